@@ -1,0 +1,198 @@
+/*
+ * dark.h -- C ABI of the B200 (sm_100a) DARKformer positive-random-feature
+ * attention library: forward pass (non-causal, causal, key-masked) and the
+ * streaming decode step.
+ *
+ * Source of the method: the DARKformer README ("Data-Aware Random Feature
+ * Kernels for Transformers", darkformer-pytorch 0.1.0 package description).
+ *   - section "Kernel": Sigma = M^T M; q and k are scaled by d^{-1/4};
+ *     phi(x; omega_j) = m^{-1/2} exp(omega_j^T M x - 1/2 x^T Sigma x),
+ *     omega_j ~ N(0, I); Att = Phi(Q)(Phi(K)^T V) / Phi(Q)(Phi(K)^T 1).
+ *   - section "Self-attention": B x L boolean key mask (true = valid), causal
+ *     constraint combined with the mask, per-head or shared geometry,
+ *     orthogonal or independent Gaussian features.
+ *   - section "Encoder-decoder model and generation": recurrent statistics
+ *     updated per appended token; a state is tied to the projection that made
+ *     it and a redraw is detected and rejected.
+ *   - section "Mixed precision": bf16 I/O with stable (fp32) accumulation.
+ *
+ * Conventions shared by every call
+ *   - Every pointer argument named as "device" must be device memory owned by
+ *     the caller; the library allocates nothing, frees nothing, and keeps no
+ *     state between calls except a process-wide projection generation counter.
+ *   - All calls are asynchronous on `stream` (a cudaStream_t passed as void*;
+ *     NULL is the legacy default stream). Argument errors are detected on the
+ *     host before anything is enqueued and returned as a status; nothing
+ *     crosses the ABI as an exception and no kernel traps.
+ *   - `dev_status` (device int, may be NULL): kernels store a nonzero
+ *     dark_status there when they detect a problem on the device
+ *     (DARK_ERR_NUMERIC: a non-finite output; DARK_ERR_TIMEOUT: a bounded
+ *     inter-block wait ran out). The caller zeroes it and reads it after the
+ *     stream is synchronised. The first error stored wins.
+ *   - Tokens use the layout [B][H][L][d] with d innermost (stride 1) and
+ *     caller-given element strides for b, h and l (NULL = contiguous).
+ */
+#ifndef DARK_H_
+#define DARK_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define DARK_ABI_VERSION 1
+
+typedef enum {
+  DARK_OK = 0,
+  DARK_ERR_INVALID_ARG = 1,   /* a size, pointer, alignment or layout is invalid  */
+  DARK_ERR_UNSUPPORTED = 2,   /* valid, but outside what this build implements    */
+  DARK_ERR_STALE_STATE = 3,   /* decode state made with another projection        */
+  DARK_ERR_CUDA = 4,          /* a CUDA launch or runtime call failed             */
+  DARK_ERR_NUMERIC = 5,       /* device: non-finite output                        */
+  DARK_ERR_TIMEOUT = 6        /* device: a bounded wait between blocks ran out    */
+} dark_status;
+
+typedef enum { DARK_F32 = 0, DARK_BF16 = 1 } dark_dtype;
+
+enum {
+  DARK_CAUSAL = 1,     /* key j is visible to query i only if j <= i (diagonal included) */
+  DARK_STABILISE = 2   /* overflow guard; see dark_attention_fwd                          */
+};
+
+/*
+ * A built projection. `w` points to caller-owned device memory holding
+ *   W' = [ c_w * (Omega_h M_h) ; c_m * M_h ]   per head, [heads][m + r][d],
+ *   c_w = d^{-1/4} * log2(e),  c_m = d^{-1/4} * sqrt(log2(e)/2),
+ * so that, for a raw token x, (W' x)_j is the feature exponent omega_j^T M x~
+ * in base 2 and sum_i (W' x)_{m+i}^2 is 1/2 x~^T Sigma x~ in base 2.
+ * DARK_F32: one fp32 plane. DARK_BF16: two bf16 planes [2][heads][m + r][d],
+ * hi = bf16(W') and lo = bf16(W' - hi); kernels use hi + lo, which keeps the
+ * exponents accurate to about 2^-16 relative (a single bf16 plane, 2^-9, moves
+ * the exponent of large features by ~1e-2 and the outputs by ~3e-2).
+ * `heads` is 1 when Omega and M are both shared by all heads, else H.
+ * `generation` is unique per dark_make_projection call in this process.
+ */
+typedef struct dark_projection {
+  int heads, m, r, d;
+  dark_dtype dtype;
+  uint64_t generation;
+  void* w;
+} dark_projection;
+
+/*
+ * Recurrent statistics of linear attention for every (batch, head):
+ *   kv = Phi(K)^T V  as [B][H][m][d] fp32,  z = Phi(K)^T 1  as [B][H][m] fp32,
+ * both device memory owned by the caller, summed over every valid key seen.
+ * `shift` is NULL unless the state was made with DARK_STABILISE: then it is a
+ * device [B][H] fp32 array holding the base-2 key constant c_K that every
+ * stored feature was divided by (2^{-c_K}); decode reuses it.
+ * `generation` ties the state to the projection that made it.
+ */
+typedef struct dark_state {
+  float* kv;
+  float* z;
+  float* shift;
+  int B, H, m, d;
+  uint64_t generation;
+} dark_state;
+
+/* ABI version of the loaded library (DARK_ABI_VERSION at build time). */
+int dark_abi_version(void);
+
+/* Human-readable name of a status code. Never NULL; static storage. */
+const char* dark_status_string(dark_status s);
+
+/* Bytes of the projection buffer for the given sizes, 0 if a size is not positive. */
+size_t dark_projection_bytes(int heads, int m, int r, int d, dark_dtype dtype);
+
+/*
+ * Builds W' (layout above) from the random features and the learned geometry
+ * (README "Kernel": W = Omega M with omega_j ~ N(0, I) in R^r, M is r x d).
+ *   omega       device fp32 [heads_omega][m][r]; heads_omega in {1, H}
+ *   geom        device fp32 [heads_geom][r][d];  heads_geom  in {1, H}
+ *   H           number of attention heads (>= 1)
+ *   dtype       DARK_BF16 or DARK_F32: the element type of W' and of the
+ *               tokens this projection will be used with
+ *   w_buf       device, w_bytes >= dark_projection_bytes(heads, ...), 16-byte
+ *               aligned; heads = max(heads_omega, heads_geom)
+ *               (for DARK_BF16 its size is 2 * heads * (m + r) * d * 2 bytes)
+ *   out         host struct filled on success (w = w_buf, a new generation)
+ * Products are accumulated in fp64, then rounded to `dtype` (hi/lo for bf16).
+ * Calling it again (a redraw) gives a new generation: states made with the
+ * old projection are rejected by dark_decode_step.
+ * Supported sizes: 4 <= d <= 256 with d a multiple of 4, 1 <= r <= 256,
+ * 1 <= m <= 1024; other positive sizes return DARK_ERR_UNSUPPORTED.
+ */
+dark_status dark_make_projection(const float* omega, int heads_omega, const float* geom,
+                                 int heads_geom, int H, int m, int r, int d, dark_dtype dtype,
+                                 void* w_buf, size_t w_bytes, void* stream,
+                                 dark_projection* out);
+
+/*
+ * Workspace bytes dark_attention_fwd needs for these sizes and flags (the
+ * largest need of any kernel path the call may take). The workspace is device
+ * memory, 256-byte aligned, owned by the caller. Its first 256 bytes hold
+ * synchronisation words: they must be zero before the workspace is first used,
+ * and every call that completes without a device error leaves them zero again,
+ * so the workspace can be reused without clearing. After a device error
+ * (dev_status != 0) zero them again. The rest needs no initialisation. Two
+ * calls in flight at the same time need two workspaces.
+ */
+size_t dark_attention_workspace_bytes(const dark_projection* proj, int B, int H, int L, int flags);
+
+/*
+ * Forward pass of PRF attention (README "Kernel", "Self-attention").
+ *   q, k, v      device, [B][H][L][d] of proj->dtype with strides qkv_strides
+ *                (elements; {b, h, l}; d stride 1; NULL = contiguous)
+ *   out          device, [B][H][L][d] of proj->dtype, strides out_strides
+ *   key_mask     device uint8 [B][L] (nonzero = valid key) or NULL = all valid.
+ *                Masked keys contribute nothing; query rows are not masked.
+ *   flags        DARK_CAUSAL: out_i uses keys j <= i only (diagonal included).
+ *                DARK_STABILISE: subtract a per-query constant (the row max of
+ *                the query exponents) and one per-(b, h) constant shared by
+ *                all keys (the max key exponent) before exponentiating; both
+ *                cancel exactly in the ratio, so outputs are unchanged in
+ *                exact arithmetic while large exponents no longer overflow.
+ *   state_out    NULL, or a state whose kv/z (and shift, with DARK_STABILISE)
+ *                receive the statistics over all valid keys; its generation is
+ *                set to proj->generation.
+ *   ws, ws_bytes workspace (see dark_attention_workspace_bytes)
+ * A query row whose visible valid keys sum to a zero denominator gets a zero
+ * output. bf16 I/O accumulates in fp32; fp32 I/O computes in fp32 throughout.
+ * Returns DARK_ERR_INVALID_ARG for inconsistent sizes or pointers,
+ * DARK_ERR_UNSUPPORTED for sizes outside dark_make_projection's limits.
+ */
+dark_status dark_attention_fwd(const dark_projection* proj, const void* q, const void* k,
+                               const void* v, void* out, const int64_t* qkv_strides,
+                               const int64_t* out_strides, int B, int H, int L,
+                               const uint8_t* key_mask, int flags, dark_state* state_out,
+                               void* ws, size_t ws_bytes, int* dev_status, void* stream);
+
+/*
+ * Zeroes a state (kv, z and, if non-NULL, shift) and ties it to `proj`, for
+ * decoding from an empty prefix.
+ */
+dark_status dark_state_init(const dark_projection* proj, dark_state* st, void* stream);
+
+/*
+ * One streaming decode step for every (batch, head) (README "Encoder-decoder
+ * model and generation"): with k_t valid, kv += phi(k_t) v_t^T and
+ * z += phi(k_t); then out_t = phi(q_t)^T kv / phi(q_t)^T z (update, then emit).
+ *   q_t, k_t, v_t, out_t  device [B][H][d] of proj->dtype, contiguous
+ *   valid                 device uint8 [B] (nonzero = this token is a valid key)
+ *                         or NULL = all valid
+ *   st                    state of sizes (B, H, proj->m, proj->d)
+ * Returns DARK_ERR_STALE_STATE, enqueuing nothing, when st->generation !=
+ * proj->generation (the projection was rebuilt after the state was made).
+ */
+dark_status dark_decode_step(const dark_projection* proj, dark_state* st, const void* q_t,
+                             const void* k_t, const void* v_t, void* out_t,
+                             const uint8_t* valid, int* dev_status, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DARK_H_ */

@@ -1,0 +1,230 @@
+// C ABI of the library (declared in include/dark.h): argument validation on the
+// host, choice between the tensor-core kernels and the generic SIMT kernels,
+// and launches on the caller's stream. Nothing here allocates device memory.
+#include <atomic>
+#include <string.h>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace {
+
+std::atomic<uint64_t> g_generation{0};
+
+constexpr int kMaxD = 256, kMaxR = 256, kMaxM = 1024;
+
+bool sizes_ok(int m, int r, int d) {
+  return m >= 1 && m <= kMaxM && r >= 1 && r <= kMaxR && d >= 4 && d <= kMaxD && d % 4 == 0;
+}
+
+bool dtype_ok(dark_dtype t) { return t == DARK_F32 || t == DARK_BF16; }
+
+size_t elt(dark_dtype t) { return t == DARK_BF16 ? 2 : 4; }
+
+bool aligned(const void* p, size_t a) { return ((uintptr_t)p % a) == 0; }
+
+dark_status from_cuda(cudaError_t e) { return e == cudaSuccess ? DARK_OK : DARK_ERR_CUDA; }
+
+bool proj_ok(const dark_projection* p) {
+  return p != nullptr && p->w != nullptr && aligned(p->w, 16) && dtype_ok(p->dtype) &&
+         sizes_ok(p->m, p->r, p->d) && p->heads >= 1;
+}
+
+enum class Path { Simt, TcCausal, TcNonCausal };
+
+Path choose_path(const dark::FwdArgs& a) {
+  if (a.flags & DARK_CAUSAL) {
+    if (dark::tc_causal_supported(a)) return Path::TcCausal;
+  } else {
+    if (dark::tc_noncausal_supported(a)) return Path::TcNonCausal;
+  }
+  return Path::Simt;
+}
+
+size_t ws_need(Path p, int B, int H, int L, int m, int d, int flags) {
+  switch (p) {
+    case Path::TcCausal: return dark::tc_causal_workspace_bytes(B, H, L, m, d);
+    case Path::TcNonCausal: return dark::tc_noncausal_workspace_bytes(B, H, L, m, d);
+    default: return dark::simt_workspace_bytes(B, H, L, m, d, flags);
+  }
+}
+
+}  // namespace
+
+extern "C" {
+
+int dark_abi_version(void) { return DARK_ABI_VERSION; }
+
+const char* dark_status_string(dark_status s) {
+  switch (s) {
+    case DARK_OK: return "DARK_OK";
+    case DARK_ERR_INVALID_ARG: return "DARK_ERR_INVALID_ARG: invalid size, pointer, alignment or layout";
+    case DARK_ERR_UNSUPPORTED: return "DARK_ERR_UNSUPPORTED: sizes outside what this build implements";
+    case DARK_ERR_STALE_STATE: return "DARK_ERR_STALE_STATE: decode state belongs to another projection";
+    case DARK_ERR_CUDA: return "DARK_ERR_CUDA: a CUDA launch or runtime call failed";
+    case DARK_ERR_NUMERIC: return "DARK_ERR_NUMERIC: non-finite output";
+    case DARK_ERR_TIMEOUT: return "DARK_ERR_TIMEOUT: a bounded wait between blocks ran out";
+  }
+  return "unknown dark_status";
+}
+
+size_t dark_projection_bytes(int heads, int m, int r, int d, dark_dtype dtype) {
+  if (heads < 1 || m < 1 || r < 1 || d < 1 || !dtype_ok(dtype)) return 0;
+  const size_t planes = dtype == DARK_BF16 ? 2 : 1;
+  return planes * (size_t)heads * (size_t)(m + r) * (size_t)d * elt(dtype);
+}
+
+dark_status dark_make_projection(const float* omega, int heads_omega, const float* geom,
+                                 int heads_geom, int H, int m, int r, int d, dark_dtype dtype,
+                                 void* w_buf, size_t w_bytes, void* stream,
+                                 dark_projection* out) {
+  if (omega == nullptr || geom == nullptr || w_buf == nullptr || out == nullptr || H < 1 ||
+      !dtype_ok(dtype))
+    return DARK_ERR_INVALID_ARG;
+  if (!(heads_omega == 1 || heads_omega == H) || !(heads_geom == 1 || heads_geom == H))
+    return DARK_ERR_INVALID_ARG;
+  if (m < 1 || r < 1 || d < 1) return DARK_ERR_INVALID_ARG;
+  if (!sizes_ok(m, r, d)) return DARK_ERR_UNSUPPORTED;
+  const int heads = heads_omega > heads_geom ? heads_omega : heads_geom;
+  if (w_bytes < dark_projection_bytes(heads, m, r, d, dtype) || !aligned(w_buf, 16))
+    return DARK_ERR_INVALID_ARG;
+  cudaError_t e = dark::launch_projection(omega, heads_omega, geom, heads_geom, heads, m, r, d,
+                                          dtype, w_buf, (cudaStream_t)stream);
+  if (e != cudaSuccess) return DARK_ERR_CUDA;
+  out->heads = heads;
+  out->m = m;
+  out->r = r;
+  out->d = d;
+  out->dtype = dtype;
+  out->w = w_buf;
+  out->generation = ++g_generation;
+  return DARK_OK;
+}
+
+size_t dark_attention_workspace_bytes(const dark_projection* proj, int B, int H, int L,
+                                      int flags) {
+  if (!proj_ok(proj) || B < 1 || H < 1 || L < 1) return 0;
+  const int m = proj->m, d = proj->d;
+  size_t need = dark::simt_workspace_bytes(B, H, L, m, d, flags);
+  const size_t tc = (flags & DARK_CAUSAL) ? dark::tc_causal_workspace_bytes(B, H, L, m, d)
+                                          : dark::tc_noncausal_workspace_bytes(B, H, L, m, d);
+  return need > tc ? need : tc;
+}
+
+dark_status dark_attention_fwd(const dark_projection* proj, const void* q, const void* k,
+                               const void* v, void* out, const int64_t* qkv_strides,
+                               const int64_t* out_strides, int B, int H, int L,
+                               const uint8_t* key_mask, int flags, dark_state* state_out,
+                               void* ws, size_t ws_bytes, int* dev_status, void* stream) {
+  if (proj == nullptr || proj->w == nullptr || !aligned(proj->w, 16) || !dtype_ok(proj->dtype))
+    return DARK_ERR_INVALID_ARG;
+  if (proj->m < 1 || proj->r < 1 || proj->d < 1) return DARK_ERR_INVALID_ARG;
+  if (!sizes_ok(proj->m, proj->r, proj->d)) return DARK_ERR_UNSUPPORTED;
+  if (q == nullptr || k == nullptr || v == nullptr || out == nullptr) return DARK_ERR_INVALID_ARG;
+  if (B < 1 || H < 1 || L < 1) return DARK_ERR_INVALID_ARG;
+  if (!(proj->heads == 1 || proj->heads == H)) return DARK_ERR_INVALID_ARG;
+  if (flags & ~(DARK_CAUSAL | DARK_STABILISE)) return DARK_ERR_INVALID_ARG;
+  if (ws == nullptr || !aligned(ws, 256)) return DARK_ERR_INVALID_ARG;
+
+  dark::FwdArgs a;
+  memset(&a, 0, sizeof(a));
+  a.heads_w = proj->heads;
+  a.m = proj->m;
+  a.r = proj->r;
+  a.d = proj->d;
+  a.dtype = proj->dtype;
+  a.w = proj->w;
+  a.q = q;
+  a.k = k;
+  a.v = v;
+  a.out = out;
+  const int64_t d = proj->d;
+  const int64_t contig[3] = {(int64_t)H * L * d, (int64_t)L * d, d};
+  for (int i = 0; i < 3; ++i) {
+    a.qs[i] = qkv_strides ? qkv_strides[i] : contig[i];
+    a.os[i] = out_strides ? out_strides[i] : contig[i];
+    if (a.qs[i] < 0 || a.os[i] < 0) return DARK_ERR_INVALID_ARG;
+  }
+  a.B = B;
+  a.H = H;
+  a.L = L;
+  a.mask = key_mask;
+  a.flags = flags;
+  if (state_out != nullptr) {
+    if (state_out->kv == nullptr || state_out->z == nullptr || state_out->B != B ||
+        state_out->H != H || state_out->m != proj->m || state_out->d != proj->d)
+      return DARK_ERR_INVALID_ARG;
+    if ((flags & DARK_STABILISE) && state_out->shift == nullptr) return DARK_ERR_INVALID_ARG;
+    a.st_kv = state_out->kv;
+    a.st_z = state_out->z;
+    a.st_shift = (flags & DARK_STABILISE) ? state_out->shift : nullptr;
+  }
+  a.ws = ws;
+  a.ws_bytes = ws_bytes;
+  a.dev_status = dev_status;
+  a.stream = (cudaStream_t)stream;
+
+  const Path p = choose_path(a);
+  if (ws_bytes < ws_need(p, B, H, L, a.m, a.d, flags)) return DARK_ERR_INVALID_ARG;
+  cudaError_t e;
+  switch (p) {
+    case Path::TcCausal: e = dark::tc_causal_forward(a); break;
+    case Path::TcNonCausal: e = dark::tc_noncausal_forward(a); break;
+    default: e = dark::simt_forward(a); break;
+  }
+  if (e != cudaSuccess) return DARK_ERR_CUDA;
+  if (state_out != nullptr) state_out->generation = proj->generation;
+  return DARK_OK;
+}
+
+dark_status dark_state_init(const dark_projection* proj, dark_state* st, void* stream) {
+  if (proj == nullptr || st == nullptr || st->kv == nullptr || st->z == nullptr)
+    return DARK_ERR_INVALID_ARG;
+  if (st->B < 1 || st->H < 1 || st->m != proj->m || st->d != proj->d) return DARK_ERR_INVALID_ARG;
+  const size_t n = (size_t)st->B * st->H;
+  cudaStream_t s = (cudaStream_t)stream;
+  cudaError_t e = cudaMemsetAsync(st->kv, 0, n * st->m * st->d * sizeof(float), s);
+  if (e == cudaSuccess) e = cudaMemsetAsync(st->z, 0, n * st->m * sizeof(float), s);
+  if (e == cudaSuccess && st->shift != nullptr) e = cudaMemsetAsync(st->shift, 0, n * sizeof(float), s);
+  if (e != cudaSuccess) return DARK_ERR_CUDA;
+  st->generation = proj->generation;
+  return DARK_OK;
+}
+
+dark_status dark_decode_step(const dark_projection* proj, dark_state* st, const void* q_t,
+                             const void* k_t, const void* v_t, void* out_t,
+                             const uint8_t* valid, int* dev_status, void* stream) {
+  if (proj == nullptr || proj->w == nullptr || !aligned(proj->w, 16) || !dtype_ok(proj->dtype) ||
+      st == nullptr)
+    return DARK_ERR_INVALID_ARG;
+  if (!sizes_ok(proj->m, proj->r, proj->d)) return DARK_ERR_UNSUPPORTED;
+  if (st->kv == nullptr || st->z == nullptr || q_t == nullptr || k_t == nullptr ||
+      v_t == nullptr || out_t == nullptr)
+    return DARK_ERR_INVALID_ARG;
+  if (st->B < 1 || st->H < 1 || st->m != proj->m || st->d != proj->d) return DARK_ERR_INVALID_ARG;
+  if (!(proj->heads == 1 || proj->heads == st->H)) return DARK_ERR_INVALID_ARG;
+  if (!aligned(st->kv, 16)) return DARK_ERR_INVALID_ARG;
+  if (st->generation != proj->generation) return DARK_ERR_STALE_STATE;
+  dark::DecodeArgs a;
+  a.heads_w = proj->heads;
+  a.m = proj->m;
+  a.r = proj->r;
+  a.d = proj->d;
+  a.dtype = proj->dtype;
+  a.w = proj->w;
+  a.kv = st->kv;
+  a.z = st->z;
+  a.shift = st->shift;
+  a.B = st->B;
+  a.H = st->H;
+  a.q = q_t;
+  a.k = k_t;
+  a.v = v_t;
+  a.out = out_t;
+  a.valid = valid;
+  a.dev_status = dev_status;
+  a.stream = (cudaStream_t)stream;
+  return from_cuda(dark::launch_decode(a));
+}
+
+}  // extern "C"

@@ -1,0 +1,222 @@
+// Streaming decode step of PRF attention (DARKformer README, section
+// "Encoder-decoder model and generation": in linear mode the recurrent
+// statistics Phi(K)^T V and Phi(K)^T 1 are updated per appended token).
+//
+// One block per (batch, head). The step is bound by reading and writing the
+// fp32 state (m x d + m floats per head), so the block first computes both
+// feature vectors (a GEMV with W' from L2), then streams its state rows with
+// coalesced 16-byte accesses, several rows in flight per thread, and folds the
+// output contraction into the same pass: out = phi(q)^T kv' / phi(q)^T z'.
+#include <math.h>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace dark {
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kBatchRows = 8;   // state rows loaded per thread before their update
+
+__device__ __forceinline__ void row_dot2(const float* __restrict__ w, size_t /*lo*/, int d,
+                                         const float* xk, const float* xq, bool both, float& ak,
+                                         float& aq) {
+  float sk = 0.f, sq = 0.f;
+  if ((d & 3) == 0) {
+    const float4* w4 = reinterpret_cast<const float4*>(w);
+    for (int c = 0; c < d / 4; ++c) {
+      const float4 u = __ldg(w4 + c);
+      sk = fmaf(u.x, xk[4 * c], sk); sk = fmaf(u.y, xk[4 * c + 1], sk);
+      sk = fmaf(u.z, xk[4 * c + 2], sk); sk = fmaf(u.w, xk[4 * c + 3], sk);
+      if (both) {
+        sq = fmaf(u.x, xq[4 * c], sq); sq = fmaf(u.y, xq[4 * c + 1], sq);
+        sq = fmaf(u.z, xq[4 * c + 2], sq); sq = fmaf(u.w, xq[4 * c + 3], sq);
+      }
+    }
+  } else {
+    for (int c = 0; c < d; ++c) {
+      sk = fmaf(w[c], xk[c], sk);
+      if (both) sq = fmaf(w[c], xq[c], sq);
+    }
+  }
+  ak = sk;
+  aq = sq;
+}
+
+// bf16 projections: the weight is hi + lo, the lo plane `lo` elements after hi.
+__device__ __forceinline__ void row_dot2(const __nv_bfloat16* __restrict__ w, size_t lo, int d,
+                                         const float* xk, const float* xq, bool both, float& ak,
+                                         float& aq) {
+  float sk = 0.f, sq = 0.f;
+  if ((d & 7) == 0) {
+    const uint4* w8 = reinterpret_cast<const uint4*>(w);
+    const uint4* l8 = reinterpret_cast<const uint4*>(w + lo);
+    for (int c = 0; c < d / 8; ++c) {
+      const uint4 u = __ldg(w8 + c);
+      const uint4 ul = __ldg(l8 + c);
+      const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&u);
+      const __nv_bfloat162* pl = reinterpret_cast<const __nv_bfloat162*>(&ul);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 fh = __bfloat1622float2(p[e]);
+        const float2 fl = __bfloat1622float2(pl[e]);
+        const float2 f = make_float2(fh.x + fl.x, fh.y + fl.y);
+        sk = fmaf(f.x, xk[8 * c + 2 * e], sk);
+        sk = fmaf(f.y, xk[8 * c + 2 * e + 1], sk);
+        if (both) {
+          sq = fmaf(f.x, xq[8 * c + 2 * e], sq);
+          sq = fmaf(f.y, xq[8 * c + 2 * e + 1], sq);
+        }
+      }
+    }
+  } else {
+    for (int c = 0; c < d; ++c) {
+      const float f = __bfloat162float(w[c]) + __bfloat162float(w[c + lo]);
+      sk = fmaf(f, xk[c], sk);
+      if (both) sq = fmaf(f, xq[c], sq);
+    }
+  }
+  ak = sk;
+  aq = sq;
+}
+
+__device__ __forceinline__ float block_sum(float v, float* scratch) {
+  v = warp_sum(v);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  __syncthreads();
+  if (lane == 0) scratch[warp] = v;
+  __syncthreads();
+  float t = lane < kThreads / 32 ? scratch[lane] : 0.f;
+  return warp_sum(t);
+}
+
+__device__ __forceinline__ float block_max(float v, float* scratch) {
+  v = warp_max(v);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  __syncthreads();
+  if (lane == 0) scratch[warp] = v;
+  __syncthreads();
+  float t = lane < kThreads / 32 ? scratch[lane] : -INFINITY;
+  return warp_max(t);
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kThreads) decode_kernel(
+    const T* __restrict__ w, int heads_w, int m, int r, int d, float* __restrict__ kv,
+    float* __restrict__ z, const float* __restrict__ shift, int H, const T* __restrict__ q,
+    const T* __restrict__ k, const T* __restrict__ v, T* __restrict__ out,
+    const uint8_t* __restrict__ valid, int* dev_status) {
+  extern __shared__ float sm[];
+  const int tpr = d / 4;                  // threads per state row (one float4 each)
+  const int rpp = kThreads / tpr;         // rows per pass
+  float* xq = sm;                         // [d]
+  float* xk = xq + d;                     // [d]
+  float* xv = xk + d;                     // [d]
+  float* pk = xv + d;                     // [m + r]
+  float* pq = pk + m + r;                 // [m]
+  float* red = pq + m;                    // [rpp][d]
+  float* scratch = red + rpp * d;         // [32]
+  const int bh = blockIdx.x, b = bh / H, h = bh % H;
+  const T* wh = w + (size_t)(heads_w == 1 ? 0 : h) * (m + r) * d;
+  const int tid = threadIdx.x;
+
+  for (int c = tid; c < d; c += kThreads) {
+    xq[c] = to_f32(q[(size_t)bh * d + c]);
+    xk[c] = to_f32(k[(size_t)bh * d + c]);
+    xv[c] = to_f32(v[(size_t)bh * d + c]);
+  }
+  __syncthreads();
+  for (int j = tid; j < m + r; j += kThreads) {
+    float ak, aq;
+    row_dot2(wh + (size_t)j * d, (size_t)heads_w * (m + r) * d, d, xk, xq, j < m, ak, aq);
+    pk[j] = ak;
+    if (j < m) pq[j] = aq;
+  }
+  __syncthreads();
+  float nrm = 0.f, qmax = -INFINITY;
+  for (int i = tid; i < r; i += kThreads) nrm = fmaf(pk[m + i], pk[m + i], nrm);
+  for (int j = tid; j < m; j += kThreads) qmax = fmaxf(qmax, pq[j]);
+  nrm = block_sum(nrm, scratch);
+  const bool stab = shift != nullptr;
+  const float qs = stab ? block_max(qmax, scratch) : 0.f;
+  const float ks = nrm + 0.5f * log2f((float)m) + (stab ? shift[bh] : 0.f);
+  const bool ok = valid == nullptr || valid[b] != 0;
+  for (int j = tid; j < m; j += kThreads) {
+    pk[j] = ok ? exp2f(pk[j] - ks) : 0.f;
+    pq[j] = exp2f(pq[j] - qs);
+  }
+  __syncthreads();
+
+  // kv' = kv + phi(k) v^T and num = phi(q)^T kv', one float4 column group per thread.
+  float4 num = make_float4(0.f, 0.f, 0.f, 0.f);
+  const int c4 = tid % tpr, r0 = tid / tpr;
+  if (r0 < rpp) {
+    const float4 vv = make_float4(xv[4 * c4], xv[4 * c4 + 1], xv[4 * c4 + 2], xv[4 * c4 + 3]);
+    float4* base = reinterpret_cast<float4*>(kv + (size_t)bh * m * d) + c4;
+    const int stride = d / 4;
+    for (int j0 = r0; j0 < m; j0 += rpp * kBatchRows) {
+      float4 s[kBatchRows];
+#pragma unroll
+      for (int u = 0; u < kBatchRows; ++u) {
+        const int j = j0 + u * rpp;
+        if (j < m) s[u] = base[(size_t)j * stride];
+      }
+#pragma unroll
+      for (int u = 0; u < kBatchRows; ++u) {
+        const int j = j0 + u * rpp;
+        if (j < m) {
+          const float fk = pk[j], fq = pq[j];
+          s[u].x = fmaf(fk, vv.x, s[u].x); s[u].y = fmaf(fk, vv.y, s[u].y);
+          s[u].z = fmaf(fk, vv.z, s[u].z); s[u].w = fmaf(fk, vv.w, s[u].w);
+          base[(size_t)j * stride] = s[u];
+          num.x = fmaf(fq, s[u].x, num.x); num.y = fmaf(fq, s[u].y, num.y);
+          num.z = fmaf(fq, s[u].z, num.z); num.w = fmaf(fq, s[u].w, num.w);
+        }
+      }
+    }
+    float* rr = red + r0 * d + 4 * c4;
+    rr[0] = num.x; rr[1] = num.y; rr[2] = num.z; rr[3] = num.w;
+  }
+  float den = 0.f;
+  for (int j = tid; j < m; j += kThreads) {
+    const float zj = z[(size_t)bh * m + j] + pk[j];
+    z[(size_t)bh * m + j] = zj;
+    den = fmaf(pq[j], zj, den);
+  }
+  den = block_sum(den, scratch);   // contains the barrier that publishes `red`
+  for (int c = tid; c < d; c += kThreads) {
+    float acc = 0.f;
+    for (int g = 0; g < rpp; ++g) acc += red[g * d + c];
+    const float o = den > 0.f ? acc / den : 0.f;
+    if (!isfinite(o)) report(dev_status, DARK_ERR_NUMERIC);
+    out[(size_t)bh * d + c] = from_f32<T>(o);
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_decode(const DecodeArgs& a) {
+  const int tpr = a.d / 4;
+  const int rpp = kThreads / tpr;
+  const size_t smem = sizeof(float) * (3 * a.d + (a.m + a.r) + a.m + rpp * a.d + 32);
+  cudaError_t err;
+  if (a.dtype == DARK_BF16) {
+    err = cudaFuncSetAttribute(decode_kernel<__nv_bfloat16>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (err != cudaSuccess) return err;
+    decode_kernel<__nv_bfloat16><<<a.B * a.H, kThreads, smem, a.stream>>>(
+        (const __nv_bfloat16*)a.w, a.heads_w, a.m, a.r, a.d, a.kv, a.z, a.shift, a.H,
+        (const __nv_bfloat16*)a.q, (const __nv_bfloat16*)a.k, (const __nv_bfloat16*)a.v,
+        (__nv_bfloat16*)a.out, a.valid, a.dev_status);
+  } else {
+    err = cudaFuncSetAttribute(decode_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)smem);
+    if (err != cudaSuccess) return err;
+    decode_kernel<float><<<a.B * a.H, kThreads, smem, a.stream>>>(
+        (const float*)a.w, a.heads_w, a.m, a.r, a.d, a.kv, a.z, a.shift, a.H, (const float*)a.q,
+        (const float*)a.k, (const float*)a.v, (float*)a.out, a.valid, a.dev_status);
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace dark

@@ -1,0 +1,71 @@
+// Internal launch interface between the C-ABI layer (api.cu) and the kernels.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "../../include/dark.h"
+
+namespace dark {
+
+// Everything one forward call needs, validated by the C-ABI layer.
+struct FwdArgs {
+  int heads_w, m, r, d;
+  dark_dtype dtype;
+  const void* w;                  // projection buffer [heads_w][m + r][d]
+  const void *q, *k, *v;
+  void* out;
+  int64_t qs[3], os[3];           // element strides {b, h, l} of q/k/v and of out
+  int B, H, L;
+  const uint8_t* mask;            // [B][L] or null
+  int flags;
+  float *st_kv, *st_z, *st_shift; // state_out arrays or null
+  void* ws;
+  size_t ws_bytes;
+  int* dev_status;
+  cudaStream_t stream;
+};
+
+inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// Every workspace starts with this many bytes of synchronisation words (zero
+// at first use, restored to zero by the kernels that use them); kernel data
+// of every path starts after it.
+constexpr size_t kWsHeader = 256;
+
+// Projection W' = [c_w Omega M ; c_m M] (one-off, fp64 accumulation).
+cudaError_t launch_projection(const float* omega, int heads_omega, const float* geom,
+                              int heads_geom, int heads_w, int m, int r, int d,
+                              dark_dtype dtype, void* w, cudaStream_t stream);
+
+// Generic SIMT forward: any strides, any supported sizes, fp32 or bf16 I/O.
+size_t simt_workspace_bytes(int B, int H, int L, int m, int d, int flags);
+cudaError_t simt_forward(const FwdArgs& a);
+
+// Tensor-core forward paths (tcgen05/TMEM/TMA). `*_supported` says whether the
+// sizes, layout and alignment fit; the launchers assume they do.
+bool tc_causal_supported(const FwdArgs& a);
+size_t tc_causal_workspace_bytes(int B, int H, int L, int m, int d);
+cudaError_t tc_causal_forward(const FwdArgs& a);
+
+bool tc_noncausal_supported(const FwdArgs& a);
+size_t tc_noncausal_workspace_bytes(int B, int H, int L, int m, int d);
+cudaError_t tc_noncausal_forward(const FwdArgs& a);
+
+// Decode step over [B][H] heads.
+struct DecodeArgs {
+  int heads_w, m, r, d;
+  dark_dtype dtype;
+  const void* w;
+  float *kv, *z, *shift;
+  int B, H;
+  const void *q, *k, *v;
+  void* out;
+  const uint8_t* valid;
+  int* dev_status;
+  cudaStream_t stream;
+};
+cudaError_t launch_decode(const DecodeArgs& a);
+
+}  // namespace dark

@@ -1,0 +1,8 @@
+// Non-causal tensor-core forward (filled in below; not yet available).
+#include "internal.h"
+
+namespace dark {
+bool tc_noncausal_supported(const FwdArgs&) { return false; }
+size_t tc_noncausal_workspace_bytes(int, int, int, int, int) { return 0; }
+cudaError_t tc_noncausal_forward(const FwdArgs&) { return cudaErrorNotSupported; }
+}  // namespace dark

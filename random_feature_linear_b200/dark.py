@@ -1,0 +1,176 @@
+"""Python binding of the C ABI in include/dark.h (ctypes; marshalling only).
+
+Every function here has the name of the C entry point it calls and does
+nothing but convert arguments: torch tensors become device pointers, the
+current torch stream becomes the cudaStream_t, statuses become exceptions.
+All computation runs in the native library ``libdark.so``; importing this
+module fails loudly if that library has not been built.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libdark.so")
+if not os.path.exists(_LIB_PATH):
+    raise ImportError(
+        f"{_LIB_PATH} is missing: build it with `python -m random_feature_linear_b200.build` "
+        "(there is no fallback implementation)")
+_lib = ctypes.CDLL(_LIB_PATH)
+
+DARK_OK, DARK_ERR_INVALID_ARG, DARK_ERR_UNSUPPORTED, DARK_ERR_STALE_STATE = 0, 1, 2, 3
+DARK_ERR_CUDA, DARK_ERR_NUMERIC, DARK_ERR_TIMEOUT = 4, 5, 6
+DARK_F32, DARK_BF16 = 0, 1
+DARK_CAUSAL, DARK_STABILISE = 1, 2
+WS_HEADER_BYTES = 256
+
+EXPORTS = ("dark_abi_version", "dark_status_string", "dark_projection_bytes",
+           "dark_make_projection", "dark_attention_workspace_bytes", "dark_attention_fwd",
+           "dark_state_init", "dark_decode_step")
+
+
+class dark_projection(ctypes.Structure):
+    _fields_ = [("heads", ctypes.c_int), ("m", ctypes.c_int), ("r", ctypes.c_int),
+                ("d", ctypes.c_int), ("dtype", ctypes.c_int), ("generation", ctypes.c_uint64),
+                ("w", ctypes.c_void_p)]
+
+
+class dark_state(ctypes.Structure):
+    _fields_ = [("kv", ctypes.c_void_p), ("z", ctypes.c_void_p), ("shift", ctypes.c_void_p),
+                ("B", ctypes.c_int), ("H", ctypes.c_int), ("m", ctypes.c_int), ("d", ctypes.c_int),
+                ("generation", ctypes.c_uint64)]
+
+
+_P = ctypes.POINTER
+_vp, _i, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+_lib.dark_abi_version.restype = _i
+_lib.dark_status_string.restype = ctypes.c_char_p
+_lib.dark_status_string.argtypes = [_i]
+_lib.dark_projection_bytes.restype = _sz
+_lib.dark_projection_bytes.argtypes = [_i, _i, _i, _i, _i]
+_lib.dark_make_projection.restype = _i
+_lib.dark_make_projection.argtypes = [_vp, _i, _vp, _i, _i, _i, _i, _i, _i, _vp, _sz, _vp,
+                                      _P(dark_projection)]
+_lib.dark_attention_workspace_bytes.restype = _sz
+_lib.dark_attention_workspace_bytes.argtypes = [_P(dark_projection), _i, _i, _i, _i]
+_lib.dark_attention_fwd.restype = _i
+_lib.dark_attention_fwd.argtypes = [_P(dark_projection), _vp, _vp, _vp, _vp, _P(ctypes.c_int64),
+                                    _P(ctypes.c_int64), _i, _i, _i, _vp, _i, _P(dark_state), _vp,
+                                    _sz, _vp, _vp]
+_lib.dark_state_init.restype = _i
+_lib.dark_state_init.argtypes = [_P(dark_projection), _P(dark_state), _vp]
+_lib.dark_decode_step.restype = _i
+_lib.dark_decode_step.argtypes = [_P(dark_projection), _P(dark_state), _vp, _vp, _vp, _vp, _vp,
+                                  _vp, _vp]
+
+
+class DarkError(RuntimeError):
+    def __init__(self, status: int):
+        self.status = status
+        super().__init__(dark_status_string(status))
+
+
+def _check(status: int) -> None:
+    if status != DARK_OK:
+        raise DarkError(status)
+
+
+def _ptr(t) -> int | None:
+    return None if t is None else t.data_ptr()
+
+
+def _stream(stream) -> int | None:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else stream
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+def dark_abi_version() -> int:
+    return _lib.dark_abi_version()
+
+
+def dark_status_string(status: int) -> str:
+    return _lib.dark_status_string(status).decode()
+
+
+def dark_projection_bytes(heads: int, m: int, r: int, d: int, dtype: int) -> int:
+    return _lib.dark_projection_bytes(heads, m, r, d, dtype)
+
+
+def dark_make_projection(omega: torch.Tensor, geom: torch.Tensor, H: int, dtype: int,
+                         w: torch.Tensor | None = None, stream=None) -> tuple:
+    """omega [H_o, m, r] and geom [H_m, r, d] fp32 device tensors.
+
+    Returns (dark_projection, w_buffer); keep the buffer alive while the
+    projection is used.
+    """
+    assert omega.dtype == torch.float32 and geom.dtype == torch.float32
+    omega, geom = omega.contiguous(), geom.contiguous()
+    ho, m, r = omega.shape
+    hg, r2, d = geom.shape
+    assert r == r2
+    heads = max(ho, hg)
+    nbytes = dark_projection_bytes(heads, m, r, d, dtype)
+    if w is None:
+        w = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=omega.device)
+    proj = dark_projection()
+    _check(_lib.dark_make_projection(_ptr(omega), ho, _ptr(geom), hg, H, m, r, d, dtype,
+                                     _ptr(w), w.numel() * w.element_size(), _stream(stream),
+                                     ctypes.byref(proj)))
+    return proj, w
+
+
+def dark_attention_workspace_bytes(proj: dark_projection, B: int, H: int, L: int,
+                                   flags: int) -> int:
+    return _lib.dark_attention_workspace_bytes(ctypes.byref(proj), B, H, L, flags)
+
+
+def make_state(proj: dark_projection, B: int, H: int, device, stabilised: bool = False):
+    """Allocates (torch) the arrays of a dark_state; returns (state, tensors)."""
+    kv = torch.zeros(B, H, proj.m, proj.d, dtype=torch.float32, device=device)
+    z = torch.zeros(B, H, proj.m, dtype=torch.float32, device=device)
+    sh = torch.zeros(B, H, dtype=torch.float32, device=device) if stabilised else None
+    st = dark_state(kv.data_ptr(), z.data_ptr(), _ptr(sh), B, H, proj.m, proj.d, 0)
+    return st, (kv, z, sh)
+
+
+def dark_attention_fwd(proj: dark_projection, q, k, v, out, B: int, H: int, L: int,
+                       key_mask=None, flags: int = 0, state_out: dark_state | None = None,
+                       ws=None, dev_status=None, stream=None, qkv_strides=None,
+                       out_strides=None) -> None:
+    """q/k/v/out are device tensors viewed as [B][H][L][d] with the given element
+    strides ({b, h, l}; None = contiguous). ws: a zero-initialised uint8 tensor."""
+    def strides(s):
+        return None if s is None else (ctypes.c_int64 * 3)(*s)
+    _check(_lib.dark_attention_fwd(
+        ctypes.byref(proj), _ptr(q), _ptr(k), _ptr(v), _ptr(out), strides(qkv_strides),
+        strides(out_strides), B, H, L, _ptr(key_mask), flags,
+        None if state_out is None else ctypes.byref(state_out), _ptr(ws),
+        0 if ws is None else ws.numel() * ws.element_size(), _ptr(dev_status), _stream(stream)))
+
+
+def dark_state_init(proj: dark_projection, st: dark_state, stream=None) -> None:
+    _check(_lib.dark_state_init(ctypes.byref(proj), ctypes.byref(st), _stream(stream)))
+
+
+def dark_decode_step(proj: dark_projection, st: dark_state, q_t, k_t, v_t, out_t, valid=None,
+                     dev_status=None, stream=None) -> None:
+    _check(_lib.dark_decode_step(ctypes.byref(proj), ctypes.byref(st), _ptr(q_t), _ptr(k_t),
+                                 _ptr(v_t), _ptr(out_t), _ptr(valid), _ptr(dev_status),
+                                 _stream(stream)))
+
+
+def alloc_workspace(proj: dark_projection, B: int, H: int, L: int, flags: int, device):
+    """A zero-filled workspace of the size dark_attention_workspace_bytes asks for."""
+    n = dark_attention_workspace_bytes(proj, B, H, L, flags)
+    return torch.zeros(max(n, WS_HEADER_BYTES), dtype=torch.uint8, device=device)
+
+
+def torch_dtype(dtype: int):
+    return torch.bfloat16 if dtype == DARK_BF16 else torch.float32

@@ -1,0 +1,116 @@
+"""Host-side checks of the C ABI that need no GPU: the library loads, exports
+every entry point declared in include/dark.h, and rejects bad arguments before
+anything is enqueued."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def D():
+    from random_feature_linear_b200 import build
+    build.build()
+    from random_feature_linear_b200 import dark
+    return dark
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "dark.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(dark_[a-z_]+)\s*\(", src)))
+
+
+def test_every_declared_symbol_is_exported(D):
+    names = _declared()
+    assert "dark_attention_fwd" in names and "dark_decode_step" in names
+    lib = ctypes.CDLL(D.library_path())
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(D.EXPORTS) <= set(names)
+
+
+def test_version_and_status_strings(D):
+    assert D.dark_abi_version() == 1
+    for s in range(7):
+        assert D.dark_status_string(s).startswith("DARK_")
+    assert "unknown" in D.dark_status_string(99)
+
+
+def test_projection_bytes(D):
+    assert D.dark_projection_bytes(8, 256, 64, 64, D.DARK_BF16) == 2 * 8 * 320 * 64 * 2
+    assert D.dark_projection_bytes(1, 64, 64, 64, D.DARK_F32) == 128 * 64 * 4
+    assert D.dark_projection_bytes(0, 64, 64, 64, D.DARK_F32) == 0
+
+
+def _fake_proj(D, **kw):
+    p = D.dark_projection()
+    p.heads, p.m, p.r, p.d, p.dtype, p.generation, p.w = 1, 64, 64, 64, D.DARK_BF16, 7, 0x1000
+    for k, v in kw.items():
+        setattr(p, k, v)
+    return p
+
+
+def test_make_projection_rejects_bad_arguments(D):
+    lib = D._lib
+    out = D.dark_projection()
+    f = 0x1000
+    # null pointers, head counts not in {1, H}, bad dtype, unsupported sizes, short buffer
+    assert lib.dark_make_projection(None, 1, f, 1, 8, 64, 64, 64, 1, f, 1 << 20, None, ctypes.byref(out)) == 1
+    assert lib.dark_make_projection(f, 3, f, 1, 8, 64, 64, 64, 1, f, 1 << 20, None, ctypes.byref(out)) == 1
+    assert lib.dark_make_projection(f, 1, f, 1, 8, 64, 64, 64, 7, f, 1 << 20, None, ctypes.byref(out)) == 1
+    assert lib.dark_make_projection(f, 1, f, 1, 8, 64, 64, 66, 1, f, 1 << 20, None, ctypes.byref(out)) == 2
+    assert lib.dark_make_projection(f, 1, f, 1, 8, 2048, 64, 64, 1, f, 1 << 30, None, ctypes.byref(out)) == 2
+    assert lib.dark_make_projection(f, 1, f, 1, 8, 64, 64, 64, 1, f, 100, None, ctypes.byref(out)) == 1
+    assert lib.dark_make_projection(f, 1, f, 1, 8, 64, 64, 64, 1, f + 2, 1 << 20, None, ctypes.byref(out)) == 1
+
+
+def test_forward_rejects_bad_arguments(D):
+    lib = D._lib
+    f = 0x10000
+    p = _fake_proj(D)
+    args = lambda **kw: dict(dict(q=f, k=f, v=f, o=f, B=2, H=1, L=16, flags=0, ws=f, wsb=1 << 30), **kw)
+
+    def call(a, proj=p):
+        return lib.dark_attention_fwd(ctypes.byref(proj), a["q"], a["k"], a["v"], a["o"], None, None,
+                                      a["B"], a["H"], a["L"], None, a["flags"], None, a["ws"], a["wsb"],
+                                      None, None)
+    assert call(args(q=None)) == 1
+    assert call(args(B=0)) == 1
+    assert call(args(L=-3)) == 1
+    assert call(args(flags=8)) == 1
+    assert call(args(ws=None)) == 1
+    assert call(args(ws=f + 16)) == 1                 # not 256-byte aligned
+    assert call(args(H=3), _fake_proj(D, heads=2)) == 1
+    assert call(args(), _fake_proj(D, d=66)) == 2
+    assert call(args(), _fake_proj(D, w=0x1002)) == 1  # W' not 16-byte aligned
+    assert call(args(wsb=16)) == 1                    # workspace too small
+    st = D.dark_state(f, f, None, 2, 1, 32, 64, 0)     # m mismatch
+    assert lib.dark_attention_fwd(ctypes.byref(p), f, f, f, f, None, None, 2, 1, 16, None, 0,
+                                  ctypes.byref(st), f, 1 << 30, None, None) == 1
+    st = D.dark_state(f, f, None, 2, 1, 64, 64, 0)     # stabilised state without shift
+    assert lib.dark_attention_fwd(ctypes.byref(p), f, f, f, f, None, None, 2, 1, 16, None, 2,
+                                  ctypes.byref(st), f, 1 << 30, None, None) == 1
+
+
+def test_decode_rejects_stale_state_before_launch(D):
+    lib = D._lib
+    f = 0x10000
+    p = _fake_proj(D, generation=5)
+    st = D.dark_state(f, f, None, 2, 1, 64, 64, 4)
+    assert lib.dark_decode_step(ctypes.byref(p), ctypes.byref(st), f, f, f, f, None, None, None) == 3
+    st = D.dark_state(f, f, None, 2, 1, 64, 32, 5)     # d mismatch
+    assert lib.dark_decode_step(ctypes.byref(p), ctypes.byref(st), f, f, f, f, None, None, None) == 1
+    st = D.dark_state(f + 4, f, None, 2, 1, 64, 64, 5)  # kv not 16-byte aligned
+    assert lib.dark_decode_step(ctypes.byref(p), ctypes.byref(st), f, f, f, f, None, None, None) == 1
+
+
+def test_workspace_query(D):
+    p = _fake_proj(D, m=256, d=64, heads=8)
+    n1 = D.dark_attention_workspace_bytes(p, 2, 8, 2048, D.DARK_CAUSAL)
+    n2 = D.dark_attention_workspace_bytes(p, 2, 8, 4096, D.DARK_CAUSAL)
+    assert n1 >= 256 and n2 > n1
+    assert D.dark_attention_workspace_bytes(p, 0, 8, 2048, 0) == 0

@@ -1,0 +1,127 @@
+"""Parity of the CUDA forward path (through the C ABI) with the fp64 oracle."""
+import numpy as np
+import pytest
+
+from oracle import dark_oracle as O
+from random_feature_linear_b200 import synth
+
+from gpu_run import check, forward
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def D(cuda_ok):
+    from random_feature_linear_b200 import dark
+    return dark
+
+
+def _oracle(inp, causal):
+    return O.attention(inp["q"], inp["k"], inp["v"], inp["omega"], inp["geom"],
+                       key_mask=inp["mask"], causal=causal)
+
+
+# Small versions of the five workload recipes: several 128-token tiles plus a
+# ragged tail, so every tile kind and the tail path run.
+SMALL = {
+    "c1": synth.WORKLOADS[1],
+    "c1-causal": synth.WORKLOADS[1].with_sizes(causal=True, L=300, B=2, H=2),
+    "c1-masked": synth.WORKLOADS[1].with_sizes(L=200, B=2, lengths=(200, 77)),
+    "c2": synth.WORKLOADS[2].with_sizes(H=2, L=300, lengths=(300, 217)),
+    "c3": synth.WORKLOADS[3].with_sizes(H=3, L=700),
+    "c4": synth.WORKLOADS[4].with_sizes(B=1, H=2, L=300),
+    "c5-prefill": synth.WORKLOADS[5].with_sizes(B=3, H=2, L=333),
+    "c2-noncausal": synth.WORKLOADS[2].with_sizes(H=2, L=260, lengths=(260, 131), causal=False),
+    "c3-causal": synth.WORKLOADS[3].with_sizes(H=2, L=385, causal=True),
+}
+
+
+@pytest.mark.parametrize("name", list(SMALL))
+def test_forward_matches_oracle(D, cuda_ok, name):
+    w = SMALL[name]
+    inp = synth.make_inputs(w)
+    res = forward(D, w, inp, cuda_ok, with_state=True)
+    assert res["status"] == 0
+    out, kv, z = _oracle(inp, w.causal)
+    check(w, res["out"], out)
+    # state over all valid keys: relative to the largest entry of each head
+    for got, ref in ((res["kv"], kv), (res["z"], z)):
+        scale = np.abs(ref).reshape(ref.shape[0], ref.shape[1], -1).max(axis=2)
+        err = np.abs(got - ref).reshape(scale.shape + (-1,)).max(axis=2) / scale
+        assert err.max() <= (1e-4 if w.dtype == "f32" else 2e-2), err.max()
+
+
+def test_strided_inputs(D, cuda_ok):
+    w = synth.WORKLOADS[2].with_sizes(H=2, L=200, lengths=(200, 150))
+    inp = synth.make_inputs(w)
+    res = forward(D, w, inp, cuda_ok, strided=True)
+    out, _, _ = _oracle(inp, True)
+    check(w, res["out"], out)
+
+
+@pytest.mark.parametrize("name", ["c1-causal", "c2", "c3"])
+def test_stabiliser_changes_nothing(D, cuda_ok, name):
+    w = SMALL[name]
+    inp = synth.make_inputs(w)
+    flags = (D.DARK_CAUSAL if w.causal else 0) | D.DARK_STABILISE
+    res = forward(D, w, inp, cuda_ok, flags=flags, with_state=True)
+    assert res["status"] == 0
+    out, kv, z = _oracle(inp, w.causal)
+    check(w, res["out"], out)
+    # the stabilised state is the true one times 2^{-shift}
+    sc = np.exp2(-res["shift"])[:, :, None]
+    zs = z * sc
+    assert np.abs(res["z"] - zs).max() <= 2e-2 * np.abs(zs).max()
+
+
+def test_stabiliser_avoids_overflow(D, cuda_ok):
+    # Query/key norms large enough that 2^exponent overflows fp32 without the
+    # stabiliser; with it, outputs stay finite and match the oracle.
+    w = synth.WORKLOADS[1].with_sizes(L=130, causal=True)
+    inp = synth.make_inputs(w)
+    inp = dict(inp, q=inp["q"] * 6.0, k=inp["k"] * 6.0)
+    lo, hi = O.exponent_range(inp["q"][0, 0], inp["omega"][0], inp["geom"][0])
+    res = forward(D, w, inp, cuda_ok, flags=D.DARK_CAUSAL | D.DARK_STABILISE)
+    assert res["status"] == 0
+    out, _, _ = _oracle(inp, True)
+    err = np.abs(res["out"] - out).max() / np.abs(out).max()
+    assert err < 1e-3
+
+
+def test_rows_without_valid_keys_are_zero(D, cuda_ok):
+    w = synth.WORKLOADS[2].with_sizes(H=2, L=257, lengths=(0, 3))
+    inp = synth.make_inputs(w)
+    res = forward(D, w, inp, cuda_ok)
+    assert res["status"] == 0
+    out, _, _ = _oracle(inp, True)
+    assert np.all(res["out"][0] == 0)
+    check(w, res["out"], out)
+
+
+@pytest.mark.parametrize("L", [1, 2, 127, 128, 129])
+def test_short_sequences(D, cuda_ok, L):
+    for base in (synth.WORKLOADS[2].with_sizes(H=2, lengths=None), synth.WORKLOADS[3].with_sizes(H=2)):
+        w = base.with_sizes(L=L)
+        inp = synth.make_inputs(w)
+        res = forward(D, w, inp, cuda_ok)
+        out, _, _ = _oracle(inp, w.causal)
+        check(w, res["out"], out)
+
+
+def test_shared_and_per_head_geometry_agree_when_equal(D, cuda_ok):
+    w = synth.WORKLOADS[2].with_sizes(H=3, L=150, lengths=None)
+    inp = synth.make_inputs(w)
+    shared = dict(inp, geom=inp["geom"][:1])
+    tiled = dict(inp, geom=np.repeat(inp["geom"][:1], 3, axis=0))
+    a = forward(D, w, shared, cuda_ok)["out"]
+    b = forward(D, w, tiled, cuda_ok)["out"]
+    np.testing.assert_array_equal(a, b)
+
+
+def test_workspace_reuse_is_deterministic(D, cuda_ok):
+    w = SMALL["c2"]
+    inp = synth.make_inputs(w)
+    r1 = forward(D, w, inp, cuda_ok)
+    r2 = forward(D, w, inp, cuda_ok, ws=r1["ws"])
+    np.testing.assert_array_equal(r1["out"], r2["out"])
+    assert r1["ws"][:256].count_nonzero().item() == 0
