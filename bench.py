@@ -1,0 +1,363 @@
+"""Benchmark of the DARKformer PRF attention forward pass on B200.
+
+Default workload: causal, key-masked bf16 attention, B=2 H=8 L=2048 d=64 r=64
+m=256 with orthogonal features and valid lengths 2048/1500 (the standard
+workload of the method's causal path; seeded synthetic inputs).
+
+One JSON line on rank 0. `value` is whole-job forward tokens/s (B*H*L per
+step, summed over ranks) with inputs resident in HBM and L2 flushed before
+every timed step; `e2e` is the same metric through the C ABI with pinned host
+buffers, host->device and device->host copies inside the timed region.
+`--impl reference` times the fp64 CPU oracle on the host cores instead.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+import torch.distributed as dist
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from random_feature_linear_b200 import synth  # noqa: E402
+
+L2_FLUSH_BYTES = 512 << 20        # > 126 MB L2
+
+
+def alg_flops(w: synth.Workload) -> float:
+    """Algorithmic FLOPs of one forward pass: per head 2Ldm (query features) +
+    2Ld(m+r) (key features and norms) + 2Lm(d+1) (state) + 2Lm(d+1) (output)."""
+    per_head = (2 * w.L * w.d * w.m + 2 * w.L * w.d * (w.m + w.r) + 4 * w.L * w.m * (w.d + 1))
+    return float(per_head * w.B * w.H)
+
+
+def alg_bytes(w: synth.Workload) -> float:
+    """Algorithmic HBM bytes: q, k, v read and out written once, plus the mask."""
+    elt = 2 if w.dtype == "bf16" else 4
+    return float(4 * w.B * w.H * w.L * w.d * elt + (w.B * w.L if w.lengths else 0))
+
+
+def load_peaks() -> dict:
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return dict(hbm=d["hbm_gbs"], bf16=d["bf16_tflops"], source="measured")
+    return dict(hbm=6650.0, bf16=1590.0, source="fallback")
+
+
+class ClockSampler:
+    """Samples SM clocks and throttle reasons with nvidia-smi while running."""
+
+    def __init__(self, index: int):
+        self.index = index
+        self.rows = []
+        self.proc = None
+        self.thread = None
+
+    def __enter__(self):
+        q = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+             "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+             "clocks_event_reasons.sw_power_cap")
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={q}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+            return self
+
+        def read():
+            for line in self.proc.stdout:
+                self.rows.append([x.strip() for x in line.split(",")])
+        self.thread = threading.Thread(target=read, daemon=True)
+        self.thread.start()
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            self.proc.wait(timeout=5)
+
+    def summary(self) -> dict:
+        rows = [r for r in self.rows if len(r) == 7 and r[0].replace(".", "").isdigit()]
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
+        sm = [float(r[0]) for r in rows]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[3 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": float(rows[0][1]),
+                "reasons": reasons, "samples": len(rows)}
+
+
+def oracle_sample(w: synth.Workload, inp: dict, max_seconds: float = 20.0):
+    """Times the fp64 oracle on whole (batch, head) slices of the workload until
+    about `max_seconds` of CPU work; returns (tokens/s, tokens, seconds, heads)."""
+    from oracle import dark_oracle as O
+    done_tokens, t_total, heads = 0, 0.0, 0
+    for b in range(w.B):
+        for h in range(w.H):
+            sl = (slice(b, b + 1), slice(h, h + 1))
+            geom = inp["geom"][h:h + 1] if inp["geom"].shape[0] > 1 else inp["geom"]
+            mask = None if inp["mask"] is None else inp["mask"][b:b + 1]
+            t0 = time.perf_counter()
+            O.attention(inp["q"][sl], inp["k"][sl], inp["v"][sl], inp["omega"], geom,
+                        key_mask=mask, causal=w.causal)
+            t_total += time.perf_counter() - t0
+            done_tokens += w.L
+            heads += 1
+            if t_total > max_seconds:
+                return done_tokens / t_total, done_tokens, t_total, heads
+    return done_tokens / t_total, done_tokens, t_total, heads
+
+
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return 1
+
+
+def count_launches(fn) -> tuple[int, list]:
+    """Kernels of the native library launched by one call of fn (CUPTI via torch.profiler)."""
+    from torch.profiler import ProfilerActivity, profile
+    with profile(activities=[ProfilerActivity.CUDA]) as prof:
+        fn()
+        torch.cuda.synchronize()
+    names = [e.name for e in prof.events() if e.device_type == torch.autograd.DeviceType.CUDA]
+    ours = [n for n in names if "dark::" in n]
+    return len(ours), sorted(set(ours))
+
+
+def run_native(args, w: synth.Workload, rank: int, world: int, dev) -> dict | None:
+    from random_feature_linear_b200 import dark as D
+    inp = synth.make_inputs(w, salt=rank)
+    dt = D.DARK_BF16 if w.dtype == "bf16" else D.DARK_F32
+    tdt = D.torch_dtype(dt)
+    omega = torch.from_numpy(inp["omega"]).to(dev)
+    geom = torch.from_numpy(inp["geom"]).to(dev)
+    proj, _wbuf = D.dark_make_projection(omega, geom, w.H, dt)
+    q, k, v = (torch.from_numpy(inp[n]).to(dev).to(tdt) for n in ("q", "k", "v"))
+    mask = None if inp["mask"] is None else torch.from_numpy(inp["mask"]).to(dev)
+    out = torch.empty_like(q)
+    flags = D.DARK_CAUSAL if w.causal else 0
+    ws = D.alloc_workspace(proj, w.B, w.H, w.L, flags, dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    flush = None if args.ncu else torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.int32, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        D.dark_attention_fwd(proj, q, k, v, out, w.B, w.H, w.L, key_mask=mask, flags=flags,
+                             ws=ws, dev_status=status)
+
+    if args.ncu:
+        # capture mode for Nsight Compute: the forward calls only (ncu flushes
+        # caches itself before every replayed kernel)
+        for _ in range(args.warmup + args.steps):
+            step()
+        torch.cuda.synchronize()
+        assert int(status.item()) == 0, D.dark_status_string(int(status.item()))
+        return None
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    if args.no_profile:
+        launches_per_step, kernel_names = 1, ["(not counted: --no-profile)"]
+    else:
+        launches_per_step, kernel_names = count_launches(step)
+
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(dev.index) as clk:
+        wall0 = time.perf_counter()
+        for i in range(args.steps):
+            flush.zero_()                       # L2 flush, outside the timed interval
+            starts[i].record(stream)
+            step()
+            ends[i].record(stream)
+        torch.cuda.synchronize()
+        wall = time.perf_counter() - wall0
+    if world > 1:
+        dist.barrier()
+    step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    total_ms = torch.tensor([sum(step_ms)], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(total_ms, op=dist.ReduceOp.MAX)
+    ms_per_step = total_ms.item() / args.steps
+    assert int(status.item()) == 0, D.dark_status_string(int(status.item()))
+
+    # end to end through the C ABI with pinned host buffers
+    hq, hk, hv = (t.cpu().pin_memory() for t in (q, k, v))
+    hmask = None if mask is None else mask.cpu().pin_memory()
+    hout = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    dmask = None if mask is None else torch.empty_like(mask)
+
+    def e2e_step():
+        dq.copy_(hq, non_blocking=True)
+        dk.copy_(hk, non_blocking=True)
+        dv.copy_(hv, non_blocking=True)
+        if dmask is not None:
+            dmask.copy_(hmask, non_blocking=True)
+        D.dark_attention_fwd(proj, dq, dk, dv, out, w.B, w.H, w.L, key_mask=dmask, flags=flags,
+                             ws=ws, dev_status=status)
+        hout.copy_(out, non_blocking=True)
+
+    for _ in range(args.warmup):
+        e2e_step()
+    torch.cuda.synchronize()
+    e_start, e_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    e_start.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    e_end.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = torch.tensor([e_start.elapsed_time(e_end) / args.steps], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(e2e_ms, op=dist.ReduceOp.MAX)
+    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv)) + (
+        0 if hmask is None else hmask.numel())
+    d2h = hout.numel() * hout.element_size()
+
+    if rank != 0:
+        return None
+    tokens = w.tokens * world
+    peaks = load_peaks()
+    t_kernel = ms_per_step / 1e3            # one launch per step on the tensor-core path
+    flops = alg_flops(w)
+    nbytes = alg_bytes(w)
+    t_tc = flops / (peaks["bf16"] * 1e12)
+    t_hbm = nbytes / (peaks["hbm"] * 1e9)
+    bound = "tensor" if t_tc >= t_hbm else "hbm"
+    if bound == "tensor":
+        achieved = flops / t_kernel / 1e12
+        roof = dict(bound="tensor", achieved=achieved, peak=peaks["bf16"], unit="TFLOP/s",
+                    frac=achieved / peaks["bf16"], traffic=None)
+    else:
+        achieved = nbytes / t_kernel / 1e9
+        roof = dict(bound="hbm", achieved=achieved, peak=peaks["hbm"], unit="GB/s",
+                    frac=achieved / peaks["hbm"], traffic=None)
+    roof["peak_source"] = peaks["source"] + " (burst)"
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        tps, ntok, secs, heads = oracle_sample(w, inp)
+        cpu = dict(value=tps, unit="tokens/s", cores=blas_threads(), kind="oracle",
+                   sample=f"{heads} of {w.B * w.H} (batch, head) slices, {ntok} tokens, {secs:.1f} s")
+    clocks = clk.summary()
+    return {
+        "metric": "DARK attention fwd tokens/s (B*H*L/s) on B200",
+        "value": tokens / (ms_per_step / 1e3),
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms_per_step,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16" if w.dtype == "bf16" else "f32",
+        "data": "synthetic (seeded numpy, orthogonal Gaussian features)",
+        "config": {"workload": w.name, "B": w.B, "H": w.H, "L": w.L, "d": w.d, "r": w.r, "m": w.m,
+                   "causal": w.causal, "lengths": list(w.lengths) if w.lengths else None,
+                   "l2": "flushed (512 MiB write) before every timed step",
+                   "parallelism": f"replicas x{world} (independent batches, no collective)"},
+        "e2e": {"value": tokens / (e2e_ms.item() / 1e3), "unit": "tokens/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "roofline": roof,
+        "roofline_other": {"t_tensor_us": t_tc * 1e6, "t_hbm_us": t_hbm * 1e6,
+                           "alg_flops": flops, "alg_bytes": nbytes},
+        "cpu_baseline": cpu,
+        "gpu_launches": launches_per_step * args.steps,
+        "kernels": kernel_names,
+        "clocks": {"sm_mhz": clocks["sm_mhz"], "sm_max_mhz": clocks["sm_max_mhz"],
+                   "reasons": clocks["reasons"]},
+        "wall_s": wall,
+        "step_ms_min": min(step_ms),
+    }
+
+
+def run_reference(args, w: synth.Workload) -> dict:
+    inp = synth.make_inputs(w)
+    for _ in range(args.warmup):
+        oracle_sample(w, inp, max_seconds=1.0)
+    vals, details = [], None
+    for _ in range(args.steps):
+        tps, ntok, secs, heads = oracle_sample(w, inp, max_seconds=args.ref_seconds)
+        vals.append(tps)
+        details = (ntok, secs, heads)
+    value = statistics.median(vals)
+    cores = blas_threads()
+    sample = f"{details[2]} of {w.B * w.H} (batch, head) slices per step, {details[0]} tokens"
+    return {
+        "impl": "reference",
+        "metric": "DARK attention fwd tokens/s (B*H*L/s) on B200",
+        "value": value, "unit": "tokens/s", "n_gpus": 1, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": w.tokens / value * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded numpy, orthogonal Gaussian features)",
+        "config": {"workload": w.name, "B": w.B, "H": w.H, "L": w.L, "d": w.d, "r": w.r,
+                   "m": w.m, "causal": w.causal},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["native", "reference"], default="native")
+    ap.add_argument("--workload", type=int, default=2, help="synthetic workload recipe (1-5)")
+    ap.add_argument("--ref-seconds", type=float, default=10.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-profile", action="store_true",
+                    help="do not count launches with the CUDA profiler (for runs under ncu)")
+    ap.add_argument("--ncu", action="store_true",
+                    help="capture mode: only warmup + steps forward calls, no timing or output")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+    w = synth.WORKLOADS[args.workload]
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args, w)), flush=True)
+        return
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+    try:
+        res = run_native(args, w, rank, world, dev)
+        if res is not None:
+            print(json.dumps(res), flush=True)
+    finally:
+        if world > 1:
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -67,10 +67,13 @@ enum {
  *   c_w = d^{-1/4} * log2(e),  c_m = d^{-1/4} * sqrt(log2(e)/2),
  * so that, for a raw token x, (W' x)_j is the feature exponent omega_j^T M x~
  * in base 2 and sum_i (W' x)_{m+i}^2 is 1/2 x~^T Sigma x~ in base 2.
- * DARK_F32: one fp32 plane. DARK_BF16: two bf16 planes [2][heads][m + r][d],
- * hi = bf16(W') and lo = bf16(W' - hi); kernels use hi + lo, which keeps the
- * exponents accurate to about 2^-16 relative (a single bf16 plane, 2^-9, moves
- * the exponent of large features by ~1e-2 and the outputs by ~3e-2).
+ * Element type of W': fp32 for DARK_F32 projections; fp16 (IEEE binary16)
+ * for DARK_BF16 projections. fp16's 11 significant bits keep the exponents of
+ * the largest features accurate to ~2e-3 (bf16's 8 bits would move them by
+ * ~1e-2 and causal outputs by ~3e-2, beyond bf16 I/O tolerance). Entries of W'
+ * must stay below 65504 in magnitude; the tensor-core kernels also convert bf16
+ * q and k to fp16 for the feature GEMM, so |q|, |k| must stay below 65504
+ * (a larger value is reported as DARK_ERR_NUMERIC).
  * `heads` is 1 when Omega and M are both shared by all heads, else H.
  * `generation` is unique per dark_make_projection call in this process.
  */
@@ -113,13 +116,12 @@ size_t dark_projection_bytes(int heads, int m, int r, int d, dark_dtype dtype);
  *   omega       device fp32 [heads_omega][m][r]; heads_omega in {1, H}
  *   geom        device fp32 [heads_geom][r][d];  heads_geom  in {1, H}
  *   H           number of attention heads (>= 1)
- *   dtype       DARK_BF16 or DARK_F32: the element type of W' and of the
- *               tokens this projection will be used with
+ *   dtype       DARK_BF16 or DARK_F32: the element type of the tokens this
+ *               projection will be used with (W' is fp16 or fp32, see above)
  *   w_buf       device, w_bytes >= dark_projection_bytes(heads, ...), 16-byte
  *               aligned; heads = max(heads_omega, heads_geom)
- *               (for DARK_BF16 its size is 2 * heads * (m + r) * d * 2 bytes)
  *   out         host struct filled on success (w = w_buf, a new generation)
- * Products are accumulated in fp64, then rounded to `dtype` (hi/lo for bf16).
+ * Products are accumulated in fp64 and rounded once to W's element type.
  * Calling it again (a redraw) gives a new generation: states made with the
  * old projection are rejected by dark_decode_step.
  * Supported sizes: 4 <= d <= 256 with d a multiple of 4, 1 <= r <= 256,

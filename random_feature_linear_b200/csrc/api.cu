@@ -70,8 +70,7 @@ const char* dark_status_string(dark_status s) {
 
 size_t dark_projection_bytes(int heads, int m, int r, int d, dark_dtype dtype) {
   if (heads < 1 || m < 1 || r < 1 || d < 1 || !dtype_ok(dtype)) return 0;
-  const size_t planes = dtype == DARK_BF16 ? 2 : 1;
-  return planes * (size_t)heads * (size_t)(m + r) * (size_t)d * elt(dtype);
+  return (size_t)heads * (size_t)(m + r) * (size_t)d * elt(dtype);
 }
 
 dark_status dark_make_projection(const float* omega, int heads_omega, const float* geom,

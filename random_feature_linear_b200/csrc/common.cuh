@@ -3,6 +3,7 @@
 
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <stdint.h>
 
 #include "../../include/dark.h"
@@ -16,12 +17,19 @@ constexpr double kLog2e = 1.4426950408889634073599246810019;
 
 __device__ __forceinline__ float to_f32(float x) { return x; }
 __device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
+__device__ __forceinline__ float to_f32(__half x) { return __half2float(x); }
+
+// Element type of the projection buffer W' for token type T: fp32 tokens use an
+// fp32 W'; bf16 tokens use an fp16 W' (11 significant bits for the exponents).
+template <typename T> struct WeightOf { using type = float; };
+template <> struct WeightOf<__nv_bfloat16> { using type = __half; };
 
 template <typename T> __device__ __forceinline__ T from_f32(float x);
 template <> __device__ __forceinline__ float from_f32<float>(float x) { return x; }
 template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) {
   return __float2bfloat16_rn(x);
 }
+template <> __device__ __forceinline__ __half from_f32<__half>(float x) { return __float2half_rn(x); }
 
 // Records the first device-side error of a call; later errors are dropped.
 __device__ __forceinline__ void report(int* dev_status, int code) {

@@ -18,9 +18,8 @@ namespace {
 constexpr int kThreads = 256;
 constexpr int kBatchRows = 8;   // state rows loaded per thread before their update
 
-__device__ __forceinline__ void row_dot2(const float* __restrict__ w, size_t /*lo*/, int d,
-                                         const float* xk, const float* xq, bool both, float& ak,
-                                         float& aq) {
+__device__ __forceinline__ void row_dot2(const float* __restrict__ w, int d, const float* xk,
+                                         const float* xq, bool both, float& ak, float& aq) {
   float sk = 0.f, sq = 0.f;
   if ((d & 3) == 0) {
     const float4* w4 = reinterpret_cast<const float4*>(w);
@@ -43,24 +42,18 @@ __device__ __forceinline__ void row_dot2(const float* __restrict__ w, size_t /*l
   aq = sq;
 }
 
-// bf16 projections: the weight is hi + lo, the lo plane `lo` elements after hi.
-__device__ __forceinline__ void row_dot2(const __nv_bfloat16* __restrict__ w, size_t lo, int d,
-                                         const float* xk, const float* xq, bool both, float& ak,
-                                         float& aq) {
+// fp16 projection rows (the weight type of bf16 tokens).
+__device__ __forceinline__ void row_dot2(const __half* __restrict__ w, int d, const float* xk,
+                                         const float* xq, bool both, float& ak, float& aq) {
   float sk = 0.f, sq = 0.f;
   if ((d & 7) == 0) {
     const uint4* w8 = reinterpret_cast<const uint4*>(w);
-    const uint4* l8 = reinterpret_cast<const uint4*>(w + lo);
     for (int c = 0; c < d / 8; ++c) {
       const uint4 u = __ldg(w8 + c);
-      const uint4 ul = __ldg(l8 + c);
-      const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&u);
-      const __nv_bfloat162* pl = reinterpret_cast<const __nv_bfloat162*>(&ul);
+      const __half2* p = reinterpret_cast<const __half2*>(&u);
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        const float2 fh = __bfloat1622float2(p[e]);
-        const float2 fl = __bfloat1622float2(pl[e]);
-        const float2 f = make_float2(fh.x + fl.x, fh.y + fl.y);
+        const float2 f = __half22float2(p[e]);
         sk = fmaf(f.x, xk[8 * c + 2 * e], sk);
         sk = fmaf(f.y, xk[8 * c + 2 * e + 1], sk);
         if (both) {
@@ -71,7 +64,7 @@ __device__ __forceinline__ void row_dot2(const __nv_bfloat16* __restrict__ w, si
     }
   } else {
     for (int c = 0; c < d; ++c) {
-      const float f = __bfloat162float(w[c]) + __bfloat162float(w[c + lo]);
+      const float f = __half2float(w[c]);
       sk = fmaf(f, xk[c], sk);
       if (both) sq = fmaf(f, xq[c], sq);
     }
@@ -102,7 +95,8 @@ __device__ __forceinline__ float block_max(float v, float* scratch) {
 
 template <typename T>
 __global__ void __launch_bounds__(kThreads) decode_kernel(
-    const T* __restrict__ w, int heads_w, int m, int r, int d, float* __restrict__ kv,
+    const typename WeightOf<T>::type* __restrict__ w, int heads_w, int m, int r, int d,
+    float* __restrict__ kv,
     float* __restrict__ z, const float* __restrict__ shift, int H, const T* __restrict__ q,
     const T* __restrict__ k, const T* __restrict__ v, T* __restrict__ out,
     const uint8_t* __restrict__ valid, int* dev_status) {
@@ -117,7 +111,7 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(
   float* red = pq + m;                    // [rpp][d]
   float* scratch = red + rpp * d;         // [32]
   const int bh = blockIdx.x, b = bh / H, h = bh % H;
-  const T* wh = w + (size_t)(heads_w == 1 ? 0 : h) * (m + r) * d;
+  const auto* wh = w + (size_t)(heads_w == 1 ? 0 : h) * (m + r) * d;
   const int tid = threadIdx.x;
 
   for (int c = tid; c < d; c += kThreads) {
@@ -128,7 +122,7 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(
   __syncthreads();
   for (int j = tid; j < m + r; j += kThreads) {
     float ak, aq;
-    row_dot2(wh + (size_t)j * d, (size_t)heads_w * (m + r) * d, d, xk, xq, j < m, ak, aq);
+    row_dot2(wh + (size_t)j * d, d, xk, xq, j < m, ak, aq);
     pk[j] = ak;
     if (j < m) pq[j] = aq;
   }
@@ -205,7 +199,7 @@ cudaError_t launch_decode(const DecodeArgs& a) {
                                cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (err != cudaSuccess) return err;
     decode_kernel<__nv_bfloat16><<<a.B * a.H, kThreads, smem, a.stream>>>(
-        (const __nv_bfloat16*)a.w, a.heads_w, a.m, a.r, a.d, a.kv, a.z, a.shift, a.H,
+        (const __half*)a.w, a.heads_w, a.m, a.r, a.d, a.kv, a.z, a.shift, a.H,
         (const __nv_bfloat16*)a.q, (const __nv_bfloat16*)a.k, (const __nv_bfloat16*)a.v,
         (__nv_bfloat16*)a.out, a.valid, a.dev_status);
   } else {

@@ -12,8 +12,7 @@
 
 namespace dark {
 
-// bf16 projections hold two planes (hi, then lo = the rounding residual of hi);
-// fp32 projections hold one plane.
+// TW: fp32 for fp32 projections, fp16 for bf16 projections.
 template <typename T>
 __global__ void projection_kernel(const float* __restrict__ omega, int heads_omega,
                                   const float* __restrict__ geom, int heads_geom, int heads_w,
@@ -32,12 +31,7 @@ __global__ void projection_kernel(const float* __restrict__ omega, int heads_ome
     } else {
       val = cm * (double)gm[(size_t)(row - m) * d + c];
     }
-    const T hi = from_f32<T>((float)val);
-    dst[c] = hi;
-    if (sizeof(T) == 2) {
-      const size_t plane = (size_t)heads_w * (m + r) * d;
-      dst[plane + c] = from_f32<T>((float)(val - (double)to_f32(hi)));
-    }
+    dst[c] = sizeof(T) == 2 ? T(__double2half(val)) : from_f32<T>((float)val);
   }
 }
 
@@ -50,8 +44,8 @@ cudaError_t launch_projection(const float* omega, int heads_omega, const float* 
   dim3 grid(m + r, heads_w);
   const int threads = d < 256 ? ((d + 31) / 32) * 32 : 256;
   if (dtype == DARK_BF16)
-    projection_kernel<__nv_bfloat16><<<grid, threads, 0, stream>>>(
-        omega, heads_omega, geom, heads_geom, heads_w, m, r, d, cw, cm, (__nv_bfloat16*)w);
+    projection_kernel<__half><<<grid, threads, 0, stream>>>(
+        omega, heads_omega, geom, heads_geom, heads_w, m, r, d, cw, cm, (__half*)w);
   else
     projection_kernel<float><<<grid, threads, 0, stream>>>(omega, heads_omega, geom, heads_geom,
                                                            heads_w, m, r, d, cw, cm, (float*)w);

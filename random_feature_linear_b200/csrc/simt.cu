@@ -60,7 +60,7 @@ __global__ void init_ck_kernel(int* ck, int n) {
 template <typename T>
 __global__ void __launch_bounds__(256) features_kernel(
     const T* __restrict__ xq, const T* __restrict__ xk, int64_t sb, int64_t sh, int64_t sl,
-    const T* __restrict__ w, size_t lo_plane, int heads_w, int m, int r, int d, int H, int L,
+    const typename WeightOf<T>::type* __restrict__ w, int heads_w, int m, int r, int d, int H, int L,
     const uint8_t* __restrict__ mask, int stabilise, float* __restrict__ phiq,
     float* __restrict__ phik, int* __restrict__ ck) {
   extern __shared__ float sm[];
@@ -73,7 +73,7 @@ __global__ void __launch_bounds__(256) features_kernel(
   const T* x = side ? xk : xq;
   const int ncols = side ? m + r : m;
   const int ld = m + r;
-  const T* wh = w + (size_t)(heads_w == 1 ? 0 : h) * (m + r) * d;
+  const auto* wh = w + (size_t)(heads_w == 1 ? 0 : h) * (m + r) * d;
 
   for (int e = threadIdx.x; e < kTF * d; e += blockDim.x) {
     const int tt = e / d, c = e % d, t = t0 + tt;
@@ -84,10 +84,9 @@ __global__ void __launch_bounds__(256) features_kernel(
     float acc[kTF];
 #pragma unroll
     for (int tt = 0; tt < kTF; ++tt) acc[tt] = 0.f;
-    const T* wr = wh + (size_t)j * d;
+    const auto* wr = wh + (size_t)j * d;
     for (int c = 0; c < d; ++c) {
-      // bf16 projections: hi plane + lo plane (lo_plane elements further on)
-      const float wv = lo_plane ? to_f32(wr[c]) + to_f32(wr[c + lo_plane]) : to_f32(wr[c]);
+      const float wv = to_f32(wr[c]);
 #pragma unroll
       for (int tt = 0; tt < kTF; ++tt) acc[tt] = fmaf(wv, xs[tt * d + c], acc[tt]);
     }
@@ -406,8 +405,8 @@ cudaError_t simt_forward_t(const FwdArgs& a) {
   err = cudaFuncSetAttribute(features_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)fsm);
   if (err != cudaSuccess) return err;
   features_kernel<T><<<dim3((a.L + kTF - 1) / kTF, bh, 2), 256, fsm, a.stream>>>(
-      (const T*)a.q, (const T*)a.k, a.qs[0], a.qs[1], a.qs[2], (const T*)a.w,
-      sizeof(T) == 2 ? (size_t)a.heads_w * (a.m + a.r) * a.d : 0, a.heads_w, a.m,
+      (const T*)a.q, (const T*)a.k, a.qs[0], a.qs[1], a.qs[2],
+      (const typename WeightOf<T>::type*)a.w, a.heads_w, a.m,
       a.r, a.d, a.H, a.L, a.mask, stab, phiq, phik, ck);
   if (stab) {
     const size_t n = (size_t)bh * a.L * a.m;

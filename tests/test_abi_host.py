@@ -41,7 +41,7 @@ def test_version_and_status_strings(D):
 
 
 def test_projection_bytes(D):
-    assert D.dark_projection_bytes(8, 256, 64, 64, D.DARK_BF16) == 2 * 8 * 320 * 64 * 2
+    assert D.dark_projection_bytes(8, 256, 64, 64, D.DARK_BF16) == 8 * 320 * 64 * 2
     assert D.dark_projection_bytes(1, 64, 64, 64, D.DARK_F32) == 128 * 64 * 4
     assert D.dark_projection_bytes(0, 64, 64, 64, D.DARK_F32) == 0
 
