@@ -32,7 +32,7 @@ bool proj_ok(const dark_projection* p) {
 
 enum class Path { Simt, TcCausal, TcNonCausal };
 
-Path choose_path(const dark::FwdArgs& a) {
+Path choose_path(dark::FwdArgs& a) {
   if (a.flags & DARK_CAUSAL) {
     if (dark::tc_causal_supported(a)) return Path::TcCausal;
   } else {
@@ -50,6 +50,80 @@ size_t ws_need(Path p, int B, int H, int L, int m, int d, int flags) {
 }
 
 }  // namespace
+
+namespace dark {
+
+dark_status fwd_prepare(const dark_projection* proj, const void* q, const void* k, const void* v,
+                        void* out, const int64_t* qkv_strides, const int64_t* out_strides, int B,
+                        int H, int L, const uint8_t* key_mask, int flags,
+                        const dark_state* state_out, int* dev_status, void* stream, FwdArgs* out_args) {
+  if (proj == nullptr || proj->w == nullptr || !aligned(proj->w, 16) || !dtype_ok(proj->dtype))
+    return DARK_ERR_INVALID_ARG;
+  if (proj->m < 1 || proj->r < 1 || proj->d < 1) return DARK_ERR_INVALID_ARG;
+  if (!sizes_ok(proj->m, proj->r, proj->d)) return DARK_ERR_UNSUPPORTED;
+  if (q == nullptr || k == nullptr || v == nullptr || out == nullptr) return DARK_ERR_INVALID_ARG;
+  if (B < 1 || H < 1 || L < 1) return DARK_ERR_INVALID_ARG;
+  if (!(proj->heads == 1 || proj->heads == H)) return DARK_ERR_INVALID_ARG;
+  if (flags & ~(DARK_CAUSAL | DARK_STABILISE)) return DARK_ERR_INVALID_ARG;
+  FwdArgs& a = *out_args;
+  memset(&a, 0, sizeof(a));
+  a.heads_w = proj->heads;
+  a.m = proj->m;
+  a.r = proj->r;
+  a.d = proj->d;
+  a.dtype = proj->dtype;
+  a.w = proj->w;
+  a.q = q;
+  a.k = k;
+  a.v = v;
+  a.out = out;
+  const int64_t d = proj->d;
+  const int64_t contig[3] = {(int64_t)H * L * d, (int64_t)L * d, d};
+  for (int i = 0; i < 3; ++i) {
+    a.qs[i] = qkv_strides ? qkv_strides[i] : contig[i];
+    a.os[i] = out_strides ? out_strides[i] : contig[i];
+    if (a.qs[i] < 0 || a.os[i] < 0) return DARK_ERR_INVALID_ARG;
+  }
+  a.B = B;
+  a.H = H;
+  a.L = L;
+  a.mask = key_mask;
+  a.flags = flags;
+  if (state_out != nullptr) {
+    if (state_out->kv == nullptr || state_out->z == nullptr || state_out->B != B ||
+        state_out->H != H || state_out->m != proj->m || state_out->d != proj->d)
+      return DARK_ERR_INVALID_ARG;
+    if ((flags & DARK_STABILISE) && state_out->shift == nullptr) return DARK_ERR_INVALID_ARG;
+    a.st_kv = state_out->kv;
+    a.st_z = state_out->z;
+    a.st_shift = (flags & DARK_STABILISE) ? state_out->shift : nullptr;
+  }
+  a.dev_status = dev_status;
+  a.stream = (cudaStream_t)stream;
+  a.path = (int)choose_path(a);   // may encode the TMA descriptors into `a`
+  return DARK_OK;
+}
+
+size_t fwd_workspace_need(const FwdArgs& a) {
+  return ws_need((Path)a.path, a.B, a.H, a.L, a.m, a.d, a.flags);
+}
+
+dark_status fwd_launch(FwdArgs& a, void* ws, size_t ws_bytes, dark_state* state_out,
+                       uint64_t generation) {
+  a.ws = ws;
+  a.ws_bytes = ws_bytes;
+  cudaError_t e;
+  switch ((Path)a.path) {
+    case Path::TcCausal: e = tc_causal_forward(a); break;
+    case Path::TcNonCausal: e = tc_noncausal_forward(a); break;
+    default: e = simt_forward(a); break;
+  }
+  if (e != cudaSuccess) return DARK_ERR_CUDA;
+  if (state_out != nullptr) state_out->generation = generation;
+  return DARK_OK;
+}
+
+}  // namespace dark
 
 extern "C" {
 
@@ -115,65 +189,13 @@ dark_status dark_attention_fwd(const dark_projection* proj, const void* q, const
                                const int64_t* out_strides, int B, int H, int L,
                                const uint8_t* key_mask, int flags, dark_state* state_out,
                                void* ws, size_t ws_bytes, int* dev_status, void* stream) {
-  if (proj == nullptr || proj->w == nullptr || !aligned(proj->w, 16) || !dtype_ok(proj->dtype))
-    return DARK_ERR_INVALID_ARG;
-  if (proj->m < 1 || proj->r < 1 || proj->d < 1) return DARK_ERR_INVALID_ARG;
-  if (!sizes_ok(proj->m, proj->r, proj->d)) return DARK_ERR_UNSUPPORTED;
-  if (q == nullptr || k == nullptr || v == nullptr || out == nullptr) return DARK_ERR_INVALID_ARG;
-  if (B < 1 || H < 1 || L < 1) return DARK_ERR_INVALID_ARG;
-  if (!(proj->heads == 1 || proj->heads == H)) return DARK_ERR_INVALID_ARG;
-  if (flags & ~(DARK_CAUSAL | DARK_STABILISE)) return DARK_ERR_INVALID_ARG;
   if (ws == nullptr || !aligned(ws, 256)) return DARK_ERR_INVALID_ARG;
-
   dark::FwdArgs a;
-  memset(&a, 0, sizeof(a));
-  a.heads_w = proj->heads;
-  a.m = proj->m;
-  a.r = proj->r;
-  a.d = proj->d;
-  a.dtype = proj->dtype;
-  a.w = proj->w;
-  a.q = q;
-  a.k = k;
-  a.v = v;
-  a.out = out;
-  const int64_t d = proj->d;
-  const int64_t contig[3] = {(int64_t)H * L * d, (int64_t)L * d, d};
-  for (int i = 0; i < 3; ++i) {
-    a.qs[i] = qkv_strides ? qkv_strides[i] : contig[i];
-    a.os[i] = out_strides ? out_strides[i] : contig[i];
-    if (a.qs[i] < 0 || a.os[i] < 0) return DARK_ERR_INVALID_ARG;
-  }
-  a.B = B;
-  a.H = H;
-  a.L = L;
-  a.mask = key_mask;
-  a.flags = flags;
-  if (state_out != nullptr) {
-    if (state_out->kv == nullptr || state_out->z == nullptr || state_out->B != B ||
-        state_out->H != H || state_out->m != proj->m || state_out->d != proj->d)
-      return DARK_ERR_INVALID_ARG;
-    if ((flags & DARK_STABILISE) && state_out->shift == nullptr) return DARK_ERR_INVALID_ARG;
-    a.st_kv = state_out->kv;
-    a.st_z = state_out->z;
-    a.st_shift = (flags & DARK_STABILISE) ? state_out->shift : nullptr;
-  }
-  a.ws = ws;
-  a.ws_bytes = ws_bytes;
-  a.dev_status = dev_status;
-  a.stream = (cudaStream_t)stream;
-
-  const Path p = choose_path(a);
-  if (ws_bytes < ws_need(p, B, H, L, a.m, a.d, flags)) return DARK_ERR_INVALID_ARG;
-  cudaError_t e;
-  switch (p) {
-    case Path::TcCausal: e = dark::tc_causal_forward(a); break;
-    case Path::TcNonCausal: e = dark::tc_noncausal_forward(a); break;
-    default: e = dark::simt_forward(a); break;
-  }
-  if (e != cudaSuccess) return DARK_ERR_CUDA;
-  if (state_out != nullptr) state_out->generation = proj->generation;
-  return DARK_OK;
+  const dark_status st = dark::fwd_prepare(proj, q, k, v, out, qkv_strides, out_strides, B, H, L,
+                                           key_mask, flags, state_out, dev_status, stream, &a);
+  if (st != DARK_OK) return st;
+  if (ws_bytes < dark::fwd_workspace_need(a)) return DARK_ERR_INVALID_ARG;
+  return dark::fwd_launch(a, ws, ws_bytes, state_out, proj->generation);
 }
 
 dark_status dark_state_init(const dark_projection* proj, dark_state* st, void* stream) {

@@ -16,7 +16,7 @@ namespace dark {
 namespace {
 
 constexpr int kThreads = 256;
-constexpr int kBatchRows = 8;   // state rows loaded per thread before their update
+constexpr int kBatchRows = 16;  // state rows held in registers per thread and pass
 
 __device__ __forceinline__ void row_dot2(const float* __restrict__ w, int d, const float* xk,
                                          const float* xq, bool both, float& ak, float& aq) {
@@ -96,9 +96,8 @@ __device__ __forceinline__ float block_max(float v, float* scratch) {
 template <typename T>
 __global__ void __launch_bounds__(kThreads) decode_kernel(
     const typename WeightOf<T>::type* __restrict__ w, int heads_w, int m, int r, int d,
-    float* __restrict__ kv,
-    float* __restrict__ z, const float* __restrict__ shift, int H, const T* __restrict__ q,
-    const T* __restrict__ k, const T* __restrict__ v, T* __restrict__ out,
+    float* __restrict__ kv, float* __restrict__ z, const float* __restrict__ shift, int H,
+    const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v, T* __restrict__ out,
     const uint8_t* __restrict__ valid, int* dev_status) {
   extern __shared__ float sm[];
   const int tpr = d / 4;                  // threads per state row (one float4 each)
@@ -113,6 +112,27 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(
   const int bh = blockIdx.x, b = bh / H, h = bh % H;
   const auto* wh = w + (size_t)(heads_w == 1 ? 0 : h) * (m + r) * d;
   const int tid = threadIdx.x;
+  const int c4 = tid % tpr, r0 = tid / tpr;
+  const bool rows_active = r0 < rpp;
+  float4* base = reinterpret_cast<float4*>(kv + (size_t)bh * m * d) + c4;
+  const int stride = d / 4;
+
+  // The state rows of the first pass are requested before anything else so
+  // that their HBM latency overlaps the feature computation below.
+  float4 s[kBatchRows];
+  if (rows_active) {
+#pragma unroll
+    for (int u = 0; u < kBatchRows; ++u) {
+      const int j = r0 + u * rpp;
+      if (j < m) s[u] = __ldcs(base + (size_t)j * stride);
+    }
+  }
+  float zpre[4];
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    const int j = tid + u * kThreads;
+    zpre[u] = j < m ? __ldcs(z + (size_t)bh * m + j) : 0.f;
+  }
 
   for (int c = tid; c < d; c += kThreads) {
     xq[c] = to_f32(q[(size_t)bh * d + c]);
@@ -143,17 +163,15 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(
 
   // kv' = kv + phi(k) v^T and num = phi(q)^T kv', one float4 column group per thread.
   float4 num = make_float4(0.f, 0.f, 0.f, 0.f);
-  const int c4 = tid % tpr, r0 = tid / tpr;
-  if (r0 < rpp) {
+  if (rows_active) {
     const float4 vv = make_float4(xv[4 * c4], xv[4 * c4 + 1], xv[4 * c4 + 2], xv[4 * c4 + 3]);
-    float4* base = reinterpret_cast<float4*>(kv + (size_t)bh * m * d) + c4;
-    const int stride = d / 4;
     for (int j0 = r0; j0 < m; j0 += rpp * kBatchRows) {
-      float4 s[kBatchRows];
+      if (j0 != r0) {
 #pragma unroll
-      for (int u = 0; u < kBatchRows; ++u) {
-        const int j = j0 + u * rpp;
-        if (j < m) s[u] = base[(size_t)j * stride];
+        for (int u = 0; u < kBatchRows; ++u) {
+          const int j = j0 + u * rpp;
+          if (j < m) s[u] = __ldcs(base + (size_t)j * stride);
+        }
       }
 #pragma unroll
       for (int u = 0; u < kBatchRows; ++u) {
@@ -162,7 +180,7 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(
           const float fk = pk[j], fq = pq[j];
           s[u].x = fmaf(fk, vv.x, s[u].x); s[u].y = fmaf(fk, vv.y, s[u].y);
           s[u].z = fmaf(fk, vv.z, s[u].z); s[u].w = fmaf(fk, vv.w, s[u].w);
-          base[(size_t)j * stride] = s[u];
+          __stcs(base + (size_t)j * stride, s[u]);
           num.x = fmaf(fq, s[u].x, num.x); num.y = fmaf(fq, s[u].y, num.y);
           num.z = fmaf(fq, s[u].z, num.z); num.w = fmaf(fq, s[u].w, num.w);
         }
@@ -172,7 +190,16 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(
     rr[0] = num.x; rr[1] = num.y; rr[2] = num.z; rr[3] = num.w;
   }
   float den = 0.f;
-  for (int j = tid; j < m; j += kThreads) {
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    const int j = tid + u * kThreads;
+    if (j < m) {
+      const float zj = zpre[u] + pk[j];
+      __stcs(z + (size_t)bh * m + j, zj);
+      den = fmaf(pq[j], zj, den);
+    }
+  }
+  for (int j = tid + 4 * kThreads; j < m; j += kThreads) {
     const float zj = z[(size_t)bh * m + j] + pk[j];
     z[(size_t)bh * m + j] = zj;
     den = fmaf(pq[j], zj, den);
@@ -195,16 +222,16 @@ cudaError_t launch_decode(const DecodeArgs& a) {
   const size_t smem = sizeof(float) * (3 * a.d + (a.m + a.r) + a.m + rpp * a.d + 32);
   cudaError_t err;
   if (a.dtype == DARK_BF16) {
-    err = cudaFuncSetAttribute(decode_kernel<__nv_bfloat16>,
-                               cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    static int done[64];
+    err = set_smem_limit_once((const void*)decode_kernel<__nv_bfloat16>, (int)smem, done);
     if (err != cudaSuccess) return err;
     decode_kernel<__nv_bfloat16><<<a.B * a.H, kThreads, smem, a.stream>>>(
         (const __half*)a.w, a.heads_w, a.m, a.r, a.d, a.kv, a.z, a.shift, a.H,
         (const __nv_bfloat16*)a.q, (const __nv_bfloat16*)a.k, (const __nv_bfloat16*)a.v,
         (__nv_bfloat16*)a.out, a.valid, a.dev_status);
   } else {
-    err = cudaFuncSetAttribute(decode_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               (int)smem);
+    static int done[64];
+    err = set_smem_limit_once((const void*)decode_kernel<float>, (int)smem, done);
     if (err != cudaSuccess) return err;
     decode_kernel<float><<<a.B * a.H, kThreads, smem, a.stream>>>(
         (const float*)a.w, a.heads_w, a.m, a.r, a.d, a.kv, a.z, a.shift, a.H, (const float*)a.q,

@@ -5,6 +5,8 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include <cuda.h>
+
 #include "../../include/dark.h"
 
 namespace dark {
@@ -25,6 +27,10 @@ struct FwdArgs {
   size_t ws_bytes;
   int* dev_status;
   cudaStream_t stream;
+  // TMA descriptors of W', q, k, v, encoded once per call by tc_make_maps
+  CUtensorMap tm_w, tm_q, tm_k, tm_v;
+  bool maps_ready;
+  int path;                       // kernel path chosen by fwd_prepare
 };
 
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -33,6 +39,16 @@ inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 // at first use, restored to zero by the kernels that use them); kernel data
 // of every path starts after it.
 constexpr size_t kWsHeader = 256;
+
+// The forward call in three steps: validate and choose the kernel path (no
+// device work), report the workspace that path needs, enqueue it.
+dark_status fwd_prepare(const dark_projection* proj, const void* q, const void* k, const void* v,
+                        void* out, const int64_t* qkv_strides, const int64_t* out_strides, int B,
+                        int H, int L, const uint8_t* key_mask, int flags,
+                        const dark_state* state_out, int* dev_status, void* stream, FwdArgs* a);
+size_t fwd_workspace_need(const FwdArgs& a);
+dark_status fwd_launch(FwdArgs& a, void* ws, size_t ws_bytes, dark_state* state_out,
+                       uint64_t generation);
 
 // Projection W' = [c_w Omega M ; c_m M] (one-off, fp64 accumulation).
 cudaError_t launch_projection(const float* omega, int heads_omega, const float* geom,
@@ -45,11 +61,20 @@ cudaError_t simt_forward(const FwdArgs& a);
 
 // Tensor-core forward paths (tcgen05/TMEM/TMA). `*_supported` says whether the
 // sizes, layout and alignment fit; the launchers assume they do.
-bool tc_causal_supported(const FwdArgs& a);
+// Alignment/stride/shape checks shared by the tensor-core paths, then the
+// TMA descriptors (false if any check fails or the driver rejects a layout).
+bool tc_make_maps(FwdArgs& a);
+// Sets a kernel's dynamic shared memory limit once per device.
+cudaError_t set_smem_limit_once(const void* kernel, int bytes, int* done_per_device);
+
+bool tc_causal_supported(FwdArgs& a);
 size_t tc_causal_workspace_bytes(int B, int H, int L, int m, int d);
 cudaError_t tc_causal_forward(const FwdArgs& a);
 
-bool tc_noncausal_supported(const FwdArgs& a);
+bool tc_noncausal_supported(FwdArgs& a);
+// Per-range key states Phi(K)^T [V | 1] as fp32 [B*H*nsplit][65][m] (tcgen05).
+cudaError_t tc_launch_key_states(const FwdArgs& a, const CUtensorMap& tw, const CUtensorMap& tk,
+                                 const CUtensorMap& tv, int ntiles, int nsplit, float* partials);
 size_t tc_noncausal_workspace_bytes(int B, int H, int L, int m, int d);
 cudaError_t tc_noncausal_forward(const FwdArgs& a);
 

@@ -14,20 +14,23 @@
 //   TMA loads of W', Q_c, K_c, V_c (128B-swizzled tiles)
 //   -> tcgen05 feature GEMMs K_c W'^T, Q_c W^T (fp16 operands, fp32 in TMEM)
 //   -> epilogue warps: key norm, exp2, key mask, bf16 Phi/Psi tiles in smem
-//   -> tcgen05 GEMMs Psi Phi^T (scores) and Phi^T [V | 1] (chunk state)
-//   -> causal mask of the scores -> intra GEMM tril(A) [V | 1]
-//   -> prefix state (hi/lo bf16 split) -> inter GEMM Psi [S | z] -> divide.
-// Phi and Psi never leave shared memory. The prefix state across chunks is
-// carried in registers when one CTA walks all chunks of a head (many heads),
-// or exchanged between CTAs by a decoupled look-back over per-chunk aggregates
-// in the workspace (few heads); every wait there is bounded and a wait that
-// runs out reports DARK_ERR_TIMEOUT instead of hanging.
-#include <atomic>
+//   -> tcgen05 GEMM Psi Phi^T (scores) -> causal mask -> intra GEMM tril(A) [V | 1]
+//   -> inter GEMM Psi [S_<c | z_<c] with the prefix split into hi + lo bf16
+//      (bf16 alone moves outputs by ~1e-2) -> divide.
+// Phi and Psi never leave shared memory. Every CTA walks a segment of
+// consecutive chunks of one head and carries the prefix state in registers,
+// adding Phi(K_c)^T [V_c | 1] after each chunk. With many heads (B*H >= #SMs)
+// a segment is the whole head; with few heads each head is cut into G
+// segments so that all SMs work, and two small launches come first: the
+// key-state kernel sums Phi(K)^T [V | 1] over each segment and a scan turns
+// the segment sums into exclusive prefixes in a fixed order (deterministic,
+// no waiting between blocks).
 #include <string.h>
 
 #include "common.cuh"
 #include "internal.h"
 #include "tc_common.cuh"
+#include "tc_keys.cuh"
 
 namespace dark {
 namespace {
@@ -36,12 +39,10 @@ using namespace tc;
 
 constexpr int kD = 64;          // head dimension handled by this kernel
 constexpr int kC = 128;         // tokens per chunk (UMMA M)
-constexpr int kThreads = 256;
+constexpr int kThreads = kFwdThreads;
 constexpr int kSms = 148;
 constexpr int kTileBytes = kC * kD * 2;   // one 128 x 64 tile of 16-bit elements
 constexpr uint32_t kTmemCols = 512;
-
-std::atomic<uint64_t> g_call{0};
 
 template <int M_, int R_>
 struct Cfg {
@@ -73,21 +74,11 @@ struct Params {
   const uint8_t* mask;
   int B, H, L, nc;              // nc = chunks per head
   int heads_w;
-  int lookback;                 // 1: one chunk per CTA + look-back; 0: one head per CTA
-  uint32_t* ticket;             // workspace header word
-  uint64_t* flags;              // [B*H*nc] look-back flags
-  float* slots;                 // [B*H*nc][2][65][m] aggregates / inclusive prefixes
-  float *st_kv, *st_z;
-  uint64_t call;
+  int nseg;                     // segments per head
+  const float* seg_prefix;      // [B*H*nseg][65][m] exclusive segment prefixes (nseg > 1)
+  float *st_kv, *st_z;          // state after the last chunk
   int* dev_status;
 };
-
-__device__ __forceinline__ bool wait_all(uint64_t* bar, uint32_t parity, int* dev_status) {
-  const bool ok = mbar_wait(bar, parity);
-  const int bad = __syncthreads_or(ok ? 0 : 1);
-  if (bad && threadIdx.x == 0) report(dev_status, DARK_ERR_TIMEOUT);
-  return bad == 0;
-}
 
 template <int M_, int R_>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -101,12 +92,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* bar_tma = (uint64_t*)(sm + G::oBar);
   uint64_t* bar_mma = bar_tma + 1;
   uint32_t* tmem_slot = (uint32_t*)(bar_tma + 2);
-  int* s_int = (int*)(bar_tma + 3);           // [0]: ticket, [1]: look-back state
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int quad = warp & 3, half = warp >> 2;
   const int row = quad * 32 + lane;           // TMEM lane = tile row of this thread
-  const bool has_feat = half < G::MB;         // owns state row `feat`
+  const bool has_feat = half < G::MB;         // owns prefix-state row `feat`
   const int feat = half * 128 + row;
 
   if (tid == 0) {
@@ -117,13 +107,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     prefetch_tmap(&tm_q);
     prefetch_tmap(&tm_k);
     prefetch_tmap(&tm_v);
-    if (p.lookback) {
-      const uint32_t t = atomicAdd(p.ticket, 1u);
-      if (t == gridDim.x - 1) atomicExch(p.ticket, 0u);   // every block has its ticket
-      s_int[0] = (int)t;
-    } else {
-      s_int[0] = blockIdx.x;
-    }
   }
   __syncwarp();
   if (warp == 0) tmem_alloc(tmem_slot, kTmemCols);
@@ -135,34 +118,30 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const uint32_t lane_tm = tmem + ((uint32_t)(quad * 32) << 16);
-  const int unit = s_int[0];
-  int bh, c_begin, c_end;
-  if (p.lookback) {
-    bh = unit / p.nc;
-    c_begin = unit % p.nc;
-    c_end = c_begin + 1;
-  } else {
-    bh = unit;
-    c_begin = 0;
-    c_end = p.nc;
-  }
+  const int bh = blockIdx.x / p.nseg, seg = blockIdx.x % p.nseg;
+  const int c_begin = (int)((long long)seg * p.nc / p.nseg);
+  const int c_end = (int)((long long)(seg + 1) * p.nc / p.nseg);
   const int b = bh / p.H, h = bh % p.H;
   const int hw = p.heads_w == 1 ? 0 : h;
 
   uint32_t ph_tma = 0, ph_mma = 0;
   float run[65];                               // prefix state row `feat` (fp32)
+  if (has_feat && seg > 0) {
+    const float* sp = p.seg_prefix + (size_t)blockIdx.x * 65 * M_;
 #pragma unroll
-  for (int i = 0; i < 65; ++i) run[i] = 0.f;
+    for (int i = 0; i < 65; ++i) run[i] = sp[(size_t)i * M_ + feat];
+  } else {
+#pragma unroll
+    for (int i = 0; i < 65; ++i) run[i] = 0.f;
+  }
   bool abort = false;
 
   for (int c = c_begin; c < c_end && !abort; ++c) {
     const int t0 = c * kC;
     // ---------------------------------------------------------------- loads
     if (tid == 0) {
-      const bool load_w = (c == c_begin) || !p.lookback;
-      mbar_arrive_expect_tx(bar_tma, (load_w ? G::kW : 0) + 3 * kTileBytes);
-      if (load_w)
-        for (int r0 = 0; r0 < G::NW; r0 += 16)
+      mbar_arrive_expect_tx(bar_tma, G::kW + 3 * kTileBytes);
+      for (int r0 = 0; r0 < G::NW; r0 += 16)
           tma_load_2d(sm + G::oW + r0 * 128, &tm_w, 0, hw * G::NW + r0, bar_tma);
       tma_load_4d(sm + G::oK, &tm_k, 0, t0, h, b, bar_tma);
       tma_load_4d(sm + G::oV, &tm_v, 0, t0, h, b, bar_tma);
@@ -170,25 +149,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     if (!wait_all(bar_tma, ph_tma, p.dev_status)) { abort = true; break; }
     ph_tma ^= 1;
-    // q, k: bf16 -> fp16 in place (the feature GEMM runs on fp16 operands)
-    {
-      bool bad = false;
-      for (int i = tid; i < 2 * kTileBytes / 16; i += kThreads) {
-        const uint32_t a = s0 + G::oQ + i * 16;        // Q then K (contiguous)
-        uint4 u = ld_shared_v4(a);
-        uint32_t* w32 = &u.x;
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const __nv_bfloat162 bv = *reinterpret_cast<const __nv_bfloat162*>(&w32[e]);
-          const float2 f = __bfloat1622float2(bv);
-          bad |= fabsf(f.x) > 65504.f || fabsf(f.y) > 65504.f;
-          const __half2 hv = __floats2half2_rn(f.x, f.y);
-          w32[e] = *reinterpret_cast<const uint32_t*>(&hv);
-        }
-        st_shared_v4(a, u.x, u.y, u.z, u.w);
-      }
-      if (bad) report(p.dev_status, DARK_ERR_NUMERIC);
-    }
+    // k, then q: bf16 -> fp16 in place (the feature GEMMs run on fp16 operands);
+    // the key GEMM starts while the query tile converts
+    to_fp16_inplace(s0 + G::oK, kTileBytes, p.dev_status);
     fence_async_smem();
     __syncthreads();
     // ------------------------------------------------------- feature GEMM K
@@ -205,6 +168,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       mma_commit(bar_mma);
     }
+    to_fp16_inplace(s0 + G::oQ, kTileBytes, p.dev_status);
+    fence_async_smem();
     if (!wait_all(bar_mma, ph_mma, p.dev_status)) { abort = true; break; }
     ph_mma ^= 1;
     tc_fence_after();
@@ -231,8 +196,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           uint32_t w4[4];
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            const float a = valid ? ex2(v[8 * g + 2 * e] - nrm) : 0.f;
-            const float bb = valid ? ex2(v[8 * g + 2 * e + 1] - nrm) : 0.f;
+            // values 5..7 of each group of 8 go through the FMA pipe
+            const float x0 = v[8 * g + 2 * e] - nrm, x1 = v[8 * g + 2 * e + 1] - nrm;
+            const float a = valid ? (2 * e >= 5 ? ex2_fma(x0) : ex2(x0)) : 0.f;
+            const float bb = valid ? (2 * e + 1 >= 5 ? ex2_fma(x1) : ex2(x1)) : 0.f;
             w4[e] = pack_bf16(a, bb);
           }
           const int f = f0 + 8 * g;
@@ -265,7 +232,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int g = 0; g < 4; ++g) {
         uint32_t w4[4];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) w4[e] = pack_bf16(ex2(v[8 * g + 2 * e]), ex2(v[8 * g + 2 * e + 1]));
+        for (int e = 0; e < 4; ++e) {
+          const float x0 = v[8 * g + 2 * e], x1 = v[8 * g + 2 * e + 1];
+          w4[e] = pack_bf16(2 * e >= 5 ? ex2_fma(x0) : ex2(x0), 2 * e + 1 >= 5 ? ex2_fma(x1) : ex2(x1));
+        }
         st_shared_v4(s0 + G::oPsi + kmajor_off(row, f0 + 8 * g, 16384), w4[0], w4[1], w4[2], w4[3]);
       }
     }
@@ -345,66 +315,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         mma(tmem + G::tNum + 64, ad, sdesc(s0 + G::oOnes + (s % 4) * 32, 16, 1024), id1, s > 0);
       }
     }
-    // ---------------------------------------------------------- prefix state
-    bool have_prefix;
-    if (p.lookback) {
-      const size_t unit_idx = (size_t)bh * p.nc + c;
-      float* slot_agg = p.slots + unit_idx * 2 * 65 * M_;
-      float* slot_inc = slot_agg + 65 * M_;
-      // publish the aggregate (chunk 0: it is already the inclusive prefix)
-      if (has_feat) {
-        float* dst = c == 0 ? slot_inc : slot_agg;
-#pragma unroll
-        for (int i = 0; i < 65; ++i) __stcg(dst + i * M_ + feat, ds[i]);
-      }
-      __threadfence();
-      __syncthreads();
-      if (tid == 0) st_release_u64(p.flags + unit_idx, (p.call << 2) | (c == 0 ? 2u : 1u));
-      // look back over the predecessors of this chunk
-      for (int pc = c - 1; pc >= 0; --pc) {
-        if (tid == 0) {
-          const uint64_t* fl = p.flags + (size_t)bh * p.nc + pc;
-          uint64_t f = ld_acquire_u64(fl);
-          const long long start = clock64();
-          while ((f >> 2) != p.call || (f & 3) == 0) {
-            if (clock64() - start > kWaitCycles) { f = 0; break; }
-            __nanosleep(64);
-            f = ld_acquire_u64(fl);
-          }
-          if (f == 0) report(p.dev_status, DARK_ERR_TIMEOUT);
-          s_int[1] = (int)(f & 3);
-        }
-        __syncthreads();
-        const int st = s_int[1];
-        __syncthreads();
-        if (st == 0) break;
-        const float* src = p.slots + ((size_t)bh * p.nc + pc) * 2 * 65 * M_ + (st == 2 ? 65 * M_ : 0);
-        if (has_feat) {
-#pragma unroll
-          for (int i = 0; i < 65; ++i) run[i] += __ldcg(src + i * M_ + feat);
-        }
-        if (st == 2) break;
-      }
-      have_prefix = c > 0;
-      // publish the inclusive prefix
-      if (c > 0) {
-        if (has_feat) {
-#pragma unroll
-          for (int i = 0; i < 65; ++i) __stcg(slot_inc + i * M_ + feat, run[i] + ds[i]);
-        }
-        __threadfence();
-        __syncthreads();
-        if (tid == 0) st_release_u64(p.flags + unit_idx, (p.call << 2) | 2u);
-      }
-      if (c == p.nc - 1 && p.st_kv != nullptr && has_feat) {
-        float* kv = p.st_kv + ((size_t)bh * M_ + feat) * kD;
-#pragma unroll
-        for (int i = 0; i < 64; ++i) kv[i] = run[i] + ds[i];
-        p.st_z[(size_t)bh * M_ + feat] = run[64] + ds[64];
-      }
-    } else {
-      have_prefix = c > 0;
-    }
+    const bool have_prefix = c > 0;
     // prefix [S | z] as hi + lo bf16 operands: S (MN-major) in the Phi region,
     // z (16 identical K-major rows) in the W' region
     if (have_prefix && has_feat) {
@@ -437,7 +348,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         st_shared_u16(zl_base + off, zlb);
       }
     }
-    if (!p.lookback && has_feat) {
+    if (has_feat) {
 #pragma unroll
       for (int i = 0; i < 65; ++i) run[i] += ds[i];
     }
@@ -493,7 +404,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_before();
     __syncthreads();
   }
-  if (!abort && !p.lookback && p.st_kv != nullptr && has_feat) {
+  if (!abort && p.st_kv != nullptr && has_feat && c_end == p.nc) {
     float* kv = p.st_kv + ((size_t)bh * M_ + feat) * kD;
 #pragma unroll
     for (int i = 0; i < 64; ++i) kv[i] = run[i];
@@ -507,19 +418,44 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
+// In place: segment sums of each head -> exclusive prefixes, in segment order.
+// All segment loads are issued before the dependent adds (at most kSms segments).
+__global__ void segment_scan_kernel(float* __restrict__ seg, int nseg, int m) {
+  const int bh = blockIdx.y;
+  const int idx = blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= 65 * m) return;
+  float* base = seg + (size_t)bh * nseg * 65 * m + idx;
+  const size_t step = (size_t)65 * m;
+  float run = 0.f;
+  for (int s0 = 0; s0 < nseg; s0 += 16) {
+    float t[16];
+#pragma unroll
+    for (int u = 0; u < 16; ++u) t[u] = s0 + u < nseg ? base[(s0 + u) * step] : 0.f;
+#pragma unroll
+    for (int u = 0; u < 16; ++u) {
+      if (s0 + u < nseg) {
+        base[(s0 + u) * step] = run;
+        run += t[u];
+      }
+    }
+  }
+}
+
 struct Layout {
-  int nc, lookback;
-  size_t off_flags, off_slots, total;
+  int nc, nseg;
+  size_t off_seg, total;
 };
 
+// Segments per head: 1 when the heads alone fill the SMs, else enough to give
+// every SM a segment (at most one per chunk).
 Layout layout(int B, int H, int L, int m) {
   Layout s;
+  const int bh = B * H;
   s.nc = (L + kC - 1) / kC;
-  s.lookback = (B * H < kSms) ? 1 : 0;
-  const size_t units = (size_t)B * H * s.nc;
-  s.off_flags = kWsHeader;
-  s.off_slots = align_up(s.off_flags + (s.lookback ? units * 8 : 0), 256);
-  s.total = align_up(s.off_slots + (s.lookback ? units * 2 * 65 * (size_t)m * 4 : 0), 256);
+  s.nseg = bh >= kSms ? 1 : kSms / bh;
+  if (s.nseg > s.nc) s.nseg = s.nc;
+  s.off_seg = kWsHeader;
+  s.total = align_up(s.off_seg + (s.nseg > 1 ? (size_t)bh * s.nseg * 65 * m * 4 : 0), 256);
   return s;
 }
 
@@ -528,6 +464,14 @@ cudaError_t launch(const FwdArgs& a, const CUtensorMap& tw, const CUtensorMap& t
                    const CUtensorMap& tk, const CUtensorMap& tv) {
   using G = Cfg<M_, R_>;
   const Layout s = layout(a.B, a.H, a.L, a.m);
+  const int bh = a.B * a.H;
+  float* seg = (float*)((char*)a.ws + s.off_seg);
+  cudaError_t e;
+  if (s.nseg > 1) {
+    e = tc_launch_key_states(a, tw, tk, tv, s.nc, s.nseg, seg);
+    if (e != cudaSuccess) return e;
+    segment_scan_kernel<<<dim3((65 * a.m + 255) / 256, bh), 256, 0, a.stream>>>(seg, s.nseg, a.m);
+  }
   Params p;
   memset(&p, 0, sizeof(p));
   p.out = (__nv_bfloat16*)a.out;
@@ -540,48 +484,26 @@ cudaError_t launch(const FwdArgs& a, const CUtensorMap& tw, const CUtensorMap& t
   p.L = a.L;
   p.nc = s.nc;
   p.heads_w = a.heads_w;
-  p.lookback = s.lookback;
-  p.ticket = (uint32_t*)a.ws;
-  p.flags = (uint64_t*)((char*)a.ws + s.off_flags);
-  p.slots = (float*)((char*)a.ws + s.off_slots);
+  p.nseg = s.nseg;
+  p.seg_prefix = seg;
   p.st_kv = a.st_kv;
   p.st_z = a.st_z;
-  p.call = ++g_call;
   p.dev_status = a.dev_status;
-  cudaError_t e = cudaFuncSetAttribute(causal_kernel<M_, R_>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)G::kSmem);
+  static int smem_set[64];
+  e = set_smem_limit_once((const void*)causal_kernel<M_, R_>, (int)G::kSmem, smem_set);
   if (e != cudaSuccess) return e;
-  const int grid = s.lookback ? a.B * a.H * s.nc : a.B * a.H;
-  causal_kernel<M_, R_><<<grid, kThreads, G::kSmem, a.stream>>>(tw, tq, tk, tv, p);
+  causal_kernel<M_, R_><<<bh * s.nseg, kThreads, G::kSmem, a.stream>>>(tw, tq, tk, tv, p);
   return cudaGetLastError();
 }
 
-bool make_maps(const FwdArgs& a, CUtensorMap* tw, CUtensorMap* tq, CUtensorMap* tk, CUtensorMap* tv) {
-  const uint64_t wd[2] = {(uint64_t)a.d, (uint64_t)a.heads_w * (a.m + a.r)};
-  const uint64_t ws[1] = {(uint64_t)a.d * 2};
-  const uint32_t wb[2] = {64, 16};
-  if (!encode_tmap(tw, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, a.w, wd, ws, wb)) return false;
-  const uint64_t xd[4] = {(uint64_t)a.d, (uint64_t)a.L, (uint64_t)a.H, (uint64_t)a.B};
-  const uint64_t xs[3] = {(uint64_t)a.qs[2] * 2, (uint64_t)a.qs[1] * 2, (uint64_t)a.qs[0] * 2};
-  const uint32_t xb[4] = {64, (uint32_t)kC, 1, 1};
-  return encode_tmap(tq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, a.q, xd, xs, xb) &&
-         encode_tmap(tk, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, a.k, xd, xs, xb) &&
-         encode_tmap(tv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, a.v, xd, xs, xb);
-}
 
-bool aligned16(const void* ptr) { return ((uintptr_t)ptr & 15) == 0; }
 
 }  // namespace
 
-bool tc_causal_supported(const FwdArgs& a) {
+bool tc_causal_supported(FwdArgs& a) {
   if (a.dtype != DARK_BF16 || a.d != kD || (a.flags & DARK_STABILISE)) return false;
   if (!(a.m == 128 || a.m == 256) || a.r % 16 != 0 || a.r < 16 || a.r > 64) return false;
-  if (!aligned16(a.q) || !aligned16(a.k) || !aligned16(a.v) || !aligned16(a.out) || !aligned16(a.w))
-    return false;
-  for (int i = 0; i < 3; ++i)
-    if (a.qs[i] % 8 != 0 || a.os[i] % 8 != 0) return false;
-  CUtensorMap t[4];
-  return make_maps(a, &t[0], &t[1], &t[2], &t[3]);
+  return tc_make_maps(a);
 }
 
 size_t tc_causal_workspace_bytes(int B, int H, int L, int m, int d) {
@@ -590,8 +512,8 @@ size_t tc_causal_workspace_bytes(int B, int H, int L, int m, int d) {
 }
 
 cudaError_t tc_causal_forward(const FwdArgs& a) {
-  CUtensorMap tw, tq, tk, tv;
-  if (!make_maps(a, &tw, &tq, &tk, &tv)) return cudaErrorInvalidValue;
+  if (!a.maps_ready) return cudaErrorInvalidValue;
+  const CUtensorMap &tw = a.tm_w, &tq = a.tm_q, &tk = a.tm_k, &tv = a.tm_v;
 #define DARK_CAUSAL_CASE(MM, RR) \
   if (a.m == MM && a.r == RR) return launch<MM, RR>(a, tw, tq, tk, tv);
   DARK_CAUSAL_CASE(256, 64)

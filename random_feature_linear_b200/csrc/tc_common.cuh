@@ -82,6 +82,15 @@ __device__ __forceinline__ void tma_load_4d(void* dst, const CUtensorMap* map, i
       "l"((uint64_t)map), "r"(x), "r"(y), "r"(z), "r"(w), "r"(smem_u32(bar))
       : "memory");
 }
+// Plain bulk copy global -> this CTA's shared memory (16-byte aligned, size a
+// multiple of 16), completing on `bar`.
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(dst)),
+      "l"((uint64_t)src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"((uint64_t)map) : "memory");
 }
@@ -194,6 +203,22 @@ __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+// 2^x on the FMA pipe, to take part of the exponentials off the MUFU unit:
+// n = round(x) from one add of 1.5 * 2^23 (n lands in the low mantissa bits),
+// 2^f for f = x - n in [-1/2, 1/2] from a cubic with 7.5e-5 maximum relative
+// error (coefficients fitted by exp2_poly.py), and 2^n added to the exponent
+// field. x is clamped to [-126, 128]: smaller results are below what bf16
+// operands keep; from 2^128 up the result saturates at ~3.4e38, the top of the
+// fp32 range (any product with it overflows in the fp32 accumulators).
+__device__ __forceinline__ float ex2_fma(float x) {
+  x = fminf(fmaxf(x, -126.f), 128.f);
+  const float big = 12582912.f;
+  const float t = x + big;
+  const float f = x - (t - big);
+  const float p = fmaf(fmaf(fmaf(0.0551716685295105f, f, 0.2426111251115799f), f,
+                            0.6932609677314758f), f, 0.9999280571937561f);
+  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
 }
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);

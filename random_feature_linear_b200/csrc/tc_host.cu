@@ -1,6 +1,7 @@
 // Host helper of the tensor-core kernels: tiled TMA descriptors.
 #include <cudaTypedefs.h>
 
+#include "internal.h"
 #include "tc_common.cuh"
 
 namespace dark {
@@ -31,6 +32,36 @@ bool encode_tmap(CUtensorMap* map, CUtensorMapDataType type, int rank, const voi
          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
+}
+
+bool tc_make_maps(FwdArgs& a) {
+  if (a.maps_ready) return true;
+  auto al16 = [](const void* p) { return ((uintptr_t)p & 15) == 0; };
+  if (a.dtype != DARK_BF16 || a.d != 64) return false;
+  if (!al16(a.q) || !al16(a.k) || !al16(a.v) || !al16(a.out) || !al16(a.w)) return false;
+  for (int i = 0; i < 3; ++i)
+    if (a.qs[i] % 8 != 0 || a.os[i] % 8 != 0) return false;
+  const uint64_t wd[2] = {(uint64_t)a.d, (uint64_t)a.heads_w * (a.m + a.r)};
+  const uint64_t wsd[1] = {(uint64_t)a.d * 2};
+  const uint32_t wb[2] = {64, 16};
+  const uint64_t xd[4] = {(uint64_t)a.d, (uint64_t)a.L, (uint64_t)a.H, (uint64_t)a.B};
+  const uint64_t xs[3] = {(uint64_t)a.qs[2] * 2, (uint64_t)a.qs[1] * 2, (uint64_t)a.qs[0] * 2};
+  const uint32_t xb[4] = {64, 128, 1, 1};
+  a.maps_ready = encode_tmap(&a.tm_w, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, a.w, wd, wsd, wb) &&
+                 encode_tmap(&a.tm_q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, a.q, xd, xs, xb) &&
+                 encode_tmap(&a.tm_k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, a.k, xd, xs, xb) &&
+                 encode_tmap(&a.tm_v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, a.v, xd, xs, xb);
+  return a.maps_ready;
+}
+
+cudaError_t set_smem_limit_once(const void* kernel, int bytes, int* done_per_device) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev >= 0 && dev < 64 && done_per_device[dev]) return cudaSuccess;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess && dev >= 0 && dev < 64) done_per_device[dev] = 1;
+  return e;
 }
 
 }  // namespace dark

@@ -1,0 +1,244 @@
+// Key-side tensor-core kernel shared by the forward paths: per range of
+// 128-token key tiles of one (batch, head), the chunk state
+// Phi(K)^T [V | 1] (DARKformer README, section "Kernel": the statistics
+// Phi(K)^T V and Phi(K)^T 1 of the associative form).
+//
+// Each CTA walks a contiguous tile range: TMA K/V tiles (double-buffered) ->
+// tcgen05 feature GEMM K W'^T (fp16 operands, fp32 in TMEM) -> epilogue: key
+// norm, exp2, key mask -> bf16 Phi tile in shared memory -> tcgen05 GEMM
+// Phi^T [V | 1] accumulated in TMEM over the range -> fp32 [65][m] partial
+// (column 64 is z). With one tile per range the partials are per-chunk
+// aggregates.
+#include "internal.h"
+#include "tc_keys.cuh"
+
+namespace dark {
+namespace {
+
+using namespace tc;
+
+constexpr int kD = 64;
+constexpr int kT = 128;
+constexpr int kThreads = kFwdThreads;
+constexpr int kTileBytes = kT * kD * 2;
+constexpr uint32_t kTmemCols = 512;
+
+struct KeyParams {
+  const uint8_t* mask;
+  int B, H, L, ntiles, nsplit, heads_w;
+  float* partials;                 // [B*H*nsplit][65][m]
+  int* dev_status;
+};
+
+template <int M_, int R_>
+struct KeyCfg {
+  static constexpr int NW = M_ + R_, MB = M_ / 128;
+  static constexpr uint32_t kW = NW * 128;
+  static constexpr uint32_t kPhi = (M_ / 64) * 16384;
+  static constexpr uint32_t oW = 0;
+  static constexpr uint32_t oK = (kW + 1023) / 1024 * 1024;   // 2 buffers
+  static constexpr uint32_t oV = oK + 2 * kTileBytes;         // 2 buffers
+  static constexpr uint32_t oPhi = oV + 2 * kTileBytes;
+  static constexpr uint32_t oOnes = oPhi + kPhi;
+  static constexpr uint32_t oBar = oOnes + 2048;
+  static constexpr uint32_t kSmem = oBar + 64 + 1024;
+  static constexpr uint32_t tP = 0, tD = 320;
+};
+
+template <int M_, int R_>
+__global__ void __launch_bounds__(kThreads, 1)
+    keys_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_k,
+                const __grid_constant__ CUtensorMap tm_v, const KeyParams p) {
+  using G = KeyCfg<M_, R_>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  const uint32_t s0 = smem_u32(sm);
+  uint64_t* bar_kv = (uint64_t*)(sm + G::oBar);     // [2]
+  uint64_t* bar_mma = bar_kv + 2;
+  uint32_t* tmem_slot = (uint32_t*)(bar_kv + 3);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int quad = warp & 3, half = warp >> 2;
+  const int row = quad * 32 + lane;
+  const int split = blockIdx.x, bh = blockIdx.y, b = bh / p.H, h = bh % p.H;
+  const int hw = p.heads_w == 1 ? 0 : h;
+  const int tb = (int)((long long)split * p.ntiles / p.nsplit);
+  const int te = (int)((long long)(split + 1) * p.ntiles / p.nsplit);
+
+  if (tid == 0) {
+    mbar_init(&bar_kv[0], 1);
+    mbar_init(&bar_kv[1], 1);
+    mbar_init(bar_mma, 1);
+    fence_mbar_init();
+    if (te > tb) {
+      mbar_arrive_expect_tx(&bar_kv[0], G::kW + 2 * kTileBytes);
+      for (int r0 = 0; r0 < G::NW; r0 += 16)
+        tma_load_2d(sm + G::oW + r0 * 128, &tm_w, 0, hw * G::NW + r0, &bar_kv[0]);
+      tma_load_4d(sm + G::oK, &tm_k, 0, tb * kT, h, b, &bar_kv[0]);
+      tma_load_4d(sm + G::oV, &tm_v, 0, tb * kT, h, b, &bar_kv[0]);
+    }
+  }
+  __syncwarp();
+  if (warp == 0) tmem_alloc(tmem_slot, kTmemCols);
+  for (int i = tid; i < 2048 / 4; i += kThreads) ((uint32_t*)(sm + G::oOnes))[i] = 0x3F803F80u;
+  fence_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t lane_tm = tmem + ((uint32_t)(quad * 32) << 16);
+
+  uint32_t ph_kv[2] = {0, 0}, ph_mma = 0;
+  bool abort = false;
+  for (int t = tb; t < te; ++t) {
+    const int i = t - tb, buf = i & 1;
+    if (!wait_all(&bar_kv[buf], ph_kv[buf], p.dev_status)) { abort = true; break; }
+    ph_kv[buf] ^= 1;
+    to_fp16_inplace(s0 + G::oK + buf * kTileBytes, kTileBytes, p.dev_status);
+    fence_async_smem();
+    __syncthreads();
+    if (tid == 0) {
+      tc_fence_after();
+      constexpr uint32_t idn0 = idesc(128, (G::NW < 256 ? G::NW : 256), false, false, true);
+      constexpr uint32_t idn1 = idesc(128, (G::NW > 256 ? G::NW - 256 : 16), false, false, true);
+#pragma unroll
+      for (int s = 0; s < kD / 16; ++s) {
+        const uint64_t ad = sdesc(s0 + G::oK + buf * kTileBytes + s * 32, 16, 1024);
+        mma(tmem + G::tP, ad, sdesc(s0 + G::oW + s * 32, 16, 1024), idn0, s > 0);
+        if (G::NW > 256)
+          mma(tmem + G::tP + 256, ad, sdesc(s0 + G::oW + 256 * 128 + s * 32, 16, 1024), idn1, s > 0);
+      }
+      mma_commit(bar_mma);
+    }
+    // this phase also covers the chunk-state GEMM of the previous tile
+    if (!wait_all(bar_mma, ph_mma, p.dev_status)) { abort = true; break; }
+    ph_mma ^= 1;
+    tc_fence_after();
+    // the other buffer is free now: prefetch the next tile into it
+    if (tid == 0 && t + 1 < te) {
+      const int nb = buf ^ 1;
+      mbar_arrive_expect_tx(&bar_kv[nb], 2 * kTileBytes);
+      tma_load_4d(sm + G::oK + nb * kTileBytes, &tm_k, 0, (t + 1) * kT, h, b, &bar_kv[nb]);
+      tma_load_4d(sm + G::oV + nb * kTileBytes, &tm_v, 0, (t + 1) * kT, h, b, &bar_kv[nb]);
+    }
+    {
+      float nrm = 0.f;
+#pragma unroll
+      for (int c0 = 0; c0 < R_; c0 += 16) {
+        float v[16];
+        tmem_ld16(lane_tm + G::tP + M_ + c0, v);
+#pragma unroll
+        for (int e = 0; e < 16; ++e) nrm = fmaf(v[e], v[e], nrm);
+      }
+      nrm += 0.5f * __log2f((float)M_);
+      const int tok = t * kT + row;
+      bool valid = tok < p.L;
+      if (valid && p.mask != nullptr) valid = p.mask[(size_t)b * p.L + tok] != 0;
+#pragma unroll 1
+      for (int f0 = half * (M_ / 2); f0 < (half + 1) * (M_ / 2); f0 += 32) {
+        float v[32];
+        tmem_ld32(lane_tm + G::tP + f0, v);
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+          uint32_t w4[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float a = valid ? ex2(v[8 * g + 2 * e] - nrm) : 0.f;
+            const float c = valid ? ex2(v[8 * g + 2 * e + 1] - nrm) : 0.f;
+            w4[e] = pack_bf16(a, c);
+          }
+          st_shared_v4(s0 + G::oPhi + kmajor_off(row, f0 + 8 * g, 16384), w4[0], w4[1], w4[2], w4[3]);
+        }
+      }
+    }
+    fence_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    if (tid == 0) {
+      tc_fence_after();
+      constexpr uint32_t idv = idesc(128, 64, true, true, false);
+      constexpr uint32_t id1 = idesc(128, 16, true, false, false);
+#pragma unroll
+      for (int mb = 0; mb < G::MB; ++mb) {
+#pragma unroll
+        for (int s = 0; s < kT / 16; ++s) {
+          const uint32_t acc = (t > tb || s > 0) ? 1u : 0u;
+          const uint64_t ad = sdesc(s0 + G::oPhi + mb * 32768 + s * 2048, 16384, 1024);
+          mma(tmem + G::tD + 80 * mb, ad, sdesc(s0 + G::oV + buf * kTileBytes + s * 2048, 16384, 1024),
+              idv, acc);
+          mma(tmem + G::tD + 80 * mb + 64, ad, sdesc(s0 + G::oOnes + (s % 4) * 32, 16, 1024), id1, acc);
+        }
+      }
+    }
+  }
+  if (!abort && te > tb) {
+    if (tid == 0) mma_commit(bar_mma);
+    if (!wait_all(bar_mma, ph_mma, p.dev_status)) abort = true;
+    tc_fence_after();
+  }
+  if (!abort && half < G::MB) {
+    const int f = half * 128 + row;
+    float* dst = p.partials + ((size_t)bh * p.nsplit + split) * 65 * M_;
+    if (te > tb) {
+      float v[32];
+      const uint32_t base = lane_tm + G::tD + 80 * half;
+      tmem_ld32(base, v);
+#pragma unroll
+      for (int e = 0; e < 32; ++e) dst[e * M_ + f] = v[e];
+      tmem_ld32(base + 32, v);
+#pragma unroll
+      for (int e = 0; e < 32; ++e) dst[(32 + e) * M_ + f] = v[e];
+      dst[64 * M_ + f] = tmem_ld1(base + 64);
+    } else {
+      for (int e = 0; e < 65; ++e) dst[e * M_ + f] = 0.f;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+
+template <int M_, int R_>
+cudaError_t launch_keys_t(const FwdArgs& a, const CUtensorMap& tw, const CUtensorMap& tk,
+                          const CUtensorMap& tv, int ntiles, int nsplit, float* partials) {
+  KeyParams kp;
+  kp.mask = a.mask;
+  kp.B = a.B;
+  kp.H = a.H;
+  kp.L = a.L;
+  kp.ntiles = ntiles;
+  kp.nsplit = nsplit;
+  kp.heads_w = a.heads_w;
+  kp.partials = partials;
+  kp.dev_status = a.dev_status;
+  using KG = KeyCfg<M_, R_>;
+  static int smem_set[64];
+  cudaError_t e = set_smem_limit_once((const void*)keys_kernel<M_, R_>, (int)KG::kSmem, smem_set);
+  if (e != cudaSuccess) return e;
+  keys_kernel<M_, R_><<<dim3(nsplit, a.B * a.H), kThreads, KG::kSmem, a.stream>>>(tw, tk, tv, kp);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t tc_launch_key_states(const FwdArgs& a, const CUtensorMap& tw, const CUtensorMap& tk,
+                                 const CUtensorMap& tv, int ntiles, int nsplit, float* partials) {
+#define DARK_KEYS_CASE(MM, RR) \
+  if (a.m == MM && a.r == RR) return launch_keys_t<MM, RR>(a, tw, tk, tv, ntiles, nsplit, partials);
+  DARK_KEYS_CASE(256, 64)
+  DARK_KEYS_CASE(256, 48)
+  DARK_KEYS_CASE(256, 32)
+  DARK_KEYS_CASE(256, 16)
+  DARK_KEYS_CASE(128, 64)
+  DARK_KEYS_CASE(128, 48)
+  DARK_KEYS_CASE(128, 32)
+  DARK_KEYS_CASE(128, 16)
+#undef DARK_KEYS_CASE
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace dark

@@ -1,0 +1,40 @@
+// Shared by the tensor-core forward kernels: bounded block-wide mbarrier wait
+// and the in-place bf16 -> fp16 conversion of a shared-memory operand tile.
+#pragma once
+
+#include "common.cuh"
+#include "tc_common.cuh"
+
+namespace dark {
+namespace tc {
+
+constexpr int kFwdThreads = 256;
+
+__device__ __forceinline__ bool wait_all(uint64_t* bar, uint32_t parity, int* dev_status) {
+  const bool ok = mbar_wait(bar, parity);
+  const int bad = __syncthreads_or(ok ? 0 : 1);
+  if (bad && threadIdx.x == 0) report(dev_status, DARK_ERR_TIMEOUT);
+  return bad == 0;
+}
+
+// bf16 -> fp16 in place for `bytes` of a shared tile (feature GEMM operand).
+__device__ __forceinline__ void to_fp16_inplace(uint32_t saddr, int bytes, int* dev_status) {
+  bool bad = false;
+  for (int i = threadIdx.x; i < bytes / 16; i += kFwdThreads) {
+    const uint32_t a = saddr + i * 16;
+    uint4 u = ld_shared_v4(a);
+    uint32_t* w32 = &u.x;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w32[e]));
+      bad |= fabsf(f.x) > 65504.f || fabsf(f.y) > 65504.f;
+      const __half2 hv = __floats2half2_rn(f.x, f.y);
+      w32[e] = *reinterpret_cast<const uint32_t*>(&hv);
+    }
+    st_shared_v4(a, u.x, u.y, u.z, u.w);
+  }
+  if (bad) report(dev_status, DARK_ERR_NUMERIC);
+}
+
+}  // namespace tc
+}  // namespace dark

@@ -19,6 +19,7 @@
 #include "common.cuh"
 #include "internal.h"
 #include "tc_common.cuh"
+#include "tc_keys.cuh"
 
 namespace dark {
 namespace {
@@ -27,7 +28,7 @@ using namespace tc;
 
 constexpr int kD = 64;
 constexpr int kT = 128;                     // tokens per tile
-constexpr int kThreads = 256;
+constexpr int kThreads = kFwdThreads;
 constexpr int kSms = 148;
 constexpr int kTileBytes = kT * kD * 2;
 constexpr uint32_t kTmemCols = 512;
@@ -37,210 +38,6 @@ constexpr uint32_t kTmemCols = 512;
 __host__ __device__ constexpr uint32_t img_s_bytes(int m) { return (uint32_t)m * 128; }
 __host__ __device__ constexpr uint32_t img_z_bytes(int m) { return (uint32_t)(m / 64) * 2048; }
 __host__ __device__ constexpr uint32_t img_bytes(int m) { return 2 * img_s_bytes(m) + 2 * img_z_bytes(m); }
-
-__device__ __forceinline__ bool wait_all(uint64_t* bar, uint32_t parity, int* dev_status) {
-  const bool ok = mbar_wait(bar, parity);
-  const int bad = __syncthreads_or(ok ? 0 : 1);
-  if (bad && threadIdx.x == 0) report(dev_status, DARK_ERR_TIMEOUT);
-  return bad == 0;
-}
-
-// bf16 -> fp16 in place for `bytes` of a shared tile (feature GEMM operand).
-__device__ __forceinline__ void to_fp16_inplace(uint32_t saddr, int bytes, int* dev_status) {
-  bool bad = false;
-  for (int i = threadIdx.x; i < bytes / 16; i += kThreads) {
-    const uint32_t a = saddr + i * 16;
-    uint4 u = ld_shared_v4(a);
-    uint32_t* w32 = &u.x;
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w32[e]));
-      bad |= fabsf(f.x) > 65504.f || fabsf(f.y) > 65504.f;
-      const __half2 hv = __floats2half2_rn(f.x, f.y);
-      w32[e] = *reinterpret_cast<const uint32_t*>(&hv);
-    }
-    st_shared_v4(a, u.x, u.y, u.z, u.w);
-  }
-  if (bad) report(dev_status, DARK_ERR_NUMERIC);
-}
-
-struct KeyParams {
-  const uint8_t* mask;
-  int B, H, L, ntiles, nsplit, heads_w;
-  float* partials;                 // [B*H*nsplit][65][m]
-  int* dev_status;
-};
-
-template <int M_, int R_>
-struct KeyCfg {
-  static constexpr int NW = M_ + R_, MB = M_ / 128;
-  static constexpr uint32_t kW = NW * 128;
-  static constexpr uint32_t kPhi = (M_ / 64) * 16384;
-  static constexpr uint32_t oW = 0;
-  static constexpr uint32_t oK = (kW + 1023) / 1024 * 1024;   // 2 buffers
-  static constexpr uint32_t oV = oK + 2 * kTileBytes;         // 2 buffers
-  static constexpr uint32_t oPhi = oV + 2 * kTileBytes;
-  static constexpr uint32_t oOnes = oPhi + kPhi;
-  static constexpr uint32_t oBar = oOnes + 2048;
-  static constexpr uint32_t kSmem = oBar + 64 + 1024;
-  static constexpr uint32_t tP = 0, tD = 320;
-};
-
-template <int M_, int R_>
-__global__ void __launch_bounds__(kThreads, 1)
-    keys_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_k,
-                const __grid_constant__ CUtensorMap tm_v, const KeyParams p) {
-  using G = KeyCfg<M_, R_>;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* sm = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-  const uint32_t s0 = smem_u32(sm);
-  uint64_t* bar_kv = (uint64_t*)(sm + G::oBar);     // [2]
-  uint64_t* bar_mma = bar_kv + 2;
-  uint32_t* tmem_slot = (uint32_t*)(bar_kv + 3);
-
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int quad = warp & 3, half = warp >> 2;
-  const int row = quad * 32 + lane;
-  const int split = blockIdx.x, bh = blockIdx.y, b = bh / p.H, h = bh % p.H;
-  const int hw = p.heads_w == 1 ? 0 : h;
-  const int tb = (int)((long long)split * p.ntiles / p.nsplit);
-  const int te = (int)((long long)(split + 1) * p.ntiles / p.nsplit);
-
-  if (tid == 0) {
-    mbar_init(&bar_kv[0], 1);
-    mbar_init(&bar_kv[1], 1);
-    mbar_init(bar_mma, 1);
-    fence_mbar_init();
-    if (te > tb) {
-      mbar_arrive_expect_tx(&bar_kv[0], G::kW + 2 * kTileBytes);
-      for (int r0 = 0; r0 < G::NW; r0 += 16)
-        tma_load_2d(sm + G::oW + r0 * 128, &tm_w, 0, hw * G::NW + r0, &bar_kv[0]);
-      tma_load_4d(sm + G::oK, &tm_k, 0, tb * kT, h, b, &bar_kv[0]);
-      tma_load_4d(sm + G::oV, &tm_v, 0, tb * kT, h, b, &bar_kv[0]);
-    }
-  }
-  __syncwarp();
-  if (warp == 0) tmem_alloc(tmem_slot, kTmemCols);
-  for (int i = tid; i < 2048 / 4; i += kThreads) ((uint32_t*)(sm + G::oOnes))[i] = 0x3F803F80u;
-  fence_async_smem();
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = *tmem_slot;
-  const uint32_t lane_tm = tmem + ((uint32_t)(quad * 32) << 16);
-
-  uint32_t ph_kv[2] = {0, 0}, ph_mma = 0;
-  bool abort = false;
-  for (int t = tb; t < te; ++t) {
-    const int i = t - tb, buf = i & 1;
-    if (!wait_all(&bar_kv[buf], ph_kv[buf], p.dev_status)) { abort = true; break; }
-    ph_kv[buf] ^= 1;
-    to_fp16_inplace(s0 + G::oK + buf * kTileBytes, kTileBytes, p.dev_status);
-    fence_async_smem();
-    __syncthreads();
-    if (tid == 0) {
-      tc_fence_after();
-      constexpr uint32_t idn0 = idesc(128, (G::NW < 256 ? G::NW : 256), false, false, true);
-      constexpr uint32_t idn1 = idesc(128, (G::NW > 256 ? G::NW - 256 : 16), false, false, true);
-#pragma unroll
-      for (int s = 0; s < kD / 16; ++s) {
-        const uint64_t ad = sdesc(s0 + G::oK + buf * kTileBytes + s * 32, 16, 1024);
-        mma(tmem + G::tP, ad, sdesc(s0 + G::oW + s * 32, 16, 1024), idn0, s > 0);
-        if (G::NW > 256)
-          mma(tmem + G::tP + 256, ad, sdesc(s0 + G::oW + 256 * 128 + s * 32, 16, 1024), idn1, s > 0);
-      }
-      mma_commit(bar_mma);
-    }
-    // this phase also covers the chunk-state GEMM of the previous tile
-    if (!wait_all(bar_mma, ph_mma, p.dev_status)) { abort = true; break; }
-    ph_mma ^= 1;
-    tc_fence_after();
-    // the other buffer is free now: prefetch the next tile into it
-    if (tid == 0 && t + 1 < te) {
-      const int nb = buf ^ 1;
-      mbar_arrive_expect_tx(&bar_kv[nb], 2 * kTileBytes);
-      tma_load_4d(sm + G::oK + nb * kTileBytes, &tm_k, 0, (t + 1) * kT, h, b, &bar_kv[nb]);
-      tma_load_4d(sm + G::oV + nb * kTileBytes, &tm_v, 0, (t + 1) * kT, h, b, &bar_kv[nb]);
-    }
-    {
-      float nrm = 0.f;
-#pragma unroll
-      for (int c0 = 0; c0 < R_; c0 += 16) {
-        float v[16];
-        tmem_ld16(lane_tm + G::tP + M_ + c0, v);
-#pragma unroll
-        for (int e = 0; e < 16; ++e) nrm = fmaf(v[e], v[e], nrm);
-      }
-      nrm += 0.5f * __log2f((float)M_);
-      const int tok = t * kT + row;
-      bool valid = tok < p.L;
-      if (valid && p.mask != nullptr) valid = p.mask[(size_t)b * p.L + tok] != 0;
-#pragma unroll 1
-      for (int f0 = half * (M_ / 2); f0 < (half + 1) * (M_ / 2); f0 += 32) {
-        float v[32];
-        tmem_ld32(lane_tm + G::tP + f0, v);
-#pragma unroll
-        for (int g = 0; g < 4; ++g) {
-          uint32_t w4[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float a = valid ? ex2(v[8 * g + 2 * e] - nrm) : 0.f;
-            const float c = valid ? ex2(v[8 * g + 2 * e + 1] - nrm) : 0.f;
-            w4[e] = pack_bf16(a, c);
-          }
-          st_shared_v4(s0 + G::oPhi + kmajor_off(row, f0 + 8 * g, 16384), w4[0], w4[1], w4[2], w4[3]);
-        }
-      }
-    }
-    fence_async_smem();
-    tc_fence_before();
-    __syncthreads();
-    if (tid == 0) {
-      tc_fence_after();
-      constexpr uint32_t idv = idesc(128, 64, true, true, false);
-      constexpr uint32_t id1 = idesc(128, 16, true, false, false);
-#pragma unroll
-      for (int mb = 0; mb < G::MB; ++mb) {
-#pragma unroll
-        for (int s = 0; s < kT / 16; ++s) {
-          const uint32_t acc = (t > tb || s > 0) ? 1u : 0u;
-          const uint64_t ad = sdesc(s0 + G::oPhi + mb * 32768 + s * 2048, 16384, 1024);
-          mma(tmem + G::tD + 80 * mb, ad, sdesc(s0 + G::oV + buf * kTileBytes + s * 2048, 16384, 1024),
-              idv, acc);
-          mma(tmem + G::tD + 80 * mb + 64, ad, sdesc(s0 + G::oOnes + (s % 4) * 32, 16, 1024), id1, acc);
-        }
-      }
-    }
-  }
-  if (!abort && te > tb) {
-    if (tid == 0) mma_commit(bar_mma);
-    if (!wait_all(bar_mma, ph_mma, p.dev_status)) abort = true;
-    tc_fence_after();
-  }
-  if (!abort && half < G::MB) {
-    const int f = half * 128 + row;
-    float* dst = p.partials + ((size_t)bh * p.nsplit + split) * 65 * M_;
-    if (te > tb) {
-      float v[32];
-      const uint32_t base = lane_tm + G::tD + 80 * half;
-      tmem_ld32(base, v);
-#pragma unroll
-      for (int e = 0; e < 32; ++e) dst[e * M_ + f] = v[e];
-      tmem_ld32(base + 32, v);
-#pragma unroll
-      for (int e = 0; e < 32; ++e) dst[(32 + e) * M_ + f] = v[e];
-      dst[64 * M_ + f] = tmem_ld1(base + 64);
-    } else {
-      for (int e = 0; e < 65; ++e) dst[e * M_ + f] = 0.f;
-    }
-  }
-  tc_fence_before();
-  __syncthreads();
-  if (warp == 0) {
-    tc_fence_after();
-    tmem_dealloc(tmem, kTmemCols);
-  }
-}
 
 // Sums the split partials of each head in split order and writes the query
 // kernel's operand image (hi + lo bf16) and, if requested, the fp32 state.
@@ -296,14 +93,6 @@ struct QueryCfg {
   static constexpr uint32_t kSmem = oBar + 64 + 1024;
   static constexpr uint32_t tP = 0, tO = 256;
 };
-
-__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
-  asm volatile(
-      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-          smem_u32(dst)),
-      "l"((uint64_t)src), "r"(bytes), "r"(smem_u32(bar))
-      : "memory");
-}
 
 template <int M_, int R_>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -479,20 +268,7 @@ Layout layout(int B, int H, int L, int m) {
   return s;
 }
 
-bool aligned16(const void* ptr) { return ((uintptr_t)ptr & 15) == 0; }
 
-bool make_maps(const FwdArgs& a, CUtensorMap* tw, CUtensorMap* tq, CUtensorMap* tk, CUtensorMap* tv) {
-  const uint64_t wd[2] = {(uint64_t)a.d, (uint64_t)a.heads_w * (a.m + a.r)};
-  const uint64_t wsd[1] = {(uint64_t)a.d * 2};
-  const uint32_t wb[2] = {64, 16};
-  if (!encode_tmap(tw, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, a.w, wd, wsd, wb)) return false;
-  const uint64_t xd[4] = {(uint64_t)a.d, (uint64_t)a.L, (uint64_t)a.H, (uint64_t)a.B};
-  const uint64_t xs[3] = {(uint64_t)a.qs[2] * 2, (uint64_t)a.qs[1] * 2, (uint64_t)a.qs[0] * 2};
-  const uint32_t xb[4] = {64, (uint32_t)kT, 1, 1};
-  return encode_tmap(tq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, a.q, xd, xs, xb) &&
-         encode_tmap(tk, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, a.k, xd, xs, xb) &&
-         encode_tmap(tv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, a.v, xd, xs, xb);
-}
 
 template <int M_, int R_>
 cudaError_t launch(const FwdArgs& a, const CUtensorMap& tw, const CUtensorMap& tq,
@@ -503,22 +279,8 @@ cudaError_t launch(const FwdArgs& a, const CUtensorMap& tw, const CUtensorMap& t
   uint8_t* images = (uint8_t*)(ws + s.off_img);
   const int bh = a.B * a.H;
 
-  KeyParams kp;
-  kp.mask = a.mask;
-  kp.B = a.B;
-  kp.H = a.H;
-  kp.L = a.L;
-  kp.ntiles = s.ntiles;
-  kp.nsplit = s.nsplit;
-  kp.heads_w = a.heads_w;
-  kp.partials = partials;
-  kp.dev_status = a.dev_status;
-  using KG = KeyCfg<M_, R_>;
-  cudaError_t e = cudaFuncSetAttribute(keys_kernel<M_, R_>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)KG::kSmem);
+  cudaError_t e = tc_launch_key_states(a, tw, tk, tv, s.ntiles, s.nsplit, partials);
   if (e != cudaSuccess) return e;
-  keys_kernel<M_, R_><<<dim3(s.nsplit, bh), kThreads, KG::kSmem, a.stream>>>(tw, tk, tv, kp);
-
   reduce_kernel<<<dim3((65 * a.m + 255) / 256, bh), 256, 0, a.stream>>>(partials, s.nsplit, a.m,
                                                                          images, a.st_kv, a.st_z);
 
@@ -536,8 +298,8 @@ cudaError_t launch(const FwdArgs& a, const CUtensorMap& tw, const CUtensorMap& t
   qp.images = images;
   qp.dev_status = a.dev_status;
   using QG = QueryCfg<M_, R_>;
-  e = cudaFuncSetAttribute(queries_kernel<M_, R_>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)QG::kSmem);
+  static int smem_set[64];
+  e = set_smem_limit_once((const void*)queries_kernel<M_, R_>, (int)QG::kSmem, smem_set);
   if (e != cudaSuccess) return e;
   const int grid = qp.total_tiles < kSms ? qp.total_tiles : kSms;
   queries_kernel<M_, R_><<<grid, kThreads, QG::kSmem, a.stream>>>(tw, tq, qp);
@@ -546,15 +308,10 @@ cudaError_t launch(const FwdArgs& a, const CUtensorMap& tw, const CUtensorMap& t
 
 }  // namespace
 
-bool tc_noncausal_supported(const FwdArgs& a) {
+bool tc_noncausal_supported(FwdArgs& a) {
   if (a.dtype != DARK_BF16 || a.d != kD || (a.flags & DARK_STABILISE)) return false;
   if (!(a.m == 128 || a.m == 256) || a.r % 16 != 0 || a.r < 16 || a.r > 64) return false;
-  if (!aligned16(a.q) || !aligned16(a.k) || !aligned16(a.v) || !aligned16(a.out) || !aligned16(a.w))
-    return false;
-  for (int i = 0; i < 3; ++i)
-    if (a.qs[i] % 8 != 0 || a.os[i] % 8 != 0) return false;
-  CUtensorMap t[4];
-  return make_maps(a, &t[0], &t[1], &t[2], &t[3]);
+  return tc_make_maps(a);
 }
 
 size_t tc_noncausal_workspace_bytes(int B, int H, int L, int m, int d) {
@@ -563,8 +320,8 @@ size_t tc_noncausal_workspace_bytes(int B, int H, int L, int m, int d) {
 }
 
 cudaError_t tc_noncausal_forward(const FwdArgs& a) {
-  CUtensorMap tw, tq, tk, tv;
-  if (!make_maps(a, &tw, &tq, &tk, &tv)) return cudaErrorInvalidValue;
+  if (!a.maps_ready) return cudaErrorInvalidValue;
+  const CUtensorMap &tw = a.tm_w, &tq = a.tm_q, &tk = a.tm_k, &tv = a.tm_v;
 #define DARK_NC_CASE(MM, RR) \
   if (a.m == MM && a.r == RR) return launch<MM, RR>(a, tw, tq, tk, tv);
   DARK_NC_CASE(256, 64)
