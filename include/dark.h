@@ -173,6 +173,31 @@ dark_status dark_attention_fwd(const dark_projection* proj, const void* q, const
                                void* ws, size_t ws_bytes, int* dev_status, void* stream);
 
 /*
+ * dark_attention_fwd without a caller workspace, for callers that cannot
+ * allocate device memory (for example code running inside a CUDA-graph capture
+ * it does not own, or under an allocator that refuses extra allocations). The
+ * method's pages have no counterpart of this call; it is a deployment aid.
+ * Arguments and results are those of dark_attention_fwd minus ws/ws_bytes; the
+ * scratch is a fixed array of dark_noalloc_scratch_bytes() (16 MiB) compiled into
+ * the library, which every GPU that loads the library keeps until the process
+ * exits. Nothing is allocated and nothing is freed.
+ *   - Returns DARK_ERR_UNSUPPORTED, enqueuing nothing, when the call needs more
+ *     scratch than that (dark_attention_workspace_bytes tells the size the call
+ *     would need with a workspace of its own).
+ *   - The first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress); make that first call before any stream capture.
+ *   - Every call shares the one array and it keeps the previous call's
+ *     contents: calls whose work overlaps on the GPU (different streams, or
+ *     different host threads without ordering) race on it. Serialise them.
+ */
+size_t dark_noalloc_scratch_bytes(void);
+dark_status dark_attention_fwd_noalloc(const dark_projection* proj, const void* q, const void* k,
+                                       const void* v, void* out, const int64_t* qkv_strides,
+                                       const int64_t* out_strides, int B, int H, int L,
+                                       const uint8_t* key_mask, int flags, dark_state* state_out,
+                                       int* dev_status, void* stream);
+
+/*
  * Zeroes a state (kv, z and, if non-NULL, shift) and ties it to `proj`, for
  * decoding from an empty prefix.
  */

@@ -28,7 +28,8 @@ WS_HEADER_BYTES = 256
 
 EXPORTS = ("dark_abi_version", "dark_status_string", "dark_projection_bytes",
            "dark_make_projection", "dark_attention_workspace_bytes", "dark_attention_fwd",
-           "dark_state_init", "dark_decode_step")
+           "dark_state_init", "dark_decode_step", "dark_noalloc_scratch_bytes",
+           "dark_attention_fwd_noalloc")
 
 
 class dark_projection(ctypes.Structure):
@@ -59,6 +60,11 @@ _lib.dark_attention_fwd.restype = _i
 _lib.dark_attention_fwd.argtypes = [_P(dark_projection), _vp, _vp, _vp, _vp, _P(ctypes.c_int64),
                                     _P(ctypes.c_int64), _i, _i, _i, _vp, _i, _P(dark_state), _vp,
                                     _sz, _vp, _vp]
+_lib.dark_noalloc_scratch_bytes.restype = _sz
+_lib.dark_attention_fwd_noalloc.restype = _i
+_lib.dark_attention_fwd_noalloc.argtypes = [_P(dark_projection), _vp, _vp, _vp, _vp,
+                                            _P(ctypes.c_int64), _P(ctypes.c_int64), _i, _i, _i,
+                                            _vp, _i, _P(dark_state), _vp, _vp]
 _lib.dark_state_init.restype = _i
 _lib.dark_state_init.argtypes = [_P(dark_projection), _P(dark_state), _vp]
 _lib.dark_decode_step.restype = _i
@@ -153,6 +159,24 @@ def dark_attention_fwd(proj: dark_projection, q, k, v, out, B: int, H: int, L: i
         strides(out_strides), B, H, L, _ptr(key_mask), flags,
         None if state_out is None else ctypes.byref(state_out), _ptr(ws),
         0 if ws is None else ws.numel() * ws.element_size(), _ptr(dev_status), _stream(stream)))
+
+
+def dark_noalloc_scratch_bytes() -> int:
+    return _lib.dark_noalloc_scratch_bytes()
+
+
+def dark_attention_fwd_noalloc(proj: dark_projection, q, k, v, out, B: int, H: int, L: int,
+                               key_mask=None, flags: int = 0,
+                               state_out: dark_state | None = None, dev_status=None,
+                               stream=None, qkv_strides=None, out_strides=None) -> None:
+    """dark_attention_fwd with the library's fixed scratch instead of a workspace."""
+    def strides(s):
+        return None if s is None else (ctypes.c_int64 * 3)(*s)
+    _check(_lib.dark_attention_fwd_noalloc(
+        ctypes.byref(proj), _ptr(q), _ptr(k), _ptr(v), _ptr(out), strides(qkv_strides),
+        strides(out_strides), B, H, L, _ptr(key_mask), flags,
+        None if state_out is None else ctypes.byref(state_out), _ptr(dev_status),
+        _stream(stream)))
 
 
 def dark_state_init(proj: dark_projection, st: dark_state, stream=None) -> None:
