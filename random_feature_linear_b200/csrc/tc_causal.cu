@@ -63,7 +63,10 @@ struct Cfg {
   static constexpr uint32_t oBar = oOnes + 2048;
   static constexpr uint32_t kSmem = oBar + 64 + 1024;     // + alignment slack
   // TMEM columns
-  static constexpr uint32_t tP = 0, tA = 0, tNum = 128, tD = 320;
+  // key features [0, M_) and norms [M_, M_ + R_); query features [256, 256 + M_)
+  // (issued once the norms are read); scores [0, 128), numerator [128, 208) and
+  // chunk state [320, 480) once both feature blocks are consumed
+  static constexpr uint32_t tP = 0, tQ = 256, tA = 0, tNum = 128, tD = 320;
   static_assert(NW <= 320 && M_ % 128 == 0 && R_ % 16 == 0, "shape");
   static_assert(tD + 80 * MB <= kTmemCols, "tmem");
 };
@@ -184,61 +187,33 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int i = 0; i < 16; ++i) nrm = fmaf(v[i], v[i], nrm);
       }
       nrm += 0.5f * __log2f((float)M_);
+      // the norm columns are read: the query GEMM may now overwrite them
+      tc_fence_before();
+      __syncthreads();
+      if (tid == 0) {
+        tc_fence_after();
+        constexpr uint32_t idq = idesc(128, (M_ < 256 ? M_ : 256), false, false, true);
+#pragma unroll
+        for (int s = 0; s < kD / 16; ++s)
+          mma(tmem + G::tQ, sdesc(s0 + G::oQ + s * 32, 16, 1024),
+              sdesc(s0 + G::oW + s * 32, 16, 1024), idq, s > 0);
+        mma_commit(bar_mma);
+      }
       const int tok = t0 + row;
       bool valid = tok < p.L;
       if (valid && p.mask != nullptr) valid = p.mask[(size_t)b * p.L + tok] != 0;
-#pragma unroll 1
-      for (int f0 = half * (M_ / 2); f0 < (half + 1) * (M_ / 2); f0 += 32) {
-        float v[32];
-        tmem_ld32(lane_tm + G::tP + f0, v);
-#pragma unroll
-        for (int g = 0; g < 4; ++g) {
-          uint32_t w4[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            // values 5..7 of each group of 8 go through the FMA pipe
-            const float x0 = v[8 * g + 2 * e] - nrm, x1 = v[8 * g + 2 * e + 1] - nrm;
-            const float a = valid ? (2 * e >= 5 ? ex2_fma(x0) : ex2(x0)) : 0.f;
-            const float bb = valid ? (2 * e + 1 >= 5 ? ex2_fma(x1) : ex2(x1)) : 0.f;
-            w4[e] = pack_bf16(a, bb);
-          }
-          const int f = f0 + 8 * g;
-          st_shared_v4(s0 + G::oPhi + kmajor_off(row, f, 16384), w4[0], w4[1], w4[2], w4[3]);
-        }
-      }
+      exp2_rows_to_smem(lane_tm + G::tP, half * (M_ / 2), (half + 1) * (M_ / 2), nrm, !valid,
+                        s0 + G::oPhi, row);
     }
     fence_async_smem();
     tc_fence_before();
     __syncthreads();
-    // ------------------------------------------------------- feature GEMM Q
-    if (tid == 0) {
-      tc_fence_after();
-      constexpr uint32_t idq = idesc(128, (M_ < 256 ? M_ : 256), false, false, true);
-#pragma unroll
-      for (int s = 0; s < kD / 16; ++s)
-        mma(tmem + G::tP, sdesc(s0 + G::oQ + s * 32, 16, 1024),
-            sdesc(s0 + G::oW + s * 32, 16, 1024), idq, s > 0);
-      mma_commit(bar_mma);
-    }
     if (!wait_all(bar_mma, ph_mma, p.dev_status)) { abort = true; break; }
     ph_mma ^= 1;
     tc_fence_after();
     // ------------------------------------------------- epilogue: Psi(Q_c)
-#pragma unroll 1
-    for (int f0 = half * (M_ / 2); f0 < (half + 1) * (M_ / 2); f0 += 32) {
-      float v[32];
-      tmem_ld32(lane_tm + G::tP + f0, v);
-#pragma unroll
-      for (int g = 0; g < 4; ++g) {
-        uint32_t w4[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float x0 = v[8 * g + 2 * e], x1 = v[8 * g + 2 * e + 1];
-          w4[e] = pack_bf16(2 * e >= 5 ? ex2_fma(x0) : ex2(x0), 2 * e + 1 >= 5 ? ex2_fma(x1) : ex2(x1));
-        }
-        st_shared_v4(s0 + G::oPsi + kmajor_off(row, f0 + 8 * g, 16384), w4[0], w4[1], w4[2], w4[3]);
-      }
-    }
+    exp2_rows_to_smem(lane_tm + G::tQ, half * (M_ / 2), (half + 1) * (M_ / 2), 0.f, false,
+                      s0 + G::oPsi, row);
     fence_async_smem();
     tc_fence_before();
     __syncthreads();
@@ -286,19 +261,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           st_shared_v4(s0 + G::oQ + kmajor_off(row, j0 + 8 * g, 16384), w4[0], w4[1], w4[2], w4[3]);
         }
       }
-    }
-    // chunk state row `feat` (the aggregate of this chunk)
-    float ds[65];
-    if (has_feat) {
-      float v[32];
-      const uint32_t base = tmem + ((uint32_t)(quad * 32) << 16) + G::tD + 80 * half;
-      tmem_ld32(base, v);
-#pragma unroll
-      for (int i = 0; i < 32; ++i) ds[i] = v[i];
-      tmem_ld32(base + 32, v);
-#pragma unroll
-      for (int i = 0; i < 32; ++i) ds[32 + i] = v[i];
-      ds[64] = tmem_ld1(base + 64);
     }
     fence_async_smem();
     tc_fence_before();
@@ -348,9 +310,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         st_shared_u16(zl_base + off, zlb);
       }
     }
+    // add this chunk's state row `feat` (Phi(K_c)^T [V_c | 1], in TMEM) to the prefix
     if (has_feat) {
+      uint32_t a[32], b2[32];
+      const uint32_t base = tmem + ((uint32_t)(quad * 32) << 16) + G::tD + 80 * half;
+      tmem_ld32_async(base, a);
+      tmem_ld32_async(base + 32, b2);
+      tmem_wait_ld(a);
+      tmem_wait_ld(b2);
 #pragma unroll
-      for (int i = 0; i < 65; ++i) run[i] += ds[i];
+      for (int i = 0; i < 32; ++i) run[i] += __uint_as_float(a[i]);
+#pragma unroll
+      for (int i = 0; i < 32; ++i) run[32 + i] += __uint_as_float(b2[i]);
+      run[64] += tmem_ld1(base + 64);
     }
     fence_async_smem();
     __syncthreads();

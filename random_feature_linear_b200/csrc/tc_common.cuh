@@ -258,6 +258,73 @@ __host__ __device__ constexpr uint32_t kmajor_off(int row, int k, uint32_t kbloc
          (uint32_t)(k % 8) * 2u;
 }
 
+// Asynchronous variant: the 32 registers are written when tmem_wait_ld(r)
+// returns; the wait names them as in/out operands so that no use of them can
+// be scheduled before it. Lets one block of columns load while another is used.
+__device__ __forceinline__ void tmem_ld32_async(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, "
+      "%12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, "
+      "%30, %31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+        "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr)
+      : "memory");
+}
+__device__ __forceinline__ void tmem_wait_ld(uint32_t (&r)[32]) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;"
+               : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]),
+                 "+r"(r[6]), "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]),
+                 "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15]), "+r"(r[16]), "+r"(r[17]),
+                 "+r"(r[18]), "+r"(r[19]), "+r"(r[20]), "+r"(r[21]), "+r"(r[22]), "+r"(r[23]),
+                 "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]), "+r"(r[29]),
+                 "+r"(r[30]), "+r"(r[31])
+               :
+               : "memory");
+}
+
+// exp2 of 32 values (minus a per-row offset) packed to bf16 and stored as four
+// 16-byte chunks of a K-major 128B-swizzled row (chunk f/8 of row `row`).
+// `zero` stores zeros instead (masked keys).
+__device__ __forceinline__ void exp2_pack_store32(const uint32_t (&r)[32], float offset, bool zero,
+                                                  uint32_t tile, int row, int f0) {
+#pragma unroll
+  for (int g = 0; g < 4; ++g) {
+    uint32_t w4[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float x0 = __uint_as_float(r[8 * g + 2 * e]) - offset;
+      const float x1 = __uint_as_float(r[8 * g + 2 * e + 1]) - offset;
+      w4[e] = zero ? 0u : pack_bf16(ex2(x0), ex2(x1));
+    }
+    st_shared_v4(tile + kmajor_off(row, f0 + 8 * g, 16384), w4[0], w4[1], w4[2], w4[3]);
+  }
+}
+
+// Columns [f_begin, f_end) of this thread's TMEM lane (32 at a time, the next
+// block's load in flight while the current one is exponentiated and stored).
+__device__ __forceinline__ void exp2_rows_to_smem(uint32_t lane_taddr, int f_begin, int f_end,
+                                                  float offset, bool zero, uint32_t tile, int row) {
+  uint32_t a[32], b[32];
+  tmem_ld32_async(lane_taddr + f_begin, a);
+  tmem_wait_ld(a);
+#pragma unroll 1
+  for (int f0 = f_begin; f0 < f_end; f0 += 64) {
+    const bool more_b = f0 + 32 < f_end, more_a = f0 + 64 < f_end;
+    if (more_b) tmem_ld32_async(lane_taddr + f0 + 32, b);
+    exp2_pack_store32(a, offset, zero, tile, row, f0);
+    if (!more_b) break;
+    tmem_wait_ld(b);
+    if (more_a) tmem_ld32_async(lane_taddr + f0 + 64, a);
+    exp2_pack_store32(b, offset, zero, tile, row, f0 + 32);
+    if (!more_a) break;
+    tmem_wait_ld(a);
+  }
+}
+
 }  // namespace tc
 
 // ------------------------------------------------------------ host helpers --

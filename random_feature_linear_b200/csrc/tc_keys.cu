@@ -88,12 +88,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = *tmem_slot;
   const uint32_t lane_tm = tmem + ((uint32_t)(quad * 32) << 16);
 
-  uint32_t ph_kv[2] = {0, 0}, ph_mma = 0;
+  uint32_t ph_kv = 0, ph_mma = 0;             // bit i: phase parity of buffer i
   bool abort = false;
   for (int t = tb; t < te; ++t) {
     const int i = t - tb, buf = i & 1;
-    if (!wait_all(&bar_kv[buf], ph_kv[buf], p.dev_status)) { abort = true; break; }
-    ph_kv[buf] ^= 1;
+    if (!wait_all(&bar_kv[buf], (ph_kv >> buf) & 1u, p.dev_status)) { abort = true; break; }
+    ph_kv ^= 1u << buf;
     to_fp16_inplace(s0 + G::oK + buf * kTileBytes, kTileBytes, p.dev_status);
     fence_async_smem();
     __syncthreads();
@@ -134,22 +134,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int tok = t * kT + row;
       bool valid = tok < p.L;
       if (valid && p.mask != nullptr) valid = p.mask[(size_t)b * p.L + tok] != 0;
-#pragma unroll 1
-      for (int f0 = half * (M_ / 2); f0 < (half + 1) * (M_ / 2); f0 += 32) {
-        float v[32];
-        tmem_ld32(lane_tm + G::tP + f0, v);
-#pragma unroll
-        for (int g = 0; g < 4; ++g) {
-          uint32_t w4[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float a = valid ? ex2(v[8 * g + 2 * e] - nrm) : 0.f;
-            const float c = valid ? ex2(v[8 * g + 2 * e + 1] - nrm) : 0.f;
-            w4[e] = pack_bf16(a, c);
-          }
-          st_shared_v4(s0 + G::oPhi + kmajor_off(row, f0 + 8 * g, 16384), w4[0], w4[1], w4[2], w4[3]);
-        }
-      }
+      exp2_rows_to_smem(lane_tm + G::tP, half * (M_ / 2), (half + 1) * (M_ / 2), nrm, !valid,
+                        s0 + G::oPhi, row);
     }
     fence_async_smem();
     tc_fence_before();

@@ -133,7 +133,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = *tmem_slot;
   const uint32_t lane_tm = tmem + ((uint32_t)(quad * 32) << 16);
 
-  uint32_t ph_q[2] = {0, 0}, ph_mma = 0, ph_head = 0;
+  uint32_t ph_q = 0, ph_mma = 0, ph_head = 0;  // ph_q bit i: parity of buffer i
   int cur_bh = -1;
   bool abort = false;
   for (int u = ub; u < ue; ++u) {
@@ -155,8 +155,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       ph_head ^= 1;
       cur_bh = bh;
     }
-    if (!wait_all(&bar_q[buf], ph_q[buf], p.dev_status)) { abort = true; break; }
-    ph_q[buf] ^= 1;
+    if (!wait_all(&bar_q[buf], (ph_q >> buf) & 1u, p.dev_status)) { abort = true; break; }
+    ph_q ^= 1u << buf;
     to_fp16_inplace(s0 + G::oQ + buf * kTileBytes, kTileBytes, p.dev_status);
     fence_async_smem();
     __syncthreads();
@@ -179,18 +179,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       tma_load_4d(sm + G::oQ + (buf ^ 1) * kTileBytes, &tm_q, 0, nt * kT, nbh % p.H, nbh / p.H,
                   &bar_q[buf ^ 1]);
     }
-#pragma unroll 1
-    for (int f0 = half * (M_ / 2); f0 < (half + 1) * (M_ / 2); f0 += 32) {
-      float v[32];
-      tmem_ld32(lane_tm + G::tP + f0, v);
-#pragma unroll
-      for (int g = 0; g < 4; ++g) {
-        uint32_t w4[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) w4[e] = pack_bf16(ex2(v[8 * g + 2 * e]), ex2(v[8 * g + 2 * e + 1]));
-        st_shared_v4(s0 + G::oPsi + kmajor_off(row, f0 + 8 * g, 16384), w4[0], w4[1], w4[2], w4[3]);
-      }
-    }
+    exp2_rows_to_smem(lane_tm + G::tP, half * (M_ / 2), (half + 1) * (M_ / 2), 0.f, false,
+                      s0 + G::oPsi, row);
     fence_async_smem();
     tc_fence_before();
     __syncthreads();
