@@ -83,18 +83,82 @@ __device__ __forceinline__ float block_sum(float v, float* scratch) {
   return warp_sum(t);
 }
 
-__device__ __forceinline__ float block_max(float v, float* scratch) {
-  v = warp_max(v);
+
+// 8 consecutive weights of a W' row as fp32 (fp16 or fp32 storage).
+__device__ __forceinline__ void load_w8(const __half* __restrict__ w, float (&f)[8]) {
+  const uint4 u = __ldg(reinterpret_cast<const uint4*>(w));
+  const __half2* h = reinterpret_cast<const __half2*>(&u);
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const float2 t = __half22float2(h[e]);
+    f[2 * e] = t.x;
+    f[2 * e + 1] = t.y;
+  }
+}
+__device__ __forceinline__ void load_w8(const float* __restrict__ w, float (&f)[8]) {
+  const float4 a = __ldg(reinterpret_cast<const float4*>(w));
+  const float4 b = __ldg(reinterpret_cast<const float4*>(w) + 1);
+  f[0] = a.x; f[1] = a.y; f[2] = a.z; f[3] = a.w;
+  f[4] = b.x; f[5] = b.y; f[6] = b.z; f[7] = b.w;
+}
+
+// Feature exponents W' k and W' q for one head into pk[0, m + r) and pq[0, m).
+// Groups of 8 lanes own one W' row at a time, each lane 8 consecutive columns;
+// every group first issues the loads of up to 8 of its rows, then reduces
+// them with shuffles, so the L2 latency of W' is paid once per batch.
+template <int kBatch, typename TW>
+__device__ __forceinline__ void feature_gemv(const TW* __restrict__ wh, int m, int r, int d,
+                                             const float* xk, const float* xq, float* pk,
+                                             float* pq) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  __syncthreads();
-  if (lane == 0) scratch[warp] = v;
-  __syncthreads();
-  float t = lane < kThreads / 32 ? scratch[lane] : -INFINITY;
-  return warp_max(t);
+  const int g = lane >> 3, cl = lane & 7;
+  const int rows = m + r;
+  constexpr int kGroups = kThreads / 8;
+  for (int c0 = 0; c0 < d; c0 += 64) {
+    float fk[8], fq[8];
+    const int col = c0 + cl * 8;
+    const bool cok = col < d;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      fk[e] = cok ? xk[col + e] : 0.f;
+      fq[e] = cok ? xq[col + e] : 0.f;
+    }
+    for (int jb = warp * 4 + g; jb < rows; jb += kBatch * kGroups) {
+      float wv[kBatch][8];
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u) {
+        const int j = jb + u * kGroups;
+        if (cok && j < rows) load_w8(wh + (size_t)j * d + col, wv[u]);
+        else {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) wv[u][e] = 0.f;
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u) {
+        const int j = jb + u * kGroups;
+        float ak = 0.f, aq = 0.f;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          ak = fmaf(wv[u][e], fk[e], ak);
+          aq = fmaf(wv[u][e], fq[e], aq);
+        }
+#pragma unroll
+        for (int o = 4; o > 0; o >>= 1) {
+          ak += __shfl_xor_sync(0xffffffffu, ak, o);
+          aq += __shfl_xor_sync(0xffffffffu, aq, o);
+        }
+        if (cl == 0 && j < rows) {
+          pk[j] = (c0 == 0 ? 0.f : pk[j]) + ak;
+          if (j < m) pq[j] = (c0 == 0 ? 0.f : pq[j]) + aq;
+        }
+      }
+    }
+  }
 }
 
 template <typename T>
-__global__ void __launch_bounds__(kThreads) decode_kernel(
+__global__ void __launch_bounds__(kThreads, 2) decode_kernel(
     const typename WeightOf<T>::type* __restrict__ w, int heads_w, int m, int r, int d,
     float* __restrict__ kv, float* __restrict__ z, const float* __restrict__ shift, int H,
     const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v, T* __restrict__ out,
@@ -111,7 +175,7 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(
   float* scratch = red + rpp * d;         // [32]
   const int bh = blockIdx.x, b = bh / H, h = bh % H;
   const auto* wh = w + (size_t)(heads_w == 1 ? 0 : h) * (m + r) * d;
-  const int tid = threadIdx.x;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int c4 = tid % tpr, r0 = tid / tpr;
   const bool rows_active = r0 < rpp;
   float4* base = reinterpret_cast<float4*>(kv + (size_t)bh * m * d) + c4;
@@ -140,20 +204,36 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(
     xv[c] = to_f32(v[(size_t)bh * d + c]);
   }
   __syncthreads();
-  for (int j = tid; j < m + r; j += kThreads) {
-    float ak, aq;
-    row_dot2(wh + (size_t)j * d, d, xk, xq, j < m, ak, aq);
-    pk[j] = ak;
-    if (j < m) pq[j] = aq;
+  // Feature exponents W' k and W' q: groups of 8 lanes own one row at a time,
+  // each lane 8 consecutive columns (held in registers), reduced by shuffles.
+  // Rows whose length is not a multiple of 8 take one thread per row instead.
+  if (d % 8 != 0) {
+    for (int j = tid; j < m + r; j += kThreads) {
+      float ak, aq;
+      row_dot2(wh + (size_t)j * d, d, xk, xq, j < m, ak, aq);
+      pk[j] = ak;
+      if (j < m) pq[j] = aq;
+    }
+  } else {
+    feature_gemv<2>(wh, m, r, d, xk, xq, pk, pq);
   }
   __syncthreads();
-  float nrm = 0.f, qmax = -INFINITY;
-  for (int i = tid; i < r; i += kThreads) nrm = fmaf(pk[m + i], pk[m + i], nrm);
-  for (int j = tid; j < m; j += kThreads) qmax = fmaxf(qmax, pq[j]);
-  nrm = block_sum(nrm, scratch);
+  // warp 0: key norm (base 2, with 1/2 log2 m) and, when stabilised, the query max
   const bool stab = shift != nullptr;
-  const float qs = stab ? block_max(qmax, scratch) : 0.f;
-  const float ks = nrm + 0.5f * log2f((float)m) + (stab ? shift[bh] : 0.f);
+  if (warp == 0) {
+    float nrm = 0.f, qmax = -INFINITY;
+    for (int i = lane; i < r; i += 32) nrm = fmaf(pk[m + i], pk[m + i], nrm);
+    if (stab)
+      for (int j = lane; j < m; j += 32) qmax = fmaxf(qmax, pq[j]);
+    nrm = warp_sum(nrm);
+    qmax = warp_max(qmax);
+    if (lane == 0) {
+      scratch[0] = nrm + 0.5f * log2f((float)m) + (stab ? shift[bh] : 0.f);
+      scratch[1] = stab ? qmax : 0.f;
+    }
+  }
+  __syncthreads();
+  const float ks = scratch[0], qs = scratch[1];
   const bool ok = valid == nullptr || valid[b] != 0;
   for (int j = tid; j < m; j += kThreads) {
     pk[j] = ok ? exp2f(pk[j] - ks) : 0.f;
@@ -199,12 +279,7 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(
       den = fmaf(pq[j], zj, den);
     }
   }
-  for (int j = tid + 4 * kThreads; j < m; j += kThreads) {
-    const float zj = z[(size_t)bh * m + j] + pk[j];
-    z[(size_t)bh * m + j] = zj;
-    den = fmaf(pq[j], zj, den);
-  }
-  den = block_sum(den, scratch);   // contains the barrier that publishes `red`
+  den = block_sum(den, scratch + 2);   // contains the barrier that publishes `red`
   for (int c = tid; c < d; c += kThreads) {
     float acc = 0.f;
     for (int g = 0; g < rpp; ++g) acc += red[g * d + c];
@@ -219,7 +294,7 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(
 cudaError_t launch_decode(const DecodeArgs& a) {
   const int tpr = a.d / 4;
   const int rpp = kThreads / tpr;
-  const size_t smem = sizeof(float) * (3 * a.d + (a.m + a.r) + a.m + rpp * a.d + 32);
+  const size_t smem = sizeof(float) * (3 * a.d + (a.m + a.r) + a.m + rpp * a.d + 40);
   cudaError_t err;
   if (a.dtype == DARK_BF16) {
     static int done[64];

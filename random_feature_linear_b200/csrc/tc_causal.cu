@@ -46,7 +46,7 @@ constexpr uint32_t kTmemCols = 512;
 
 template <int M_, int R_>
 struct Cfg {
-  static constexpr int M = M_, R = R_, MB = M_ / 128;
+  static constexpr int MB = M_ / 128;
   static constexpr int NW = M_ + R_;                      // W' rows
   static constexpr uint32_t kW = NW * 128;                // W' bytes (fp16, 128 B rows)
   static constexpr uint32_t kZ = (M_ / 64) * 2048;        // one z16 operand (hi or lo)
