@@ -112,3 +112,14 @@ def test_redraw_makes_state_stale(D, cuda_ok):
     # the old projection still accepts it
     D.dark_decode_step(res["proj"], res["state"], q, q, q, torch.empty_like(q))
     torch.cuda.synchronize()
+
+
+def test_decode_shared_projection(D, cuda_ok):
+    # one W' for all heads (shared Omega and M)
+    w = synth.WORKLOADS[5].with_sizes(B=5, H=3, L=140, per_head_geom=False)
+    inp = synth.make_inputs(w)
+    stream = synth.decode_stream(w, 3)
+    got, _ = _decode_run(D, cuda_ok, w, inp, stream, 3)
+    ref = _oracle_decode(inp, stream, 3)
+    for g, r in zip(got, ref):
+        check(w, g[:, :, None], r[:, :, None])
