@@ -13,6 +13,7 @@ buffers, host->device and device->host copies inside the timed region.
 from __future__ import annotations
 
 import argparse
+import hashlib
 import json
 import os
 import statistics
@@ -30,6 +31,26 @@ sys.path.insert(0, ROOT)
 from random_feature_linear_b200 import synth  # noqa: E402
 
 L2_FLUSH_BYTES = 512 << 20        # > 126 MB L2
+
+
+METRIC = "DARK attention fwd tokens/s (B\u00b7H\u00b7L/s) on 1 B200; % of BF16-tensor/HBM roofline"
+
+# DRAM bytes (read + write) per forward call from one ncu capture of the causal
+# masked workload (B2 H8 L2048 d64 r64 m256), summed over its three launches.
+# Reported only while the kernel sources hash to what was captured.
+_CAUSAL_SOURCES = ("tc_causal.cu", "tc_keys.cu", "tc_keys.cuh", "tc_common.cuh")
+_NCU_TRAFFIC = {2: ("7fee9498405bfb98", 8.760320e6 + 9.592320e6 + 21.514240e6)}
+
+
+def captured_traffic(cfg: int):
+    if cfg not in _NCU_TRAFFIC:
+        return None
+    digest, nbytes = _NCU_TRAFFIC[cfg]
+    h = hashlib.sha256()
+    for f in _CAUSAL_SOURCES:
+        with open(os.path.join(ROOT, "random_feature_linear_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return nbytes if h.hexdigest()[:16] == digest else None
 
 
 def alg_flops(w: synth.Workload) -> float:
@@ -269,7 +290,7 @@ def run_native(args, w: synth.Workload, rank: int, world: int, dev) -> dict | No
         return None
     tokens = w.tokens * world
     peaks = load_peaks()
-    t_kernel = ms_per_step / 1e3            # one launch per step on the tensor-core path
+    t_kernel = ms_per_step / 1e3            # the whole forward call (its launches back to back)
     flops = alg_flops(w)
     nbytes = alg_bytes(w)
     t_tc = flops / (peaks["bf16"] * 1e12)
@@ -284,6 +305,10 @@ def run_native(args, w: synth.Workload, rank: int, world: int, dev) -> dict | No
         roof = dict(bound="hbm", achieved=achieved, peak=peaks["hbm"], unit="GB/s",
                     frac=achieved / peaks["hbm"], traffic=None)
     roof["peak_source"] = peaks["source"] + " (burst)"
+    short = sorted({k.replace("(anonymous namespace)::", "").split("(")[0].split("<")[0].split("::")[-1]
+                    for k in kernel_names if "dark::" in k})
+    roof["kernel"] = "forward call" + (" (" + ", ".join(short) + ")" if short else "")
+    roof["traffic"] = captured_traffic(args.workload)
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
         tps, ntok, secs, heads = oracle_sample(w, inp)
@@ -291,7 +316,7 @@ def run_native(args, w: synth.Workload, rank: int, world: int, dev) -> dict | No
                    sample=f"{heads} of {w.B * w.H} (batch, head) slices, {ntok} tokens, {secs:.1f} s")
     clocks = clk.summary()
     return {
-        "metric": "DARK attention fwd tokens/s (B*H*L/s) on B200",
+        "metric": METRIC,
         "value": tokens / (ms_per_step / 1e3),
         "unit": "tokens/s",
         "n_gpus": world,
@@ -323,6 +348,163 @@ def run_native(args, w: synth.Workload, rank: int, world: int, dev) -> dict | No
     }
 
 
+DECODE_METRIC = "DARK decode step tokens/s (B\u00b7H rows per step) on 1 B200; % of HBM roofline"
+
+
+def decode_bytes(w: synth.Workload) -> float:
+    """Algorithmic HBM bytes of one decode step: the fp32 (KV, z) state read and
+    written once, plus q, k, v in and out."""
+    state = w.B * w.H * w.m * (w.d + 1) * 4
+    io = 4 * w.B * w.H * w.d * (2 if w.dtype == "bf16" else 4)
+    return 2 * state + io
+
+
+def oracle_decode_sample(w: synth.Workload, kv, z, stream, omega, geom, max_seconds: float = 10.0):
+    """Times fp64 oracle decode steps over all (batch, head) slices; returns
+    (rows/s, steps done, seconds)."""
+    from oracle import dark_oracle as O
+    done, t_total = 0, 0.0
+    while t_total < max_seconds and done < stream["q"].shape[0]:
+        t0 = time.perf_counter()
+        _, kv, z = O.decode_step(kv, z, stream["q"][done], stream["k"][done], stream["v"][done],
+                                 omega, geom)
+        t_total += time.perf_counter() - t0
+        done += 1
+    return done * w.B * w.H / t_total, done, t_total
+
+
+def run_decode(args, rank: int, world: int, dev) -> dict | None:
+    """Streaming decode (workload 5): a causal prefill fills the (KV, z) state
+    outside the timed region; each timed iteration is one decode step replayed
+    from a CUDA graph, with the L2 flushed before it (the state then comes from
+    HBM). A 1024-step graph, state L2-warm, is reported beside it."""
+    from random_feature_linear_b200 import dark as D
+    w = synth.WORKLOADS[5]
+    inp = synth.make_inputs(w, salt=rank)
+    dt = D.DARK_BF16
+    omega = torch.from_numpy(inp["omega"]).to(dev)
+    geom = torch.from_numpy(inp["geom"]).to(dev)
+    proj, _wbuf = D.dark_make_projection(omega, geom, w.H, dt)
+    q, k, v = (torch.from_numpy(inp[n]).to(dev).to(torch.bfloat16) for n in ("q", "k", "v"))
+    out = torch.empty_like(q)
+    st, st_t = D.make_state(proj, w.B, w.H, dev)
+    ws = D.alloc_workspace(proj, w.B, w.H, w.L, D.DARK_CAUSAL, dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    D.dark_attention_fwd(proj, q, k, v, out, w.B, w.H, w.L, flags=D.DARK_CAUSAL, state_out=st,
+                         ws=ws, dev_status=status)
+    n_graph = 1024
+    stream_np = synth.decode_stream(w, n_graph, salt=rank)
+    sq, sk, sv = (torch.from_numpy(stream_np[n]).to(dev).to(torch.bfloat16) for n in ("q", "k", "v"))
+    so = torch.empty_like(sq)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.int32, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def one(i):
+        D.dark_decode_step(proj, st, sq[i], sk[i], sv[i], so[i], dev_status=status)
+
+    for i in range(args.warmup):
+        one(i)
+    torch.cuda.synchronize()
+    launches, kernel_names = (1, ["(not counted: --no-profile)"]) if args.no_profile else \
+        count_launches(lambda: one(0))
+    side = torch.cuda.Stream()
+    side.wait_stream(stream)
+    g1, gall = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+    with torch.cuda.stream(side):
+        with torch.cuda.graph(g1, stream=side):
+            one(0)
+        with torch.cuda.graph(gall, stream=side):
+            for i in range(n_graph):
+                one(i)
+    stream.wait_stream(side)
+    torch.cuda.synchronize()
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(dev.index) as clk:
+        for i in range(args.steps):
+            flush.zero_()
+            starts[i].record(stream)
+            g1.replay()
+            ends[i].record(stream)
+        torch.cuda.synchronize()
+    step_ms = [a.elapsed_time(b) for a, b in zip(starts, ends)]
+    ms = torch.tensor([statistics.median(step_ms)], dtype=torch.float64, device=dev)
+    # 1024 consecutive steps in one graph (state stays in L2 between steps)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    gall.replay()
+    torch.cuda.synchronize()
+    e0.record(stream)
+    gall.replay()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    warm_ms = e0.elapsed_time(e1) / n_graph
+    if int(status.item()) != 0:
+        raise RuntimeError(D.dark_status_string(int(status.item())))
+    # end to end: pinned host q, k, v in, the call, out back to the host, per step
+    hq, hk, hv = (t[:args.steps].cpu().pin_memory() for t in (sq, sk, sv))
+    ho = torch.empty_like(hq[0]).pin_memory()
+    dq, dk, dv = (torch.empty_like(sq[0]) for _ in range(3))
+    do = torch.empty_like(dq)
+    e0.record(stream)
+    for i in range(args.steps):
+        dq.copy_(hq[i], non_blocking=True)
+        dk.copy_(hk[i], non_blocking=True)
+        dv.copy_(hv[i], non_blocking=True)
+        D.dark_decode_step(proj, st, dq, dk, dv, do, dev_status=status)
+        ho.copy_(do, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = torch.tensor([e0.elapsed_time(e1) / args.steps], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(ms, op=dist.ReduceOp.MAX)
+        dist.all_reduce(e2e_ms, op=dist.ReduceOp.MAX)
+    if rank != 0:
+        return None
+    rows = w.B * w.H * world
+    t = ms.item() / 1e3
+    peaks = load_peaks()
+    nbytes = decode_bytes(w)
+    achieved = nbytes / t / 1e9
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        kv0 = st_t[0][:1].double().cpu().numpy()
+        z0 = st_t[1][:1].double().cpu().numpy()
+        sub = {n: stream_np[n][:, :1] for n in ("q", "k", "v")}
+        rps, nsteps, secs = oracle_decode_sample(w.with_sizes(B=1), kv0, z0, sub, inp["omega"],
+                                                 inp["geom"])
+        cpu = dict(value=rps, unit="tokens/s", cores=blas_threads(), kind="oracle",
+                   sample=f"batch row 0 ({w.H} heads), {nsteps} decode steps, {secs:.1f} s")
+    clocks = clk.summary()
+    return {
+        "metric": DECODE_METRIC, "value": rows / t, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms.item(),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded numpy, orthogonal Gaussian features)",
+        "config": {"workload": "decode after a 4096-token causal prefill (B64 H8 d64 r64 m256, "
+                               "fp32 state)", "B": w.B, "H": w.H, "d": w.d, "r": w.r, "m": w.m,
+                   "l2": "flushed (512 MiB write) before every timed step",
+                   "timing": "CUDA events around a one-step CUDA-graph replay",
+                   "parallelism": f"replicas x{world} (independent batches, no collective)"},
+        "e2e": {"value": rows / (e2e_ms.item() / 1e3), "unit": "tokens/s",
+                "h2d_bytes_per_step": 3 * dq.numel() * dq.element_size(),
+                "d2h_bytes_per_step": do.numel() * do.element_size()},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm"], "unit": "GB/s",
+                     "frac": achieved / peaks["hbm"], "traffic": None,
+                     "peak_source": peaks["source"], "kernel": "decode_kernel"},
+        "warm_graph_1024": {"ms_per_step": warm_ms, "value": rows / (warm_ms / 1e3),
+                            "GBps_algorithmic": nbytes / (warm_ms / 1e3) / 1e9,
+                            "note": "state L2-resident between steps"},
+        "cpu_baseline": cpu,
+        "gpu_launches": launches * args.steps,
+        "kernels": kernel_names,
+        "clocks": {"sm_mhz": clocks["sm_mhz"], "sm_max_mhz": clocks["sm_max_mhz"],
+                   "reasons": clocks["reasons"], "samples": clocks["samples"]},
+    }
+
+
 def run_reference(args, w: synth.Workload) -> dict:
     inp = synth.make_inputs(w)
     for _ in range(args.warmup):
@@ -337,7 +519,7 @@ def run_reference(args, w: synth.Workload) -> dict:
     sample = f"{details[2]} of {w.B * w.H} (batch, head) slices per step, {details[0]} tokens"
     return {
         "impl": "reference",
-        "metric": "DARK attention fwd tokens/s (B*H*L/s) on B200",
+        "metric": METRIC,
         "value": value, "unit": "tokens/s", "n_gpus": 1, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": w.tokens / value * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
@@ -362,6 +544,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-profile", action="store_true",
                     help="do not count launches with the CUDA profiler (for runs under ncu)")
+    ap.add_argument("--decode", action="store_true",
+                    help="time the streaming decode step (workload 5) instead of the forward")
     ap.add_argument("--ncu", action="store_true",
                     help="capture mode: only warmup + steps forward calls, no timing or output")
     args = ap.parse_args()
@@ -382,7 +566,8 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=dev)
     try:
-        res = run_native(args, w, rank, world, dev)
+        res = run_decode(args, rank, world, dev) if args.decode else \
+            run_native(args, w, rank, world, dev)
         if res is not None:
             print(json.dumps(res), flush=True)
     finally:
