@@ -30,20 +30,22 @@ bool proj_ok(const dark_projection* p) {
          sizes_ok(p->m, p->r, p->d) && p->heads >= 1;
 }
 
-enum class Path { Simt, TcCausal, TcNonCausal };
+enum class Path { Simt, TcCausal, TcNonCausal, TcWide };
 
 Path choose_path(dark::FwdArgs& a) {
   if (a.flags & DARK_CAUSAL) {
     if (dark::tc_causal_supported(a)) return Path::TcCausal;
+    if (dark::tc_wide_supported(a)) return Path::TcWide;
   } else {
     if (dark::tc_noncausal_supported(a)) return Path::TcNonCausal;
   }
   return Path::Simt;
 }
 
-size_t ws_need(Path p, int B, int H, int L, int m, int d, int flags) {
+size_t ws_need(Path p, int B, int H, int L, int m, int r, int d, int flags) {
   switch (p) {
     case Path::TcCausal: return dark::tc_causal_workspace_bytes(B, H, L, m, d);
+    case Path::TcWide: return dark::tc_wide_workspace_bytes(B, H, L, m, d, r);
     case Path::TcNonCausal: return dark::tc_noncausal_workspace_bytes(B, H, L, m, d);
     default: return dark::simt_workspace_bytes(B, H, L, m, d, flags);
   }
@@ -105,7 +107,7 @@ dark_status fwd_prepare(const dark_projection* proj, const void* q, const void* 
 }
 
 size_t fwd_workspace_need(const FwdArgs& a) {
-  return ws_need((Path)a.path, a.B, a.H, a.L, a.m, a.d, a.flags);
+  return ws_need((Path)a.path, a.B, a.H, a.L, a.m, a.r, a.d, a.flags);
 }
 
 dark_status fwd_launch(FwdArgs& a, void* ws, size_t ws_bytes, dark_state* state_out,
@@ -116,6 +118,7 @@ dark_status fwd_launch(FwdArgs& a, void* ws, size_t ws_bytes, dark_state* state_
   switch ((Path)a.path) {
     case Path::TcCausal: e = tc_causal_forward(a); break;
     case Path::TcNonCausal: e = tc_noncausal_forward(a); break;
+    case Path::TcWide: e = tc_wide_forward(a); break;
     default: e = simt_forward(a); break;
   }
   if (e != cudaSuccess) return DARK_ERR_CUDA;
@@ -181,7 +184,10 @@ size_t dark_attention_workspace_bytes(const dark_projection* proj, int B, int H,
   size_t need = dark::simt_workspace_bytes(B, H, L, m, d, flags);
   const size_t tc = (flags & DARK_CAUSAL) ? dark::tc_causal_workspace_bytes(B, H, L, m, d)
                                           : dark::tc_noncausal_workspace_bytes(B, H, L, m, d);
-  return need > tc ? need : tc;
+  const size_t wide =
+      (flags & DARK_CAUSAL) ? dark::tc_wide_workspace_bytes(B, H, L, m, d, proj->r) : 0;
+  if (need < tc) need = tc;
+  return need > wide ? need : wide;
 }
 
 dark_status dark_attention_fwd(const dark_projection* proj, const void* q, const void* k,

@@ -78,6 +78,12 @@ cudaError_t tc_launch_key_states(const FwdArgs& a, const CUtensorMap& tw, const 
 size_t tc_noncausal_workspace_bytes(int B, int H, int L, int m, int d);
 cudaError_t tc_noncausal_forward(const FwdArgs& a);
 
+// Wide heads (d = 128..256, m up to 512), causal: features/scores launch, then
+// a value-block launch carrying the state in TMEM (tcgen05).
+bool tc_wide_supported(FwdArgs& a);
+size_t tc_wide_workspace_bytes(int B, int H, int L, int m, int d, int r);
+cudaError_t tc_wide_forward(const FwdArgs& a);
+
 // Decode step over [B][H] heads.
 struct DecodeArgs {
   int heads_w, m, r, d;

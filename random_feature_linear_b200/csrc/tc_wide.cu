@@ -1,0 +1,805 @@
+// Causal (and key-masked) PRF attention forward for wide heads (d = 128..256,
+// m up to 512) on sm_100a tensor cores.
+//
+// DARKformer README, section "Kernel": phi(x) = m^{-1/2} exp(omega^T M x~ -
+// 1/2 |M x~|^2) and out = Phi(Q)(Phi(K)^T V) / Phi(Q)(Phi(K)^T 1); section
+// "Self-attention": the causal constraint (diagonal included) combined with the
+// key mask. Per 128-token chunk c (Psi drops the per-query factors of phi):
+//
+//   num_c = tril(Psi(Q_c) Phi(K_c)^T) [V_c | 1] + Psi(Q_c) [S_<c | z_<c]
+//   out_c = num_c[:, :d] / num_c[:, d]
+//   [S_<=c | z_<=c] = [S_<c | z_<c] + Phi(K_c)^T [V_c | 1]
+//
+// At d = 256, m = 512 one head's state [S | z] is 512 x 257 fp32 (526 KB),
+// more than one SM's shared memory or TMEM, so it cannot ride along with one
+// CTA as in the d = 64 kernel. The work is split in two launches:
+//
+//  1. features_kernel, one CTA per (head, chunk): the feature GEMMs K_c W'^T
+//     and Q_c W^T (fp16 operands, fp32 in TMEM) share every streamed W' slab;
+//     the epilogue warps turn them into Phi(K_c), Psi(Q_c) (bf16) in 64-feature
+//     blocks while the next block's GEMM runs, the scores Psi Phi^T accumulate
+//     on the tensor cores block by block, and Phi, Psi and the masked causal
+//     scores A_c are bulk-copied to the workspace as ready shared-memory operand
+//     images (128B-swizzled, so the second launch copies them back verbatim).
+//  2. values_kernel, one CTA per (head, 64 value columns): walks the chunks in
+//     order with its slice of the state, m x (64 + 1) fp32, resident in TMEM
+//     (m/128 tiles of 128 features x 80 columns). Per chunk and feature tile f
+//     the epilogue warps copy S_f to shared memory as hi + lo bf16 operands
+//     (bf16 alone moves outputs by ~1e-2), then the tensor cores run
+//       num += Psi_f [S_f | z_f]  (hi and lo)   and   S_f += Phi_f^T [V_c | 1]
+//     after num = A_c [V_c | 1]; the epilogue divides and stores out_c.
+//
+// In both kernels warp 8 is the producer (TMA / bulk copies) and the MMA
+// issuer; warps 0-7 are the epilogue (TMEM lane quadrant = warp % 4). Every
+// wait is bounded: a wait that runs out records DARK_ERR_TIMEOUT and raises the
+// CTA's abort flag, every role leaves its loop, in-flight copies are waited for
+// (bounded), and TMEM is freed.
+#include <string.h>
+
+#include "common.cuh"
+#include "internal.h"
+#include "tc_common.cuh"
+
+namespace dark {
+namespace {
+
+using namespace tc;
+
+constexpr int kC = 128;              // tokens per chunk (UMMA M)
+constexpr int kEpiThreads = 256;     // warps 0-7
+constexpr int kThreads = kEpiThreads + 32;
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kSmemBudget = 229376;   // 224 KB of operands + barriers + alignment slack
+
+// ------------------------------------------------------------ sync helpers --
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+// shared -> global bulk copy (16-byte aligned, size a multiple of 16)
+__device__ __forceinline__ void bulk_store(void* gdst, uint32_t ssrc, uint32_t bytes) {
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"((uint64_t)gdst),
+               "r"(ssrc), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() {
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+__device__ __forceinline__ void bulk_wait_read_all() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+__device__ __forceinline__ void bulk_wait_all() {
+  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+}
+// Barrier 1 over the 256 epilogue threads; true if any of them passes `bad`.
+__device__ __forceinline__ bool epi_sync_or(bool bad) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "barrier.cta.red.or.pred q, 1, 256, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)bad)
+      : "memory");
+  return r != 0;
+}
+__device__ __forceinline__ void epi_sync() { asm volatile("barrier.cta.sync 1, 256;" ::: "memory"); }
+
+// Bounded wait of one thread. A wait that runs out records DARK_ERR_TIMEOUT and
+// raises the abort flag; a raised flag ends every other wait of the CTA.
+__device__ __forceinline__ bool wait_one(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                         int* dev_status) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const long long t0 = clock64();
+  while (!mbar_try_wait(bar, parity)) {
+    if (*abort_flag) return false;
+    if (clock64() - t0 > kWaitCycles) {
+      *abort_flag = 1;
+      report(dev_status, DARK_ERR_TIMEOUT);
+      return false;
+    }
+  }
+  return true;
+}
+// The same for the epilogue warps: all 256 wait, then agree.
+__device__ __forceinline__ bool epi_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                         int* dev_status) {
+  const bool ok = wait_one(bar, parity, abort_flag, dev_status);
+  return !epi_sync_or(!ok);
+}
+// Epilogue warp -> producer/MMA thread: one arrival per warp (barrier count 8).
+__device__ __forceinline__ void warp_arrive(uint64_t* bar) {
+  __syncwarp();
+  if ((threadIdx.x & 31) == 0) mbar_arrive(bar);
+}
+
+// ================================================================ launch 1 ==
+template <int D_, int M_, int R_>
+struct FeatCfg {
+  static constexpr int DS = D_ / 64;                       // 64-column slabs of d
+  static constexpr int NNORM = R_ / 64, NFEAT = M_ / 64;   // W' items of 64 rows
+  static constexpr int NITEMS = NNORM + NFEAT;
+  static constexpr uint32_t kX = DS * 16384;               // one 128-token tile, fp16
+  static constexpr uint32_t kSlot = DS * 8192;             // 64 W' rows x d, fp16
+  static constexpr uint32_t oXK = 0, oXQ = kX, oST = 2 * kX;   // staging: Phi_n | Psi_n, later A
+  static constexpr uint32_t oW = oST + 32768;
+  static constexpr int kSlotsFit = (int)((kSmemBudget - oW) / kSlot);
+  static constexpr int NSLOT = kSlotsFit > 6 ? 6 : kSlotsFit;
+  static constexpr uint32_t oBar = oW + NSLOT * kSlot;
+  static constexpr uint32_t kSmem = oBar + 1024 + 1024 + 1024;   // barriers, norm exchange, slack
+  // TMEM: norms [0, R_) first; then P blocks (keys at 128 b, queries at 128 b + 64,
+  // b = block parity) over the same columns; scores [256, 384)
+  static constexpr uint32_t tS = 256;
+  static_assert(D_ % 64 == 0 && D_ >= 128 && D_ <= 256, "d");
+  static_assert(M_ % 128 == 0 && M_ <= 512 && R_ % 64 == 0 && R_ >= 64 && R_ <= 256, "m, r");
+  static_assert(NSLOT >= 2, "shared memory");
+};
+
+// Bytes of one chunk's record in the workspace: Phi image, Psi image, A image.
+__host__ __device__ constexpr size_t chunk_record_bytes(int m) {
+  return (size_t)2 * m * 256 + 32768;
+}
+
+struct FeatParams {
+  const uint8_t* mask;
+  uint8_t* img;            // chunk records [B*H][nc]
+  int B, H, L, nc, heads_w;
+  int* dev_status;
+};
+
+template <int D_, int M_, int R_>
+__global__ void __launch_bounds__(kThreads, 1)
+    features_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_q,
+                    const __grid_constant__ CUtensorMap tm_k, const FeatParams p) {
+  using G = FeatCfg<D_, M_, R_>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  const uint32_t s0 = smem_u32(sm);
+  uint64_t* bars = (uint64_t*)(sm + G::oBar);
+  uint64_t* bar_x = bars + 0;
+  uint64_t* bar_conv = bars + 1;        // epilogue: tiles converted to fp16 (8 arrivals)
+  uint64_t* bar_norm = bars + 2;        // MMA: norm GEMM done
+  uint64_t* bar_nread = bars + 3;       // epilogue: norm columns read (8)
+  uint64_t* bar_pfull = bars + 4;       // [2] MMA: P block ready
+  uint64_t* bar_stage = bars + 6;       // epilogue: P block read, staging written (8)
+  uint64_t* bar_sfree = bars + 7;       // MMA: scores GEMM of the staged block done
+  uint64_t* bar_full = bars + 8;        // [NSLOT] W' slot loaded
+  uint64_t* bar_empty = bars + 16;      // [NSLOT] W' slot read by the MMAs
+  uint32_t* tmem_slot = (uint32_t*)(bars + 24);
+  volatile int* abort_flag = (volatile int*)(bars + 25);
+  float* nrm_x = (float*)(sm + G::oBar + 1024);   // [2][128] norm halves
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int bh = blockIdx.x / p.nc, c = blockIdx.x % p.nc;
+  const int b = bh / p.H, h = bh % p.H;
+  const int hw = p.heads_w == 1 ? 0 : h;
+  const int t0 = c * kC;
+  uint8_t* rec = p.img + ((size_t)bh * p.nc + c) * chunk_record_bytes(M_);
+
+  if (tid == 0) {
+    mbar_init(bar_x, 1);
+    mbar_init(bar_conv, 8);
+    mbar_init(bar_norm, 1);
+    mbar_init(bar_nread, 8);
+    mbar_init(bar_pfull + 0, 1);
+    mbar_init(bar_pfull + 1, 1);
+    mbar_init(bar_stage, 8);
+    mbar_init(bar_sfree, 1);
+    for (int i = 0; i < G::NSLOT; ++i) {
+      mbar_init(bar_full + i, 1);
+      mbar_init(bar_empty + i, 1);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0) tmem_alloc(tmem_slot, kTmemCols);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 8) {
+    // ------------------------------------------- producer and MMA issuer
+    if (lane == 0) {
+      prefetch_tmap(&tm_w);
+      prefetch_tmap(&tm_q);
+      prefetch_tmap(&tm_k);
+      mbar_arrive_expect_tx(bar_x, 2 * G::kX);
+      for (int s = 0; s < G::DS; ++s) {
+        tma_load_4d(sm + G::oXK + s * 16384, &tm_k, 64 * s, t0, h, b, bar_x);
+        tma_load_4d(sm + G::oXQ + s * 16384, &tm_q, 64 * s, t0, h, b, bar_x);
+      }
+      int issued = 0, waited = 0;   // W' items loaded / waited for, in order
+      auto load_item = [&](int i) {
+        const int slot = i % G::NSLOT;
+        const int row0 = i < G::NNORM ? M_ + 64 * i : 64 * (i - G::NNORM);
+        mbar_arrive_expect_tx(bar_full + slot, G::kSlot);
+        for (int s = 0; s < G::DS; ++s)
+          tma_load_2d(sm + G::oW + slot * G::kSlot + s * 8192, &tm_w, 64 * s,
+                      hw * (M_ + R_) + row0, bar_full + slot);
+      };
+      for (; issued < G::NSLOT && issued < G::NITEMS; ++issued) load_item(issued);
+      const uint32_t sXK = s0 + G::oXK, sXQ = s0 + G::oXQ;
+      // after issuing item i: refill the slot item i-1 used, once its MMAs are done
+      auto refill = [&](int i) -> bool {
+        if (i < 1 || issued >= G::NITEMS) return true;
+        const int j = i - 1;
+        if (!wait_one(bar_empty + j % G::NSLOT, (j / G::NSLOT) & 1, abort_flag, p.dev_status))
+          return false;
+        load_item(issued++);
+        return true;
+      };
+      auto feat_block = [&](int n) -> bool {   // K and Q GEMMs of feature block n
+        const int i = G::NNORM + n, slot = i % G::NSLOT;
+        if (!wait_one(bar_full + slot, (i / G::NSLOT) & 1, abort_flag, p.dev_status)) return false;
+        ++waited;
+        tc_fence_after();
+        const uint32_t sw = s0 + G::oW + slot * G::kSlot;
+        const uint32_t tp = tmem + 128 * (n & 1);
+        constexpr uint32_t id = idesc(128, 64, false, false, true);
+#pragma unroll
+        for (int s = 0; s < G::DS; ++s)
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const uint64_t bd = sdesc(sw + s * 8192 + k * 32, 16, 1024);
+            mma(tp, sdesc(sXK + s * 16384 + k * 32, 16, 1024), bd, id, (s | k) != 0);
+            mma(tp + 64, sdesc(sXQ + s * 16384 + k * 32, 16, 1024), bd, id, (s | k) != 0);
+          }
+        mma_commit(bar_empty + slot);
+        mma_commit(bar_pfull + (n & 1));
+        return refill(i);
+      };
+      bool ok = wait_one(bar_conv, 0, abort_flag, p.dev_status);
+      // ---- norm GEMM: columns [0, R_)
+      for (int i = 0; ok && i < G::NNORM; ++i) {
+        const int slot = i % G::NSLOT;
+        if (!(ok = wait_one(bar_full + slot, (i / G::NSLOT) & 1, abort_flag, p.dev_status))) break;
+        ++waited;
+        tc_fence_after();
+        const uint32_t sw = s0 + G::oW + slot * G::kSlot;
+        constexpr uint32_t id = idesc(128, 64, false, false, true);
+#pragma unroll
+        for (int s = 0; s < G::DS; ++s)
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            mma(tmem + 64 * i, sdesc(sXK + s * 16384 + k * 32, 16, 1024),
+                sdesc(sw + s * 8192 + k * 32, 16, 1024), id, (s | k) != 0);
+        mma_commit(bar_empty + slot);
+        ok = refill(i);
+      }
+      if (ok) mma_commit(bar_norm);
+      // ---- feature blocks (P buffers overwrite the norm columns once read)
+      if (ok) ok = wait_one(bar_nread, 0, abort_flag, p.dev_status);
+      if (ok) ok = feat_block(0);
+      if (ok && G::NFEAT > 1) ok = feat_block(1);
+      for (int n = 0; ok && n < G::NFEAT; ++n) {
+        // block n staged by the epilogue: scores += Psi_n Phi_n^T
+        if (!(ok = wait_one(bar_stage, n & 1, abort_flag, p.dev_status))) break;
+        tc_fence_after();
+        constexpr uint32_t ids = idesc(128, 128, false, false, false);
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+          mma(tmem + G::tS, sdesc(s0 + G::oST + 16384 + k * 32, 16, 1024),
+              sdesc(s0 + G::oST + k * 32, 16, 1024), ids, (n | k) != 0);
+        mma_commit(bar_sfree);
+        if (n + 2 < G::NFEAT) ok = feat_block(n + 2);
+      }
+      // leave no copy in flight: the token tiles and the W' items not waited for
+      if (!ok) {
+        mbar_wait(bar_x, 0);
+        for (int i = waited; i < issued; ++i) mbar_wait(bar_full + i % G::NSLOT, (i / G::NSLOT) & 1);
+      }
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int etid = tid, quad = warp & 3, half = warp >> 2;
+    const int row = quad * 32 + lane;
+    const uint32_t lane_tm = tmem + ((uint32_t)(quad * 32) << 16);
+    const int tok = t0 + row;
+    bool valid = tok < p.L;
+    if (valid && p.mask != nullptr) valid = p.mask[(size_t)b * p.L + tok] != 0;
+    bool ok = epi_wait(bar_x, 0, abort_flag, p.dev_status);
+    if (ok) {
+      // bf16 -> fp16 in place (both tiles; |x| >= 65504 is reported)
+      bool bad = false;
+      for (int i = etid; i < (int)(2 * G::kX / 16); i += kEpiThreads) {
+        const uint32_t a = s0 + G::oXK + i * 16;
+        uint4 u = ld_shared_v4(a);
+        uint32_t* w32 = &u.x;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w32[e]));
+          bad |= fabsf(f.x) > 65504.f || fabsf(f.y) > 65504.f;
+          const __half2 hv = __floats2half2_rn(f.x, f.y);
+          w32[e] = *reinterpret_cast<const uint32_t*>(&hv);
+        }
+        st_shared_v4(a, u.x, u.y, u.z, u.w);
+      }
+      if (bad) report(p.dev_status, DARK_ERR_NUMERIC);
+      fence_async_smem();
+      warp_arrive(bar_conv);
+      ok = epi_wait(bar_norm, 0, abort_flag, p.dev_status);
+    }
+    float nrm = 0.f;
+    if (ok) {
+      tc_fence_after();
+      float part = 0.f;
+#pragma unroll 1
+      for (int c0 = half * (R_ / 2); c0 < (half + 1) * (R_ / 2); c0 += 32) {
+        float v[32];
+        tmem_ld32(lane_tm + c0, v);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) part = fmaf(v[i], v[i], part);
+      }
+      nrm_x[half * 128 + row] = part;
+      tc_fence_before();
+      epi_sync();
+      nrm = nrm_x[row] + nrm_x[128 + row] + 0.5f * __log2f((float)M_);
+      warp_arrive(bar_nread);
+    }
+    uint8_t* g_phi = rec;
+    uint8_t* g_psi = rec + (size_t)M_ * 256;
+    const uint32_t st_phi = s0 + G::oST, st_psi = s0 + G::oST + 16384;
+    for (int n = 0; ok && n < G::NFEAT; ++n) {
+      if (!(ok = epi_wait(bar_pfull + (n & 1), (n >> 1) & 1, abort_flag, p.dev_status))) break;
+      if (n > 0) {
+        // staging is free once the scores GEMM and the bulk stores of block n-1 read it
+        if (!(ok = epi_wait(bar_sfree, (n - 1) & 1, abort_flag, p.dev_status))) break;
+        if (etid == 0) bulk_wait_read_all();
+        epi_sync();
+      }
+      tc_fence_after();
+      const uint32_t tp = lane_tm + 128 * (n & 1);
+      if (half == 0)
+        exp2_rows_to_smem(tp, 0, 64, nrm, !valid, st_phi, row);
+      else
+        exp2_rows_to_smem(tp + 64, 0, 64, 0.f, false, st_psi, row);
+      tc_fence_before();
+      fence_async_smem();
+      epi_sync();
+      if (etid == 0) {
+        bulk_store(g_phi + (size_t)n * 16384, st_phi, 16384);
+        bulk_store(g_psi + (size_t)n * 16384, st_psi, 16384);
+        bulk_commit();
+      }
+      warp_arrive(bar_stage);
+    }
+    // ------------------------------ masked causal scores -> A image
+    if (ok) ok = epi_wait(bar_sfree, (G::NFEAT - 1) & 1, abort_flag, p.dev_status);
+    if (ok) {
+      if (etid == 0) bulk_wait_read_all();
+      epi_sync();
+      tc_fence_after();
+      float v[32];
+#pragma unroll
+      for (int j0 = half * 64; j0 < half * 64 + 64; j0 += 32) {
+        tmem_ld32(lane_tm + G::tS + j0, v);
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+          uint32_t w4[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int j = j0 + 8 * g + 2 * e;
+            w4[e] = pack_bf16(j <= row ? v[8 * g + 2 * e] : 0.f,
+                              j + 1 <= row ? v[8 * g + 2 * e + 1] : 0.f);
+          }
+          st_shared_v4(s0 + G::oST + kmajor_off(row, j0 + 8 * g, 16384), w4[0], w4[1], w4[2], w4[3]);
+        }
+      }
+      tc_fence_before();
+      fence_async_smem();
+      epi_sync();
+      if (etid == 0) {
+        bulk_store(rec + (size_t)2 * M_ * 256, s0 + G::oST, 32768);
+        bulk_commit();
+      }
+    }
+    if (etid == 0) bulk_wait_all();
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// ================================================================ launch 2 ==
+template <int M_>
+struct ValCfg {
+  static constexpr int NT = M_ / 128;        // feature tiles of the state
+  static constexpr int NITEM = 2 * NT;       // per chunk: Psi_f, Phi_f (32 KB each)
+  static constexpr int NSLOT = 3;
+  static constexpr uint32_t oA = 0;          // A_c image, 32 KB
+  static constexpr uint32_t oV = 32768;      // V_c slices, 2 x 16 KB
+  static constexpr uint32_t oR = 65536;      // ring, NSLOT x 32 KB
+  static constexpr uint32_t oS = oR + NSLOT * 32768;   // S hi | S lo | z hi | z lo
+  static constexpr uint32_t oOnes = oS + 40960;
+  static constexpr uint32_t oBar = oOnes + 2048;
+  static constexpr uint32_t kSmem = oBar + 1024 + 1024;
+  // TMEM: state tile f at columns 80 f (64 values, then z in 16 columns); numerator after
+  static constexpr uint32_t tNum = 80 * NT;
+  static_assert(M_ % 128 == 0 && M_ <= 512 && tNum + 80 <= kTmemCols, "m");
+};
+
+struct ValParams {
+  const uint8_t* img;
+  __nv_bfloat16* out;
+  int64_t ob, oh, ol;
+  int B, H, L, nc, nvb;
+  float *st_kv, *st_z;
+  int d;
+  int* dev_status;
+};
+
+template <int M_>
+__global__ void __launch_bounds__(kThreads, 1)
+    values_kernel(const __grid_constant__ CUtensorMap tm_v, const ValParams p) {
+  using G = ValCfg<M_>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  const uint32_t s0 = smem_u32(sm);
+  uint64_t* bars = (uint64_t*)(sm + G::oBar);
+  uint64_t* bar_av = bars + 0;          // [2] A_c and V_c slice loaded
+  uint64_t* bar_aempty = bars + 2;      // MMA: intra GEMM (reads A_c) done
+  uint64_t* bar_vempty = bars + 3;      // [2] MMA: every GEMM of the chunk done (V slot free)
+  uint64_t* bar_simg = bars + 5;        // epilogue: S image of tile f written (8)
+  uint64_t* bar_sfree = bars + 6;       // MMA: inter GEMM of tile f done (S image free)
+  uint64_t* bar_nfull = bars + 7;       // MMA: numerator of the chunk complete
+  uint64_t* bar_nfree = bars + 8;       // epilogue: numerator read (8)
+  uint64_t* bar_full = bars + 9;        // [3] ring slot loaded
+  uint64_t* bar_empty = bars + 12;      // [3] ring slot read
+  uint32_t* tmem_slot = (uint32_t*)(bars + 16);
+  volatile int* abort_flag = (volatile int*)(bars + 17);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int bh = blockIdx.x / p.nvb, vb = blockIdx.x % p.nvb;
+  const int b = bh / p.H, h = bh % p.H;
+  const size_t rec_bytes = chunk_record_bytes(M_);
+  const uint8_t* recs = p.img + (size_t)bh * p.nc * rec_bytes;
+
+  if (tid == 0) {
+    mbar_init(bar_av + 0, 1);
+    mbar_init(bar_av + 1, 1);
+    mbar_init(bar_aempty, 1);
+    mbar_init(bar_vempty + 0, 1);
+    mbar_init(bar_vempty + 1, 1);
+    mbar_init(bar_simg, 8);
+    mbar_init(bar_sfree, 1);
+    mbar_init(bar_nfull, 1);
+    mbar_init(bar_nfree, 8);
+    for (int i = 0; i < G::NSLOT; ++i) {
+      mbar_init(bar_full + i, 1);
+      mbar_init(bar_empty + i, 1);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  // ones tile (bf16 1.0): 16 rows x 64, K-major, for the z / denominator columns
+  for (int i = tid; i < 2048 / 4; i += kThreads) ((uint32_t*)(sm + G::oOnes))[i] = 0x3F803F80u;
+  fence_async_smem();
+  if (warp == 0) tmem_alloc(tmem_slot, kTmemCols);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 8) {
+    // ------------------------------------------- producer and MMA issuer
+    if (lane == 0) {
+      prefetch_tmap(&tm_v);
+      const int total = p.nc * G::NITEM;
+      int issued = 0, waited = 0;        // ring items loaded / waited for, in order
+      int av_issued = 0, av_waited = 0;  // chunks whose A_c, V_c were loaded / waited for
+      auto load_item = [&](int g) {
+        const int c = g / G::NITEM, i = g % G::NITEM, f = i >> 1;
+        const uint8_t* src = recs + (size_t)c * rec_bytes + ((i & 1) ? 0 : (size_t)M_ * 256) +
+                             (size_t)f * 32768;
+        const int slot = g % G::NSLOT;
+        mbar_arrive_expect_tx(bar_full + slot, 32768);
+        bulk_load(sm + G::oR + slot * 32768, src, 32768, bar_full + slot);
+      };
+      auto load_av = [&](int c) -> bool {
+        if (c > 0 && !wait_one(bar_aempty, (c - 1) & 1, abort_flag, p.dev_status)) return false;
+        if (c > 1 && !wait_one(bar_vempty + (c & 1), ((c - 2) >> 1) & 1, abort_flag, p.dev_status))
+          return false;
+        mbar_arrive_expect_tx(bar_av + (c & 1), 32768 + 16384);
+        bulk_load(sm + G::oA, recs + (size_t)c * rec_bytes + (size_t)2 * M_ * 256, 32768,
+                  bar_av + (c & 1));
+        tma_load_4d(sm + G::oV + (c & 1) * 16384, &tm_v, 64 * vb, c * kC, h, b, bar_av + (c & 1));
+        av_issued = c + 1;
+        return true;
+      };
+      // after issuing the MMAs of item g: refill the slot item g-1 used
+      auto refill = [&](int g) -> bool {
+        if (g < 1 || issued >= total) return true;
+        const int j = g - 1;
+        if (!wait_one(bar_empty + j % G::NSLOT, (j / G::NSLOT) & 1, abort_flag, p.dev_status))
+          return false;
+        load_item(issued++);
+        return true;
+      };
+      bool ok = load_av(0);
+      for (; ok && issued < G::NSLOT && issued < total; ++issued) load_item(issued);
+      const uint32_t sA = s0 + G::oA, sSh = s0 + G::oS, sSl = sSh + 16384;
+      const uint32_t sZh = sSh + 32768, sZl = sZh + 4096, sOnes = s0 + G::oOnes;
+      const uint32_t tnum = tmem + G::tNum;
+      for (int c = 0; ok && c < p.nc; ++c) {
+        if (!(ok = wait_one(bar_av + (c & 1), (c >> 1) & 1, abort_flag, p.dev_status))) break;
+        ++av_waited;
+        if (c > 0 && !(ok = wait_one(bar_nfree, (c - 1) & 1, abort_flag, p.dev_status))) break;
+        tc_fence_after();
+        const uint32_t sV = s0 + G::oV + (c & 1) * 16384;
+        // num = A_c [V_c | 1]
+        {
+          constexpr uint32_t idv = idesc(128, 64, false, true, false);
+          constexpr uint32_t id1 = idesc(128, 16, false, false, false);
+#pragma unroll
+          for (int s = 0; s < kC / 16; ++s) {
+            const uint64_t ad = sdesc(sA + (s / 4) * 16384 + (s % 4) * 32, 16, 1024);
+            mma(tnum, ad, sdesc(sV + s * 2048, 16384, 1024), idv, s > 0);
+            mma(tnum + 64, ad, sdesc(sOnes + (s % 4) * 32, 16, 1024), id1, s > 0);
+          }
+          mma_commit(bar_aempty);
+        }
+        for (int f = 0; ok && f < G::NT; ++f) {
+          const int g = c * G::NITEM + 2 * f;
+          if (!(ok = wait_one(bar_simg, (c * G::NT + f) & 1, abort_flag, p.dev_status))) break;
+          if (!(ok = wait_one(bar_full + g % G::NSLOT, (g / G::NSLOT) & 1, abort_flag, p.dev_status)))
+            break;
+          ++waited;
+          tc_fence_after();
+          // num += Psi_f [S_f | z_f], S and z as hi + lo bf16
+          {
+            const uint32_t sPsi = s0 + G::oR + (g % G::NSLOT) * 32768;
+            constexpr uint32_t idv = idesc(128, 64, false, true, false);
+            constexpr uint32_t id1 = idesc(128, 16, false, false, false);
+#pragma unroll
+            for (int s = 0; s < 8; ++s) {
+              const uint64_t ad = sdesc(sPsi + (s / 4) * 16384 + (s % 4) * 32, 16, 1024);
+              mma(tnum, ad, sdesc(sSh + s * 2048, 16384, 1024), idv, 1);
+              mma(tnum, ad, sdesc(sSl + s * 2048, 16384, 1024), idv, 1);
+              mma(tnum + 64, ad, sdesc(sZh + (s / 4) * 2048 + (s % 4) * 32, 16, 1024), id1, 1);
+              mma(tnum + 64, ad, sdesc(sZl + (s / 4) * 2048 + (s % 4) * 32, 16, 1024), id1, 1);
+            }
+            mma_commit(bar_sfree);
+            mma_commit(bar_empty + g % G::NSLOT);
+          }
+          if (!(ok = refill(g))) break;
+          if (f == 0 && c + 1 < p.nc && !(ok = load_av(c + 1))) break;
+          if (!(ok = wait_one(bar_full + (g + 1) % G::NSLOT, ((g + 1) / G::NSLOT) & 1, abort_flag,
+                              p.dev_status)))
+            break;
+          ++waited;
+          tc_fence_after();
+          // S_f += Phi_f^T [V_c | 1]
+          {
+            const uint32_t sPhi = s0 + G::oR + ((g + 1) % G::NSLOT) * 32768;
+            const uint32_t ts = tmem + 80 * f;
+            constexpr uint32_t idv = idesc(128, 64, true, true, false);
+            constexpr uint32_t id1 = idesc(128, 16, true, false, false);
+#pragma unroll
+            for (int s = 0; s < kC / 16; ++s) {
+              const uint64_t ad = sdesc(sPhi + s * 2048, 16384, 1024);
+              mma(ts, ad, sdesc(sV + s * 2048, 16384, 1024), idv, (c > 0) || (s > 0));
+              mma(ts + 64, ad, sdesc(sOnes + (s % 4) * 32, 16, 1024), id1, (c > 0) || (s > 0));
+            }
+            mma_commit(bar_empty + (g + 1) % G::NSLOT);
+          }
+          if (!(ok = refill(g + 1))) break;
+        }
+        if (!ok) break;
+        mma_commit(bar_nfull);
+        mma_commit(bar_vempty + (c & 1));
+      }
+      if (!ok) {
+        // leave no copy in flight
+        for (int g = waited; g < issued; ++g) mbar_wait(bar_full + g % G::NSLOT, (g / G::NSLOT) & 1);
+        for (int c = av_waited; c < av_issued; ++c) mbar_wait(bar_av + (c & 1), (c >> 1) & 1);
+      }
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int quad = warp & 3, half = warp >> 2;
+    const int row = quad * 32 + lane;               // TMEM lane: feature of a tile / query row
+    const uint32_t lane_tm = tmem + ((uint32_t)(quad * 32) << 16);
+    const uint32_t sSh = s0 + G::oS, sSl = sSh + 16384, sZh = sSh + 32768, sZl = sZh + 4096;
+    bool ok = true;
+    for (int c = 0; ok && c < p.nc; ++c) {
+      for (int f = 0; f < G::NT; ++f) {
+        const int k = c * G::NT + f;
+        if (k > 0 && !(ok = epi_wait(bar_sfree, (k - 1) & 1, abort_flag, p.dev_status))) break;
+        tc_fence_after();
+        // S_f (row `row` of the tile) as hi + lo bf16: MN-major values, K-major z
+        float x[33];
+        if (c == 0) {
+#pragma unroll
+          for (int i = 0; i < 33; ++i) x[i] = 0.f;
+        } else {
+          uint32_t a[32];
+          tmem_ld32_async(lane_tm + 80 * f + 32 * half, a);
+          tmem_wait_ld(a);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) x[i] = __uint_as_float(a[i]);
+          x[32] = half == 0 ? tmem_ld1(lane_tm + 80 * f + 64) : 0.f;
+        }
+        const uint32_t rowoff = (uint32_t)(row / 8) * 1024 + (uint32_t)(row % 8) * 128;
+#pragma unroll
+        for (int cg = 0; cg < 4; ++cg) {
+          uint32_t hi4[4], lo4[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float x0 = x[8 * cg + 2 * e], x1 = x[8 * cg + 2 * e + 1];
+            const __nv_bfloat162 hv = __floats2bfloat162_rn(x0, x1);
+            const float2 hf = __bfloat1622float2(hv);
+            hi4[e] = *reinterpret_cast<const uint32_t*>(&hv);
+            lo4[e] = pack_bf16(x0 - hf.x, x1 - hf.y);
+          }
+          const uint32_t off = rowoff + (uint32_t)(((4 * half + cg) ^ (row % 8)) * 16);
+          st_shared_v4(sSh + off, hi4[0], hi4[1], hi4[2], hi4[3]);
+          st_shared_v4(sSl + off, lo4[0], lo4[1], lo4[2], lo4[3]);
+        }
+        if (half == 0) {
+          const __nv_bfloat16 zh = __float2bfloat16_rn(x[32]);
+          const __nv_bfloat16 zl = __float2bfloat16_rn(x[32] - __bfloat162float(zh));
+          const uint16_t zhb = *reinterpret_cast<const uint16_t*>(&zh);
+          const uint16_t zlb = *reinterpret_cast<const uint16_t*>(&zl);
+#pragma unroll
+          for (int n = 0; n < 16; ++n) {
+            const uint32_t off = (uint32_t)(row / 64) * 2048 + kmajor_off(n, row % 64, 0);
+            st_shared_u16(sZh + off, zhb);
+            st_shared_u16(sZl + off, zlb);
+          }
+        }
+        tc_fence_before();
+        fence_async_smem();
+        warp_arrive(bar_simg);
+      }
+      if (!ok) break;
+      // ---------------------------------------------- out_c = num / den
+      if (!(ok = epi_wait(bar_nfull, c & 1, abort_flag, p.dev_status))) break;
+      tc_fence_after();
+      {
+        uint32_t a[32];
+        tmem_ld32_async(lane_tm + G::tNum + 32 * half, a);
+        tmem_wait_ld(a);
+        const float den = tmem_ld1(lane_tm + G::tNum + 64);
+        const int tok = c * kC + row;
+        if (tok < p.L) {
+          const float inv = den > 0.f ? 1.f / den : 0.f;
+          uint32_t w[16];
+          bool bad = !isfinite(den);
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const float o0 = __uint_as_float(a[2 * e]) * inv, o1 = __uint_as_float(a[2 * e + 1]) * inv;
+            bad |= !isfinite(o0) || !isfinite(o1);
+            w[e] = pack_bf16(o0, o1);
+          }
+          if (bad) report(p.dev_status, DARK_ERR_NUMERIC);
+          uint4* dst = reinterpret_cast<uint4*>(p.out + (int64_t)b * p.ob + (int64_t)h * p.oh +
+                                                (int64_t)tok * p.ol + 64 * vb + 32 * half);
+#pragma unroll
+          for (int q4 = 0; q4 < 4; ++q4)
+            dst[q4] = make_uint4(w[4 * q4], w[4 * q4 + 1], w[4 * q4 + 2], w[4 * q4 + 3]);
+        }
+      }
+      tc_fence_before();
+      warp_arrive(bar_nfree);
+    }
+    // final state [S | z] (every GEMM of the last chunk is complete)
+    if (ok && p.st_kv != nullptr) {
+      tc_fence_after();
+      for (int f = 0; f < G::NT; ++f) {
+        uint32_t a[32];
+        tmem_ld32_async(lane_tm + 80 * f + 32 * half, a);
+        tmem_wait_ld(a);
+        const int feat = 128 * f + row;
+        float* kv = p.st_kv + ((size_t)bh * M_ + feat) * p.d + 64 * vb + 32 * half;
+#pragma unroll
+        for (int i = 0; i < 32; ++i) kv[i] = __uint_as_float(a[i]);
+        const float z = tmem_ld1(lane_tm + 80 * f + 64);
+        if (vb == 0 && half == 0) p.st_z[(size_t)bh * M_ + feat] = z;
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// ------------------------------------------------------------------ host --
+bool make_wide_maps(FwdArgs& a) {
+  auto al16 = [](const void* p) { return ((uintptr_t)p & 15) == 0; };
+  if (!al16(a.q) || !al16(a.k) || !al16(a.v) || !al16(a.out) || !al16(a.w)) return false;
+  for (int i = 0; i < 3; ++i)
+    if (a.qs[i] % 8 != 0 || a.os[i] % 8 != 0) return false;
+  const uint64_t wd[2] = {(uint64_t)a.d, (uint64_t)a.heads_w * (a.m + a.r)};
+  const uint64_t wsd[1] = {(uint64_t)a.d * 2};
+  const uint32_t wb[2] = {64, 64};
+  const uint64_t xd[4] = {(uint64_t)a.d, (uint64_t)a.L, (uint64_t)a.H, (uint64_t)a.B};
+  const uint64_t xs[3] = {(uint64_t)a.qs[2] * 2, (uint64_t)a.qs[1] * 2, (uint64_t)a.qs[0] * 2};
+  const uint32_t xb[4] = {64, 128, 1, 1};
+  a.maps_ready = encode_tmap(&a.tm_w, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, a.w, wd, wsd, wb) &&
+                 encode_tmap(&a.tm_q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, a.q, xd, xs, xb) &&
+                 encode_tmap(&a.tm_k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, a.k, xd, xs, xb) &&
+                 encode_tmap(&a.tm_v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, a.v, xd, xs, xb);
+  return a.maps_ready;
+}
+
+bool shape_ok(int d, int m, int r) {
+  return (d == 256 && m == 512 && r == 256) || (d == 128 && m == 256 && r == 128) ||
+         (d == 128 && m == 128 && r == 64);
+}
+
+template <int D_, int M_, int R_>
+cudaError_t launch(const FwdArgs& a) {
+  using F = FeatCfg<D_, M_, R_>;
+  using V = ValCfg<M_>;
+  const int nc = (a.L + kC - 1) / kC;
+  uint8_t* img = (uint8_t*)a.ws + kWsHeader;
+  FeatParams fp;
+  fp.mask = a.mask;
+  fp.img = img;
+  fp.B = a.B;
+  fp.H = a.H;
+  fp.L = a.L;
+  fp.nc = nc;
+  fp.heads_w = a.heads_w;
+  fp.dev_status = a.dev_status;
+  static int smem_f[64], smem_v[64];
+  cudaError_t e = set_smem_limit_once((const void*)features_kernel<D_, M_, R_>, (int)F::kSmem, smem_f);
+  if (e != cudaSuccess) return e;
+  e = set_smem_limit_once((const void*)values_kernel<M_>, (int)V::kSmem, smem_v);
+  if (e != cudaSuccess) return e;
+  features_kernel<D_, M_, R_><<<a.B * a.H * nc, kThreads, F::kSmem, a.stream>>>(a.tm_w, a.tm_q,
+                                                                                 a.tm_k, fp);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  ValParams vp;
+  memset(&vp, 0, sizeof(vp));
+  vp.img = img;
+  vp.out = (__nv_bfloat16*)a.out;
+  vp.ob = a.os[0];
+  vp.oh = a.os[1];
+  vp.ol = a.os[2];
+  vp.B = a.B;
+  vp.H = a.H;
+  vp.L = a.L;
+  vp.nc = nc;
+  vp.nvb = D_ / 64;
+  vp.st_kv = a.st_kv;
+  vp.st_z = a.st_z;
+  vp.d = D_;
+  vp.dev_status = a.dev_status;
+  values_kernel<M_><<<a.B * a.H * (D_ / 64), kThreads, V::kSmem, a.stream>>>(a.tm_v, vp);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+bool tc_wide_supported(FwdArgs& a) {
+  if (a.dtype != DARK_BF16 || !(a.flags & DARK_CAUSAL) || (a.flags & DARK_STABILISE)) return false;
+  if (!shape_ok(a.d, a.m, a.r)) return false;
+  return make_wide_maps(a);
+}
+
+size_t tc_wide_workspace_bytes(int B, int H, int L, int m, int d, int r) {
+  if (!shape_ok(d, m, r)) return 0;
+  const size_t nc = (size_t)(L + kC - 1) / kC;
+  return align_up(kWsHeader + (size_t)B * H * nc * chunk_record_bytes(m), 256);
+}
+
+cudaError_t tc_wide_forward(const FwdArgs& a) {
+  if (!a.maps_ready) return cudaErrorInvalidValue;
+  if (a.d == 256 && a.m == 512 && a.r == 256) return launch<256, 512, 256>(a);
+  if (a.d == 128 && a.m == 256 && a.r == 128) return launch<128, 256, 128>(a);
+  if (a.d == 128 && a.m == 128 && a.r == 64) return launch<128, 128, 64>(a);
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace dark

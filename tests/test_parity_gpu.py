@@ -33,6 +33,12 @@ SMALL = {
     "c5-prefill": synth.WORKLOADS[5].with_sizes(B=3, H=2, L=333),
     "c2-noncausal": synth.WORKLOADS[2].with_sizes(H=2, L=260, lengths=(260, 131), causal=False),
     "c3-causal": synth.WORKLOADS[3].with_sizes(H=2, L=385, causal=True),
+    # wide heads (two-launch tensor-core path): key mask, ragged tails, other d/m/r
+    "c4-masked": synth.WORKLOADS[4].with_sizes(B=2, H=1, L=260, lengths=(260, 100)),
+    "wide-d128-m256": synth.WORKLOADS[4].with_sizes(B=2, H=2, L=270, d=128, r=128, m=256,
+                                                      lengths=(270, 150)),
+    "wide-d128-m128-shared": synth.WORKLOADS[4].with_sizes(B=1, H=3, L=140, d=128, r=64, m=128,
+                                                             per_head_geom=False),
 }
 
 
