@@ -406,22 +406,29 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // ================================================================ launch 2 ==
+// Every MMA of this launch uses the widest N its operands allow: an M=128,
+// K=16 MMA re-reads its 4 KB A slice from shared memory, so narrow N would be
+// limited by shared-memory bandwidth rather than by the tensor cores.
 template <int M_>
 struct ValCfg {
   static constexpr int NT = M_ / 128;        // feature tiles of the state
-  static constexpr int NITEM = 2 * NT;       // per chunk: Psi_f, Phi_f (32 KB each)
-  static constexpr int NSLOT = 3;
-  static constexpr uint32_t oA = 0;          // A_c image, 32 KB
-  static constexpr uint32_t oV = 32768;      // V_c slices, 2 x 16 KB
-  static constexpr uint32_t oR = 65536;      // ring, NSLOT x 32 KB
-  static constexpr uint32_t oS = oR + NSLOT * 32768;   // S hi | S lo | z hi | z lo
-  static constexpr uint32_t oOnes = oS + 40960;
-  static constexpr uint32_t oBar = oOnes + 2048;
+  static constexpr int NITEM = 1 + 2 * NT;   // ring items per chunk: Psi_0, A_c, Phi_0, (Psi_f, Phi_f)...
+  static constexpr int NSLOT = 4;            // ring slots of 32 KB
+  static constexpr uint32_t oV = 0;          // V_c slices, 2 x 16 KB (MN-major, 64 values)
+  static constexpr uint32_t oOnes = 32768;   // 128 x 64 block, 1.0 in column 0: [V | 1] operand
+  static constexpr uint32_t oR = 49152;      // ring
+  static constexpr uint32_t oS = oR + NSLOT * 32768;   // [S hi | S lo | (z hi, z lo)], 3 x 16 KB
+  static constexpr uint32_t oBar = oS + 49152;
   static constexpr uint32_t kSmem = oBar + 1024 + 1024;
-  // TMEM: state tile f at columns 80 f (64 values, then z in 16 columns); numerator after
+  // TMEM: state tile f at columns 80 f (64 values, z in column 64); numerator
+  // [num hi (64) | num lo (64) | den hi | den lo | 14 zero columns]
   static constexpr uint32_t tNum = 80 * NT;
-  static_assert(M_ % 128 == 0 && M_ <= 512 && tNum + 80 <= kTmemCols, "m");
+  static_assert(M_ % 128 == 0 && M_ <= 512 && tNum + 144 <= kTmemCols, "m");
+  static_assert(NT <= 4, "tiles");
 };
+// ring item index of Psi_f / Phi_f / A_c inside a chunk
+__device__ __forceinline__ int item_psi(int f) { return f == 0 ? 0 : 2 * f + 1; }
+__device__ __forceinline__ int item_phi(int f) { return 2 * f + 2; }
 
 struct ValParams {
   const uint8_t* img;
@@ -441,17 +448,17 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* sm = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   const uint32_t s0 = smem_u32(sm);
   uint64_t* bars = (uint64_t*)(sm + G::oBar);
-  uint64_t* bar_av = bars + 0;          // [2] A_c and V_c slice loaded
-  uint64_t* bar_aempty = bars + 2;      // MMA: intra GEMM (reads A_c) done
-  uint64_t* bar_vempty = bars + 3;      // [2] MMA: every GEMM of the chunk done (V slot free)
-  uint64_t* bar_simg = bars + 5;        // epilogue: S image of tile f written (8)
-  uint64_t* bar_sfree = bars + 6;       // MMA: inter GEMM of tile f done (S image free)
-  uint64_t* bar_nfull = bars + 7;       // MMA: numerator of the chunk complete
-  uint64_t* bar_nfree = bars + 8;       // epilogue: numerator read (8)
-  uint64_t* bar_full = bars + 9;        // [3] ring slot loaded
-  uint64_t* bar_empty = bars + 12;      // [3] ring slot read
-  uint32_t* tmem_slot = (uint32_t*)(bars + 16);
-  volatile int* abort_flag = (volatile int*)(bars + 17);
+  uint64_t* bar_v = bars + 0;           // [2] V_c slice loaded (slot c & 1)
+  uint64_t* bar_vempty = bars + 2;      // [2] MMA: every GEMM of the chunk done (V slot free)
+  uint64_t* bar_simg = bars + 4;        // epilogue: S image written (8 arrivals)
+  uint64_t* bar_sfree = bars + 5;       // MMA: inter GEMM reading the S image done
+  uint64_t* bar_nfull = bars + 6;       // MMA: numerator complete
+  uint64_t* bar_nfree = bars + 7;       // epilogue: numerator read (8)
+  uint64_t* bar_ds = bars + 8;          // [NT] MMA: state tile f updated by the chunk
+  uint64_t* bar_full = bars + 16;       // [NSLOT] ring slot loaded
+  uint64_t* bar_empty = bars + 20;      // [NSLOT] ring slot read
+  uint32_t* tmem_slot = (uint32_t*)(bars + 24);
+  volatile int* abort_flag = (volatile int*)(bars + 25);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int bh = blockIdx.x / p.nvb, vb = blockIdx.x % p.nvb;
@@ -460,15 +467,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint8_t* recs = p.img + (size_t)bh * p.nc * rec_bytes;
 
   if (tid == 0) {
-    mbar_init(bar_av + 0, 1);
-    mbar_init(bar_av + 1, 1);
-    mbar_init(bar_aempty, 1);
-    mbar_init(bar_vempty + 0, 1);
-    mbar_init(bar_vempty + 1, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bar_v + i, 1);
+      mbar_init(bar_vempty + i, 1);
+    }
     mbar_init(bar_simg, 8);
     mbar_init(bar_sfree, 1);
     mbar_init(bar_nfull, 1);
     mbar_init(bar_nfree, 8);
+    for (int f = 0; f < G::NT; ++f) mbar_init(bar_ds + f, 1);
     for (int i = 0; i < G::NSLOT; ++i) {
       mbar_init(bar_full + i, 1);
       mbar_init(bar_empty + i, 1);
@@ -476,8 +483,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     *abort_flag = 0;
     fence_mbar_init();
   }
-  // ones tile (bf16 1.0): 16 rows x 64, K-major, for the z / denominator columns
-  for (int i = tid; i < 2048 / 4; i += kThreads) ((uint32_t*)(sm + G::oOnes))[i] = 0x3F803F80u;
+  // zeroed S image and ones block: 1.0 (bf16) at column 0 of each of its 128
+  // 128-byte rows (128B swizzle puts it in 16-byte chunk row % 8)
+  for (int i = tid; i < (int)((16384 + 49152) / 16); i += kThreads) {
+    const uint32_t off = i < 1024 ? G::oOnes + i * 16 : G::oS + (i - 1024) * 16;
+    st_shared_v4(s0 + off, 0u, 0u, 0u, 0u);
+  }
+  __syncthreads();
+  if (tid < 128) st_shared_u16(s0 + G::oOnes + (tid / 8) * 1024 + (tid % 8) * 144, 0x3F80);
   fence_async_smem();
   if (warp == 0) tmem_alloc(tmem_slot, kTmemCols);
   tc_fence_before();
@@ -491,112 +504,119 @@ __global__ void __launch_bounds__(kThreads, 1)
       prefetch_tmap(&tm_v);
       const int total = p.nc * G::NITEM;
       int issued = 0, waited = 0;        // ring items loaded / waited for, in order
-      int av_issued = 0, av_waited = 0;  // chunks whose A_c, V_c were loaded / waited for
+      int v_issued = 0, v_waited = 0;    // V slices loaded / waited for
       auto load_item = [&](int g) {
-        const int c = g / G::NITEM, i = g % G::NITEM, f = i >> 1;
-        const uint8_t* src = recs + (size_t)c * rec_bytes + ((i & 1) ? 0 : (size_t)M_ * 256) +
-                             (size_t)f * 32768;
+        const int c = g / G::NITEM, i = g % G::NITEM;
+        const uint8_t* rc = recs + (size_t)c * rec_bytes;
+        const uint8_t* src;
+        if (i == 1) {
+          src = rc + (size_t)2 * M_ * 256;                         // A_c
+        } else if (i == 0 || (i & 1)) {
+          src = rc + (size_t)M_ * 256 + (size_t)(i == 0 ? 0 : (i - 1) / 2) * 32768;   // Psi_f
+        } else {
+          src = rc + (size_t)((i - 2) / 2) * 32768;                  // Phi_f
+        }
         const int slot = g % G::NSLOT;
         mbar_arrive_expect_tx(bar_full + slot, 32768);
         bulk_load(sm + G::oR + slot * 32768, src, 32768, bar_full + slot);
       };
-      auto load_av = [&](int c) -> bool {
-        if (c > 0 && !wait_one(bar_aempty, (c - 1) & 1, abort_flag, p.dev_status)) return false;
+      auto load_v = [&](int c) -> bool {
         if (c > 1 && !wait_one(bar_vempty + (c & 1), ((c - 2) >> 1) & 1, abort_flag, p.dev_status))
           return false;
-        mbar_arrive_expect_tx(bar_av + (c & 1), 32768 + 16384);
-        bulk_load(sm + G::oA, recs + (size_t)c * rec_bytes + (size_t)2 * M_ * 256, 32768,
-                  bar_av + (c & 1));
-        tma_load_4d(sm + G::oV + (c & 1) * 16384, &tm_v, 64 * vb, c * kC, h, b, bar_av + (c & 1));
-        av_issued = c + 1;
+        mbar_arrive_expect_tx(bar_v + (c & 1), 16384);
+        tma_load_4d(sm + G::oV + (c & 1) * 16384, &tm_v, 64 * vb, c * kC, h, b, bar_v + (c & 1));
+        v_issued = c + 1;
         return true;
       };
-      // after issuing the MMAs of item g: refill the slot item g-1 used
+      // after issuing the MMAs of item g: keep items up to g + NSLOT - 1 loaded;
+      // each load waits for the item that last used its slot (at most item g - 1)
       auto refill = [&](int g) -> bool {
-        if (g < 1 || issued >= total) return true;
-        const int j = g - 1;
-        if (!wait_one(bar_empty + j % G::NSLOT, (j / G::NSLOT) & 1, abort_flag, p.dev_status))
-          return false;
-        load_item(issued++);
+        while (issued <= g + G::NSLOT - 1 && issued < total) {
+          const int j = issued - G::NSLOT;
+          if (j >= 0 &&
+              !wait_one(bar_empty + j % G::NSLOT, (j / G::NSLOT) & 1, abort_flag, p.dev_status))
+            return false;
+          load_item(issued++);
+        }
         return true;
       };
-      bool ok = load_av(0);
+      auto wait_item = [&](int g) -> bool {
+        if (!wait_one(bar_full + g % G::NSLOT, (g / G::NSLOT) & 1, abort_flag, p.dev_status))
+          return false;
+        ++waited;
+        return true;
+      };
+      auto slot_addr = [&](int g) -> uint32_t { return s0 + G::oR + (g % G::NSLOT) * 32768; };
+      bool ok = load_v(0);
       for (; ok && issued < G::NSLOT && issued < total; ++issued) load_item(issued);
-      const uint32_t sA = s0 + G::oA, sSh = s0 + G::oS, sSl = sSh + 16384;
-      const uint32_t sZh = sSh + 32768, sZl = sZh + 4096, sOnes = s0 + G::oOnes;
       const uint32_t tnum = tmem + G::tNum;
+      const uint32_t sS = s0 + G::oS, sOnes = s0 + G::oOnes;
       for (int c = 0; ok && c < p.nc; ++c) {
-        if (!(ok = wait_one(bar_av + (c & 1), (c >> 1) & 1, abort_flag, p.dev_status))) break;
-        ++av_waited;
+        const int j = c & 1, g0 = c * G::NITEM;
+        const uint32_t sV = s0 + G::oV + j * 16384;
+        const uint32_t lbo_v1 = G::oOnes - (G::oV + j * 16384);   // [V | 1]: ones block after V
+        if (!(ok = wait_one(bar_v + j, (c >> 1) & 1, abort_flag, p.dev_status))) break;
+        ++v_waited;
         if (c > 0 && !(ok = wait_one(bar_nfree, (c - 1) & 1, abort_flag, p.dev_status))) break;
-        tc_fence_after();
-        const uint32_t sV = s0 + G::oV + (c & 1) * 16384;
-        // num = A_c [V_c | 1]
-        {
-          constexpr uint32_t idv = idesc(128, 64, false, true, false);
-          constexpr uint32_t id1 = idesc(128, 16, false, false, false);
-#pragma unroll
-          for (int s = 0; s < kC / 16; ++s) {
-            const uint64_t ad = sdesc(sA + (s / 4) * 16384 + (s % 4) * 32, 16, 1024);
-            mma(tnum, ad, sdesc(sV + s * 2048, 16384, 1024), idv, s > 0);
-            mma(tnum + 64, ad, sdesc(sOnes + (s % 4) * 32, 16, 1024), id1, s > 0);
-          }
-          mma_commit(bar_aempty);
-        }
         for (int f = 0; ok && f < G::NT; ++f) {
-          const int g = c * G::NITEM + 2 * f;
-          if (!(ok = wait_one(bar_simg, (c * G::NT + f) & 1, abort_flag, p.dev_status))) break;
-          if (!(ok = wait_one(bar_full + g % G::NSLOT, (g / G::NSLOT) & 1, abort_flag, p.dev_status)))
-            break;
-          ++waited;
+          const int k = c * G::NT + f;
+          const int gP = g0 + item_psi(f), gF = g0 + item_phi(f);
+          if (!(ok = wait_one(bar_simg, k & 1, abort_flag, p.dev_status))) break;
+          if (!(ok = wait_item(gP))) break;
           tc_fence_after();
-          // num += Psi_f [S_f | z_f], S and z as hi + lo bf16
+          // num[:, 0:144] (+)= Psi_f [S_hi | S_lo | (z_hi, z_lo)]; the first one of
+          // the chunk starts the numerator
           {
-            const uint32_t sPsi = s0 + G::oR + (g % G::NSLOT) * 32768;
-            constexpr uint32_t idv = idesc(128, 64, false, true, false);
-            constexpr uint32_t id1 = idesc(128, 16, false, false, false);
+            const uint32_t sPsi = slot_addr(gP);
+            constexpr uint32_t id = idesc(128, 144, false, true, false);
 #pragma unroll
-            for (int s = 0; s < 8; ++s) {
-              const uint64_t ad = sdesc(sPsi + (s / 4) * 16384 + (s % 4) * 32, 16, 1024);
-              mma(tnum, ad, sdesc(sSh + s * 2048, 16384, 1024), idv, 1);
-              mma(tnum, ad, sdesc(sSl + s * 2048, 16384, 1024), idv, 1);
-              mma(tnum + 64, ad, sdesc(sZh + (s / 4) * 2048 + (s % 4) * 32, 16, 1024), id1, 1);
-              mma(tnum + 64, ad, sdesc(sZl + (s / 4) * 2048 + (s % 4) * 32, 16, 1024), id1, 1);
-            }
+            for (int s = 0; s < 8; ++s)
+              mma(tnum, sdesc(sPsi + (s / 4) * 16384 + (s % 4) * 32, 16, 1024),
+                  sdesc(sS + s * 2048, 16384, 1024), id, (f > 0) || (s > 0));
             mma_commit(bar_sfree);
-            mma_commit(bar_empty + g % G::NSLOT);
           }
-          if (!(ok = refill(g))) break;
-          if (f == 0 && c + 1 < p.nc && !(ok = load_av(c + 1))) break;
-          if (!(ok = wait_one(bar_full + (g + 1) % G::NSLOT, ((g + 1) / G::NSLOT) & 1, abort_flag,
-                              p.dev_status)))
-            break;
-          ++waited;
+          if (f == 0) {
+            // num[:, 0:64] += A_c V_c ; den: num[:, 128] += A_c 1
+            if (!(ok = wait_item(g0 + 1))) break;
+            tc_fence_after();
+            const uint32_t sA = slot_addr(g0 + 1);
+            constexpr uint32_t idv = idesc(128, 64, false, true, false);
+            constexpr uint32_t id1 = idesc(128, 16, false, true, false);
+#pragma unroll
+            for (int s = 0; s < kC / 16; ++s) {
+              const uint64_t ad = sdesc(sA + (s / 4) * 16384 + (s % 4) * 32, 16, 1024);
+              mma(tnum, ad, sdesc(sV + s * 2048, 16384, 1024), idv, 1);
+              mma(tnum + 128, ad, sdesc(sOnes + s * 2048, 16384, 1024), id1, 1);
+            }
+          }
+          mma_commit(bar_empty + gP % G::NSLOT);
+          if (f == 0) mma_commit(bar_empty + (g0 + 1) % G::NSLOT);
+          if (!(ok = refill(gP))) break;
+          if (f == 0 && c + 1 < p.nc && !(ok = load_v(c + 1))) break;
+          if (!(ok = wait_item(gF))) break;
           tc_fence_after();
           // S_f += Phi_f^T [V_c | 1]
           {
-            const uint32_t sPhi = s0 + G::oR + ((g + 1) % G::NSLOT) * 32768;
+            const uint32_t sPhi = slot_addr(gF);
             const uint32_t ts = tmem + 80 * f;
-            constexpr uint32_t idv = idesc(128, 64, true, true, false);
-            constexpr uint32_t id1 = idesc(128, 16, true, false, false);
+            constexpr uint32_t id = idesc(128, 80, true, true, false);
 #pragma unroll
-            for (int s = 0; s < kC / 16; ++s) {
-              const uint64_t ad = sdesc(sPhi + s * 2048, 16384, 1024);
-              mma(ts, ad, sdesc(sV + s * 2048, 16384, 1024), idv, (c > 0) || (s > 0));
-              mma(ts + 64, ad, sdesc(sOnes + (s % 4) * 32, 16, 1024), id1, (c > 0) || (s > 0));
-            }
-            mma_commit(bar_empty + (g + 1) % G::NSLOT);
+            for (int s = 0; s < kC / 16; ++s)
+              mma(ts, sdesc(sPhi + s * 2048, 16384, 1024), sdesc(sV + s * 2048, lbo_v1, 1024), id,
+                  (c > 0) || (s > 0));
+            mma_commit(bar_ds + f);
+            mma_commit(bar_empty + gF % G::NSLOT);
           }
-          if (!(ok = refill(g + 1))) break;
+          if (!(ok = refill(gF))) break;
         }
         if (!ok) break;
         mma_commit(bar_nfull);
-        mma_commit(bar_vempty + (c & 1));
+        mma_commit(bar_vempty + j);
       }
       if (!ok) {
         // leave no copy in flight
         for (int g = waited; g < issued; ++g) mbar_wait(bar_full + g % G::NSLOT, (g / G::NSLOT) & 1);
-        for (int c = av_waited; c < av_issued; ++c) mbar_wait(bar_av + (c & 1), (c >> 1) & 1);
+        for (int c = v_waited; c < v_issued; ++c) mbar_wait(bar_v + (c & 1), (c >> 1) & 1);
       }
     }
     __syncwarp();
@@ -605,14 +625,51 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int quad = warp & 3, half = warp >> 2;
     const int row = quad * 32 + lane;               // TMEM lane: feature of a tile / query row
     const uint32_t lane_tm = tmem + ((uint32_t)(quad * 32) << 16);
-    const uint32_t sSh = s0 + G::oS, sSl = sSh + 16384, sZh = sSh + 32768, sZl = sZh + 4096;
+    const uint32_t sSh = s0 + G::oS, sSl = sSh + 16384, sZ = sSh + 32768;
     bool ok = true;
+    // out_c = (num hi + num lo) / (den hi + den lo)
+    auto output = [&](int c) -> bool {
+      if (!epi_wait(bar_nfull, c & 1, abort_flag, p.dev_status)) return false;
+      tc_fence_after();
+      const uint32_t tn = lane_tm + G::tNum;
+      uint32_t a[32], l[32];
+      tmem_ld32_async(tn + 32 * half, a);
+      tmem_ld32_async(tn + 64 + 32 * half, l);
+      tmem_wait_ld(a);
+      tmem_wait_ld(l);
+      const float den = tmem_ld1(tn + 128) + tmem_ld1(tn + 129);
+      const int tok = c * kC + row;
+      if (tok < p.L) {
+        const float inv = den > 0.f ? 1.f / den : 0.f;
+        uint32_t w[16];
+        bool bad = !isfinite(den);
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const float o0 = (__uint_as_float(a[2 * e]) + __uint_as_float(l[2 * e])) * inv;
+          const float o1 = (__uint_as_float(a[2 * e + 1]) + __uint_as_float(l[2 * e + 1])) * inv;
+          bad |= !isfinite(o0) || !isfinite(o1);
+          w[e] = pack_bf16(o0, o1);
+        }
+        if (bad) report(p.dev_status, DARK_ERR_NUMERIC);
+        uint4* dst = reinterpret_cast<uint4*>(p.out + (int64_t)b * p.ob + (int64_t)h * p.oh +
+                                              (int64_t)tok * p.ol + 64 * vb + 32 * half);
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4)
+          dst[q4] = make_uint4(w[4 * q4], w[4 * q4 + 1], w[4 * q4 + 2], w[4 * q4 + 3]);
+      }
+      tc_fence_before();
+      warp_arrive(bar_nfree);
+      return true;
+    };
     for (int c = 0; ok && c < p.nc; ++c) {
       for (int f = 0; f < G::NT; ++f) {
         const int k = c * G::NT + f;
+        // the S image is free once the previous tile's inter GEMM read it;
+        // tile f holds S_<c once the previous chunk's update of it is done
         if (k > 0 && !(ok = epi_wait(bar_sfree, (k - 1) & 1, abort_flag, p.dev_status))) break;
+        if (c > 0 && !(ok = epi_wait(bar_ds + f, (c - 1) & 1, abort_flag, p.dev_status))) break;
         tc_fence_after();
-        // S_f (row `row` of the tile) as hi + lo bf16: MN-major values, K-major z
+        // row `row` of S_f as hi + lo bf16 (MN-major: the feature is the K row)
         float x[33];
         if (c == 0) {
 #pragma unroll
@@ -642,53 +699,21 @@ __global__ void __launch_bounds__(kThreads, 1)
           st_shared_v4(sSl + off, lo4[0], lo4[1], lo4[2], lo4[3]);
         }
         if (half == 0) {
-          const __nv_bfloat16 zh = __float2bfloat16_rn(x[32]);
-          const __nv_bfloat16 zl = __float2bfloat16_rn(x[32] - __bfloat162float(zh));
-          const uint16_t zhb = *reinterpret_cast<const uint16_t*>(&zh);
-          const uint16_t zlb = *reinterpret_cast<const uint16_t*>(&zl);
-#pragma unroll
-          for (int n = 0; n < 16; ++n) {
-            const uint32_t off = (uint32_t)(row / 64) * 2048 + kmajor_off(n, row % 64, 0);
-            st_shared_u16(sZh + off, zhb);
-            st_shared_u16(sZl + off, zlb);
-          }
+          // (z hi, z lo) in columns 0, 1 of the third block (16-byte chunk row % 8)
+          const float zh = __bfloat162float(__float2bfloat16_rn(x[32]));
+          asm volatile("st.shared.b32 [%0], %1;" ::"r"(sZ + rowoff + (uint32_t)(row % 8) * 16),
+                       "r"(pack_bf16(zh, x[32] - zh))
+                       : "memory");
         }
         tc_fence_before();
         fence_async_smem();
         warp_arrive(bar_simg);
+        // the previous chunk's output, while the tensor cores start on this one
+        if (f == 0 && c > 0 && !(ok = output(c - 1))) break;
       }
-      if (!ok) break;
-      // ---------------------------------------------- out_c = num / den
-      if (!(ok = epi_wait(bar_nfull, c & 1, abort_flag, p.dev_status))) break;
-      tc_fence_after();
-      {
-        uint32_t a[32];
-        tmem_ld32_async(lane_tm + G::tNum + 32 * half, a);
-        tmem_wait_ld(a);
-        const float den = tmem_ld1(lane_tm + G::tNum + 64);
-        const int tok = c * kC + row;
-        if (tok < p.L) {
-          const float inv = den > 0.f ? 1.f / den : 0.f;
-          uint32_t w[16];
-          bool bad = !isfinite(den);
-#pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const float o0 = __uint_as_float(a[2 * e]) * inv, o1 = __uint_as_float(a[2 * e + 1]) * inv;
-            bad |= !isfinite(o0) || !isfinite(o1);
-            w[e] = pack_bf16(o0, o1);
-          }
-          if (bad) report(p.dev_status, DARK_ERR_NUMERIC);
-          uint4* dst = reinterpret_cast<uint4*>(p.out + (int64_t)b * p.ob + (int64_t)h * p.oh +
-                                                (int64_t)tok * p.ol + 64 * vb + 32 * half);
-#pragma unroll
-          for (int q4 = 0; q4 < 4; ++q4)
-            dst[q4] = make_uint4(w[4 * q4], w[4 * q4 + 1], w[4 * q4 + 2], w[4 * q4 + 3]);
-        }
-      }
-      tc_fence_before();
-      warp_arrive(bar_nfree);
     }
-    // final state [S | z] (every GEMM of the last chunk is complete)
+    if (ok) ok = output(p.nc - 1);
+    // final state [S | z]: every GEMM of the last chunk is complete
     if (ok && p.st_kv != nullptr) {
       tc_fence_after();
       for (int f = 0; f < G::NT; ++f) {
