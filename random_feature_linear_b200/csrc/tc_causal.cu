@@ -49,8 +49,8 @@ struct Cfg {
   static constexpr int MB = M_ / 128;
   static constexpr int NW = M_ + R_;                      // W' rows
   static constexpr uint32_t kW = NW * 128;                // W' bytes (fp16, 128 B rows)
-  static constexpr uint32_t kZ = (M_ / 64) * 2048;        // one z16 operand (hi or lo)
-  static constexpr uint32_t kWReg = (kW > 2 * kZ ? kW : 2 * kZ);
+  static constexpr uint32_t kZ = (M_ / 64) * 2048;        // the 16-row z operand
+  static constexpr uint32_t kWReg = (kW > kZ ? kW : kZ);
   static constexpr uint32_t kPhi = (M_ / 64) * 16384;     // 128 tokens x M_ features, bf16
   // shared memory offsets (all 1024-byte aligned)
   static constexpr uint32_t oW = 0;
@@ -64,9 +64,10 @@ struct Cfg {
   static constexpr uint32_t kSmem = oBar + 64 + 1024;     // + alignment slack
   // TMEM columns
   // key features [0, M_) and norms [M_, M_ + R_); query features [256, 256 + M_)
-  // (issued once the norms are read); scores [0, 128), numerator [128, 208) and
-  // chunk state [320, 480) once both feature blocks are consumed
-  static constexpr uint32_t tP = 0, tQ = 256, tA = 0, tNum = 128, tD = 320;
+  // (issued once the norms are read); once both feature blocks are consumed:
+  // scores [0, 128), numerator hi | lo [128, 256), denominator hi, lo at 256,
+  // 257 (16 columns) and chunk state [320, 480)
+  static constexpr uint32_t tP = 0, tQ = 256, tA = 0, tNum = 128, tDen = 256, tD = 320;
   static_assert(NW <= 320 && M_ % 128 == 0 && R_ % 16 == 0, "shape");
   static_assert(tD + 80 * MB <= kTmemCols, "tmem");
 };
@@ -113,8 +114,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   __syncwarp();
   if (warp == 0) tmem_alloc(tmem_slot, kTmemCols);
-  // ones tile (bf16 1.0) for the z columns: 16 rows x 64 keys, K-major
-  for (int i = tid; i < 2048 / 4; i += kThreads) ((uint32_t*)(sm + G::oOnes))[i] = 0x3F803F80u;
+  // ones operand for the z / denominator columns: 16 rows x 64 keys, K-major,
+  // 1.0 in row 0 (its first 128 bytes) and zeros in rows 1-15, so that each
+  // sum lands in a single column
+  for (int i = tid; i < 2048 / 4; i += kThreads)
+    ((uint32_t*)(sm + G::oOnes))[i] = i < 32 ? 0x3F803F80u : 0u;
   fence_async_smem();
   tc_fence_before();
   __syncthreads();
@@ -244,7 +248,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (!wait_all(bar_mma, ph_mma, p.dev_status)) { abort = true; break; }
     ph_mma ^= 1;
     tc_fence_after();
-    // ----------------------- causal mask of the scores -> bf16 A operand (Q/K tiles)
+    // ---- causal mask of the scores -> bf16 A operand (Q tile region); the
+    // prefix [S_<c | z_<c] as operands; this chunk's state added to the prefix
     {
       float v[32];
 #pragma unroll
@@ -262,24 +267,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     }
-    fence_async_smem();
-    tc_fence_before();
-    __syncthreads();
-    // -------------------------------------------- intra-chunk GEMM tril(A) [V|1]
-    if (tid == 0) {
-      tc_fence_after();
-      constexpr uint32_t idv = idesc(128, 64, false, true, false);
-      constexpr uint32_t id1 = idesc(128, 16, false, false, false);
-#pragma unroll
-      for (int s = 0; s < kC / 16; ++s) {
-        const uint64_t ad = sdesc(s0 + G::oQ + (s / 4) * 16384 + (s % 4) * 32, 16, 1024);
-        mma(tmem + G::tNum, ad, sdesc(s0 + G::oV + s * 2048, 16384, 1024), idv, s > 0);
-        mma(tmem + G::tNum + 64, ad, sdesc(s0 + G::oOnes + (s % 4) * 32, 16, 1024), id1, s > 0);
-      }
-    }
     const bool have_prefix = c > 0;
-    // prefix [S | z] as hi + lo bf16 operands: S (MN-major) in the Phi region,
-    // z (16 identical K-major rows) in the W' region
+    // S hi, S lo: MN-major blocks of M_ feature rows in the Phi region (M_ * 128
+    // bytes apart); z hi, z lo: rows 0 and 1 of a 16-row K-major operand in the
+    // W' region (rows 2-15 zero)
     if (have_prefix && has_feat) {
       const uint32_t sh = s0 + G::oPhi, sl = sh + M_ * 128;
       const uint32_t rowoff = (uint32_t)(feat / 8) * 1024 + (uint32_t)(feat % 8) * 128;
@@ -300,14 +291,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       const __nv_bfloat16 zh = __float2bfloat16_rn(run[64]);
       const __nv_bfloat16 zl = __float2bfloat16_rn(run[64] - __bfloat162float(zh));
-      const uint16_t zhb = *reinterpret_cast<const uint16_t*>(&zh);
-      const uint16_t zlb = *reinterpret_cast<const uint16_t*>(&zl);
-      const uint32_t zh_base = s0 + G::oW, zl_base = zh_base + G::kZ;
-#pragma unroll
-      for (int n = 0; n < 16; ++n) {
-        const uint32_t off = (uint32_t)(feat / 64) * 2048 + kmajor_off(n, feat % 64, 0);
-        st_shared_u16(zh_base + off, zhb);
-        st_shared_u16(zl_base + off, zlb);
+      const uint32_t zb = s0 + G::oW + (uint32_t)(feat / 64) * 2048;
+      st_shared_u16(zb + kmajor_off(0, feat % 64, 0), *reinterpret_cast<const uint16_t*>(&zh));
+      st_shared_u16(zb + kmajor_off(1, feat % 64, 0), *reinterpret_cast<const uint16_t*>(&zl));
+    }
+    if (have_prefix) {
+      for (int i = tid; i < (M_ / 64) * 14 * 8; i += kThreads) {
+        const int blk = i / 112, n = 2 + (i % 112) / 8, ch = i % 8;
+        st_shared_v4(s0 + G::oW + blk * 2048 + (n / 8) * 1024 + (n % 8) * 128 + ch * 16, 0u, 0u, 0u, 0u);
       }
     }
     // add this chunk's state row `feat` (Phi(K_c)^T [V_c | 1], in TMEM) to the prefix
@@ -325,24 +316,32 @@ __global__ void __launch_bounds__(kThreads, 1)
       run[64] += tmem_ld1(base + 64);
     }
     fence_async_smem();
+    tc_fence_before();
     __syncthreads();
-    // -------------------------------------------------- inter-chunk GEMM Psi [S|z]
+    // ---- [num hi | num lo] = Psi [S hi | S lo], [den hi, den lo] = Psi [z hi; z lo]
+    // (one N = 128 and one N = 16 MMA per K-step), then num hi += tril(A) V and
+    // den hi += tril(A) 1, all in one commit group
     if (tid == 0) {
       tc_fence_after();
       if (have_prefix) {
-        constexpr uint32_t idv = idesc(128, 64, false, true, false);
-        constexpr uint32_t id1 = idesc(128, 16, false, false, false);
+        constexpr uint32_t ids = idesc(128, 128, false, true, false);
+        constexpr uint32_t idz = idesc(128, 16, false, false, false);
 #pragma unroll
-        for (int part = 0; part < 2; ++part) {
-          const uint32_t sb = s0 + G::oPhi + part * M_ * 128;
-          const uint32_t zb = s0 + G::oW + part * G::kZ;
-#pragma unroll
-          for (int s = 0; s < M_ / 16; ++s) {
-            const uint64_t ad = sdesc(s0 + G::oPsi + (s / 4) * 16384 + (s % 4) * 32, 16, 1024);
-            mma(tmem + G::tNum, ad, sdesc(sb + s * 2048, 16384, 1024), idv, 1);
-            mma(tmem + G::tNum + 64, ad, sdesc(zb + (s / 4) * 2048 + (s % 4) * 32, 16, 1024), id1, 1);
-          }
+        for (int s = 0; s < M_ / 16; ++s) {
+          const uint64_t ad = sdesc(s0 + G::oPsi + (s / 4) * 16384 + (s % 4) * 32, 16, 1024);
+          mma(tmem + G::tNum, ad, sdesc(s0 + G::oPhi + s * 2048, M_ * 128, 1024), ids, s > 0);
+          mma(tmem + G::tDen, ad, sdesc(s0 + G::oW + (s / 4) * 2048 + (s % 4) * 32, 16, 1024), idz,
+              s > 0);
         }
+      }
+      constexpr uint32_t idv = idesc(128, 64, false, true, false);
+      constexpr uint32_t id1 = idesc(128, 16, false, false, false);
+#pragma unroll
+      for (int s = 0; s < kC / 16; ++s) {
+        const uint64_t ad = sdesc(s0 + G::oQ + (s / 4) * 16384 + (s % 4) * 32, 16, 1024);
+        const uint32_t acc = (have_prefix || s > 0) ? 1u : 0u;
+        mma(tmem + G::tNum, ad, sdesc(s0 + G::oV + s * 2048, 16384, 1024), idv, acc);
+        mma(tmem + G::tDen, ad, sdesc(s0 + G::oOnes + (s % 4) * 32, 16, 1024), id1, acc);
       }
       mma_commit(bar_mma);
     }
@@ -351,9 +350,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     // ------------------------------------------------------------- output
     {
-      const float den = tmem_ld1(lane_tm + G::tNum + 64);
+      float den = tmem_ld1(lane_tm + G::tDen);
       float v[32];
       tmem_ld32(lane_tm + G::tNum + half * 32, v);
+      if (have_prefix) {
+        float vl[32];
+        tmem_ld32(lane_tm + G::tNum + 64 + half * 32, vl);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) v[i] += vl[i];
+        den += tmem_ld1(lane_tm + G::tDen + 1);
+      }
       const int tok = t0 + row;
       if (tok < p.L) {
         const float inv = den > 0.f ? 1.f / den : 0.f;

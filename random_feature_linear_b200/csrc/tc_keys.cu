@@ -38,10 +38,13 @@ struct KeyCfg {
   static constexpr uint32_t oW = 0;
   static constexpr uint32_t oK = (kW + 1023) / 1024 * 1024;   // 2 buffers
   static constexpr uint32_t oV = oK + 2 * kTileBytes;         // 2 buffers
-  static constexpr uint32_t oPhi = oV + 2 * kTileBytes;
-  static constexpr uint32_t oOnes = oPhi + kPhi;
-  static constexpr uint32_t oBar = oOnes + 2048;
+  // 128 x 64 block of bf16 ones after the V buffers: [V | 1] is one MN-major
+  // operand of N = 80 (64-wide blocks LBO apart), one MMA per K-step
+  static constexpr uint32_t oOnes = oV + 2 * kTileBytes;
+  static constexpr uint32_t oPhi = oOnes + kTileBytes;
+  static constexpr uint32_t oBar = oPhi + kPhi;
   static constexpr uint32_t kSmem = oBar + 64 + 1024;
+  static_assert(kSmem <= 232448, "shared memory");
   static constexpr uint32_t tP = 0, tD = 320;
 };
 
@@ -80,7 +83,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   __syncwarp();
   if (warp == 0) tmem_alloc(tmem_slot, kTmemCols);
-  for (int i = tid; i < 2048 / 4; i += kThreads) ((uint32_t*)(sm + G::oOnes))[i] = 0x3F803F80u;
+  for (int i = tid; i < kTileBytes / 4; i += kThreads) ((uint32_t*)(sm + G::oOnes))[i] = 0x3F803F80u;
   fence_async_smem();
   tc_fence_before();
   __syncthreads();
@@ -142,17 +145,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     if (tid == 0) {
       tc_fence_after();
-      constexpr uint32_t idv = idesc(128, 64, true, true, false);
-      constexpr uint32_t id1 = idesc(128, 16, true, false, false);
+      // chunk state [S | z] += Phi^T [V | 1] (z in column 64 and its copies)
+      constexpr uint32_t id = idesc(128, 80, true, true, false);
+      const uint32_t sv = s0 + G::oV + buf * kTileBytes;
+      const uint32_t lbo = G::oOnes - (G::oV + buf * kTileBytes);
 #pragma unroll
       for (int mb = 0; mb < G::MB; ++mb) {
 #pragma unroll
         for (int s = 0; s < kT / 16; ++s) {
           const uint32_t acc = (t > tb || s > 0) ? 1u : 0u;
-          const uint64_t ad = sdesc(s0 + G::oPhi + mb * 32768 + s * 2048, 16384, 1024);
-          mma(tmem + G::tD + 80 * mb, ad, sdesc(s0 + G::oV + buf * kTileBytes + s * 2048, 16384, 1024),
-              idv, acc);
-          mma(tmem + G::tD + 80 * mb + 64, ad, sdesc(s0 + G::oOnes + (s % 4) * 32, 16, 1024), id1, acc);
+          mma(tmem + G::tD + 80 * mb, sdesc(s0 + G::oPhi + mb * 32768 + s * 2048, 16384, 1024),
+              sdesc(sv + s * 2048, lbo, 1024), id, acc);
         }
       }
     }

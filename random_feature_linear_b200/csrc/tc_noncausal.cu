@@ -33,11 +33,13 @@ constexpr int kSms = 148;
 constexpr int kTileBytes = kT * kD * 2;
 constexpr uint32_t kTmemCols = 512;
 
-// Byte sizes of the query kernel's B-operand image of [S | z] (per head):
-// S hi, S lo (MN-major, 128 B per feature), z hi, z lo (16 identical K-major rows).
+// The query kernel's B operand [S hi | S lo | (z hi, z lo)] per head: three
+// MN-major blocks of m feature rows x 128 B, so that one MMA per K-step (N =
+// 64 + 64 + 16) yields both halves of the numerator and of the denominator
+// (every MMA with N <= 144 costs about the same, so fewer and wider is faster).
+// The third block holds z hi, z lo in columns 0, 1 and zeros up to column 15.
 __host__ __device__ constexpr uint32_t img_s_bytes(int m) { return (uint32_t)m * 128; }
-__host__ __device__ constexpr uint32_t img_z_bytes(int m) { return (uint32_t)(m / 64) * 2048; }
-__host__ __device__ constexpr uint32_t img_bytes(int m) { return 2 * img_s_bytes(m) + 2 * img_z_bytes(m); }
+__host__ __device__ constexpr uint32_t img_bytes(int m) { return 3 * img_s_bytes(m); }
 
 // Sums the split partials of each head in split order and writes the query
 // kernel's operand image (hi + lo bf16) and, if requested, the fp32 state.
@@ -54,20 +56,18 @@ __global__ void reduce_kernel(const float* __restrict__ partials, int nsplit, in
   const __nv_bfloat16 hi = __float2bfloat16_rn(acc);
   const __nv_bfloat16 lo = __float2bfloat16_rn(acc - __bfloat162float(hi));
   uint8_t* img = images + (size_t)bh * img_bytes(m);
+  const uint32_t row = (uint32_t)(f / 8) * 1024 + (uint32_t)(f % 8) * 128;
   if (col < 64) {
-    const uint32_t off = (uint32_t)(f / 8) * 1024 + (uint32_t)(f % 8) * 128 +
-                         (uint32_t)((((col / 8) ^ (f % 8)) * 16)) + (uint32_t)(col % 8) * 2;
+    const uint32_t off = row + (uint32_t)((((col / 8) ^ (f % 8)) * 16)) + (uint32_t)(col % 8) * 2;
     *reinterpret_cast<__nv_bfloat16*>(img + off) = hi;
     *reinterpret_cast<__nv_bfloat16*>(img + img_s_bytes(m) + off) = lo;
     if (st_kv != nullptr) st_kv[((size_t)bh * m + f) * 64 + col] = acc;
   } else {
-    uint8_t* zh = img + 2 * img_s_bytes(m);
-    uint8_t* zl = zh + img_z_bytes(m);
-    for (int n = 0; n < 16; ++n) {
-      const uint32_t off = (uint32_t)(f / 64) * 2048 + kmajor_off(n, f % 64, 0);
-      *reinterpret_cast<__nv_bfloat16*>(zh + off) = hi;
-      *reinterpret_cast<__nv_bfloat16*>(zl + off) = lo;
-    }
+    // columns 0-7 and 8-15 of the third block: (z hi, z lo, 0, ...), zeros
+    uint8_t* zz = img + 2 * img_s_bytes(m) + row;
+    const uint32_t w0 = (uint32_t)__bfloat16_as_ushort(hi) | ((uint32_t)__bfloat16_as_ushort(lo) << 16);
+    *reinterpret_cast<uint4*>(zz + (uint32_t)((0 ^ (f % 8)) * 16)) = make_uint4(w0, 0u, 0u, 0u);
+    *reinterpret_cast<uint4*>(zz + (uint32_t)((1 ^ (f % 8)) * 16)) = make_uint4(0u, 0u, 0u, 0u);
     if (st_z != nullptr) st_z[(size_t)bh * m + f] = acc;
   }
 }
@@ -92,6 +92,7 @@ struct QueryCfg {
   static constexpr uint32_t oBar = oPsi + kPsi;
   static constexpr uint32_t kSmem = oBar + 64 + 1024;
   static constexpr uint32_t tP = 0, tO = 256;
+  static_assert(kSmem <= 232448, "shared memory");
 };
 
 template <int M_, int R_>
@@ -186,29 +187,24 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     if (tid == 0) {
       tc_fence_after();
-      constexpr uint32_t idv = idesc(128, 64, false, true, false);
-      constexpr uint32_t id1 = idesc(128, 16, false, false, false);
+      // [num hi | num lo | den hi, den lo] = Psi [S hi | S lo | (z hi, z lo)]
+      constexpr uint32_t id = idesc(128, 144, false, true, false);
 #pragma unroll
-      for (int part = 0; part < 2; ++part) {
-        const uint32_t sb = s0 + G::oImg + part * img_s_bytes(M_);
-        const uint32_t zb = s0 + G::oImg + 2 * img_s_bytes(M_) + part * img_z_bytes(M_);
-#pragma unroll
-        for (int s = 0; s < M_ / 16; ++s) {
-          const uint64_t ad = sdesc(s0 + G::oPsi + (s / 4) * 16384 + (s % 4) * 32, 16, 1024);
-          const uint32_t acc = (part > 0 || s > 0) ? 1u : 0u;
-          mma(tmem + G::tO, ad, sdesc(sb + s * 2048, 16384, 1024), idv, acc);
-          mma(tmem + G::tO + 64, ad, sdesc(zb + (s / 4) * 2048 + (s % 4) * 32, 16, 1024), id1, acc);
-        }
-      }
+      for (int s = 0; s < M_ / 16; ++s)
+        mma(tmem + G::tO, sdesc(s0 + G::oPsi + (s / 4) * 16384 + (s % 4) * 32, 16, 1024),
+            sdesc(s0 + G::oImg + s * 2048, img_s_bytes(M_), 1024), id, s > 0);
       mma_commit(bar_mma);
     }
     if (!wait_all(bar_mma, ph_mma, p.dev_status)) { abort = true; break; }
     ph_mma ^= 1;
     tc_fence_after();
     {
-      const float den = tmem_ld1(lane_tm + G::tO + 64);
-      float v[32];
+      const float den = tmem_ld1(lane_tm + G::tO + 128) + tmem_ld1(lane_tm + G::tO + 129);
+      float v[32], vl[32];
       tmem_ld32(lane_tm + G::tO + half * 32, v);
+      tmem_ld32(lane_tm + G::tO + 64 + half * 32, vl);
+#pragma unroll
+      for (int i = 0; i < 32; ++i) v[i] += vl[i];
       const int tok = t * kT + row;
       if (tok < p.L) {
         const float inv = den > 0.f ? 1.f / den : 0.f;
