@@ -50,14 +50,19 @@ struct Cfg {
   static constexpr int NW = M_ + R_;                      // W' rows
   static constexpr uint32_t kW = NW * 128;                // W' bytes (fp16, 128 B rows)
   static constexpr uint32_t kZ = (M_ / 64) * 2048;        // the 16-row z operand
-  static constexpr uint32_t kWReg = (kW > kZ ? kW : kZ);
+  // after the feature GEMMs the W' region holds the z operand and keys 64-127
+  // of the masked-score operand (keys 0-63 sit in the Q tile)
+  static constexpr uint32_t oA1 = kZ;
+  static constexpr uint32_t kWReg = (kW > kZ + 16384 ? kW : kZ + 16384);
   static constexpr uint32_t kPhi = (M_ / 64) * 16384;     // 128 tokens x M_ features, bf16
   // shared memory offsets (all 1024-byte aligned)
   static constexpr uint32_t oW = 0;
   static constexpr uint32_t oQ = (oW + kWReg + 1023) / 1024 * 1024;
-  static constexpr uint32_t oK = oQ + kTileBytes;
-  static constexpr uint32_t oV = oK + kTileBytes;
-  static constexpr uint32_t oPhi = oV + kTileBytes;
+  // V, then K: once the key GEMM is done the K tile is refilled with bf16 ones,
+  // so that [V | 1] is one MN-major operand of N = 80 (blocks 16 KB apart)
+  static constexpr uint32_t oV = oQ + kTileBytes;
+  static constexpr uint32_t oK = oV + kTileBytes;
+  static constexpr uint32_t oPhi = oK + kTileBytes;
   static constexpr uint32_t oPsi = oPhi + kPhi;
   static constexpr uint32_t oOnes = oPsi + kPhi;
   static constexpr uint32_t oBar = oOnes + 2048;
@@ -218,10 +223,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------- epilogue: Psi(Q_c)
     exp2_rows_to_smem(lane_tm + G::tQ, half * (M_ / 2), (half + 1) * (M_ / 2), 0.f, false,
                       s0 + G::oPsi, row);
+    for (int i = tid; i < kTileBytes / 16; i += kThreads)   // the key tile is consumed
+      st_shared_v4(s0 + G::oK + i * 16, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u);
     fence_async_smem();
     tc_fence_before();
     __syncthreads();
-    // -------------------------------- scores Psi Phi^T and chunk state Phi^T [V|1]
+    // ------------------ scores Psi Phi^T and chunk state Phi^T [V | 1] (N = 80)
     if (tid == 0) {
       tc_fence_after();
       constexpr uint32_t ids = idesc(128, 128, false, false, false);
@@ -231,24 +238,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         mma(tmem + G::tA, sdesc(s0 + G::oPsi + off, 16, 1024), sdesc(s0 + G::oPhi + off, 16, 1024),
             ids, s > 0);
       }
-      constexpr uint32_t idv = idesc(128, 64, true, true, false);
-      constexpr uint32_t id1 = idesc(128, 16, true, false, false);
+      constexpr uint32_t idv = idesc(128, 80, true, true, false);
 #pragma unroll
       for (int mb = 0; mb < G::MB; ++mb) {
 #pragma unroll
-        for (int s = 0; s < kC / 16; ++s) {
-          const uint64_t ad = sdesc(s0 + G::oPhi + mb * 32768 + s * 2048, 16384, 1024);
-          mma(tmem + G::tD + 80 * mb, ad, sdesc(s0 + G::oV + s * 2048, 16384, 1024), idv, s > 0);
-          mma(tmem + G::tD + 80 * mb + 64, ad, sdesc(s0 + G::oOnes + (s % 4) * 32, 16, 1024), id1,
-              s > 0);
-        }
+        for (int s = 0; s < kC / 16; ++s)
+          mma(tmem + G::tD + 80 * mb, sdesc(s0 + G::oPhi + mb * 32768 + s * 2048, 16384, 1024),
+              sdesc(s0 + G::oV + s * 2048, G::oK - G::oV, 1024), idv, s > 0);
       }
       mma_commit(bar_mma);
     }
     if (!wait_all(bar_mma, ph_mma, p.dev_status)) { abort = true; break; }
     ph_mma ^= 1;
     tc_fence_after();
-    // ---- causal mask of the scores -> bf16 A operand (Q tile region); the
+    // ---- causal mask of the scores -> bf16 A operand (Q tile, W' region); the
     // prefix [S_<c | z_<c] as operands; this chunk's state added to the prefix
     {
       float v[32];
@@ -263,7 +266,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int j = j0 + 8 * g + 2 * e;
             w4[e] = pack_bf16(j <= row ? v[8 * g + 2 * e] : 0.f, j + 1 <= row ? v[8 * g + 2 * e + 1] : 0.f);
           }
-          st_shared_v4(s0 + G::oQ + kmajor_off(row, j0 + 8 * g, 16384), w4[0], w4[1], w4[2], w4[3]);
+          const uint32_t blk = j0 < 64 ? s0 + G::oQ : s0 + G::oW + G::oA1;
+          st_shared_v4(blk + kmajor_off(row, (j0 % 64) + 8 * g, 0), w4[0], w4[1], w4[2], w4[3]);
         }
       }
     }
@@ -338,7 +342,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       constexpr uint32_t id1 = idesc(128, 16, false, false, false);
 #pragma unroll
       for (int s = 0; s < kC / 16; ++s) {
-        const uint64_t ad = sdesc(s0 + G::oQ + (s / 4) * 16384 + (s % 4) * 32, 16, 1024);
+        const uint32_t ablk = s < 4 ? s0 + G::oQ : s0 + G::oW + G::oA1;
+        const uint64_t ad = sdesc(ablk + (s % 4) * 32, 16, 1024);
         const uint32_t acc = (have_prefix || s > 0) ? 1u : 0u;
         mma(tmem + G::tNum, ad, sdesc(s0 + G::oV + s * 2048, 16384, 1024), idv, acc);
         mma(tmem + G::tDen, ad, sdesc(s0 + G::oOnes + (s % 4) * 32, 16, 1024), id1, acc);
