@@ -29,8 +29,8 @@
 //       num += Psi_f [S_f | z_f]  (hi and lo)   and   S_f += Phi_f^T [V_c | 1]
 //     after num = A_c [V_c | 1]; the epilogue divides and stores out_c.
 //
-// In both kernels warp 8 is the producer (TMA / bulk copies) and the MMA
-// issuer; warps 0-7 are the epilogue (TMEM lane quadrant = warp % 4). Every
+// In both kernels warp 9 is the producer (TMA / bulk copies), warp 8 issues
+// the MMAs and warps 0-7 are the epilogue (TMEM lane quadrant = warp % 4). Every
 // wait is bounded: a wait that runs out records DARK_ERR_TIMEOUT and raises the
 // CTA's abort flag, every role leaves its loop, in-flight copies are waited for
 // (bounded), and TMEM is freed.
@@ -47,7 +47,7 @@ using namespace tc;
 
 constexpr int kC = 128;              // tokens per chunk (UMMA M)
 constexpr int kEpiThreads = 256;     // warps 0-7
-constexpr int kThreads = kEpiThreads + 32;
+constexpr int kThreadsF = kEpiThreads + 64;   // + MMA warp 8 + producer warp 9
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kSmemBudget = 229376;   // 224 KB of operands + barriers + alignment slack
 
@@ -117,7 +117,9 @@ __device__ __forceinline__ void warp_arrive(uint64_t* bar) {
 template <int D_, int M_, int R_>
 struct FeatCfg {
   static constexpr int DS = D_ / 64;                       // 64-column slabs of d
-  static constexpr int NNORM = R_ / 64, NFEAT = M_ / 64;   // W' items of 64 rows
+  // W' items: first one per d slab with all R_ norm rows (one N = R_ MMA per
+  // K-step), then 64 feature rows over all of d
+  static constexpr int NNORM = DS, NFEAT = M_ / 64;
   static constexpr int NITEMS = NNORM + NFEAT;
   static constexpr uint32_t kX = DS * 16384;               // one 128-token tile, fp16
   static constexpr uint32_t kSlot = DS * 8192;             // 64 W' rows x d, fp16
@@ -133,6 +135,7 @@ struct FeatCfg {
   static_assert(D_ % 64 == 0 && D_ >= 128 && D_ <= 256, "d");
   static_assert(M_ % 128 == 0 && M_ <= 512 && R_ % 64 == 0 && R_ >= 64 && R_ <= 256, "m, r");
   static_assert(NSLOT >= 2, "shared memory");
+  static_assert(R_ * 128 <= kSlot, "norm item");
 };
 
 // Bytes of one chunk's record in the workspace: Phi image, Psi image, A image.
@@ -148,7 +151,7 @@ struct FeatParams {
 };
 
 template <int D_, int M_, int R_>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreadsF, 1)
     features_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_q,
                     const __grid_constant__ CUtensorMap tm_k, const FeatParams p) {
   using G = FeatCfg<D_, M_, R_>;
@@ -165,8 +168,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* bar_sfree = bars + 7;       // MMA: scores GEMM of the staged block done
   uint64_t* bar_full = bars + 8;        // [NSLOT] W' slot loaded
   uint64_t* bar_empty = bars + 16;      // [NSLOT] W' slot read by the MMAs
-  uint32_t* tmem_slot = (uint32_t*)(bars + 24);
-  volatile int* abort_flag = (volatile int*)(bars + 25);
+  uint64_t* bar_drain = bars + 24;      // MMA: everything issued has completed (abort path)
+  uint32_t* tmem_slot = (uint32_t*)(bars + 25);
+  volatile int* abort_flag = (volatile int*)(bars + 26);
   float* nrm_x = (float*)(sm + G::oBar + 1024);   // [2][128] norm halves
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -185,6 +189,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(bar_pfull + 1, 1);
     mbar_init(bar_stage, 8);
     mbar_init(bar_sfree, 1);
+    mbar_init(bar_drain, 1);
     for (int i = 0; i < G::NSLOT; ++i) {
       mbar_init(bar_full + i, 1);
       mbar_init(bar_empty + i, 1);
@@ -198,8 +203,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 8) {
-    // ------------------------------------------- producer and MMA issuer
+  if (warp == 9) {
+    // ------------------------------------------------------------ producer
+    // the token tiles, then the W' items in consumption order, each into the
+    // slot its predecessor NSLOT back has left
     if (lane == 0) {
       prefetch_tmap(&tm_w);
       prefetch_tmap(&tm_q);
@@ -209,30 +216,42 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_load_4d(sm + G::oXK + s * 16384, &tm_k, 64 * s, t0, h, b, bar_x);
         tma_load_4d(sm + G::oXQ + s * 16384, &tm_q, 64 * s, t0, h, b, bar_x);
       }
-      int issued = 0, waited = 0;   // W' items loaded / waited for, in order
-      auto load_item = [&](int i) {
+      int last[G::NSLOT];
+      for (int i = 0; i < G::NSLOT; ++i) last[i] = -1;
+      bool ok = true;
+      for (int i = 0; ok && i < G::NITEMS; ++i) {
         const int slot = i % G::NSLOT;
-        const int row0 = i < G::NNORM ? M_ + 64 * i : 64 * (i - G::NNORM);
-        mbar_arrive_expect_tx(bar_full + slot, G::kSlot);
-        for (int s = 0; s < G::DS; ++s)
-          tma_load_2d(sm + G::oW + slot * G::kSlot + s * 8192, &tm_w, 64 * s,
-                      hw * (M_ + R_) + row0, bar_full + slot);
-      };
-      for (; issued < G::NSLOT && issued < G::NITEMS; ++issued) load_item(issued);
+        if (i >= G::NSLOT &&
+            !(ok = wait_one(bar_empty + slot, ((i / G::NSLOT) - 1) & 1, abort_flag, p.dev_status)))
+          break;
+        uint8_t* dst = sm + G::oW + slot * G::kSlot;
+        if (i < G::NNORM) {          // norm rows, d slab i
+          mbar_arrive_expect_tx(bar_full + slot, R_ * 128);
+          for (int j = 0; j < R_ / 64; ++j)
+            tma_load_2d(dst + j * 8192, &tm_w, 64 * i, hw * (M_ + R_) + M_ + 64 * j, bar_full + slot);
+        } else {                     // feature rows 64 (i - NNORM) .. + 63, all of d
+          mbar_arrive_expect_tx(bar_full + slot, G::kSlot);
+          for (int s = 0; s < G::DS; ++s)
+            tma_load_2d(dst + s * 8192, &tm_w, 64 * s, hw * (M_ + R_) + 64 * (i - G::NNORM),
+                        bar_full + slot);
+        }
+        last[slot] = i;
+      }
+      if (!ok) {
+        // leave no copy in flight (a completed phase passes at once)
+        mbar_wait(bar_x, 0);
+        for (int i = 0; i < G::NSLOT; ++i)
+          if (last[i] >= 0) mbar_wait(bar_full + i, (last[i] / G::NSLOT) & 1);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 8) {
+    // ---------------------------------------------------------- MMA issuer
+    if (lane == 0) {
       const uint32_t sXK = s0 + G::oXK, sXQ = s0 + G::oXQ;
-      // after issuing item i: refill the slot item i-1 used, once its MMAs are done
-      auto refill = [&](int i) -> bool {
-        if (i < 1 || issued >= G::NITEMS) return true;
-        const int j = i - 1;
-        if (!wait_one(bar_empty + j % G::NSLOT, (j / G::NSLOT) & 1, abort_flag, p.dev_status))
-          return false;
-        load_item(issued++);
-        return true;
-      };
       auto feat_block = [&](int n) -> bool {   // K and Q GEMMs of feature block n
         const int i = G::NNORM + n, slot = i % G::NSLOT;
         if (!wait_one(bar_full + slot, (i / G::NSLOT) & 1, abort_flag, p.dev_status)) return false;
-        ++waited;
         tc_fence_after();
         const uint32_t sw = s0 + G::oW + slot * G::kSlot;
         const uint32_t tp = tmem + 128 * (n & 1);
@@ -247,25 +266,21 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         mma_commit(bar_empty + slot);
         mma_commit(bar_pfull + (n & 1));
-        return refill(i);
+        return true;
       };
       bool ok = wait_one(bar_conv, 0, abort_flag, p.dev_status);
-      // ---- norm GEMM: columns [0, R_)
+      // ---- norm GEMM: columns [0, R_), one N = R_ MMA per K-step
       for (int i = 0; ok && i < G::NNORM; ++i) {
         const int slot = i % G::NSLOT;
         if (!(ok = wait_one(bar_full + slot, (i / G::NSLOT) & 1, abort_flag, p.dev_status))) break;
-        ++waited;
         tc_fence_after();
         const uint32_t sw = s0 + G::oW + slot * G::kSlot;
-        constexpr uint32_t id = idesc(128, 64, false, false, true);
+        constexpr uint32_t id = idesc(128, R_, false, false, true);
 #pragma unroll
-        for (int s = 0; s < G::DS; ++s)
-#pragma unroll
-          for (int k = 0; k < 4; ++k)
-            mma(tmem + 64 * i, sdesc(sXK + s * 16384 + k * 32, 16, 1024),
-                sdesc(sw + s * 8192 + k * 32, 16, 1024), id, (s | k) != 0);
+        for (int k = 0; k < 4; ++k)
+          mma(tmem, sdesc(sXK + i * 16384 + k * 32, 16, 1024), sdesc(sw + k * 32, 16, 1024), id,
+              (i | k) != 0);
         mma_commit(bar_empty + slot);
-        ok = refill(i);
       }
       if (ok) mma_commit(bar_norm);
       // ---- feature blocks (P buffers overwrite the norm columns once read)
@@ -284,10 +299,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         mma_commit(bar_sfree);
         if (n + 2 < G::NFEAT) ok = feat_block(n + 2);
       }
-      // leave no copy in flight: the token tiles and the W' items not waited for
       if (!ok) {
-        mbar_wait(bar_x, 0);
-        for (int i = waited; i < issued; ++i) mbar_wait(bar_full + i % G::NSLOT, (i / G::NSLOT) & 1);
+        // let every issued MMA finish before TMEM is released
+        mma_commit(bar_drain);
+        mbar_wait(bar_drain, 0);
       }
     }
     __syncwarp();
@@ -440,8 +455,10 @@ struct ValParams {
   int* dev_status;
 };
 
+constexpr int kThreadsV = kEpiThreads + 64;   // + MMA warp 8 + producer warp 9
+
 template <int M_>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreadsV, 1)
     values_kernel(const __grid_constant__ CUtensorMap tm_v, const ValParams p) {
   using G = ValCfg<M_>;
   extern __shared__ uint8_t smem_raw[];
@@ -457,8 +474,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* bar_ds = bars + 8;          // [NT] MMA: state tile f updated by the chunk
   uint64_t* bar_full = bars + 16;       // [NSLOT] ring slot loaded
   uint64_t* bar_empty = bars + 20;      // [NSLOT] ring slot read
-  uint32_t* tmem_slot = (uint32_t*)(bars + 24);
-  volatile int* abort_flag = (volatile int*)(bars + 25);
+  uint64_t* bar_drain = bars + 24;      // MMA: everything issued has completed (abort path)
+  uint32_t* tmem_slot = (uint32_t*)(bars + 25);
+  volatile int* abort_flag = (volatile int*)(bars + 26);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int bh = blockIdx.x / p.nvb, vb = blockIdx.x % p.nvb;
@@ -476,6 +494,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(bar_nfull, 1);
     mbar_init(bar_nfree, 8);
     for (int f = 0; f < G::NT; ++f) mbar_init(bar_ds + f, 1);
+    mbar_init(bar_drain, 1);
     for (int i = 0; i < G::NSLOT; ++i) {
       mbar_init(bar_full + i, 1);
       mbar_init(bar_empty + i, 1);
@@ -485,7 +504,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   // zeroed S image and ones block: 1.0 (bf16) at column 0 of each of its 128
   // 128-byte rows (128B swizzle puts it in 16-byte chunk row % 8)
-  for (int i = tid; i < (int)((16384 + 49152) / 16); i += kThreads) {
+  for (int i = tid; i < (int)((16384 + 49152) / 16); i += kThreadsV) {
     const uint32_t off = i < 1024 ? G::oOnes + i * 16 : G::oS + (i - 1024) * 16;
     st_shared_v4(s0 + off, 0u, 0u, 0u, 0u);
   }
@@ -498,57 +517,60 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 8) {
-    // ------------------------------------------- producer and MMA issuer
+  if (warp == 9) {
+    // ------------------------------------------------------------ producer
+    // ring items in consumption order, each into the slot its predecessor
+    // NSLOT back has left; the V slice of chunk c before the chunk's first item
     if (lane == 0) {
       prefetch_tmap(&tm_v);
       const int total = p.nc * G::NITEM;
-      int issued = 0, waited = 0;        // ring items loaded / waited for, in order
-      int v_issued = 0, v_waited = 0;    // V slices loaded / waited for
-      auto load_item = [&](int g) {
+      int last[G::NSLOT], vlast[2] = {-1, -1};
+      for (int i = 0; i < G::NSLOT; ++i) last[i] = -1;
+      bool ok = true;
+      for (int g = 0; ok && g < total; ++g) {
         const int c = g / G::NITEM, i = g % G::NITEM;
+        if (i == 0) {
+          if (c > 1 &&
+              !(ok = wait_one(bar_vempty + (c & 1), ((c - 2) >> 1) & 1, abort_flag, p.dev_status)))
+            break;
+          mbar_arrive_expect_tx(bar_v + (c & 1), 16384);
+          tma_load_4d(sm + G::oV + (c & 1) * 16384, &tm_v, 64 * vb, c * kC, h, b, bar_v + (c & 1));
+          vlast[c & 1] = c;
+        }
+        const int slot = g % G::NSLOT;
+        if (g >= G::NSLOT &&
+            !(ok = wait_one(bar_empty + slot, ((g / G::NSLOT) - 1) & 1, abort_flag, p.dev_status)))
+          break;
         const uint8_t* rc = recs + (size_t)c * rec_bytes;
         const uint8_t* src;
         if (i == 1) {
-          src = rc + (size_t)2 * M_ * 256;                         // A_c
+          src = rc + (size_t)2 * M_ * 256;                                          // A_c
         } else if (i == 0 || (i & 1)) {
           src = rc + (size_t)M_ * 256 + (size_t)(i == 0 ? 0 : (i - 1) / 2) * 32768;   // Psi_f
         } else {
-          src = rc + (size_t)((i - 2) / 2) * 32768;                  // Phi_f
+          src = rc + (size_t)((i - 2) / 2) * 32768;                                   // Phi_f
         }
-        const int slot = g % G::NSLOT;
         mbar_arrive_expect_tx(bar_full + slot, 32768);
         bulk_load(sm + G::oR + slot * 32768, src, 32768, bar_full + slot);
-      };
-      auto load_v = [&](int c) -> bool {
-        if (c > 1 && !wait_one(bar_vempty + (c & 1), ((c - 2) >> 1) & 1, abort_flag, p.dev_status))
-          return false;
-        mbar_arrive_expect_tx(bar_v + (c & 1), 16384);
-        tma_load_4d(sm + G::oV + (c & 1) * 16384, &tm_v, 64 * vb, c * kC, h, b, bar_v + (c & 1));
-        v_issued = c + 1;
-        return true;
-      };
-      // after issuing the MMAs of item g: keep items up to g + NSLOT - 1 loaded;
-      // each load waits for the item that last used its slot (at most item g - 1)
-      auto refill = [&](int g) -> bool {
-        while (issued <= g + G::NSLOT - 1 && issued < total) {
-          const int j = issued - G::NSLOT;
-          if (j >= 0 &&
-              !wait_one(bar_empty + j % G::NSLOT, (j / G::NSLOT) & 1, abort_flag, p.dev_status))
-            return false;
-          load_item(issued++);
-        }
-        return true;
-      };
+        last[slot] = g;
+      }
+      if (!ok) {
+        // leave no copy in flight (a completed phase passes at once)
+        for (int i = 0; i < G::NSLOT; ++i)
+          if (last[i] >= 0) mbar_wait(bar_full + i, (last[i] / G::NSLOT) & 1);
+        for (int j = 0; j < 2; ++j)
+          if (vlast[j] >= 0) mbar_wait(bar_v + j, (vlast[j] >> 1) & 1);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 8) {
+    // ---------------------------------------------------------- MMA issuer
+    if (lane == 0) {
       auto wait_item = [&](int g) -> bool {
-        if (!wait_one(bar_full + g % G::NSLOT, (g / G::NSLOT) & 1, abort_flag, p.dev_status))
-          return false;
-        ++waited;
-        return true;
+        return wait_one(bar_full + g % G::NSLOT, (g / G::NSLOT) & 1, abort_flag, p.dev_status);
       };
       auto slot_addr = [&](int g) -> uint32_t { return s0 + G::oR + (g % G::NSLOT) * 32768; };
-      bool ok = load_v(0);
-      for (; ok && issued < G::NSLOT && issued < total; ++issued) load_item(issued);
+      bool ok = true;
       const uint32_t tnum = tmem + G::tNum;
       const uint32_t sS = s0 + G::oS, sOnes = s0 + G::oOnes;
       for (int c = 0; ok && c < p.nc; ++c) {
@@ -556,7 +578,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t sV = s0 + G::oV + j * 16384;
         const uint32_t lbo_v1 = G::oOnes - (G::oV + j * 16384);   // [V | 1]: ones block after V
         if (!(ok = wait_one(bar_v + j, (c >> 1) & 1, abort_flag, p.dev_status))) break;
-        ++v_waited;
         if (c > 0 && !(ok = wait_one(bar_nfree, (c - 1) & 1, abort_flag, p.dev_status))) break;
         for (int f = 0; ok && f < G::NT; ++f) {
           const int k = c * G::NT + f;
@@ -591,8 +612,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           mma_commit(bar_empty + gP % G::NSLOT);
           if (f == 0) mma_commit(bar_empty + (g0 + 1) % G::NSLOT);
-          if (!(ok = refill(gP))) break;
-          if (f == 0 && c + 1 < p.nc && !(ok = load_v(c + 1))) break;
           if (!(ok = wait_item(gF))) break;
           tc_fence_after();
           // S_f += Phi_f^T [V_c | 1]
@@ -607,16 +626,15 @@ __global__ void __launch_bounds__(kThreads, 1)
             mma_commit(bar_ds + f);
             mma_commit(bar_empty + gF % G::NSLOT);
           }
-          if (!(ok = refill(gF))) break;
         }
         if (!ok) break;
         mma_commit(bar_nfull);
         mma_commit(bar_vempty + j);
       }
       if (!ok) {
-        // leave no copy in flight
-        for (int g = waited; g < issued; ++g) mbar_wait(bar_full + g % G::NSLOT, (g / G::NSLOT) & 1);
-        for (int c = v_waited; c < v_issued; ++c) mbar_wait(bar_v + (c & 1), (c >> 1) & 1);
+        // let every issued MMA finish before TMEM is released
+        mma_commit(bar_drain);
+        mbar_wait(bar_drain, 0);
       }
     }
     __syncwarp();
@@ -781,7 +799,7 @@ cudaError_t launch(const FwdArgs& a) {
   if (e != cudaSuccess) return e;
   e = set_smem_limit_once((const void*)values_kernel<M_>, (int)V::kSmem, smem_v);
   if (e != cudaSuccess) return e;
-  features_kernel<D_, M_, R_><<<a.B * a.H * nc, kThreads, F::kSmem, a.stream>>>(a.tm_w, a.tm_q,
+  features_kernel<D_, M_, R_><<<a.B * a.H * nc, kThreadsF, F::kSmem, a.stream>>>(a.tm_w, a.tm_q,
                                                                                  a.tm_k, fp);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
@@ -801,7 +819,7 @@ cudaError_t launch(const FwdArgs& a) {
   vp.st_z = a.st_z;
   vp.d = D_;
   vp.dev_status = a.dev_status;
-  values_kernel<M_><<<a.B * a.H * (D_ / 64), kThreads, V::kSmem, a.stream>>>(a.tm_v, vp);
+  values_kernel<M_><<<a.B * a.H * (D_ / 64), kThreadsV, V::kSmem, a.stream>>>(a.tm_v, vp);
   return cudaGetLastError();
 }
 
