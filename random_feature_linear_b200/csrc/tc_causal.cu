@@ -21,10 +21,10 @@
 // consecutive chunks of one head and carries the prefix state in registers,
 // adding Phi(K_c)^T [V_c | 1] after each chunk. With many heads (B*H >= #SMs)
 // a segment is the whole head; with few heads each head is cut into G
-// segments so that all SMs work, and two small launches come first: the
-// key-state kernel sums Phi(K)^T [V | 1] over each segment and a scan turns
-// the segment sums into exclusive prefixes in a fixed order (deterministic,
-// no waiting between blocks).
+// segments so that all SMs work, and a key-state launch comes first: it sums
+// Phi(K)^T [V | 1] over each segment, and each CTA adds the sums of the
+// segments before its own in segment order (deterministic, no waiting
+// between blocks).
 #include <string.h>
 
 #include "common.cuh"
@@ -84,7 +84,7 @@ struct Params {
   int B, H, L, nc;              // nc = chunks per head
   int heads_w;
   int nseg;                     // segments per head
-  const float* seg_prefix;      // [B*H*nseg][65][m] exclusive segment prefixes (nseg > 1)
+  const float* seg_sums;        // [B*H*nseg][65][m] per-segment key states (nseg > 1)
   float *st_kv, *st_z;          // state after the last chunk
   int* dev_status;
 };
@@ -138,14 +138,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   uint32_t ph_tma = 0, ph_mma = 0;
   float run[65];                               // prefix state row `feat` (fp32)
-  if (has_feat && seg > 0) {
-    const float* sp = p.seg_prefix + (size_t)blockIdx.x * 65 * M_;
 #pragma unroll
-    for (int i = 0; i < 65; ++i) run[i] = sp[(size_t)i * M_ + feat];
-  } else {
-#pragma unroll
-    for (int i = 0; i < 65; ++i) run[i] = 0.f;
-  }
+  for (int i = 0; i < 65; ++i) run[i] = 0.f;
   bool abort = false;
 
   for (int c = c_begin; c < c_end && !abort; ++c) {
@@ -158,6 +152,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       tma_load_4d(sm + G::oK, &tm_k, 0, t0, h, b, bar_tma);
       tma_load_4d(sm + G::oV, &tm_v, 0, t0, h, b, bar_tma);
       tma_load_4d(sm + G::oQ, &tm_q, 0, t0, h, b, bar_tma);
+    }
+    if (c == c_begin && seg > 0 && has_feat) {
+      // exclusive prefix of this segment: the earlier segments' key states,
+      // added in segment order while the first chunk's tiles load
+      for (int g = 0; g < seg; ++g) {
+        const float* sp = p.seg_sums + (size_t)(bh * p.nseg + g) * 65 * M_ + feat;
+#pragma unroll
+        for (int i = 0; i < 65; ++i) run[i] += sp[(size_t)i * M_];
+      }
     }
     if (!wait_all(bar_tma, ph_tma, p.dev_status)) { abort = true; break; }
     ph_tma ^= 1;
@@ -401,29 +404,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-// In place: segment sums of each head -> exclusive prefixes, in segment order.
-// All segment loads are issued before the dependent adds (at most kSms segments).
-__global__ void segment_scan_kernel(float* __restrict__ seg, int nseg, int m) {
-  const int bh = blockIdx.y;
-  const int idx = blockIdx.x * blockDim.x + threadIdx.x;
-  if (idx >= 65 * m) return;
-  float* base = seg + (size_t)bh * nseg * 65 * m + idx;
-  const size_t step = (size_t)65 * m;
-  float run = 0.f;
-  for (int s0 = 0; s0 < nseg; s0 += 16) {
-    float t[16];
-#pragma unroll
-    for (int u = 0; u < 16; ++u) t[u] = s0 + u < nseg ? base[(s0 + u) * step] : 0.f;
-#pragma unroll
-    for (int u = 0; u < 16; ++u) {
-      if (s0 + u < nseg) {
-        base[(s0 + u) * step] = run;
-        run += t[u];
-      }
-    }
-  }
-}
-
 struct Layout {
   int nc, nseg;
   size_t off_seg, total;
@@ -453,7 +433,6 @@ cudaError_t launch(const FwdArgs& a, const CUtensorMap& tw, const CUtensorMap& t
   if (s.nseg > 1) {
     e = tc_launch_key_states(a, tw, tk, tv, s.nc, s.nseg, seg);
     if (e != cudaSuccess) return e;
-    segment_scan_kernel<<<dim3((65 * a.m + 255) / 256, bh), 256, 0, a.stream>>>(seg, s.nseg, a.m);
   }
   Params p;
   memset(&p, 0, sizeof(p));
@@ -468,7 +447,7 @@ cudaError_t launch(const FwdArgs& a, const CUtensorMap& tw, const CUtensorMap& t
   p.nc = s.nc;
   p.heads_w = a.heads_w;
   p.nseg = s.nseg;
-  p.seg_prefix = seg;
+  p.seg_sums = seg;
   p.st_kv = a.st_kv;
   p.st_z = a.st_z;
   p.dev_status = a.dev_status;
