@@ -142,17 +142,20 @@ __global__ void __launch_bounds__(kThreads, 1)
   for (int i = 0; i < 65; ++i) run[i] = 0.f;
   bool abort = false;
 
+  // W', K, V and Q tiles of the chunk starting at token t (one thread)
+  auto issue_loads = [&](int t) {
+    mbar_arrive_expect_tx(bar_tma, G::kW + 3 * kTileBytes);
+    for (int r0 = 0; r0 < G::NW; r0 += 16)
+      tma_load_2d(sm + G::oW + r0 * 128, &tm_w, 0, hw * G::NW + r0, bar_tma);
+    tma_load_4d(sm + G::oK, &tm_k, 0, t, h, b, bar_tma);
+    tma_load_4d(sm + G::oV, &tm_v, 0, t, h, b, bar_tma);
+    tma_load_4d(sm + G::oQ, &tm_q, 0, t, h, b, bar_tma);
+  };
   for (int c = c_begin; c < c_end && !abort; ++c) {
     const int t0 = c * kC;
     // ---------------------------------------------------------------- loads
-    if (tid == 0) {
-      mbar_arrive_expect_tx(bar_tma, G::kW + 3 * kTileBytes);
-      for (int r0 = 0; r0 < G::NW; r0 += 16)
-          tma_load_2d(sm + G::oW + r0 * 128, &tm_w, 0, hw * G::NW + r0, bar_tma);
-      tma_load_4d(sm + G::oK, &tm_k, 0, t0, h, b, bar_tma);
-      tma_load_4d(sm + G::oV, &tm_v, 0, t0, h, b, bar_tma);
-      tma_load_4d(sm + G::oQ, &tm_q, 0, t0, h, b, bar_tma);
-    }
+    // (for later chunks they were issued during the previous chunk's output)
+    if (tid == 0 && c == c_begin) issue_loads(t0);
     if (c == c_begin && seg > 0 && has_feat) {
       // exclusive prefix of this segment: the earlier segments' key states,
       // added in segment order while the first chunk's tiles load
@@ -356,6 +359,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (!wait_all(bar_mma, ph_mma, p.dev_status)) { abort = true; break; }
     ph_mma ^= 1;
     tc_fence_after();
+    // every tile region has been read: the next chunk's tiles load during the output
+    if (tid == 0 && c + 1 < c_end) issue_loads(t0 + kC);
     // ------------------------------------------------------------- output
     {
       float den = tmem_ld1(lane_tm + G::tDen);
