@@ -11,6 +11,7 @@
 
 #include "common.cuh"
 #include "internal.h"
+#include "tc_common.cuh"
 
 namespace dark {
 namespace {
@@ -84,9 +85,15 @@ __device__ __forceinline__ float block_sum(float v, float* scratch) {
 }
 
 
-// 8 consecutive weights of a W' row as fp32 (fp16 or fp32 storage).
+// W' of one head is copied to shared memory (one bulk copy at the start,
+// overlapping the state prefetch) when it is at most this large; the feature
+// GEMV then reads it there instead of paying L2 latency per batch of rows.
+constexpr size_t kStageW = 64 * 1024;
+
+// 8 consecutive weights of a W' row as fp32 (fp16 or fp32 storage; the row is
+// in global memory or, when staged, in shared memory: a generic load).
 __device__ __forceinline__ void load_w8(const __half* __restrict__ w, float (&f)[8]) {
-  const uint4 u = __ldg(reinterpret_cast<const uint4*>(w));
+  const uint4 u = *reinterpret_cast<const uint4*>(w);
   const __half2* h = reinterpret_cast<const __half2*>(&u);
 #pragma unroll
   for (int e = 0; e < 4; ++e) {
@@ -96,8 +103,8 @@ __device__ __forceinline__ void load_w8(const __half* __restrict__ w, float (&f)
   }
 }
 __device__ __forceinline__ void load_w8(const float* __restrict__ w, float (&f)[8]) {
-  const float4 a = __ldg(reinterpret_cast<const float4*>(w));
-  const float4 b = __ldg(reinterpret_cast<const float4*>(w) + 1);
+  const float4 a = *reinterpret_cast<const float4*>(w);
+  const float4 b = *(reinterpret_cast<const float4*>(w) + 1);
   f[0] = a.x; f[1] = a.y; f[2] = a.z; f[3] = a.w;
   f[4] = b.x; f[5] = b.y; f[6] = b.z; f[7] = b.w;
 }
@@ -162,8 +169,9 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(
     const typename WeightOf<T>::type* __restrict__ w, int heads_w, int m, int r, int d,
     float* __restrict__ kv, float* __restrict__ z, const float* __restrict__ shift, int H,
     const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v, T* __restrict__ out,
-    const uint8_t* __restrict__ valid, int* dev_status) {
-  extern __shared__ float sm[];
+    const uint8_t* __restrict__ valid, int* dev_status, int stage_w) {
+  using TW = typename WeightOf<T>::type;
+  extern __shared__ __align__(16) float sm[];
   const int tpr = d / 4;                  // threads per state row (one float4 each)
   const int rpp = kThreads / tpr;         // rows per pass
   float* xq = sm;                         // [d]
@@ -173,9 +181,23 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(
   float* pq = pk + m + r;                 // [m]
   float* red = pq + m;                    // [rpp][d]
   float* scratch = red + rpp * d;         // [32]
+  // 16-byte aligned tail: the copy barrier, then the staged W' rows [m + r][d]
+  const size_t tail = ((size_t)(3 * d + (m + r) + m + rpp * d + 32) * 4 + 15) / 16 * 16;
+  uint64_t* bar_w = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(sm) + tail);
+  TW* w_sm = reinterpret_cast<TW*>(reinterpret_cast<uint8_t*>(sm) + tail + 16);
   const int bh = blockIdx.x, b = bh / H, h = bh % H;
-  const auto* wh = w + (size_t)(heads_w == 1 ? 0 : h) * (m + r) * d;
+  const TW* wg = w + (size_t)(heads_w == 1 ? 0 : h) * (m + r) * d;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const uint32_t w_bytes = (uint32_t)((size_t)(m + r) * d * sizeof(TW));
+  if (stage_w && tid == 0) {
+    tc::mbar_init(bar_w, 1);
+    tc::fence_mbar_init();
+    tc::mbar_arrive_expect_tx(bar_w, w_bytes);
+    for (uint32_t o = 0; o < w_bytes; o += 16384)
+      tc::bulk_load(reinterpret_cast<uint8_t*>(w_sm) + o, reinterpret_cast<const uint8_t*>(wg) + o,
+                    w_bytes - o < 16384 ? w_bytes - o : 16384, bar_w);
+  }
+  const TW* wh = stage_w ? w_sm : wg;
   const int c4 = tid % tpr, r0 = tid / tpr;
   const bool rows_active = r0 < rpp;
   float4* base = reinterpret_cast<float4*>(kv + (size_t)bh * m * d) + c4;
@@ -204,6 +226,18 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(
     xv[c] = to_f32(v[(size_t)bh * d + c]);
   }
   __syncthreads();
+  if (stage_w) {
+    // W' in shared memory (bounded wait; on a time-out nothing is written)
+    const bool arrived = tc::mbar_wait(bar_w, 0);
+    if (__syncthreads_or(arrived ? 0 : 1)) {
+      if (tid == 0) {
+        report(dev_status, DARK_ERR_TIMEOUT);
+        tc::mbar_wait(bar_w, 0);   // the copy must not land after the block is gone
+      }
+      __syncthreads();
+      return;
+    }
+  }
   // Feature exponents W' k and W' q: groups of 8 lanes own one row at a time,
   // each lane 8 consecutive columns (held in registers), reduced by shuffles.
   // Rows whose length is not a multiple of 8 take one thread per row instead.
@@ -294,23 +328,33 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(
 cudaError_t launch_decode(const DecodeArgs& a) {
   const int tpr = a.d / 4;
   const int rpp = kThreads / tpr;
-  const size_t smem = sizeof(float) * (3 * a.d + (a.m + a.r) + a.m + rpp * a.d + 40);
+  const size_t welt = a.dtype == DARK_BF16 ? sizeof(__half) : sizeof(float);
+  const size_t w_bytes = (size_t)(a.m + a.r) * a.d * welt;
+  // staged W': each head's rows 16-byte aligned for the bulk copy, and rows of
+  // a multiple of 8 elements (the 8-lane GEMV, the only one reading it there)
+  const int stage_w = w_bytes <= kStageW && w_bytes % 16 == 0 && a.d % 8 == 0 &&
+                      ((uintptr_t)a.w & 15) == 0;
+  const size_t tail = (sizeof(float) * (3 * a.d + (a.m + a.r) + a.m + rpp * a.d + 32) + 15) / 16 * 16;
+  const size_t smem = tail + (stage_w ? 16 + w_bytes : 0);
+  // one opt-in per device that covers every size: at most 4128 floats of
+  // vectors and partial sums (d <= 256, m <= 1024, r <= 256) plus staged W'
+  constexpr int kSmemOptIn = 96 * 1024;
   cudaError_t err;
   if (a.dtype == DARK_BF16) {
     static int done[64];
-    err = set_smem_limit_once((const void*)decode_kernel<__nv_bfloat16>, (int)smem, done);
+    err = set_smem_limit_once((const void*)decode_kernel<__nv_bfloat16>, kSmemOptIn, done);
     if (err != cudaSuccess) return err;
     decode_kernel<__nv_bfloat16><<<a.B * a.H, kThreads, smem, a.stream>>>(
         (const __half*)a.w, a.heads_w, a.m, a.r, a.d, a.kv, a.z, a.shift, a.H,
         (const __nv_bfloat16*)a.q, (const __nv_bfloat16*)a.k, (const __nv_bfloat16*)a.v,
-        (__nv_bfloat16*)a.out, a.valid, a.dev_status);
+        (__nv_bfloat16*)a.out, a.valid, a.dev_status, stage_w);
   } else {
     static int done[64];
-    err = set_smem_limit_once((const void*)decode_kernel<float>, (int)smem, done);
+    err = set_smem_limit_once((const void*)decode_kernel<float>, kSmemOptIn, done);
     if (err != cudaSuccess) return err;
     decode_kernel<float><<<a.B * a.H, kThreads, smem, a.stream>>>(
         (const float*)a.w, a.heads_w, a.m, a.r, a.d, a.kv, a.z, a.shift, a.H, (const float*)a.q,
-        (const float*)a.k, (const float*)a.v, (float*)a.out, a.valid, a.dev_status);
+        (const float*)a.k, (const float*)a.v, (float*)a.out, a.valid, a.dev_status, stage_w);
   }
   return cudaGetLastError();
 }
