@@ -164,6 +164,79 @@ __device__ __forceinline__ void feature_gemv(const TW* __restrict__ wh, int m, i
   }
 }
 
+// 8 consecutive weights of a staged W' row (shared memory) as fp32.
+__device__ __forceinline__ void load_w8_shared(uint32_t saddr, const __half*, float (&f)[8]) {
+  const uint4 u = tc::ld_shared_v4(saddr);
+  const __half2* h = reinterpret_cast<const __half2*>(&u);
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const float2 t = __half22float2(h[e]);
+    f[2 * e] = t.x;
+    f[2 * e + 1] = t.y;
+  }
+}
+__device__ __forceinline__ void load_w8_shared(uint32_t saddr, const float*, float (&f)[8]) {
+  const uint4 a = tc::ld_shared_v4(saddr), b = tc::ld_shared_v4(saddr + 16);
+  f[0] = __uint_as_float(a.x); f[1] = __uint_as_float(a.y);
+  f[2] = __uint_as_float(a.z); f[3] = __uint_as_float(a.w);
+  f[4] = __uint_as_float(b.x); f[5] = __uint_as_float(b.y);
+  f[6] = __uint_as_float(b.z); f[7] = __uint_as_float(b.w);
+}
+
+// The feature GEMV on staged W' rows (d a multiple of 8): 8-lane groups, one
+// row at a time per group, all rows of a group in flight together; also
+// returns this thread's share of sum_i (W'_{m+i} k)^2 (the key norm), which
+// lanes 0 of the groups hold and the caller reduces.
+template <typename TW>
+__device__ __forceinline__ float feature_gemv_shared(const TW* w_sm, int m, int r, int d,
+                                                     const float* xk, const float* xq, float* pk,
+                                                     float* pq) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int g = lane >> 3, cl = lane & 7;
+  const int rows = m + r;
+  constexpr int kGroups = kThreads / 8;
+  const uint32_t wbase = tc::smem_u32(w_sm);
+  float nrm = 0.f;
+  for (int c0 = 0; c0 < d; c0 += 64) {
+    const int col = c0 + cl * 8;
+    const bool cok = col < d;
+    float fk[8], fq[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      fk[e] = cok ? xk[col + e] : 0.f;
+      fq[e] = cok ? xq[col + e] : 0.f;
+    }
+#pragma unroll 4
+    for (int j = warp * 4 + g; j < rows; j += kGroups) {
+      float wv[8];
+      if (cok) {
+        load_w8_shared(wbase + (uint32_t)(((size_t)j * d + col) * sizeof(TW)), (const TW*)nullptr, wv);
+      } else {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) wv[e] = 0.f;
+      }
+      float ak = 0.f, aq = 0.f;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        ak = fmaf(wv[e], fk[e], ak);
+        aq = fmaf(wv[e], fq[e], aq);
+      }
+#pragma unroll
+      for (int o = 4; o > 0; o >>= 1) {
+        ak += __shfl_xor_sync(0xffffffffu, ak, o);
+        aq += __shfl_xor_sync(0xffffffffu, aq, o);
+      }
+      if (cl == 0) {
+        const float tk = (c0 == 0 ? 0.f : pk[j]) + ak;
+        pk[j] = tk;
+        if (j < m) pq[j] = (c0 == 0 ? 0.f : pq[j]) + aq;
+        else if (c0 + 64 >= d) nrm = fmaf(tk, tk, nrm);   // norm row, all columns summed
+      }
+    }
+  }
+  return nrm;
+}
+
 template <typename T>
 __global__ void __launch_bounds__(kThreads, 2) decode_kernel(
     const typename WeightOf<T>::type* __restrict__ w, int heads_w, int m, int r, int d,
@@ -203,8 +276,12 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(
   float4* base = reinterpret_cast<float4*>(kv + (size_t)bh * m * d) + c4;
   const int stride = d / 4;
 
-  // The state rows of the first pass are requested before anything else so
-  // that their HBM latency overlaps the feature computation below.
+  // The step's tokens first (they gate the feature GEMV), then the state rows
+  // of the first pass, whose HBM latency overlaps the feature computation.
+  const bool has_c = tid < d;             // d <= kThreads: one element per thread
+  const T q_e = has_c ? q[(size_t)bh * d + tid] : T(0.f);
+  const T k_e = has_c ? k[(size_t)bh * d + tid] : T(0.f);
+  const T v_e = has_c ? v[(size_t)bh * d + tid] : T(0.f);
   float4 s[kBatchRows];
   if (rows_active) {
 #pragma unroll
@@ -220,10 +297,10 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(
     zpre[u] = j < m ? __ldcs(z + (size_t)bh * m + j) : 0.f;
   }
 
-  for (int c = tid; c < d; c += kThreads) {
-    xq[c] = to_f32(q[(size_t)bh * d + c]);
-    xk[c] = to_f32(k[(size_t)bh * d + c]);
-    xv[c] = to_f32(v[(size_t)bh * d + c]);
+  if (has_c) {
+    xq[tid] = to_f32(q_e);
+    xk[tid] = to_f32(k_e);
+    xv[tid] = to_f32(v_e);
   }
   __syncthreads();
   if (stage_w) {
@@ -241,33 +318,47 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(
   // Feature exponents W' k and W' q: groups of 8 lanes own one row at a time,
   // each lane 8 consecutive columns (held in registers), reduced by shuffles.
   // Rows whose length is not a multiple of 8 take one thread per row instead.
-  if (d % 8 != 0) {
-    for (int j = tid; j < m + r; j += kThreads) {
-      float ak, aq;
-      row_dot2(wh + (size_t)j * d, d, xk, xq, j < m, ak, aq);
-      pk[j] = ak;
-      if (j < m) pq[j] = aq;
-    }
-  } else {
-    feature_gemv<2>(wh, m, r, d, xk, xq, pk, pq);
-  }
-  __syncthreads();
-  // warp 0: key norm (base 2, with 1/2 log2 m) and, when stabilised, the query max
   const bool stab = shift != nullptr;
-  if (warp == 0) {
-    float nrm = 0.f, qmax = -INFINITY;
-    for (int i = lane; i < r; i += 32) nrm = fmaf(pk[m + i], pk[m + i], nrm);
-    if (stab)
-      for (int j = lane; j < m; j += 32) qmax = fmaxf(qmax, pq[j]);
-    nrm = warp_sum(nrm);
-    qmax = warp_max(qmax);
-    if (lane == 0) {
-      scratch[0] = nrm + 0.5f * log2f((float)m) + (stab ? shift[bh] : 0.f);
-      scratch[1] = stab ? qmax : 0.f;
+  float ks, qs;
+  if (stage_w && !stab) {
+    // GEMV on the staged rows; the key norm from per-warp partial sums
+    const float part = warp_sum(feature_gemv_shared(w_sm, m, r, d, xk, xq, pk, pq));
+    if (lane == 0) scratch[2 + warp] = part;
+    __syncthreads();
+    float nrm = 0.f;
+#pragma unroll
+    for (int i = 0; i < kThreads / 32; ++i) nrm += scratch[2 + i];
+    ks = nrm + 0.5f * log2f((float)m);
+    qs = 0.f;
+  } else {
+    if (d % 8 != 0) {
+      for (int j = tid; j < m + r; j += kThreads) {
+        float ak, aq;
+        row_dot2(wh + (size_t)j * d, d, xk, xq, j < m, ak, aq);
+        pk[j] = ak;
+        if (j < m) pq[j] = aq;
+      }
+    } else {
+      feature_gemv<2>(wh, m, r, d, xk, xq, pk, pq);
     }
+    __syncthreads();
+    // warp 0: key norm (base 2, with 1/2 log2 m) and, when stabilised, the query max
+    if (warp == 0) {
+      float nrm = 0.f, qmax = -INFINITY;
+      for (int i = lane; i < r; i += 32) nrm = fmaf(pk[m + i], pk[m + i], nrm);
+      if (stab)
+        for (int j = lane; j < m; j += 32) qmax = fmaxf(qmax, pq[j]);
+      nrm = warp_sum(nrm);
+      qmax = warp_max(qmax);
+      if (lane == 0) {
+        scratch[0] = nrm + 0.5f * log2f((float)m) + (stab ? shift[bh] : 0.f);
+        scratch[1] = stab ? qmax : 0.f;
+      }
+    }
+    __syncthreads();
+    ks = scratch[0];
+    qs = scratch[1];
   }
-  __syncthreads();
-  const float ks = scratch[0], qs = scratch[1];
   const bool ok = valid == nullptr || valid[b] != 0;
   for (int j = tid; j < m; j += kThreads) {
     pk[j] = ok ? exp2f(pk[j] - ks) : 0.f;
