@@ -54,6 +54,21 @@ def captured_traffic(cfg: int):
     return nbytes if h.hexdigest()[:16] == digest else None
 
 
+# Nominal exp2 rate of the special-function units: 16 per clock per SM x 148
+# SMs x 1.965 GHz (an explanatory third bound next to tensor and HBM time).
+MUFU_EX2_PER_S = 16 * 148 * 1.965e9
+
+
+def max_over_ranks(value: float, device) -> float:
+    """The largest of every rank's value (the job's time is its slowest rank's);
+    the value itself on one rank or without a process group."""
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 def alg_flops(w: synth.Workload) -> float:
     """Algorithmic FLOPs of one forward pass: per head 2Ldm (query features) +
     2Ld(m+r) (key features and norms) + 2Lm(d+1) (state) + 2Lm(d+1) (output)."""
@@ -246,10 +261,7 @@ def run_native(args, w: synth.Workload, rank: int, world: int, dev) -> dict | No
     if world > 1:
         dist.barrier()
     step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
-    total_ms = torch.tensor([sum(step_ms)], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(total_ms, op=dist.ReduceOp.MAX)
-    ms_per_step = total_ms.item() / args.steps
+    ms_per_step = max_over_ranks(sum(step_ms), dev) / args.steps
     assert int(status.item()) == 0, D.dark_status_string(int(status.item()))
 
     # end to end through the C ABI with pinned host buffers
@@ -280,9 +292,7 @@ def run_native(args, w: synth.Workload, rank: int, world: int, dev) -> dict | No
         e2e_step()
     e_end.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = torch.tensor([e_start.elapsed_time(e_end) / args.steps], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(e2e_ms, op=dist.ReduceOp.MAX)
+    e2e_ms = max_over_ranks(e_start.elapsed_time(e_end) / args.steps, dev)
     h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv)) + (
         0 if hmask is None else hmask.numel())
     d2h = hout.numel() * hout.element_size()
@@ -334,10 +344,11 @@ def run_native(args, w: synth.Workload, rank: int, world: int, dev) -> dict | No
                    "l2": "flushed (512 MiB write) before every timed step",
                    "timing": "CUDA events around one CUDA-graph replay of the forward call per step",
                    "parallelism": f"replicas x{world} (independent batches, no collective)"},
-        "e2e": {"value": tokens / (e2e_ms.item() / 1e3), "unit": "tokens/s",
+        "e2e": {"value": tokens / (e2e_ms / 1e3), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "roofline": roof,
         "roofline_other": {"t_tensor_us": t_tc * 1e6, "t_hbm_us": t_hbm * 1e6,
+                           "t_mufu_us_nominal": 2.0 * w.tokens * w.m / MUFU_EX2_PER_S * 1e6,
                            "alg_flops": flops, "alg_bytes": nbytes},
         "cpu_baseline": cpu,
         "gpu_launches": launches_per_step * args.steps,
@@ -439,7 +450,7 @@ def run_decode(args, rank: int, world: int, dev) -> dict | None:
             ends[i].record(stream)
         torch.cuda.synchronize()
     step_ms = [a.elapsed_time(b) for a, b in zip(starts, ends)]
-    ms = torch.tensor([statistics.median(step_ms)], dtype=torch.float64, device=dev)
+    ms = statistics.median(step_ms)
     # 1024 consecutive steps in one graph (state stays in L2 between steps)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     gall.replay()
@@ -465,14 +476,12 @@ def run_decode(args, rank: int, world: int, dev) -> dict | None:
         ho.copy_(do, non_blocking=True)
     e1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = torch.tensor([e0.elapsed_time(e1) / args.steps], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(ms, op=dist.ReduceOp.MAX)
-        dist.all_reduce(e2e_ms, op=dist.ReduceOp.MAX)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, dev)
+    ms = max_over_ranks(ms, dev)
     if rank != 0:
         return None
     rows = w.B * w.H * world
-    t = ms.item() / 1e3
+    t = ms / 1e3
     peaks = load_peaks()
     nbytes = decode_bytes(w)
     achieved = nbytes / t / 1e9
@@ -488,7 +497,7 @@ def run_decode(args, rank: int, world: int, dev) -> dict | None:
     clocks = clk.summary()
     return {
         "metric": DECODE_METRIC, "value": rows / t, "unit": "tokens/s", "n_gpus": world,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms.item(),
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded numpy, orthogonal Gaussian features)",
         "config": {"workload": "decode after a 4096-token causal prefill (B64 H8 d64 r64 m256, "
@@ -496,7 +505,7 @@ def run_decode(args, rank: int, world: int, dev) -> dict | None:
                    "l2": "flushed (512 MiB write) before every timed step",
                    "timing": "CUDA events around a one-step CUDA-graph replay",
                    "parallelism": f"replicas x{world} (independent batches, no collective)"},
-        "e2e": {"value": rows / (e2e_ms.item() / 1e3), "unit": "tokens/s",
+        "e2e": {"value": rows / (e2e_ms / 1e3), "unit": "tokens/s",
                 "h2d_bytes_per_step": 3 * dq.numel() * dq.element_size(),
                 "d2h_bytes_per_step": do.numel() * do.element_size()},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm"], "unit": "GB/s",
