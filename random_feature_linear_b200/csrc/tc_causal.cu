@@ -156,15 +156,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ---------------------------------------------------------------- loads
     // (for later chunks they were issued during the previous chunk's output)
     if (tid == 0 && c == c_begin) issue_loads(t0);
-    if (c == c_begin && seg > 0 && has_feat) {
-      // exclusive prefix of this segment: the earlier segments' key states,
-      // added in segment order while the first chunk's tiles load
-      for (int g = 0; g < seg; ++g) {
-        const float* sp = p.seg_sums + (size_t)(bh * p.nseg + g) * 65 * M_ + feat;
-#pragma unroll
-        for (int i = 0; i < 65; ++i) run[i] += sp[(size_t)i * M_];
-      }
-    }
     if (!wait_all(bar_tma, ph_tma, p.dev_status)) { abort = true; break; }
     ph_tma ^= 1;
     // k, then q: bf16 -> fp16 in place (the feature GEMMs run on fp16 operands);
@@ -253,6 +244,19 @@ __global__ void __launch_bounds__(kThreads, 1)
               sdesc(s0 + G::oV + s * 2048, G::oK - G::oV, 1024), idv, s > 0);
       }
       mma_commit(bar_mma);
+    }
+    if (c == c_begin && seg > 0) {
+      // exclusive prefix of this segment: the earlier segments' key states
+      // (written by the key-state launch, which may still be finishing: this
+      // launch starts early and waits for it only here), added in segment order
+      asm volatile("griddepcontrol.wait;" ::: "memory");
+      if (has_feat) {
+        for (int g = 0; g < seg; ++g) {
+          const float* sp = p.seg_sums + (size_t)(bh * p.nseg + g) * 65 * M_ + feat;
+#pragma unroll
+          for (int i = 0; i < 65; ++i) run[i] += sp[(size_t)i * M_];
+        }
+      }
     }
     if (!wait_all(bar_mma, ph_mma, p.dev_status)) { abort = true; break; }
     ph_mma ^= 1;
@@ -459,8 +463,21 @@ cudaError_t launch(const FwdArgs& a, const CUtensorMap& tw, const CUtensorMap& t
   static int smem_set[64];
   e = set_smem_limit_once((const void*)causal_kernel<M_, R_>, (int)G::kSmem, smem_set);
   if (e != cudaSuccess) return e;
-  causal_kernel<M_, R_><<<bh * s.nseg, kThreads, G::kSmem, a.stream>>>(tw, tq, tk, tv, p);
-  return cudaGetLastError();
+  // after the key-state launch: programmatic dependent launch, so that CTAs
+  // start on SMs the key-state CTAs leave and wait for its results only where
+  // they read them
+  cudaLaunchConfig_t cfg;
+  memset(&cfg, 0, sizeof(cfg));
+  cfg.gridDim = dim3(bh * s.nseg);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = G::kSmem;
+  cfg.stream = a.stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = s.nseg > 1 ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, causal_kernel<M_, R_>, tw, tq, tk, tv, p);
 }
 
 

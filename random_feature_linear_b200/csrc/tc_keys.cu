@@ -89,6 +89,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // a launch that follows with programmatic serialization may start now; it
+  // waits for this grid's results where it reads them
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const uint32_t lane_tm = tmem + ((uint32_t)(quad * 32) << 16);
 
   uint32_t ph_kv = 0, ph_mma = 0;             // bit i: phase parity of buffer i
