@@ -123,3 +123,28 @@ def test_decode_shared_projection(D, cuda_ok):
     ref = _oracle_decode(inp, stream, 3)
     for g, r in zip(got, ref):
         check(w, g[:, :, None], r[:, :, None])
+
+
+@pytest.mark.parametrize("dims", [(128, 256, 128), (256, 512, 256)])
+def test_decode_after_wide_prefill(D, cuda_ok, dims):
+    # prefill on the wide-head path (state carried in TMEM value blocks), then
+    # decode; at d=128 W' (96 KB) is read from L2, at d=256 as well (384 KB)
+    d, m, r = dims
+    w = synth.WORKLOADS[4].with_sizes(B=1, H=2, L=200, d=d, r=r, m=m)
+    inp = synth.make_inputs(w)
+    stream = synth.decode_stream(w, 3)
+    got, _ = _decode_run(D, cuda_ok, w, inp, stream, 3)
+    ref = _oracle_decode(inp, stream, 3)
+    for g, r_ in zip(got, ref):
+        check(w, g[:, :, None], r_[:, :, None])
+
+
+def test_decode_staged_projection_small_m(D, cuda_ok):
+    # m=128, r=32, d=64: W' (20 KB) staged in shared memory, 3 passes of rows
+    w = synth.WORKLOADS[5].with_sizes(B=2, H=3, L=150, m=128, r=32)
+    inp = synth.make_inputs(w)
+    stream = synth.decode_stream(w, 4)
+    got, _ = _decode_run(D, cuda_ok, w, inp, stream, 4)
+    ref = _oracle_decode(inp, stream, 4)
+    for g, r_ in zip(got, ref):
+        check(w, g[:, :, None], r_[:, :, None])

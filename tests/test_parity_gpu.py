@@ -57,11 +57,17 @@ def test_forward_matches_oracle(D, cuda_ok, name):
         assert err.max() <= (1e-4 if w.dtype == "f32" else 2e-2), err.max()
 
 
-def test_strided_inputs(D, cuda_ok):
-    w = synth.WORKLOADS[2].with_sizes(H=2, L=200, lengths=(200, 150))
+@pytest.mark.parametrize("recipe", ["c2", "wide-d128", "c3"])
+def test_strided_inputs(D, cuda_ok, recipe):
+    # q, k, v interleaved as [B][L][3][H][d] and out as [B][L][H][d]
+    w = {"c2": synth.WORKLOADS[2].with_sizes(H=2, L=200, lengths=(200, 150)),
+         "wide-d128": synth.WORKLOADS[4].with_sizes(B=2, H=2, L=150, d=128, r=128, m=256,
+                                                    lengths=(150, 90)),
+         "c3": synth.WORKLOADS[3].with_sizes(H=2, L=300)}[recipe]
     inp = synth.make_inputs(w)
     res = forward(D, w, inp, cuda_ok, strided=True)
-    out, _, _ = _oracle(inp, True)
+    assert res["status"] == 0
+    out, _, _ = _oracle(inp, w.causal)
     check(w, res["out"], out)
 
 
