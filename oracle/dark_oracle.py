@@ -17,7 +17,10 @@ Kernels for Transformers", darkformer-pytorch 0.1.0 package description):
   attention combines the token mask with the causal constraint.
 * section "Encoder-decoder model and generation": in linear mode the prompt is
   processed once and recurrent statistics (Phi(K)^T V, Phi(K)^T 1) are then
-  updated per appended token.
+  updated per appended token; decoder cross-attention summarises the encoded
+  source once per layer.
+* section "Cross-attention": queries attend over a separate context; query and
+  context masks are separate; there is no causal option.
 
 Readings where the pages are silent (each is listed with its reason in the
 design notes of this repository):
@@ -29,6 +32,8 @@ design notes of this repository):
   denominator and its output is defined as 0.
 * decode: the new key/value pair is added to the state first, then the output
   for the new query is emitted (the same inclusive rule as causal prefill).
+* cross-attention: the context mask drops context positions; a masked query
+  row outputs 0 (the pages do not say what the query mask does).
 
 Everything is computed in fp64 with plain numpy; bf16/fp32 inputs are upcast
 exactly. Parity of every function here is pinned by ``tests/test_oracle_pins.py``
@@ -185,6 +190,63 @@ def decode_step(kv, z, q_t, k_t, v_t, omega, geom, valid=None):
             den = pq @ z[b, h]
             out[b, h] = (pq @ kv[b, h]) / den if den > 0 else 0.0
     return out, kv, z
+
+
+def cross_attention(q, k, v, omega, geom, query_mask=None, context_mask=None):
+    """Cross-attention of queries over a separate context (README,
+    "Cross-attention": separate query and context masks, no causal option).
+
+    q: [B, H, Lq, d]; k, v: [B, H, Lk, d]; query_mask: [B, Lq]; context_mask:
+    [B, Lk] (nonzero = valid, None = all valid). out_i = sum_j kappa_hat(q_i, k_j)
+    v_j / sum_j kappa_hat(q_i, k_j) over the valid context positions j, written
+    out pair by pair; a masked query row, or one whose denominator is zero,
+    outputs 0. Returns (out [B, H, Lq, d], kv [B, H, m, d], z [B, H, m]), the
+    context summary Phi(K)^T V and Phi(K)^T 1 ("summarised once per layer").
+    """
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    B, H, Lq, d = q.shape
+    Lk = k.shape[2]
+    m = omega.shape[1]
+    out = np.zeros((B, H, Lq, d))
+    kv = np.zeros((B, H, m, d))
+    zz = np.zeros((B, H, m))
+    for b in range(B):
+        ctx = np.ones(Lk, bool) if context_mask is None else np.asarray(context_mask[b]) != 0
+        qry = np.ones(Lq, bool) if query_mask is None else np.asarray(query_mask[b]) != 0
+        for h in range(H):
+            om, gm = _head(omega, h), _head(geom, h)
+            phq = feature_map(q[b, h], om, gm)
+            phk = feature_map(k[b, h], om, gm)
+            for i in range(Lq):
+                if not qry[i]:
+                    continue
+                num = np.zeros(d)
+                den = 0.0
+                for j in range(Lk):
+                    if ctx[j]:
+                        w = float(phq[i] @ phk[j])
+                        num += w * v[b, h, j]
+                        den += w
+                out[b, h, i] = num / den if den > 0 else 0.0
+            kv[b, h] = (phk * ctx[:, None]).T @ v[b, h]
+            zz[b, h] = (phk * ctx[:, None]).sum(axis=0)
+    return out, kv, zz
+
+
+def cross_decode_step(kv, z, q_t, omega, geom):
+    """One decoder step of cross-attention against a fixed context summary
+    (README, "Encoder-decoder model and generation": the encoded source is
+    summarised once per layer): out_t = phi(q_t)^T kv / phi(q_t)^T z; the
+    summary is not changed. q_t: [B, H, d]; kv: [B, H, m, d]; z: [B, H, m]."""
+    kv, z, q_t = _f64(kv), _f64(z), _f64(q_t)
+    B, H, d = q_t.shape
+    out = np.zeros((B, H, d))
+    for b in range(B):
+        for h in range(H):
+            pq = feature_map(q_t[b, h], _head(omega, h), _head(geom, h))
+            den = pq @ z[b, h]
+            out[b, h] = (pq @ kv[b, h]) / den if den > 0 else 0.0
+    return out
 
 
 def exponent_range(x, omega, geom):
