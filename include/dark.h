@@ -42,7 +42,7 @@
 extern "C" {
 #endif
 
-#define DARK_ABI_VERSION 1
+#define DARK_ABI_VERSION 2
 
 typedef enum {
   DARK_OK = 0,
@@ -217,6 +217,54 @@ dark_status dark_state_init(const dark_projection* proj, dark_state* st, void* s
 dark_status dark_decode_step(const dark_projection* proj, dark_state* st, const void* q_t,
                              const void* k_t, const void* v_t, void* out_t,
                              const uint8_t* valid, int* dev_status, void* stream);
+
+/*
+ * Workspace bytes dark_cross_attention_fwd needs (0 for invalid arguments or
+ * DARK_CAUSAL). Same rules as dark_attention_workspace_bytes.
+ */
+size_t dark_cross_attention_workspace_bytes(const dark_projection* proj, int B, int H, int Lq,
+                                            int Lk, int flags);
+
+/*
+ * Cross-attention of Lq queries over an Lk-token context (README
+ * "Cross-attention": separate query and context masks, no causal option):
+ * out_i = phi(q_i)^T S / phi(q_i)^T z with S = Phi(K)^T V and z = Phi(K)^T 1
+ * over the valid context positions.
+ *   q            device, [B][H][Lq][d] of proj->dtype, strides q_strides
+ *                (elements; {b, h, l}; d stride 1; NULL = contiguous)
+ *   query_mask   device uint8 [B][Lq] or NULL; a masked query row (0) gets a
+ *                zero output (the pages leave the query mask's effect open:
+ *                this library's reading)
+ *   k, v         device, [B][H][Lk][d], strides kv_strides (NULL = contiguous)
+ *   context_mask device uint8 [B][Lk] (nonzero = valid context position) or NULL
+ *   out          device, [B][H][Lq][d], strides out_strides (NULL = contiguous)
+ *   flags        0 or DARK_STABILISE; DARK_CAUSAL returns DARK_ERR_INVALID_ARG
+ *   context_out  NULL, or a state that receives the context summary (S, z)
+ *                ("summarised once per layer" for decoding, see
+ *                dark_cross_decode_step); its generation is set
+ *   ws, ws_bytes workspace (dark_cross_attention_workspace_bytes)
+ * Errors as dark_attention_fwd.
+ */
+dark_status dark_cross_attention_fwd(const dark_projection* proj, const void* q,
+                                     const int64_t* q_strides, int Lq, const uint8_t* query_mask,
+                                     const void* k, const void* v, const int64_t* kv_strides,
+                                     int Lk, const uint8_t* context_mask, void* out,
+                                     const int64_t* out_strides, int B, int H, int flags,
+                                     dark_state* context_out, void* ws, size_t ws_bytes,
+                                     int* dev_status, void* stream);
+
+/*
+ * One decoder step of cross-attention against a context summary made by
+ * dark_cross_attention_fwd (README "Encoder-decoder model and generation":
+ * decoder cross-attention summarises the encoded source once per layer):
+ * out_t = phi(q_t)^T S / phi(q_t)^T z. The summary is read, never written.
+ *   q_t, out_t   device [B][H][d] of proj->dtype, contiguous
+ *   context      state of sizes (B, H, proj->m, proj->d)
+ * Returns DARK_ERR_STALE_STATE, enqueuing nothing, when context->generation !=
+ * proj->generation.
+ */
+dark_status dark_cross_decode_step(const dark_projection* proj, const dark_state* context,
+                                   const void* q_t, void* out_t, int* dev_status, void* stream);
 
 #ifdef __cplusplus
 }

@@ -42,12 +42,12 @@ Path choose_path(dark::FwdArgs& a) {
   return Path::Simt;
 }
 
-size_t ws_need(Path p, int B, int H, int L, int m, int r, int d, int flags) {
+size_t ws_need(Path p, int B, int H, int Lq, int Lk, int m, int r, int d, int flags) {
   switch (p) {
-    case Path::TcCausal: return dark::tc_causal_workspace_bytes(B, H, L, m, d);
-    case Path::TcWide: return dark::tc_wide_workspace_bytes(B, H, L, m, d, r);
-    case Path::TcNonCausal: return dark::tc_noncausal_workspace_bytes(B, H, L, m, d);
-    default: return dark::simt_workspace_bytes(B, H, L, m, d, flags);
+    case Path::TcCausal: return dark::tc_causal_workspace_bytes(B, H, Lq, m, d);
+    case Path::TcWide: return dark::tc_wide_workspace_bytes(B, H, Lq, m, d, r);
+    case Path::TcNonCausal: return dark::tc_noncausal_workspace_bytes(B, H, Lq, Lk, m, d);
+    default: return dark::simt_workspace_bytes(B, H, Lq, Lk, m, d, flags);
   }
 }
 
@@ -55,16 +55,19 @@ size_t ws_need(Path p, int B, int H, int L, int m, int r, int d, int flags) {
 
 namespace dark {
 
-dark_status fwd_prepare(const dark_projection* proj, const void* q, const void* k, const void* v,
-                        void* out, const int64_t* qkv_strides, const int64_t* out_strides, int B,
-                        int H, int L, const uint8_t* key_mask, int flags,
-                        const dark_state* state_out, int* dev_status, void* stream, FwdArgs* out_args) {
+dark_status fwd_prepare_general(const dark_projection* proj, const void* q,
+                                const int64_t* q_strides, int Lq, const uint8_t* query_mask,
+                                const void* k, const void* v, const int64_t* kv_strides, int Lk,
+                                const uint8_t* key_mask, void* out, const int64_t* out_strides,
+                                int B, int H, int flags, const dark_state* state_out,
+                                int* dev_status, void* stream, FwdArgs* out_args) {
   if (proj == nullptr || proj->w == nullptr || !aligned(proj->w, 16) || !dtype_ok(proj->dtype))
     return DARK_ERR_INVALID_ARG;
   if (proj->m < 1 || proj->r < 1 || proj->d < 1) return DARK_ERR_INVALID_ARG;
   if (!sizes_ok(proj->m, proj->r, proj->d)) return DARK_ERR_UNSUPPORTED;
   if (q == nullptr || k == nullptr || v == nullptr || out == nullptr) return DARK_ERR_INVALID_ARG;
-  if (B < 1 || H < 1 || L < 1) return DARK_ERR_INVALID_ARG;
+  if (B < 1 || H < 1 || Lq < 1 || Lk < 1) return DARK_ERR_INVALID_ARG;
+  if ((flags & DARK_CAUSAL) && Lq != Lk) return DARK_ERR_INVALID_ARG;
   if (!(proj->heads == 1 || proj->heads == H)) return DARK_ERR_INVALID_ARG;
   if (flags & ~(DARK_CAUSAL | DARK_STABILISE)) return DARK_ERR_INVALID_ARG;
   FwdArgs& a = *out_args;
@@ -80,16 +83,20 @@ dark_status fwd_prepare(const dark_projection* proj, const void* q, const void* 
   a.v = v;
   a.out = out;
   const int64_t d = proj->d;
-  const int64_t contig[3] = {(int64_t)H * L * d, (int64_t)L * d, d};
+  const int64_t cq[3] = {(int64_t)H * Lq * d, (int64_t)Lq * d, d};
+  const int64_t ck[3] = {(int64_t)H * Lk * d, (int64_t)Lk * d, d};
   for (int i = 0; i < 3; ++i) {
-    a.qs[i] = qkv_strides ? qkv_strides[i] : contig[i];
-    a.os[i] = out_strides ? out_strides[i] : contig[i];
-    if (a.qs[i] < 0 || a.os[i] < 0) return DARK_ERR_INVALID_ARG;
+    a.qs[i] = q_strides ? q_strides[i] : cq[i];
+    a.ks[i] = kv_strides ? kv_strides[i] : ck[i];
+    a.os[i] = out_strides ? out_strides[i] : cq[i];
+    if (a.qs[i] < 0 || a.ks[i] < 0 || a.os[i] < 0) return DARK_ERR_INVALID_ARG;
   }
   a.B = B;
   a.H = H;
-  a.L = L;
+  a.L = Lq;
+  a.Lk = Lk;
   a.mask = key_mask;
+  a.qmask = query_mask;
   a.flags = flags;
   if (state_out != nullptr) {
     if (state_out->kv == nullptr || state_out->z == nullptr || state_out->B != B ||
@@ -106,8 +113,18 @@ dark_status fwd_prepare(const dark_projection* proj, const void* q, const void* 
   return DARK_OK;
 }
 
+dark_status fwd_prepare(const dark_projection* proj, const void* q, const void* k, const void* v,
+                        void* out, const int64_t* qkv_strides, const int64_t* out_strides, int B,
+                        int H, int L, const uint8_t* key_mask, int flags,
+                        const dark_state* state_out, int* dev_status, void* stream,
+                        FwdArgs* out_args) {
+  return fwd_prepare_general(proj, q, qkv_strides, L, nullptr, k, v, qkv_strides, L, key_mask,
+                             out, out_strides, B, H, flags, state_out, dev_status, stream,
+                             out_args);
+}
+
 size_t fwd_workspace_need(const FwdArgs& a) {
-  return ws_need((Path)a.path, a.B, a.H, a.L, a.m, a.r, a.d, a.flags);
+  return ws_need((Path)a.path, a.B, a.H, a.L, a.Lk, a.m, a.r, a.d, a.flags);
 }
 
 dark_status fwd_launch(FwdArgs& a, void* ws, size_t ws_bytes, dark_state* state_out,
@@ -181,9 +198,9 @@ size_t dark_attention_workspace_bytes(const dark_projection* proj, int B, int H,
                                       int flags) {
   if (!proj_ok(proj) || B < 1 || H < 1 || L < 1) return 0;
   const int m = proj->m, d = proj->d;
-  size_t need = dark::simt_workspace_bytes(B, H, L, m, d, flags);
+  size_t need = dark::simt_workspace_bytes(B, H, L, L, m, d, flags);
   const size_t tc = (flags & DARK_CAUSAL) ? dark::tc_causal_workspace_bytes(B, H, L, m, d)
-                                          : dark::tc_noncausal_workspace_bytes(B, H, L, m, d);
+                                          : dark::tc_noncausal_workspace_bytes(B, H, L, L, m, d);
   const size_t wide =
       (flags & DARK_CAUSAL) ? dark::tc_wide_workspace_bytes(B, H, L, m, d, proj->r) : 0;
   if (need < tc) need = tc;
@@ -202,6 +219,66 @@ dark_status dark_attention_fwd(const dark_projection* proj, const void* q, const
   if (st != DARK_OK) return st;
   if (ws_bytes < dark::fwd_workspace_need(a)) return DARK_ERR_INVALID_ARG;
   return dark::fwd_launch(a, ws, ws_bytes, state_out, proj->generation);
+}
+
+size_t dark_cross_attention_workspace_bytes(const dark_projection* proj, int B, int H, int Lq,
+                                            int Lk, int flags) {
+  if (!proj_ok(proj) || B < 1 || H < 1 || Lq < 1 || Lk < 1 || (flags & DARK_CAUSAL)) return 0;
+  const size_t simt = dark::simt_workspace_bytes(B, H, Lq, Lk, proj->m, proj->d, flags);
+  const size_t tc = dark::tc_noncausal_workspace_bytes(B, H, Lq, Lk, proj->m, proj->d);
+  return simt > tc ? simt : tc;
+}
+
+dark_status dark_cross_attention_fwd(const dark_projection* proj, const void* q,
+                                     const int64_t* q_strides, int Lq, const uint8_t* query_mask,
+                                     const void* k, const void* v, const int64_t* kv_strides,
+                                     int Lk, const uint8_t* context_mask, void* out,
+                                     const int64_t* out_strides, int B, int H, int flags,
+                                     dark_state* context_out, void* ws, size_t ws_bytes,
+                                     int* dev_status, void* stream) {
+  if (ws == nullptr || !aligned(ws, 256)) return DARK_ERR_INVALID_ARG;
+  if (flags & DARK_CAUSAL) return DARK_ERR_INVALID_ARG;
+  dark::FwdArgs a;
+  const dark_status st = dark::fwd_prepare_general(
+      proj, q, q_strides, Lq, query_mask, k, v, kv_strides, Lk, context_mask, out, out_strides,
+      B, H, flags, context_out, dev_status, stream, &a);
+  if (st != DARK_OK) return st;
+  if (ws_bytes < dark::fwd_workspace_need(a)) return DARK_ERR_INVALID_ARG;
+  return dark::fwd_launch(a, ws, ws_bytes, context_out, proj->generation);
+}
+
+dark_status dark_cross_decode_step(const dark_projection* proj, const dark_state* context,
+                                   const void* q_t, void* out_t, int* dev_status, void* stream) {
+  if (proj == nullptr || proj->w == nullptr || !aligned(proj->w, 16) || !dtype_ok(proj->dtype) ||
+      context == nullptr)
+    return DARK_ERR_INVALID_ARG;
+  if (!sizes_ok(proj->m, proj->r, proj->d)) return DARK_ERR_UNSUPPORTED;
+  if (context->kv == nullptr || context->z == nullptr || q_t == nullptr || out_t == nullptr)
+    return DARK_ERR_INVALID_ARG;
+  if (context->B < 1 || context->H < 1 || context->m != proj->m || context->d != proj->d)
+    return DARK_ERR_INVALID_ARG;
+  if (!(proj->heads == 1 || proj->heads == context->H)) return DARK_ERR_INVALID_ARG;
+  if (!aligned(context->kv, 16)) return DARK_ERR_INVALID_ARG;
+  if (context->generation != proj->generation) return DARK_ERR_STALE_STATE;
+  dark::DecodeArgs a;
+  memset(&a, 0, sizeof(a));
+  a.heads_w = proj->heads;
+  a.m = proj->m;
+  a.r = proj->r;
+  a.d = proj->d;
+  a.dtype = proj->dtype;
+  a.w = proj->w;
+  a.kv = context->kv;
+  a.z = context->z;
+  a.shift = context->shift;
+  a.B = context->B;
+  a.H = context->H;
+  a.q = q_t;
+  a.out = out_t;
+  a.update = 0;
+  a.dev_status = dev_status;
+  a.stream = (cudaStream_t)stream;
+  return from_cuda(dark::launch_decode(a));
 }
 
 dark_status dark_state_init(const dark_projection* proj, dark_state* st, void* stream) {
@@ -249,6 +326,7 @@ dark_status dark_decode_step(const dark_projection* proj, dark_state* st, const 
   a.v = v_t;
   a.out = out_t;
   a.valid = valid;
+  a.update = 1;
   a.dev_status = dev_status;
   a.stream = (cudaStream_t)stream;
   return from_cuda(dark::launch_decode(a));

@@ -242,7 +242,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(
     const typename WeightOf<T>::type* __restrict__ w, int heads_w, int m, int r, int d,
     float* __restrict__ kv, float* __restrict__ z, const float* __restrict__ shift, int H,
     const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v, T* __restrict__ out,
-    const uint8_t* __restrict__ valid, int* dev_status, int stage_w) {
+    const uint8_t* __restrict__ valid, int* dev_status, int stage_w, int update) {
   using TW = typename WeightOf<T>::type;
   extern __shared__ __align__(16) float sm[];
   const int tpr = d / 4;                  // threads per state row (one float4 each)
@@ -278,10 +278,11 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(
 
   // The step's tokens first (they gate the feature GEMV), then the state rows
   // of the first pass, whose HBM latency overlaps the feature computation.
+  // (update == 0: cross-attention against a fixed context; k and v are unused)
   const bool has_c = tid < d;             // d <= kThreads: one element per thread
   const T q_e = has_c ? q[(size_t)bh * d + tid] : T(0.f);
-  const T k_e = has_c ? k[(size_t)bh * d + tid] : T(0.f);
-  const T v_e = has_c ? v[(size_t)bh * d + tid] : T(0.f);
+  const T k_e = has_c && update ? k[(size_t)bh * d + tid] : T(0.f);
+  const T v_e = has_c && update ? v[(size_t)bh * d + tid] : T(0.f);
   float4 s[kBatchRows];
   if (rows_active) {
 #pragma unroll
@@ -359,7 +360,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(
     ks = scratch[0];
     qs = scratch[1];
   }
-  const bool ok = valid == nullptr || valid[b] != 0;
+  const bool ok = update && (valid == nullptr || valid[b] != 0);
   for (int j = tid; j < m; j += kThreads) {
     pk[j] = ok ? exp2f(pk[j] - ks) : 0.f;
     pq[j] = exp2f(pq[j] - qs);
@@ -385,7 +386,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(
           const float fk = pk[j], fq = pq[j];
           s[u].x = fmaf(fk, vv.x, s[u].x); s[u].y = fmaf(fk, vv.y, s[u].y);
           s[u].z = fmaf(fk, vv.z, s[u].z); s[u].w = fmaf(fk, vv.w, s[u].w);
-          __stcs(base + (size_t)j * stride, s[u]);
+          if (update) __stcs(base + (size_t)j * stride, s[u]);
           num.x = fmaf(fq, s[u].x, num.x); num.y = fmaf(fq, s[u].y, num.y);
           num.z = fmaf(fq, s[u].z, num.z); num.w = fmaf(fq, s[u].w, num.w);
         }
@@ -400,7 +401,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(
     const int j = tid + u * kThreads;
     if (j < m) {
       const float zj = zpre[u] + pk[j];
-      __stcs(z + (size_t)bh * m + j, zj);
+      if (update) __stcs(z + (size_t)bh * m + j, zj);
       den = fmaf(pq[j], zj, den);
     }
   }
@@ -438,14 +439,15 @@ cudaError_t launch_decode(const DecodeArgs& a) {
     decode_kernel<__nv_bfloat16><<<a.B * a.H, kThreads, smem, a.stream>>>(
         (const __half*)a.w, a.heads_w, a.m, a.r, a.d, a.kv, a.z, a.shift, a.H,
         (const __nv_bfloat16*)a.q, (const __nv_bfloat16*)a.k, (const __nv_bfloat16*)a.v,
-        (__nv_bfloat16*)a.out, a.valid, a.dev_status, stage_w);
+        (__nv_bfloat16*)a.out, a.valid, a.dev_status, stage_w, a.update);
   } else {
     static int done[64];
     err = set_smem_limit_once((const void*)decode_kernel<float>, kSmemOptIn, done);
     if (err != cudaSuccess) return err;
     decode_kernel<float><<<a.B * a.H, kThreads, smem, a.stream>>>(
         (const float*)a.w, a.heads_w, a.m, a.r, a.d, a.kv, a.z, a.shift, a.H, (const float*)a.q,
-        (const float*)a.k, (const float*)a.v, (float*)a.out, a.valid, a.dev_status, stage_w);
+        (const float*)a.k, (const float*)a.v, (float*)a.out, a.valid, a.dev_status, stage_w,
+        a.update);
   }
   return cudaGetLastError();
 }

@@ -18,9 +18,11 @@ struct FwdArgs {
   const void* w;                  // projection buffer [heads_w][m + r][d]
   const void *q, *k, *v;
   void* out;
-  int64_t qs[3], os[3];           // element strides {b, h, l} of q/k/v and of out
-  int B, H, L;
-  const uint8_t* mask;            // [B][L] or null
+  int64_t qs[3], ks[3], os[3];    // element strides {b, h, l} of q, of k/v, of out
+  int B, H, L;                    // L: queries (and keys, for self-attention)
+  int Lk;                         // keys/values: L, or the context length
+  const uint8_t* mask;            // keys [B][Lk] or null
+  const uint8_t* qmask;           // queries [B][L] or null (cross-attention)
   int flags;
   float *st_kv, *st_z, *st_shift; // state_out arrays or null
   void* ws;
@@ -42,6 +44,15 @@ constexpr size_t kWsHeader = 256;
 
 // The forward call in three steps: validate and choose the kernel path (no
 // device work), report the workspace that path needs, enqueue it.
+// Lq queries (strides q_strides, optional query mask) over Lk keys/values
+// (strides kv_strides, optional key mask); self-attention passes Lq = Lk and the
+// same strides for both.
+dark_status fwd_prepare_general(const dark_projection* proj, const void* q,
+                                const int64_t* q_strides, int Lq, const uint8_t* query_mask,
+                                const void* k, const void* v, const int64_t* kv_strides, int Lk,
+                                const uint8_t* key_mask, void* out, const int64_t* out_strides,
+                                int B, int H, int flags, const dark_state* state_out,
+                                int* dev_status, void* stream, FwdArgs* a);
 dark_status fwd_prepare(const dark_projection* proj, const void* q, const void* k, const void* v,
                         void* out, const int64_t* qkv_strides, const int64_t* out_strides, int B,
                         int H, int L, const uint8_t* key_mask, int flags,
@@ -56,7 +67,7 @@ cudaError_t launch_projection(const float* omega, int heads_omega, const float* 
                               dark_dtype dtype, void* w, cudaStream_t stream);
 
 // Generic SIMT forward: any strides, any supported sizes, fp32 or bf16 I/O.
-size_t simt_workspace_bytes(int B, int H, int L, int m, int d, int flags);
+size_t simt_workspace_bytes(int B, int H, int Lq, int Lk, int m, int d, int flags);
 cudaError_t simt_forward(const FwdArgs& a);
 
 // Tensor-core forward paths (tcgen05/TMEM/TMA). `*_supported` says whether the
@@ -75,7 +86,7 @@ bool tc_noncausal_supported(FwdArgs& a);
 // Per-range key states Phi(K)^T [V | 1] as fp32 [B*H*nsplit][65][m] (tcgen05).
 cudaError_t tc_launch_key_states(const FwdArgs& a, const CUtensorMap& tw, const CUtensorMap& tk,
                                  const CUtensorMap& tv, int ntiles, int nsplit, float* partials);
-size_t tc_noncausal_workspace_bytes(int B, int H, int L, int m, int d);
+size_t tc_noncausal_workspace_bytes(int B, int H, int Lq, int Lk, int m, int d);
 cudaError_t tc_noncausal_forward(const FwdArgs& a);
 
 // Wide heads (d = 128..256, m up to 512), causal: features/scores launch, then
@@ -94,6 +105,7 @@ struct DecodeArgs {
   const void *q, *k, *v;
   void* out;
   const uint8_t* valid;
+  int update;                     // 1: add (k, v) to the state first; 0: read it only
   int* dev_status;
   cudaStream_t stream;
 };

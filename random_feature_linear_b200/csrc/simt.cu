@@ -1,4 +1,5 @@
-// Generic SIMT forward pass of PRF attention.
+// Generic SIMT forward pass of PRF attention (self-attention, and cross-attention
+// of Lq queries over Lk context keys).
 //
 // This is the fp32-I/O path (fp32 FFMA throughout, so no TF32 rounding enters
 // the exponent) and the path for any size, stride or alignment that the
@@ -30,24 +31,25 @@ struct SimtLayout {
   size_t off_ck, off_phiq, off_phik, off_s, total;
 };
 
-SimtLayout simt_layout(int B, int H, int L, int m, int d, int flags) {
+// Lq queries attend over Lk keys (Lq = Lk for self-attention; causal only then).
+SimtLayout simt_layout(int B, int H, int Lq, int Lk, int m, int d, int flags) {
   SimtLayout s;
   const int bh = B * H;
   if (flags & DARK_CAUSAL) {
     s.chunk_len = kCausalChunk;
-    s.nc = (L + kCausalChunk - 1) / kCausalChunk;
+    s.nc = (Lk + kCausalChunk - 1) / kCausalChunk;
   } else {
     int ns = (2 * kSms + bh - 1) / bh;
-    const int max_ns = (L + 63) / 64;
+    const int max_ns = (Lk + 63) / 64;
     if (ns > max_ns) ns = max_ns;
     if (ns < 1) ns = 1;
-    s.chunk_len = (L + ns - 1) / ns;
-    s.nc = (L + s.chunk_len - 1) / s.chunk_len;
+    s.chunk_len = (Lk + ns - 1) / ns;
+    s.nc = (Lk + s.chunk_len - 1) / s.chunk_len;
   }
   s.off_ck = kWsHeader;
   s.off_phiq = align_up(s.off_ck + sizeof(int) * (size_t)bh, 256);
-  s.off_phik = align_up(s.off_phiq + sizeof(float) * (size_t)bh * L * m, 256);
-  s.off_s = align_up(s.off_phik + sizeof(float) * (size_t)bh * L * m, 256);
+  s.off_phik = align_up(s.off_phiq + sizeof(float) * (size_t)bh * Lq * m, 256);
+  s.off_s = align_up(s.off_phik + sizeof(float) * (size_t)bh * Lk * m, 256);
   s.total = align_up(s.off_s + sizeof(float) * (size_t)bh * s.nc * m * (d + 1), 256);
   return s;
 }
@@ -59,8 +61,9 @@ __global__ void init_ck_kernel(int* ck, int n) {
 
 template <typename T>
 __global__ void __launch_bounds__(256) features_kernel(
-    const T* __restrict__ xq, const T* __restrict__ xk, int64_t sb, int64_t sh, int64_t sl,
-    const typename WeightOf<T>::type* __restrict__ w, int heads_w, int m, int r, int d, int H, int L,
+    const T* __restrict__ xq, int64_t qb, int64_t qh, int64_t ql, int Lq,
+    const T* __restrict__ xk, int64_t kb, int64_t kh, int64_t kl, int Lk,
+    const typename WeightOf<T>::type* __restrict__ w, int heads_w, int m, int r, int d, int H,
     const uint8_t* __restrict__ mask, int stabilise, float* __restrict__ phiq,
     float* __restrict__ phik, int* __restrict__ ck) {
   extern __shared__ float sm[];
@@ -70,7 +73,10 @@ __global__ void __launch_bounds__(256) features_kernel(
   const int side = blockIdx.z;       // 0: queries, 1: keys
   const int bh = blockIdx.y, b = bh / H, h = bh % H;
   const int t0 = blockIdx.x * kTF;
+  const int L = side ? Lk : Lq;
+  if (t0 >= L) return;               // the grid covers the longer side
   const T* x = side ? xk : xq;
+  const int64_t sb = side ? kb : qb, sh = side ? kh : qh, sl = side ? kl : ql;
   const int ncols = side ? m + r : m;
   const int ld = m + r;
   const auto* wh = w + (size_t)(heads_w == 1 ? 0 : h) * (m + r) * d;
@@ -243,7 +249,8 @@ __global__ void __launch_bounds__(256) out_kernel(
     const float* __restrict__ phiq, const float* __restrict__ phik,
     const float* __restrict__ chunk_s, const T* __restrict__ v, int64_t vb, int64_t vh,
     int64_t vl, T* __restrict__ out, int64_t ob, int64_t oh, int64_t ol, int m, int d, int H,
-    int L, int causal, int chunk_len, int nc, int* dev_status) {
+    int L, int causal, int chunk_len, int nc, const uint8_t* __restrict__ qmask,
+    int* dev_status) {
   extern __shared__ float sm[];
   const int dd = d + 1;
   const int ET = (dd + 63) / 64;
@@ -369,7 +376,8 @@ __global__ void __launch_bounds__(256) out_kernel(
   for (int i = 0; i < 4; ++i) {
     const int row = ty * 4 + i, t = q0 + row;
     if (t >= L) continue;
-    const float dn = den[row];
+    // a masked query row (cross-attention) outputs 0
+    const float dn = (qmask == nullptr || qmask[(size_t)b * L + t] != 0) ? den[row] : 0.f;
 #pragma unroll
     for (int et = 0; et < 5; ++et) {
       if (et < ET) {
@@ -389,7 +397,7 @@ __global__ void __launch_bounds__(256) out_kernel(
 
 template <typename T>
 cudaError_t simt_forward_t(const FwdArgs& a) {
-  const SimtLayout s = simt_layout(a.B, a.H, a.L, a.m, a.d, a.flags);
+  const SimtLayout s = simt_layout(a.B, a.H, a.L, a.Lk, a.m, a.d, a.flags);
   char* ws = (char*)a.ws;
   int* ck = (int*)(ws + s.off_ck);
   float* phiq = (float*)(ws + s.off_phiq);
@@ -404,16 +412,17 @@ cudaError_t simt_forward_t(const FwdArgs& a) {
   const size_t fsm = sizeof(float) * kTF * (a.d + a.m + a.r);
   err = cudaFuncSetAttribute(features_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)fsm);
   if (err != cudaSuccess) return err;
-  features_kernel<T><<<dim3((a.L + kTF - 1) / kTF, bh, 2), 256, fsm, a.stream>>>(
-      (const T*)a.q, (const T*)a.k, a.qs[0], a.qs[1], a.qs[2],
-      (const typename WeightOf<T>::type*)a.w, a.heads_w, a.m,
-      a.r, a.d, a.H, a.L, a.mask, stab, phiq, phik, ck);
+  const int lmax = a.L > a.Lk ? a.L : a.Lk;
+  features_kernel<T><<<dim3((lmax + kTF - 1) / kTF, bh, 2), 256, fsm, a.stream>>>(
+      (const T*)a.q, a.qs[0], a.qs[1], a.qs[2], a.L, (const T*)a.k, a.ks[0], a.ks[1], a.ks[2],
+      a.Lk, (const typename WeightOf<T>::type*)a.w, a.heads_w, a.m, a.r, a.d, a.H, a.mask, stab,
+      phiq, phik, ck);
   if (stab) {
-    const size_t n = (size_t)bh * a.L * a.m;
-    expshift_kernel<<<(unsigned)((n + 255) / 256), 256, 0, a.stream>>>(phik, ck, a.L, a.m, n);
+    const size_t n = (size_t)bh * a.Lk * a.m;
+    expshift_kernel<<<(unsigned)((n + 255) / 256), 256, 0, a.stream>>>(phik, ck, a.Lk, a.m, n);
   }
   chunk_state_kernel<T><<<dim3(s.nc, bh), 256, 0, a.stream>>>(
-      phik, (const T*)a.v, a.qs[0], a.qs[1], a.qs[2], a.m, a.d, a.H, a.L, s.chunk_len, s.nc, cs);
+      phik, (const T*)a.v, a.ks[0], a.ks[1], a.ks[2], a.m, a.d, a.H, a.Lk, s.chunk_len, s.nc, cs);
   scan_kernel<<<dim3((a.m * (a.d + 1) + 255) / 256, bh), 256, 0, a.stream>>>(
       cs, a.m, a.d, s.nc, causal, a.st_kv, a.st_z, stab ? a.st_shift : nullptr, ck);
   const int ddp = ((a.d + 1 + 63) / 64) * 64;
@@ -421,15 +430,15 @@ cudaError_t simt_forward_t(const FwdArgs& a) {
   err = cudaFuncSetAttribute(out_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)osm);
   if (err != cudaSuccess) return err;
   out_kernel<T><<<dim3((a.L + 63) / 64, bh), 256, osm, a.stream>>>(
-      phiq, phik, cs, (const T*)a.v, a.qs[0], a.qs[1], a.qs[2], (T*)a.out, a.os[0], a.os[1],
-      a.os[2], a.m, a.d, a.H, a.L, causal, s.chunk_len, s.nc, a.dev_status);
+      phiq, phik, cs, (const T*)a.v, a.ks[0], a.ks[1], a.ks[2], (T*)a.out, a.os[0], a.os[1],
+      a.os[2], a.m, a.d, a.H, a.L, causal, s.chunk_len, s.nc, a.qmask, a.dev_status);
   return cudaGetLastError();
 }
 
 }  // namespace
 
-size_t simt_workspace_bytes(int B, int H, int L, int m, int d, int flags) {
-  return simt_layout(B, H, L, m, d, flags).total;
+size_t simt_workspace_bytes(int B, int H, int Lq, int Lk, int m, int d, int flags) {
+  return simt_layout(B, H, Lq, Lk, m, d, flags).total;
 }
 
 cudaError_t simt_forward(const FwdArgs& a) {

@@ -40,17 +40,20 @@ bool tc_make_maps(FwdArgs& a) {
   if (a.dtype != DARK_BF16 || a.d != 64) return false;
   if (!al16(a.q) || !al16(a.k) || !al16(a.v) || !al16(a.out) || !al16(a.w)) return false;
   for (int i = 0; i < 3; ++i)
-    if (a.qs[i] % 8 != 0 || a.os[i] % 8 != 0) return false;
+    if (a.qs[i] % 8 != 0 || a.ks[i] % 8 != 0 || a.os[i] % 8 != 0) return false;
   const uint64_t wd[2] = {(uint64_t)a.d, (uint64_t)a.heads_w * (a.m + a.r)};
   const uint64_t wsd[1] = {(uint64_t)a.d * 2};
   const uint32_t wb[2] = {64, 16};
-  const uint64_t xd[4] = {(uint64_t)a.d, (uint64_t)a.L, (uint64_t)a.H, (uint64_t)a.B};
-  const uint64_t xs[3] = {(uint64_t)a.qs[2] * 2, (uint64_t)a.qs[1] * 2, (uint64_t)a.qs[0] * 2};
+  // queries: L tokens with strides qs; keys and values: Lk tokens with strides ks
+  const uint64_t qd[4] = {(uint64_t)a.d, (uint64_t)a.L, (uint64_t)a.H, (uint64_t)a.B};
+  const uint64_t qst[3] = {(uint64_t)a.qs[2] * 2, (uint64_t)a.qs[1] * 2, (uint64_t)a.qs[0] * 2};
+  const uint64_t kd[4] = {(uint64_t)a.d, (uint64_t)a.Lk, (uint64_t)a.H, (uint64_t)a.B};
+  const uint64_t kst[3] = {(uint64_t)a.ks[2] * 2, (uint64_t)a.ks[1] * 2, (uint64_t)a.ks[0] * 2};
   const uint32_t xb[4] = {64, 128, 1, 1};
   a.maps_ready = encode_tmap(&a.tm_w, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, a.w, wd, wsd, wb) &&
-                 encode_tmap(&a.tm_q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, a.q, xd, xs, xb) &&
-                 encode_tmap(&a.tm_k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, a.k, xd, xs, xb) &&
-                 encode_tmap(&a.tm_v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, a.v, xd, xs, xb);
+                 encode_tmap(&a.tm_q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, a.q, qd, qst, xb) &&
+                 encode_tmap(&a.tm_k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, a.k, kd, kst, xb) &&
+                 encode_tmap(&a.tm_v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, a.v, kd, kst, xb);
   return a.maps_ready;
 }
 

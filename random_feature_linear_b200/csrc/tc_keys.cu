@@ -201,7 +201,7 @@ cudaError_t launch_keys_t(const FwdArgs& a, const CUtensorMap& tw, const CUtenso
   kp.mask = a.mask;
   kp.B = a.B;
   kp.H = a.H;
-  kp.L = a.L;
+  kp.L = a.Lk;                    // keys (= L for self-attention)
   kp.ntiles = ntiles;
   kp.nsplit = nsplit;
   kp.heads_w = a.heads_w;

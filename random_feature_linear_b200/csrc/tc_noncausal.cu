@@ -75,7 +75,8 @@ __global__ void reduce_kernel(const float* __restrict__ partials, int nsplit, in
 struct QueryParams {
   __nv_bfloat16* out;
   int64_t ob, oh, ol;
-  int B, H, L, ntiles, heads_w, total_tiles;
+  int B, H, L, ntiles, heads_w, total_tiles;   // L, ntiles: queries
+  const uint8_t* qmask;         // [B][L] or null: a masked query row outputs 0
   const uint8_t* images;
   int* dev_status;
 };
@@ -207,7 +208,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int i = 0; i < 32; ++i) v[i] += vl[i];
       const int tok = t * kT + row;
       if (tok < p.L) {
-        const float inv = den > 0.f ? 1.f / den : 0.f;
+        const bool live = p.qmask == nullptr || p.qmask[(size_t)b * p.L + tok] != 0;
+        const float inv = live && den > 0.f ? 1.f / den : 0.f;
         uint32_t w[16];
         bool bad = !isfinite(den);
 #pragma unroll
@@ -237,14 +239,17 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 struct Layout {
-  int ntiles, nsplit;
+  int ntiles, nsplit;           // key tiles per head and key ranges per head
+  int qtiles;                   // query tiles per head
   size_t off_part, off_img, total;
 };
 
-Layout layout(int B, int H, int L, int m) {
+// Lq queries over Lk keys (equal for self-attention).
+Layout layout(int B, int H, int Lq, int Lk, int m) {
   Layout s;
   const int bh = B * H;
-  s.ntiles = (L + kT - 1) / kT;
+  s.ntiles = (Lk + kT - 1) / kT;
+  s.qtiles = (Lq + kT - 1) / kT;
   s.nsplit = kSms / bh;
   if (s.nsplit < 1) s.nsplit = 1;
   if (s.nsplit > s.ntiles) s.nsplit = s.ntiles;
@@ -259,7 +264,7 @@ Layout layout(int B, int H, int L, int m) {
 template <int M_, int R_>
 cudaError_t launch(const FwdArgs& a, const CUtensorMap& tw, const CUtensorMap& tq,
                    const CUtensorMap& tk, const CUtensorMap& tv) {
-  const Layout s = layout(a.B, a.H, a.L, a.m);
+  const Layout s = layout(a.B, a.H, a.L, a.Lk, a.m);
   char* ws = (char*)a.ws;
   float* partials = (float*)(ws + s.off_part);
   uint8_t* images = (uint8_t*)(ws + s.off_img);
@@ -278,9 +283,10 @@ cudaError_t launch(const FwdArgs& a, const CUtensorMap& tw, const CUtensorMap& t
   qp.B = a.B;
   qp.H = a.H;
   qp.L = a.L;
-  qp.ntiles = s.ntiles;
+  qp.ntiles = s.qtiles;
   qp.heads_w = a.heads_w;
-  qp.total_tiles = bh * s.ntiles;
+  qp.total_tiles = bh * s.qtiles;
+  qp.qmask = a.qmask;
   qp.images = images;
   qp.dev_status = a.dev_status;
   using QG = QueryCfg<M_, R_>;
@@ -300,9 +306,9 @@ bool tc_noncausal_supported(FwdArgs& a) {
   return tc_make_maps(a);
 }
 
-size_t tc_noncausal_workspace_bytes(int B, int H, int L, int m, int d) {
+size_t tc_noncausal_workspace_bytes(int B, int H, int Lq, int Lk, int m, int d) {
   if (d != kD || !(m == 128 || m == 256)) return 0;
-  return layout(B, H, L, m).total;
+  return layout(B, H, Lq, Lk, m).total;
 }
 
 cudaError_t tc_noncausal_forward(const FwdArgs& a) {

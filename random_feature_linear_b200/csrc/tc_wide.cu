@@ -760,7 +760,7 @@ bool make_wide_maps(FwdArgs& a) {
   auto al16 = [](const void* p) { return ((uintptr_t)p & 15) == 0; };
   if (!al16(a.q) || !al16(a.k) || !al16(a.v) || !al16(a.out) || !al16(a.w)) return false;
   for (int i = 0; i < 3; ++i)
-    if (a.qs[i] % 8 != 0 || a.os[i] % 8 != 0) return false;
+    if (a.qs[i] % 8 != 0 || a.ks[i] != a.qs[i] || a.os[i] % 8 != 0) return false;
   const uint64_t wd[2] = {(uint64_t)a.d, (uint64_t)a.heads_w * (a.m + a.r)};
   const uint64_t wsd[1] = {(uint64_t)a.d * 2};
   const uint32_t wb[2] = {64, 64};

@@ -29,7 +29,8 @@ WS_HEADER_BYTES = 256
 EXPORTS = ("dark_abi_version", "dark_status_string", "dark_projection_bytes",
            "dark_make_projection", "dark_attention_workspace_bytes", "dark_attention_fwd",
            "dark_state_init", "dark_decode_step", "dark_noalloc_scratch_bytes",
-           "dark_attention_fwd_noalloc")
+           "dark_attention_fwd_noalloc", "dark_cross_attention_workspace_bytes",
+           "dark_cross_attention_fwd", "dark_cross_decode_step")
 
 
 class dark_projection(ctypes.Structure):
@@ -70,6 +71,15 @@ _lib.dark_state_init.argtypes = [_P(dark_projection), _P(dark_state), _vp]
 _lib.dark_decode_step.restype = _i
 _lib.dark_decode_step.argtypes = [_P(dark_projection), _P(dark_state), _vp, _vp, _vp, _vp, _vp,
                                   _vp, _vp]
+_lib.dark_cross_attention_workspace_bytes.restype = _sz
+_lib.dark_cross_attention_workspace_bytes.argtypes = [_P(dark_projection), _i, _i, _i, _i, _i]
+_lib.dark_cross_attention_fwd.restype = _i
+_lib.dark_cross_attention_fwd.argtypes = [_P(dark_projection), _vp, _P(ctypes.c_int64), _i, _vp,
+                                          _vp, _vp, _P(ctypes.c_int64), _i, _vp, _vp,
+                                          _P(ctypes.c_int64), _i, _i, _i, _P(dark_state), _vp,
+                                          _sz, _vp, _vp]
+_lib.dark_cross_decode_step.restype = _i
+_lib.dark_cross_decode_step.argtypes = [_P(dark_projection), _P(dark_state), _vp, _vp, _vp, _vp]
 
 
 class DarkError(RuntimeError):
@@ -188,6 +198,40 @@ def dark_decode_step(proj: dark_projection, st: dark_state, q_t, k_t, v_t, out_t
     _check(_lib.dark_decode_step(ctypes.byref(proj), ctypes.byref(st), _ptr(q_t), _ptr(k_t),
                                  _ptr(v_t), _ptr(out_t), _ptr(valid), _ptr(dev_status),
                                  _stream(stream)))
+
+
+def dark_cross_attention_workspace_bytes(proj: dark_projection, B: int, H: int, Lq: int, Lk: int,
+                                         flags: int) -> int:
+    return _lib.dark_cross_attention_workspace_bytes(ctypes.byref(proj), B, H, Lq, Lk, flags)
+
+
+def dark_cross_attention_fwd(proj: dark_projection, q, k, v, out, B: int, H: int, Lq: int, Lk: int,
+                             query_mask=None, context_mask=None, flags: int = 0,
+                             context_out: dark_state | None = None, ws=None, dev_status=None,
+                             stream=None, q_strides=None, kv_strides=None,
+                             out_strides=None) -> None:
+    """q/out viewed as [B][H][Lq][d], k/v as [B][H][Lk][d] with the given element
+    strides ({b, h, l}; None = contiguous). ws: a zero-initialised uint8 tensor."""
+    def strides(s):
+        return None if s is None else (ctypes.c_int64 * 3)(*s)
+    _check(_lib.dark_cross_attention_fwd(
+        ctypes.byref(proj), _ptr(q), strides(q_strides), Lq, _ptr(query_mask), _ptr(k), _ptr(v),
+        strides(kv_strides), Lk, _ptr(context_mask), _ptr(out), strides(out_strides), B, H, flags,
+        None if context_out is None else ctypes.byref(context_out), _ptr(ws),
+        0 if ws is None else ws.numel() * ws.element_size(), _ptr(dev_status), _stream(stream)))
+
+
+def dark_cross_decode_step(proj: dark_projection, context: dark_state, q_t, out_t,
+                           dev_status=None, stream=None) -> None:
+    _check(_lib.dark_cross_decode_step(ctypes.byref(proj), ctypes.byref(context), _ptr(q_t),
+                                       _ptr(out_t), _ptr(dev_status), _stream(stream)))
+
+
+def alloc_cross_workspace(proj: dark_projection, B: int, H: int, Lq: int, Lk: int, flags: int,
+                          device):
+    """A zero-filled workspace of the size dark_cross_attention_workspace_bytes asks for."""
+    n = dark_cross_attention_workspace_bytes(proj, B, H, Lq, Lk, flags)
+    return torch.zeros(max(n, WS_HEADER_BYTES), dtype=torch.uint8, device=device)
 
 
 def alloc_workspace(proj: dark_projection, B: int, H: int, L: int, flags: int, device):

@@ -34,7 +34,8 @@ def test_every_declared_symbol_is_exported(D):
 
 
 def test_version_and_status_strings(D):
-    assert D.dark_abi_version() == 1
+    hdr = open(os.path.join(ROOT, "include", "dark.h")).read()
+    assert D.dark_abi_version() == int(re.search(r"#define DARK_ABI_VERSION (\d+)", hdr).group(1))
     for s in range(7):
         assert D.dark_status_string(s).startswith("DARK_")
     assert "unknown" in D.dark_status_string(99)
@@ -114,3 +115,37 @@ def test_workspace_query(D):
     n2 = D.dark_attention_workspace_bytes(p, 2, 8, 4096, D.DARK_CAUSAL)
     assert n1 >= 256 and n2 > n1
     assert D.dark_attention_workspace_bytes(p, 0, 8, 2048, 0) == 0
+
+
+def test_cross_attention_rejects_bad_arguments(D):
+    lib = D._lib
+    f = 0x10000
+    p = _fake_proj(D)
+
+    def call(q=f, Lq=16, k=f, v=f, Lk=40, o=f, B=2, H=1, flags=0, ws=f, wsb=1 << 30, ctx=None):
+        return lib.dark_cross_attention_fwd(ctypes.byref(p), q, None, Lq, None, k, v, None, Lk,
+                                            None, o, None, B, H, flags, ctx, ws, wsb, None, None)
+
+    assert call(flags=D.DARK_CAUSAL) == 1            # no causal cross-attention
+    assert call(Lq=0) == 1 and call(Lk=0) == 1 and call(B=0) == 1
+    assert call(q=None) == 1 and call(k=None) == 1 and call(o=None) == 1
+    assert call(ws=None) == 1 and call(ws=f + 8) == 1
+    assert call(flags=8) == 1
+    st = D.dark_state(f, f, None, 2, 1, 64, 32, 0)      # d mismatch
+    assert call(ctx=ctypes.byref(st)) == 1
+    # workspace: none for causal, some for valid sizes, growing with the context
+    assert D.dark_cross_attention_workspace_bytes(p, 2, 1, 16, 40, D.DARK_CAUSAL) == 0
+    small = D.dark_cross_attention_workspace_bytes(p, 2, 1, 16, 40, 0)
+    big = D.dark_cross_attention_workspace_bytes(p, 2, 1, 16, 4000, 0)
+    assert 0 < small < big
+
+
+def test_cross_decode_rejects_stale_and_bad_arguments(D):
+    lib = D._lib
+    f = 0x10000
+    p = _fake_proj(D)
+    st = D.dark_state(f, f, None, 2, 1, 64, 64, p.generation)
+    assert lib.dark_cross_decode_step(ctypes.byref(p), None, f, f, None, None) == 1
+    assert lib.dark_cross_decode_step(ctypes.byref(p), ctypes.byref(st), None, f, None, None) == 1
+    stale = D.dark_state(f, f, None, 2, 1, 64, 64, p.generation + 1)
+    assert lib.dark_cross_decode_step(ctypes.byref(p), ctypes.byref(stale), f, f, None, None) == 3
