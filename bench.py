@@ -522,6 +522,164 @@ def run_decode(args, rank: int, world: int, dev) -> dict | None:
     }
 
 
+CROSS_METRIC = ("DARK cross-attention fwd tokens/s (B·H·(Lq+Lk)/s) on 1 B200; "
+                "% of BF16-tensor/HBM roofline")
+CROSS_LQ, CROSS_LK = 256, 1024
+
+
+def cross_workload() -> synth.Workload:
+    """The README's cross-attention example (8 heads of 64, 256 features, 256
+    queries over 1024 context tokens, batch 2) with the causal recipe's draws."""
+    return synth.WORKLOADS[2].with_sizes(B=2, H=8, L=CROSS_LQ, causal=False, lengths=None)
+
+
+def cross_flops_bytes(w: synth.Workload, lq: int, lk: int) -> tuple[float, float]:
+    """Per head 2 Lq d m (query features) + 2 Lk d (m+r) (context features and
+    norms) + 2 Lk m (d+1) (summary) + 2 Lq m (d+1) (output); bytes: q and out
+    over Lq tokens, k and v over Lk tokens, once each, plus both masks."""
+    per_head = 2 * lq * w.d * w.m + 2 * lk * w.d * (w.m + w.r) + 2 * (lq + lk) * w.m * (w.d + 1)
+    elt = 2 if w.dtype == "bf16" else 4
+    nbytes = 2 * w.B * w.H * (lq + lk) * w.d * elt + w.B * (lq + lk)
+    return float(per_head * w.B * w.H), float(nbytes)
+
+
+def run_cross(args, rank: int, world: int, dev) -> dict | None:
+    """Cross-attention forward of queries over a separate context (both masks
+    given, all valid as in the README example); timed like the self-attention
+    forward: one CUDA-graph replay per step, L2 flushed before each."""
+    from random_feature_linear_b200 import dark as D
+    w, lq, lk = cross_workload(), CROSS_LQ, CROSS_LK
+    iq = synth.make_inputs(w, salt=rank)
+    ik = synth.make_inputs(w.with_sizes(L=lk), salt=rank + 1000)
+    tdt = D.torch_dtype(D.DARK_BF16)
+    proj, _wbuf = D.dark_make_projection(torch.from_numpy(iq["omega"]).to(dev),
+                                         torch.from_numpy(iq["geom"]).to(dev), w.H, D.DARK_BF16)
+    q = torch.from_numpy(iq["q"]).to(dev).to(tdt)
+    k, v = (torch.from_numpy(ik[n]).to(dev).to(tdt) for n in ("k", "v"))
+    qm = torch.ones(w.B, lq, dtype=torch.uint8, device=dev)
+    cm = torch.ones(w.B, lk, dtype=torch.uint8, device=dev)
+    out = torch.empty_like(q)
+    ws = D.alloc_cross_workspace(proj, w.B, w.H, lq, lk, 0, dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.int32, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def call(q_, k_, v_, qm_, cm_):
+        D.dark_cross_attention_fwd(proj, q_, k_, v_, out, w.B, w.H, lq, lk, query_mask=qm_,
+                                   context_mask=cm_, ws=ws, dev_status=status)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        call(q, k, v, qm, cm)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    side = torch.cuda.Stream()
+    side.wait_stream(stream)
+    with torch.cuda.stream(side):
+        call(q, k, v, qm, cm)
+        side.synchronize()
+        with torch.cuda.graph(graph, stream=side):
+            call(q, k, v, qm, cm)
+    stream.wait_stream(side)
+    torch.cuda.synchronize()
+    launches_per_step, kernel_names = (1, ["(not counted: --no-profile)"]) if args.no_profile \
+        else count_launches(lambda: call(q, k, v, qm, cm))
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(dev.index) as clk:
+        for i in range(args.steps):
+            flush.zero_()
+            starts[i].record(stream)
+            graph.replay()
+            ends[i].record(stream)
+        torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    ms_per_step = max_over_ranks(sum(s.elapsed_time(e) for s, e in zip(starts, ends)), dev) \
+        / args.steps
+    assert int(status.item()) == 0, D.dark_status_string(int(status.item()))
+
+    host = [t.cpu().pin_memory() for t in (q, k, v, qm, cm)]
+    devb = [torch.empty_like(t) for t in (q, k, v, qm, cm)]
+    hout = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+
+    def e2e_step():
+        for dst, src in zip(devb, host):
+            dst.copy_(src, non_blocking=True)
+        call(*devb)
+        hout.copy_(out, non_blocking=True)
+
+    for _ in range(args.warmup):
+        e2e_step()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    e0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, dev)
+    if rank != 0:
+        return None
+    tokens = w.B * w.H * (lq + lk) * world
+    peaks = load_peaks()
+    flops, nbytes = cross_flops_bytes(w, lq, lk)
+    t = ms_per_step / 1e3
+    t_tc, t_hbm = flops / (peaks["bf16"] * 1e12), nbytes / (peaks["hbm"] * 1e9)
+    if t_tc >= t_hbm:
+        roof = dict(bound="tensor", achieved=flops / t / 1e12, peak=peaks["bf16"], unit="TFLOP/s")
+    else:
+        roof = dict(bound="hbm", achieved=nbytes / t / 1e9, peak=peaks["hbm"], unit="GB/s")
+    roof.update(frac=roof["achieved"] / roof["peak"], traffic=None,
+                peak_source=peaks["source"] + " (burst)", kernel="cross-attention forward call")
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        from oracle import dark_oracle as O
+        qn, kn, vn = iq["q"], ik["k"], ik["v"]
+        t0, heads = time.perf_counter(), 0
+        for b in range(w.B):
+            for h in range(w.H):
+                sl = (slice(b, b + 1), slice(h, h + 1))
+                O.cross_attention(qn[sl], kn[sl], vn[sl], iq["omega"], iq["geom"][h:h + 1])
+                heads += 1
+                if time.perf_counter() - t0 > 10.0:
+                    break
+            else:
+                continue
+            break
+        secs = time.perf_counter() - t0
+        cpu = dict(value=heads * (lq + lk) / secs, unit="tokens/s", cores=blas_threads(),
+                   kind="oracle", sample=f"{heads} of {w.B * w.H} (batch, head) slices, {secs:.1f} s")
+    clocks = clk.summary()
+    return {
+        "metric": CROSS_METRIC, "value": tokens / t, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded numpy, orthogonal Gaussian features)",
+        "config": {"workload": f"cross-attention bf16 (B{w.B} H{w.H} Lq{lq} Lk{lk} d{w.d} r{w.r} "
+                               f"m{w.m}, all-valid query and context masks)",
+                   "l2": "flushed (512 MiB write) before every timed step",
+                   "timing": "CUDA events around one CUDA-graph replay of the forward call per step",
+                   "parallelism": f"replicas x{world} (independent batches, no collective)"},
+        "e2e": {"value": tokens / (e2e_ms / 1e3), "unit": "tokens/s",
+                "h2d_bytes_per_step": sum(x.numel() * x.element_size() for x in host),
+                "d2h_bytes_per_step": hout.numel() * hout.element_size()},
+        "roofline": roof,
+        "roofline_other": {"t_tensor_us": t_tc * 1e6, "t_hbm_us": t_hbm * 1e6,
+                           "alg_flops": flops, "alg_bytes": nbytes},
+        "cpu_baseline": cpu,
+        "gpu_launches": launches_per_step * args.steps,
+        "kernels": kernel_names,
+        "clocks": {"sm_mhz": clocks["sm_mhz"], "sm_max_mhz": clocks["sm_max_mhz"],
+                   "reasons": clocks["reasons"], "samples": clocks["samples"]},
+    }
+
+
 def run_reference(args, w: synth.Workload) -> dict:
     inp = synth.make_inputs(w)
     for _ in range(args.warmup):
@@ -563,6 +721,8 @@ def main():
                     help="do not count launches with the CUDA profiler (for runs under ncu)")
     ap.add_argument("--decode", action="store_true",
                     help="time the streaming decode step (workload 5) instead of the forward")
+    ap.add_argument("--cross", action="store_true",
+                    help="time cross-attention (256 queries over 1024 context tokens) instead")
     ap.add_argument("--ncu", action="store_true",
                     help="capture mode: only warmup + steps forward calls, no timing or output")
     args = ap.parse_args()
@@ -583,8 +743,12 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=dev)
     try:
-        res = run_decode(args, rank, world, dev) if args.decode else \
-            run_native(args, w, rank, world, dev)
+        if args.decode:
+            res = run_decode(args, rank, world, dev)
+        elif args.cross:
+            res = run_cross(args, rank, world, dev)
+        else:
+            res = run_native(args, w, rank, world, dev)
         if res is not None:
             print(json.dumps(res), flush=True)
     finally:
