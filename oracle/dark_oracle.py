@@ -253,3 +253,76 @@ def exponent_range(x, omega, geom):
     """(min, max) natural-log exponent of phi over x, m^{-1/2} included."""
     e = feature_exponents(x, omega, geom) - 0.5 * np.log(np.asarray(omega).shape[0])
     return float(e.min()), float(e.max())
+
+
+def attention_backward(q, k, v, omega, geom, dout, key_mask=None, causal=False):
+    """Gradients of sum(dout * attention(q, k, v, omega, geom, key_mask, causal))
+    with respect to q, k, v and the geometry M (README, "Kernel": M is the
+    learned factor of Sigma = M^T M; Omega is a fixed draw and gets none).
+
+    The chain rule of the forward above, step by step for each (batch, head):
+      S_i, z_i  = the key statistics query i sees (all valid keys, or the
+                  valid keys j <= i when causal);
+      num_i = phi(q_i) S_i, den_i = phi(q_i) . z_i, o_i = num_i / den_i;
+      w_i = g_i / den_i, c_i = (g_i . o_i) / den_i (zero when den_i = 0);
+      dphi(q_i) = S_i w_i - z_i c_i;
+      dS_j = sum over the queries i that see key j of phi(q_i) w_i^T,
+      dz_j = -sum of phi(q_i) c_i over the same queries;
+      dv_j = dS_j^T phi(k_j), dphi(k_j) = dS_j v_j + dz_j (valid keys only).
+    Through phi(x)_j = m^{-1/2} exp(omega_j . u - |u|^2 / 2), u = M x~, x~ = d^{-1/4} x:
+      a_j = dphi_j phi_j;  du = Omega^T a - (sum_j a_j) u;
+      dx = d^{-1/4} M^T du;  dM += du x~^T.
+    q, k, v, dout: [B, H, L, d]; omega: [H_o, m, r]; geom: [H_m, r, d].
+    Returns (dq, dk, dv [B, H, L, d], dgeom [H_m, r, d]), dgeom summed over
+    batches and over the heads that share it.
+    """
+    q, k, v, g_all = _f64(q), _f64(k), _f64(v), _f64(dout)
+    omega, geom = _f64(omega), _f64(geom)
+    B, H, L, d = q.shape
+    m = omega.shape[1]
+    s = d ** -0.25
+    dq, dk, dv = np.zeros_like(q), np.zeros_like(k), np.zeros_like(v)
+    dgeom = np.zeros_like(geom)
+    for b in range(B):
+        valid = np.ones(L, bool) if key_mask is None else np.asarray(key_mask[b]) != 0
+        for h in range(H):
+            om, gm = _head(omega, h), _head(geom, h)
+            phq = feature_map(q[b, h], om, gm)
+            phk = feature_map(k[b, h], om, gm) * valid[:, None]
+            vv, g = v[b, h], g_all[b, h]
+            contrib = np.einsum("jf,je->jfe", phk, vv)          # phi(k_j) v_j^T
+            if causal:
+                S = np.cumsum(contrib, axis=0)                  # S_i over keys j <= i
+                z = np.cumsum(phk, axis=0)
+            else:
+                S = np.broadcast_to(contrib.sum(axis=0), (L, m, d))
+                z = np.broadcast_to(phk.sum(axis=0), (L, m))
+            num = np.einsum("if,ife->ie", phq, S)
+            den = np.einsum("if,if->i", phq, z)
+            ok = den > 0
+            safe = np.where(ok, den, 1.0)
+            o = np.where(ok[:, None], num / safe[:, None], 0.0)
+            w = np.where(ok[:, None], g / safe[:, None], 0.0)
+            c = np.where(ok, np.einsum("ie,ie->i", g, o) / safe, 0.0)
+            dphq = np.einsum("ife,ie->if", S, w) - z * c[:, None]
+            gq = np.einsum("if,ie->ife", phq, w)                # phi(q_i) w_i^T
+            gz = -phq * c[:, None]
+            if causal:
+                # key j is seen by the queries i >= j: suffix sums
+                dS = np.cumsum(gq[::-1], axis=0)[::-1]
+                dz = np.cumsum(gz[::-1], axis=0)[::-1]
+            else:
+                dS = np.broadcast_to(gq.sum(axis=0), (L, m, d))
+                dz = np.broadcast_to(gz.sum(axis=0), (L, m))
+            dv[b, h] = np.einsum("jfe,jf->je", dS, phk) * valid[:, None]
+            dphk = (np.einsum("jfe,je->jf", dS, vv) + dz) * valid[:, None]
+            ghm = np.zeros_like(gm)
+            for x, dph, ph, dst in ((q[b, h], dphq, phq, dq), (k[b, h], dphk, phk, dk)):
+                xs = x * s
+                u = xs @ gm.T
+                a = dph * ph
+                du = a @ om - a.sum(axis=1, keepdims=True) * u
+                dst[b, h] = s * (du @ gm)
+                ghm += du.T @ xs
+            dgeom[0 if geom.shape[0] == 1 else h] += ghm
+    return dq, dk, dv, dgeom
