@@ -680,6 +680,162 @@ def run_cross(args, rank: int, world: int, dev) -> dict | None:
     }
 
 
+BWD_METRIC = ("DARK attention bwd tokens/s (B·H·L/s, dq dk dv dM) on 1 B200; "
+              "% of FP32-FFMA roofline")
+# fp32 FFMA peak: 148 SMs x 128 lanes x 2 FLOP x 1.965 GHz (the backward kernels
+# are SIMT fp32 throughout)
+FFMA_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
+
+
+def bwd_flops(w: synth.Workload) -> float:
+    """Algorithmic FLOPs of one backward pass, per head: features 2Ldm (queries)
+    + 2Ld(m+r) (keys); five m x (d+1) contractions over L (forward statistics,
+    [num | den], dphi(q), gradient statistics, dv with dphi(k)); dx 2Ldm +
+    2Ld(m+r) + 2Ldr (key norms); dW' 4L(m+r)d. Causal diagonal tiles excluded."""
+    L, d, m, r = w.L, w.d, w.m, w.r
+    per_head = (2 * L * d * m + 2 * L * d * (m + r) + 5 * 2 * L * m * (d + 1)
+                + 2 * L * d * m + 2 * L * d * (m + r) + 2 * L * d * r + 4 * L * (m + r) * d)
+    return float(per_head * w.B * w.H)
+
+
+def run_backward(args, w: synth.Workload, rank: int, world: int, dev) -> dict | None:
+    """Backward pass of the workload's attention (gradients of q, k, v and M for
+    a seeded upstream gradient); timed like the forward."""
+    from random_feature_linear_b200 import dark as D
+    inp = synth.make_inputs(w, salt=rank)
+    dout_np = synth.make_cotangent(w, salt=rank)
+    dt = D.DARK_BF16 if w.dtype == "bf16" else D.DARK_F32
+    tdt = D.torch_dtype(dt)
+    omega = torch.from_numpy(inp["omega"]).to(dev)
+    geom = torch.from_numpy(inp["geom"]).to(dev)
+    q, k, v = (torch.from_numpy(inp[n]).to(dev).to(tdt) for n in ("q", "k", "v"))
+    g = torch.from_numpy(dout_np).to(dev).to(tdt)
+    mask = None if inp["mask"] is None else torch.from_numpy(inp["mask"]).to(dev)
+    dq, dk, dv = (torch.empty_like(q) for _ in range(3))
+    dgeom = torch.empty_like(geom)
+    flags = D.DARK_CAUSAL if w.causal else 0
+    ws = D.alloc_bwd_workspace(omega, geom, w.B, w.H, w.L, dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.int32, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def call(q_, k_, v_, g_, m_):
+        D.dark_attention_bwd(omega, geom, q_, k_, v_, g_, dq, dk, dv, w.B, w.H, w.L, dt,
+                             key_mask=m_, flags=flags, dgeom=dgeom, ws=ws, dev_status=status)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        call(q, k, v, g, mask)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0, D.dark_status_string(int(status.item()))
+    graph = torch.cuda.CUDAGraph()
+    side = torch.cuda.Stream()
+    side.wait_stream(stream)
+    with torch.cuda.stream(side):
+        call(q, k, v, g, mask)
+        side.synchronize()
+        with torch.cuda.graph(graph, stream=side):
+            call(q, k, v, g, mask)
+    stream.wait_stream(side)
+    torch.cuda.synchronize()
+    launches_per_step, kernel_names = (1, ["(not counted: --no-profile)"]) if args.no_profile \
+        else count_launches(lambda: call(q, k, v, g, mask))
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(dev.index) as clk:
+        for i in range(args.steps):
+            flush.zero_()
+            starts[i].record(stream)
+            graph.replay()
+            ends[i].record(stream)
+        torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    ms_per_step = max_over_ranks(sum(s.elapsed_time(e) for s, e in zip(starts, ends)), dev) \
+        / args.steps
+
+    srcs = [q, k, v, g] + ([] if mask is None else [mask])
+    host = [t.cpu().pin_memory() for t in srcs]
+    devb = [torch.empty_like(t) for t in srcs]
+    outs = [dq, dk, dv, dgeom]
+    houts = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in outs]
+
+    def e2e_step():
+        for dst, src in zip(devb, host):
+            dst.copy_(src, non_blocking=True)
+        call(devb[0], devb[1], devb[2], devb[3], devb[4] if mask is not None else None)
+        for dst, src in zip(houts, outs):
+            dst.copy_(src, non_blocking=True)
+
+    for _ in range(args.warmup):
+        e2e_step()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    e0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, dev)
+    assert int(status.item()) == 0, D.dark_status_string(int(status.item()))
+    if rank != 0:
+        return None
+    tokens = w.tokens * world
+    t = ms_per_step / 1e3
+    flops = bwd_flops(w)
+    peaks = load_peaks()
+    roof = dict(bound="alu", achieved=flops / t / 1e12, peak=FFMA_TFLOPS, unit="TFLOP/s",
+                frac=flops / t / 1e12 / FFMA_TFLOPS, traffic=None,
+                peak_source="derived: 148 SMs x 128 FP32 lanes x 2 x 1.965 GHz",
+                kernel="backward call (SIMT fp32)")
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        from oracle import dark_oracle as O
+        t0, heads = time.perf_counter(), 0
+        for h in range(w.H):
+            sl = (slice(0, 1), slice(h, h + 1))
+            gm = inp["geom"][h:h + 1] if inp["geom"].shape[0] > 1 else inp["geom"]
+            O.attention_backward(inp["q"][sl], inp["k"][sl], inp["v"][sl], inp["omega"], gm,
+                                 dout_np[sl], key_mask=None if inp["mask"] is None
+                                 else inp["mask"][:1], causal=w.causal)
+            heads += 1
+            if time.perf_counter() - t0 > 10.0:
+                break
+        secs = time.perf_counter() - t0
+        cpu = dict(value=heads * w.L / secs, unit="tokens/s", cores=blas_threads(), kind="oracle",
+                   sample=f"{heads} of {w.B * w.H} (batch, head) slices, {secs:.1f} s")
+    clocks = clk.summary()
+    return {
+        "metric": BWD_METRIC, "value": tokens / t, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16" if w.dtype == "bf16" else "f32",
+        "data": "synthetic (seeded numpy, orthogonal Gaussian features; dout ~ N(0,1))",
+        "config": {"workload": "backward of " + w.name, "B": w.B, "H": w.H, "L": w.L, "d": w.d,
+                   "r": w.r, "m": w.m, "causal": w.causal,
+                   "l2": "flushed (512 MiB write) before every timed step",
+                   "timing": "CUDA events around one CUDA-graph replay of the backward call per step",
+                   "parallelism": f"replicas x{world} (independent batches, no collective)"},
+        "e2e": {"value": tokens / (e2e_ms / 1e3), "unit": "tokens/s",
+                "h2d_bytes_per_step": sum(x.numel() * x.element_size() for x in host),
+                "d2h_bytes_per_step": sum(x.numel() * x.element_size() for x in houts)},
+        "roofline": roof,
+        "roofline_other": {"alg_flops": flops,
+                           "frac_of_bf16_tensor_peak": flops / t / 1e12 / peaks["bf16"],
+                           "t_ffma_us": flops / (FFMA_TFLOPS * 1e12) * 1e6},
+        "cpu_baseline": cpu,
+        "gpu_launches": launches_per_step * args.steps,
+        "kernels": kernel_names,
+        "clocks": {"sm_mhz": clocks["sm_mhz"], "sm_max_mhz": clocks["sm_max_mhz"],
+                   "reasons": clocks["reasons"], "samples": clocks["samples"]},
+    }
+
+
 def run_reference(args, w: synth.Workload) -> dict:
     inp = synth.make_inputs(w)
     for _ in range(args.warmup):
@@ -721,6 +877,8 @@ def main():
                     help="do not count launches with the CUDA profiler (for runs under ncu)")
     ap.add_argument("--decode", action="store_true",
                     help="time the streaming decode step (workload 5) instead of the forward")
+    ap.add_argument("--backward", action="store_true",
+                    help="time the backward pass of --workload instead of the forward")
     ap.add_argument("--cross", action="store_true",
                     help="time cross-attention (256 queries over 1024 context tokens) instead")
     ap.add_argument("--ncu", action="store_true",
@@ -747,6 +905,8 @@ def main():
             res = run_decode(args, rank, world, dev)
         elif args.cross:
             res = run_cross(args, rank, world, dev)
+        elif args.backward:
+            res = run_backward(args, w, rank, world, dev)
         else:
             res = run_native(args, w, rank, world, dev)
         if res is not None:

@@ -1,7 +1,7 @@
 /*
  * dark.h -- C ABI of the B200 (sm_100a) DARKformer positive-random-feature
- * attention library: forward pass (non-causal, causal, key-masked) and the
- * streaming decode step.
+ * attention library: forward pass (non-causal, causal, key-masked), its
+ * backward pass, cross-attention and the streaming decode steps.
  *
  * Source of the method: the DARKformer README ("Data-Aware Random Feature
  * Kernels for Transformers", darkformer-pytorch 0.1.0 package description).
@@ -42,7 +42,7 @@
 extern "C" {
 #endif
 
-#define DARK_ABI_VERSION 2
+#define DARK_ABI_VERSION 3
 
 typedef enum {
   DARK_OK = 0,
@@ -265,6 +265,49 @@ dark_status dark_cross_attention_fwd(const dark_projection* proj, const void* q,
  */
 dark_status dark_cross_decode_step(const dark_projection* proj, const dark_state* context,
                                    const void* q_t, void* out_t, int* dev_status, void* stream);
+
+/*
+ * Backward pass of self-attention (dark_attention_fwd without query mask):
+ * gradients of sum(dout * out) with respect to q, k, v and the geometry M.
+ * README, section "Kernel": M (r x d per head, or shared) is the learned factor
+ * of Sigma = M^T M, whose learning is the method's point; Omega is a fixed draw
+ * of the projection and gets no gradient. Section "Self-attention": the key mask
+ * and the causal constraint act as in the forward pass. A query row with no
+ * visible valid key has output 0 and contributes no gradient; masked keys get
+ * zero dk and dv.
+ *
+ * The projection is rebuilt in fp32 from omega and geom (the forward's W' for
+ * bf16 is fp16), features are recomputed, and every step accumulates in fp32.
+ *   omega        device fp32 [heads_omega][m][r]  (heads_omega = 1 or H)
+ *   geom         device fp32 [heads_geom][r][d]   (heads_geom = 1 or H)
+ *   dtype        element type of q, k, v, dout, dq, dk, dv
+ *   q, k, v      device [B][H][L][d], element strides qkv_strides {b, h, l}
+ *   dout         device [B][H][L][d], strides dout_strides (NULL = contiguous)
+ *   key_mask     device uint8 [B][L] (nonzero = valid) or NULL
+ *   flags        DARK_CAUSAL and/or DARK_STABILISE (a per-head key shift; the
+ *                gradients do not depend on it)
+ *   dq, dk, dv   device [B][H][L][d], strides grad_strides; overwritten. They
+ *                must not overlap each other or any input.
+ *   dgeom        device fp32 [heads_geom][r][d], overwritten with the gradient
+ *                summed over batches and over the heads sharing M; NULL skips it.
+ *   ws, ws_bytes device workspace of at least
+ *                dark_attention_bwd_workspace_bytes(...) bytes, 256-byte
+ *                aligned; no initial contents are required.
+ * Errors: DARK_ERR_INVALID_ARG for a null pointer, a bad head count, flag,
+ * stride or workspace; DARK_ERR_UNSUPPORTED for sizes outside the library's
+ * limits or B*H > 65535; DARK_ERR_CUDA for a failed launch; the device may store
+ * DARK_ERR_NUMERIC in dev_status for a non-finite gradient.
+ */
+size_t dark_attention_bwd_workspace_bytes(int heads_omega, int heads_geom, int m, int r, int d,
+                                          int B, int H, int L);
+dark_status dark_attention_bwd(const float* omega, int heads_omega, const float* geom,
+                               int heads_geom, int m, int r, int d, dark_dtype dtype,
+                               const void* q, const void* k, const void* v,
+                               const int64_t* qkv_strides, const void* dout,
+                               const int64_t* dout_strides, int B, int H, int L,
+                               const uint8_t* key_mask, int flags, void* dq, void* dk, void* dv,
+                               const int64_t* grad_strides, float* dgeom, void* ws,
+                               size_t ws_bytes, int* dev_status, void* stream);
 
 #ifdef __cplusplus
 }

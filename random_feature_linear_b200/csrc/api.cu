@@ -281,6 +281,72 @@ dark_status dark_cross_decode_step(const dark_projection* proj, const dark_state
   return from_cuda(dark::launch_decode(a));
 }
 
+size_t dark_attention_bwd_workspace_bytes(int heads_omega, int heads_geom, int m, int r, int d,
+                                          int B, int H, int L) {
+  if (heads_omega < 1 || heads_geom < 1 || B < 1 || H < 1 || L < 1 || !sizes_ok(m, r, d))
+    return 0;
+  const int heads_w = heads_omega > heads_geom ? heads_omega : heads_geom;
+  return dark::bwd_workspace_bytes(B, H, L, m, r, d, heads_w);
+}
+
+dark_status dark_attention_bwd(const float* omega, int heads_omega, const float* geom,
+                               int heads_geom, int m, int r, int d, dark_dtype dtype,
+                               const void* q, const void* k, const void* v,
+                               const int64_t* qkv_strides, const void* dout,
+                               const int64_t* dout_strides, int B, int H, int L,
+                               const uint8_t* key_mask, int flags, void* dq, void* dk, void* dv,
+                               const int64_t* grad_strides, float* dgeom, void* ws,
+                               size_t ws_bytes, int* dev_status, void* stream) {
+  if (omega == nullptr || geom == nullptr || !dtype_ok(dtype)) return DARK_ERR_INVALID_ARG;
+  if (q == nullptr || k == nullptr || v == nullptr || dout == nullptr || dq == nullptr ||
+      dk == nullptr || dv == nullptr || ws == nullptr)
+    return DARK_ERR_INVALID_ARG;
+  if (B < 1 || H < 1 || L < 1 || m < 1 || r < 1 || d < 1) return DARK_ERR_INVALID_ARG;
+  if (!(heads_omega == 1 || heads_omega == H) || !(heads_geom == 1 || heads_geom == H))
+    return DARK_ERR_INVALID_ARG;
+  if (flags & ~(DARK_CAUSAL | DARK_STABILISE)) return DARK_ERR_INVALID_ARG;
+  if (!sizes_ok(m, r, d)) return DARK_ERR_UNSUPPORTED;
+  if ((int64_t)B * H > 65535) return DARK_ERR_UNSUPPORTED;   // grid y/z bound
+  if (!aligned(ws, 256) || ws_bytes < dark_attention_bwd_workspace_bytes(
+                                          heads_omega, heads_geom, m, r, d, B, H, L))
+    return DARK_ERR_INVALID_ARG;
+  dark::BwdArgs a;
+  memset(&a, 0, sizeof(a));
+  a.omega = omega;
+  a.geom = geom;
+  a.heads_omega = heads_omega;
+  a.heads_geom = heads_geom;
+  a.heads_w = heads_omega > heads_geom ? heads_omega : heads_geom;
+  a.m = m;
+  a.r = r;
+  a.d = d;
+  a.dtype = dtype;
+  a.q = q;
+  a.k = k;
+  a.v = v;
+  a.dout = dout;
+  a.dq = dq;
+  a.dk = dk;
+  a.dv = dv;
+  const int64_t c[3] = {(int64_t)H * L * d, (int64_t)L * d, (int64_t)d};
+  for (int i = 0; i < 3; ++i) {
+    a.xs[i] = qkv_strides ? qkv_strides[i] : c[i];
+    a.gs[i] = dout_strides ? dout_strides[i] : c[i];
+    a.ds[i] = grad_strides ? grad_strides[i] : c[i];
+    if (a.xs[i] < 0 || a.gs[i] < 0 || a.ds[i] < 0) return DARK_ERR_INVALID_ARG;
+  }
+  a.dgeom = dgeom;
+  a.B = B;
+  a.H = H;
+  a.L = L;
+  a.mask = key_mask;
+  a.flags = flags;
+  a.ws = ws;
+  a.dev_status = dev_status;
+  a.stream = (cudaStream_t)stream;
+  return from_cuda(dark::launch_backward(a));
+}
+
 dark_status dark_state_init(const dark_projection* proj, dark_state* st, void* stream) {
   if (proj == nullptr || st == nullptr || st->kv == nullptr || st->z == nullptr)
     return DARK_ERR_INVALID_ARG;

@@ -111,4 +111,23 @@ struct DecodeArgs {
 };
 cudaError_t launch_decode(const DecodeArgs& a);
 
+// Backward pass of self-attention (SIMT, fp32 arithmetic).
+struct BwdArgs {
+  const float *omega, *geom;      // [heads_omega][m][r], [heads_geom][r][d]
+  int heads_omega, heads_geom, heads_w, m, r, d;
+  dark_dtype dtype;
+  const void *q, *k, *v, *dout;
+  void *dq, *dk, *dv;
+  int64_t xs[3], gs[3], ds[3];    // element strides {b, h, l}: q/k/v, dout, dq/dk/dv
+  float* dgeom;                   // [heads_geom][r][d] or null
+  int B, H, L;
+  const uint8_t* mask;
+  int flags;
+  void* ws;
+  int* dev_status;
+  cudaStream_t stream;
+};
+size_t bwd_workspace_bytes(int B, int H, int L, int m, int r, int d, int heads_w);
+cudaError_t launch_backward(const BwdArgs& a);
+
 }  // namespace dark

@@ -30,7 +30,8 @@ EXPORTS = ("dark_abi_version", "dark_status_string", "dark_projection_bytes",
            "dark_make_projection", "dark_attention_workspace_bytes", "dark_attention_fwd",
            "dark_state_init", "dark_decode_step", "dark_noalloc_scratch_bytes",
            "dark_attention_fwd_noalloc", "dark_cross_attention_workspace_bytes",
-           "dark_cross_attention_fwd", "dark_cross_decode_step")
+           "dark_cross_attention_fwd", "dark_cross_decode_step",
+           "dark_attention_bwd_workspace_bytes", "dark_attention_bwd")
 
 
 class dark_projection(ctypes.Structure):
@@ -80,6 +81,13 @@ _lib.dark_cross_attention_fwd.argtypes = [_P(dark_projection), _vp, _P(ctypes.c_
                                           _sz, _vp, _vp]
 _lib.dark_cross_decode_step.restype = _i
 _lib.dark_cross_decode_step.argtypes = [_P(dark_projection), _P(dark_state), _vp, _vp, _vp, _vp]
+_lib.dark_attention_bwd_workspace_bytes.restype = _sz
+_lib.dark_attention_bwd_workspace_bytes.argtypes = [_i] * 8
+_lib.dark_attention_bwd.restype = _i
+_lib.dark_attention_bwd.argtypes = [_vp, _i, _vp, _i, _i, _i, _i, _i, _vp, _vp, _vp,
+                                    _P(ctypes.c_int64), _vp, _P(ctypes.c_int64), _i, _i, _i, _vp,
+                                    _i, _vp, _vp, _vp, _P(ctypes.c_int64), _vp, _vp, _sz, _vp,
+                                    _vp]
 
 
 class DarkError(RuntimeError):
@@ -95,6 +103,31 @@ def _check(status: int) -> None:
 
 def _ptr(t) -> int | None:
     return None if t is None else t.data_ptr()
+
+
+def _strides(given, *tensors):
+    """Element strides {b, h, l} of [B][H][L][d] tensors for the C ABI: the given
+    ones, else the tensors' own, which must agree and have a unit d stride."""
+    if given is None:
+        own = {tuple(t.stride()) for t in tensors}
+        if len(own) != 1:
+            raise ValueError("tensors sharing one stride argument have different strides")
+        s = own.pop()
+        if len(s) != 4 or s[3] != 1:
+            raise ValueError("expected [B][H][L][d] tensors with a unit d stride")
+        given = s[:3]
+    return (ctypes.c_int64 * 3)(*given)
+
+
+def _dense(t, name):
+    """Arrays without stride arguments cross the ABI as dense row-major buffers."""
+    if t is not None and not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t
+
+
+def _dptr(t, name) -> int | None:
+    return _ptr(_dense(t, name))
 
 
 def _stream(stream) -> int | None:
@@ -161,12 +194,10 @@ def dark_attention_fwd(proj: dark_projection, q, k, v, out, B: int, H: int, L: i
                        ws=None, dev_status=None, stream=None, qkv_strides=None,
                        out_strides=None) -> None:
     """q/k/v/out are device tensors viewed as [B][H][L][d] with the given element
-    strides ({b, h, l}; None = contiguous). ws: a zero-initialised uint8 tensor."""
-    def strides(s):
-        return None if s is None else (ctypes.c_int64 * 3)(*s)
+    strides ({b, h, l}; None = the tensors' own). ws: a zero-initialised uint8 tensor."""
     _check(_lib.dark_attention_fwd(
-        ctypes.byref(proj), _ptr(q), _ptr(k), _ptr(v), _ptr(out), strides(qkv_strides),
-        strides(out_strides), B, H, L, _ptr(key_mask), flags,
+        ctypes.byref(proj), _ptr(q), _ptr(k), _ptr(v), _ptr(out), _strides(qkv_strides, q, k, v),
+        _strides(out_strides, out), B, H, L, _dptr(key_mask, "key_mask"), flags,
         None if state_out is None else ctypes.byref(state_out), _ptr(ws),
         0 if ws is None else ws.numel() * ws.element_size(), _ptr(dev_status), _stream(stream)))
 
@@ -180,11 +211,9 @@ def dark_attention_fwd_noalloc(proj: dark_projection, q, k, v, out, B: int, H: i
                                state_out: dark_state | None = None, dev_status=None,
                                stream=None, qkv_strides=None, out_strides=None) -> None:
     """dark_attention_fwd with the library's fixed scratch instead of a workspace."""
-    def strides(s):
-        return None if s is None else (ctypes.c_int64 * 3)(*s)
     _check(_lib.dark_attention_fwd_noalloc(
-        ctypes.byref(proj), _ptr(q), _ptr(k), _ptr(v), _ptr(out), strides(qkv_strides),
-        strides(out_strides), B, H, L, _ptr(key_mask), flags,
+        ctypes.byref(proj), _ptr(q), _ptr(k), _ptr(v), _ptr(out), _strides(qkv_strides, q, k, v),
+        _strides(out_strides, out), B, H, L, _dptr(key_mask, "key_mask"), flags,
         None if state_out is None else ctypes.byref(state_out), _ptr(dev_status),
         _stream(stream)))
 
@@ -195,9 +224,9 @@ def dark_state_init(proj: dark_projection, st: dark_state, stream=None) -> None:
 
 def dark_decode_step(proj: dark_projection, st: dark_state, q_t, k_t, v_t, out_t, valid=None,
                      dev_status=None, stream=None) -> None:
-    _check(_lib.dark_decode_step(ctypes.byref(proj), ctypes.byref(st), _ptr(q_t), _ptr(k_t),
-                                 _ptr(v_t), _ptr(out_t), _ptr(valid), _ptr(dev_status),
-                                 _stream(stream)))
+    _check(_lib.dark_decode_step(ctypes.byref(proj), ctypes.byref(st), _dptr(q_t, "q_t"),
+                                 _dptr(k_t, "k_t"), _dptr(v_t, "v_t"), _dptr(out_t, "out_t"),
+                                 _dptr(valid, "valid"), _ptr(dev_status), _stream(stream)))
 
 
 def dark_cross_attention_workspace_bytes(proj: dark_projection, B: int, H: int, Lq: int, Lk: int,
@@ -211,20 +240,20 @@ def dark_cross_attention_fwd(proj: dark_projection, q, k, v, out, B: int, H: int
                              stream=None, q_strides=None, kv_strides=None,
                              out_strides=None) -> None:
     """q/out viewed as [B][H][Lq][d], k/v as [B][H][Lk][d] with the given element
-    strides ({b, h, l}; None = contiguous). ws: a zero-initialised uint8 tensor."""
-    def strides(s):
-        return None if s is None else (ctypes.c_int64 * 3)(*s)
+    strides ({b, h, l}; None = the tensors' own). ws: a zero-initialised uint8 tensor."""
     _check(_lib.dark_cross_attention_fwd(
-        ctypes.byref(proj), _ptr(q), strides(q_strides), Lq, _ptr(query_mask), _ptr(k), _ptr(v),
-        strides(kv_strides), Lk, _ptr(context_mask), _ptr(out), strides(out_strides), B, H, flags,
+        ctypes.byref(proj), _ptr(q), _strides(q_strides, q), Lq, _dptr(query_mask, "query_mask"), _ptr(k), _ptr(v),
+        _strides(kv_strides, k, v), Lk, _dptr(context_mask, "context_mask"), _ptr(out), _strides(out_strides, out),
+        B, H, flags,
         None if context_out is None else ctypes.byref(context_out), _ptr(ws),
         0 if ws is None else ws.numel() * ws.element_size(), _ptr(dev_status), _stream(stream)))
 
 
 def dark_cross_decode_step(proj: dark_projection, context: dark_state, q_t, out_t,
                            dev_status=None, stream=None) -> None:
-    _check(_lib.dark_cross_decode_step(ctypes.byref(proj), ctypes.byref(context), _ptr(q_t),
-                                       _ptr(out_t), _ptr(dev_status), _stream(stream)))
+    _check(_lib.dark_cross_decode_step(ctypes.byref(proj), ctypes.byref(context),
+                                       _dptr(q_t, "q_t"), _dptr(out_t, "out_t"), _ptr(dev_status),
+                                       _stream(stream)))
 
 
 def alloc_cross_workspace(proj: dark_projection, B: int, H: int, Lq: int, Lk: int, flags: int,
@@ -232,6 +261,41 @@ def alloc_cross_workspace(proj: dark_projection, B: int, H: int, Lq: int, Lk: in
     """A zero-filled workspace of the size dark_cross_attention_workspace_bytes asks for."""
     n = dark_cross_attention_workspace_bytes(proj, B, H, Lq, Lk, flags)
     return torch.zeros(max(n, WS_HEADER_BYTES), dtype=torch.uint8, device=device)
+
+
+def dark_attention_bwd_workspace_bytes(heads_omega: int, heads_geom: int, m: int, r: int, d: int,
+                                       B: int, H: int, L: int) -> int:
+    return _lib.dark_attention_bwd_workspace_bytes(heads_omega, heads_geom, m, r, d, B, H, L)
+
+
+def dark_attention_bwd(omega, geom, q, k, v, dout, dq, dk, dv, B: int, H: int, L: int,
+                       dtype: int, key_mask=None, flags: int = 0, dgeom=None, ws=None,
+                       dev_status=None, stream=None, qkv_strides=None, dout_strides=None,
+                       grad_strides=None) -> None:
+    """Gradients of sum(dout * out) of self-attention. omega: fp32 device tensor
+    [H_o, m, r]; geom: fp32 [H_m, r, d]; q/k/v/dout/dq/dk/dv viewed as
+    [B][H][L][d] with element strides ({b, h, l}; None = the tensors' own); dgeom: fp32
+    [H_m, r, d] or None; ws: see alloc_bwd_workspace."""
+    assert omega.dtype == torch.float32 and geom.dtype == torch.float32
+    omega, geom = omega.contiguous(), geom.contiguous()
+    if dgeom is not None:
+        _dense(dgeom, "dgeom")
+    ho, m, r = omega.shape
+    hg, _, d = geom.shape
+    _check(_lib.dark_attention_bwd(
+        _ptr(omega), ho, _ptr(geom), hg, m, r, d, dtype, _ptr(q), _ptr(k), _ptr(v),
+        _strides(qkv_strides, q, k, v), _ptr(dout), _strides(dout_strides, dout), B, H, L,
+        _dptr(key_mask, "key_mask"), flags, _ptr(dq), _ptr(dk), _ptr(dv), _strides(grad_strides, dq, dk, dv),
+        _ptr(dgeom), _ptr(ws),
+        0 if ws is None else ws.numel() * ws.element_size(), _ptr(dev_status), _stream(stream)))
+
+
+def alloc_bwd_workspace(omega, geom, B: int, H: int, L: int, device):
+    """A workspace of the size dark_attention_bwd_workspace_bytes asks for."""
+    ho, m, r = omega.shape
+    hg, _, d = geom.shape
+    n = dark_attention_bwd_workspace_bytes(ho, hg, m, r, d, B, H, L)
+    return torch.empty(max(n, WS_HEADER_BYTES), dtype=torch.uint8, device=device)
 
 
 def alloc_workspace(proj: dark_projection, B: int, H: int, L: int, flags: int, device):

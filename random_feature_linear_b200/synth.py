@@ -21,7 +21,7 @@ from __future__ import annotations
 import dataclasses
 import numpy as np
 
-TID_OMEGA, TID_GEOM, TID_Q, TID_K, TID_V, TID_STREAM = 1, 2, 3, 4, 5, 6
+TID_OMEGA, TID_GEOM, TID_Q, TID_K, TID_V, TID_STREAM, TID_GRAD = 1, 2, 3, 4, 5, 6, 7
 
 
 @dataclasses.dataclass(frozen=True)
@@ -161,6 +161,12 @@ def make_inputs(w: Workload, salt: int = 0) -> dict:
         for b, n in enumerate(w.lengths):
             mask[b, :n] = 1
     return dict(omega=omega, geom=geom, q=q, k=k, v=v, mask=mask)
+
+
+def make_cotangent(w: Workload, salt: int = 0) -> np.ndarray:
+    """Upstream gradient dout ~ N(0, 1) of the attention output, [B, H, L, d]
+    (bf16-exact where the workload's I/O is bf16)."""
+    return _io(w, _rng(w, TID_GRAD, salt).standard_normal((w.B, w.H, w.L, w.d)))
 
 
 def decode_stream(w: Workload, steps: int, salt: int = 0) -> dict:

@@ -149,3 +149,27 @@ def test_cross_decode_rejects_stale_and_bad_arguments(D):
     assert lib.dark_cross_decode_step(ctypes.byref(p), ctypes.byref(st), None, f, None, None) == 1
     stale = D.dark_state(f, f, None, 2, 1, 64, 64, p.generation + 1)
     assert lib.dark_cross_decode_step(ctypes.byref(p), ctypes.byref(stale), f, f, None, None) == 3
+
+
+def test_backward_rejects_bad_arguments(D):
+    lib = D._lib
+    f = 0x10000
+    need = D.dark_attention_bwd_workspace_bytes(1, 2, 64, 32, 64, 2, 2, 100)
+
+    def call(om=f, ho=1, gm=f, hg=2, m=64, r=32, d=64, dt=D.DARK_BF16, q=f, g=f, B=2, H=2, L=100,
+             flags=0, dq=f, ws=f, wsb=need, strides=None):
+        return lib.dark_attention_bwd(om, ho, gm, hg, m, r, d, dt, q, f, f, strides, g, None, B, H,
+                                      L, None, flags, dq, f, f, None, None, ws, wsb, None, None)
+
+    assert call(om=None) == 1 and call(gm=None) == 1 and call(q=None) == 1
+    assert call(g=None) == 1 and call(dq=None) == 1 and call(ws=None) == 1
+    assert call(ho=3) == 1 and call(hg=0) == 1            # heads must be 1 or H
+    assert call(B=0) == 1 and call(L=0) == 1
+    assert call(flags=4) == 1 and call(dt=7) == 1
+    assert call(d=6) == 2 and call(m=4096) == 2           # outside the library's sizes
+    assert call(ws=f + 64) == 1 and call(wsb=need - 1) == 1
+    assert call(strides=(ctypes.c_int64 * 3)(-1, 64, 64)) == 1
+    assert call(B=300, H=300, hg=1, wsb=1 << 62) == 2      # grid bound on B*H
+    # workspace size: zero for bad sizes, growing with L
+    assert D.dark_attention_bwd_workspace_bytes(1, 2, 64, 32, 64, 0, 2, 100) == 0
+    assert need < D.dark_attention_bwd_workspace_bytes(1, 2, 64, 32, 64, 2, 2, 1000)
