@@ -40,7 +40,7 @@ METRIC = "DARK attention fwd tokens/s (B\u00b7H\u00b7L/s) on 1 B200; % of BF16-t
 # (key states, causal chunks; no bytes written back within either launch).
 # Reported only while the kernel sources hash to what was captured.
 _CAUSAL_SOURCES = ("tc_causal.cu", "tc_keys.cu", "tc_keys.cuh", "tc_common.cuh")
-_NCU_TRAFFIC = {2: ("0d90ad241e86d6f0", 8.758528e6 + 21.510912e6)}
+_NCU_TRAFFIC = {2: ("2d9f70c43543c0ba", 8.759040e6 + 21.510656e6)}
 
 
 def captured_traffic(cfg: int):

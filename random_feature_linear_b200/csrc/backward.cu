@@ -76,22 +76,48 @@ __global__ void fill_ordered_kernel(int* p, int n, float v) {
   if (i < n) p[i] = float_to_ordered(v);
 }
 
-// One 64 x 64 output tile of A B^T accumulated over K in chunks of 32, from two
-// shared staging buffers [64][33] filled by the caller's loaders: thread (ty, tx)
-// owns rows ty*4.. and columns tx*4...
-__device__ __forceinline__ void fma_tile(const float* As, const float* Bs, float (&acc)[4][4]) {
+// Tile GEMM building blocks. Operand tiles are staged k-major in shared memory,
+// [32 k][kLd] for 64 rows or columns (the 4 extra floats keep every row 16-byte
+// aligned), so one k step reads one float4 of A and one of B for 16 FMAs.
+// Thread (ty, tx) = (threadIdx / 16, threadIdx % 16) owns output rows ty*4..+3
+// and columns tx*4..+3 of a 64 x 64 tile.
+constexpr int kLd = 68;
+
+__device__ __forceinline__ float4 ld4(const float* p) {
+  return *reinterpret_cast<const float4*>(p);
+}
+
+// acc[i][j] += sum_kk A[kk][ty*4+i] B[kk][tx*4+j], kk < 32 (A, B k-major, stride kLd).
+__device__ __forceinline__ void fma_tile(const float* A, const float* B, float (&acc)[4][4]) {
   const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
 #pragma unroll 8
   for (int kk = 0; kk < 32; ++kk) {
-    float a[4], b[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) a[i] = As[(ty * 4 + i) * 33 + kk];
-#pragma unroll
-    for (int j = 0; j < 4; ++j) b[j] = Bs[(tx * 4 + j) * 33 + kk];
+    const float4 a4 = ld4(A + kk * kLd + ty * 4), b4 = ld4(B + kk * kLd + tx * 4);
+    const float a[4] = {a4.x, a4.y, a4.z, a4.w}, b[4] = {b4.x, b4.y, b4.z, b4.w};
 #pragma unroll
     for (int i = 0; i < 4; ++i)
 #pragma unroll
       for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
+  }
+}
+
+// Stages dst[kk][row] = get(row, kk) for 64 rows x 32 k from a source whose
+// rows are contiguous in k (consecutive threads read consecutive k).
+template <class Get>
+__device__ __forceinline__ void stage_t(float* dst, Get get) {
+  for (int e = threadIdx.x; e < 64 * 32; e += blockDim.x) {
+    const int row = e >> 5, kk = e & 31;
+    dst[kk * kLd + row] = get(row, kk);
+  }
+}
+
+// Stages dst[kk][col] = get(kk, col) for 32 k x 64 columns from a source whose
+// rows are contiguous in the column index.
+template <class Get>
+__device__ __forceinline__ void stage_n(float* dst, Get get) {
+  for (int e = threadIdx.x; e < 32 * 64; e += blockDim.x) {
+    const int kk = e >> 6, col = e & 63;
+    dst[kk * kLd + col] = get(kk, col);
   }
 }
 
@@ -112,8 +138,8 @@ __global__ void __launch_bounds__(256) bwd_features_kernel(
     const float* __restrict__ w, int heads_w, int m, int r, int d, int H, int L,
     const uint8_t* __restrict__ mask, int stabilise, float* __restrict__ phiq,
     float* __restrict__ phik, int* __restrict__ ck) {
-  __shared__ float Xs[kT * 33];
-  __shared__ float Ws[64 * 33];
+  __shared__ __align__(16) float Xs[32 * kLd];
+  __shared__ __align__(16) float Ws[32 * kLd];
   __shared__ float rowc[kT];
   __shared__ int rowmax[kT];
   const int side = blockIdx.z;
@@ -132,11 +158,12 @@ __global__ void __launch_bounds__(256) bwd_features_kernel(
   auto tile = [&](int c0, float (&acc)[4][4]) {
     zero(acc);
     for (int k0 = 0; k0 < d; k0 += 32) {
-      for (int e = threadIdx.x; e < kT * 32; e += blockDim.x) {
-        const int t = e >> 5, c = e & 31;
-        Xs[t * 33 + c] = (t0 + t < L && k0 + c < d) ? to_f32(x[(int64_t)(t0 + t) * sl + k0 + c]) : 0.f;
-        Ws[t * 33 + c] = (c0 + t < m + r && k0 + c < d) ? wh[(size_t)(c0 + t) * d + k0 + c] : 0.f;
-      }
+      stage_t(Xs, [&](int t, int kk) {
+        return (t0 + t < L && k0 + kk < d) ? to_f32(x[(int64_t)(t0 + t) * sl + k0 + kk]) : 0.f;
+      });
+      stage_t(Ws, [&](int j, int kk) {
+        return (c0 + j < m + r && k0 + kk < d) ? wh[(size_t)(c0 + j) * d + k0 + kk] : 0.f;
+      });
       __syncthreads();
       fma_tile(Xs, Ws, acc);
       __syncthreads();
@@ -242,8 +269,8 @@ template <class U>
 __global__ void __launch_bounds__(256) chunk_state_kernel(const float* __restrict__ A, U u, int m,
                                                           int d, int L, int nt,
                                                           float* __restrict__ st) {
-  __shared__ float As[32 * 65];
-  __shared__ float Bs[32 * 65];
+  __shared__ __align__(16) float As[32 * kLd];
+  __shared__ __align__(16) float Bs[32 * kLd];
   const int c = blockIdx.x, bh = blockIdx.y;
   const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
   const int dd = d + 1;
@@ -255,24 +282,16 @@ __global__ void __launch_bounds__(256) chunk_state_kernel(const float* __restric
       float acc[4][4];
       zero(acc);
       for (int k0 = tb; k0 < te; k0 += 32) {
-        for (int e = threadIdx.x; e < 32 * 64; e += blockDim.x) {
-          const int tt = e >> 6, f = e & 63, t = k0 + tt;
-          As[tt * 65 + f] = (t < te && f0 + f < m) ? a[(size_t)t * m + f0 + f] : 0.f;
-          Bs[tt * 65 + f] = t < te ? u(bh, t, e0 + f) : 0.f;
-        }
+        stage_n(As, [&](int kk, int f) {
+          const int t = k0 + kk;
+          return (t < te && f0 + f < m) ? a[(size_t)t * m + f0 + f] : 0.f;
+        });
+        stage_n(Bs, [&](int kk, int col) {
+          const int t = k0 + kk;
+          return t < te ? u(bh, t, e0 + col) : 0.f;
+        });
         __syncthreads();
-#pragma unroll 8
-        for (int kk = 0; kk < 32; ++kk) {
-          float x[4], y[4];
-#pragma unroll
-          for (int i = 0; i < 4; ++i) x[i] = As[kk * 65 + ty * 4 + i];
-#pragma unroll
-          for (int j = 0; j < 4; ++j) y[j] = Bs[kk * 65 + tx * 4 + j];
-#pragma unroll
-          for (int i = 0; i < 4; ++i)
-#pragma unroll
-            for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(x[i], y[j], acc[i][j]);
-        }
+        fma_tile(As, Bs, acc);
         __syncthreads();
       }
 #pragma unroll
@@ -290,17 +309,26 @@ __global__ void __launch_bounds__(256) chunk_state_kernel(const float* __restric
 }
 
 // mode 0: exclusive prefix over tiles (causal forward statistics); 1: exclusive
-// suffix (causal gradient statistics); 2: total into tile 0 (non-causal).
+// suffix (causal gradient statistics); 2: total into tile 0 (non-causal). Eight
+// tiles' values are loaded before any is stored, so the loads overlap.
 __global__ void tile_scan_kernel(float* __restrict__ st, int n, int nt, int mode) {
   const int idx = blockIdx.x * blockDim.x + threadIdx.x;
   if (idx >= n) return;
   float* base = st + (size_t)blockIdx.y * nt * n + idx;
   float run = 0.f;
-  for (int s = 0; s < nt; ++s) {
-    const int c = mode == 1 ? nt - 1 - s : s;
-    const float t = base[(size_t)c * n];
-    if (mode != 2) base[(size_t)c * n] = run;
-    run += t;
+  for (int s0 = 0; s0 < nt; s0 += 8) {
+    float v[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int s = s0 + u, c = mode == 1 ? nt - 1 - s : s;
+      v[u] = s < nt ? base[(size_t)c * n] : 0.f;
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int s = s0 + u, c = mode == 1 ? nt - 1 - s : s;
+      if (s < nt && mode != 2) base[(size_t)c * n] = run;
+      run += v[u];
+    }
   }
   if (mode == 2) base[0] = run;
 }
@@ -311,22 +339,24 @@ __global__ void tile_scan_kernel(float* __restrict__ st, int n, int nt, int mode
 // SIDE 1 (keys): X = Phi(K), Y = Phi(Q), state = dS over later tiles (or all
 // queries), U = [w | -c]; phase 1 gives dv; P = [v | 1]. Phase 2 on both sides:
 // dphi(X) = P state^T + tri(P U^T) Y, then coef = ln2 * X * dphi.
-// tri keeps key <= query within the tile (causal only).
-template <typename T, int SIDE>
-__global__ void __launch_bounds__(256) pass_kernel(
+// tri keeps key <= query within the tile (causal only). ET = ceil((d + 1) / 64)
+// column blocks of [num | den] per thread.
+template <typename T, int SIDE, int ET>
+__global__ void __launch_bounds__(256, ET <= 3 ? 2 : 1) pass_kernel(
     const float* __restrict__ phiq, const float* __restrict__ phik,
     const float* __restrict__ state, const T* __restrict__ v, int64_t vb, int64_t vh, int64_t vl,
     const T* __restrict__ g, int64_t gb, int64_t gh, int64_t gl, float* __restrict__ wq,
     T* __restrict__ dv, int64_t ob, int64_t oh, int64_t ol, float* __restrict__ coef, int m,
     int r, int d, int H, int L, int nt, int causal, int* dev_status) {
-  extern __shared__ float sm[];
-  const int dd = d + 1, ET = (dd + 63) / 64, ddp = ET * 64;
-  float* Xs = sm;                 // [64][33]
-  float* Ys = Xs + 64 * 33;       // [64][33]
-  float* Sc = Ys + 64 * 33;       // [64][65]  masked tile of X Y^T, then of P U^T
-  float* Bt = Sc + 64 * 65;       // [32][ddp]
-  float* Ps = Bt + 32 * ddp;      // [64][ddp]
-  float* rowv = Ps + 64 * ddp;    // [64]
+  extern __shared__ __align__(16) float sm[];
+  constexpr int ddp = ET * 64;
+  const int dd = d + 1;
+  float* Xk = sm;                 // [32][kLd]  A staging
+  float* Yk = Xk + 32 * kLd;      // [32][kLd]  B staging
+  float* ScT = Yk + 32 * kLd;     // [64 k][kLd] masked tile of X Y^T, then of P U^T (k-major)
+  float* Bt = ScT + 64 * kLd;     // [32][ddp]  phase-1 B operand (state rows, U rows)
+  float* PsT = Bt + 32 * ddp;     // [ddp][kLd] P, k-major
+  float* rowv = PsT + ddp * kLd;  // [64]
   const int c = blockIdx.x, bh = blockIdx.y, b = bh / H, h = bh % H;
   const int t0 = c * kT;
   const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
@@ -342,84 +372,85 @@ __global__ void __launch_bounds__(256) pass_kernel(
     return wrow[(size_t)t * dd + e];
   };
   auto keep = [](int row, int col) { return SIDE == 0 ? col <= row : col >= row; };
+  // masked 64 x 64 tile from registers into ScT[col][row] (k-major for the next GEMM)
+  auto store_masked = [&](const float (&s4)[4][4]) {
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int col = tx * 4 + j;
+      float4 o;
+      o.x = keep(ty * 4 + 0, col) ? s4[0][j] : 0.f;
+      o.y = keep(ty * 4 + 1, col) ? s4[1][j] : 0.f;
+      o.z = keep(ty * 4 + 2, col) ? s4[2][j] : 0.f;
+      o.w = keep(ty * 4 + 3, col) ? s4[3][j] : 0.f;
+      *reinterpret_cast<float4*>(ScT + col * kLd + ty * 4) = o;
+    }
+  };
 
   // ---- phase 1: acc = X state + tri(X Y^T) U ----
-  float acc[5][4][4];
+  float acc[ET][4][4];
 #pragma unroll
-  for (int et = 0; et < 5; ++et)
+  for (int et = 0; et < ET; ++et)
 #pragma unroll
     for (int i = 0; i < 4; ++i)
 #pragma unroll
       for (int j = 0; j < 4; ++j) acc[et][i][j] = 0.f;
-  auto acc_from = [&](const float* A, int lda) {   // acc += A[64][32] Bt[32][ddp]
+  auto acc_from = [&](const float* A) {   // acc += A[32 k][64 rows] (k-major) Bt[32][ddp]
+#pragma unroll 4
     for (int kk = 0; kk < 32; ++kk) {
-      float a[4];
+      const float4 a4 = ld4(A + kk * kLd + ty * 4);
+      const float a[4] = {a4.x, a4.y, a4.z, a4.w};
 #pragma unroll
-      for (int i = 0; i < 4; ++i) a[i] = A[(ty * 4 + i) * lda + kk];
+      for (int et = 0; et < ET; ++et) {
+        const float4 b4 = ld4(Bt + kk * ddp + et * 64 + tx * 4);
+        const float bb[4] = {b4.x, b4.y, b4.z, b4.w};
 #pragma unroll
-      for (int et = 0; et < 5; ++et) {
-        if (et < ET) {
+        for (int i = 0; i < 4; ++i)
 #pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const float bv = Bt[kk * ddp + et * 64 + tx * 4 + j];
-#pragma unroll
-            for (int i = 0; i < 4; ++i) acc[et][i][j] = fmaf(a[i], bv, acc[et][i][j]);
-          }
-        }
+          for (int j = 0; j < 4; ++j) acc[et][i][j] = fmaf(a[i], bb[j], acc[et][i][j]);
       }
     }
   };
+  float s4[4][4];
+  zero(s4);
   for (int f0 = 0; f0 < m; f0 += 32) {
-    for (int e = threadIdx.x; e < 64 * 32; e += blockDim.x) {
-      const int i = e >> 5, kk = e & 31;
-      Xs[i * 33 + kk] = (t0 + i < L && f0 + kk < m) ? X[(size_t)(t0 + i) * m + f0 + kk] : 0.f;
-    }
+    stage_t(Xk, [&](int i, int kk) {
+      return (t0 + i < L && f0 + kk < m) ? X[(size_t)(t0 + i) * m + f0 + kk] : 0.f;
+    });
+    if (causal)
+      stage_t(Yk, [&](int j, int kk) {
+        return (t0 + j < L && f0 + kk < m) ? Y[(size_t)(t0 + j) * m + f0 + kk] : 0.f;
+      });
     for (int e = threadIdx.x; e < 32 * ddp; e += blockDim.x) {
       const int kk = e / ddp, col = e % ddp;
       Bt[e] = (f0 + kk < m && col < dd) ? st[(size_t)(f0 + kk) * dd + col] : 0.f;
     }
     __syncthreads();
-    acc_from(Xs, 33);
+    acc_from(Xk);
+    if (causal) fma_tile(Xk, Yk, s4);
     __syncthreads();
   }
   if (causal) {
-    float s4[4][4];
-    zero(s4);
-    for (int f0 = 0; f0 < m; f0 += 32) {
-      for (int e = threadIdx.x; e < 64 * 32; e += blockDim.x) {
-        const int i = e >> 5, kk = e & 31;
-        const bool in = f0 + kk < m;
-        Xs[i * 33 + kk] = (t0 + i < L && in) ? X[(size_t)(t0 + i) * m + f0 + kk] : 0.f;
-        Ys[i * 33 + kk] = (t0 + i < L && in) ? Y[(size_t)(t0 + i) * m + f0 + kk] : 0.f;
-      }
-      __syncthreads();
-      fma_tile(Xs, Ys, s4);
-      __syncthreads();
-    }
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-#pragma unroll
-      for (int j = 0; j < 4; ++j)
-        Sc[(ty * 4 + i) * 65 + tx * 4 + j] = keep(ty * 4 + i, tx * 4 + j) ? s4[i][j] : 0.f;
+    store_masked(s4);
     for (int k0 = 0; k0 < 64; k0 += 32) {
       for (int e = threadIdx.x; e < 32 * ddp; e += blockDim.x) {
         const int kk = e / ddp, col = e % ddp;
         Bt[e] = U(t0 + k0 + kk, col);
       }
       __syncthreads();
-      acc_from(Sc + k0, 65);
+      acc_from(ScT + k0 * kLd);
       __syncthreads();
     }
   }
 
-  // ---- epilogue of phase 1 ----
+  // ---- epilogue of phase 1: P into PsT (k-major) ----
+  auto put_p = [&](int row, int col, float p) { PsT[col * kLd + row] = p; };
   if (SIDE == 0) {
     // den = column d of [num | den]
 #pragma unroll
-    for (int et = 0; et < 5; ++et)
+    for (int et = 0; et < ET; ++et)
 #pragma unroll
       for (int j = 0; j < 4; ++j)
-        if (et < ET && et * 64 + tx * 4 + j == d) {
+        if (et * 64 + tx * 4 + j == d) {
 #pragma unroll
           for (int i = 0; i < 4; ++i) rowv[ty * 4 + i] = acc[et][i][j];
         }
@@ -430,28 +461,27 @@ __global__ void __launch_bounds__(256) pass_kernel(
       const int row = ty * 4 + i, t = t0 + row;
       const float den = rowv[row];
       const float inv = (t < L && den > 0.f) ? 1.f / den : 0.f;
-      float gv[5][4];
+      float gv[ET][4];
       float go = 0.f;
 #pragma unroll
-      for (int et = 0; et < 5; ++et)
+      for (int et = 0; et < ET; ++et)
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
           const int col = et * 64 + tx * 4 + j;
-          gv[et][j] = (et < ET && col < d && t < L) ? to_f32(gh_[(int64_t)t * gl + col]) : 0.f;
-          go = fmaf(gv[et][j], et < ET ? acc[et][i][j] : 0.f, go);
+          gv[et][j] = (col < d && t < L) ? to_f32(gh_[(int64_t)t * gl + col]) : 0.f;
+          go = fmaf(gv[et][j], acc[et][i][j], go);
         }
       // the 16 threads of a row are 16 consecutive lanes
 #pragma unroll
       for (int o = 8; o > 0; o >>= 1) go += __shfl_xor_sync(0xffffffffu, go, o);
       const float cc = go * inv * inv;
 #pragma unroll
-      for (int et = 0; et < 5; ++et)
+      for (int et = 0; et < ET; ++et)
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
           const int col = et * 64 + tx * 4 + j;
-          if (et >= ET) continue;
           const float p = col < d ? gv[et][j] * inv : (col == d ? -cc : 0.f);
-          Ps[row * ddp + col] = p;
+          put_p(row, col, p);
           if (t < L && col < dd) wrow[(size_t)t * dd + col] = p;
           if (col < dd && !isfinite(p)) report(dev_status, DARK_ERR_NUMERIC);
         }
@@ -462,17 +492,18 @@ __global__ void __launch_bounds__(256) pass_kernel(
     for (int i = 0; i < 4; ++i) {
       const int row = ty * 4 + i, t = t0 + row;
 #pragma unroll
-      for (int et = 0; et < 5; ++et)
+      for (int et = 0; et < ET; ++et)
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
           const int col = et * 64 + tx * 4 + j;
-          if (et >= ET) continue;
           if (t < L && col < d) {
             const float gval = acc[et][i][j];
             if (!isfinite(gval)) report(dev_status, DARK_ERR_NUMERIC);
             dvh[(int64_t)t * ol + col] = from_f32<T>(gval);
           }
-          Ps[row * ddp + col] = t < L ? (col < d ? to_f32(vh_[(int64_t)t * vl + col]) : (col == d ? 1.f : 0.f)) : 0.f;
+          put_p(row, col, t < L ? (col < d ? to_f32(vh_[(int64_t)t * vl + col])
+                                           : (col == d ? 1.f : 0.f))
+                                : 0.f);
         }
     }
   }
@@ -480,23 +511,14 @@ __global__ void __launch_bounds__(256) pass_kernel(
 
   // ---- phase 2: dphi(X) = P state^T + tri(P U^T) Y ----
   if (causal) {
-    float s4[4][4];
     zero(s4);
     for (int e0 = 0; e0 < ddp; e0 += 32) {
-      for (int e = threadIdx.x; e < 64 * 32; e += blockDim.x) {
-        const int i = e >> 5, kk = e & 31;
-        Xs[i * 33 + kk] = Ps[i * ddp + e0 + kk];
-        Ys[i * 33 + kk] = U(t0 + i, e0 + kk);
-      }
+      stage_t(Yk, [&](int j, int kk) { return U(t0 + j, e0 + kk); });
       __syncthreads();
-      fma_tile(Xs, Ys, s4);
+      fma_tile(PsT + e0 * kLd, Yk, s4);
       __syncthreads();
     }
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-#pragma unroll
-      for (int j = 0; j < 4; ++j)
-        Sc[(ty * 4 + i) * 65 + tx * 4 + j] = keep(ty * 4 + i, tx * 4 + j) ? s4[i][j] : 0.f;
+    store_masked(s4);
     __syncthreads();
   }
   const int mr = m + r;
@@ -505,24 +527,21 @@ __global__ void __launch_bounds__(256) pass_kernel(
     float a2[4][4];
     zero(a2);
     for (int e0 = 0; e0 < ddp; e0 += 32) {
-      for (int e = threadIdx.x; e < 64 * 32; e += blockDim.x) {
-        const int i = e >> 5, kk = e & 31;
-        Xs[i * 33 + kk] = Ps[i * ddp + e0 + kk];
-        Ys[i * 33 + kk] = (f0 + i < m && e0 + kk < dd) ? st[(size_t)(f0 + i) * dd + e0 + kk] : 0.f;
-      }
+      stage_t(Yk, [&](int f, int kk) {
+        return (f0 + f < m && e0 + kk < dd) ? st[(size_t)(f0 + f) * dd + e0 + kk] : 0.f;
+      });
       __syncthreads();
-      fma_tile(Xs, Ys, a2);
+      fma_tile(PsT + e0 * kLd, Yk, a2);
       __syncthreads();
     }
     if (causal) {
       for (int k0 = 0; k0 < 64; k0 += 32) {
-        for (int e = threadIdx.x; e < 64 * 32; e += blockDim.x) {
-          const int f = e >> 5, kk = e & 31, t = t0 + k0 + kk;
-          Ys[f * 33 + kk] = (t < L && f0 + f < m) ? Y[(size_t)t * m + f0 + f] : 0.f;
-          Xs[f * 33 + kk] = Sc[f * 65 + k0 + kk];
-        }
+        stage_n(Yk, [&](int kk, int f) {
+          const int t = t0 + k0 + kk;
+          return (t < L && f0 + f < m) ? Y[(size_t)t * m + f0 + f] : 0.f;
+        });
         __syncthreads();
-        fma_tile(Xs, Ys, a2);
+        fma_tile(ScT + k0 * kLd, Yk, a2);
         __syncthreads();
       }
     }
@@ -547,8 +566,8 @@ __global__ void __launch_bounds__(256) dx_kernel(
     const float* __restrict__ w, int heads_w, int m, int r, int d, int H, int L,
     float* __restrict__ cfq, float* __restrict__ cfk, T* __restrict__ dq, T* __restrict__ dk,
     int64_t ob, int64_t oh, int64_t ol, int* dev_status) {
-  __shared__ float As[64 * 33];
-  __shared__ float Bs[64 * 33];
+  __shared__ __align__(16) float As[32 * kLd];
+  __shared__ __align__(16) float Bs[32 * kLd];
   __shared__ float rsum[kT];
   const int side = blockIdx.z;
   const int bh = blockIdx.y, b = bh / H, h = bh % H;
@@ -573,11 +592,12 @@ __global__ void __launch_bounds__(256) dx_kernel(
     for (int c0 = 0; c0 < r; c0 += 64) {
       zero(acc);
       for (int k0 = 0; k0 < d; k0 += 32) {
-        for (int e = threadIdx.x; e < 64 * 32; e += blockDim.x) {
-          const int i = e >> 5, kk = e & 31;
-          As[i * 33 + kk] = (t0 + i < L && k0 + kk < d) ? to_f32(x[(int64_t)(t0 + i) * sl + k0 + kk]) : 0.f;
-          Bs[i * 33 + kk] = (c0 + i < r && k0 + kk < d) ? wh[(size_t)(m + c0 + i) * d + k0 + kk] : 0.f;
-        }
+        stage_t(As, [&](int i, int kk) {
+          return (t0 + i < L && k0 + kk < d) ? to_f32(x[(int64_t)(t0 + i) * sl + k0 + kk]) : 0.f;
+        });
+        stage_t(Bs, [&](int i, int kk) {
+          return (c0 + i < r && k0 + kk < d) ? wh[(size_t)(m + c0 + i) * d + k0 + kk] : 0.f;
+        });
         __syncthreads();
         fma_tile(As, Bs, acc);
         __syncthreads();
@@ -605,12 +625,12 @@ __global__ void __launch_bounds__(256) dx_kernel(
   for (int c0 = 0; c0 < d; c0 += 64) {
     zero(acc);
     for (int k0 = 0; k0 < kend; k0 += 32) {
-      for (int e = threadIdx.x; e < 64 * 32; e += blockDim.x) {
-        const int i = e >> 5, kk = e & 31;
-        As[i * 33 + kk] = (t0 + i < L && k0 + kk < kend) ? cf[(size_t)(t0 + i) * mr + k0 + kk] : 0.f;
-        const int jj = e >> 6, cc = e & 63;     // W' rows k0 + jj, columns c0 + cc
-        Bs[cc * 33 + jj] = (k0 + jj < kend && c0 + cc < d) ? wh[(size_t)(k0 + jj) * d + c0 + cc] : 0.f;
-      }
+      stage_t(As, [&](int i, int kk) {
+        return (t0 + i < L && k0 + kk < kend) ? cf[(size_t)(t0 + i) * mr + k0 + kk] : 0.f;
+      });
+      stage_n(Bs, [&](int kk, int cc) {
+        return (k0 + kk < kend && c0 + cc < d) ? wh[(size_t)(k0 + kk) * d + c0 + cc] : 0.f;
+      });
       __syncthreads();
       fma_tile(As, Bs, acc);
       __syncthreads();
@@ -637,8 +657,8 @@ __global__ void __launch_bounds__(256) dw_kernel(
     const T* __restrict__ xq, const T* __restrict__ xk, int64_t sb, int64_t sh, int64_t sl,
     const float* __restrict__ cfq, const float* __restrict__ cfk, int m, int r, int d, int H,
     int L, int heads_w, int nsplit, float* __restrict__ G) {
-  __shared__ float As[64 * 33];
-  __shared__ float Bs[64 * 33];
+  __shared__ __align__(16) float As[32 * kLd];
+  __shared__ __align__(16) float Bs[32 * kLd];
   const int mr = m + r;
   const int j0 = blockIdx.x * 64, c0 = blockIdx.y * 64;
   const int bh = blockIdx.z / nsplit, split = blockIdx.z % nsplit;
@@ -652,11 +672,14 @@ __global__ void __launch_bounds__(256) dw_kernel(
     const T* x = (side ? xk : xq) + (int64_t)b * sb + (int64_t)h * sh;
     const float* cf = (side ? cfk : cfq) + (size_t)bh * L * mr;
     for (int k0 = tb; k0 < te; k0 += 32) {
-      for (int e = threadIdx.x; e < 32 * 64; e += blockDim.x) {
-        const int tt = e >> 6, f = e & 63, t = k0 + tt;
-        As[f * 33 + tt] = (t < te && j0 + f < mr) ? cf[(size_t)t * mr + j0 + f] : 0.f;
-        Bs[f * 33 + tt] = (t < te && c0 + f < d) ? to_f32(x[(int64_t)t * sl + c0 + f]) : 0.f;
-      }
+      stage_n(As, [&](int kk, int f) {
+        const int t = k0 + kk;
+        return (t < te && j0 + f < mr) ? cf[(size_t)t * mr + j0 + f] : 0.f;
+      });
+      stage_n(Bs, [&](int kk, int f) {
+        const int t = k0 + kk;
+        return (t < te && c0 + f < d) ? to_f32(x[(int64_t)t * sl + c0 + f]) : 0.f;
+      });
       __syncthreads();
       fma_tile(As, Bs, acc);
       __syncthreads();
@@ -696,9 +719,49 @@ __global__ void dgeom_kernel(const float* __restrict__ G, const float* __restric
   }
 }
 
-size_t pass_smem_bytes(int d) {
-  const int ddp = ((d + 1 + 63) / 64) * 64;
-  return sizeof(float) * (64 * 33 * 2 + 64 * 65 + 32 * ddp + 64 * ddp + 64);
+size_t pass_smem_bytes(int et) {
+  const int ddp = et * 64;
+  return sizeof(float) * (32 * kLd * 2 + 64 * kLd + 32 * ddp + ddp * kLd + 64);
+}
+
+struct PassArgs {
+  const float *phiq, *phik, *state;
+  const void* v;
+  int64_t vb, vh, vl;
+  const void* g;
+  int64_t gb, gh, gl;
+  float* wq;
+  void* dv;
+  int64_t ob, oh, ol;
+  float* coef;
+  int m, r, d, H, L, nt, causal;
+  int* dev_status;
+};
+
+template <typename T, int SIDE, int ET>
+cudaError_t launch_pass_et(const PassArgs& p, dim3 grid, cudaStream_t stream) {
+  static int smem_set[64];
+  const size_t bytes = pass_smem_bytes(ET);
+  cudaError_t err = set_smem_limit_once((const void*)pass_kernel<T, SIDE, ET>, (int)bytes, smem_set);
+  if (err != cudaSuccess) return err;
+  pass_kernel<T, SIDE, ET><<<grid, 256, bytes, stream>>>(
+      p.phiq, p.phik, p.state, (const T*)p.v, p.vb, p.vh, p.vl, (const T*)p.g, p.gb, p.gh, p.gl,
+      p.wq, (T*)p.dv, p.ob, p.oh, p.ol, p.coef, p.m, p.r, p.d, p.H, p.L, p.nt, p.causal,
+      p.dev_status);
+  return cudaGetLastError();
+}
+
+// ET = ceil((d + 1) / 64) column blocks; d <= 256 gives at most 5.
+template <typename T, int SIDE>
+cudaError_t launch_pass(const PassArgs& p, dim3 grid, cudaStream_t stream) {
+  switch ((p.d + 1 + 63) / 64) {
+    case 1: return launch_pass_et<T, SIDE, 1>(p, grid, stream);
+    case 2: return launch_pass_et<T, SIDE, 2>(p, grid, stream);
+    case 3: return launch_pass_et<T, SIDE, 3>(p, grid, stream);
+    case 4: return launch_pass_et<T, SIDE, 4>(p, grid, stream);
+    case 5: return launch_pass_et<T, SIDE, 5>(p, grid, stream);
+    default: return cudaErrorInvalidValue;
+  }
 }
 
 template <typename T>
@@ -740,22 +803,23 @@ cudaError_t backward_t(const BwdArgs& a) {
       phik, ValuesOnes<T>{v, a.xs[0], a.xs[1], a.xs[2], a.H, d}, m, d, L, nt, cs);
   tile_scan_kernel<<<scan_grid, 256, 0, a.stream>>>(cs, n_st, nt, causal ? 0 : 2);
 
-  const size_t psm = pass_smem_bytes(d);
-  // the opt-in is set once per device, for the largest head (d = 256)
-  static int smem_set[2][64];
-  err = set_smem_limit_once((const void*)pass_kernel<T, 0>, (int)pass_smem_bytes(256), smem_set[0]);
+  PassArgs pa{phiq, phik, cs, v, a.xs[0], a.xs[1], a.xs[2], a.dout, a.gs[0], a.gs[1], a.gs[2],
+              wq, nullptr, 0, 0, 0, cfq, m, r, d, a.H, L, nt, causal, a.dev_status};
+  err = launch_pass<T, 0>(pa, dim3(nt, bh), a.stream);
   if (err != cudaSuccess) return err;
-  err = set_smem_limit_once((const void*)pass_kernel<T, 1>, (int)pass_smem_bytes(256), smem_set[1]);
-  if (err != cudaSuccess) return err;
-  pass_kernel<T, 0><<<dim3(nt, bh), 256, psm, a.stream>>>(
-      phiq, phik, cs, v, a.xs[0], a.xs[1], a.xs[2], (const T*)a.dout, a.gs[0], a.gs[1], a.gs[2],
-      wq, nullptr, 0, 0, 0, cfq, m, r, d, a.H, L, nt, causal, a.dev_status);
   chunk_state_kernel<StoredRows><<<dim3(nt, bh), 256, 0, a.stream>>>(
       phiq, StoredRows{wq, L, d + 1}, m, d, L, nt, dsn);
   tile_scan_kernel<<<scan_grid, 256, 0, a.stream>>>(dsn, n_st, nt, causal ? 1 : 2);
-  pass_kernel<T, 1><<<dim3(nt, bh), 256, psm, a.stream>>>(
-      phiq, phik, dsn, v, a.xs[0], a.xs[1], a.xs[2], nullptr, 0, 0, 0, wq, (T*)a.dv, a.ds[0],
-      a.ds[1], a.ds[2], cfk, m, r, d, a.H, L, nt, causal, a.dev_status);
+  pa.state = dsn;
+  pa.g = nullptr;
+  pa.gb = pa.gh = pa.gl = 0;
+  pa.dv = a.dv;
+  pa.ob = a.ds[0];
+  pa.oh = a.ds[1];
+  pa.ol = a.ds[2];
+  pa.coef = cfk;
+  err = launch_pass<T, 1>(pa, dim3(nt, bh), a.stream);
+  if (err != cudaSuccess) return err;
   dx_kernel<T><<<dim3(nt, bh, 2), 256, 0, a.stream>>>(
       q, k, a.xs[0], a.xs[1], a.xs[2], wf, a.heads_w, m, r, d, a.H, L, cfq, cfk, (T*)a.dq,
       (T*)a.dk, a.ds[0], a.ds[1], a.ds[2], a.dev_status);
