@@ -326,3 +326,41 @@ def attention_backward(q, k, v, omega, geom, dout, key_mask=None, causal=False):
                 ghm += du.T @ xs
             dgeom[0 if geom.shape[0] == 1 else h] += ghm
     return dq, dk, dv, dgeom
+
+
+def exact_attention(q, k, v, geom, key_mask=None, causal=False):
+    """The learned kernel evaluated exactly (README, "Attention modes": the exact
+    path applies the learned geometry to queries and keys before scaled dot-product
+    attention): out_i = sum_j softmax_j(u_i . w_j) v_j with u = M q~, w = M k~,
+    x~ = d^{-1/4} x, so the scores are q^T Sigma k / sqrt(d), over the valid keys
+    (and j <= i when causal). A row with no visible key outputs 0.
+
+    q, k, v: [B, H, L, d]; geom: [H_m, r, d]; key_mask: [B, L] or None.
+    """
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    B, H, L, d = q.shape
+    out = np.zeros((B, H, L, d))
+    s = d ** -0.25
+    for b in range(B):
+        valid = np.ones(L, bool) if key_mask is None else np.asarray(key_mask[b]) != 0
+        for h in range(H):
+            gm = _f64(_head(geom, h))
+            u = (q[b, h] * s) @ gm.T
+            w = (k[b, h] * s) @ gm.T
+            scores = u @ w.T
+            keep = np.broadcast_to(valid[None, :], (L, L)).copy()
+            if causal:
+                keep &= np.tril(np.ones((L, L), bool))
+            for i in range(L):
+                if not keep[i].any():
+                    continue
+                z = scores[i][keep[i]]
+                p = np.exp(z - z.max())
+                out[b, h, i] = (p / p.sum()) @ v[b, h][keep[i]]
+    return out
+
+
+def uses_exact(L: int, exact_threshold: int) -> bool:
+    """Auto mode (README, "Attention modes"): exact attention through the
+    threshold, linear attention above it."""
+    return exact_threshold > 0 and L <= exact_threshold
