@@ -836,6 +836,49 @@ def run_backward(args, w: synth.Workload, rank: int, world: int, dev) -> dict | 
     }
 
 
+SAMPLE_METRIC = "DARK projection draw (orthogonal Omega, Philox4x64-10) draws/s on 1 B200"
+
+
+def run_sample(args, rank: int, world: int, dev) -> dict | None:
+    """Device draws of an orthogonal Omega for the causal workload's shape (m 256,
+    r 64) and the large-head workload's (m 512, r 256): CUDA events around each
+    draw (Gaussians, fp64 Gram-Schmidt per block, scaled rows)."""
+    from random_feature_linear_b200 import dark as D
+    res = {}
+    launches = 0
+    for name, m, r in (("m256 r64", 256, 64), ("m512 r256", 512, 256)):
+        om = torch.empty(1, m, r, dtype=torch.float32, device=dev)
+        ws = torch.empty(max(D.dark_sample_omega_workspace_bytes(1, m, r, True), 256),
+                         dtype=torch.uint8, device=dev)
+        for i in range(args.warmup):
+            D.dark_sample_omega(1, i, om, ws=ws)
+        torch.cuda.synchronize()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(args.steps)]
+        for i, (a, b) in enumerate(ev):
+            a.record()
+            D.dark_sample_omega(1, 1000 + i, om, ws=ws)
+            b.record()
+        torch.cuda.synchronize()
+        ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in ev) / args.steps, dev)
+        res[name] = ms
+        launches += 3 * args.steps
+    if rank != 0:
+        return None
+    main = res["m256 r64"]
+    return {
+        "metric": SAMPLE_METRIC, "value": world / (main / 1e3), "unit": "draws/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": main,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (counter-based generator)",
+        "config": {"workload": "orthogonal Omega draw, m 256 r 64 (one head); also m 512 r 256",
+                   "ms_per_draw": res,
+                   "timing": "CUDA events around each draw; one draw per step"},
+        "roofline": None,
+        "gpu_launches": launches,
+    }
+
+
 def run_reference(args, w: synth.Workload) -> dict:
     inp = synth.make_inputs(w)
     for _ in range(args.warmup):
@@ -877,6 +920,8 @@ def main():
                     help="do not count launches with the CUDA profiler (for runs under ncu)")
     ap.add_argument("--decode", action="store_true",
                     help="time the streaming decode step (workload 5) instead of the forward")
+    ap.add_argument("--sample", action="store_true",
+                    help="time device draws of an orthogonal projection instead")
     ap.add_argument("--backward", action="store_true",
                     help="time the backward pass of --workload instead of the forward")
     ap.add_argument("--cross", action="store_true",
@@ -907,6 +952,8 @@ def main():
             res = run_cross(args, rank, world, dev)
         elif args.backward:
             res = run_backward(args, w, rank, world, dev)
+        elif args.sample:
+            res = run_sample(args, rank, world, dev)
         else:
             res = run_native(args, w, rank, world, dev)
         if res is not None:

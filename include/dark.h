@@ -1,7 +1,8 @@
 /*
  * dark.h -- C ABI of the B200 (sm_100a) DARKformer positive-random-feature
  * attention library: forward pass (non-causal, causal, key-masked), its
- * backward pass, cross-attention and the streaming decode steps.
+ * backward pass, cross-attention, the streaming decode steps and the projection
+ * sampler with its redraw schedule.
  *
  * Source of the method: the DARKformer README ("Data-Aware Random Feature
  * Kernels for Transformers", darkformer-pytorch 0.1.0 package description).
@@ -42,7 +43,7 @@
 extern "C" {
 #endif
 
-#define DARK_ABI_VERSION 3
+#define DARK_ABI_VERSION 4
 
 typedef enum {
   DARK_OK = 0,
@@ -308,6 +309,60 @@ dark_status dark_attention_bwd(const float* omega, int heads_omega, const float*
                                const uint8_t* key_mask, int flags, void* dq, void* dk, void* dv,
                                const int64_t* grad_strides, float* dgeom, void* ws,
                                size_t ws_bytes, int* dev_status, void* stream);
+
+/*
+ * Projection sampler: Omega drawn on the device, reproducibly from (seed, draw).
+ * README, section "Kernel": omega_j ~ N(0, I_r); section "Self-attention":
+ * orthogonal Gaussian blocks by default, independent Gaussian features when
+ * orthogonal_features=False; section "Projection lifecycle": projection_seed makes
+ * the draws reproducible.
+ *
+ * Generator (the pages fix none): Philox4x64-10 with key (seed, draw) and counter
+ * (block, head, purpose, 0); the block's four 64-bit words give two Box-Muller pairs
+ * (u1 = 1 - u(x_a), u2 = u(x_b), u(x) = (x >> 11) 2^-53). Stream element e of
+ * (head, purpose) is word e % 4 of block e / 4.
+ *   independent: Omega[h][j][i] = z(h, 0, j r + i);
+ *   orthogonal:  per block b of r rows, G[i][k] = z(h, 0, b r^2 + i r + k), G = Q R
+ *                with diag(R) > 0 (fp64 Gram-Schmidt with re-orthogonalisation),
+ *                row i = ||(z(h, 1, b r^2 + i r + k))_k|| * Q[:, i]; a partial last
+ *                block keeps its first rows.
+ *   omega     device fp32 [heads][m][r], written
+ *   ws        device workspace of dark_sample_omega_workspace_bytes(...) bytes,
+ *             256-byte aligned (none needed for independent features: NULL is fine)
+ * Errors: DARK_ERR_INVALID_ARG for a null or misaligned pointer, bad sizes or a
+ * short workspace; DARK_ERR_UNSUPPORTED for m > 1024, r > 256 or heads > 65535;
+ * DARK_ERR_CUDA for a failed launch.
+ */
+size_t dark_sample_omega_workspace_bytes(int heads, int m, int r, int orthogonal);
+dark_status dark_sample_omega(uint64_t seed, uint64_t draw, int heads, int m, int r,
+                              int orthogonal, float* omega, void* ws, size_t ws_bytes,
+                              void* stream);
+
+/*
+ * Redraw schedule of one projection (host only; README, section "Projection
+ * lifecycle"). The current projection is dark_sample_omega(seed, draw, ...).
+ *   interval > 0: a redraw falls due after that many training forwards and happens
+ *   at the start of the next training forward; evaluation forwards do not count;
+ *   interval <= 0: no scheduled redraws. While fixed, a redraw falling due is
+ *   dropped (the interval restarts) and ordinary requests are refused; a forced
+ *   request redraws once. Every redraw restarts the interval. deterministic != 0
+ *   fixes the projection at construction.
+ */
+typedef struct dark_redraw_schedule {
+  uint64_t seed;       /* projection seed */
+  uint64_t draw;       /* redraws so far: the current projection's draw index */
+  int64_t interval;    /* training forwards between scheduled redraws; 0: none */
+  int64_t count;       /* training forwards since the interval last restarted */
+  int fixed;           /* 1: ordinary redraws are ignored */
+} dark_redraw_schedule;
+
+dark_status dark_redraw_schedule_init(dark_redraw_schedule* s, uint64_t seed, int64_t interval,
+                                      int deterministic);
+/* At the start of a forward: 1 if a redraw happened (draw advanced), else 0. */
+int dark_redraw_on_forward(dark_redraw_schedule* s, int training);
+/* A manual redraw request: 1 if granted (draw advanced), else 0. */
+int dark_redraw_request(dark_redraw_schedule* s, int force);
+void dark_redraw_set_fixed(dark_redraw_schedule* s, int fixed);
 
 #ifdef __cplusplus
 }

@@ -347,6 +347,61 @@ dark_status dark_attention_bwd(const float* omega, int heads_omega, const float*
   return from_cuda(dark::launch_backward(a));
 }
 
+size_t dark_sample_omega_workspace_bytes(int heads, int m, int r, int orthogonal) {
+  if (heads < 1 || m < 1 || r < 1 || m > kMaxM || r > kMaxR) return 0;
+  return dark::omega_workspace_bytes(heads, m, r, orthogonal);
+}
+
+dark_status dark_sample_omega(uint64_t seed, uint64_t draw, int heads, int m, int r,
+                              int orthogonal, float* omega, void* ws, size_t ws_bytes,
+                              void* stream) {
+  if (omega == nullptr || !aligned(omega, 4) || heads < 1 || m < 1 || r < 1)
+    return DARK_ERR_INVALID_ARG;
+  if (m > kMaxM || r > kMaxR || heads > 65535) return DARK_ERR_UNSUPPORTED;
+  if (orthogonal) {
+    const size_t need = dark::omega_workspace_bytes(heads, m, r, 1);
+    if (ws == nullptr || !aligned(ws, 256) || ws_bytes < need) return DARK_ERR_INVALID_ARG;
+  }
+  return from_cuda(dark::launch_sample_omega(seed, draw, heads, m, r, orthogonal ? 1 : 0, omega,
+                                             ws, (cudaStream_t)stream));
+}
+
+dark_status dark_redraw_schedule_init(dark_redraw_schedule* s, uint64_t seed, int64_t interval,
+                                      int deterministic) {
+  if (s == nullptr) return DARK_ERR_INVALID_ARG;
+  s->seed = seed;
+  s->draw = 0;
+  s->interval = interval > 0 ? interval : 0;
+  s->count = 0;
+  s->fixed = deterministic ? 1 : 0;
+  return DARK_OK;
+}
+
+int dark_redraw_on_forward(dark_redraw_schedule* s, int training) {
+  if (s == nullptr || !training) return 0;
+  int redrew = 0;
+  if (s->interval > 0 && s->count >= s->interval) {
+    s->count = 0;                 // a redraw falling due while fixed is dropped
+    if (!s->fixed) {
+      ++s->draw;
+      redrew = 1;
+    }
+  }
+  ++s->count;
+  return redrew;
+}
+
+int dark_redraw_request(dark_redraw_schedule* s, int force) {
+  if (s == nullptr || (s->fixed && !force)) return 0;
+  ++s->draw;
+  s->count = 0;
+  return 1;
+}
+
+void dark_redraw_set_fixed(dark_redraw_schedule* s, int fixed) {
+  if (s != nullptr) s->fixed = fixed ? 1 : 0;
+}
+
 dark_status dark_state_init(const dark_projection* proj, dark_state* st, void* stream) {
   if (proj == nullptr || st == nullptr || st->kv == nullptr || st->z == nullptr)
     return DARK_ERR_INVALID_ARG;

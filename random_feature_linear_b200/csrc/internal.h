@@ -130,4 +130,10 @@ struct BwdArgs {
 size_t bwd_workspace_bytes(int B, int H, int L, int m, int r, int d, int heads_w);
 cudaError_t launch_backward(const BwdArgs& a);
 
+// Projection sampler (Philox4x64-10 + Box-Muller; orthogonal blocks by fp64
+// Gram-Schmidt).
+size_t omega_workspace_bytes(int heads, int m, int r, int orthogonal);
+cudaError_t launch_sample_omega(uint64_t seed, uint64_t draw, int heads, int m, int r,
+                                int orthogonal, float* omega, void* ws, cudaStream_t stream);
+
 }  // namespace dark

@@ -31,7 +31,9 @@ EXPORTS = ("dark_abi_version", "dark_status_string", "dark_projection_bytes",
            "dark_state_init", "dark_decode_step", "dark_noalloc_scratch_bytes",
            "dark_attention_fwd_noalloc", "dark_cross_attention_workspace_bytes",
            "dark_cross_attention_fwd", "dark_cross_decode_step",
-           "dark_attention_bwd_workspace_bytes", "dark_attention_bwd")
+           "dark_attention_bwd_workspace_bytes", "dark_attention_bwd",
+           "dark_sample_omega_workspace_bytes", "dark_sample_omega", "dark_redraw_schedule_init",
+           "dark_redraw_on_forward", "dark_redraw_request", "dark_redraw_set_fixed")
 
 
 class dark_projection(ctypes.Structure):
@@ -44,6 +46,11 @@ class dark_state(ctypes.Structure):
     _fields_ = [("kv", ctypes.c_void_p), ("z", ctypes.c_void_p), ("shift", ctypes.c_void_p),
                 ("B", ctypes.c_int), ("H", ctypes.c_int), ("m", ctypes.c_int), ("d", ctypes.c_int),
                 ("generation", ctypes.c_uint64)]
+
+
+class dark_redraw_schedule(ctypes.Structure):
+    _fields_ = [("seed", ctypes.c_uint64), ("draw", ctypes.c_uint64),
+                ("interval", ctypes.c_int64), ("count", ctypes.c_int64), ("fixed", ctypes.c_int)]
 
 
 _P = ctypes.POINTER
@@ -81,6 +88,20 @@ _lib.dark_cross_attention_fwd.argtypes = [_P(dark_projection), _vp, _P(ctypes.c_
                                           _sz, _vp, _vp]
 _lib.dark_cross_decode_step.restype = _i
 _lib.dark_cross_decode_step.argtypes = [_P(dark_projection), _P(dark_state), _vp, _vp, _vp, _vp]
+_lib.dark_sample_omega_workspace_bytes.restype = _sz
+_lib.dark_sample_omega_workspace_bytes.argtypes = [_i, _i, _i, _i]
+_lib.dark_sample_omega.restype = _i
+_lib.dark_sample_omega.argtypes = [ctypes.c_uint64, ctypes.c_uint64, _i, _i, _i, _i, _vp, _vp, _sz,
+                                   _vp]
+_lib.dark_redraw_schedule_init.restype = _i
+_lib.dark_redraw_schedule_init.argtypes = [_P(dark_redraw_schedule), ctypes.c_uint64,
+                                           ctypes.c_int64, _i]
+_lib.dark_redraw_on_forward.restype = _i
+_lib.dark_redraw_on_forward.argtypes = [_P(dark_redraw_schedule), _i]
+_lib.dark_redraw_request.restype = _i
+_lib.dark_redraw_request.argtypes = [_P(dark_redraw_schedule), _i]
+_lib.dark_redraw_set_fixed.restype = None
+_lib.dark_redraw_set_fixed.argtypes = [_P(dark_redraw_schedule), _i]
 _lib.dark_attention_bwd_workspace_bytes.restype = _sz
 _lib.dark_attention_bwd_workspace_bytes.argtypes = [_i] * 8
 _lib.dark_attention_bwd.restype = _i
@@ -302,6 +323,50 @@ def alloc_workspace(proj: dark_projection, B: int, H: int, L: int, flags: int, d
     """A zero-filled workspace of the size dark_attention_workspace_bytes asks for."""
     n = dark_attention_workspace_bytes(proj, B, H, L, flags)
     return torch.zeros(max(n, WS_HEADER_BYTES), dtype=torch.uint8, device=device)
+
+
+def dark_sample_omega_workspace_bytes(heads: int, m: int, r: int, orthogonal: bool) -> int:
+    return _lib.dark_sample_omega_workspace_bytes(heads, m, r, int(orthogonal))
+
+
+def dark_sample_omega(seed: int, draw: int, omega, orthogonal: bool = True, ws=None,
+                      stream=None) -> None:
+    """Fills the fp32 device tensor omega [heads, m, r] from (seed, draw)."""
+    _dense(omega, "omega")
+    assert omega.dtype == torch.float32 and omega.dim() == 3
+    heads, m, r = omega.shape
+    if orthogonal and ws is None:
+        n = dark_sample_omega_workspace_bytes(heads, m, r, True)
+        ws = torch.empty(max(n, 256), dtype=torch.uint8, device=omega.device)
+    _check(_lib.dark_sample_omega(seed, draw, heads, m, r, int(orthogonal), _ptr(omega), _ptr(ws),
+                                  0 if ws is None else ws.numel() * ws.element_size(),
+                                  _stream(stream)))
+
+
+class RedrawSchedule:
+    """The library's redraw schedule (dark_redraw_schedule) with Python method names."""
+
+    def __init__(self, seed: int, interval: int | None = None, deterministic: bool = False):
+        self.s = dark_redraw_schedule()
+        _check(_lib.dark_redraw_schedule_init(ctypes.byref(self.s), seed,
+                                              0 if interval is None else interval,
+                                              int(deterministic)))
+
+    @property
+    def draw(self) -> int:
+        return self.s.draw
+
+    def forward(self, training: bool) -> bool:
+        return bool(_lib.dark_redraw_on_forward(ctypes.byref(self.s), int(training)))
+
+    def redraw(self, force: bool = False) -> bool:
+        return bool(_lib.dark_redraw_request(ctypes.byref(self.s), int(force)))
+
+    def fix(self) -> None:
+        _lib.dark_redraw_set_fixed(ctypes.byref(self.s), 1)
+
+    def unfix(self) -> None:
+        _lib.dark_redraw_set_fixed(ctypes.byref(self.s), 0)
 
 
 def torch_dtype(dtype: int):

@@ -173,3 +173,47 @@ def test_backward_rejects_bad_arguments(D):
     # workspace size: zero for bad sizes, growing with L
     assert D.dark_attention_bwd_workspace_bytes(1, 2, 64, 32, 64, 0, 2, 100) == 0
     assert need < D.dark_attention_bwd_workspace_bytes(1, 2, 64, 32, 64, 2, 2, 1000)
+
+
+def test_redraw_schedule_matches_oracle(D):
+    # random sequences of forwards (training or evaluation), manual and forced
+    # redraws, fix and unfix: the library's schedule and the oracle's take the
+    # same decisions
+    import random
+
+    from oracle import dark_sampler as S
+    rng = random.Random(5)
+    for trial in range(40):
+        interval = rng.choice([None, 1, 2, 3, 5])
+        det = rng.random() < 0.2
+        lib, ref = D.RedrawSchedule(9, interval, det), S.RedrawSchedule(9, interval, det)
+        for _ in range(60):
+            op = rng.randrange(6)
+            if op <= 2:
+                tr = op != 2
+                assert lib.forward(tr) == ref.forward(tr)
+            elif op == 3:
+                f = rng.random() < 0.3
+                assert lib.redraw(f) == ref.redraw(f)
+            elif op == 4:
+                lib.fix()
+                ref.fix()
+            else:
+                lib.unfix()
+                ref.unfix()
+            assert lib.draw == ref.draw
+
+
+def test_sampler_rejects_bad_arguments(D):
+    lib = D._lib
+    f = 0x10000
+    need = D.dark_sample_omega_workspace_bytes(1, 256, 64, True)
+    assert need > 0 and D.dark_sample_omega_workspace_bytes(1, 256, 64, False) == 0
+    assert lib.dark_sample_omega(1, 0, 1, 256, 64, 1, None, f, need, None) == 1
+    assert lib.dark_sample_omega(1, 0, 1, 256, 64, 1, f + 2, f, need, None) == 1
+    assert lib.dark_sample_omega(1, 0, 0, 256, 64, 1, f, f, need, None) == 1
+    assert lib.dark_sample_omega(1, 0, 1, 256, 64, 1, f, None, need, None) == 1
+    assert lib.dark_sample_omega(1, 0, 1, 256, 64, 1, f, f, need - 8, None) == 1
+    assert lib.dark_sample_omega(1, 0, 1, 256, 64, 1, f, f + 16, need, None) == 1
+    assert lib.dark_sample_omega(1, 0, 1, 256, 512, 1, f, f, 1 << 40, None) == 2
+    assert lib.dark_sample_omega(1, 0, 1, 4096, 64, 0, f, None, 0, None) == 2
