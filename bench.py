@@ -152,7 +152,7 @@ class ClockSampler:
                 "samples": len(self.samples)}
 
 
-def oracle_sample(w: synth.Workload, inp: dict, max_seconds: float = 20.0):
+def oracle_sample(w: synth.Workload, inp: dict, max_seconds: float = 20.0, exact: bool = False):
     """Times the fp64 oracle on whole (batch, head) slices of the workload until
     about `max_seconds` of CPU work; returns (tokens/s, tokens, seconds, heads)."""
     from oracle import dark_oracle as O
@@ -163,8 +163,12 @@ def oracle_sample(w: synth.Workload, inp: dict, max_seconds: float = 20.0):
             geom = inp["geom"][h:h + 1] if inp["geom"].shape[0] > 1 else inp["geom"]
             mask = None if inp["mask"] is None else inp["mask"][b:b + 1]
             t0 = time.perf_counter()
-            O.attention(inp["q"][sl], inp["k"][sl], inp["v"][sl], inp["omega"], geom,
-                        key_mask=mask, causal=w.causal)
+            if exact:
+                O.exact_attention(inp["q"][sl], inp["k"][sl], inp["v"][sl], geom,
+                                  key_mask=mask, causal=w.causal)
+            else:
+                O.attention(inp["q"][sl], inp["k"][sl], inp["v"][sl], inp["omega"], geom,
+                            key_mask=mask, causal=w.causal)
             t_total += time.perf_counter() - t0
             done_tokens += w.L
             heads += 1
@@ -204,7 +208,7 @@ def run_native(args, w: synth.Workload, rank: int, world: int, dev) -> dict | No
     q, k, v = (torch.from_numpy(inp[n]).to(dev).to(tdt) for n in ("q", "k", "v"))
     mask = None if inp["mask"] is None else torch.from_numpy(inp["mask"]).to(dev)
     out = torch.empty_like(q)
-    flags = D.DARK_CAUSAL if w.causal else 0
+    flags = (D.DARK_CAUSAL if w.causal else 0) | (D.DARK_EXACT if args.exact else 0)
     ws = D.alloc_workspace(proj, w.B, w.H, w.L, flags, dev)
     status = torch.zeros(1, dtype=torch.int32, device=dev)
     flush = None if args.ncu else torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.int32, device=dev)
@@ -306,28 +310,36 @@ def run_native(args, w: synth.Workload, rank: int, world: int, dev) -> dict | No
     nbytes = alg_bytes(w)
     t_tc = flops / (peaks["bf16"] * 1e12)
     t_hbm = nbytes / (peaks["hbm"] * 1e9)
-    bound = "tensor" if t_tc >= t_hbm else "hbm"
-    if bound == "tensor":
+    if args.exact:
+        flops = exact_flops(w)
         achieved = flops / t_kernel / 1e12
-        roof = dict(bound="tensor", achieved=achieved, peak=peaks["bf16"], unit="TFLOP/s",
-                    frac=achieved / peaks["bf16"], traffic=None)
+        roof = dict(bound="alu", achieved=achieved, peak=FFMA_TFLOPS, unit="TFLOP/s",
+                    frac=achieved / FFMA_TFLOPS, traffic=None,
+                    peak_source="derived: 148 SMs x 128 FP32 lanes x 2 x 1.965 GHz",
+                    kernel="exact-mode call (SIMT fp32)")
     else:
-        achieved = nbytes / t_kernel / 1e9
-        roof = dict(bound="hbm", achieved=achieved, peak=peaks["hbm"], unit="GB/s",
-                    frac=achieved / peaks["hbm"], traffic=None)
-    roof["peak_source"] = peaks["source"] + " (burst)"
-    short = sorted({k.replace("(anonymous namespace)::", "").split("(")[0].split("<")[0].split("::")[-1]
-                    for k in kernel_names if "dark::" in k})
-    roof["kernel"] = "forward call" + (" (" + ", ".join(short) + ")" if short else "")
-    roof["traffic"] = captured_traffic(args.workload)
+        bound = "tensor" if t_tc >= t_hbm else "hbm"
+        if bound == "tensor":
+            achieved = flops / t_kernel / 1e12
+            roof = dict(bound="tensor", achieved=achieved, peak=peaks["bf16"], unit="TFLOP/s",
+                        frac=achieved / peaks["bf16"], traffic=None)
+        else:
+            achieved = nbytes / t_kernel / 1e9
+            roof = dict(bound="hbm", achieved=achieved, peak=peaks["hbm"], unit="GB/s",
+                        frac=achieved / peaks["hbm"], traffic=None)
+        roof["peak_source"] = peaks["source"] + " (burst)"
+        short = sorted({k.replace("(anonymous namespace)::", "").split("(")[0].split("<")[0].split("::")[-1]
+                        for k in kernel_names if "dark::" in k})
+        roof["kernel"] = "forward call" + (" (" + ", ".join(short) + ")" if short else "")
+        roof["traffic"] = captured_traffic(args.workload)
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
-        tps, ntok, secs, heads = oracle_sample(w, inp)
+        tps, ntok, secs, heads = oracle_sample(w, inp, exact=args.exact)
         cpu = dict(value=tps, unit="tokens/s", cores=blas_threads(), kind="oracle",
                    sample=f"{heads} of {w.B * w.H} (batch, head) slices, {ntok} tokens, {secs:.1f} s")
     clocks = clk.summary()
     return {
-        "metric": METRIC,
+        "metric": EXACT_METRIC if args.exact else METRIC,
         "value": tokens / (ms_per_step / 1e3),
         "unit": "tokens/s",
         "n_gpus": world,
@@ -339,7 +351,8 @@ def run_native(args, w: synth.Workload, rank: int, world: int, dev) -> dict | No
         "vs_baseline": None,
         "dtype": "bf16" if w.dtype == "bf16" else "f32",
         "data": "synthetic (seeded numpy, orthogonal Gaussian features)",
-        "config": {"workload": w.name, "B": w.B, "H": w.H, "L": w.L, "d": w.d, "r": w.r, "m": w.m,
+        "config": {"workload": ("exact mode: " if args.exact else "") + w.name, "B": w.B, "H": w.H,
+                   "L": w.L, "d": w.d, "r": w.r, "m": w.m,
                    "causal": w.causal, "lengths": list(w.lengths) if w.lengths else None,
                    "l2": "flushed (512 MiB write) before every timed step",
                    "timing": "CUDA events around one CUDA-graph replay of the forward call per step",
@@ -680,6 +693,17 @@ def run_cross(args, rank: int, world: int, dev) -> dict | None:
     }
 
 
+EXACT_METRIC = ("DARK exact learned-kernel attention fwd tokens/s (B·H·L/s) on 1 B200; "
+                "% of FP32-FFMA roofline")
+
+
+def exact_flops(w: synth.Workload) -> float:
+    """Exact mode per head: projections 2·2Ldr, then per visible (query, key) pair
+    2r (score) + 2d (P V); L^2/2 pairs when causal."""
+    pairs = w.L * (w.L + 1) / 2 if w.causal else w.L * w.L
+    return float((4 * w.L * w.d * w.r + pairs * 2 * (w.r + w.d)) * w.B * w.H)
+
+
 BWD_METRIC = ("DARK attention bwd tokens/s (B·H·L/s, dq dk dv dM) on 1 B200; "
               "% of FP32-FFMA roofline")
 # fp32 FFMA peak: 148 SMs x 128 lanes x 2 FLOP x 1.965 GHz (the backward kernels
@@ -920,6 +944,8 @@ def main():
                     help="do not count launches with the CUDA profiler (for runs under ncu)")
     ap.add_argument("--decode", action="store_true",
                     help="time the streaming decode step (workload 5) instead of the forward")
+    ap.add_argument("--exact", action="store_true",
+                    help="time the exact learned-kernel mode of --workload instead")
     ap.add_argument("--sample", action="store_true",
                     help="time device draws of an orthogonal projection instead")
     ap.add_argument("--backward", action="store_true",

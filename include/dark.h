@@ -43,7 +43,7 @@
 extern "C" {
 #endif
 
-#define DARK_ABI_VERSION 4
+#define DARK_ABI_VERSION 5
 
 typedef enum {
   DARK_OK = 0,
@@ -59,7 +59,8 @@ typedef enum { DARK_F32 = 0, DARK_BF16 = 1 } dark_dtype;
 
 enum {
   DARK_CAUSAL = 1,     /* key j is visible to query i only if j <= i (diagonal included) */
-  DARK_STABILISE = 2   /* overflow guard; see dark_attention_fwd                          */
+  DARK_STABILISE = 2,  /* overflow guard; see dark_attention_fwd                          */
+  DARK_EXACT = 4       /* the learned kernel evaluated exactly (softmax); see below        */
 };
 
 /*
@@ -309,6 +310,25 @@ dark_status dark_attention_bwd(const float* omega, int heads_omega, const float*
                                const uint8_t* key_mask, int flags, void* dq, void* dk, void* dv,
                                const int64_t* grad_strides, float* dgeom, void* ws,
                                size_t ws_bytes, int* dev_status, void* stream);
+
+/*
+ * Exact mode (README, section "Attention modes": the exact path applies the
+ * learned geometry to queries and keys before scaled dot-product attention).
+ * DARK_EXACT in the flags of dark_attention_fwd, dark_attention_fwd_noalloc or
+ * dark_cross_attention_fwd evaluates
+ *   out_i = sum_j softmax_j(u_i . w_j) v_j,  u = M q~, w = M k~, x~ = d^{-1/4} x,
+ * (scores q^T Sigma k / sqrt(d)) over the valid keys (j <= i with DARK_CAUSAL)
+ * instead of the random-feature estimate. M is read from the projection's last r
+ * rows (c_m M); Omega is not used. A query row with no visible key outputs 0.
+ * state_out / context_out must be NULL (the mode keeps no recurrent statistics);
+ * DARK_STABILISE is accepted and has no effect (the softmax is computed with a
+ * running maximum). The workspace queries account for the flag.
+ *
+ * Auto mode ("exact_threshold"): exact attention through the threshold, linear
+ * attention above it. dark_auto_uses_exact returns 1 when L <= exact_threshold and
+ * exact_threshold > 0; the caller then adds DARK_EXACT.
+ */
+int dark_auto_uses_exact(int L, int exact_threshold);
 
 /*
  * Projection sampler: Omega drawn on the device, reproducibly from (seed, draw).

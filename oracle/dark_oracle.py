@@ -328,31 +328,35 @@ def attention_backward(q, k, v, omega, geom, dout, key_mask=None, causal=False):
     return dq, dk, dv, dgeom
 
 
-def exact_attention(q, k, v, geom, key_mask=None, causal=False):
+def exact_attention(q, k, v, geom, key_mask=None, causal=False, query_mask=None):
     """The learned kernel evaluated exactly (README, "Attention modes": the exact
     path applies the learned geometry to queries and keys before scaled dot-product
     attention): out_i = sum_j softmax_j(u_i . w_j) v_j with u = M q~, w = M k~,
     x~ = d^{-1/4} x, so the scores are q^T Sigma k / sqrt(d), over the valid keys
-    (and j <= i when causal). A row with no visible key outputs 0.
+    (and j <= i when causal). A row with no visible key, or a masked query row,
+    outputs 0.
 
-    q, k, v: [B, H, L, d]; geom: [H_m, r, d]; key_mask: [B, L] or None.
+    q: [B, H, Lq, d]; k, v: [B, H, Lk, d] (Lk = Lq when causal); geom: [H_m, r, d];
+    key_mask: [B, Lk] or None; query_mask: [B, Lq] or None.
     """
     q, k, v = _f64(q), _f64(k), _f64(v)
-    B, H, L, d = q.shape
-    out = np.zeros((B, H, L, d))
+    B, H, Lq, d = q.shape
+    Lk = k.shape[2]
+    out = np.zeros((B, H, Lq, d))
     s = d ** -0.25
     for b in range(B):
-        valid = np.ones(L, bool) if key_mask is None else np.asarray(key_mask[b]) != 0
+        valid = np.ones(Lk, bool) if key_mask is None else np.asarray(key_mask[b]) != 0
+        live = np.ones(Lq, bool) if query_mask is None else np.asarray(query_mask[b]) != 0
         for h in range(H):
             gm = _f64(_head(geom, h))
             u = (q[b, h] * s) @ gm.T
             w = (k[b, h] * s) @ gm.T
             scores = u @ w.T
-            keep = np.broadcast_to(valid[None, :], (L, L)).copy()
+            keep = np.broadcast_to(valid[None, :], (Lq, Lk)).copy()
             if causal:
-                keep &= np.tril(np.ones((L, L), bool))
-            for i in range(L):
-                if not keep[i].any():
+                keep &= np.tril(np.ones((Lq, Lk), bool))
+            for i in range(Lq):
+                if not live[i] or not keep[i].any():
                     continue
                 z = scores[i][keep[i]]
                 p = np.exp(z - z.max())

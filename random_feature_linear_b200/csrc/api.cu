@@ -30,9 +30,10 @@ bool proj_ok(const dark_projection* p) {
          sizes_ok(p->m, p->r, p->d) && p->heads >= 1;
 }
 
-enum class Path { Simt, TcCausal, TcNonCausal, TcWide };
+enum class Path { Simt, TcCausal, TcNonCausal, TcWide, Exact };
 
 Path choose_path(dark::FwdArgs& a) {
+  if (a.flags & DARK_EXACT) return Path::Exact;
   if (a.flags & DARK_CAUSAL) {
     if (dark::tc_causal_supported(a)) return Path::TcCausal;
     if (dark::tc_wide_supported(a)) return Path::TcWide;
@@ -47,6 +48,7 @@ size_t ws_need(Path p, int B, int H, int Lq, int Lk, int m, int r, int d, int fl
     case Path::TcCausal: return dark::tc_causal_workspace_bytes(B, H, Lq, m, d);
     case Path::TcWide: return dark::tc_wide_workspace_bytes(B, H, Lq, m, d, r);
     case Path::TcNonCausal: return dark::tc_noncausal_workspace_bytes(B, H, Lq, Lk, m, d);
+    case Path::Exact: return dark::exact_workspace_bytes(B, H, Lq, Lk, r);
     default: return dark::simt_workspace_bytes(B, H, Lq, Lk, m, d, flags);
   }
 }
@@ -69,7 +71,9 @@ dark_status fwd_prepare_general(const dark_projection* proj, const void* q,
   if (B < 1 || H < 1 || Lq < 1 || Lk < 1) return DARK_ERR_INVALID_ARG;
   if ((flags & DARK_CAUSAL) && Lq != Lk) return DARK_ERR_INVALID_ARG;
   if (!(proj->heads == 1 || proj->heads == H)) return DARK_ERR_INVALID_ARG;
-  if (flags & ~(DARK_CAUSAL | DARK_STABILISE)) return DARK_ERR_INVALID_ARG;
+  if (flags & ~(DARK_CAUSAL | DARK_STABILISE | DARK_EXACT)) return DARK_ERR_INVALID_ARG;
+  // the exact mode keeps no recurrent statistics
+  if ((flags & DARK_EXACT) && state_out != nullptr) return DARK_ERR_INVALID_ARG;
   FwdArgs& a = *out_args;
   memset(&a, 0, sizeof(a));
   a.heads_w = proj->heads;
@@ -136,6 +140,7 @@ dark_status fwd_launch(FwdArgs& a, void* ws, size_t ws_bytes, dark_state* state_
     case Path::TcCausal: e = tc_causal_forward(a); break;
     case Path::TcNonCausal: e = tc_noncausal_forward(a); break;
     case Path::TcWide: e = tc_wide_forward(a); break;
+    case Path::Exact: e = exact_forward(a); break;
     default: e = simt_forward(a); break;
   }
   if (e != cudaSuccess) return DARK_ERR_CUDA;
@@ -197,6 +202,7 @@ dark_status dark_make_projection(const float* omega, int heads_omega, const floa
 size_t dark_attention_workspace_bytes(const dark_projection* proj, int B, int H, int L,
                                       int flags) {
   if (!proj_ok(proj) || B < 1 || H < 1 || L < 1) return 0;
+  if (flags & DARK_EXACT) return dark::exact_workspace_bytes(B, H, L, L, proj->r);
   const int m = proj->m, d = proj->d;
   size_t need = dark::simt_workspace_bytes(B, H, L, L, m, d, flags);
   const size_t tc = (flags & DARK_CAUSAL) ? dark::tc_causal_workspace_bytes(B, H, L, m, d)
@@ -224,6 +230,7 @@ dark_status dark_attention_fwd(const dark_projection* proj, const void* q, const
 size_t dark_cross_attention_workspace_bytes(const dark_projection* proj, int B, int H, int Lq,
                                             int Lk, int flags) {
   if (!proj_ok(proj) || B < 1 || H < 1 || Lq < 1 || Lk < 1 || (flags & DARK_CAUSAL)) return 0;
+  if (flags & DARK_EXACT) return dark::exact_workspace_bytes(B, H, Lq, Lk, proj->r);
   const size_t simt = dark::simt_workspace_bytes(B, H, Lq, Lk, proj->m, proj->d, flags);
   const size_t tc = dark::tc_noncausal_workspace_bytes(B, H, Lq, Lk, proj->m, proj->d);
   return simt > tc ? simt : tc;
@@ -345,6 +352,10 @@ dark_status dark_attention_bwd(const float* omega, int heads_omega, const float*
   a.dev_status = dev_status;
   a.stream = (cudaStream_t)stream;
   return from_cuda(dark::launch_backward(a));
+}
+
+int dark_auto_uses_exact(int L, int exact_threshold) {
+  return exact_threshold > 0 && L <= exact_threshold ? 1 : 0;
 }
 
 size_t dark_sample_omega_workspace_bytes(int heads, int m, int r, int orthogonal) {

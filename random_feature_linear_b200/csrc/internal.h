@@ -95,6 +95,10 @@ bool tc_wide_supported(FwdArgs& a);
 size_t tc_wide_workspace_bytes(int B, int H, int L, int m, int d, int r);
 cudaError_t tc_wide_forward(const FwdArgs& a);
 
+// Exact learned-kernel attention (softmax over u = M q~, w = M k~), SIMT fp32.
+size_t exact_workspace_bytes(int B, int H, int Lq, int Lk, int r);
+cudaError_t exact_forward(const FwdArgs& a);
+
 // Decode step over [B][H] heads.
 struct DecodeArgs {
   int heads_w, m, r, d;

@@ -23,7 +23,7 @@ _lib = ctypes.CDLL(_LIB_PATH)
 DARK_OK, DARK_ERR_INVALID_ARG, DARK_ERR_UNSUPPORTED, DARK_ERR_STALE_STATE = 0, 1, 2, 3
 DARK_ERR_CUDA, DARK_ERR_NUMERIC, DARK_ERR_TIMEOUT = 4, 5, 6
 DARK_F32, DARK_BF16 = 0, 1
-DARK_CAUSAL, DARK_STABILISE = 1, 2
+DARK_CAUSAL, DARK_STABILISE, DARK_EXACT = 1, 2, 4
 WS_HEADER_BYTES = 256
 
 EXPORTS = ("dark_abi_version", "dark_status_string", "dark_projection_bytes",
@@ -33,7 +33,8 @@ EXPORTS = ("dark_abi_version", "dark_status_string", "dark_projection_bytes",
            "dark_cross_attention_fwd", "dark_cross_decode_step",
            "dark_attention_bwd_workspace_bytes", "dark_attention_bwd",
            "dark_sample_omega_workspace_bytes", "dark_sample_omega", "dark_redraw_schedule_init",
-           "dark_redraw_on_forward", "dark_redraw_request", "dark_redraw_set_fixed")
+           "dark_redraw_on_forward", "dark_redraw_request", "dark_redraw_set_fixed",
+           "dark_auto_uses_exact")
 
 
 class dark_projection(ctypes.Structure):
@@ -88,6 +89,8 @@ _lib.dark_cross_attention_fwd.argtypes = [_P(dark_projection), _vp, _P(ctypes.c_
                                           _sz, _vp, _vp]
 _lib.dark_cross_decode_step.restype = _i
 _lib.dark_cross_decode_step.argtypes = [_P(dark_projection), _P(dark_state), _vp, _vp, _vp, _vp]
+_lib.dark_auto_uses_exact.restype = _i
+_lib.dark_auto_uses_exact.argtypes = [_i, _i]
 _lib.dark_sample_omega_workspace_bytes.restype = _sz
 _lib.dark_sample_omega_workspace_bytes.argtypes = [_i, _i, _i, _i]
 _lib.dark_sample_omega.restype = _i
@@ -323,6 +326,10 @@ def alloc_workspace(proj: dark_projection, B: int, H: int, L: int, flags: int, d
     """A zero-filled workspace of the size dark_attention_workspace_bytes asks for."""
     n = dark_attention_workspace_bytes(proj, B, H, L, flags)
     return torch.zeros(max(n, WS_HEADER_BYTES), dtype=torch.uint8, device=device)
+
+
+def dark_auto_uses_exact(L: int, exact_threshold: int) -> bool:
+    return bool(_lib.dark_auto_uses_exact(L, exact_threshold))
 
 
 def dark_sample_omega_workspace_bytes(heads: int, m: int, r: int, orthogonal: bool) -> int:

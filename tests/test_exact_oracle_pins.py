@@ -64,6 +64,31 @@ def test_random_features_converge_to_the_exact_kernel():
     assert errs[1] < 0.05 and errs[1] < errs[0] / 4
 
 
+def test_cross_form_and_query_mask():
+    # queries over a separate context: equal to the self-attention form when the
+    # context is the same tokens; a masked query row is zero, the rest unchanged
+    q, k, v, gm = _inputs(7)
+    mask = np.array([[1, 1, 0, 1, 1, 1, 1, 1, 0], [1] * 9], np.uint8)
+    a = O.exact_attention(q, k, v, gm, key_mask=mask)
+    qm = np.array([[1, 0, 1, 1, 1, 1, 1, 1, 1], [1, 1, 1, 0, 0, 1, 1, 1, 1]], np.uint8)
+    b = O.exact_attention(q, k, v, gm, key_mask=mask, query_mask=qm)
+    dead = np.broadcast_to((qm == 0)[:, None, :, None], a.shape)
+    assert np.all(b[dead] == 0.0) and np.array_equal(a[~dead], b[~dead])
+    # a longer context: rows against torch SDPA with the key mask as attn_mask
+    rng = np.random.default_rng(8)
+    k2, v2 = rng.standard_normal((2, 2, 13, 8)), rng.standard_normal((2, 2, 13, 8))
+    cm = np.ones((2, 13), np.uint8)
+    cm[0, 4:7] = 0
+    got = O.exact_attention(q, k2, v2, gm, key_mask=cm)
+    s = 8 ** -0.25
+    tg = torch.tensor(gm)
+    u = torch.einsum("bhld,hrd->bhlr", torch.tensor(q) * s, tg)
+    w = torch.einsum("bhld,hrd->bhlr", torch.tensor(k2) * s, tg)
+    keep = torch.tensor(cm != 0)[:, None, None, :].expand(2, 2, 9, 13)
+    ref = F.scaled_dot_product_attention(u, w, torch.tensor(v2), attn_mask=keep, scale=1.0)
+    assert np.abs(got - ref.numpy()).max() <= 1e-12
+
+
 def test_auto_policy():
     assert O.uses_exact(1024, 1024) and not O.uses_exact(1025, 1024)
     assert not O.uses_exact(16, 0)
