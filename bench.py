@@ -313,10 +313,16 @@ def run_native(args, w: synth.Workload, rank: int, world: int, dev) -> dict | No
     if args.exact:
         flops = exact_flops(w)
         achieved = flops / t_kernel / 1e12
-        roof = dict(bound="alu", achieved=achieved, peak=FFMA_TFLOPS, unit="TFLOP/s",
-                    frac=achieved / FFMA_TFLOPS, traffic=None,
-                    peak_source="derived: 148 SMs x 128 FP32 lanes x 2 x 1.965 GHz",
-                    kernel="exact-mode call (SIMT fp32)")
+        if w.dtype == "bf16" and w.d == 64 and w.r % 16 == 0 and w.r <= 64:
+            roof = dict(bound="tensor", achieved=achieved, peak=peaks["bf16"], unit="TFLOP/s",
+                        frac=achieved / peaks["bf16"], traffic=None,
+                        peak_source=peaks["source"] + " (burst)",
+                        kernel="exact-mode call (exact_tc_kernel, tcgen05)")
+        else:
+            roof = dict(bound="alu", achieved=achieved, peak=FFMA_TFLOPS, unit="TFLOP/s",
+                        frac=achieved / FFMA_TFLOPS, traffic=None,
+                        peak_source="derived: 148 SMs x 128 FP32 lanes x 2 x 1.965 GHz",
+                        kernel="exact-mode call (SIMT fp32)")
     else:
         bound = "tensor" if t_tc >= t_hbm else "hbm"
         if bound == "tensor":

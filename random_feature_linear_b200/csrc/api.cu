@@ -30,10 +30,10 @@ bool proj_ok(const dark_projection* p) {
          sizes_ok(p->m, p->r, p->d) && p->heads >= 1;
 }
 
-enum class Path { Simt, TcCausal, TcNonCausal, TcWide, Exact };
+enum class Path { Simt, TcCausal, TcNonCausal, TcWide, Exact, TcExact };
 
 Path choose_path(dark::FwdArgs& a) {
-  if (a.flags & DARK_EXACT) return Path::Exact;
+  if (a.flags & DARK_EXACT) return dark::tc_exact_supported(a) ? Path::TcExact : Path::Exact;
   if (a.flags & DARK_CAUSAL) {
     if (dark::tc_causal_supported(a)) return Path::TcCausal;
     if (dark::tc_wide_supported(a)) return Path::TcWide;
@@ -49,6 +49,7 @@ size_t ws_need(Path p, int B, int H, int Lq, int Lk, int m, int r, int d, int fl
     case Path::TcWide: return dark::tc_wide_workspace_bytes(B, H, Lq, m, d, r);
     case Path::TcNonCausal: return dark::tc_noncausal_workspace_bytes(B, H, Lq, Lk, m, d);
     case Path::Exact: return dark::exact_workspace_bytes(B, H, Lq, Lk, r);
+    case Path::TcExact: return dark::kWsHeader;
     default: return dark::simt_workspace_bytes(B, H, Lq, Lk, m, d, flags);
   }
 }
@@ -141,6 +142,7 @@ dark_status fwd_launch(FwdArgs& a, void* ws, size_t ws_bytes, dark_state* state_
     case Path::TcNonCausal: e = tc_noncausal_forward(a); break;
     case Path::TcWide: e = tc_wide_forward(a); break;
     case Path::Exact: e = exact_forward(a); break;
+    case Path::TcExact: e = tc_exact_forward(a); break;
     default: e = simt_forward(a); break;
   }
   if (e != cudaSuccess) return DARK_ERR_CUDA;

@@ -98,6 +98,9 @@ cudaError_t tc_wide_forward(const FwdArgs& a);
 // Exact learned-kernel attention (softmax over u = M q~, w = M k~), SIMT fp32.
 size_t exact_workspace_bytes(int B, int H, int Lq, int Lk, int r);
 cudaError_t exact_forward(const FwdArgs& a);
+// ... and on tcgen05 for bf16, d = 64, r in {16, 32, 48, 64} (no workspace).
+bool tc_exact_supported(FwdArgs& a);
+cudaError_t tc_exact_forward(const FwdArgs& a);
 
 // Decode step over [B][H] heads.
 struct DecodeArgs {

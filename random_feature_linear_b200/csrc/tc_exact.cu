@@ -1,0 +1,350 @@
+// Exact learned-kernel attention on sm_100a tensor cores (bf16 I/O, d = 64,
+// r <= 64): out_i = sum_j softmax_j(u_i . w_j) v_j with u = M q~, w = M k~
+// (README, section "Attention modes": the exact path applies the learned
+// geometry to queries and keys before scaled dot-product attention).
+//
+// One CTA (256 threads) per 128-query tile of one (batch, head):
+//   Q tile (TMA, bf16 -> fp16) x W'_bot^T -> 2 p_q (fp16, a K-major operand; the
+//   projection's last r rows are c_m M, so 2 p_q . p_k is the score in base 2);
+//   per 128-key tile:
+//     K tile (TMA) x W'_bot^T -> p_k (fp16 operand)        tcgen05, N = r
+//     scores S = (2 p_q) p_k^T                              tcgen05, N = 128
+//     key mask, causal mask, running row maximum (the two thread halves of a
+//     row exchange their maxima), P = 2^(S - max) as bf16 into shared memory
+//     [num | den] = P [V | 1]                               tcgen05, N = 80
+//     O = O * 2^(old max - new max) + num, l likewise with den (registers)
+//   out = O / l.
+// The next key tile loads while the current scores are processed, the next
+// value tile while the next projection runs. Every wait is bounded; a wait
+// that runs out stores DARK_ERR_TIMEOUT and the CTA leaves its loop.
+#include <string.h>
+
+#include "common.cuh"
+#include "internal.h"
+#include "tc_common.cuh"
+#include "tc_keys.cuh"
+
+namespace dark {
+namespace {
+
+using namespace tc;
+
+constexpr int kD = 64;
+constexpr int kT = 128;                    // queries per CTA, keys per tile
+constexpr int kThreads = kFwdThreads;
+constexpr int kTile = kT * kD * 2;         // one 128 x 64 tile of 16-bit elements
+constexpr uint32_t kTmemCols = 256;
+
+// shared memory (all 1024-byte aligned)
+constexpr uint32_t oW = 0;                 // W'_bot: up to 64 rows x 128 B (fp16)
+constexpr uint32_t oQ = 8192;              // Q tile, then 2 p_q (fp16, K-major)
+constexpr uint32_t oK = oQ + kTile;        // K tile, then p_k (fp16, K-major)
+constexpr uint32_t oV = oK + kTile;        // V tile (bf16, keys x d)
+constexpr uint32_t oOnes = oV + kTile;     // bf16 ones: [V | 1] as one N = 80 operand
+constexpr uint32_t oP = oOnes + kTile;     // P: 128 queries x 128 keys bf16, two K blocks
+constexpr uint32_t oMax = oP + 2 * kTile;  // row maxima of the two thread halves
+constexpr uint32_t oBar = oMax + 2 * kT * 4;
+constexpr uint32_t kSmem = oBar + 64 + 1024;
+// TMEM columns: scores [0, 128); projection [128, 128 + r) and, later in the
+// same tile, [num | den] [128, 208)
+constexpr uint32_t tS = 0, tX = 128;
+
+struct Params {
+  __nv_bfloat16* out;
+  int64_t ob, oh, ol;
+  const uint8_t* kmask;                    // [B][Lk] or null
+  const uint8_t* qmask;                    // [B][Lq] or null
+  int B, H, Lq, Lk, nq, causal, heads_w, m, r;
+  int* dev_status;
+};
+
+// Projection epilogue: this thread's row of the N = r projection in TMEM, times
+// `scale`, as fp16 into a K-major 128B-swizzled tile (columns r..63 zero).
+__device__ __forceinline__ void proj_to_smem(uint32_t lane_taddr, int r, float scale,
+                                             uint32_t tile, int row, int half) {
+  const int c0 = half * 32;
+  uint32_t w[16];
+  if (c0 < r) {
+    float v[32];
+    tmem_ld32(lane_taddr + c0, v);
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+      const float a = c0 + 2 * e < r ? v[2 * e] * scale : 0.f;
+      const float b = c0 + 2 * e + 1 < r ? v[2 * e + 1] * scale : 0.f;
+      const __half2 hv = __floats2half2_rn(a, b);
+      w[e] = *reinterpret_cast<const uint32_t*>(&hv);
+    }
+  } else {
+#pragma unroll
+    for (int e = 0; e < 16; ++e) w[e] = 0u;
+  }
+#pragma unroll
+  for (int g = 0; g < 4; ++g)
+    st_shared_v4(tile + kmajor_off(row, c0 + 8 * g, 0), w[4 * g], w[4 * g + 1], w[4 * g + 2],
+                 w[4 * g + 3]);
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    exact_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_q,
+                    const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                    const Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  const uint32_t s0 = smem_u32(sm);
+  uint64_t* bar_k = (uint64_t*)(sm + oBar);     // Q, W' (first), then each K tile
+  uint64_t* bar_v = bar_k + 1;                  // each V tile
+  uint64_t* bar_mma = bar_k + 2;
+  uint32_t* tmem_slot = (uint32_t*)(bar_k + 3);
+  float* smax = (float*)(sm + oMax);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int quad = warp & 3, half = warp >> 2;
+  const int row = quad * 32 + lane;
+
+  if (tid == 0) {
+    mbar_init(bar_k, 1);
+    mbar_init(bar_v, 1);
+    mbar_init(bar_mma, 1);
+    fence_mbar_init();
+    prefetch_tmap(&tm_w);
+    prefetch_tmap(&tm_q);
+    prefetch_tmap(&tm_k);
+    prefetch_tmap(&tm_v);
+  }
+  __syncwarp();
+  if (warp == 0) tmem_alloc(tmem_slot, kTmemCols);
+  for (int i = tid; i < kTile / 16; i += kThreads)
+    st_shared_v4(s0 + oOnes + i * 16, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u);
+  fence_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t lane_tm = tmem + ((uint32_t)(quad * 32) << 16);
+  const int bh = blockIdx.x / p.nq, qt = blockIdx.x % p.nq;
+  const int b = bh / p.H, h = bh % p.H;
+  const int hw = p.heads_w == 1 ? 0 : h;
+  const int q0 = qt * kT;
+  const int qi = q0 + row;
+  const int nk = p.causal ? qt + 1 : (p.Lk + kT - 1) / kT;
+  const int r = p.r;
+
+  uint32_t ph_k = 0, ph_v = 0, ph_mma = 0;
+  bool abort = false;
+  float o[32], l = 0.f, mrow = -INFINITY;
+#pragma unroll
+  for (int i = 0; i < 32; ++i) o[i] = 0.f;
+
+  // ---- Q and W'_bot, then K_0 and V_0
+  if (tid == 0) {
+    mbar_arrive_expect_tx(bar_k, (uint32_t)r * 128 + kTile);
+    for (int r0 = 0; r0 < r; r0 += 16)
+      tma_load_2d(sm + oW + r0 * 128, &tm_w, 0, hw * (p.m + r) + p.m + r0, bar_k);
+    tma_load_4d(sm + oQ, &tm_q, 0, q0, h, b, bar_k);
+  }
+  if (!wait_all(bar_k, ph_k, p.dev_status)) abort = true;
+  ph_k ^= 1;
+  if (!abort) {
+    if (tid == 0) {
+      mbar_arrive_expect_tx(bar_k, kTile);
+      tma_load_4d(sm + oK, &tm_k, 0, 0, h, b, bar_k);
+      mbar_arrive_expect_tx(bar_v, kTile);
+      tma_load_4d(sm + oV, &tm_v, 0, 0, h, b, bar_v);
+    }
+    to_fp16_inplace(s0 + oQ, kTile, p.dev_status);
+    fence_async_smem();
+    __syncthreads();
+    if (tid == 0) {
+      tc_fence_after();
+      const uint32_t idp = idesc(128, r, false, false, true);
+#pragma unroll
+      for (int s = 0; s < kD / 16; ++s)
+        mma(tmem + tX, sdesc(s0 + oQ + s * 32, 16, 1024), sdesc(s0 + oW + s * 32, 16, 1024), idp,
+            s > 0);
+      mma_commit(bar_mma);
+    }
+    if (!wait_all(bar_mma, ph_mma, p.dev_status)) abort = true;
+    ph_mma ^= 1;
+    tc_fence_after();
+    // the projection MMA has read the Q tile: 2 p_q over it
+    if (!abort) proj_to_smem(lane_tm + tX, r, 2.f, s0 + oQ, row, half);
+    fence_async_smem();
+    tc_fence_before();
+    __syncthreads();
+  }
+
+  for (int j = 0; j < nk && !abort; ++j) {
+    const int k0 = j * kT;
+    // ---- K_j: projection p_k
+    if (!wait_all(bar_k, ph_k, p.dev_status)) { abort = true; break; }
+    ph_k ^= 1;
+    to_fp16_inplace(s0 + oK, kTile, p.dev_status);
+    fence_async_smem();
+    __syncthreads();
+    if (tid == 0) {
+      tc_fence_after();
+      const uint32_t idp = idesc(128, r, false, false, true);
+#pragma unroll
+      for (int s = 0; s < kD / 16; ++s)
+        mma(tmem + tX, sdesc(s0 + oK + s * 32, 16, 1024), sdesc(s0 + oW + s * 32, 16, 1024), idp,
+            s > 0);
+      mma_commit(bar_mma);
+    }
+    if (!wait_all(bar_mma, ph_mma, p.dev_status)) { abort = true; break; }
+    ph_mma ^= 1;
+    tc_fence_after();
+    proj_to_smem(lane_tm + tX, r, 1.f, s0 + oK, row, half);
+    fence_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    // ---- scores S = (2 p_q) p_k^T
+    if (tid == 0) {
+      tc_fence_after();
+      constexpr uint32_t ids = idesc(128, 128, false, false, true);
+#pragma unroll
+      for (int s = 0; s < kD / 16; ++s)
+        mma(tmem + tS, sdesc(s0 + oQ + s * 32, 16, 1024), sdesc(s0 + oK + s * 32, 16, 1024), ids,
+            s > 0);
+      mma_commit(bar_mma);
+    }
+    if (!wait_all(bar_mma, ph_mma, p.dev_status)) { abort = true; break; }
+    ph_mma ^= 1;
+    tc_fence_after();
+    // the scores MMA has read p_k: the next key tile may load over it
+    if (tid == 0 && j + 1 < nk) {
+      mbar_arrive_expect_tx(bar_k, kTile);
+      tma_load_4d(sm + oK, &tm_k, 0, k0 + kT, h, b, bar_k);
+    }
+    // ---- masks, row maximum, P = 2^(S - max) (this half: keys half*64 .. +63)
+    float sv[64];
+    {
+      float v[32];
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        tmem_ld32(lane_tm + tS + half * 64 + c * 32, v);
+#pragma unroll
+        for (int e = 0; e < 32; ++e) sv[c * 32 + e] = v[e];
+      }
+    }
+    float tmax = -INFINITY;
+#pragma unroll
+    for (int e = 0; e < 64; ++e) {
+      const int key = k0 + half * 64 + e;
+      bool ok = key < p.Lk && (!p.causal || key <= qi);
+      if (ok && p.kmask != nullptr) ok = p.kmask[(size_t)b * p.Lk + key] != 0;
+      sv[e] = ok ? sv[e] : -INFINITY;
+      tmax = fmaxf(tmax, sv[e]);
+    }
+    smax[half * kT + row] = tmax;
+    __syncthreads();
+    const float nmax = fmaxf(mrow, fmaxf(smax[row], smax[kT + row]));
+    const float off = nmax == -INFINITY ? 0.f : nmax;
+    const float scale = nmax == -INFINITY ? 1.f : ex2(mrow - nmax);
+    mrow = nmax;
+#pragma unroll
+    for (int g = 0; g < 8; ++g) {
+      uint32_t w4[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float x0 = sv[8 * g + 2 * e], x1 = sv[8 * g + 2 * e + 1];
+        w4[e] = pack_bf16(x0 == -INFINITY ? 0.f : ex2(x0 - off), x1 == -INFINITY ? 0.f : ex2(x1 - off));
+      }
+      st_shared_v4(s0 + oP + kmajor_off(row, half * 64 + 8 * g, 16384), w4[0], w4[1], w4[2], w4[3]);
+    }
+    fence_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    // ---- [num | den] = P [V | 1]
+    if (!wait_all(bar_v, ph_v, p.dev_status)) { abort = true; break; }
+    ph_v ^= 1;
+    if (tid == 0) {
+      tc_fence_after();
+      constexpr uint32_t idv = idesc(128, 80, false, true, false);
+#pragma unroll
+      for (int s = 0; s < kT / 16; ++s)
+        mma(tmem + tX, sdesc(s0 + oP + (s / 4) * 16384 + (s % 4) * 32, 16, 1024),
+            sdesc(s0 + oV + s * 2048, oOnes - oV, 1024), idv, s > 0);
+      mma_commit(bar_mma);
+    }
+    if (!wait_all(bar_mma, ph_mma, p.dev_status)) { abort = true; break; }
+    ph_mma ^= 1;
+    tc_fence_after();
+    // the value MMA has read V: the next value tile may load
+    if (tid == 0 && j + 1 < nk) {
+      mbar_arrive_expect_tx(bar_v, kTile);
+      tma_load_4d(sm + oV, &tm_v, 0, k0 + kT, h, b, bar_v);
+    }
+    {
+      float v[32];
+      tmem_ld32(lane_tm + tX + half * 32, v);
+      const float den = tmem_ld1(lane_tm + tX + 64);
+#pragma unroll
+      for (int i = 0; i < 32; ++i) o[i] = fmaf(o[i], scale, v[i]);
+      l = fmaf(l, scale, den);
+    }
+    tc_fence_before();
+    __syncthreads();
+  }
+  if (!abort && qi < p.Lq) {
+    const bool live = p.qmask == nullptr || p.qmask[(size_t)b * p.Lq + qi] != 0;
+    const float inv = (live && l > 0.f) ? 1.f / l : 0.f;
+    uint32_t w[16];
+    bool bad = false;
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+      const float a = o[2 * e] * inv, c = o[2 * e + 1] * inv;
+      bad |= !isfinite(a) || !isfinite(c);
+      w[e] = pack_bf16(a, c);
+    }
+    if (bad) report(p.dev_status, DARK_ERR_NUMERIC);
+    uint4* dst = reinterpret_cast<uint4*>(p.out + (int64_t)b * p.ob + (int64_t)h * p.oh +
+                                          (int64_t)qi * p.ol + half * 32);
+#pragma unroll
+    for (int q4 = 0; q4 < 4; ++q4)
+      dst[q4] = make_uint4(w[4 * q4], w[4 * q4 + 1], w[4 * q4 + 2], w[4 * q4 + 3]);
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+}  // namespace
+
+bool tc_exact_supported(FwdArgs& a) {
+  if (a.dtype != DARK_BF16 || a.d != kD || a.r % 16 != 0 || a.r < 16 || a.r > 64) return false;
+  if (a.os[2] % 8 != 0) return false;          // 16-byte output stores
+  return tc_make_maps(a);
+}
+
+cudaError_t tc_exact_forward(const FwdArgs& a) {
+  if (!a.maps_ready) return cudaErrorInvalidValue;
+  Params p;
+  memset(&p, 0, sizeof(p));
+  p.out = (__nv_bfloat16*)a.out;
+  p.ob = a.os[0];
+  p.oh = a.os[1];
+  p.ol = a.os[2];
+  p.kmask = a.mask;
+  p.qmask = a.qmask;
+  p.B = a.B;
+  p.H = a.H;
+  p.Lq = a.L;
+  p.Lk = a.Lk;
+  p.nq = (a.L + kT - 1) / kT;
+  p.causal = (a.flags & DARK_CAUSAL) ? 1 : 0;
+  p.heads_w = a.heads_w;
+  p.m = a.m;
+  p.r = a.r;
+  p.dev_status = a.dev_status;
+  static int smem_set[64];
+  cudaError_t e = set_smem_limit_once((const void*)exact_tc_kernel, (int)kSmem, smem_set);
+  if (e != cudaSuccess) return e;
+  exact_tc_kernel<<<a.B * a.H * p.nq, kThreads, kSmem, a.stream>>>(a.tm_w, a.tm_q, a.tm_k, a.tm_v,
+                                                                   p);
+  return cudaGetLastError();
+}
+
+}  // namespace dark
