@@ -84,7 +84,7 @@ __device__ __forceinline__ void proj_to_smem(uint32_t lane_taddr, int r, float s
                  w[4 * g + 3]);
 }
 
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads, 2)
     exact_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_q,
                     const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                     const Params p) {
@@ -121,7 +121,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const uint32_t lane_tm = tmem + ((uint32_t)(quad * 32) << 16);
-  const int bh = blockIdx.x / p.nq, qt = blockIdx.x % p.nq;
+  // query tiles in decreasing order of work first (causal: tile qt walks qt + 1
+  // key tiles), so that the short ones fill in behind the long ones
+  const int nbh = p.B * p.H;
+  const int bh = blockIdx.x % nbh, qt = p.nq - 1 - blockIdx.x / nbh;
   const int b = bh / p.H, h = bh % p.H;
   const int hw = p.heads_w == 1 ? 0 : h;
   const int q0 = qt * kT;
@@ -215,25 +218,22 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_arrive_expect_tx(bar_k, kTile);
       tma_load_4d(sm + oK, &tm_k, 0, k0 + kT, h, b, bar_k);
     }
-    // ---- masks, row maximum, P = 2^(S - max) (this half: keys half*64 .. +63)
-    float sv[64];
-    {
-      float v[32];
-#pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        tmem_ld32(lane_tm + tS + half * 64 + c * 32, v);
-#pragma unroll
-        for (int e = 0; e < 32; ++e) sv[c * 32 + e] = v[e];
-      }
-    }
-    float tmax = -INFINITY;
-#pragma unroll
-    for (int e = 0; e < 64; ++e) {
-      const int key = k0 + half * 64 + e;
+    // ---- masks, row maximum, P = 2^(S - max) (this half: keys half*64 .. +63);
+    // the scores are read from TMEM twice (maximum, then exponentials) rather
+    // than held in registers
+    auto visible = [&](int key) {
       bool ok = key < p.Lk && (!p.causal || key <= qi);
       if (ok && p.kmask != nullptr) ok = p.kmask[(size_t)b * p.Lk + key] != 0;
-      sv[e] = ok ? sv[e] : -INFINITY;
-      tmax = fmaxf(tmax, sv[e]);
+      return ok;
+    };
+    float tmax = -INFINITY;
+#pragma unroll
+    for (int c = 0; c < 2; ++c) {
+      float v[32];
+      tmem_ld32(lane_tm + tS + half * 64 + c * 32, v);
+#pragma unroll
+      for (int e = 0; e < 32; ++e)
+        if (visible(k0 + half * 64 + c * 32 + e)) tmax = fmaxf(tmax, v[e]);
     }
     smax[half * kT + row] = tmax;
     __syncthreads();
@@ -242,14 +242,22 @@ __global__ void __launch_bounds__(kThreads, 1)
     const float scale = nmax == -INFINITY ? 1.f : ex2(mrow - nmax);
     mrow = nmax;
 #pragma unroll
-    for (int g = 0; g < 8; ++g) {
-      uint32_t w4[4];
+    for (int c = 0; c < 2; ++c) {
+      float v[32];
+      tmem_ld32(lane_tm + tS + half * 64 + c * 32, v);
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float x0 = sv[8 * g + 2 * e], x1 = sv[8 * g + 2 * e + 1];
-        w4[e] = pack_bf16(x0 == -INFINITY ? 0.f : ex2(x0 - off), x1 == -INFINITY ? 0.f : ex2(x1 - off));
+      for (int g = 0; g < 4; ++g) {
+        uint32_t w4[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int j0 = c * 32 + 8 * g + 2 * e, key = k0 + half * 64 + j0;
+          const float p0 = visible(key) ? ex2(v[8 * g + 2 * e] - off) : 0.f;
+          const float p1 = visible(key + 1) ? ex2(v[8 * g + 2 * e + 1] - off) : 0.f;
+          w4[e] = pack_bf16(p0, p1);
+        }
+        st_shared_v4(s0 + oP + kmajor_off(row, half * 64 + c * 32 + 8 * g, 16384), w4[0], w4[1],
+                     w4[2], w4[3]);
       }
-      st_shared_v4(s0 + oP + kmajor_off(row, half * 64 + 8 * g, 16384), w4[0], w4[1], w4[2], w4[3]);
     }
     fence_async_smem();
     tc_fence_before();
@@ -342,6 +350,18 @@ cudaError_t tc_exact_forward(const FwdArgs& a) {
   static int smem_set[64];
   cudaError_t e = set_smem_limit_once((const void*)exact_tc_kernel, (int)kSmem, smem_set);
   if (e != cudaSuccess) return e;
+  // two CTAs per SM (2 x 106 KB of shared memory, 2 x 256 TMEM columns); set
+  // once per device, outside any later stream capture
+  static int carveout_set[64];
+  int dev = 0;
+  e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev >= 0 && dev < 64 && !carveout_set[dev]) {
+    e = cudaFuncSetAttribute((const void*)exact_tc_kernel,
+                             cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+    if (e != cudaSuccess) return e;
+    carveout_set[dev] = 1;
+  }
   exact_tc_kernel<<<a.B * a.H * p.nq, kThreads, kSmem, a.stream>>>(a.tm_w, a.tm_q, a.tm_k, a.tm_v,
                                                                    p);
   return cudaGetLastError();
