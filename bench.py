@@ -700,7 +700,7 @@ def run_cross(args, rank: int, world: int, dev) -> dict | None:
 
 
 EXACT_METRIC = ("DARK exact learned-kernel attention fwd tokens/s (B·H·L/s) on 1 B200; "
-                "% of FP32-FFMA roofline")
+                "% of BF16-tensor roofline (tcgen05 path) or FP32-FFMA (SIMT path)")
 
 
 def exact_flops(w: synth.Workload) -> float:

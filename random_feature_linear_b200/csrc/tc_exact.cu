@@ -43,7 +43,8 @@ constexpr uint32_t oV = oK + kTile;        // V tile (bf16, keys x d)
 constexpr uint32_t oOnes = oV + kTile;     // bf16 ones: [V | 1] as one N = 80 operand
 constexpr uint32_t oP = oOnes + kTile;     // P: 128 queries x 128 keys bf16, two K blocks
 constexpr uint32_t oMax = oP + 2 * kTile;  // row maxima of the two thread halves
-constexpr uint32_t oBar = oMax + 2 * kT * 4;
+constexpr uint32_t oKv = oMax + 2 * kT * 4; // validity of the tile's 128 keys (bytes)
+constexpr uint32_t oBar = oKv + kT;
 constexpr uint32_t kSmem = oBar + 64 + 1024;
 // TMEM columns: scores [0, 128); projection [128, 128 + r) and, later in the
 // same tile, [num | den] [128, 208)
@@ -96,6 +97,7 @@ __global__ void __launch_bounds__(kThreads, 2)
   uint64_t* bar_mma = bar_k + 2;
   uint32_t* tmem_slot = (uint32_t*)(bar_k + 3);
   float* smax = (float*)(sm + oMax);
+  uint8_t* kval = sm + oKv;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int quad = warp & 3, half = warp >> 2;
@@ -210,6 +212,12 @@ __global__ void __launch_bounds__(kThreads, 2)
             s > 0);
       mma_commit(bar_mma);
     }
+    // key validity of this tile, read from global memory once (the wait below
+    // is a block-wide barrier)
+    if (tid < kT) {
+      const int key = k0 + tid;
+      kval[tid] = (key < p.Lk && (p.kmask == nullptr || p.kmask[(size_t)b * p.Lk + key] != 0)) ? 1 : 0;
+    }
     if (!wait_all(bar_mma, ph_mma, p.dev_status)) { abort = true; break; }
     ph_mma ^= 1;
     tc_fence_after();
@@ -221,11 +229,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     // ---- masks, row maximum, P = 2^(S - max) (this half: keys half*64 .. +63);
     // the scores are read from TMEM twice (maximum, then exponentials) rather
     // than held in registers
-    auto visible = [&](int key) {
-      bool ok = key < p.Lk && (!p.causal || key <= qi);
-      if (ok && p.kmask != nullptr) ok = p.kmask[(size_t)b * p.Lk + key] != 0;
-      return ok;
-    };
+    auto visible = [&](int key) { return kval[key - k0] != 0 && (!p.causal || key <= qi); };
     float tmax = -INFINITY;
 #pragma unroll
     for (int c = 0; c < 2; ++c) {
