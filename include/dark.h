@@ -241,8 +241,8 @@ size_t dark_cross_attention_workspace_bytes(const dark_projection* proj, int B, 
  *   context_mask device uint8 [B][Lk] (nonzero = valid context position) or NULL
  *   out          device, [B][H][Lq][d], strides out_strides (NULL = contiguous)
  *   flags        0 or DARK_STABILISE; DARK_CAUSAL returns DARK_ERR_INVALID_ARG
- *   context_out  NULL, or a state that receives the context summary (S, z)
- *                ("summarised once per layer" for decoding, see
+ *   context_out  NULL, or a state that receives the context summary (S, z),
+ *                which decoding reuses at every step (see
  *                dark_cross_decode_step); its generation is set
  *   ws, ws_bytes workspace (dark_cross_attention_workspace_bytes)
  * Errors as dark_attention_fwd.
@@ -312,8 +312,8 @@ dark_status dark_attention_bwd(const float* omega, int heads_omega, const float*
                                size_t ws_bytes, int* dev_status, void* stream);
 
 /*
- * Exact mode (README, section "Attention modes": the exact path applies the
- * learned geometry to queries and keys before scaled dot-product attention).
+ * Exact mode (README, section "Attention modes": M acts on queries and keys and
+ * ordinary softmax attention with scaled scores follows).
  * DARK_EXACT in the flags of dark_attention_fwd, dark_attention_fwd_noalloc or
  * dark_cross_attention_fwd evaluates
  *   out_i = sum_j softmax_j(u_i . w_j) v_j,  u = M q~, w = M k~, x~ = d^{-1/4} x,
@@ -324,8 +324,8 @@ dark_status dark_attention_bwd(const float* omega, int heads_omega, const float*
  * DARK_STABILISE is accepted and has no effect (the softmax is computed with a
  * running maximum). The workspace queries account for the flag.
  *
- * Auto mode ("exact_threshold"): exact attention through the threshold, linear
- * attention above it. dark_auto_uses_exact returns 1 when L <= exact_threshold and
+ * Auto mode ("exact_threshold"): the exact mode for sequences up to the threshold
+ * length, random features for longer ones. dark_auto_uses_exact returns 1 when L <= exact_threshold and
  * exact_threshold > 0; the caller then adds DARK_EXACT.
  */
 int dark_auto_uses_exact(int L, int exact_threshold);
@@ -361,8 +361,9 @@ dark_status dark_sample_omega(uint64_t seed, uint64_t draw, int heads, int m, in
 /*
  * Redraw schedule of one projection (host only; README, section "Projection
  * lifecycle"). The current projection is dark_sample_omega(seed, draw, ...).
- *   interval > 0: a redraw falls due after that many training forwards and happens
- *   at the start of the next training forward; evaluation forwards do not count;
+ *   interval > 0: once that many training forwards have run, a redraw happens at
+ *   the start of the next training forward; forwards outside training are not
+ *   counted;
  *   interval <= 0: no scheduled redraws. While fixed, a redraw falling due is
  *   dropped (the interval restarts) and ordinary requests are refused; a forced
  *   request redraws once. Every redraw restarts the interval. deterministic != 0

@@ -201,7 +201,7 @@ def cross_attention(q, k, v, omega, geom, query_mask=None, context_mask=None):
     v_j / sum_j kappa_hat(q_i, k_j) over the valid context positions j, written
     out pair by pair; a masked query row, or one whose denominator is zero,
     outputs 0. Returns (out [B, H, Lq, d], kv [B, H, m, d], z [B, H, m]), the
-    context summary Phi(K)^T V and Phi(K)^T 1 ("summarised once per layer").
+    context summary Phi(K)^T V and Phi(K)^T 1 that a decoder reuses at every step.
     """
     q, k, v = _f64(q), _f64(k), _f64(v)
     B, H, Lq, d = q.shape
@@ -235,8 +235,8 @@ def cross_attention(q, k, v, omega, geom, query_mask=None, context_mask=None):
 
 def cross_decode_step(kv, z, q_t, omega, geom):
     """One decoder step of cross-attention against a fixed context summary
-    (README, "Encoder-decoder model and generation": the encoded source is
-    summarised once per layer): out_t = phi(q_t)^T kv / phi(q_t)^T z; the
+    (README, "Encoder-decoder model and generation": each layer's decoder reuses
+    one summary of the encoder output): out_t = phi(q_t)^T kv / phi(q_t)^T z; the
     summary is not changed. q_t: [B, H, d]; kv: [B, H, m, d]; z: [B, H, m]."""
     kv, z, q_t = _f64(kv), _f64(z), _f64(q_t)
     B, H, d = q_t.shape
@@ -329,9 +329,9 @@ def attention_backward(q, k, v, omega, geom, dout, key_mask=None, causal=False):
 
 
 def exact_attention(q, k, v, geom, key_mask=None, causal=False, query_mask=None):
-    """The learned kernel evaluated exactly (README, "Attention modes": the exact
-    path applies the learned geometry to queries and keys before scaled dot-product
-    attention): out_i = sum_j softmax_j(u_i . w_j) v_j with u = M q~, w = M k~,
+    """The learned kernel evaluated exactly (README, "Attention modes": in the
+    exact mode M acts on queries and keys and ordinary softmax attention with
+    scaled scores follows): out_i = sum_j softmax_j(u_i . w_j) v_j with u = M q~, w = M k~,
     x~ = d^{-1/4} x, so the scores are q^T Sigma k / sqrt(d), over the valid keys
     (and j <= i when causal). A row with no visible key, or a masked query row,
     outputs 0.
@@ -365,6 +365,6 @@ def exact_attention(q, k, v, geom, key_mask=None, causal=False, query_mask=None)
 
 
 def uses_exact(L: int, exact_threshold: int) -> bool:
-    """Auto mode (README, "Attention modes"): exact attention through the
-    threshold, linear attention above it."""
+    """Auto mode (README, "Attention modes"): the exact mode for sequences up
+    to the threshold length, random features for longer ones."""
     return exact_threshold > 0 and L <= exact_threshold

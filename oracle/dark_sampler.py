@@ -10,10 +10,10 @@ Sources:
 * DARKformer README ("Data-Aware Random Feature Kernels for Transformers"),
   section "Self-attention": ``orthogonal_features`` chooses orthogonal Gaussian
   blocks (default) or independent Gaussian features; omega_j ~ N(0, I) (section
-  "Kernel"). Section "Projection lifecycle": projections stay fixed until a redraw;
-  ``feature_redraw_interval`` redraws after that many training forwards,
-  evaluation forwards do not count; fixed projections ignore ordinary redraws,
-  ``force`` overrides once; ``projection_seed`` makes the draws reproducible.
+  "Kernel"). Section "Projection lifecycle": a projection is kept until it is
+  redrawn; with a redraw interval a new draw falls due once that many training
+  forwards have run, and forwards outside training are not counted; a fixed
+  projection refuses redraws unless one is forced; a seed reproduces the draws.
 * Philox4x64-10: Salmon, Moraes, Dror and Shaw, "Parallel random numbers: as easy
   as 1, 2, 3" (SC 2011): ten rounds of two 64 x 64 -> 128-bit multiplies with the
   round constants below and a Weyl-sequence key schedule.
@@ -102,7 +102,7 @@ class RedrawSchedule:
 
     interval None: no scheduled redraws; a positive interval redraws after that
     many training forwards (the redraw happens before the next forward, which then
-    uses the new draw). Evaluation forwards do not count. While fixed, a scheduled
+    uses the new draw). Forwards outside training are not counted. While fixed, a scheduled
     redraw that falls due is dropped (the interval restarts) and ordinary manual
     redraws are ignored; a forced manual redraw happens once. Any redraw restarts
     the interval. ``deterministic`` fixes the projection at construction.

@@ -1,6 +1,6 @@
-// Exact learned-kernel attention (README, section "Attention modes": the exact
-// path applies the learned geometry to queries and keys before scaled dot-product
-// attention): out_i = sum_j softmax_j(u_i . w_j) v_j with u = M q~, w = M k~,
+// Exact learned-kernel attention (README, section "Attention modes": in the exact
+// mode M acts on queries and keys and ordinary softmax attention with scaled
+// scores follows): out_i = sum_j softmax_j(u_i . w_j) v_j with u = M q~, w = M k~,
 // x~ = d^{-1/4} x, i.e. scores q^T Sigma k / sqrt(d), over the valid keys (j <= i
 // when causal). A query row with no visible key, or a masked query row in
 // cross-attention, outputs 0.

@@ -4,11 +4,10 @@
 //
 // DARKformer README, section "Kernel": omega_j ~ N(0, I_r); section
 // "Self-attention": orthogonal Gaussian blocks by default, independent features
-// with orthogonal_features=False; section "Projection lifecycle": projections stay
-// fixed until a redraw, a positive feature_redraw_interval redraws after that many
-// training forwards (evaluation forwards do not count), fixed projections ignore
-// ordinary redraws and a forced one happens once, projection_seed makes the draws
-// reproducible.
+// with orthogonal_features=False; section "Projection lifecycle": a projection is
+// kept until it is redrawn, a redraw interval makes one fall due after that many
+// training forwards (forwards outside training are not counted), a fixed
+// projection refuses redraws unless one is forced, and a seed reproduces them.
 //
 // Generator: Philox4x64-10 (Salmon, Moraes, Dror, Shaw, "Parallel random numbers:
 // as easy as 1, 2, 3", SC 2011), key (seed, draw), counter (block, head, purpose,

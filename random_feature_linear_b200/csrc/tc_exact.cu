@@ -1,7 +1,7 @@
 // Exact learned-kernel attention on sm_100a tensor cores (bf16 I/O, d = 64,
 // r <= 64): out_i = sum_j softmax_j(u_i . w_j) v_j with u = M q~, w = M k~
-// (README, section "Attention modes": the exact path applies the learned
-// geometry to queries and keys before scaled dot-product attention).
+// (README, section "Attention modes": in the exact mode M acts on queries and
+// keys and ordinary softmax attention with scaled scores follows).
 //
 // One CTA (256 threads) per 128-query tile of one (batch, head):
 //   Q tile (TMA, bf16 -> fp16) x W'_bot^T -> 2 p_q (fp16, a K-major operand; the

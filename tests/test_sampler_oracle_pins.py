@@ -82,7 +82,7 @@ def test_redraw_schedule_rules():
         s.forward(training=True)
         draws.append(s.draw)
     assert draws == [0, 0, 0, 1, 1, 1, 2]
-    # evaluation forwards do not advance the schedule
+    # forwards outside training are not counted
     s2 = S.RedrawSchedule(seed=7, interval=2)
     seq = [s2.forward(t) for t in (True, False, False, True, True)]
     assert seq == [False, False, False, False, True] and s2.draw == 1
