@@ -14,7 +14,7 @@
  *     orthogonal or independent Gaussian features.
  *   - section "Encoder-decoder model and generation": recurrent statistics
  *     updated per appended token; a state is tied to the projection that made
- *     it and a redraw is detected and rejected.
+ *     it, and statistics from before a redraw are refused.
  *   - section "Mixed precision": bf16 I/O with stable (fp32) accumulation.
  *
  * Conventions shared by every call

@@ -13,8 +13,8 @@ Kernels for Transformers", darkformer-pytorch 0.1.0 package description):
   modules scale both q and k by d_h^{-1/4}; the positive random feature map is
   phi(x; omega_j) = m^{-1/2} exp(omega_j^T M x - 1/2 x^T Sigma x) with
   omega_j ~ N(0, I); attention is Phi(Q)(Phi(K)^T V) / Phi(Q)(Phi(K)^T 1).
-* section "Self-attention": a boolean B x L mask marks valid tokens; causal
-  attention combines the token mask with the causal constraint.
+* section "Self-attention": a boolean B x L mask marks valid tokens; in causal
+  attention a key must be both valid and not later than the query.
 * section "Encoder-decoder model and generation": in linear mode the prompt is
   processed once and recurrent statistics (Phi(K)^T V, Phi(K)^T 1) are then
   updated per appended token; decoder cross-attention summarises the encoded

@@ -100,9 +100,10 @@ def sample_omega(seed: int, draw: int, heads: int, m: int, r: int,
 class RedrawSchedule:
     """The projection lifecycle of the README's "Projection lifecycle" section.
 
-    interval None: no scheduled redraws; a positive interval redraws after that
-    many training forwards (the redraw happens before the next forward, which then
-    uses the new draw). Forwards outside training are not counted. While fixed, a scheduled
+    interval None: no scheduled redraws. With a positive interval a redraw falls
+    due once that many training forwards have run; it happens at the start of the
+    next training forward, which uses the new draw. Forwards outside training are
+    not counted. While fixed, a scheduled
     redraw that falls due is dropped (the interval restarts) and ordinary manual
     redraws are ignored; a forced manual redraw happens once. Any redraw restarts
     the interval. ``deterministic`` fixes the projection at construction.
