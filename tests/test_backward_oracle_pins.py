@@ -5,6 +5,8 @@ mathematics fixes, independently of the oracle's own chain rule:
 * central finite differences of the pinned forward, entry by entry;
 * reverse-mode autograd (torch, fp64) over a different formulation of the same
   function: the explicit L x L matrix of kernel estimates, row-normalised;
+* closed forms: dv = A^T dout with A the row-normalised matrix of kernel
+  estimates; one token gives dv = dout and no other gradient;
 * invariants: shared geometry collects the per-head gradients, a batch row with
   no valid key has zero gradients.
 """
@@ -122,3 +124,34 @@ def test_rows_without_visible_keys_have_zero_gradients():
     assert np.all(dq[1, :, :2] == 0)
     assert np.all(dk[1, :, :2] == 0) and np.all(dv[1, :, :2] == 0)
     assert np.abs(dq[1, :, 2:]).max() > 0
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_value_gradient_is_the_transposed_attention_matrix(causal):
+    # out = A v with A the row-normalised matrix of kernel estimates over the
+    # visible keys, so dv = A^T dout exactly (a closed form, from the L x L matrix)
+    q, k, v, om, gm, g = _inputs(11, L=12, heads_geom=2, heads_omega=1)
+    mask = np.ones((2, 12), np.uint8)
+    mask[1, [2, 7]] = 0
+    _, _, dv, _ = O.attention_backward(q, k, v, om, gm, g, key_mask=mask, causal=causal)
+    for b in range(2):
+        for h in range(2):
+            phq = O.feature_map(q[b, h], om[0], gm[h])
+            phk = O.feature_map(k[b, h], om[0], gm[h])
+            kmat = phq @ phk.T
+            kmat[:, mask[b] == 0] = 0.0
+            if causal:
+                kmat = np.tril(kmat)
+            a = kmat / kmat.sum(axis=1, keepdims=True)
+            ref = a.T @ g[b, h]
+            assert np.abs(dv[b, h] - ref).max() <= 1e-12 * np.abs(ref).max()
+
+
+def test_single_token_closed_form():
+    # one token: out = v exactly, so dv = dout and every other gradient is zero
+    q, k, v, om, gm, g = _inputs(12, L=1)
+    dq, dk, dv, dgm = O.attention_backward(q, k, v, om, gm, g, causal=True)
+    assert np.abs(dv - g).max() <= 1e-12
+    scale = np.abs(g).max()
+    for x in (dq, dk, dgm):
+        assert np.abs(x).max() <= 1e-12 * scale
