@@ -217,3 +217,21 @@ def test_sampler_rejects_bad_arguments(D):
     assert lib.dark_sample_omega(1, 0, 1, 256, 64, 1, f, f + 16, need, None) == 1
     assert lib.dark_sample_omega(1, 0, 1, 256, 512, 1, f, f, 1 << 40, None) == 2
     assert lib.dark_sample_omega(1, 0, 1, 4096, 64, 0, f, None, 0, None) == 2
+
+
+def test_binding_takes_strides_from_the_tensors(D):
+    import torch
+    x = torch.zeros(2, 3, 5, 8)
+    assert list(D._strides(None, x)) == [120, 40, 8]
+    # a [B][L][H][d] buffer viewed as [B][H][L][d]
+    y = torch.zeros(2, 5, 3, 8).permute(0, 2, 1, 3)
+    assert list(D._strides(None, y, y)) == [120, 8, 24]
+    # explicit strides win
+    assert list(D._strides((1, 2, 3), x)) == [1, 2, 3]
+    with pytest.raises(ValueError):
+        D._strides(None, x, y)                     # q, k, v must share one layout
+    with pytest.raises(ValueError):
+        D._strides(None, torch.zeros(2, 3, 8, 5).transpose(2, 3))   # d must be innermost
+    with pytest.raises(ValueError):
+        D._dense(torch.zeros(4, 6)[:, ::2], "mask")  # arrays without strides must be dense
+    assert D._dense(None, "mask") is None
