@@ -337,3 +337,47 @@ def test_exponents_stay_in_range_for_workloads():
         inp = synth.make_inputs(w)
         lo, hi = O.exponent_range(inp["k"][0, 0], inp["omega"][0], inp["geom"][0])
         assert -80 < lo and hi < 40, (cfg, lo, hi)
+
+
+def test_feature_exponents_hand_values():
+    # README, "Kernel": the exponent of phi_j(x) is omega_j^T M x~ - 1/2 |M x~|^2
+    # (x~ = d^{-1/4} x) and phi carries the factor m^{-1/2}. Hand-derived cases:
+    # (1) the two-token example (d = r = 1, M = 1, Omega = [1; -1]): x = 1 gives
+    #     [1 - 1/2, -1 - 1/2], x = -1 gives [-3/2, 1/2], x = -1/2 gives [-5/8, 3/8].
+    g = json.load(open(os.path.join(GOLDEN, "two_token_worked_example.json")))
+    om, gm = np.array(g["omega"]), np.array(g["geom"])
+    x = np.array([[1.0], [-1.0], [-0.5]])
+    e = O.feature_exponents(x, om, gm)
+    np.testing.assert_allclose(e, [[0.5, -1.5], [-1.5, 0.5], [-0.625, 0.375]], atol=1e-15)
+    lo, hi = O.exponent_range(x, om, gm)
+    assert abs(lo - (-1.5 - 0.5 * np.log(2))) < 1e-15 and abs(hi - (0.5 - 0.5 * np.log(2))) < 1e-15
+    # (2) d = r = 4 so that d^{-1/4} = 2^{-1/2} matters, M = 2 I: x = (sqrt 2, 0, 0, 0)
+    #     gives x~ = e_1, M x~ = 2 e_1 and 1/2 |M x~|^2 = 2; omega = e_1, e_2, -e_1
+    #     and 3 e_1 + e_4 give exponents 2 - 2, 0 - 2, -2 - 2 and 6 - 2.
+    om4 = np.array([[1.0, 0, 0, 0], [0, 1.0, 0, 0], [-1.0, 0, 0, 0], [3.0, 0, 0, 1.0]])
+    x4 = np.array([[np.sqrt(2.0), 0, 0, 0]])
+    e4 = O.feature_exponents(x4, om4, 2.0 * np.eye(4))
+    np.testing.assert_allclose(e4, [[0.0, -2.0, -4.0, 4.0]], atol=1e-14)
+    lo4, hi4 = O.exponent_range(x4, om4, 2.0 * np.eye(4))
+    assert abs(lo4 - (-4.0 - np.log(2))) < 1e-14 and abs(hi4 - (4.0 - np.log(2))) < 1e-14
+    # (3) low rank, r = 2 < d = 4: M x~ keeps two coordinates only
+    gm2 = np.array([[1.0, 1.0, 0, 0], [0, 0, 2.0, 0]])
+    x2 = np.array([[2.0, 0.0, 1.0, 5.0]]) * np.sqrt(2.0)      # x~ = (2, 0, 1, 5)
+    om2 = np.array([[1.0, 0.0], [0.0, -1.0]])
+    # M x~ = (2, 2), 1/2 |M x~|^2 = 4; exponents 2 - 4 and -2 - 4
+    np.testing.assert_allclose(O.feature_exponents(x2, om2, gm2), [[-2.0, -6.0]], atol=1e-14)
+
+
+def test_feature_exponents_agree_with_feature_map():
+    # exponent_range bounds log(phi) itself: the log of the pinned feature map
+    # (times sqrt(m) for the exponents) on random recipes, with per-head geometry
+    rng = np.random.default_rng(11)
+    for d, r, m in ((64, 64, 256), (64, 32, 128), (16, 8, 8)):
+        x = rng.standard_normal((50, d))
+        om = rng.standard_normal((m, r))
+        gm = np.eye(r, d) + 0.1 * rng.standard_normal((r, d))
+        phi = O.feature_map(x, om, gm)
+        np.testing.assert_allclose(O.feature_exponents(x, om, gm), np.log(phi * np.sqrt(m)),
+                                   rtol=0, atol=1e-12)
+        lo, hi = O.exponent_range(x, om, gm)
+        assert abs(lo - np.log(phi).min()) < 1e-12 and abs(hi - np.log(phi).max()) < 1e-12
