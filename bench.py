@@ -1,8 +1,10 @@
 """Benchmark of the DARKformer PRF attention forward pass on B200.
 
-Default workload: causal, key-masked bf16 attention, B=2 H=8 L=2048 d=64 r=64
-m=256 with orthogonal features and valid lengths 2048/1500 (the standard
-workload of the method's causal path; seeded synthetic inputs).
+Default workload: the large-head causal forward, bf16, B=4 H=8 L=8192 d=256
+r=256 m=512 with orthogonal features and anisotropic queries and keys (the
+largest single-GPU configuration of the method's forward path; seeded
+synthetic inputs), followed by the streaming decode step (B=64 H=8 d=64
+m=256 after a 4096-token prefill), reported under the key "decode".
 
 One JSON line on rank 0. `value` is whole-job forward tokens/s (B*H*L per
 step, summed over ranks) with inputs resident in HBM and L2 flushed before
@@ -177,13 +179,43 @@ def oracle_sample(w: synth.Workload, inp: dict, max_seconds: float = 20.0, exact
     return done_tokens / t_total, done_tokens, t_total, heads
 
 
-def blas_threads() -> int:
+def host_cores() -> int:
+    """Cores this process may run on (its CPU affinity set)."""
+    return len(os.sched_getaffinity(0))
+
+
+def cpu_model() -> str:
     try:
-        from threadpoolctl import threadpool_info
-        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
-        return max(n) if n else 1
-    except Exception:
-        return 1
+        with open("/proc/cpuinfo") as fh:
+            for line in fh:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
+class oracle_threads:
+    """Runs the oracle's numpy/BLAS work on every core of the affinity set, so
+    that the reported core count is the thread count actually used."""
+
+    def __enter__(self):
+        self.n = host_cores()
+        self.ctl = None
+        try:
+            from threadpoolctl import threadpool_limits
+            self.ctl = threadpool_limits(limits=self.n)
+        except Exception:
+            self.ctl = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.ctl is not None:
+            self.ctl.restore_original_limits()
+
+
+def cpu_info(n: int) -> dict:
+    return {"cores": n, "cpu_model": cpu_model()}
 
 
 def count_launches(fn) -> tuple[int, list]:
@@ -340,8 +372,9 @@ def run_native(args, w: synth.Workload, rank: int, world: int, dev) -> dict | No
         roof["traffic"] = captured_traffic(args.workload)
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
-        tps, ntok, secs, heads = oracle_sample(w, inp, exact=args.exact)
-        cpu = dict(value=tps, unit="tokens/s", cores=blas_threads(), kind="oracle",
+        with oracle_threads() as ot:
+            tps, ntok, secs, heads = oracle_sample(w, inp, exact=args.exact)
+        cpu = dict(value=tps, unit="tokens/s", kind="oracle", **cpu_info(ot.n),
                    sample=f"{heads} of {w.B * w.H} (batch, head) slices, {ntok} tokens, {secs:.1f} s")
     clocks = clk.summary()
     return {
@@ -509,9 +542,10 @@ def run_decode(args, rank: int, world: int, dev) -> dict | None:
         kv0 = st_t[0][:1].double().cpu().numpy()
         z0 = st_t[1][:1].double().cpu().numpy()
         sub = {n: stream_np[n][:, :1] for n in ("q", "k", "v")}
-        rps, nsteps, secs = oracle_decode_sample(w.with_sizes(B=1), kv0, z0, sub, inp["omega"],
-                                                 inp["geom"])
-        cpu = dict(value=rps, unit="tokens/s", cores=blas_threads(), kind="oracle",
+        with oracle_threads() as ot:
+            rps, nsteps, secs = oracle_decode_sample(w.with_sizes(B=1), kv0, z0, sub,
+                                                     inp["omega"], inp["geom"])
+        cpu = dict(value=rps, unit="tokens/s", kind="oracle", **cpu_info(ot.n),
                    sample=f"batch row 0 ({w.H} heads), {nsteps} decode steps, {secs:.1f} s")
     clocks = clk.summary()
     return {
@@ -660,19 +694,20 @@ def run_cross(args, rank: int, world: int, dev) -> dict | None:
     if world == 1 and not args.no_cpu_baseline:
         from oracle import dark_oracle as O
         qn, kn, vn = iq["q"], ik["k"], ik["v"]
-        t0, heads = time.perf_counter(), 0
-        for b in range(w.B):
-            for h in range(w.H):
-                sl = (slice(b, b + 1), slice(h, h + 1))
-                O.cross_attention(qn[sl], kn[sl], vn[sl], iq["omega"], iq["geom"][h:h + 1])
-                heads += 1
-                if time.perf_counter() - t0 > 10.0:
-                    break
-            else:
-                continue
-            break
-        secs = time.perf_counter() - t0
-        cpu = dict(value=heads * (lq + lk) / secs, unit="tokens/s", cores=blas_threads(),
+        with oracle_threads() as ot:
+            t0, heads = time.perf_counter(), 0
+            for b in range(w.B):
+                for h in range(w.H):
+                    sl = (slice(b, b + 1), slice(h, h + 1))
+                    O.cross_attention(qn[sl], kn[sl], vn[sl], iq["omega"], iq["geom"][h:h + 1])
+                    heads += 1
+                    if time.perf_counter() - t0 > 10.0:
+                        break
+                else:
+                    continue
+                break
+            secs = time.perf_counter() - t0
+        cpu = dict(value=heads * (lq + lk) / secs, unit="tokens/s", **cpu_info(ot.n),
                    kind="oracle", sample=f"{heads} of {w.B * w.H} (batch, head) slices, {secs:.1f} s")
     clocks = clk.summary()
     return {
@@ -826,18 +861,19 @@ def run_backward(args, w: synth.Workload, rank: int, world: int, dev) -> dict | 
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
         from oracle import dark_oracle as O
-        t0, heads = time.perf_counter(), 0
-        for h in range(w.H):
-            sl = (slice(0, 1), slice(h, h + 1))
-            gm = inp["geom"][h:h + 1] if inp["geom"].shape[0] > 1 else inp["geom"]
-            O.attention_backward(inp["q"][sl], inp["k"][sl], inp["v"][sl], inp["omega"], gm,
-                                 dout_np[sl], key_mask=None if inp["mask"] is None
-                                 else inp["mask"][:1], causal=w.causal)
-            heads += 1
-            if time.perf_counter() - t0 > 10.0:
-                break
-        secs = time.perf_counter() - t0
-        cpu = dict(value=heads * w.L / secs, unit="tokens/s", cores=blas_threads(), kind="oracle",
+        with oracle_threads() as ot:
+            t0, heads = time.perf_counter(), 0
+            for h in range(w.H):
+                sl = (slice(0, 1), slice(h, h + 1))
+                gm = inp["geom"][h:h + 1] if inp["geom"].shape[0] > 1 else inp["geom"]
+                O.attention_backward(inp["q"][sl], inp["k"][sl], inp["v"][sl], inp["omega"], gm,
+                                     dout_np[sl], key_mask=None if inp["mask"] is None
+                                     else inp["mask"][:1], causal=w.causal)
+                heads += 1
+                if time.perf_counter() - t0 > 10.0:
+                    break
+            secs = time.perf_counter() - t0
+        cpu = dict(value=heads * w.L / secs, unit="tokens/s", **cpu_info(ot.n), kind="oracle",
                    sample=f"{heads} of {w.B * w.H} (batch, head) slices, {secs:.1f} s")
     clocks = clk.summary()
     return {
@@ -911,15 +947,15 @@ def run_sample(args, rank: int, world: int, dev) -> dict | None:
 
 def run_reference(args, w: synth.Workload) -> dict:
     inp = synth.make_inputs(w)
-    for _ in range(args.warmup):
-        oracle_sample(w, inp, max_seconds=1.0)
-    vals, details = [], None
-    for _ in range(args.steps):
-        tps, ntok, secs, heads = oracle_sample(w, inp, max_seconds=args.ref_seconds)
-        vals.append(tps)
-        details = (ntok, secs, heads)
+    with oracle_threads() as ot:
+        for _ in range(args.warmup):
+            oracle_sample(w, inp, max_seconds=1.0)
+        vals, details = [], None
+        for _ in range(args.steps):
+            tps, ntok, secs, heads = oracle_sample(w, inp, max_seconds=args.ref_seconds)
+            vals.append(tps)
+            details = (ntok, secs, heads)
     value = statistics.median(vals)
-    cores = blas_threads()
     sample = f"{details[2]} of {w.B * w.H} (batch, head) slices per step, {details[0]} tokens"
     return {
         "impl": "reference",
@@ -930,8 +966,8 @@ def run_reference(args, w: synth.Workload) -> dict:
         "data": "synthetic (seeded numpy, orthogonal Gaussian features)",
         "config": {"workload": w.name, "B": w.B, "H": w.H, "L": w.L, "d": w.d, "r": w.r,
                    "m": w.m, "causal": w.causal},
-        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
-                         "sample": sample},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "kind": "oracle",
+                         "sample": sample, **cpu_info(ot.n)},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
@@ -943,8 +979,11 @@ def main():
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["native", "reference"], default="native")
-    ap.add_argument("--workload", type=int, default=2, help="synthetic workload recipe (1-5)")
-    ap.add_argument("--ref-seconds", type=float, default=10.0)
+    ap.add_argument("--workload", type=int, default=4, help="synthetic workload recipe (1-5)")
+    ap.add_argument("--ref-seconds", type=float, default=None,
+                    help="CPU seconds per reference step (default: about 120 s over all steps)")
+    ap.add_argument("--no-decode", action="store_true",
+                    help="leave the decode step out of the forward run's JSON line")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-profile", action="store_true",
                     help="do not count launches with the CUDA profiler (for runs under ncu)")
@@ -962,10 +1001,22 @@ def main():
                     help="capture mode: only warmup + steps forward calls, no timing or output")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
+    if args.ref_seconds is None:
+        args.ref_seconds = max(1.0, min(10.0, 120.0 / max(args.steps + args.warmup, 1)))
     w = synth.WORKLOADS[args.workload]
 
+    if "WORLD_SIZE" not in os.environ and args.gpus > 1:
+        # one process per GPU: relaunch this command under torchrun
+        cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1",
+               f"--nproc-per-node={args.gpus}", "--master-addr", "127.0.0.1",
+               "--master-port", os.environ.get("MASTER_PORT", "29511"),
+               os.path.abspath(__file__), *sys.argv[1:]]
+        os.execv(sys.executable, cmd)
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
+    if world != args.gpus:
+        raise SystemExit(f"bench.py: --gpus {args.gpus} but WORLD_SIZE is {world}; "
+                         "launch one process per GPU (torchrun --nproc-per-node N)")
     if args.impl == "reference":
         if rank == 0:
             print(json.dumps(run_reference(args, w)), flush=True)
@@ -988,6 +1039,10 @@ def main():
             res = run_sample(args, rank, world, dev)
         else:
             res = run_native(args, w, rank, world, dev)
+            if not (args.no_decode or args.ncu or args.exact):
+                dec = run_decode(args, rank, world, dev)
+                if res is not None:
+                    res["decode"] = dec
         if res is not None:
             print(json.dumps(res), flush=True)
     finally:

@@ -176,9 +176,10 @@ dark_status dark_attention_fwd(const dark_projection* proj, const void* q, const
 
 /*
  * dark_attention_fwd without a caller workspace, for callers that cannot
- * allocate device memory (for example code running inside a CUDA-graph capture
- * it does not own, or under an allocator that refuses extra allocations). The
- * method's pages have no counterpart of this call; it is a deployment aid.
+ * allocate device memory (for example a runtime that hands the library only the
+ * tensors of the call, or code under an allocator that refuses extra
+ * allocations). The method's pages have no counterpart of this call; it is a
+ * deployment aid.
  * Arguments and results are those of dark_attention_fwd minus ws/ws_bytes; the
  * scratch is a fixed array of dark_noalloc_scratch_bytes() (16 MiB) compiled into
  * the library, which every GPU that loads the library keeps until the process
@@ -188,6 +189,9 @@ dark_status dark_attention_fwd(const dark_projection* proj, const void* q, const
  *     would need with a workspace of its own).
  *   - The first call on each device looks up the array's device address
  *     (cudaGetSymbolAddress); make that first call before any stream capture.
+ *     The address is kept for the life of the process: after cudaDeviceReset
+ *     (or any other teardown of the device's primary context) do not call this
+ *     entry point again in that process.
  *   - Every call shares the one array and it keeps the previous call's
  *     contents: calls whose work overlaps on the GPU (different streams, or
  *     different host threads without ordering) race on it. Serialise them.

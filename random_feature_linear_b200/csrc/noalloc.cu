@@ -1,8 +1,7 @@
 // dark_attention_fwd_noalloc: the forward pass for callers that cannot
 // allocate device memory. Some hosts run this library where cudaMalloc is not
-// available to them: inside a CUDA-graph capture they do not control, under an
-// allocator that forbids extra allocations, or in a runtime that hands the
-// library only the tensors of the call. They still own their inputs and
+// available to them: under an allocator that forbids extra allocations, or in a
+// runtime that hands the library only the tensors of the call. They still own their inputs and
 // outputs; the scratch that dark_attention_fwd takes as a caller workspace
 // comes here from one fixed array compiled into the library.
 #include <mutex>
@@ -20,7 +19,9 @@ constexpr int kMaxDevices = 64;
 std::mutex g_mu;
 void* g_scratch_addr[kMaxDevices];
 
-// Device address of the array on the current device; looked up once per device.
+// Device address of the array on the current device; looked up once per device
+// and kept for the life of the process (the header tells callers not to use
+// this entry point after a device reset, which would invalidate it).
 // In host code `g_noalloc_scratch` only names a host-side shadow, so its address
 // must come from cudaGetSymbolAddress with the device current.
 cudaError_t scratch_for_current_device(void** out) {

@@ -204,22 +204,6 @@ __device__ __forceinline__ float ex2(float x) {
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
-// 2^x on the FMA pipe, to take part of the exponentials off the MUFU unit:
-// n = round(x) from one add of 1.5 * 2^23 (n lands in the low mantissa bits),
-// 2^f for f = x - n in [-1/2, 1/2] from a cubic with 7.5e-5 maximum relative
-// error (coefficients fitted by exp2_poly.py), and 2^n added to the exponent
-// field. x is clamped to [-126, 128]: smaller results are below what bf16
-// operands keep; from 2^128 up the result saturates at ~3.4e38, the top of the
-// fp32 range (any product with it overflows in the fp32 accumulators).
-__device__ __forceinline__ float ex2_fma(float x) {
-  x = fminf(fmaxf(x, -126.f), 128.f);
-  const float big = 12582912.f;
-  const float t = x + big;
-  const float f = x - (t - big);
-  const float p = fmaf(fmaf(fmaf(0.0551716685295105f, f, 0.2426111251115799f), f,
-                            0.6932609677314758f), f, 0.9999280571937561f);
-  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
-}
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<const uint32_t*>(&v);
@@ -241,15 +225,6 @@ __device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
                : "memory");
   return v;
 }
-__device__ __forceinline__ void st_release_u64(uint64_t* p, uint64_t v) {
-  asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
-}
-__device__ __forceinline__ uint64_t ld_acquire_u64(const uint64_t* p) {
-  uint64_t v;
-  asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
-  return v;
-}
-
 // Byte offset of element (row, k) in a K-major 128B-swizzled tile whose 64-element
 // K blocks are `kblock_bytes` apart (16-bit elements; rows grouped 8 per atom).
 __host__ __device__ constexpr uint32_t kmajor_off(int row, int k, uint32_t kblock_bytes) {

@@ -1,17 +1,21 @@
 """dark_attention_fwd_noalloc against dark_attention_fwd (GPU, through the C ABI).
 
-The no-allocation entry point serves callers that cannot call cudaMalloc (code
-inside someone else's CUDA-graph capture, or under an allocator that refuses
-extra allocations): its scratch is a fixed array inside the library. It must
-give the same results as the workspace entry point, call after call, even
-though every call reuses the same scratch. This file is collected last so that
-a run stopping at its first failure has run everything else before it.
+The no-allocation entry point serves callers that cannot call cudaMalloc (a
+runtime that hands the library only the tensors of the call, or an allocator
+that refuses extra allocations): its scratch is a fixed array inside the
+library. It must give the same results as the workspace entry point, and the
+fp64 oracle's within the forward tolerances, call after call, even though every
+call reuses the same scratch. This file is collected last so that a run
+stopping at its first failure has run everything else before it.
 """
 import numpy as np
 import pytest
 import torch
 
+from oracle import dark_oracle as O
 from random_feature_linear_b200 import synth
+
+from gpu_run import check
 
 pytestmark = pytest.mark.gpu
 
@@ -69,6 +73,10 @@ def test_noalloc_matches_workspace_entry_twice(D, cuda_ok, w):
             assert np.abs(got - ref).max() <= 2e-2
         np.testing.assert_allclose(kv, kv_ref, rtol=1e-4, atol=1e-6 * np.abs(kv_ref).max())
         np.testing.assert_allclose(z, z_ref, rtol=1e-4, atol=1e-6 * np.abs(z_ref).max())
+        # and the fp64 oracle on the same inputs
+        want, _, _ = O.attention(inp["q"], inp["k"], inp["v"], inp["omega"], inp["geom"],
+                                 key_mask=inp["mask"], causal=w.causal)
+        check(w, got, want)
 
 
 def test_noalloc_rejects_calls_beyond_its_scratch(D, cuda_ok):
