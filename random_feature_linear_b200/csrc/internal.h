@@ -75,6 +75,8 @@ cudaError_t simt_forward(const FwdArgs& a);
 // Alignment/stride/shape checks shared by the tensor-core paths, then the
 // TMA descriptors (false if any check fails or the driver rejects a layout).
 bool tc_make_maps(FwdArgs& a);
+// Streaming multiprocessors of the current device (looked up once per device).
+int num_sms();
 // Sets a kernel's dynamic shared memory limit once per device.
 cudaError_t set_smem_limit_once(const void* kernel, int bytes, int* done_per_device);
 

@@ -57,6 +57,19 @@ bool tc_make_maps(FwdArgs& a) {
   return a.maps_ready;
 }
 
+int num_sms() {
+  static int count[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  if (count[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+      n = 148;
+    count[dev] = n;
+  }
+  return count[dev];
+}
+
 cudaError_t set_smem_limit_once(const void* kernel, int bytes, int* done_per_device) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);

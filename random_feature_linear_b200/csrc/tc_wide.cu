@@ -114,28 +114,39 @@ __device__ __forceinline__ void warp_arrive(uint64_t* bar) {
 }
 
 // ================================================================ launch 1 ==
+// Persistent: each CTA walks a contiguous range of (head, chunk) items. Per
+// item the key and query tiles sit side by side in shared memory as one
+// 256-token operand [K_c ; Q_c] (fp16, d in 64-column slabs), so that every
+// feature GEMM is a full-width MMA: W'_f (128 feature rows, M = 128) times the
+// 256 tokens (N = 256), accumulated over d. The TMEM result holds feature f of
+// the block in lane f and token t in column t (keys 0-127, queries 128-255),
+// which is exactly the layout the value launch wants for its operands:
+// Phi_f^T with features as rows (the A operand of the state update) and
+// Psi_f^T with features as rows (the MN-major A operand of the prefix
+// product). The key norms come first from a tokens x r GEMM (keys as M) and go
+// to shared memory as one base-2 offset per key, +inf for masked keys (whose
+// features are then exp2(-inf) = 0).
 template <int D_, int M_, int R_>
 struct FeatCfg {
-  static constexpr int DS = D_ / 64;                       // 64-column slabs of d
-  // W' items: first one per d slab with all R_ norm rows (one N = R_ MMA per
-  // K-step), then 64 feature rows over all of d
-  static constexpr int NNORM = DS, NFEAT = M_ / 64;
-  static constexpr int NITEMS = NNORM + NFEAT;
-  static constexpr uint32_t kX = DS * 16384;               // one 128-token tile, fp16
-  static constexpr uint32_t kSlot = DS * 8192;             // 64 W' rows x d, fp16
-  static constexpr uint32_t oXK = 0, oXQ = kX, oST = 2 * kX;   // staging: Phi_n | Psi_n, later A
-  static constexpr uint32_t oW = oST + 32768;
-  static constexpr int kSlotsFit = (int)((kSmemBudget - oW) / kSlot);
+  static constexpr int DS = D_ / 64;                     // 64-column slabs of d
+  static constexpr int NB = M_ / 128;                    // feature blocks of 128
+  static constexpr int NRH = R_ > 128 ? R_ / 128 : 1;    // norm row groups per slab
+  static constexpr int NRROWS = R_ > 128 ? 128 : R_;     // rows per norm item
+  static constexpr int NNORM = DS * NRH;                 // ring items: norm rows first,
+  static constexpr int NITEMS = NNORM + NB * DS;         // then W' block f, slab s
+  static constexpr uint32_t kXSlab = 32768;              // 256 token rows x 128 B
+  static constexpr uint32_t oX = 0;
+  static constexpr uint32_t oST = DS * kXSlab;           // staging: Phi_f | Psi_f (32 KB each)
+  static constexpr uint32_t oW = oST + 65536;            // ring of 16 KB slots
+  static constexpr int kSlotsFit = (int)((kSmemBudget - oW) / 16384);
   static constexpr int NSLOT = kSlotsFit > 6 ? 6 : kSlotsFit;
-  static constexpr uint32_t oBar = oW + NSLOT * kSlot;
-  static constexpr uint32_t kSmem = oBar + 1024 + 1024 + 1024;   // barriers, norm exchange, slack
-  // TMEM: norms [0, R_) first; then P blocks (keys at 128 b, queries at 128 b + 64,
-  // b = block parity) over the same columns; scores [256, 384)
-  static constexpr uint32_t tS = 256;
+  static constexpr uint32_t oBar = oW + NSLOT * 16384;
+  static constexpr uint32_t kSmem = oBar + 2048 + 1024;  // barriers, norms, exchange, slack
+  static constexpr uint32_t tF = 0, tN = 256;            // TMEM: F block | norms, then scores
   static_assert(D_ % 64 == 0 && D_ >= 128 && D_ <= 256, "d");
-  static_assert(M_ % 128 == 0 && M_ <= 512 && R_ % 64 == 0 && R_ >= 64 && R_ <= 256, "m, r");
+  static_assert(M_ % 128 == 0 && M_ <= 512, "m");
+  static_assert(R_ % 64 == 0 && R_ >= 64 && R_ <= 256, "r");
   static_assert(NSLOT >= 2, "shared memory");
-  static_assert(R_ * 128 <= kSlot, "norm item");
 };
 
 // Bytes of one chunk's record in the workspace: Phi image, Psi image, A image.
@@ -146,7 +157,7 @@ __host__ __device__ constexpr size_t chunk_record_bytes(int m) {
 struct FeatParams {
   const uint8_t* mask;
   uint8_t* img;            // chunk records [B*H][nc]
-  int B, H, L, nc, heads_w;
+  int B, H, L, nc, heads_w, nitems;
   int* dev_status;
 };
 
@@ -159,36 +170,41 @@ __global__ void __launch_bounds__(kThreadsF, 1)
   uint8_t* sm = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   const uint32_t s0 = smem_u32(sm);
   uint64_t* bars = (uint64_t*)(sm + G::oBar);
-  uint64_t* bar_x = bars + 0;
-  uint64_t* bar_conv = bars + 1;        // epilogue: tiles converted to fp16 (8 arrivals)
-  uint64_t* bar_norm = bars + 2;        // MMA: norm GEMM done
-  uint64_t* bar_nread = bars + 3;       // epilogue: norm columns read (8)
-  uint64_t* bar_pfull = bars + 4;       // [2] MMA: P block ready
-  uint64_t* bar_stage = bars + 6;       // epilogue: P block read, staging written (8)
-  uint64_t* bar_sfree = bars + 7;       // MMA: scores GEMM of the staged block done
-  uint64_t* bar_full = bars + 8;        // [NSLOT] W' slot loaded
-  uint64_t* bar_empty = bars + 16;      // [NSLOT] W' slot read by the MMAs
-  uint64_t* bar_drain = bars + 24;      // MMA: everything issued has completed (abort path)
-  uint32_t* tmem_slot = (uint32_t*)(bars + 25);
-  volatile int* abort_flag = (volatile int*)(bars + 26);
-  float* nrm_x = (float*)(sm + G::oBar + 1024);   // [2][128] norm halves
+  uint64_t* bar_x = bars + 0;       // producer: token tiles loaded
+  uint64_t* bar_conv = bars + 1;    // epilogue: tiles converted; TMEM norm/score region free (8)
+  uint64_t* bar_norm = bars + 2;    // MMA: norm GEMM done
+  uint64_t* bar_nread = bars + 3;   // epilogue: norms read (8)
+  uint64_t* bar_ffull = bars + 4;   // MMA: feature block in TMEM
+  uint64_t* bar_ffree = bars + 5;   // epilogue: feature block read (8)
+  uint64_t* bar_stage = bars + 6;   // epilogue: Phi_f, Psi_f staged (8)
+  uint64_t* bar_sfree = bars + 7;   // MMA: scores GEMM of the staged block done
+  uint64_t* bar_xfree = bars + 8;   // MMA: every GEMM reading the token tiles done
+  uint64_t* bar_sc = bars + 9;      // MMA: scores complete
+  uint64_t* bar_drain = bars + 10;  // MMA: everything issued has completed (abort path)
+  uint64_t* bar_full = bars + 16;   // [NSLOT] ring slot loaded
+  uint64_t* bar_empty = bars + 24;  // [NSLOT] ring slot read by the MMAs
+  uint32_t* tmem_slot = (uint32_t*)(bars + 32);
+  volatile int* abort_flag = (volatile int*)(bars + 33);
+  float* nrm_s = (float*)(sm + G::oBar + 1024);          // [128] key offsets
+  float* nrm_x = (float*)(sm + G::oBar + 1536);          // [128] second half sums
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int bh = blockIdx.x / p.nc, c = blockIdx.x % p.nc;
-  const int b = bh / p.H, h = bh % p.H;
-  const int hw = p.heads_w == 1 ? 0 : h;
-  const int t0 = c * kC;
-  uint8_t* rec = p.img + ((size_t)bh * p.nc + c) * chunk_record_bytes(M_);
+  // this CTA's contiguous range of (head, chunk) items
+  const int per = p.nitems / gridDim.x, extra = p.nitems % gridDim.x;
+  const int it0 = blockIdx.x * per + (blockIdx.x < extra ? blockIdx.x : extra);
+  const int nit = per + (blockIdx.x < extra ? 1 : 0);
 
   if (tid == 0) {
     mbar_init(bar_x, 1);
     mbar_init(bar_conv, 8);
     mbar_init(bar_norm, 1);
     mbar_init(bar_nread, 8);
-    mbar_init(bar_pfull + 0, 1);
-    mbar_init(bar_pfull + 1, 1);
+    mbar_init(bar_ffull, 1);
+    mbar_init(bar_ffree, 8);
     mbar_init(bar_stage, 8);
     mbar_init(bar_sfree, 1);
+    mbar_init(bar_xfree, 1);
+    mbar_init(bar_sc, 1);
     mbar_init(bar_drain, 1);
     for (int i = 0; i < G::NSLOT; ++i) {
       mbar_init(bar_full + i, 1);
@@ -205,41 +221,52 @@ __global__ void __launch_bounds__(kThreadsF, 1)
 
   if (warp == 9) {
     // ------------------------------------------------------------ producer
-    // the token tiles, then the W' items in consumption order, each into the
-    // slot its predecessor NSLOT back has left
+    // per item: the token tiles (once the previous item's GEMMs have read
+    // them), then the ring items in consumption order
     if (lane == 0) {
       prefetch_tmap(&tm_w);
       prefetch_tmap(&tm_q);
       prefetch_tmap(&tm_k);
-      mbar_arrive_expect_tx(bar_x, 2 * G::kX);
-      for (int s = 0; s < G::DS; ++s) {
-        tma_load_4d(sm + G::oXK + s * 16384, &tm_k, 64 * s, t0, h, b, bar_x);
-        tma_load_4d(sm + G::oXQ + s * 16384, &tm_q, 64 * s, t0, h, b, bar_x);
-      }
       int last[G::NSLOT];
       for (int i = 0; i < G::NSLOT; ++i) last[i] = -1;
       bool ok = true;
-      for (int i = 0; ok && i < G::NITEMS; ++i) {
-        const int slot = i % G::NSLOT;
-        if (i >= G::NSLOT &&
-            !(ok = wait_one(bar_empty + slot, ((i / G::NSLOT) - 1) & 1, abort_flag, p.dev_status)))
-          break;
-        uint8_t* dst = sm + G::oW + slot * G::kSlot;
-        if (i < G::NNORM) {          // norm rows, d slab i
-          mbar_arrive_expect_tx(bar_full + slot, R_ * 128);
-          for (int j = 0; j < R_ / 64; ++j)
-            tma_load_2d(dst + j * 8192, &tm_w, 64 * i, hw * (M_ + R_) + M_ + 64 * j, bar_full + slot);
-        } else {                     // feature rows 64 (i - NNORM) .. + 63, all of d
-          mbar_arrive_expect_tx(bar_full + slot, G::kSlot);
-          for (int s = 0; s < G::DS; ++s)
-            tma_load_2d(dst + s * 8192, &tm_w, 64 * s, hw * (M_ + R_) + 64 * (i - G::NNORM),
-                        bar_full + slot);
+      int xlast = -1;
+      int g = 0;   // ring items issued so far (over all items)
+      for (int j = 0; ok && j < nit; ++j) {
+        const int item = it0 + j, bh = item / p.nc, c = item % p.nc;
+        const int b = bh / p.H, h = bh % p.H, hw = p.heads_w == 1 ? 0 : h;
+        if (j > 0 && !(ok = wait_one(bar_xfree, (j - 1) & 1, abort_flag, p.dev_status))) break;
+        mbar_arrive_expect_tx(bar_x, 2 * G::DS * 16384);
+        for (int s = 0; s < G::DS; ++s) {
+          tma_load_4d(sm + G::oX + s * G::kXSlab, &tm_k, 64 * s, c * kC, h, b, bar_x);
+          tma_load_4d(sm + G::oX + s * G::kXSlab + 16384, &tm_q, 64 * s, c * kC, h, b, bar_x);
         }
-        last[slot] = i;
+        xlast = j;
+        for (int i = 0; i < G::NITEMS; ++i, ++g) {
+          const int slot = g % G::NSLOT;
+          if (g >= G::NSLOT &&
+              !(ok = wait_one(bar_empty + slot, ((g / G::NSLOT) - 1) & 1, abort_flag, p.dev_status)))
+            break;
+          uint8_t* dst = sm + G::oW + slot * 16384;
+          const int wrow0 = hw * (M_ + R_);
+          if (i < G::NNORM) {          // norm rows: slab i / NRH, row group i % NRH
+            const int s = i / G::NRH, rg = i % G::NRH;
+            mbar_arrive_expect_tx(bar_full + slot, G::NRROWS * 128);
+            for (int q = 0; q < G::NRROWS / 64; ++q)
+              tma_load_2d(dst + q * 8192, &tm_w, 64 * s, wrow0 + M_ + rg * 128 + 64 * q,
+                          bar_full + slot);
+          } else {                     // feature rows of block f, d slab s
+            const int f = (i - G::NNORM) / G::DS, s = (i - G::NNORM) % G::DS;
+            mbar_arrive_expect_tx(bar_full + slot, 16384);
+            tma_load_2d(dst, &tm_w, 64 * s, wrow0 + 128 * f, bar_full + slot);
+            tma_load_2d(dst + 8192, &tm_w, 64 * s, wrow0 + 128 * f + 64, bar_full + slot);
+          }
+          last[slot] = g;
+        }
       }
       if (!ok) {
         // leave no copy in flight (a completed phase passes at once)
-        mbar_wait(bar_x, 0);
+        if (xlast >= 0) mbar_wait(bar_x, xlast & 1);
         for (int i = 0; i < G::NSLOT; ++i)
           if (last[i] >= 0) mbar_wait(bar_full + i, (last[i] / G::NSLOT) & 1);
       }
@@ -248,56 +275,72 @@ __global__ void __launch_bounds__(kThreadsF, 1)
   } else if (warp == 8) {
     // ---------------------------------------------------------- MMA issuer
     if (lane == 0) {
-      const uint32_t sXK = s0 + G::oXK, sXQ = s0 + G::oXQ;
-      auto feat_block = [&](int n) -> bool {   // K and Q GEMMs of feature block n
-        const int i = G::NNORM + n, slot = i % G::NSLOT;
-        if (!wait_one(bar_full + slot, (i / G::NSLOT) & 1, abort_flag, p.dev_status)) return false;
-        tc_fence_after();
-        const uint32_t sw = s0 + G::oW + slot * G::kSlot;
-        const uint32_t tp = tmem + 128 * (n & 1);
-        constexpr uint32_t id = idesc(128, 64, false, false, true);
-#pragma unroll
-        for (int s = 0; s < G::DS; ++s)
-#pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            const uint64_t bd = sdesc(sw + s * 8192 + k * 32, 16, 1024);
-            mma(tp, sdesc(sXK + s * 16384 + k * 32, 16, 1024), bd, id, (s | k) != 0);
-            mma(tp + 64, sdesc(sXQ + s * 16384 + k * 32, 16, 1024), bd, id, (s | k) != 0);
-          }
-        mma_commit(bar_empty + slot);
-        mma_commit(bar_pfull + (n & 1));
-        return true;
+      bool ok = true;
+      int g = 0, nblk = 0;   // ring items consumed, feature blocks issued (all items)
+      auto wait_item = [&](int gi) -> bool {
+        return wait_one(bar_full + gi % G::NSLOT, (gi / G::NSLOT) & 1, abort_flag, p.dev_status);
       };
-      bool ok = wait_one(bar_conv, 0, abort_flag, p.dev_status);
-      // ---- norm GEMM: columns [0, R_), one N = R_ MMA per K-step
-      for (int i = 0; ok && i < G::NNORM; ++i) {
-        const int slot = i % G::NSLOT;
-        if (!(ok = wait_one(bar_full + slot, (i / G::NSLOT) & 1, abort_flag, p.dev_status))) break;
-        tc_fence_after();
-        const uint32_t sw = s0 + G::oW + slot * G::kSlot;
-        constexpr uint32_t id = idesc(128, R_, false, false, true);
+      auto slot_addr = [&](int gi) -> uint32_t { return s0 + G::oW + (gi % G::NSLOT) * 16384; };
+      // scores += Psi_f Phi_f^T from the staging (both MN-major, features as K)
+      auto scores = [&](int f) {
+        constexpr uint32_t id = idesc(128, 128, true, true, false);
 #pragma unroll
-        for (int k = 0; k < 4; ++k)
-          mma(tmem, sdesc(sXK + i * 16384 + k * 32, 16, 1024), sdesc(sw + k * 32, 16, 1024), id,
-              (i | k) != 0);
-        mma_commit(bar_empty + slot);
-      }
-      if (ok) mma_commit(bar_norm);
-      // ---- feature blocks (P buffers overwrite the norm columns once read)
-      if (ok) ok = wait_one(bar_nread, 0, abort_flag, p.dev_status);
-      if (ok) ok = feat_block(0);
-      if (ok && G::NFEAT > 1) ok = feat_block(1);
-      for (int n = 0; ok && n < G::NFEAT; ++n) {
-        // block n staged by the epilogue: scores += Psi_n Phi_n^T
-        if (!(ok = wait_one(bar_stage, n & 1, abort_flag, p.dev_status))) break;
-        tc_fence_after();
-        constexpr uint32_t ids = idesc(128, 128, false, false, false);
-#pragma unroll
-        for (int k = 0; k < 4; ++k)
-          mma(tmem + G::tS, sdesc(s0 + G::oST + 16384 + k * 32, 16, 1024),
-              sdesc(s0 + G::oST + k * 32, 16, 1024), ids, (n | k) != 0);
+        for (int k = 0; k < 8; ++k)
+          mma(tmem + G::tN, sdesc(s0 + G::oST + 32768 + k * 2048, 16384, 1024),
+              sdesc(s0 + G::oST + k * 2048, 16384, 1024), id, (f | k) != 0);
         mma_commit(bar_sfree);
-        if (n + 2 < G::NFEAT) ok = feat_block(n + 2);
+      };
+      for (int j = 0; ok && j < nit; ++j) {
+        if (!(ok = wait_one(bar_conv, j & 1, abort_flag, p.dev_status))) break;
+        tc_fence_after();
+        // ---- key norms: (keys x d) (d x r), r in groups of up to 128 columns
+        for (int i = 0; ok && i < G::NNORM; ++i, ++g) {
+          const int s = i / G::NRH, rg = i % G::NRH;
+          if (!(ok = wait_item(g))) break;
+          tc_fence_after();
+          constexpr uint32_t id = idesc(128, G::NRROWS, false, false, true);
+          const uint32_t sw = slot_addr(g), sx = s0 + G::oX + s * G::kXSlab;
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            mma(tmem + G::tN + 128 * rg, sdesc(sx + k * 32, 16, 1024), sdesc(sw + k * 32, 16, 1024),
+                id, (s | k) != 0);
+          mma_commit(bar_empty + g % G::NSLOT);
+        }
+        if (!ok) break;
+        mma_commit(bar_norm);
+        // ---- feature blocks: F = W'_f [K_c ; Q_c]^T, one N = 256 MMA per K-step
+        for (int f = 0; ok && f < G::NB; ++f, ++nblk) {
+          if (nblk > 0 && !(ok = wait_one(bar_ffree, (nblk - 1) & 1, abort_flag, p.dev_status)))
+            break;
+          tc_fence_after();
+          constexpr uint32_t id = idesc(128, 256, false, false, true);
+          for (int s = 0; ok && s < G::DS; ++s, ++g) {
+            if (!(ok = wait_item(g))) break;
+            tc_fence_after();
+            const uint32_t sw = slot_addr(g), sx = s0 + G::oX + s * G::kXSlab;
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+              mma(tmem + G::tF, sdesc(sw + k * 32, 16, 1024), sdesc(sx + k * 32, 16, 1024), id,
+                  (s | k) != 0);
+            mma_commit(bar_empty + g % G::NSLOT);
+          }
+          if (!ok) break;
+          mma_commit(bar_ffull);
+          if (f == G::NB - 1) mma_commit(bar_xfree);
+          // scores of the previous block, staged meanwhile by the epilogue
+          if (f > 0) {
+            if (f == 1 && !(ok = wait_one(bar_nread, j & 1, abort_flag, p.dev_status))) break;
+            if (!(ok = wait_one(bar_stage, (nblk - 1) & 1, abort_flag, p.dev_status))) break;
+            tc_fence_after();
+            scores(f - 1);
+          }
+        }
+        if (!ok) break;
+        if (G::NB == 1 && !(ok = wait_one(bar_nread, j & 1, abort_flag, p.dev_status))) break;
+        if (!(ok = wait_one(bar_stage, (nblk - 1) & 1, abort_flag, p.dev_status))) break;
+        tc_fence_after();
+        scores(G::NB - 1);
+        mma_commit(bar_sc);
       }
       if (!ok) {
         // let every issued MMA finish before TMEM is released
@@ -309,97 +352,133 @@ __global__ void __launch_bounds__(kThreadsF, 1)
   } else {
     // ------------------------------------------------------------ epilogue
     const int etid = tid, quad = warp & 3, half = warp >> 2;
-    const int row = quad * 32 + lane;
+    const int row = quad * 32 + lane;                    // TMEM lane
     const uint32_t lane_tm = tmem + ((uint32_t)(quad * 32) << 16);
-    const int tok = t0 + row;
-    bool valid = tok < p.L;
-    if (valid && p.mask != nullptr) valid = p.mask[(size_t)b * p.L + tok] != 0;
-    bool ok = epi_wait(bar_x, 0, abort_flag, p.dev_status);
-    if (ok) {
-      // bf16 -> fp16 in place (both tiles; |x| >= 65504 is reported)
-      bool bad = false;
-      for (int i = etid; i < (int)(2 * G::kX / 16); i += kEpiThreads) {
-        const uint32_t a = s0 + G::oXK + i * 16;
-        uint4 u = ld_shared_v4(a);
-        uint32_t* w32 = &u.x;
+    bool ok = true;
+    int nblk = 0;
+    for (int j = 0; ok && j < nit; ++j) {
+      const int item = it0 + j, bh = item / p.nc, c = item % p.nc;
+      const int b = bh / p.H;
+      uint8_t* rec = p.img + (size_t)item * chunk_record_bytes(M_);
+      if (!(ok = epi_wait(bar_x, j & 1, abort_flag, p.dev_status))) break;
+      // bf16 -> fp16 in place (|x| >= 65504 is reported)
+      {
+        bool bad = false;
+        for (int i = etid; i < (int)(G::DS * G::kXSlab / 16); i += kEpiThreads) {
+          const uint32_t a = s0 + G::oX + i * 16;
+          uint4 u = ld_shared_v4(a);
+          uint32_t* w32 = &u.x;
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w32[e]));
-          bad |= fabsf(f.x) > 65504.f || fabsf(f.y) > 65504.f;
-          const __half2 hv = __floats2half2_rn(f.x, f.y);
-          w32[e] = *reinterpret_cast<const uint32_t*>(&hv);
+          for (int e = 0; e < 4; ++e) {
+            const float2 f2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w32[e]));
+            bad |= fabsf(f2.x) > 65504.f || fabsf(f2.y) > 65504.f;
+            const __half2 hv = __floats2half2_rn(f2.x, f2.y);
+            w32[e] = *reinterpret_cast<const uint32_t*>(&hv);
+          }
+          st_shared_v4(a, u.x, u.y, u.z, u.w);
         }
-        st_shared_v4(a, u.x, u.y, u.z, u.w);
+        if (bad) report(p.dev_status, DARK_ERR_NUMERIC);
       }
-      if (bad) report(p.dev_status, DARK_ERR_NUMERIC);
       fence_async_smem();
+      tc_fence_before();
       warp_arrive(bar_conv);
-      ok = epi_wait(bar_norm, 0, abort_flag, p.dev_status);
-    }
-    float nrm = 0.f;
-    if (ok) {
+      // ---- key offsets: sum of squares of the norm columns + 1/2 log2 m;
+      // +inf for a masked or missing key
+      if (!(ok = epi_wait(bar_norm, j & 1, abort_flag, p.dev_status))) break;
       tc_fence_after();
-      float part = 0.f;
+      {
+        float part = 0.f;
 #pragma unroll 1
-      for (int c0 = half * (R_ / 2); c0 < (half + 1) * (R_ / 2); c0 += 32) {
-        float v[32];
-        tmem_ld32(lane_tm + c0, v);
+        for (int c0 = half * (R_ / 2); c0 < (half + 1) * (R_ / 2); c0 += 32) {
+          float v[32];
+          tmem_ld32(lane_tm + G::tN + c0, v);
 #pragma unroll
-        for (int i = 0; i < 32; ++i) part = fmaf(v[i], v[i], part);
-      }
-      nrm_x[half * 128 + row] = part;
-      tc_fence_before();
-      epi_sync();
-      nrm = nrm_x[row] + nrm_x[128 + row] + 0.5f * __log2f((float)M_);
-      warp_arrive(bar_nread);
-    }
-    uint8_t* g_phi = rec;
-    uint8_t* g_psi = rec + (size_t)M_ * 256;
-    const uint32_t st_phi = s0 + G::oST, st_psi = s0 + G::oST + 16384;
-    for (int n = 0; ok && n < G::NFEAT; ++n) {
-      if (!(ok = epi_wait(bar_pfull + (n & 1), (n >> 1) & 1, abort_flag, p.dev_status))) break;
-      if (n > 0) {
-        // staging is free once the scores GEMM and the bulk stores of block n-1 read it
-        if (!(ok = epi_wait(bar_sfree, (n - 1) & 1, abort_flag, p.dev_status))) break;
-        if (etid == 0) bulk_wait_read_all();
+          for (int i = 0; i < 32; ++i) part = fmaf(v[i], v[i], part);
+        }
+        if (half == 1) nrm_x[row] = part;
         epi_sync();
+        if (half == 0) {
+          const int tok = c * kC + row;
+          bool valid = tok < p.L;
+          if (valid && p.mask != nullptr) valid = p.mask[(size_t)b * p.L + tok] != 0;
+          nrm_s[row] = valid ? part + nrm_x[row] + 0.5f * __log2f((float)M_) : __int_as_float(0x7f800000);
+        }
+        tc_fence_before();
+        epi_sync();
+        warp_arrive(bar_nread);
       }
-      tc_fence_after();
-      const uint32_t tp = lane_tm + 128 * (n & 1);
-      if (half == 0)
-        exp2_rows_to_smem(tp, 0, 64, nrm, !valid, st_phi, row);
-      else
-        exp2_rows_to_smem(tp + 64, 0, 64, 0.f, false, st_psi, row);
-      tc_fence_before();
-      fence_async_smem();
-      epi_sync();
-      if (etid == 0) {
-        bulk_store(g_phi + (size_t)n * 16384, st_phi, 16384);
-        bulk_store(g_psi + (size_t)n * 16384, st_psi, 16384);
-        bulk_commit();
+      // ---- feature blocks: Phi_f (keys, half 0) and Psi_f (queries, half 1)
+      for (int f = 0; ok && f < G::NB; ++f, ++nblk) {
+        if (!(ok = epi_wait(bar_ffull, nblk & 1, abort_flag, p.dev_status))) break;
+        tc_fence_after();
+        uint32_t v[4][32];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) tmem_ld32_async(lane_tm + G::tF + 128 * half + 32 * q, v[q]);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) tmem_wait_ld(v[q]);
+        tc_fence_before();
+        warp_arrive(bar_ffree);
+        // exp2 and bf16 packing (keys: minus the key offset)
+        uint32_t pk[64];
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const int t = 32 * q + 2 * e;
+            float x0 = __uint_as_float(v[q][2 * e]), x1 = __uint_as_float(v[q][2 * e + 1]);
+            if (half == 0) {
+              x0 -= nrm_s[t];
+              x1 -= nrm_s[t + 1];
+            }
+            pk[16 * q + e] = pack_bf16(ex2(x0), ex2(x1));
+          }
+        // the staging is free once the previous block's scores GEMM and bulk
+        // stores (or the previous item's A image store) have read it
+        if (nblk > 0) {
+          if (f > 0 && !(ok = epi_wait(bar_sfree, (nblk - 1) & 1, abort_flag, p.dev_status))) break;
+          if (etid == 0) bulk_wait_read_all();
+          epi_sync();
+        }
+        const uint32_t st = s0 + G::oST + 32768 * half;
+#pragma unroll
+        for (int cc = 0; cc < 16; ++cc) {
+          const uint32_t off = (uint32_t)(cc >> 3) * 16384 + (uint32_t)(row >> 3) * 1024 +
+                               (uint32_t)(row & 7) * 128 + (uint32_t)(((cc & 7) ^ (row & 7)) * 16);
+          st_shared_v4(st + off, pk[4 * cc], pk[4 * cc + 1], pk[4 * cc + 2], pk[4 * cc + 3]);
+        }
+        fence_async_smem();
+        epi_sync();
+        if (etid == 0) {
+          bulk_store(rec + (size_t)f * 32768, s0 + G::oST, 32768);
+          bulk_store(rec + (size_t)M_ * 256 + (size_t)f * 32768, s0 + G::oST + 32768, 32768);
+          bulk_commit();
+        }
+        warp_arrive(bar_stage);
       }
-      warp_arrive(bar_stage);
-    }
-    // ------------------------------ masked causal scores -> A image
-    if (ok) ok = epi_wait(bar_sfree, (G::NFEAT - 1) & 1, abort_flag, p.dev_status);
-    if (ok) {
+      if (!ok) break;
+      // ---- masked causal scores -> A image (query rows, keys as K)
+      if (!(ok = epi_wait(bar_sc, j & 1, abort_flag, p.dev_status))) break;
       if (etid == 0) bulk_wait_read_all();
       epi_sync();
       tc_fence_after();
-      float v[32];
+      {
+        uint32_t a[2][32];
+        tmem_ld32_async(lane_tm + G::tN + 64 * half, a[0]);
+        tmem_ld32_async(lane_tm + G::tN + 64 * half + 32, a[1]);
+        tmem_wait_ld(a[0]);
+        tmem_wait_ld(a[1]);
 #pragma unroll
-      for (int j0 = half * 64; j0 < half * 64 + 64; j0 += 32) {
-        tmem_ld32(lane_tm + G::tS + j0, v);
-#pragma unroll
-        for (int g = 0; g < 4; ++g) {
+        for (int cc = 0; cc < 8; ++cc) {
           uint32_t w4[4];
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            const int j = j0 + 8 * g + 2 * e;
-            w4[e] = pack_bf16(j <= row ? v[8 * g + 2 * e] : 0.f,
-                              j + 1 <= row ? v[8 * g + 2 * e + 1] : 0.f);
+            const int jj = 64 * half + 8 * cc + 2 * e;
+            const uint32_t* src = a[cc >> 2] + 8 * (cc & 3) + 2 * e;
+            w4[e] = pack_bf16(jj <= row ? __uint_as_float(src[0]) : 0.f,
+                              jj + 1 <= row ? __uint_as_float(src[1]) : 0.f);
           }
-          st_shared_v4(s0 + G::oST + kmajor_off(row, j0 + 8 * g, 16384), w4[0], w4[1], w4[2], w4[3]);
+          st_shared_v4(s0 + G::oST + kmajor_off(row, 64 * half + 8 * cc, 16384), w4[0], w4[1],
+                       w4[2], w4[3]);
         }
       }
       tc_fence_before();
@@ -589,11 +668,11 @@ __global__ void __launch_bounds__(kThreadsV, 1)
           // the chunk starts the numerator
           {
             const uint32_t sPsi = slot_addr(gP);
-            constexpr uint32_t id = idesc(128, 144, false, true, false);
+            constexpr uint32_t id = idesc(128, 144, true, true, false);
 #pragma unroll
             for (int s = 0; s < 8; ++s)
-              mma(tnum, sdesc(sPsi + (s / 4) * 16384 + (s % 4) * 32, 16, 1024),
-                  sdesc(sS + s * 2048, 16384, 1024), id, (f > 0) || (s > 0));
+              mma(tnum, sdesc(sPsi + s * 2048, 16384, 1024), sdesc(sS + s * 2048, 16384, 1024), id,
+                  (f > 0) || (s > 0));
             mma_commit(bar_sfree);
           }
           if (f == 0) {
@@ -618,11 +697,11 @@ __global__ void __launch_bounds__(kThreadsV, 1)
           {
             const uint32_t sPhi = slot_addr(gF);
             const uint32_t ts = tmem + 80 * f;
-            constexpr uint32_t id = idesc(128, 80, true, true, false);
+            constexpr uint32_t id = idesc(128, 80, false, true, false);
 #pragma unroll
             for (int s = 0; s < kC / 16; ++s)
-              mma(ts, sdesc(sPhi + s * 2048, 16384, 1024), sdesc(sV + s * 2048, lbo_v1, 1024), id,
-                  (c > 0) || (s > 0));
+              mma(ts, sdesc(sPhi + (s / 4) * 16384 + (s % 4) * 32, 16, 1024),
+                  sdesc(sV + s * 2048, lbo_v1, 1024), id, (c > 0) || (s > 0));
             mma_commit(bar_ds + f);
             mma_commit(bar_empty + gF % G::NSLOT);
           }
@@ -799,8 +878,9 @@ cudaError_t launch(const FwdArgs& a) {
   if (e != cudaSuccess) return e;
   e = set_smem_limit_once((const void*)values_kernel<M_>, (int)V::kSmem, smem_v);
   if (e != cudaSuccess) return e;
-  features_kernel<D_, M_, R_><<<a.B * a.H * nc, kThreadsF, F::kSmem, a.stream>>>(a.tm_w, a.tm_q,
-                                                                                 a.tm_k, fp);
+  fp.nitems = a.B * a.H * nc;
+  const int grid_f = fp.nitems < num_sms() ? fp.nitems : num_sms();
+  features_kernel<D_, M_, R_><<<grid_f, kThreadsF, F::kSmem, a.stream>>>(a.tm_w, a.tm_q, a.tm_k, fp);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   ValParams vp;

@@ -98,3 +98,49 @@ def test_full_size_forward(D, cuda_ok, cfg):
                                             inp["omega"], inp["geom"][h:h + 1])
                 kvs[(b, h)] = (kv2[0, 0], z2[0, 0])
                 assert np.abs(o[b, h] - ro[0, 0]).max() <= TOL_BF16
+
+
+def test_full_size_decode_1024_steps(D, cuda_ok):
+    # Workload 5 as specified: a 4096-token causal prefill of the whole batch
+    # (B64 H8 d64 m256) followed by 1024 single-token decode steps of the whole
+    # batch through the C ABI. Every step's output on sampled heads is compared
+    # with the oracle's decode recurrence continued from its own prefill state
+    # (README, "Encoder-decoder model and generation": update, then emit), and
+    # the final fp32 state (kv, z) with the oracle's, relative to its largest
+    # entry, so that drift of the carried state over 1024 updates is checked.
+    w = synth.WORKLOADS[5]
+    steps = 1024
+    inp = synth.make_inputs(w)
+    res = forward(D, w, inp, cuda_ok, with_state=True)
+    assert res["status"] == 0
+    stream = synth.decode_stream(w, steps)
+    sq, sk, sv = (to_dev(stream[nm], torch.bfloat16, cuda_ok) for nm in ("q", "k", "v"))
+    outs = torch.empty_like(sq)
+    status = torch.zeros(1, dtype=torch.int32, device=cuda_ok)
+    for t in range(steps):
+        D.dark_decode_step(res["proj"], res["state"], sq[t], sk[t], sv[t], outs[t],
+                           dev_status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    got = outs.double().cpu().numpy()                        # [steps, B, H, d]
+    assert np.all(np.isfinite(got))
+    kv_end = res["state_tensors"][0].double().cpu().numpy()
+    z_end = res["state_tensors"][1].double().cpu().numpy()
+    rng = np.random.default_rng(55)
+    bh = [(b, h) for b in range(w.B) for h in range(w.H)]
+    heads = [bh[i] for i in sorted(set([0, len(bh) - 1] + rng.integers(0, len(bh), 2).tolist()))]
+    for (b, h) in heads:
+        gm = inp["geom"][h:h + 1]
+        phk = O.feature_map(inp["k"][b, h], inp["omega"][0], inp["geom"][h])
+        kv = (phk.T @ inp["v"][b, h].astype(np.float64))[None, None]
+        z = phk.sum(axis=0)[None, None]
+        worst = 0.0
+        for t in range(steps):
+            sl = (slice(b, b + 1), slice(h, h + 1))
+            ro, kv, z = O.decode_step(kv, z, stream["q"][t][sl], stream["k"][t][sl],
+                                      stream["v"][t][sl], inp["omega"], gm)
+            worst = max(worst, float(np.abs(got[t, b, h] - ro[0, 0]).max()))
+        assert worst <= TOL_BF16, (b, h, worst)
+        # the same bar as the prefill state above (bf16 feature operands)
+        assert np.abs(kv_end[b, h] - kv[0, 0]).max() <= TOL_BF16 * np.abs(kv).max(), (b, h)
+        assert np.abs(z_end[b, h] - z[0, 0]).max() <= TOL_BF16 * np.abs(z).max(), (b, h)
