@@ -43,7 +43,7 @@
 extern "C" {
 #endif
 
-#define DARK_ABI_VERSION 5
+#define DARK_ABI_VERSION 6
 
 typedef enum {
   DARK_OK = 0,
@@ -108,6 +108,18 @@ int dark_abi_version(void);
 
 /* Human-readable name of a status code. Never NULL; static storage. */
 const char* dark_status_string(dark_status s);
+
+/*
+ * Testing hook for the device time-out path; the method's pages have no
+ * counterpart of it. With cycles > 0, every tensor-core forward kernel launched
+ * afterwards first waits on a barrier that nothing completes, for at most
+ * `cycles` SM clock cycles, and then takes the path of a wait that ran out: it
+ * records DARK_ERR_TIMEOUT in *dev_status, waits (bounded) for its own copies
+ * and MMAs still in flight, frees its TMEM and returns without writing its
+ * outputs. 0 (the default) turns the hook off. Process-wide: set it only while
+ * no other host thread calls the library.
+ */
+void dark_set_test_stall_cycles(long long cycles);
 
 /* Bytes of the projection buffer for the given sizes, 0 if a size is not positive. */
 size_t dark_projection_bytes(int heads, int m, int r, int d, dark_dtype dtype);

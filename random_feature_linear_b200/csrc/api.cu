@@ -152,9 +152,20 @@ dark_status fwd_launch(FwdArgs& a, void* ws, size_t ws_bytes, dark_state* state_
 
 }  // namespace dark
 
+namespace dark {
+namespace {
+std::atomic<long long> g_test_stall{0};
+}
+long long test_stall_cycles() { return g_test_stall.load(std::memory_order_relaxed); }
+}  // namespace dark
+
 extern "C" {
 
 int dark_abi_version(void) { return DARK_ABI_VERSION; }
+
+void dark_set_test_stall_cycles(long long cycles) {
+  dark::g_test_stall.store(cycles > 0 ? cycles : 0, std::memory_order_relaxed);
+}
 
 const char* dark_status_string(dark_status s) {
   switch (s) {

@@ -75,6 +75,9 @@ cudaError_t simt_forward(const FwdArgs& a);
 // Alignment/stride/shape checks shared by the tensor-core paths, then the
 // TMA descriptors (false if any check fails or the driver rejects a layout).
 bool tc_make_maps(FwdArgs& a);
+// Cycles of the testing stall every tensor-core forward kernel takes first
+// (0: none); set through dark_set_test_stall_cycles.
+long long test_stall_cycles();
 // Streaming multiprocessors of the current device (looked up once per device).
 int num_sms();
 // Sets a kernel's dynamic shared memory limit once per device.

@@ -87,6 +87,7 @@ struct Params {
   const float* seg_sums;        // [B*H*nseg][65][m] per-segment key states (nseg > 1)
   float *st_kv, *st_z;          // state after the last chunk
   int* dev_status;
+  long long stall;              // testing stall before the first wait (0: none)
 };
 
 template <int M_, int R_>
@@ -101,6 +102,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* bar_tma = (uint64_t*)(sm + G::oBar);
   uint64_t* bar_mma = bar_tma + 1;
   uint32_t* tmem_slot = (uint32_t*)(bar_tma + 2);
+  uint64_t* bar_drain = bar_tma + 3;    // abort path: the issued MMAs completed
+  uint64_t* bar_never = bar_tma + 4;    // completed by nothing (testing stall)
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int quad = warp & 3, half = warp >> 2;
@@ -111,6 +114,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (tid == 0) {
     mbar_init(bar_tma, 1);
     mbar_init(bar_mma, 1);
+    mbar_init(bar_drain, 1);
+    mbar_init(bar_never, 1);
     fence_mbar_init();
     prefetch_tmap(&tm_w);
     prefetch_tmap(&tm_q);
@@ -141,9 +146,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
   for (int i = 0; i < 65; ++i) run[i] = 0.f;
   bool abort = false;
+  int tma_issued = 0, tma_waited = 0;          // load phases started / waited for
 
   // W', K, V and Q tiles of the chunk starting at token t (one thread)
   auto issue_loads = [&](int t) {
+    ++tma_issued;
     mbar_arrive_expect_tx(bar_tma, G::kW + 3 * kTileBytes);
     for (int r0 = 0; r0 < G::NW; r0 += 16)
       tma_load_2d(sm + G::oW + r0 * 128, &tm_w, 0, hw * G::NW + r0, bar_tma);
@@ -156,8 +163,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ---------------------------------------------------------------- loads
     // (for later chunks they were issued during the previous chunk's output)
     if (tid == 0 && c == c_begin) issue_loads(t0);
+    if (c == c_begin && p.stall > 0 && !wait_all(bar_never, 0, p.dev_status, p.stall)) {
+      abort = true;
+      break;
+    }
     if (!wait_all(bar_tma, ph_tma, p.dev_status)) { abort = true; break; }
     ph_tma ^= 1;
+    ++tma_waited;
     // k, then q: bf16 -> fp16 in place (the feature GEMMs run on fp16 operands);
     // the key GEMM starts while the query tile converts
     to_fp16_inplace(s0 + G::oK, kTileBytes, p.dev_status);
@@ -405,6 +417,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int i = 0; i < 64; ++i) kv[i] = run[i];
     p.st_z[(size_t)bh * M_ + feat] = run[64];
   }
+  if (abort && tid == 0) {
+    // no copy or MMA of this CTA may still be running when TMEM is freed
+    drain_loads(bar_tma, tma_issued, tma_waited);
+    drain_mmas(bar_drain);
+  }
   tc_fence_before();
   __syncthreads();
   if (warp == 0) {
@@ -460,6 +477,7 @@ cudaError_t launch(const FwdArgs& a, const CUtensorMap& tw, const CUtensorMap& t
   p.st_kv = a.st_kv;
   p.st_z = a.st_z;
   p.dev_status = a.dev_status;
+  p.stall = test_stall_cycles();
   static int smem_set[64];
   e = set_smem_limit_once((const void*)causal_kernel<M_, R_>, (int)G::kSmem, smem_set);
   if (e != cudaSuccess) return e;

@@ -54,14 +54,31 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
-// Waits for the phase with the given parity; false if it did not complete in time.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+// Waits for the phase with the given parity; false if it did not complete
+// within `limit` cycles.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
+                                          long long limit = kWaitCycles) {
   if (mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
   while (!mbar_try_wait(bar, parity)) {
-    if (clock64() - t0 > kWaitCycles) return false;
+    if (clock64() - t0 > limit) return false;
   }
   return true;
+}
+// Abort path of a CTA after a wait ran out: a bounded wait for the last of
+// `issued` load phases started on `bar` when only `waited` of them were waited
+// for (a completed phase passes at once), so that no copy is still writing
+// into shared memory when the CTA exits.
+__device__ __forceinline__ void drain_loads(uint64_t* bar, int issued, int waited) {
+  if (issued > waited) mbar_wait(bar, (uint32_t)(issued - 1) & 1u);
+}
+// Abort path, on the thread that issued the MMAs: a bounded wait until every
+// MMA it issued has completed (before TMEM is released).
+__device__ __forceinline__ void drain_mmas(uint64_t* bar_drain) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                   smem_u32(bar_drain))
+               : "memory");
+  mbar_wait(bar_drain, 0);
 }
 
 // --------------------------------------------------------------------- TMA --

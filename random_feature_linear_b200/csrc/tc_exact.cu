@@ -57,6 +57,7 @@ struct Params {
   const uint8_t* qmask;                    // [B][Lq] or null
   int B, H, Lq, Lk, nq, causal, heads_w, m, r;
   int* dev_status;
+  long long stall;                         // testing stall before the first wait (0: none)
 };
 
 // Projection epilogue: this thread's row of the N = r projection in TMEM, times
@@ -96,6 +97,8 @@ __global__ void __launch_bounds__(kThreads, 2)
   uint64_t* bar_v = bar_k + 1;                  // each V tile
   uint64_t* bar_mma = bar_k + 2;
   uint32_t* tmem_slot = (uint32_t*)(bar_k + 3);
+  uint64_t* bar_drain = bar_k + 4;              // abort path: the issued MMAs completed
+  uint64_t* bar_never = bar_k + 5;              // completed by nothing (testing stall)
   float* smax = (float*)(sm + oMax);
   uint8_t* kval = sm + oKv;
 
@@ -107,6 +110,8 @@ __global__ void __launch_bounds__(kThreads, 2)
     mbar_init(bar_k, 1);
     mbar_init(bar_v, 1);
     mbar_init(bar_mma, 1);
+    mbar_init(bar_drain, 1);
+    mbar_init(bar_never, 1);
     fence_mbar_init();
     prefetch_tmap(&tm_w);
     prefetch_tmap(&tm_q);
@@ -136,6 +141,7 @@ __global__ void __launch_bounds__(kThreads, 2)
 
   uint32_t ph_k = 0, ph_v = 0, ph_mma = 0;
   bool abort = false;
+  int k_issued = 1, k_waited = 0, v_issued = 0, v_waited = 0;   // load phases started / waited
   float o[32], l = 0.f, mrow = -INFINITY;
 #pragma unroll
   for (int i = 0; i < 32; ++i) o[i] = 0.f;
@@ -147,9 +153,13 @@ __global__ void __launch_bounds__(kThreads, 2)
       tma_load_2d(sm + oW + r0 * 128, &tm_w, 0, hw * (p.m + r) + p.m + r0, bar_k);
     tma_load_4d(sm + oQ, &tm_q, 0, q0, h, b, bar_k);
   }
-  if (!wait_all(bar_k, ph_k, p.dev_status)) abort = true;
+  if (p.stall > 0 && !wait_all(bar_never, 0, p.dev_status, p.stall)) abort = true;
+  if (!abort && !wait_all(bar_k, ph_k, p.dev_status)) abort = true;
   ph_k ^= 1;
   if (!abort) {
+    ++k_waited;
+    ++k_issued;
+    ++v_issued;
     if (tid == 0) {
       mbar_arrive_expect_tx(bar_k, kTile);
       tma_load_4d(sm + oK, &tm_k, 0, 0, h, b, bar_k);
@@ -183,6 +193,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     // ---- K_j: projection p_k
     if (!wait_all(bar_k, ph_k, p.dev_status)) { abort = true; break; }
     ph_k ^= 1;
+    ++k_waited;
     to_fp16_inplace(s0 + oK, kTile, p.dev_status);
     fence_async_smem();
     __syncthreads();
@@ -222,6 +233,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     ph_mma ^= 1;
     tc_fence_after();
     // the scores MMA has read p_k: the next key tile may load over it
+    if (j + 1 < nk) ++k_issued;
     if (tid == 0 && j + 1 < nk) {
       mbar_arrive_expect_tx(bar_k, kTile);
       tma_load_4d(sm + oK, &tm_k, 0, k0 + kT, h, b, bar_k);
@@ -269,6 +281,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     // ---- [num | den] = P [V | 1]
     if (!wait_all(bar_v, ph_v, p.dev_status)) { abort = true; break; }
     ph_v ^= 1;
+    ++v_waited;
     if (tid == 0) {
       tc_fence_after();
       constexpr uint32_t idv = idesc(128, 80, false, true, false);
@@ -282,6 +295,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     ph_mma ^= 1;
     tc_fence_after();
     // the value MMA has read V: the next value tile may load
+    if (j + 1 < nk) ++v_issued;
     if (tid == 0 && j + 1 < nk) {
       mbar_arrive_expect_tx(bar_v, kTile);
       tma_load_4d(sm + oV, &tm_v, 0, k0 + kT, h, b, bar_v);
@@ -296,6 +310,12 @@ __global__ void __launch_bounds__(kThreads, 2)
     }
     tc_fence_before();
     __syncthreads();
+  }
+  if (abort && tid == 0) {
+    // no copy or MMA of this CTA may still be running when TMEM is freed
+    drain_loads(bar_k, k_issued, k_waited);
+    drain_loads(bar_v, v_issued, v_waited);
+    drain_mmas(bar_drain);
   }
   if (!abort && qi < p.Lq) {
     const bool live = p.qmask == nullptr || p.qmask[(size_t)b * p.Lq + qi] != 0;
@@ -351,6 +371,7 @@ cudaError_t tc_exact_forward(const FwdArgs& a) {
   p.m = a.m;
   p.r = a.r;
   p.dev_status = a.dev_status;
+  p.stall = test_stall_cycles();
   static int smem_set[64];
   cudaError_t e = set_smem_limit_once((const void*)exact_tc_kernel, (int)kSmem, smem_set);
   if (e != cudaSuccess) return e;

@@ -28,6 +28,7 @@ struct KeyParams {
   int B, H, L, ntiles, nsplit, heads_w;
   float* partials;                 // [B*H*nsplit][65][m]
   int* dev_status;
+  long long stall;                 // testing stall before the first wait (0: none)
 };
 
 template <int M_, int R_>
@@ -59,6 +60,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* bar_kv = (uint64_t*)(sm + G::oBar);     // [2]
   uint64_t* bar_mma = bar_kv + 2;
   uint32_t* tmem_slot = (uint32_t*)(bar_kv + 3);
+  uint64_t* bar_drain = bar_kv + 4;     // abort path: the issued MMAs completed
+  uint64_t* bar_never = bar_kv + 5;     // completed by nothing (testing stall)
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int quad = warp & 3, half = warp >> 2;
@@ -72,6 +75,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(&bar_kv[0], 1);
     mbar_init(&bar_kv[1], 1);
     mbar_init(bar_mma, 1);
+    mbar_init(bar_drain, 1);
+    mbar_init(bar_never, 1);
     fence_mbar_init();
     if (te > tb) {
       mbar_arrive_expect_tx(&bar_kv[0], G::kW + 2 * kTileBytes);
@@ -96,10 +101,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   uint32_t ph_kv = 0, ph_mma = 0;             // bit i: phase parity of buffer i
   bool abort = false;
-  for (int t = tb; t < te; ++t) {
+  int issued[2] = {te > tb ? 1 : 0, 0}, waited[2] = {0, 0};   // load phases per buffer
+  if (te > tb && p.stall > 0 && !wait_all(bar_never, 0, p.dev_status, p.stall)) abort = true;
+  for (int t = tb; t < te && !abort; ++t) {
     const int i = t - tb, buf = i & 1;
     if (!wait_all(&bar_kv[buf], (ph_kv >> buf) & 1u, p.dev_status)) { abort = true; break; }
     ph_kv ^= 1u << buf;
+    ++waited[buf];
     to_fp16_inplace(s0 + G::oK + buf * kTileBytes, kTileBytes, p.dev_status);
     fence_async_smem();
     __syncthreads();
@@ -123,6 +131,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // the other buffer is free now: prefetch the next tile into it
     if (tid == 0 && t + 1 < te) {
       const int nb = buf ^ 1;
+      ++issued[nb];
       mbar_arrive_expect_tx(&bar_kv[nb], 2 * kTileBytes);
       tma_load_4d(sm + G::oK + nb * kTileBytes, &tm_k, 0, (t + 1) * kT, h, b, &bar_kv[nb]);
       tma_load_4d(sm + G::oV + nb * kTileBytes, &tm_v, 0, (t + 1) * kT, h, b, &bar_kv[nb]);
@@ -168,6 +177,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (!wait_all(bar_mma, ph_mma, p.dev_status)) abort = true;
     tc_fence_after();
   }
+  if (abort && tid == 0) {
+    // no copy or MMA of this CTA may still be running when TMEM is freed
+    drain_loads(&bar_kv[0], issued[0], waited[0]);
+    drain_loads(&bar_kv[1], issued[1], waited[1]);
+    drain_mmas(bar_drain);
+  }
   if (!abort && half < G::MB) {
     const int f = half * 128 + row;
     float* dst = p.partials + ((size_t)bh * p.nsplit + split) * 65 * M_;
@@ -207,6 +222,7 @@ cudaError_t launch_keys_t(const FwdArgs& a, const CUtensorMap& tw, const CUtenso
   kp.heads_w = a.heads_w;
   kp.partials = partials;
   kp.dev_status = a.dev_status;
+  kp.stall = test_stall_cycles();
   using KG = KeyCfg<M_, R_>;
   static int smem_set[64];
   cudaError_t e = set_smem_limit_once((const void*)keys_kernel<M_, R_>, (int)KG::kSmem, smem_set);

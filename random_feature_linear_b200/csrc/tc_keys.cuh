@@ -10,8 +10,11 @@ namespace tc {
 
 constexpr int kFwdThreads = 256;
 
-__device__ __forceinline__ bool wait_all(uint64_t* bar, uint32_t parity, int* dev_status) {
-  const bool ok = mbar_wait(bar, parity);
+// Every thread of the CTA waits (bounded by `limit` cycles); false on all of
+// them if any wait ran out (DARK_ERR_TIMEOUT is then recorded).
+__device__ __forceinline__ bool wait_all(uint64_t* bar, uint32_t parity, int* dev_status,
+                                         long long limit = kWaitCycles) {
+  const bool ok = mbar_wait(bar, parity, limit);
   const int bad = __syncthreads_or(ok ? 0 : 1);
   if (bad && threadIdx.x == 0) report(dev_status, DARK_ERR_TIMEOUT);
   return bad == 0;

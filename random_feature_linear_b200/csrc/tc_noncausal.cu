@@ -79,6 +79,7 @@ struct QueryParams {
   const uint8_t* qmask;         // [B][L] or null: a masked query row outputs 0
   const uint8_t* images;
   int* dev_status;
+  long long stall;              // testing stall before the first wait (0: none)
 };
 
 template <int M_, int R_>
@@ -108,6 +109,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* bar_mma = bar_q + 2;
   uint64_t* bar_head = bar_q + 3;
   uint32_t* tmem_slot = (uint32_t*)(bar_q + 4);
+  uint64_t* bar_drain = bar_q + 5;      // abort path: the issued MMAs completed
+  uint64_t* bar_never = bar_q + 6;      // completed by nothing (testing stall)
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int quad = warp & 3, half = warp >> 2;
@@ -120,6 +123,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(&bar_q[1], 1);
     mbar_init(bar_mma, 1);
     mbar_init(bar_head, 1);
+    mbar_init(bar_drain, 1);
+    mbar_init(bar_never, 1);
     fence_mbar_init();
     if (ue > ub) {
       const int bh = ub / p.ntiles, t = ub % p.ntiles;
@@ -138,13 +143,17 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint32_t ph_q = 0, ph_mma = 0, ph_head = 0;  // ph_q bit i: parity of buffer i
   int cur_bh = -1;
   bool abort = false;
-  for (int u = ub; u < ue; ++u) {
+  // load phases started / waited for: query buffers, head operands
+  int q_issued[2] = {ue > ub ? 1 : 0, 0}, q_waited[2] = {0, 0}, h_issued = 0, h_waited = 0;
+  if (ue > ub && p.stall > 0 && !wait_all(bar_never, 0, p.dev_status, p.stall)) abort = true;
+  for (int u = ub; u < ue && !abort; ++u) {
     const int i = u - ub, buf = i & 1;
     const int bh = u / p.ntiles, t = u % p.ntiles, b = bh / p.H, h = bh % p.H;
     if (bh != cur_bh) {
       // W' rows and the [S | z] image of this head (all earlier MMAs have completed)
       if (tid == 0) {
         const int hw = p.heads_w == 1 ? 0 : h;
+        ++h_issued;
         mbar_arrive_expect_tx(bar_head, G::kWq + img_bytes(M_));
         for (int r0 = 0; r0 < M_; r0 += 16)
           tma_load_2d(sm + G::oW + r0 * 128, &tm_w, 0, hw * G::NW + r0, bar_head);
@@ -155,10 +164,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (!wait_all(bar_head, ph_head, p.dev_status)) { abort = true; break; }
       ph_head ^= 1;
+      ++h_waited;
       cur_bh = bh;
     }
     if (!wait_all(&bar_q[buf], (ph_q >> buf) & 1u, p.dev_status)) { abort = true; break; }
     ph_q ^= 1u << buf;
+    ++q_waited[buf];
     to_fp16_inplace(s0 + G::oQ + buf * kTileBytes, kTileBytes, p.dev_status);
     fence_async_smem();
     __syncthreads();
@@ -177,6 +188,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // prefetch the next query tile into the other buffer (its GEMM completed)
     if (tid == 0 && u + 1 < ue) {
       const int nbh = (u + 1) / p.ntiles, nt = (u + 1) % p.ntiles;
+      ++q_issued[buf ^ 1];
       mbar_arrive_expect_tx(&bar_q[buf ^ 1], kTileBytes);
       tma_load_4d(sm + G::oQ + (buf ^ 1) * kTileBytes, &tm_q, 0, nt * kT, nbh % p.H, nbh / p.H,
                   &bar_q[buf ^ 1]);
@@ -229,7 +241,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_before();
     __syncthreads();
   }
-  (void)abort;
+  if (abort && tid == 0) {
+    // no copy or MMA of this CTA may still be running when TMEM is freed
+    drain_loads(bar_head, h_issued, h_waited);
+    drain_loads(&bar_q[0], q_issued[0], q_waited[0]);
+    drain_loads(&bar_q[1], q_issued[1], q_waited[1]);
+    drain_mmas(bar_drain);
+  }
   tc_fence_before();
   __syncthreads();
   if (warp == 0) {
@@ -289,6 +307,7 @@ cudaError_t launch(const FwdArgs& a, const CUtensorMap& tw, const CUtensorMap& t
   qp.qmask = a.qmask;
   qp.images = images;
   qp.dev_status = a.dev_status;
+  qp.stall = test_stall_cycles();
   using QG = QueryCfg<M_, R_>;
   static int smem_set[64];
   e = set_smem_limit_once((const void*)queries_kernel<M_, R_>, (int)QG::kSmem, smem_set);

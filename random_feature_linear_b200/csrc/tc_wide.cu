@@ -88,12 +88,12 @@ __device__ __forceinline__ void epi_sync() { asm volatile("barrier.cta.sync 1, 2
 // Bounded wait of one thread. A wait that runs out records DARK_ERR_TIMEOUT and
 // raises the abort flag; a raised flag ends every other wait of the CTA.
 __device__ __forceinline__ bool wait_one(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
-                                         int* dev_status) {
+                                         int* dev_status, long long limit = kWaitCycles) {
   if (mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
   while (!mbar_try_wait(bar, parity)) {
     if (*abort_flag) return false;
-    if (clock64() - t0 > kWaitCycles) {
+    if (clock64() - t0 > limit) {
       *abort_flag = 1;
       report(dev_status, DARK_ERR_TIMEOUT);
       return false;
@@ -103,8 +103,8 @@ __device__ __forceinline__ bool wait_one(uint64_t* bar, uint32_t parity, volatil
 }
 // The same for the epilogue warps: all 256 wait, then agree.
 __device__ __forceinline__ bool epi_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
-                                         int* dev_status) {
-  const bool ok = wait_one(bar, parity, abort_flag, dev_status);
+                                         int* dev_status, long long limit = kWaitCycles) {
+  const bool ok = wait_one(bar, parity, abort_flag, dev_status, limit);
   return !epi_sync_or(!ok);
 }
 // Epilogue warp -> producer/MMA thread: one arrival per warp (barrier count 8).
@@ -149,16 +149,20 @@ struct FeatCfg {
   static_assert(NSLOT >= 2, "shared memory");
 };
 
-// Bytes of one chunk's record in the workspace: Phi image, Psi image, A image.
-__host__ __device__ constexpr size_t chunk_record_bytes(int m) {
-  return (size_t)2 * m * 256 + 32768;
-}
+// One chunk's record in the workspace: the Phi image (m/128 blocks of 128
+// features x 128 tokens), the Psi image (the same), the masked score image A
+// (128 queries x 128 keys), dz = the chunk's key-feature sums (m floats) and
+// the row sums of A over keys 0-63 and over keys 64-127 (2 x 128 floats).
+__host__ __device__ constexpr size_t chunk_dz_off(int m) { return (size_t)2 * m * 256 + 32768; }
+__host__ __device__ constexpr size_t chunk_den_off(int m) { return chunk_dz_off(m) + (size_t)4 * m; }
+__host__ __device__ constexpr size_t chunk_record_bytes(int m) { return chunk_den_off(m) + 1024; }
 
 struct FeatParams {
   const uint8_t* mask;
   uint8_t* img;            // chunk records [B*H][nc]
   int B, H, L, nc, heads_w, nitems;
   int* dev_status;
+  long long stall;         // testing stall before the first wait (0: none)
 };
 
 template <int D_, int M_, int R_>
@@ -181,6 +185,7 @@ __global__ void __launch_bounds__(kThreadsF, 1)
   uint64_t* bar_xfree = bars + 8;   // MMA: every GEMM reading the token tiles done
   uint64_t* bar_sc = bars + 9;      // MMA: scores complete
   uint64_t* bar_drain = bars + 10;  // MMA: everything issued has completed (abort path)
+  uint64_t* bar_never = bars + 11;  // completed by nothing (testing stall)
   uint64_t* bar_full = bars + 16;   // [NSLOT] ring slot loaded
   uint64_t* bar_empty = bars + 24;  // [NSLOT] ring slot read by the MMAs
   uint32_t* tmem_slot = (uint32_t*)(bars + 32);
@@ -206,6 +211,7 @@ __global__ void __launch_bounds__(kThreadsF, 1)
     mbar_init(bar_xfree, 1);
     mbar_init(bar_sc, 1);
     mbar_init(bar_drain, 1);
+    mbar_init(bar_never, 1);
     for (int i = 0; i < G::NSLOT; ++i) {
       mbar_init(bar_full + i, 1);
       mbar_init(bar_empty + i, 1);
@@ -356,6 +362,7 @@ __global__ void __launch_bounds__(kThreadsF, 1)
     const uint32_t lane_tm = tmem + ((uint32_t)(quad * 32) << 16);
     bool ok = true;
     int nblk = 0;
+    if (nit > 0 && p.stall > 0) ok = epi_wait(bar_never, 0, abort_flag, p.dev_status, p.stall);
     for (int j = 0; ok && j < nit; ++j) {
       const int item = it0 + j, bh = item / p.nc, c = item % p.nc;
       const int b = bh / p.H;
@@ -418,8 +425,10 @@ __global__ void __launch_bounds__(kThreadsF, 1)
         for (int q = 0; q < 4; ++q) tmem_wait_ld(v[q]);
         tc_fence_before();
         warp_arrive(bar_ffree);
-        // exp2 and bf16 packing (keys: minus the key offset)
+        // exp2 and bf16 packing (keys: minus the key offset; their sum over the
+        // chunk, of the rounded values, is the chunk's increment of z)
         uint32_t pk[64];
+        float dz = 0.f;
 #pragma unroll
         for (int q = 0; q < 4; ++q)
 #pragma unroll
@@ -430,8 +439,15 @@ __global__ void __launch_bounds__(kThreadsF, 1)
               x0 -= nrm_s[t];
               x1 -= nrm_s[t + 1];
             }
-            pk[16 * q + e] = pack_bf16(ex2(x0), ex2(x1));
+            const __nv_bfloat162 pv = __floats2bfloat162_rn(ex2(x0), ex2(x1));
+            pk[16 * q + e] = *reinterpret_cast<const uint32_t*>(&pv);
+            if (half == 0) {
+              const float2 pf = __bfloat1622float2(pv);
+              dz += pf.x + pf.y;
+            }
           }
+        if (half == 0)
+          *reinterpret_cast<float*>(rec + chunk_dz_off(M_) + 4 * (128 * f + row)) = dz;
         // the staging is free once the previous block's scores GEMM and bulk
         // stores (or the previous item's A image store) have read it
         if (nblk > 0) {
@@ -467,6 +483,7 @@ __global__ void __launch_bounds__(kThreadsF, 1)
         tmem_ld32_async(lane_tm + G::tN + 64 * half + 32, a[1]);
         tmem_wait_ld(a[0]);
         tmem_wait_ld(a[1]);
+        float rs = 0.f;      // row sum of the rounded masked scores over this key half
 #pragma unroll
         for (int cc = 0; cc < 8; ++cc) {
           uint32_t w4[4];
@@ -474,12 +491,16 @@ __global__ void __launch_bounds__(kThreadsF, 1)
           for (int e = 0; e < 4; ++e) {
             const int jj = 64 * half + 8 * cc + 2 * e;
             const uint32_t* src = a[cc >> 2] + 8 * (cc & 3) + 2 * e;
-            w4[e] = pack_bf16(jj <= row ? __uint_as_float(src[0]) : 0.f,
-                              jj + 1 <= row ? __uint_as_float(src[1]) : 0.f);
+            const __nv_bfloat162 pv = __floats2bfloat162_rn(jj <= row ? __uint_as_float(src[0]) : 0.f,
+                                                            jj + 1 <= row ? __uint_as_float(src[1]) : 0.f);
+            w4[e] = *reinterpret_cast<const uint32_t*>(&pv);
+            const float2 pf = __bfloat1622float2(pv);
+            rs += pf.x + pf.y;
           }
           st_shared_v4(s0 + G::oST + kmajor_off(row, 64 * half + 8 * cc, 16384), w4[0], w4[1],
                        w4[2], w4[3]);
         }
+        *reinterpret_cast<float*>(rec + chunk_den_off(M_) + 4 * (128 * half + row)) = rs;
       }
       tc_fence_before();
       fence_async_smem();
@@ -500,145 +521,260 @@ __global__ void __launch_bounds__(kThreadsF, 1)
 }
 
 // ================================================================ launch 2 ==
-// Every MMA of this launch uses the widest N its operands allow: an M=128,
-// K=16 MMA re-reads its 4 KB A slice from shared memory, so narrow N would be
-// limited by shared-memory bandwidth rather than by the tensor cores.
-template <int M_>
+// One CTA per (head, value block of 128 columns, feature half). The CTA keeps
+// its block of the state, S[f, v] for its NTC tiles of 128 features and 128
+// value columns, in TMEM (NTC x 128 columns) and walks the chunks in order.
+// Per chunk c, with Psi_t, Phi_t the images of its feature tiles t:
+//
+//   num  = sum_t Psi_t [S_t hi | S_t lo]      (one N = 256 MMA per K-step)
+//        + A_c[:, my keys] V_c                (intra-chunk part, split by keys)
+//   S_t += Phi_t^T V_c
+//   den  = sum_t Psi_t z_t + rowsum(A_c[:, my keys])   (CUDA cores, fp32)
+//
+// with z_t the running key-feature sums of the CTA's features (z_<c; the
+// per-chunk increments come from the features launch). With m >= 256 the two
+// feature halves of a head form a cluster of two CTAs: each finishes half of
+// the chunk's query rows and sends the partner its partial result for the
+// other half through distributed shared memory, as num/den in fp16 plus den
+// in fp32 (out = (num + den' o') / (den + den')).
+//
+// Warp 9 streams V_c (TMA) and the images (bulk copies) through a 3-slot ring;
+// warp 8 issues the MMAs; warps 0-7 are the epilogue. The S operand [S hi | S lo]
+// is rebuilt from TMEM for every chunk in halves of 64 features: epilogue group
+// h (the four warps whose TMEM lanes hold features 64h..64h+63) fills buffer h
+// while the MMAs read the other one.
+template <int D_, int M_>
 struct ValCfg {
-  static constexpr int NT = M_ / 128;        // feature tiles of the state
-  static constexpr int NITEM = 1 + 2 * NT;   // ring items per chunk: Psi_0, A_c, Phi_0, (Psi_f, Phi_f)...
-  static constexpr int NSLOT = 4;            // ring slots of 32 KB
-  static constexpr uint32_t oV = 0;          // V_c slices, 2 x 16 KB (MN-major, 64 values)
-  static constexpr uint32_t oOnes = 32768;   // 128 x 64 block, 1.0 in column 0: [V | 1] operand
-  static constexpr uint32_t oR = 49152;      // ring
-  static constexpr uint32_t oS = oR + NSLOT * 32768;   // [S hi | S lo | (z hi, z lo)], 3 x 16 KB
-  static constexpr uint32_t oBar = oS + 49152;
+  static constexpr int FS = M_ >= 256 ? 2 : 1;          // feature halves (cluster size)
+  static constexpr int VS = D_ / 128;                   // value blocks of 128 columns
+  static constexpr int NTC = M_ / (FS * 128);           // feature tiles of this CTA
+  static constexpr int NI = 2 * NTC + 1;                // ring items per chunk
+  static constexpr int NSLOT = 3;
+  static constexpr uint32_t oV = 0;                     // V_c block: 2 x 16 KB (MN-major)
+  static constexpr uint32_t oS = 32768;                 // S operand halves: 2 x 32 KB
+  static constexpr uint32_t oR = oS + 65536;            // ring: NSLOT x 32 KB
+  static constexpr uint32_t oX = oR + NSLOT * 32768;    // received o' (fp16 [64][128]) + den'
+  static constexpr uint32_t oSm = oX + 16384 + 1024;    // [2] small items: dz [NTC*128], den_a [256]
+  static constexpr uint32_t kSmB = NTC * 512 + 1024;
+  static constexpr uint32_t oZ = oSm + 2 * kSmB;        // z [NTC*128], den partials [2][2][128]
+  static constexpr uint32_t oBar = oZ + NTC * 512 + 2048;
   static constexpr uint32_t kSmem = oBar + 1024 + 1024;
-  // TMEM: state tile f at columns 80 f (64 values, z in column 64); numerator
-  // [num hi (64) | num lo (64) | den hi | den lo | 14 zero columns]
-  static constexpr uint32_t tNum = 80 * NT;
-  static_assert(M_ % 128 == 0 && M_ <= 512 && tNum + 144 <= kTmemCols, "m");
-  static_assert(NT <= 4, "tiles");
+  static constexpr uint32_t tNum = 256;                 // TMEM: S tiles [0, 128 NTC), num [256, 512)
+  static_assert(D_ % 128 == 0 && D_ <= 256 && NTC >= 1 && NTC <= 2, "shape");
+  static_assert(kSmem <= 232448, "shared memory");
 };
-// ring item index of Psi_f / Phi_f / A_c inside a chunk
-__device__ __forceinline__ int item_psi(int f) { return f == 0 ? 0 : 2 * f + 1; }
-__device__ __forceinline__ int item_phi(int f) { return 2 * f + 2; }
 
 struct ValParams {
   const uint8_t* img;
   __nv_bfloat16* out;
   int64_t ob, oh, ol;
-  int B, H, L, nc, nvb;
+  int B, H, L, nc;
   float *st_kv, *st_z;
-  int d;
   int* dev_status;
+  long long stall;         // testing stall before the first wait (0: none)
 };
 
 constexpr int kThreadsV = kEpiThreads + 64;   // + MMA warp 8 + producer warp 9
 
-template <int M_>
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::
+                   : "memory");
+}
+// Address of the same shared-memory location in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t peer_addr(uint32_t saddr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ void st_peer_v4(uint32_t a, uint32_t x, uint32_t y, uint32_t z, uint32_t w) {
+  asm volatile("st.shared::cluster.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(x), "r"(y), "r"(z),
+               "r"(w)
+               : "memory");
+}
+__device__ __forceinline__ void st_peer_f32(uint32_t a, float x) {
+  asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(a), "f"(x) : "memory");
+}
+// Arrival on a peer CTA's mbarrier, ordered after this thread's earlier writes.
+__device__ __forceinline__ void arrive_peer(uint32_t bar_addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar_addr)
+               : "memory");
+}
+// Wait for a barrier that peers arrive on (acquire at cluster scope), bounded.
+__device__ __forceinline__ bool wait_cluster(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                             int* dev_status) {
+  const uint32_t a = smem_u32(bar);
+  auto probe = [&]() -> bool {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.b32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(a), "r"(parity)
+        : "memory");
+    return ok != 0;
+  };
+  if (probe()) return true;
+  const long long t0 = clock64();
+  while (!probe()) {
+    if (*abort_flag) return false;
+    if (clock64() - t0 > kWaitCycles) {
+      *abort_flag = 1;
+      report(dev_status, DARK_ERR_TIMEOUT);
+      return false;
+    }
+  }
+  return true;
+}
+// Named barrier 2 + g over the 128 threads of epilogue group g; true if any
+// of them passes `bad`.
+__device__ __forceinline__ bool grp_sync_or(int g, bool bad) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "barrier.cta.red.or.pred q, %2, 128, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)bad), "r"(2 + g)
+      : "memory");
+  return r != 0;
+}
+__device__ __forceinline__ bool grp_wait(int g, uint64_t* bar, uint32_t parity,
+                                         volatile int* abort_flag, int* dev_status) {
+  const bool ok = wait_one(bar, parity, abort_flag, dev_status);
+  return !grp_sync_or(g, !ok);
+}
+
+template <int D_, int M_>
 __global__ void __launch_bounds__(kThreadsV, 1)
     values_kernel(const __grid_constant__ CUtensorMap tm_v, const ValParams p) {
-  using G = ValCfg<M_>;
+  using G = ValCfg<D_, M_>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   const uint32_t s0 = smem_u32(sm);
   uint64_t* bars = (uint64_t*)(sm + G::oBar);
-  uint64_t* bar_v = bars + 0;           // [2] V_c slice loaded (slot c & 1)
-  uint64_t* bar_vempty = bars + 2;      // [2] MMA: every GEMM of the chunk done (V slot free)
-  uint64_t* bar_simg = bars + 4;        // epilogue: S image written (8 arrivals)
-  uint64_t* bar_sfree = bars + 5;       // MMA: inter GEMM reading the S image done
-  uint64_t* bar_nfull = bars + 6;       // MMA: numerator complete
-  uint64_t* bar_nfree = bars + 7;       // epilogue: numerator read (8)
-  uint64_t* bar_ds = bars + 8;          // [NT] MMA: state tile f updated by the chunk
+  uint64_t* bar_v = bars + 0;           // V_c and the chunk's small items loaded
+  uint64_t* bar_vfree = bars + 1;       // MMA: every GEMM reading V_c done
+  uint64_t* bar_smfree = bars + 2;      // [2] epilogue: small items of buffer i consumed (8)
+  uint64_t* bar_simg = bars + 4;        // [2] group h: S operand half written (4)
+  uint64_t* bar_sfree = bars + 6;       // [2] MMA: GEMM reading S operand half h done
+  uint64_t* bar_ds = bars + 8;          // [2] MMA: state tile t updated by the chunk
+  uint64_t* bar_den = bars + 10;        // [2] epilogue: Psi_t read for the denominators (8)
+  uint64_t* bar_nfull = bars + 12;      // MMA: numerator complete
+  uint64_t* bar_nfree = bars + 13;      // epilogue: numerator read (8)
+  uint64_t* bar_recv = bars + 14;       // peer: its half-result for my rows arrived (128)
+  uint64_t* bar_rfree = bars + 15;      // peer: my previous half-result consumed (128)
   uint64_t* bar_full = bars + 16;       // [NSLOT] ring slot loaded
   uint64_t* bar_empty = bars + 20;      // [NSLOT] ring slot read
   uint64_t* bar_drain = bars + 24;      // MMA: everything issued has completed (abort path)
-  uint32_t* tmem_slot = (uint32_t*)(bars + 25);
-  volatile int* abort_flag = (volatile int*)(bars + 26);
+  uint64_t* bar_never = bars + 25;      // completed by nothing (testing stall)
+  uint32_t* tmem_slot = (uint32_t*)(bars + 26);
+  volatile int* abort_flag = (volatile int*)(bars + 27);
+  float* zs = (float*)(sm + G::oZ);                    // [NTC*128] z_<c of my features
+  float* den_part = (float*)(sm + G::oZ + G::NTC * 512);   // [2 parity][2 groups][128]
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int bh = blockIdx.x / p.nvb, vb = blockIdx.x % p.nvb;
+  const int fh = G::FS == 2 ? (int)cluster_rank() : 0;
+  const int unit = blockIdx.x / G::FS;                 // (head, value block)
+  const int bh = unit / G::VS, vb = unit % G::VS;
   const int b = bh / p.H, h = bh % p.H;
   const size_t rec_bytes = chunk_record_bytes(M_);
   const uint8_t* recs = p.img + (size_t)bh * p.nc * rec_bytes;
+  const int ft0 = fh * G::NTC;                         // first global feature tile of this CTA
 
   if (tid == 0) {
+    mbar_init(bar_v, 1);
+    mbar_init(bar_vfree, 1);
     for (int i = 0; i < 2; ++i) {
-      mbar_init(bar_v + i, 1);
-      mbar_init(bar_vempty + i, 1);
+      mbar_init(bar_smfree + i, 8);
+      mbar_init(bar_simg + i, 4);
+      mbar_init(bar_sfree + i, 1);
+      mbar_init(bar_ds + i, 1);
+      mbar_init(bar_den + i, 8);
     }
-    mbar_init(bar_simg, 8);
-    mbar_init(bar_sfree, 1);
     mbar_init(bar_nfull, 1);
     mbar_init(bar_nfree, 8);
-    for (int f = 0; f < G::NT; ++f) mbar_init(bar_ds + f, 1);
-    mbar_init(bar_drain, 1);
+    mbar_init(bar_recv, 128);
+    mbar_init(bar_rfree, 128);
     for (int i = 0; i < G::NSLOT; ++i) {
       mbar_init(bar_full + i, 1);
       mbar_init(bar_empty + i, 1);
     }
+    mbar_init(bar_drain, 1);
+    mbar_init(bar_never, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
-  // zeroed S image and ones block: 1.0 (bf16) at column 0 of each of its 128
-  // 128-byte rows (128B swizzle puts it in 16-byte chunk row % 8)
-  for (int i = tid; i < (int)((16384 + 49152) / 16); i += kThreadsV) {
-    const uint32_t off = i < 1024 ? G::oOnes + i * 16 : G::oS + (i - 1024) * 16;
-    st_shared_v4(s0 + off, 0u, 0u, 0u, 0u);
-  }
-  __syncthreads();
-  if (tid < 128) st_shared_u16(s0 + G::oOnes + (tid / 8) * 1024 + (tid % 8) * 144, 0x3F80);
-  fence_async_smem();
+  for (int i = tid; i < G::NTC * 128 + 512; i += kThreadsV) zs[i] = 0.f;   // z and den partials
   if (warp == 0) tmem_alloc(tmem_slot, kTmemCols);
   tc_fence_before();
   __syncthreads();
+  if (G::FS == 2) cluster_sync();     // both CTAs' barriers exist before any peer arrives
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
+  // ring item index (within a chunk) of Psi_t, Phi_t and A: Psi_0, .., Psi_{NTC-1}, A, Phi_0, ..
+  auto item_psi = [](int t) { return t; };
+  auto item_a = []() { return G::NTC; };
+  auto item_phi = [](int t) { return G::NTC + 1 + t; };
+
   if (warp == 9) {
     // ------------------------------------------------------------ producer
-    // ring items in consumption order, each into the slot its predecessor
-    // NSLOT back has left; the V slice of chunk c before the chunk's first item
     if (lane == 0) {
       prefetch_tmap(&tm_v);
-      const int total = p.nc * G::NITEM;
-      int last[G::NSLOT], vlast[2] = {-1, -1};
+      int last[G::NSLOT];
       for (int i = 0; i < G::NSLOT; ++i) last[i] = -1;
+      int vlast = -1;
       bool ok = true;
-      for (int g = 0; ok && g < total; ++g) {
-        const int c = g / G::NITEM, i = g % G::NITEM;
-        if (i == 0) {
-          if (c > 1 &&
-              !(ok = wait_one(bar_vempty + (c & 1), ((c - 2) >> 1) & 1, abort_flag, p.dev_status)))
-            break;
-          mbar_arrive_expect_tx(bar_v + (c & 1), 16384);
-          tma_load_4d(sm + G::oV + (c & 1) * 16384, &tm_v, 64 * vb, c * kC, h, b, bar_v + (c & 1));
-          vlast[c & 1] = c;
-        }
-        const int slot = g % G::NSLOT;
-        if (g >= G::NSLOT &&
-            !(ok = wait_one(bar_empty + slot, ((g / G::NSLOT) - 1) & 1, abort_flag, p.dev_status)))
-          break;
+      for (int c = 0; ok && c < p.nc; ++c) {
         const uint8_t* rc = recs + (size_t)c * rec_bytes;
-        const uint8_t* src;
-        if (i == 1) {
-          src = rc + (size_t)2 * M_ * 256;                                          // A_c
-        } else if (i == 0 || (i & 1)) {
-          src = rc + (size_t)M_ * 256 + (size_t)(i == 0 ? 0 : (i - 1) / 2) * 32768;   // Psi_f
-        } else {
-          src = rc + (size_t)((i - 2) / 2) * 32768;                                   // Phi_f
+        for (int i = 0; ok && i < G::NI; ++i) {
+          if (i == G::NTC) {
+            // V_c (once the previous chunk's GEMMs have read V_{c-1}) and the
+            // chunk's small items (into the buffer of chunk c - 2, once consumed)
+            if (c > 0 && !(ok = wait_one(bar_vfree, (c - 1) & 1, abort_flag, p.dev_status))) break;
+            if (c > 1 && !(ok = wait_one(bar_smfree + (c & 1), ((c >> 1) - 1) & 1, abort_flag,
+                                         p.dev_status)))
+              break;
+            const uint32_t dzb = G::NTC * 512, dab = G::FS == 2 ? 512 : 1024;
+            mbar_arrive_expect_tx(bar_v, 32768 + dzb + dab);
+            tma_load_4d(sm + G::oV, &tm_v, 128 * vb, c * kC, h, b, bar_v);
+            tma_load_4d(sm + G::oV + 16384, &tm_v, 128 * vb + 64, c * kC, h, b, bar_v);
+            uint8_t* smb = sm + G::oSm + (c & 1) * G::kSmB;
+            bulk_load(smb, rc + chunk_dz_off(M_) + (size_t)ft0 * 512, dzb, bar_v);
+            bulk_load(smb + dzb, rc + chunk_den_off(M_) + (G::FS == 2 ? 512 * fh : 0), dab, bar_v);
+            vlast = c;
+          }
+          const int g = c * G::NI + i, slot = g % G::NSLOT;
+          if (g >= G::NSLOT &&
+              !(ok = wait_one(bar_empty + slot, ((g / G::NSLOT) - 1) & 1, abort_flag, p.dev_status)))
+            break;
+          const uint8_t* src;
+          uint32_t bytes = 32768;
+          if (i < G::NTC) {
+            src = rc + (size_t)M_ * 256 + (size_t)(ft0 + i) * 32768;           // Psi_t
+          } else if (i == G::NTC) {
+            src = rc + (size_t)2 * M_ * 256 + (G::FS == 2 ? 16384 * fh : 0);    // A (my keys)
+            bytes = G::FS == 2 ? 16384 : 32768;
+          } else {
+            src = rc + (size_t)(ft0 + i - G::NTC - 1) * 32768;                 // Phi_t
+          }
+          mbar_arrive_expect_tx(bar_full + slot, bytes);
+          bulk_load(sm + G::oR + slot * 32768, src, bytes, bar_full + slot);
+          last[slot] = g;
         }
-        mbar_arrive_expect_tx(bar_full + slot, 32768);
-        bulk_load(sm + G::oR + slot * 32768, src, 32768, bar_full + slot);
-        last[slot] = g;
       }
       if (!ok) {
         // leave no copy in flight (a completed phase passes at once)
+        if (vlast >= 0) mbar_wait(bar_v, vlast & 1);
         for (int i = 0; i < G::NSLOT; ++i)
           if (last[i] >= 0) mbar_wait(bar_full + i, (last[i] / G::NSLOT) & 1);
-        for (int j = 0; j < 2; ++j)
-          if (vlast[j] >= 0) mbar_wait(bar_v + j, (vlast[j] >> 1) & 1);
       }
     }
     __syncwarp();
@@ -650,65 +786,68 @@ __global__ void __launch_bounds__(kThreadsV, 1)
       };
       auto slot_addr = [&](int g) -> uint32_t { return s0 + G::oR + (g % G::NSLOT) * 32768; };
       bool ok = true;
-      const uint32_t tnum = tmem + G::tNum;
-      const uint32_t sS = s0 + G::oS, sOnes = s0 + G::oOnes;
+      const uint32_t tnum = tmem + G::tNum, sV = s0 + G::oV;
       for (int c = 0; ok && c < p.nc; ++c) {
-        const int j = c & 1, g0 = c * G::NITEM;
-        const uint32_t sV = s0 + G::oV + j * 16384;
-        const uint32_t lbo_v1 = G::oOnes - (G::oV + j * 16384);   // [V | 1]: ones block after V
-        if (!(ok = wait_one(bar_v + j, (c >> 1) & 1, abort_flag, p.dev_status))) break;
-        if (c > 0 && !(ok = wait_one(bar_nfree, (c - 1) & 1, abort_flag, p.dev_status))) break;
-        for (int f = 0; ok && f < G::NT; ++f) {
-          const int k = c * G::NT + f;
-          const int gP = g0 + item_psi(f), gF = g0 + item_phi(f);
-          if (!(ok = wait_one(bar_simg, k & 1, abort_flag, p.dev_status))) break;
+        const int g0 = c * G::NI;
+        // ---- num = sum_t Psi_t [S_t hi | S_t lo], in halves of 64 features
+        for (int t = 0; ok && t < G::NTC; ++t) {
+          const int gP = g0 + item_psi(t);
           if (!(ok = wait_item(gP))) break;
-          tc_fence_after();
-          // num[:, 0:144] (+)= Psi_f [S_hi | S_lo | (z_hi, z_lo)]; the first one of
-          // the chunk starts the numerator
-          {
-            const uint32_t sPsi = slot_addr(gP);
-            constexpr uint32_t id = idesc(128, 144, true, true, false);
-#pragma unroll
-            for (int s = 0; s < 8; ++s)
-              mma(tnum, sdesc(sPsi + s * 2048, 16384, 1024), sdesc(sS + s * 2048, 16384, 1024), id,
-                  (f > 0) || (s > 0));
-            mma_commit(bar_sfree);
-          }
-          if (f == 0) {
-            // num[:, 0:64] += A_c V_c ; den: num[:, 128] += A_c 1
-            if (!(ok = wait_item(g0 + 1))) break;
+          for (int hh = 0; ok && hh < 2; ++hh) {
+            const int k = c * G::NTC + t;          // use of S operand half hh
+            if (!(ok = wait_one(bar_simg + hh, k & 1, abort_flag, p.dev_status))) break;
+            if (t == 0 && hh == 0 && c > 0 &&
+                !(ok = wait_one(bar_nfree, (c - 1) & 1, abort_flag, p.dev_status)))
+              break;
             tc_fence_after();
-            const uint32_t sA = slot_addr(g0 + 1);
-            constexpr uint32_t idv = idesc(128, 64, false, true, false);
-            constexpr uint32_t id1 = idesc(128, 16, false, true, false);
+            constexpr uint32_t id = idesc(128, 256, true, true, false);
+            const uint32_t sP = slot_addr(gP), sS = s0 + G::oS + hh * 32768;
 #pragma unroll
-            for (int s = 0; s < kC / 16; ++s) {
-              const uint64_t ad = sdesc(sA + (s / 4) * 16384 + (s % 4) * 32, 16, 1024);
-              mma(tnum, ad, sdesc(sV + s * 2048, 16384, 1024), idv, 1);
-              mma(tnum + 128, ad, sdesc(sOnes + s * 2048, 16384, 1024), id1, 1);
-            }
+            for (int s = 0; s < 4; ++s)
+              mma(tnum, sdesc(sP + (4 * hh + s) * 2048, 16384, 1024), sdesc(sS + s * 2048, 8192, 1024),
+                  id, (t | hh | s) != 0);
+            mma_commit(bar_sfree + hh);
           }
+          if (!ok) break;
+          // the epilogue reads Psi_t too (denominators): release its slot after that
+          if (!(ok = wait_one(bar_den + t, c & 1, abort_flag, p.dev_status))) break;
           mma_commit(bar_empty + gP % G::NSLOT);
-          if (f == 0) mma_commit(bar_empty + (g0 + 1) % G::NSLOT);
+        }
+        if (!ok) break;
+        // ---- num[:, hi] += A_c[:, my keys] V_c[my keys]
+        const int gA = g0 + item_a();
+        if (!(ok = wait_item(gA))) break;
+        if (!(ok = wait_one(bar_v, c & 1, abort_flag, p.dev_status))) break;
+        tc_fence_after();
+        {
+          constexpr uint32_t id = idesc(128, 128, false, true, false);
+          const uint32_t sA = slot_addr(gA);
+          constexpr int NKS = G::FS == 2 ? 4 : 8;
+#pragma unroll
+          for (int s = 0; s < NKS; ++s) {
+            const int key_step = (G::FS == 2 ? 4 * fh : 0) + s;
+            mma(tnum, sdesc(sA + (s / 4) * 16384 + (s % 4) * 32, 16, 1024),
+                sdesc(sV + key_step * 2048, 16384, 1024), id, 1u);
+          }
+          mma_commit(bar_empty + gA % G::NSLOT);
+        }
+        // ---- S_t += Phi_t^T V_c
+        for (int t = 0; ok && t < G::NTC; ++t) {
+          const int gF = g0 + item_phi(t);
           if (!(ok = wait_item(gF))) break;
           tc_fence_after();
-          // S_f += Phi_f^T [V_c | 1]
-          {
-            const uint32_t sPhi = slot_addr(gF);
-            const uint32_t ts = tmem + 80 * f;
-            constexpr uint32_t id = idesc(128, 80, false, true, false);
+          constexpr uint32_t id = idesc(128, 128, false, true, false);
+          const uint32_t sF = slot_addr(gF);
 #pragma unroll
-            for (int s = 0; s < kC / 16; ++s)
-              mma(ts, sdesc(sPhi + (s / 4) * 16384 + (s % 4) * 32, 16, 1024),
-                  sdesc(sV + s * 2048, lbo_v1, 1024), id, (c > 0) || (s > 0));
-            mma_commit(bar_ds + f);
-            mma_commit(bar_empty + gF % G::NSLOT);
-          }
+          for (int s = 0; s < kC / 16; ++s)
+            mma(tmem + 128 * t, sdesc(sF + (s / 4) * 16384 + (s % 4) * 32, 16, 1024),
+                sdesc(sV + s * 2048, 16384, 1024), id, (c > 0) || (s > 0));
+          mma_commit(bar_ds + t);
+          mma_commit(bar_empty + gF % G::NSLOT);
         }
         if (!ok) break;
         mma_commit(bar_nfull);
-        mma_commit(bar_vempty + j);
+        mma_commit(bar_vfree);
       }
       if (!ok) {
         // let every issued MMA finish before TMEM is released
@@ -719,115 +858,201 @@ __global__ void __launch_bounds__(kThreadsV, 1)
     __syncwarp();
   } else {
     // ------------------------------------------------------------ epilogue
-    const int quad = warp & 3, half = warp >> 2;
-    const int row = quad * 32 + lane;               // TMEM lane: feature of a tile / query row
+    const int quad = warp & 3, colh = warp >> 2;
+    const int row = quad * 32 + lane;               // TMEM lane
+    const int grp = quad >> 1;                      // lanes 64 grp .. 64 grp + 63
+    const int gi = (colh << 6) | ((quad & 1) << 5) | lane;   // 0..127 within the group
     const uint32_t lane_tm = tmem + ((uint32_t)(quad * 32) << 16);
-    const uint32_t sSh = s0 + G::oS, sSl = sSh + 16384, sZ = sSh + 32768;
+    const int hrow = row - 64 * grp;                // feature row within the half
     bool ok = true;
-    // out_c = (num hi + num lo) / (den hi + den lo)
-    auto output = [&](int c) -> bool {
-      if (!epi_wait(bar_nfull, c & 1, abort_flag, p.dev_status)) return false;
-      tc_fence_after();
-      const uint32_t tn = lane_tm + G::tNum;
-      uint32_t a[32], l[32];
-      tmem_ld32_async(tn + 32 * half, a);
-      tmem_ld32_async(tn + 64 + 32 * half, l);
-      tmem_wait_ld(a);
-      tmem_wait_ld(l);
-      const float den = tmem_ld1(tn + 128) + tmem_ld1(tn + 129);
-      const int tok = c * kC + row;
-      if (tok < p.L) {
-        const float inv = den > 0.f ? 1.f / den : 0.f;
-        uint32_t w[16];
-        bool bad = !isfinite(den);
-#pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const float o0 = (__uint_as_float(a[2 * e]) + __uint_as_float(l[2 * e])) * inv;
-          const float o1 = (__uint_as_float(a[2 * e + 1]) + __uint_as_float(l[2 * e + 1])) * inv;
-          bad |= !isfinite(o0) || !isfinite(o1);
-          w[e] = pack_bf16(o0, o1);
-        }
-        if (bad) report(p.dev_status, DARK_ERR_NUMERIC);
-        uint4* dst = reinterpret_cast<uint4*>(p.out + (int64_t)b * p.ob + (int64_t)h * p.oh +
-                                              (int64_t)tok * p.ol + 64 * vb + 32 * half);
-#pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4)
-          dst[q4] = make_uint4(w[4 * q4], w[4 * q4 + 1], w[4 * q4 + 2], w[4 * q4 + 3]);
-      }
-      tc_fence_before();
-      warp_arrive(bar_nfree);
-      return true;
-    };
+    if (p.stall > 0) ok = epi_wait(bar_never, 0, abort_flag, p.dev_status, p.stall);
+    float den_acc = 0.f;                            // den partial of token gi (this group)
+    const uint32_t peer = (uint32_t)(1 - fh);
     for (int c = 0; ok && c < p.nc; ++c) {
-      for (int f = 0; f < G::NT; ++f) {
-        const int k = c * G::NT + f;
-        // the S image is free once the previous tile's inter GEMM read it;
-        // tile f holds S_<c once the previous chunk's update of it is done
-        if (k > 0 && !(ok = epi_wait(bar_sfree, (k - 1) & 1, abort_flag, p.dev_status))) break;
-        if (c > 0 && !(ok = epi_wait(bar_ds + f, (c - 1) & 1, abort_flag, p.dev_status))) break;
+      const int g0 = c * G::NI;
+      // ---------------- per feature tile: S operand half, then the denominators
+      for (int t = 0; ok && t < G::NTC; ++t) {
+        const int k = c * G::NTC + t;
+        if (k > 0 && !(ok = grp_wait(grp, bar_sfree + grp, (k - 1) & 1, abort_flag, p.dev_status)))
+          break;
+        if (c > 0 && !(ok = grp_wait(grp, bar_ds + t, (c - 1) & 1, abort_flag, p.dev_status))) break;
         tc_fence_after();
-        // row `row` of S_f as hi + lo bf16 (MN-major: the feature is the K row)
-        float x[33];
-        if (c == 0) {
-#pragma unroll
-          for (int i = 0; i < 33; ++i) x[i] = 0.f;
+        // this thread: feature hrow of half grp, value columns 64 colh .. 64 colh + 63
+        uint32_t a[2][32];
+        if (c > 0) {
+          tmem_ld32_async(lane_tm + 128 * t + 64 * colh, a[0]);
+          tmem_ld32_async(lane_tm + 128 * t + 64 * colh + 32, a[1]);
+          tmem_wait_ld(a[0]);
+          tmem_wait_ld(a[1]);
         } else {
-          uint32_t a[32];
-          tmem_ld32_async(lane_tm + 80 * f + 32 * half, a);
-          tmem_wait_ld(a);
 #pragma unroll
-          for (int i = 0; i < 32; ++i) x[i] = __uint_as_float(a[i]);
-          x[32] = half == 0 ? tmem_ld1(lane_tm + 80 * f + 64) : 0.f;
+          for (int i = 0; i < 32; ++i) a[0][i] = a[1][i] = 0u;
         }
-        const uint32_t rowoff = (uint32_t)(row / 8) * 1024 + (uint32_t)(row % 8) * 128;
+        const uint32_t sS = s0 + G::oS + grp * 32768;
+        const uint32_t rowoff = (uint32_t)(hrow >> 3) * 1024 + (uint32_t)(hrow & 7) * 128;
 #pragma unroll
-        for (int cg = 0; cg < 4; ++cg) {
+        for (int cg = 0; cg < 8; ++cg) {
           uint32_t hi4[4], lo4[4];
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            const float x0 = x[8 * cg + 2 * e], x1 = x[8 * cg + 2 * e + 1];
+            const int i = 8 * cg + 2 * e;
+            const float x0 = __uint_as_float(a[i >> 5][i & 31]);
+            const float x1 = __uint_as_float(a[(i + 1) >> 5][(i + 1) & 31]);
             const __nv_bfloat162 hv = __floats2bfloat162_rn(x0, x1);
             const float2 hf = __bfloat1622float2(hv);
             hi4[e] = *reinterpret_cast<const uint32_t*>(&hv);
             lo4[e] = pack_bf16(x0 - hf.x, x1 - hf.y);
           }
-          const uint32_t off = rowoff + (uint32_t)(((4 * half + cg) ^ (row % 8)) * 16);
-          st_shared_v4(sSh + off, hi4[0], hi4[1], hi4[2], hi4[3]);
-          st_shared_v4(sSl + off, lo4[0], lo4[1], lo4[2], lo4[3]);
-        }
-        if (half == 0) {
-          // (z hi, z lo) in columns 0, 1 of the third block (16-byte chunk row % 8)
-          const float zh = __bfloat162float(__float2bfloat16_rn(x[32]));
-          asm volatile("st.shared.b32 [%0], %1;" ::"r"(sZ + rowoff + (uint32_t)(row % 8) * 16),
-                       "r"(pack_bf16(zh, x[32] - zh))
-                       : "memory");
+          const uint32_t off = rowoff + (uint32_t)((cg ^ (hrow & 7)) * 16);
+          st_shared_v4(sS + colh * 8192 + off, hi4[0], hi4[1], hi4[2], hi4[3]);          // hi block
+          st_shared_v4(sS + (2 + colh) * 8192 + off, lo4[0], lo4[1], lo4[2], lo4[3]);   // lo block
         }
         tc_fence_before();
         fence_async_smem();
-        warp_arrive(bar_simg);
-        // the previous chunk's output, while the tensor cores start on this one
-        if (f == 0 && c > 0 && !(ok = output(c - 1))) break;
+        warp_arrive(bar_simg + grp);
+        // ---- den partial of token gi over features 64 grp .. + 63 of tile t
+        const int gP = g0 + item_psi(t);
+        if (!(ok = grp_wait(grp, bar_full + gP % G::NSLOT, (gP / G::NSLOT) & 1, abort_flag,
+                            p.dev_status)))
+          break;
+        {
+          const uint8_t* psi = sm + G::oR + (gP % G::NSLOT) * 32768 + (gi >> 6) * 16384;
+          const float* zt = zs + 128 * t + 64 * grp;
+          const int tc8 = (gi & 63) >> 3, tin = gi & 7;
+          float acc = 0.f;
+#pragma unroll 8
+          for (int j = 0; j < 64; ++j) {
+            const int f = 64 * grp + j;
+            const __nv_bfloat16 v = *reinterpret_cast<const __nv_bfloat16*>(
+                psi + (f >> 3) * 1024 + (f & 7) * 128 + ((tc8 ^ (f & 7)) << 4) + tin * 2);
+            acc = fmaf(__bfloat162float(v), zt[j], acc);
+          }
+          den_acc += acc;
+        }
+        // z_<c+1 = z_<c + dz_c for these 64 features, once every thread has read
+        // them and the chunk's small items have arrived
+        if (!(ok = grp_wait(grp, bar_v, c & 1, abort_flag, p.dev_status))) break;
+        if (gi < 64) {
+          const float* dz = (const float*)(sm + G::oSm + (c & 1) * G::kSmB);
+          zs[128 * t + 64 * grp + gi] += dz[128 * t + 64 * grp + gi];
+        }
+        warp_arrive(bar_den + t);
       }
-    }
-    if (ok) ok = output(p.nc - 1);
-    // final state [S | z]: every GEMM of the last chunk is complete
-    if (ok && p.st_kv != nullptr) {
+      if (!ok) break;
+      // ---------------- output of chunk c
+      den_part[((c & 1) * 2 + grp) * 128 + gi] = den_acc;
+      den_acc = 0.f;
+      if (!(ok = epi_wait(bar_nfull, c & 1, abort_flag, p.dev_status))) break;
       tc_fence_after();
-      for (int f = 0; f < G::NT; ++f) {
-        uint32_t a[32];
-        tmem_ld32_async(lane_tm + 80 * f + 32 * half, a);
-        tmem_wait_ld(a);
-        const int feat = 128 * f + row;
-        float* kv = p.st_kv + ((size_t)bh * M_ + feat) * p.d + 64 * vb + 32 * half;
+      float num[64];
+      {
+        uint32_t hi[2][32], lo[2][32];
+        tmem_ld32_async(lane_tm + G::tNum + 64 * colh, hi[0]);
+        tmem_ld32_async(lane_tm + G::tNum + 64 * colh + 32, hi[1]);
+        tmem_ld32_async(lane_tm + G::tNum + 128 + 64 * colh, lo[0]);
+        tmem_ld32_async(lane_tm + G::tNum + 128 + 64 * colh + 32, lo[1]);
+        tmem_wait_ld(hi[0]);
+        tmem_wait_ld(hi[1]);
+        tmem_wait_ld(lo[0]);
+        tmem_wait_ld(lo[1]);
 #pragma unroll
-        for (int i = 0; i < 32; ++i) kv[i] = __uint_as_float(a[i]);
-        const float z = tmem_ld1(lane_tm + 80 * f + 64);
-        if (vb == 0 && half == 0) p.st_z[(size_t)bh * M_ + feat] = z;
+        for (int i = 0; i < 64; ++i)
+          num[i] = __uint_as_float(hi[i >> 5][i & 31]) + __uint_as_float(lo[i >> 5][i & 31]);
+      }
+      tc_fence_before();
+      warp_arrive(bar_nfree);
+      // den = the two groups' partials for query row `row` + rowsum(A_c[row, my keys])
+      const float* da = (const float*)(sm + G::oSm + (c & 1) * G::kSmB + G::NTC * 512);
+      const float den = den_part[((c & 1) * 2 + 0) * 128 + row] +
+                        den_part[((c & 1) * 2 + 1) * 128 + row] + da[row] +
+                        (G::FS == 1 ? da[128 + row] : 0.f);
+      const int tok = c * kC + row;
+      if (G::FS == 1 || (row >> 6) == fh) {
+        // a row this CTA finishes
+        float dp = 0.f;
+        uint32_t op[32];
+        if (G::FS == 2) {
+          if (!(ok = wait_cluster(bar_recv, c & 1, abort_flag, p.dev_status))) break;
+          const uint32_t xr = s0 + G::oX + (uint32_t)(row & 63) * 256 + colh * 128;
+#pragma unroll
+          for (int q4 = 0; q4 < 8; ++q4) {
+            const uint4 u = ld_shared_v4(xr + q4 * 16);
+            op[4 * q4] = u.x;
+            op[4 * q4 + 1] = u.y;
+            op[4 * q4 + 2] = u.z;
+            op[4 * q4 + 3] = u.w;
+          }
+          dp = ((const float*)(sm + G::oX + 16384))[row & 63];
+        }
+        const float dt = den + dp;
+        if (tok < p.L) {
+          const float inv = dt > 0.f ? 1.f / dt : 0.f;
+          uint32_t w[32];
+          bool bad = !isfinite(dt);
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            float o0 = num[2 * e], o1 = num[2 * e + 1];
+            if (G::FS == 2) {
+              const float2 of = __half22float2(*reinterpret_cast<const __half2*>(&op[e]));
+              o0 = fmaf(dp, of.x, o0);
+              o1 = fmaf(dp, of.y, o1);
+            }
+            o0 *= inv;
+            o1 *= inv;
+            bad |= !isfinite(o0) || !isfinite(o1);
+            w[e] = pack_bf16(o0, o1);
+          }
+          if (bad) report(p.dev_status, DARK_ERR_NUMERIC);
+          uint4* dst = reinterpret_cast<uint4*>(p.out + (int64_t)b * p.ob + (int64_t)h * p.oh +
+                                                (int64_t)tok * p.ol + 128 * vb + 64 * colh);
+#pragma unroll
+          for (int q4 = 0; q4 < 8; ++q4)
+            dst[q4] = make_uint4(w[4 * q4], w[4 * q4 + 1], w[4 * q4 + 2], w[4 * q4 + 3]);
+        }
+        if (G::FS == 2) arrive_peer(peer_addr(smem_u32(bar_rfree), peer));
+      } else {
+        // a row the peer finishes: send num/den (fp16) and den
+        if (c > 0 && !(ok = wait_cluster(bar_rfree, (c - 1) & 1, abort_flag, p.dev_status))) break;
+        const float inv = den > 0.f ? 1.f / den : 0.f;
+        uint32_t w[32];
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          const __half2 hv = __floats2half2_rn(num[2 * e] * inv, num[2 * e + 1] * inv);
+          w[e] = *reinterpret_cast<const uint32_t*>(&hv);
+        }
+        const uint32_t xr = peer_addr(s0 + G::oX + (uint32_t)(row & 63) * 256 + colh * 128, peer);
+#pragma unroll
+        for (int q4 = 0; q4 < 8; ++q4)
+          st_peer_v4(xr + q4 * 16, w[4 * q4], w[4 * q4 + 1], w[4 * q4 + 2], w[4 * q4 + 3]);
+        if (colh == 0) st_peer_f32(peer_addr(s0 + G::oX + 16384 + (uint32_t)(row & 63) * 4, peer), den);
+        arrive_peer(peer_addr(smem_u32(bar_recv), peer));
+      }
+      warp_arrive(bar_smfree + (c & 1));
+    }
+    // final state: S_t (my features x my 128 value columns) and z (first value block)
+    if (ok && p.st_kv != nullptr) {
+      for (int t = 0; ok && t < G::NTC; ++t)
+        ok = epi_wait(bar_ds + t, (p.nc - 1) & 1, abort_flag, p.dev_status);
+      if (ok) {
+        tc_fence_after();
+        for (int t = 0; t < G::NTC; ++t) {
+          uint32_t a[2][32];
+          tmem_ld32_async(lane_tm + 128 * t + 64 * colh, a[0]);
+          tmem_ld32_async(lane_tm + 128 * t + 64 * colh + 32, a[1]);
+          tmem_wait_ld(a[0]);
+          tmem_wait_ld(a[1]);
+          const int feat = 128 * (ft0 + t) + row;
+          float* kv = p.st_kv + ((size_t)bh * M_ + feat) * D_ + 128 * vb + 64 * colh;
+#pragma unroll
+          for (int i = 0; i < 64; ++i) kv[i] = __uint_as_float(a[i >> 5][i & 31]);
+          if (vb == 0 && colh == 0) p.st_z[(size_t)bh * M_ + feat] = zs[128 * t + row];
+        }
       }
     }
   }
   tc_fence_before();
   __syncthreads();
+  if (G::FS == 2) cluster_sync();     // no peer may still write into this CTA
   if (warp == 0) {
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
@@ -861,7 +1086,7 @@ bool shape_ok(int d, int m, int r) {
 template <int D_, int M_, int R_>
 cudaError_t launch(const FwdArgs& a) {
   using F = FeatCfg<D_, M_, R_>;
-  using V = ValCfg<M_>;
+  using V = ValCfg<D_, M_>;
   const int nc = (a.L + kC - 1) / kC;
   uint8_t* img = (uint8_t*)a.ws + kWsHeader;
   FeatParams fp;
@@ -873,10 +1098,11 @@ cudaError_t launch(const FwdArgs& a) {
   fp.nc = nc;
   fp.heads_w = a.heads_w;
   fp.dev_status = a.dev_status;
+  fp.stall = test_stall_cycles();
   static int smem_f[64], smem_v[64];
   cudaError_t e = set_smem_limit_once((const void*)features_kernel<D_, M_, R_>, (int)F::kSmem, smem_f);
   if (e != cudaSuccess) return e;
-  e = set_smem_limit_once((const void*)values_kernel<M_>, (int)V::kSmem, smem_v);
+  e = set_smem_limit_once((const void*)values_kernel<D_, M_>, (int)V::kSmem, smem_v);
   if (e != cudaSuccess) return e;
   fp.nitems = a.B * a.H * nc;
   const int grid_f = fp.nitems < num_sms() ? fp.nitems : num_sms();
@@ -894,12 +1120,27 @@ cudaError_t launch(const FwdArgs& a) {
   vp.H = a.H;
   vp.L = a.L;
   vp.nc = nc;
-  vp.nvb = D_ / 64;
   vp.st_kv = a.st_kv;
   vp.st_z = a.st_z;
-  vp.d = D_;
   vp.dev_status = a.dev_status;
-  values_kernel<M_><<<a.B * a.H * (D_ / 64), kThreadsV, V::kSmem, a.stream>>>(a.tm_v, vp);
+  vp.stall = test_stall_cycles();
+  // one CTA per (head, 128 value columns, feature half); the feature halves
+  // of a (head, value block) form a cluster
+  cudaLaunchConfig_t cfg;
+  memset(&cfg, 0, sizeof(cfg));
+  cfg.gridDim = dim3(a.B * a.H * V::VS * V::FS);
+  cfg.blockDim = dim3(kThreadsV);
+  cfg.dynamicSmemBytes = V::kSmem;
+  cfg.stream = a.stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = V::FS;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, values_kernel<D_, M_>, a.tm_v, vp);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

@@ -34,7 +34,7 @@ EXPORTS = ("dark_abi_version", "dark_status_string", "dark_projection_bytes",
            "dark_attention_bwd_workspace_bytes", "dark_attention_bwd",
            "dark_sample_omega_workspace_bytes", "dark_sample_omega", "dark_redraw_schedule_init",
            "dark_redraw_on_forward", "dark_redraw_request", "dark_redraw_set_fixed",
-           "dark_auto_uses_exact")
+           "dark_auto_uses_exact", "dark_set_test_stall_cycles")
 
 
 class dark_projection(ctypes.Structure):
@@ -58,6 +58,8 @@ _P = ctypes.POINTER
 _vp, _i, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
 _lib.dark_abi_version.restype = _i
 _lib.dark_status_string.restype = ctypes.c_char_p
+_lib.dark_set_test_stall_cycles.argtypes = [ctypes.c_longlong]
+_lib.dark_set_test_stall_cycles.restype = None
 _lib.dark_status_string.argtypes = [_i]
 _lib.dark_projection_bytes.restype = _sz
 _lib.dark_projection_bytes.argtypes = [_i, _i, _i, _i, _i]
@@ -170,6 +172,11 @@ def dark_abi_version() -> int:
 
 def dark_status_string(status: int) -> str:
     return _lib.dark_status_string(status).decode()
+
+
+def dark_set_test_stall_cycles(cycles: int) -> None:
+    """Testing hook of the device time-out path (0 turns it off); see dark.h."""
+    _lib.dark_set_test_stall_cycles(int(cycles))
 
 
 def dark_projection_bytes(heads: int, m: int, r: int, d: int, dtype: int) -> int:
