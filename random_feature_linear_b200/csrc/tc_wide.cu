@@ -55,10 +55,13 @@ constexpr uint32_t kSmemBudget = 229376;   // 224 KB of operands + barriers + al
 __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
-// shared -> global bulk copy (16-byte aligned, size a multiple of 16)
-__device__ __forceinline__ void bulk_store(void* gdst, uint32_t ssrc, uint32_t bytes) {
-  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"((uint64_t)gdst),
-               "r"(ssrc), "r"(bytes)
+// shared -> global bulk copy (16-byte aligned, size a multiple of 16) with an
+// L2 eviction policy for the written lines
+__device__ __forceinline__ void bulk_store_hint(void* gdst, uint32_t ssrc, uint32_t bytes,
+                                                uint64_t policy) {
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group.L2::cache_hint [%0], [%1], %2, %3;" ::"l"(
+                   (uint64_t)gdst),
+               "r"(ssrc), "r"(bytes), "l"(policy)
                : "memory");
 }
 __device__ __forceinline__ void bulk_commit() {
@@ -233,6 +236,8 @@ __global__ void __launch_bounds__(kThreadsF, 1)
       prefetch_tmap(&tm_w);
       prefetch_tmap(&tm_q);
       prefetch_tmap(&tm_k);
+      // projection rows are re-read for every chunk: keep them in L2
+      const uint64_t keep = l2_evict_last(), once = l2_evict_first();
       int last[G::NSLOT];
       for (int i = 0; i < G::NSLOT; ++i) last[i] = -1;
       bool ok = true;
@@ -244,8 +249,9 @@ __global__ void __launch_bounds__(kThreadsF, 1)
         if (j > 0 && !(ok = wait_one(bar_xfree, (j - 1) & 1, abort_flag, p.dev_status))) break;
         mbar_arrive_expect_tx(bar_x, 2 * G::DS * 16384);
         for (int s = 0; s < G::DS; ++s) {
-          tma_load_4d(sm + G::oX + s * G::kXSlab, &tm_k, 64 * s, c * kC, h, b, bar_x);
-          tma_load_4d(sm + G::oX + s * G::kXSlab + 16384, &tm_q, 64 * s, c * kC, h, b, bar_x);
+          tma_load_4d_hint(sm + G::oX + s * G::kXSlab, &tm_k, 64 * s, c * kC, h, b, bar_x, once);
+          tma_load_4d_hint(sm + G::oX + s * G::kXSlab + 16384, &tm_q, 64 * s, c * kC, h, b, bar_x,
+                           once);
         }
         xlast = j;
         for (int i = 0; i < G::NITEMS; ++i, ++g) {
@@ -259,13 +265,13 @@ __global__ void __launch_bounds__(kThreadsF, 1)
             const int s = i / G::NRH, rg = i % G::NRH;
             mbar_arrive_expect_tx(bar_full + slot, G::NRROWS * 128);
             for (int q = 0; q < G::NRROWS / 64; ++q)
-              tma_load_2d(dst + q * 8192, &tm_w, 64 * s, wrow0 + M_ + rg * 128 + 64 * q,
-                          bar_full + slot);
+              tma_load_2d_hint(dst + q * 8192, &tm_w, 64 * s, wrow0 + M_ + rg * 128 + 64 * q,
+                               bar_full + slot, keep);
           } else {                     // feature rows of block f, d slab s
             const int f = (i - G::NNORM) / G::DS, s = (i - G::NNORM) % G::DS;
             mbar_arrive_expect_tx(bar_full + slot, 16384);
-            tma_load_2d(dst, &tm_w, 64 * s, wrow0 + 128 * f, bar_full + slot);
-            tma_load_2d(dst + 8192, &tm_w, 64 * s, wrow0 + 128 * f + 64, bar_full + slot);
+            tma_load_2d_hint(dst, &tm_w, 64 * s, wrow0 + 128 * f, bar_full + slot, keep);
+            tma_load_2d_hint(dst + 8192, &tm_w, 64 * s, wrow0 + 128 * f + 64, bar_full + slot, keep);
           }
           last[slot] = g;
         }
@@ -371,6 +377,7 @@ __global__ void __launch_bounds__(kThreadsF, 1)
       // bf16 -> fp16 in place (|x| >= 65504 is reported)
       {
         bool bad = false;
+#pragma unroll 4
         for (int i = etid; i < (int)(G::DS * G::kXSlab / 16); i += kEpiThreads) {
           const uint32_t a = s0 + G::oX + i * 16;
           uint4 u = ld_shared_v4(a);
@@ -465,8 +472,11 @@ __global__ void __launch_bounds__(kThreadsF, 1)
         fence_async_smem();
         epi_sync();
         if (etid == 0) {
-          bulk_store(rec + (size_t)f * 32768, s0 + G::oST, 32768);
-          bulk_store(rec + (size_t)M_ * 256 + (size_t)f * 32768, s0 + G::oST + 32768, 32768);
+          // the images stream through L2 once: evict them before the projection rows
+          const uint64_t once = l2_evict_first();
+          bulk_store_hint(rec + (size_t)f * 32768, s0 + G::oST, 32768, once);
+          bulk_store_hint(rec + (size_t)M_ * 256 + (size_t)f * 32768, s0 + G::oST + 32768, 32768,
+                          once);
           bulk_commit();
         }
         warp_arrive(bar_stage);
@@ -506,7 +516,7 @@ __global__ void __launch_bounds__(kThreadsF, 1)
       fence_async_smem();
       epi_sync();
       if (etid == 0) {
-        bulk_store(rec + (size_t)2 * M_ * 256, s0 + G::oST, 32768);
+        bulk_store_hint(rec + (size_t)2 * M_ * 256, s0 + G::oST, 32768, l2_evict_first());
         bulk_commit();
       }
     }
@@ -548,13 +558,18 @@ struct ValCfg {
   static constexpr int FS = M_ >= 256 ? 2 : 1;          // feature halves (cluster size)
   static constexpr int VS = D_ / 128;                   // value blocks of 128 columns
   static constexpr int NTC = M_ / (FS * 128);           // feature tiles of this CTA
-  static constexpr int NI = 2 * NTC + 1;                // ring items per chunk
-  static constexpr int NSLOT = 3;
+  // ring items of 16 KB per chunk: Psi_t in halves of 64 features (2 per tile),
+  // A (my key block, or both), Phi_t in blocks of 64 tokens (2 per tile)
+  static constexpr int NA = FS == 2 ? 1 : 2;
+  static constexpr int NI = 4 * NTC + NA;
+  static constexpr int NSLOT = 5;
   static constexpr uint32_t oV = 0;                     // V_c block: 2 x 16 KB (MN-major)
   static constexpr uint32_t oS = 32768;                 // S operand halves: 2 x 32 KB
-  static constexpr uint32_t oR = oS + 65536;            // ring: NSLOT x 32 KB
-  static constexpr uint32_t oX = oR + NSLOT * 32768;    // received o' (fp16 [64][128]) + den'
-  static constexpr uint32_t oSm = oX + 16384 + 1024;    // [2] small items: dz [NTC*128], den_a [256]
+  static constexpr uint32_t oR = oS + 65536;            // ring: NSLOT x 16 KB
+  static constexpr uint32_t kXB = 16384 + 1024;         // received o' (fp16 [64][128]) + den' [64]
+  static constexpr uint32_t kXBytes = 16384 + 256;      // bytes the peer sends per chunk
+  static constexpr uint32_t oX = oR + NSLOT * 16384;    // [2] receive buffers (chunk parity)
+  static constexpr uint32_t oSm = oX + 2 * kXB;         // [2] small items: dz [NTC*128], den_a [256]
   static constexpr uint32_t kSmB = NTC * 512 + 1024;
   static constexpr uint32_t oZ = oSm + 2 * kSmB;        // z [NTC*128], den partials [2][2][128]
   static constexpr uint32_t oBar = oZ + NTC * 512 + 2048;
@@ -591,17 +606,24 @@ __device__ __forceinline__ uint32_t peer_addr(uint32_t saddr, uint32_t rank) {
   asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
   return r;
 }
-__device__ __forceinline__ void st_peer_v4(uint32_t a, uint32_t x, uint32_t y, uint32_t z, uint32_t w) {
-  asm volatile("st.shared::cluster.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(x), "r"(y), "r"(z),
-               "r"(w)
+// Arrival on a peer CTA's mbarrier, not ordered after this thread's writes
+// (the caller's earlier reads are complete: their values have been used).
+__device__ __forceinline__ void arrive_peer_relaxed(uint32_t bar_addr) {
+  asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar_addr)
                : "memory");
 }
-__device__ __forceinline__ void st_peer_f32(uint32_t a, float x) {
-  asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(a), "f"(x) : "memory");
+// Asynchronous stores into a peer CTA's shared memory; the bytes count towards
+// the transaction count of the peer's mbarrier at `bar_addr`.
+__device__ __forceinline__ void st_async_v4(uint32_t a, uint32_t x, uint32_t y, uint32_t z,
+                                            uint32_t w, uint32_t bar_addr) {
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.b32 [%0], {%1, %2, %3, %4}, [%5];" ::"r"(
+                   a),
+               "r"(x), "r"(y), "r"(z), "r"(w), "r"(bar_addr)
+               : "memory");
 }
-// Arrival on a peer CTA's mbarrier, ordered after this thread's earlier writes.
-__device__ __forceinline__ void arrive_peer(uint32_t bar_addr) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar_addr)
+__device__ __forceinline__ void st_async_f32(uint32_t a, float x, uint32_t bar_addr) {
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.b32 [%0], %1, [%2];" ::"r"(a),
+               "r"(__float_as_uint(x)), "r"(bar_addr)
                : "memory");
 }
 // Wait for a barrier that peers arrive on (acquire at cluster scope), bounded.
@@ -665,17 +687,17 @@ __global__ void __launch_bounds__(kThreadsV, 1)
   uint64_t* bar_simg = bars + 4;        // [2] group h: S operand half written (4)
   uint64_t* bar_sfree = bars + 6;       // [2] MMA: GEMM reading S operand half h done
   uint64_t* bar_ds = bars + 8;          // [2] MMA: state tile t updated by the chunk
-  uint64_t* bar_den = bars + 10;        // [2] epilogue: Psi_t read for the denominators (8)
-  uint64_t* bar_nfull = bars + 12;      // MMA: numerator complete
-  uint64_t* bar_nfree = bars + 13;      // epilogue: numerator read (8)
-  uint64_t* bar_recv = bars + 14;       // peer: its half-result for my rows arrived (128)
-  uint64_t* bar_rfree = bars + 15;      // peer: my previous half-result consumed (128)
-  uint64_t* bar_full = bars + 16;       // [NSLOT] ring slot loaded
-  uint64_t* bar_empty = bars + 20;      // [NSLOT] ring slot read
-  uint64_t* bar_drain = bars + 24;      // MMA: everything issued has completed (abort path)
-  uint64_t* bar_never = bars + 25;      // completed by nothing (testing stall)
-  uint32_t* tmem_slot = (uint32_t*)(bars + 26);
-  volatile int* abort_flag = (volatile int*)(bars + 27);
+  uint64_t* bar_den = bars + 10;        // [2 t][2 h] group h: Psi_{t,h} read for the denominators (4)
+  uint64_t* bar_nfull = bars + 14;      // MMA: numerator complete
+  uint64_t* bar_nfree = bars + 15;      // epilogue: numerator read (8)
+  uint64_t* bar_recv = bars + 38;       // [2] peer: its half-result for my rows arrived (128)
+  uint64_t* bar_rfree = bars + 40;      // [2] peer: my half-result in its buffer consumed (128)
+  uint64_t* bar_drain = bars + 18;      // MMA: everything issued has completed (abort path)
+  uint64_t* bar_never = bars + 19;      // completed by nothing (testing stall)
+  uint64_t* bar_full = bars + 20;       // [NSLOT] ring slot loaded
+  uint64_t* bar_empty = bars + 28;      // [NSLOT] ring slot read
+  uint32_t* tmem_slot = (uint32_t*)(bars + 36);
+  volatile int* abort_flag = (volatile int*)(bars + 37);
   float* zs = (float*)(sm + G::oZ);                    // [NTC*128] z_<c of my features
   float* den_part = (float*)(sm + G::oZ + G::NTC * 512);   // [2 parity][2 groups][128]
 
@@ -696,12 +718,15 @@ __global__ void __launch_bounds__(kThreadsV, 1)
       mbar_init(bar_simg + i, 4);
       mbar_init(bar_sfree + i, 1);
       mbar_init(bar_ds + i, 1);
-      mbar_init(bar_den + i, 8);
+      mbar_init(bar_den + i, 4);
+      mbar_init(bar_den + 2 + i, 4);
     }
     mbar_init(bar_nfull, 1);
     mbar_init(bar_nfree, 8);
-    mbar_init(bar_recv, 128);
-    mbar_init(bar_rfree, 128);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bar_recv + i, 1);
+      mbar_init(bar_rfree + i, 1);
+    }
     for (int i = 0; i < G::NSLOT; ++i) {
       mbar_init(bar_full + i, 1);
       mbar_init(bar_empty + i, 1);
@@ -710,6 +735,9 @@ __global__ void __launch_bounds__(kThreadsV, 1)
     mbar_init(bar_never, 1);
     *abort_flag = 0;
     fence_mbar_init();
+    // the peer's half-results for chunks 0 and 1 (its stores complete these)
+    if (G::FS == 2)
+      for (int i = 0; i < 2 && i < p.nc; ++i) mbar_arrive_expect_tx(bar_recv + i, G::kXBytes);
   }
   for (int i = tid; i < G::NTC * 128 + 512; i += kThreadsV) zs[i] = 0.f;   // z and den partials
   if (warp == 0) tmem_alloc(tmem_slot, kTmemCols);
@@ -720,9 +748,11 @@ __global__ void __launch_bounds__(kThreadsV, 1)
   const uint32_t tmem = *tmem_slot;
 
   // ring item index (within a chunk) of Psi_t, Phi_t and A: Psi_0, .., Psi_{NTC-1}, A, Phi_0, ..
-  auto item_psi = [](int t) { return t; };
-  auto item_a = []() { return G::NTC; };
-  auto item_phi = [](int t) { return G::NTC + 1 + t; };
+  // ring items of a chunk: Psi_{t,h} (features 64h.. of tile t), then A_j (key
+  // block j), then Phi_{t,kb} (tokens 64kb.. of tile t)
+  auto item_psi = [](int t, int hh) { return 2 * t + hh; };
+  auto item_a = [](int j) { return 2 * G::NTC + j; };
+  auto item_phi = [](int t, int kb) { return 2 * G::NTC + G::NA + 2 * t + kb; };
 
   if (warp == 9) {
     // ------------------------------------------------------------ producer
@@ -735,7 +765,7 @@ __global__ void __launch_bounds__(kThreadsV, 1)
       for (int c = 0; ok && c < p.nc; ++c) {
         const uint8_t* rc = recs + (size_t)c * rec_bytes;
         for (int i = 0; ok && i < G::NI; ++i) {
-          if (i == G::NTC) {
+          if (i == 2 * G::NTC) {
             // V_c (once the previous chunk's GEMMs have read V_{c-1}) and the
             // chunk's small items (into the buffer of chunk c - 2, once consumed)
             if (c > 0 && !(ok = wait_one(bar_vfree, (c - 1) & 1, abort_flag, p.dev_status))) break;
@@ -755,18 +785,21 @@ __global__ void __launch_bounds__(kThreadsV, 1)
           if (g >= G::NSLOT &&
               !(ok = wait_one(bar_empty + slot, ((g / G::NSLOT) - 1) & 1, abort_flag, p.dev_status)))
             break;
-          const uint8_t* src;
-          uint32_t bytes = 32768;
-          if (i < G::NTC) {
-            src = rc + (size_t)M_ * 256 + (size_t)(ft0 + i) * 32768;           // Psi_t
-          } else if (i == G::NTC) {
-            src = rc + (size_t)2 * M_ * 256 + (G::FS == 2 ? 16384 * fh : 0);    // A (my keys)
-            bytes = G::FS == 2 ? 16384 : 32768;
+          uint8_t* dst = sm + G::oR + slot * 16384;
+          mbar_arrive_expect_tx(bar_full + slot, 16384);
+          if (i < 2 * G::NTC) {
+            // Psi_{t,h}: rows 64h.. of both token blocks of the tile's image
+            const uint8_t* src = rc + (size_t)M_ * 256 + (size_t)(ft0 + i / 2) * 32768 + (i & 1) * 8192;
+            bulk_load(dst, src, 8192, bar_full + slot);
+            bulk_load(dst + 8192, src + 16384, 8192, bar_full + slot);
+          } else if (i < 2 * G::NTC + G::NA) {
+            const int j = G::FS == 2 ? fh : i - 2 * G::NTC;                      // A, key block j
+            bulk_load(dst, rc + (size_t)2 * M_ * 256 + 16384 * j, 16384, bar_full + slot);
           } else {
-            src = rc + (size_t)(ft0 + i - G::NTC - 1) * 32768;                 // Phi_t
+            const int q = i - 2 * G::NTC - G::NA;                               // Phi_{t,kb}
+            bulk_load(dst, rc + (size_t)(ft0 + q / 2) * 32768 + (q & 1) * 16384, 16384,
+                      bar_full + slot);
           }
-          mbar_arrive_expect_tx(bar_full + slot, bytes);
-          bulk_load(sm + G::oR + slot * 32768, src, bytes, bar_full + slot);
           last[slot] = g;
         }
       }
@@ -784,17 +817,17 @@ __global__ void __launch_bounds__(kThreadsV, 1)
       auto wait_item = [&](int g) -> bool {
         return wait_one(bar_full + g % G::NSLOT, (g / G::NSLOT) & 1, abort_flag, p.dev_status);
       };
-      auto slot_addr = [&](int g) -> uint32_t { return s0 + G::oR + (g % G::NSLOT) * 32768; };
+      auto slot_addr = [&](int g) -> uint32_t { return s0 + G::oR + (g % G::NSLOT) * 16384; };
       bool ok = true;
       const uint32_t tnum = tmem + G::tNum, sV = s0 + G::oV;
       for (int c = 0; ok && c < p.nc; ++c) {
         const int g0 = c * G::NI;
         // ---- num = sum_t Psi_t [S_t hi | S_t lo], in halves of 64 features
         for (int t = 0; ok && t < G::NTC; ++t) {
-          const int gP = g0 + item_psi(t);
-          if (!(ok = wait_item(gP))) break;
           for (int hh = 0; ok && hh < 2; ++hh) {
+            const int gP = g0 + item_psi(t, hh);
             const int k = c * G::NTC + t;          // use of S operand half hh
+            if (!(ok = wait_item(gP))) break;
             if (!(ok = wait_one(bar_simg + hh, k & 1, abort_flag, p.dev_status))) break;
             if (t == 0 && hh == 0 && c > 0 &&
                 !(ok = wait_one(bar_nfree, (c - 1) & 1, abort_flag, p.dev_status)))
@@ -803,47 +836,50 @@ __global__ void __launch_bounds__(kThreadsV, 1)
             constexpr uint32_t id = idesc(128, 256, true, true, false);
             const uint32_t sP = slot_addr(gP), sS = s0 + G::oS + hh * 32768;
 #pragma unroll
-            for (int s = 0; s < 4; ++s)
-              mma(tnum, sdesc(sP + (4 * hh + s) * 2048, 16384, 1024), sdesc(sS + s * 2048, 8192, 1024),
-                  id, (t | hh | s) != 0);
+            for (int st = 0; st < 4; ++st)
+              mma(tnum, sdesc(sP + st * 2048, 8192, 1024), sdesc(sS + st * 2048, 8192, 1024), id,
+                  (t | hh | st) != 0);
             mma_commit(bar_sfree + hh);
           }
-          if (!ok) break;
-          // the epilogue reads Psi_t too (denominators): release its slot after that
-          if (!(ok = wait_one(bar_den + t, c & 1, abort_flag, p.dev_status))) break;
-          mma_commit(bar_empty + gP % G::NSLOT);
         }
+        // the epilogue reads the Psi items too (denominators): release them after that
+        for (int t = 0; ok && t < G::NTC; ++t)
+          for (int hh = 0; ok && hh < 2; ++hh) {
+            if (!(ok = wait_one(bar_den + 2 * t + hh, c & 1, abort_flag, p.dev_status))) break;
+            mma_commit(bar_empty + (g0 + item_psi(t, hh)) % G::NSLOT);
+          }
         if (!ok) break;
         // ---- num[:, hi] += A_c[:, my keys] V_c[my keys]
-        const int gA = g0 + item_a();
-        if (!(ok = wait_item(gA))) break;
-        if (!(ok = wait_one(bar_v, c & 1, abort_flag, p.dev_status))) break;
-        tc_fence_after();
-        {
-          constexpr uint32_t id = idesc(128, 128, false, true, false);
-          const uint32_t sA = slot_addr(gA);
-          constexpr int NKS = G::FS == 2 ? 4 : 8;
-#pragma unroll
-          for (int s = 0; s < NKS; ++s) {
-            const int key_step = (G::FS == 2 ? 4 * fh : 0) + s;
-            mma(tnum, sdesc(sA + (s / 4) * 16384 + (s % 4) * 32, 16, 1024),
-                sdesc(sV + key_step * 2048, 16384, 1024), id, 1u);
-          }
-          mma_commit(bar_empty + gA % G::NSLOT);
-        }
-        // ---- S_t += Phi_t^T V_c
-        for (int t = 0; ok && t < G::NTC; ++t) {
-          const int gF = g0 + item_phi(t);
-          if (!(ok = wait_item(gF))) break;
+        for (int j = 0; ok && j < G::NA; ++j) {
+          const int gA = g0 + item_a(j);
+          if (!(ok = wait_item(gA))) break;
+          if (j == 0 && !(ok = wait_one(bar_v, c & 1, abort_flag, p.dev_status))) break;
           tc_fence_after();
           constexpr uint32_t id = idesc(128, 128, false, true, false);
-          const uint32_t sF = slot_addr(gF);
+          const uint32_t sA = slot_addr(gA);
+          const int kb = G::FS == 2 ? fh : j;      // key block of V
 #pragma unroll
-          for (int s = 0; s < kC / 16; ++s)
-            mma(tmem + 128 * t, sdesc(sF + (s / 4) * 16384 + (s % 4) * 32, 16, 1024),
-                sdesc(sV + s * 2048, 16384, 1024), id, (c > 0) || (s > 0));
+          for (int st = 0; st < 4; ++st)
+            mma(tnum, sdesc(sA + st * 32, 16, 1024), sdesc(sV + (4 * kb + st) * 2048, 16384, 1024), id,
+                1u);
+          mma_commit(bar_empty + gA % G::NSLOT);
+        }
+        // ---- S_t += Phi_t^T V_c, in blocks of 64 tokens
+        for (int t = 0; ok && t < G::NTC; ++t) {
+          for (int kb = 0; ok && kb < 2; ++kb) {
+            const int gF = g0 + item_phi(t, kb);
+            if (!(ok = wait_item(gF))) break;
+            tc_fence_after();
+            constexpr uint32_t id = idesc(128, 128, false, true, false);
+            const uint32_t sF = slot_addr(gF);
+#pragma unroll
+            for (int st = 0; st < 4; ++st)
+              mma(tmem + 128 * t, sdesc(sF + st * 32, 16, 1024),
+                  sdesc(sV + (4 * kb + st) * 2048, 16384, 1024), id, (c > 0) || (kb > 0) || (st > 0));
+            mma_commit(bar_empty + gF % G::NSLOT);
+          }
+          if (!ok) break;
           mma_commit(bar_ds + t);
-          mma_commit(bar_empty + gF % G::NSLOT);
         }
         if (!ok) break;
         mma_commit(bar_nfull);
@@ -866,83 +902,182 @@ __global__ void __launch_bounds__(kThreadsV, 1)
     const int hrow = row - 64 * grp;                // feature row within the half
     bool ok = true;
     if (p.stall > 0) ok = epi_wait(bar_never, 0, abort_flag, p.dev_status, p.stall);
-    float den_acc = 0.f;                            // den partial of token gi (this group)
+    // denominators: this thread sums features 8a + fi (a = 0..7) of a half for
+    // the 8 tokens of chunk tcd; the 8 lanes fi of a quarter-warp then reduce
+    const int fi = lane & 7;
+    const int tcd = (((quad & 1) | (colh << 1)) << 2) | (lane >> 3);   // 0..15
+    float dacc[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) dacc[e] = 0.f;
+    uint32_t po[32];                               // o of my rows, previous chunk (fp16 pairs)
+    float pden = 0.f;
+#pragma unroll
+    for (int e = 0; e < 32; ++e) po[e] = 0u;
     const uint32_t peer = (uint32_t)(1 - fh);
-    for (int c = 0; ok && c < p.nc; ++c) {
-      const int g0 = c * G::NI;
-      // ---------------- per feature tile: S operand half, then the denominators
-      for (int t = 0; ok && t < G::NTC; ++t) {
-        const int k = c * G::NTC + t;
-        if (k > 0 && !(ok = grp_wait(grp, bar_sfree + grp, (k - 1) & 1, abort_flag, p.dev_status)))
-          break;
-        if (c > 0 && !(ok = grp_wait(grp, bar_ds + t, (c - 1) & 1, abort_flag, p.dev_status))) break;
-        tc_fence_after();
-        // this thread: feature hrow of half grp, value columns 64 colh .. 64 colh + 63
-        uint32_t a[2][32];
-        if (c > 0) {
-          tmem_ld32_async(lane_tm + 128 * t + 64 * colh, a[0]);
-          tmem_ld32_async(lane_tm + 128 * t + 64 * colh + 32, a[1]);
-          tmem_wait_ld(a[0]);
-          tmem_wait_ld(a[1]);
-        } else {
+    // out[row] of chunk cc from 64 fp32 numerators and 1/den (bf16); false if not finite
+    auto store_row = [&](int cc, const float* nm, float invd, float dd) -> bool {
+      uint32_t w[32];
+      bool bad = !isfinite(dd);
 #pragma unroll
-          for (int i = 0; i < 32; ++i) a[0][i] = a[1][i] = 0u;
+      for (int e = 0; e < 32; ++e) {
+        const float o0 = nm[2 * e] * invd, o1 = nm[2 * e + 1] * invd;
+        bad |= !isfinite(o0) || !isfinite(o1);
+        w[e] = pack_bf16(o0, o1);
+      }
+      uint4* dst = reinterpret_cast<uint4*>(p.out + (int64_t)b * p.ob + (int64_t)h * p.oh +
+                                            (int64_t)(cc * kC + row) * p.ol + 128 * vb + 64 * colh);
+#pragma unroll
+      for (int q4 = 0; q4 < 8; ++q4)
+        dst[q4] = make_uint4(w[4 * q4], w[4 * q4 + 1], w[4 * q4 + 2], w[4 * q4 + 3]);
+      return !bad;
+    };
+    // rows of chunk cc this CTA finishes: (den o + den' o') / (den + den') with
+    // o, den kept from that chunk and o', den' from the peer's buffer cc & 1
+    auto finish_prev = [&](int cc) -> bool {
+      const bool arrived = wait_cluster(bar_recv + (cc & 1), (cc >> 1) & 1, abort_flag, p.dev_status);
+      if (grp_sync_or(grp, !arrived)) return false;
+      const uint32_t xb = s0 + G::oX + (cc & 1) * G::kXB;
+      const uint32_t xr = xb + (uint32_t)(row & 63) * 256 + colh * 128;
+      const float dp = *reinterpret_cast<const float*>(sm + G::oX + (cc & 1) * G::kXB + 16384 +
+                                                       (row & 63) * 4);
+      float nm[64];
+#pragma unroll
+      for (int q4 = 0; q4 < 8; ++q4) {
+        const uint4 u = ld_shared_v4(xr + q4 * 16);
+        const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 of = __half22float2(*reinterpret_cast<const __half2*>(&w4[e]));
+          const float2 mf = __half22float2(*reinterpret_cast<const __half2*>(&po[4 * q4 + e]));
+          nm[8 * q4 + 2 * e] = fmaf(pden, mf.x, dp * of.x);
+          nm[8 * q4 + 2 * e + 1] = fmaf(pden, mf.y, dp * of.y);
         }
-        const uint32_t sS = s0 + G::oS + grp * 32768;
-        const uint32_t rowoff = (uint32_t)(hrow >> 3) * 1024 + (uint32_t)(hrow & 7) * 128;
+      }
+      // every reader of the group is done: expect the peer's chunk cc + 2 in this
+      // buffer and tell the peer it may send it
+      grp_sync_or(grp, false);
+      if (gi == 0) {
+        if (cc + 2 < p.nc) mbar_arrive_expect_tx(bar_recv + (cc & 1), G::kXBytes);
+        arrive_peer_relaxed(peer_addr(smem_u32(bar_rfree + (cc & 1)), peer));
+      }
+      const float dt = pden + dp;
+      if (cc * kC + row < p.L && !store_row(cc, nm, dt > 0.f ? 1.f / dt : 0.f, dt))
+        report(p.dev_status, DARK_ERR_NUMERIC);
+      return true;
+    };
+    // S operand half of feature tile t for chunk c (group grp's features)
+    auto conv = [&](int c, int t) -> bool {
+      const int k = c * G::NTC + t;
+      if (k > 0 && !(ok = grp_wait(grp, bar_sfree + grp, (k - 1) & 1, abort_flag, p.dev_status)))
+        return false;
+      if (c > 0 && !(ok = grp_wait(grp, bar_ds + t, (c - 1) & 1, abort_flag, p.dev_status))) return false;
+      tc_fence_after();
+      // this thread: feature hrow of half grp, value columns 64 colh .. 64 colh + 63
+      uint32_t a[2][32];
+      if (c > 0) {
+        tmem_ld32_async(lane_tm + 128 * t + 64 * colh, a[0]);
+        tmem_ld32_async(lane_tm + 128 * t + 64 * colh + 32, a[1]);
+        tmem_wait_ld(a[0]);
+        tmem_wait_ld(a[1]);
+      } else {
 #pragma unroll
-        for (int cg = 0; cg < 8; ++cg) {
-          uint32_t hi4[4], lo4[4];
+        for (int i = 0; i < 32; ++i) a[0][i] = a[1][i] = 0u;
+      }
+      const uint32_t sS = s0 + G::oS + grp * 32768;
+      const uint32_t rowoff = (uint32_t)(hrow >> 3) * 1024 + (uint32_t)(hrow & 7) * 128;
+#pragma unroll
+      for (int cg = 0; cg < 8; ++cg) {
+        uint32_t hi4[4], lo4[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int i = 8 * cg + 2 * e;
+          const float x0 = __uint_as_float(a[i >> 5][i & 31]);
+          const float x1 = __uint_as_float(a[(i + 1) >> 5][(i + 1) & 31]);
+          const __nv_bfloat162 hv = __floats2bfloat162_rn(x0, x1);
+          const float2 hf = __bfloat1622float2(hv);
+          hi4[e] = *reinterpret_cast<const uint32_t*>(&hv);
+          lo4[e] = pack_bf16(x0 - hf.x, x1 - hf.y);
+        }
+        const uint32_t off = rowoff + (uint32_t)((cg ^ (hrow & 7)) * 16);
+        st_shared_v4(sS + colh * 8192 + off, hi4[0], hi4[1], hi4[2], hi4[3]);          // hi block
+        st_shared_v4(sS + (2 + colh) * 8192 + off, lo4[0], lo4[1], lo4[2], lo4[3]);   // lo block
+      }
+      tc_fence_before();
+      fence_async_smem();
+      warp_arrive(bar_simg + grp);
+      return true;
+    };
+    // denominator partials from Psi_{t,grp} of chunk c, then z_<c+1 for the half
+    auto den_tile = [&](int c, int t) -> bool {
+      const int g0 = c * G::NI;
+      // ---- den partial of token gi over features 64 grp .. + 63 of tile t
+      const int gP = g0 + item_psi(t, grp);
+      if (!(ok = grp_wait(grp, bar_full + gP % G::NSLOT, (gP / G::NSLOT) & 1, abort_flag,
+                          p.dev_status)))
+        return false;
+      {
+        // Psi_{t,h}: token block tcd >> 3, rows = features of the half
+        const uint32_t psi = s0 + G::oR + (gP % G::NSLOT) * 16384 + (tcd >> 3) * 8192 +
+                             (uint32_t)fi * 128 + (uint32_t)(((tcd & 7) ^ fi) << 4);
+        const float* zt = zs + 128 * t + 64 * grp + fi;
+        float acc[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+#pragma unroll
+        for (int a8 = 0; a8 < 8; ++a8) {
+          const uint4 u = ld_shared_v4(psi + a8 * 1024);
+          const float zf = zt[8 * a8];
+          const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            const int i = 8 * cg + 2 * e;
-            const float x0 = __uint_as_float(a[i >> 5][i & 31]);
-            const float x1 = __uint_as_float(a[(i + 1) >> 5][(i + 1) & 31]);
-            const __nv_bfloat162 hv = __floats2bfloat162_rn(x0, x1);
-            const float2 hf = __bfloat1622float2(hv);
-            hi4[e] = *reinterpret_cast<const uint32_t*>(&hv);
-            lo4[e] = pack_bf16(x0 - hf.x, x1 - hf.y);
+            acc[2 * e] = fmaf(__uint_as_float(w4[e] << 16), zf, acc[2 * e]);
+            acc[2 * e + 1] = fmaf(__uint_as_float(w4[e] & 0xFFFF0000u), zf, acc[2 * e + 1]);
           }
-          const uint32_t off = rowoff + (uint32_t)((cg ^ (hrow & 7)) * 16);
-          st_shared_v4(sS + colh * 8192 + off, hi4[0], hi4[1], hi4[2], hi4[3]);          // hi block
-          st_shared_v4(sS + (2 + colh) * 8192 + off, lo4[0], lo4[1], lo4[2], lo4[3]);   // lo block
         }
-        tc_fence_before();
-        fence_async_smem();
-        warp_arrive(bar_simg + grp);
-        // ---- den partial of token gi over features 64 grp .. + 63 of tile t
-        const int gP = g0 + item_psi(t);
-        if (!(ok = grp_wait(grp, bar_full + gP % G::NSLOT, (gP / G::NSLOT) & 1, abort_flag,
-                            p.dev_status)))
-          break;
-        {
-          const uint8_t* psi = sm + G::oR + (gP % G::NSLOT) * 32768 + (gi >> 6) * 16384;
-          const float* zt = zs + 128 * t + 64 * grp;
-          const int tc8 = (gi & 63) >> 3, tin = gi & 7;
-          float acc = 0.f;
-#pragma unroll 8
-          for (int j = 0; j < 64; ++j) {
-            const int f = 64 * grp + j;
-            const __nv_bfloat16 v = *reinterpret_cast<const __nv_bfloat16*>(
-                psi + (f >> 3) * 1024 + (f & 7) * 128 + ((tc8 ^ (f & 7)) << 4) + tin * 2);
-            acc = fmaf(__bfloat162float(v), zt[j], acc);
-          }
-          den_acc += acc;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          float x = acc[e];
+          x += __shfl_xor_sync(0xffffffffu, x, 1);
+          x += __shfl_xor_sync(0xffffffffu, x, 2);
+          x += __shfl_xor_sync(0xffffffffu, x, 4);
+          dacc[e] += x;
         }
-        // z_<c+1 = z_<c + dz_c for these 64 features, once every thread has read
-        // them and the chunk's small items have arrived
-        if (!(ok = grp_wait(grp, bar_v, c & 1, abort_flag, p.dev_status))) break;
-        if (gi < 64) {
-          const float* dz = (const float*)(sm + G::oSm + (c & 1) * G::kSmB);
-          zs[128 * t + 64 * grp + gi] += dz[128 * t + 64 * grp + gi];
-        }
-        warp_arrive(bar_den + t);
       }
-      if (!ok) break;
-      // ---------------- output of chunk c
-      den_part[((c & 1) * 2 + grp) * 128 + gi] = den_acc;
-      den_acc = 0.f;
-      if (!(ok = epi_wait(bar_nfull, c & 1, abort_flag, p.dev_status))) break;
+      // z_<c+1 = z_<c + dz_c for these 64 features, once every thread has read
+      // them and the chunk's small items have arrived
+      if (!(ok = grp_wait(grp, bar_v, c & 1, abort_flag, p.dev_status))) return false;
+      if (gi < 64) {
+        const float* dz = (const float*)(sm + G::oSm + (c & 1) * G::kSmB);
+        zs[128 * t + 64 * grp + gi] += dz[128 * t + 64 * grp + gi];
+      }
+      warp_arrive(bar_den + 2 * t + grp);
+      return true;
+    };
+    // this chunk's denominator partials, for the rows of the output phase (read
+    // by other threads after the agreement at the top of the chunk)
+    auto put_den = [&](int c) {
+      if (fi == 0) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) den_part[((c & 1) * 2 + grp) * 128 + 8 * tcd + e] = dacc[e];
+      }
+#pragma unroll
+      for (int e = 0; e < 8; ++e) dacc[e] = 0.f;
+    };
+    for (int t = 0; ok && t < G::NTC; ++t) ok = conv(0, t) && den_tile(0, t);
+    put_den(0);
+    // Every epilogue thread passes the agreement at the top of each chunk (the
+    // only point where both groups wait together); a failure inside a chunk
+    // skips to it, so that the groups always leave the loop together.
+    for (int c = 0; c < p.nc; ++c) {
+      if (epi_sync_or(!ok)) {
+        ok = false;
+        break;
+      }
+      // ---------------- output of chunk c, part 1: numerators and denominators
+      if (!wait_one(bar_nfull, c & 1, abort_flag, p.dev_status)) {
+        ok = false;
+        continue;
+      }
       tc_fence_after();
       float num[64];
       {
@@ -966,69 +1101,56 @@ __global__ void __launch_bounds__(kThreadsV, 1)
       const float den = den_part[((c & 1) * 2 + 0) * 128 + row] +
                         den_part[((c & 1) * 2 + 1) * 128 + row] + da[row] +
                         (G::FS == 1 ? da[128 + row] : 0.f);
-      const int tok = c * kC + row;
-      if (G::FS == 1 || (row >> 6) == fh) {
-        // a row this CTA finishes
-        float dp = 0.f;
-        uint32_t op[32];
-        if (G::FS == 2) {
-          if (!(ok = wait_cluster(bar_recv, c & 1, abort_flag, p.dev_status))) break;
-          const uint32_t xr = s0 + G::oX + (uint32_t)(row & 63) * 256 + colh * 128;
-#pragma unroll
-          for (int q4 = 0; q4 < 8; ++q4) {
-            const uint4 u = ld_shared_v4(xr + q4 * 16);
-            op[4 * q4] = u.x;
-            op[4 * q4 + 1] = u.y;
-            op[4 * q4 + 2] = u.z;
-            op[4 * q4 + 3] = u.w;
-          }
-          dp = ((const float*)(sm + G::oX + 16384))[row & 63];
-        }
-        const float dt = den + dp;
-        if (tok < p.L) {
-          const float inv = dt > 0.f ? 1.f / dt : 0.f;
-          uint32_t w[32];
-          bool bad = !isfinite(dt);
-#pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            float o0 = num[2 * e], o1 = num[2 * e + 1];
-            if (G::FS == 2) {
-              const float2 of = __half22float2(*reinterpret_cast<const __half2*>(&op[e]));
-              o0 = fmaf(dp, of.x, o0);
-              o1 = fmaf(dp, of.y, o1);
-            }
-            o0 *= inv;
-            o1 *= inv;
-            bad |= !isfinite(o0) || !isfinite(o1);
-            w[e] = pack_bf16(o0, o1);
-          }
-          if (bad) report(p.dev_status, DARK_ERR_NUMERIC);
-          uint4* dst = reinterpret_cast<uint4*>(p.out + (int64_t)b * p.ob + (int64_t)h * p.oh +
-                                                (int64_t)tok * p.ol + 128 * vb + 64 * colh);
-#pragma unroll
-          for (int q4 = 0; q4 < 8; ++q4)
-            dst[q4] = make_uint4(w[4 * q4], w[4 * q4 + 1], w[4 * q4 + 2], w[4 * q4 + 3]);
-        }
-        if (G::FS == 2) arrive_peer(peer_addr(smem_u32(bar_rfree), peer));
+      const float inv = den > 0.f ? 1.f / den : 0.f;
+      uint32_t o[32];
+      if (G::FS == 1) {
+        if (c * kC + row < p.L && !store_row(c, num, inv, den)) report(p.dev_status, DARK_ERR_NUMERIC);
       } else {
-        // a row the peer finishes: send num/den (fp16) and den
-        if (c > 0 && !(ok = wait_cluster(bar_rfree, (c - 1) & 1, abort_flag, p.dev_status))) break;
-        const float inv = den > 0.f ? 1.f / den : 0.f;
-        uint32_t w[32];
 #pragma unroll
         for (int e = 0; e < 32; ++e) {
           const __half2 hv = __floats2half2_rn(num[2 * e] * inv, num[2 * e + 1] * inv);
-          w[e] = *reinterpret_cast<const uint32_t*>(&hv);
+          o[e] = *reinterpret_cast<const uint32_t*>(&hv);
         }
-        const uint32_t xr = peer_addr(s0 + G::oX + (uint32_t)(row & 63) * 256 + colh * 128, peer);
+      }
+      // the next chunk's S operands and denominators, so that its MMAs start now
+      if (c + 1 < p.nc) {
+        for (int t = 0; ok && t < G::NTC; ++t) ok = conv(c + 1, t) && den_tile(c + 1, t);
+        if (!ok) continue;
+        put_den(c + 1);
+      }
+      // ---------------- output of chunk c, part 2: the exchange between the halves
+      if (G::FS == 2) {
+        if ((row >> 6) == fh) {
+          // a row this CTA finishes: chunk c - 1's, whose other half has arrived
+          // by now; this chunk's part waits in registers until the next chunk
+          if (c > 0 && !(ok = finish_prev(c - 1))) continue;
 #pragma unroll
-        for (int q4 = 0; q4 < 8; ++q4)
-          st_peer_v4(xr + q4 * 16, w[4 * q4], w[4 * q4 + 1], w[4 * q4 + 2], w[4 * q4 + 3]);
-        if (colh == 0) st_peer_f32(peer_addr(s0 + G::oX + 16384 + (uint32_t)(row & 63) * 4, peer), den);
-        arrive_peer(peer_addr(smem_u32(bar_recv), peer));
+          for (int e = 0; e < 32; ++e) po[e] = o[e];
+          pden = den;
+        } else {
+          // a row the peer finishes: num/den (fp16) and den into its buffer c & 1,
+          // once it has consumed what the buffer held (chunk c - 2)
+          if (c > 1) {
+            const bool freed = wait_cluster(bar_rfree + (c & 1), ((c >> 1) - 1) & 1, abort_flag,
+                                            p.dev_status);
+            if (grp_sync_or(grp, !freed)) {
+              ok = false;
+              continue;
+            }
+          }
+          const uint32_t xb = s0 + G::oX + (c & 1) * G::kXB;
+          const uint32_t xr = peer_addr(xb + (uint32_t)(row & 63) * 256 + colh * 128, peer);
+          const uint32_t rb = peer_addr(smem_u32(bar_recv + (c & 1)), peer);
+#pragma unroll
+          for (int q4 = 0; q4 < 8; ++q4)
+            st_async_v4(xr + q4 * 16, o[4 * q4], o[4 * q4 + 1], o[4 * q4 + 2], o[4 * q4 + 3], rb);
+          if (colh == 0) st_async_f32(peer_addr(xb + 16384 + (uint32_t)(row & 63) * 4, peer), den, rb);
+        }
       }
       warp_arrive(bar_smfree + (c & 1));
     }
+    if (ok && G::FS == 2 && (row >> 6) == fh && p.nc > 0) ok = finish_prev(p.nc - 1);
+    ok = !epi_sync_or(!ok);
     // final state: S_t (my features x my 128 value columns) and z (first value block)
     if (ok && p.st_kv != nullptr) {
       for (int t = 0; ok && t < G::NTC; ++t)
