@@ -148,3 +148,33 @@ def test_decode_staged_projection_small_m(D, cuda_ok):
     ref = _oracle_decode(inp, stream, 4)
     for g, r_ in zip(got, ref):
         check(w, g[:, :, None], r_[:, :, None])
+
+
+@pytest.mark.parametrize("per_head", [True, False], ids=["per-head-geometry", "shared-geometry"])
+def test_decode_many_heads(D, cuda_ok, per_head):
+    # More heads than twice the SM count: the streaming path (one block per SM
+    # walking heads in projection order, state copied through shared memory),
+    # with invalid tokens in some batch rows and heads of one projection row
+    # spread over several blocks
+    w = synth.WORKLOADS[5].with_sizes(B=41, H=8, L=130, per_head_geom=per_head)
+    inp = synth.make_inputs(w)
+    steps = 3
+    stream = synth.decode_stream(w, steps)
+    rng = np.random.default_rng(5)
+    valid = (rng.random((steps, w.B)) > 0.2).astype(np.uint8)
+    got, res = _decode_run(D, cuda_ok, w, inp, stream, steps, valid=valid)
+    ref = _oracle_decode(inp, stream, steps, valid=valid)
+    for g, r in zip(got, ref):
+        check(w, g[:, :, None], r[:, :, None])
+    # the state after the steps: the oracle's recurrence over prefill and steps
+    _, kv, z = O.attention(inp["q"], inp["k"], inp["v"], inp["omega"], inp["geom"],
+                           key_mask=inp["mask"], causal=True)
+    for t in range(steps):
+        _, kv, z = O.decode_step(kv, z, stream["q"][t], stream["k"][t], stream["v"][t],
+                                 inp["omega"], inp["geom"], valid=valid[t])
+    kv_g = res["state_tensors"][0].double().cpu().numpy()
+    z_g = res["state_tensors"][1].double().cpu().numpy()
+    for got_s, ref_s in ((kv_g, kv), (z_g, z)):
+        scale = np.abs(ref_s).reshape(w.B, w.H, -1).max(axis=2)
+        err = np.abs(got_s - ref_s).reshape(w.B, w.H, -1).max(axis=2) / scale
+        assert err.max() <= 2e-2, err.max()
