@@ -746,10 +746,13 @@ def exact_flops(w: synth.Workload) -> float:
 
 
 BWD_METRIC = ("DARK attention bwd tokens/s (B·H·L/s, dq dk dv dM) on 1 B200; "
-              "% of FP32-FFMA roofline")
-# fp32 FFMA peak: 148 SMs x 128 lanes x 2 FLOP x 1.965 GHz (the backward kernels
-# are SIMT fp32 throughout)
+              "% of TF32-tensor roofline (bf16 I/O) or FP32-FFMA (fp32 I/O)")
+# fp32 FFMA peak: 148 SMs x 128 lanes x 2 FLOP x 1.965 GHz (the fp32-I/O backward
+# kernels are SIMT fp32 throughout)
 FFMA_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
+# dense tf32 / bf16 tensor throughput, nominal (1.1 and 2.25 PFLOP/s): the tf32
+# peak is the measured bf16 peak times this ratio
+TF32_OVER_BF16 = 1.1 / 2.25
 
 
 def bwd_flops(w: synth.Workload) -> float:
@@ -854,10 +857,18 @@ def run_backward(args, w: synth.Workload, rank: int, world: int, dev) -> dict | 
     t = ms_per_step / 1e3
     flops = bwd_flops(w)
     peaks = load_peaks()
-    roof = dict(bound="alu", achieved=flops / t / 1e12, peak=FFMA_TFLOPS, unit="TFLOP/s",
-                frac=flops / t / 1e12 / FFMA_TFLOPS, traffic=None,
-                peak_source="derived: 148 SMs x 128 FP32 lanes x 2 x 1.965 GHz",
-                kernel="backward call (SIMT fp32)")
+    if any("tbf_" in n for n in kernel_names):
+        tf32 = peaks["bf16"] * TF32_OVER_BF16
+        roof = dict(bound="tensor", achieved=flops / t / 1e12, peak=tf32, unit="TFLOP/s",
+                    frac=flops / t / 1e12 / tf32, traffic=None,
+                    peak_source=f"{peaks['source']} bf16 x {TF32_OVER_BF16:.3f} "
+                                "(nominal dense tf32 / bf16)",
+                    kernel="backward call (tcgen05 kind::tf32)")
+    else:
+        roof = dict(bound="alu", achieved=flops / t / 1e12, peak=FFMA_TFLOPS, unit="TFLOP/s",
+                    frac=flops / t / 1e12 / FFMA_TFLOPS, traffic=None,
+                    peak_source="derived: 148 SMs x 128 FP32 lanes x 2 x 1.965 GHz",
+                    kernel="backward call (SIMT fp32)")
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
         from oracle import dark_oracle as O
@@ -973,17 +984,37 @@ def run_reference(args, w: synth.Workload) -> dict:
     }
 
 
+def decode_in_child(args) -> dict:
+    """The decode line attached to a one-GPU forward run, measured by a fresh
+    process (`bench.py --decode`): the CUDA profiler that counts launches
+    records kernels in the first session of a process only."""
+    import subprocess
+    cmd = [sys.executable, os.path.abspath(__file__), "--decode", "--steps", str(args.steps),
+           "--warmup", str(args.warmup)]
+    cmd += ["--no-cpu-baseline"] if args.no_cpu_baseline else []
+    cmd += ["--no-profile"] if args.no_profile else []
+    env = {k: v for k, v in os.environ.items() if k not in ("WORLD_SIZE", "RANK", "LOCAL_RANK")}
+    p = subprocess.run(cmd, capture_output=True, text=True, timeout=900, env=env)
+    lines = [ln for ln in p.stdout.splitlines() if ln.startswith("{")]
+    if p.returncode != 0 or not lines:
+        raise RuntimeError(f"decode run failed (rc {p.returncode}): {p.stderr[-2000:]}")
+    return json.loads(lines[-1])
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["native", "reference"], default="native")
-    ap.add_argument("--workload", type=int, default=4, help="synthetic workload recipe (1-5)")
+    ap.add_argument("--workload", type=int, default=None,
+                    help="synthetic workload recipe (1-5); default 4 for the forward, 2 for "
+                         "--backward and --exact")
     ap.add_argument("--ref-seconds", type=float, default=None,
                     help="CPU seconds per reference step (default: about 120 s over all steps)")
     ap.add_argument("--no-decode", action="store_true",
-                    help="leave the decode step out of the forward run's JSON line")
+                    help="leave the decode step out of the forward run's JSON line (it is "
+                         "attached to one-GPU runs only)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-profile", action="store_true",
                     help="do not count launches with the CUDA profiler (for runs under ncu)")
@@ -1003,6 +1034,8 @@ def main():
     args.warmup = max(args.warmup, 3)
     if args.ref_seconds is None:
         args.ref_seconds = max(1.0, min(10.0, 120.0 / max(args.steps + args.warmup, 1)))
+    if args.workload is None:
+        args.workload = 2 if (args.backward or args.exact) else 4
     w = synth.WORKLOADS[args.workload]
 
     if "WORLD_SIZE" not in os.environ and args.gpus > 1:
@@ -1039,10 +1072,8 @@ def main():
             res = run_sample(args, rank, world, dev)
         else:
             res = run_native(args, w, rank, world, dev)
-            if not (args.no_decode or args.ncu or args.exact):
-                dec = run_decode(args, rank, world, dev)
-                if res is not None:
-                    res["decode"] = dec
+            if not (args.no_decode or args.ncu or args.exact) and world == 1:
+                res["decode"] = decode_in_child(args)
         if res is not None:
             print(json.dumps(res), flush=True)
     finally:

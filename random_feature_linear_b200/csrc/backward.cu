@@ -793,11 +793,35 @@ cudaError_t backward_t(const BwdArgs& a) {
 }  // namespace
 
 size_t bwd_workspace_bytes(int B, int H, int L, int m, int r, int d, int heads_w) {
-  return bwd_layout(B, H, L, m, r, d, heads_w).total;
+  const size_t simt = bwd_layout(B, H, L, m, r, d, heads_w).total;
+  const size_t tc = tc_bwd_workspace_bytes(B, H, L, m, r, d, heads_w);
+  return simt > tc ? simt : tc;
 }
 
 cudaError_t launch_backward(const BwdArgs& a) {
+  if (tc_backward_supported(a)) return launch_backward_tc(a);
   return a.dtype == DARK_BF16 ? backward_t<__nv_bfloat16>(a) : backward_t<float>(a);
+}
+
+// Steps shared with the tensor-core backward (tc_backward.cu).
+cudaError_t bwd_fill_ordered(int* p, int n, float v, cudaStream_t s) {
+  fill_ordered_kernel<<<(n + 255) / 256, 256, 0, s>>>(p, n, v);
+  return cudaGetLastError();
+}
+cudaError_t bwd_shift_keys(float* phik, const int* ck, int L, int m, size_t n, cudaStream_t s) {
+  bwd_shift_keys_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(phik, ck, L, m, n);
+  return cudaGetLastError();
+}
+cudaError_t bwd_tile_scan(float* st, int n, int nt, int bh, int mode, cudaStream_t s) {
+  tile_scan_kernel<<<dim3((n + 255) / 256, bh), 256, 0, s>>>(st, n, nt, mode);
+  return cudaGetLastError();
+}
+cudaError_t bwd_dgeom(const float* G, const BwdArgs& a) {
+  const double sc = pow((double)a.d, -0.25);
+  dgeom_kernel<<<dim3(a.r, a.heads_geom), 128, 0, a.stream>>>(
+      G, a.omega, a.heads_omega, a.heads_geom, a.heads_w, a.m, a.r, a.d, (float)(sc * kLog2e),
+      (float)(sc * sqrt(0.5 * kLog2e)), a.dgeom);
+  return cudaGetLastError();
 }
 
 }  // namespace dark

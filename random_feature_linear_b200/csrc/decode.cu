@@ -237,47 +237,6 @@ __device__ __forceinline__ float feature_gemv_shared(const TW* w_sm, int m, int 
   return nrm;
 }
 
-// The feature GEMV on staged fp16 W' rows (d a multiple of 8): one thread per
-// row, the row's chunks of 8 columns visited from a per-row rotation so that
-// the threads of a warp read different banks; no shuffles. Returns this
-// thread's share of sum_i (W'_{m+i} k)^2 (the key norm).
-__device__ __forceinline__ float feature_gemv_rows(const __half* w_sm, int m, int r, int d,
-                                                   const float* xk, const float* xq, float* pk,
-                                                   float* pq, int nthreads) {
-  const int nch = d / 8;
-  float nrm = 0.f;
-  for (int j = threadIdx.x; j < m + r; j += nthreads) {
-    const uint4* wr = reinterpret_cast<const uint4*>(w_sm + (size_t)j * d);
-    float ak = 0.f, aq = 0.f;
-    const bool want_q = j < m;
-#pragma unroll 4
-    for (int cc = 0; cc < nch; ++cc) {
-      int c = cc + j;
-      c -= (c / nch) * nch;
-      const uint4 u = wr[c];
-      const __half2* hp = reinterpret_cast<const __half2*>(&u);
-      const float4 k0 = *reinterpret_cast<const float4*>(xk + 8 * c);
-      const float4 k1 = *reinterpret_cast<const float4*>(xk + 8 * c + 4);
-      const float2 w0 = __half22float2(hp[0]), w1 = __half22float2(hp[1]);
-      const float2 w2 = __half22float2(hp[2]), w3 = __half22float2(hp[3]);
-      ak = fmaf(w0.x, k0.x, ak); ak = fmaf(w0.y, k0.y, ak); ak = fmaf(w1.x, k0.z, ak);
-      ak = fmaf(w1.y, k0.w, ak); ak = fmaf(w2.x, k1.x, ak); ak = fmaf(w2.y, k1.y, ak);
-      ak = fmaf(w3.x, k1.z, ak); ak = fmaf(w3.y, k1.w, ak);
-      if (want_q) {
-        const float4 q0 = *reinterpret_cast<const float4*>(xq + 8 * c);
-        const float4 q1 = *reinterpret_cast<const float4*>(xq + 8 * c + 4);
-        aq = fmaf(w0.x, q0.x, aq); aq = fmaf(w0.y, q0.y, aq); aq = fmaf(w1.x, q0.z, aq);
-        aq = fmaf(w1.y, q0.w, aq); aq = fmaf(w2.x, q1.x, aq); aq = fmaf(w2.y, q1.y, aq);
-        aq = fmaf(w3.x, q1.z, aq); aq = fmaf(w3.y, q1.w, aq);
-      }
-    }
-    pk[j] = ak;
-    if (want_q) pq[j] = aq;
-    else nrm = fmaf(ak, ak, nrm);
-  }
-  return nrm;
-}
-
 template <typename T>
 __global__ void __launch_bounds__(kThreads, 2) decode_kernel(
     const typename WeightOf<T>::type* __restrict__ w, int heads_w, int m, int r, int d,
@@ -364,12 +323,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(
   float ks, qs;
   if (stage_w && !stab) {
     // GEMV on the staged rows; the key norm from per-warp partial sums
-    float part;
-    if constexpr (sizeof(TW) == 2)
-      part = warp_sum(feature_gemv_rows(reinterpret_cast<const __half*>(w_sm), m, r, d, xk, xq, pk,
-                                        pq, kThreads));
-    else
-      part = warp_sum(feature_gemv_shared(w_sm, m, r, d, xk, xq, pk, pq));
+    const float part = warp_sum(feature_gemv_shared(w_sm, m, r, d, xk, xq, pk, pq));
     if (lane == 0) scratch[2 + warp] = part;
     __syncthreads();
     float nrm = 0.f;
@@ -462,237 +416,9 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(
 }
 
 
-// ---------------------------------------------------------------------------
-// Streaming decode step for many heads (the common case: bf16 tokens, fp16
-// W', no stabiliser). The step reads and writes every head's fp32 state once,
-// so it is bound by HBM bandwidth if enough state is in flight. One persistent
-// block per SM walks a contiguous range of heads in projection order (item
-// i -> head i / B, batch i % B, so that consecutive items share W'); each
-// head's state [kv | z] is copied into one of two shared-memory buffers with a
-// single bulk copy (the next head's copy is in flight while this one is
-// updated), updated in place, and copied back with a bulk store. W' of the
-// current projection head is staged once, with the next one prefetched into a
-// second buffer when the head changes.
-constexpr int kStreamThreads = 256;
-
-struct StreamLayout {
-  uint32_t state, wbytes, oS, oW, oV, total;
-};
-__host__ __device__ inline StreamLayout stream_layout(int m, int r, int d) {
-  StreamLayout L;
-  L.state = (uint32_t)m * (d + 1) * 4;                       // [kv (m x d) | z (m)] fp32
-  L.wbytes = (uint32_t)(m + r) * d * 2;                      // fp16 W' of one head
-  L.oS = 0;
-  L.oW = (2 * L.state + 127) / 128 * 128;
-  L.oV = L.oW + (2 * L.wbytes + 127) / 128 * 128;
-  const int rpp = kStreamThreads / (d / 4);
-  // xq, xk, xv [d]; pk [m + r]; pq [m]; red [rpp][d]; scratch [40]; 4 barriers
-  L.total = L.oV + (uint32_t)(3 * d + (m + r) + m + rpp * d + 40) * 4 + 64;
-  return L;
-}
-
-__global__ void __launch_bounds__(kStreamThreads, 1) decode_stream_kernel(
-    const __half* __restrict__ w, int heads_w, int m, int r, int d, float* __restrict__ kv,
-    float* __restrict__ z, int B, int H, const __nv_bfloat16* __restrict__ q,
-    const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ v,
-    __nv_bfloat16* __restrict__ out, const uint8_t* __restrict__ valid, int* dev_status, int nitems) {
-  extern __shared__ __align__(128) uint8_t smem[];
-  const StreamLayout L = stream_layout(m, r, d);
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int tpr = d / 4, rpp = kStreamThreads / tpr;
-  float* xq = reinterpret_cast<float*>(smem + L.oV);
-  float* xk = xq + d;
-  float* xv = xk + d;
-  float* pk = xv + d;                     // [m + r]
-  float* pq = pk + m + r;                 // [m]
-  float* red = pq + m;                    // [rpp][d]
-  float* scratch = red + rpp * d;         // [40]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(
-      smem + ((L.oV + (uint32_t)(3 * d + (m + r) + m + rpp * d + 40) * 4 + 15) / 16 * 16));
-  uint64_t* bar_s = bars;                 // [2] state buffer loaded
-  uint64_t* bar_w = bars + 2;             // [2] W' buffer loaded
-  const int per = nitems / gridDim.x, extra = nitems % gridDim.x;
-  const int it0 = blockIdx.x * per + (blockIdx.x < extra ? blockIdx.x : extra);
-  const int nit = per + (blockIdx.x < extra ? 1 : 0);
-  auto head_of = [&](int i) { return i / B; };
-  auto bh_of = [&](int i) { return (i % B) * H + i / B; };
-  auto whead = [&](int h) -> const __half* {
-    return w + (size_t)(heads_w == 1 ? 0 : h) * (m + r) * d;
-  };
-  // bulk copy of item j's state into buffer j & 1 / of W' for head h into buffer sel
-  auto load_state = [&](int j) {
-    const int bh = bh_of(it0 + j);
-    uint64_t* bar = bar_s + (j & 1);
-    uint8_t* dst = smem + L.oS + (j & 1) * L.state;
-    const uint32_t kvb = (uint32_t)m * d * 4;
-    tc::mbar_arrive_expect_tx(bar, L.state);
-    for (uint32_t o = 0; o < kvb; o += 32768)
-      tc::bulk_load(dst + o, reinterpret_cast<const uint8_t*>(kv + (size_t)bh * m * d) + o,
-                    kvb - o < 32768 ? kvb - o : 32768, bar);
-    tc::bulk_load(dst + kvb, z + (size_t)bh * m, (uint32_t)m * 4, bar);
-  };
-  auto load_w = [&](int h, int sel) {
-    const uint8_t* src = reinterpret_cast<const uint8_t*>(whead(h));
-    tc::mbar_arrive_expect_tx(bar_w + sel, L.wbytes);
-    for (uint32_t o = 0; o < L.wbytes; o += 32768)
-      tc::bulk_load(smem + L.oW + sel * L.wbytes + o, src + o,
-                    L.wbytes - o < 32768 ? L.wbytes - o : 32768, bar_w + sel);
-  };
-  if (tid == 0) {
-    for (int i = 0; i < 4; ++i) tc::mbar_init(bars + i, 1);
-    tc::fence_mbar_init();
-    if (nit > 0) {
-      load_w(head_of(it0), 0);
-      load_state(0);
-      if (nit > 1) load_state(1);
-    }
-  }
-  __syncthreads();
-  int wsel = 0, wphase[2] = {0, 0};
-  int s_last[2] = {nit > 0 ? 0 : -1, nit > 1 ? 1 : -1};   // last item loaded into each buffer
-  int w_loads[2] = {nit > 0 ? 1 : 0, 0};                    // W' loads issued per buffer
-  bool ok = true;
-  for (int j = 0; j < nit && ok; ++j) {
-    const int i = it0 + j, h = head_of(i), bh = bh_of(i), b = i % B;
-    float* st = reinterpret_cast<float*>(smem + L.oS + (j & 1) * L.state);
-    float* zs = st + (size_t)m * d;
-    if (j > 0 && h != head_of(i - 1)) wsel ^= 1;
-    const __half* w_sm = reinterpret_cast<const __half*>(smem + L.oW + wsel * L.wbytes);
-    if (tid < d) {
-      xq[tid] = __bfloat162float(q[(size_t)bh * d + tid]);
-      xk[tid] = __bfloat162float(k[(size_t)bh * d + tid]);
-      xv[tid] = __bfloat162float(v[(size_t)bh * d + tid]);
-    }
-    // W' of this head: wait for its load when the head changes
-    const bool new_w = j == 0 || h != head_of(i - 1);
-    bool w_ok = true;
-    if (new_w) {
-      w_ok = tc::mbar_wait(bar_w + wsel, wphase[wsel] & 1);
-      wphase[wsel] ^= 1;            // the next load into this buffer completes the next phase
-    }
-    if (__syncthreads_or(w_ok ? 0 : 1)) {
-      ok = false;
-      break;
-    }
-    // feature exponents and the key norm (one thread per W' row)
-    const float part = warp_sum(feature_gemv_rows(w_sm, m, r, d, xk, xq, pk, pq, kStreamThreads));
-    if (lane == 0) scratch[8 + warp] = part;
-    // the buffers of item j - 1 (state) and of the next head's W' are free now:
-    // prefetch item j + 1's state once the store of item j - 1 has read it
-    if (tid == 0) {
-      if (j + 1 < nit && j >= 1) {
-        asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
-        load_state(j + 1);
-        s_last[(j + 1) & 1] = j + 1;
-      }
-      if (j + 1 < nit && head_of(i + 1) != h) {
-        load_w(head_of(i + 1), wsel ^ 1);
-        ++w_loads[wsel ^ 1];
-      }
-    }
-    __syncthreads();
-    float nrm = 0.f;
-#pragma unroll
-    for (int u = 0; u < kStreamThreads / 32; ++u) nrm += scratch[8 + u];
-    const float ks = nrm + 0.5f * log2f((float)m);
-    const bool upd = valid == nullptr || valid[b] != 0;
-    for (int jj = tid; jj < m; jj += kStreamThreads) {
-      pk[jj] = upd ? exp2f(pk[jj] - ks) : 0.f;
-      pq[jj] = exp2f(pq[jj]);
-    }
-    // this item's state
-    const bool s_ok = tc::mbar_wait(bar_s + (j & 1), (j >> 1) & 1);
-    if (__syncthreads_or(s_ok ? 0 : 1)) {
-      ok = false;
-      break;
-    }
-    // kv' = kv + phi(k) v^T and num = phi(q)^T kv', in place, one float4 column
-    // group per thread
-    const int c4 = tid % tpr, r0 = tid / tpr;
-    float4 num = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (r0 < rpp) {
-      const float4 vv = make_float4(xv[4 * c4], xv[4 * c4 + 1], xv[4 * c4 + 2], xv[4 * c4 + 3]);
-      float4* s4 = reinterpret_cast<float4*>(st) + c4;
-#pragma unroll 4
-      for (int row = r0; row < m; row += rpp) {
-        float4 x = s4[(size_t)row * tpr];
-        const float fk = pk[row], fq = pq[row];
-        x.x = fmaf(fk, vv.x, x.x); x.y = fmaf(fk, vv.y, x.y);
-        x.z = fmaf(fk, vv.z, x.z); x.w = fmaf(fk, vv.w, x.w);
-        s4[(size_t)row * tpr] = x;
-        num.x = fmaf(fq, x.x, num.x); num.y = fmaf(fq, x.y, num.y);
-        num.z = fmaf(fq, x.z, num.z); num.w = fmaf(fq, x.w, num.w);
-      }
-      float* rr = red + r0 * d + 4 * c4;
-      rr[0] = num.x; rr[1] = num.y; rr[2] = num.z; rr[3] = num.w;
-    }
-    float den = 0.f;
-    for (int jj = tid; jj < m; jj += kStreamThreads) {
-      const float zj = zs[jj] + pk[jj];
-      zs[jj] = zj;
-      den = fmaf(pq[jj], zj, den);
-    }
-    den = warp_sum(den);
-    if (lane == 0) scratch[warp] = den;
-    tc::fence_async_smem();           // the state writes above, for the bulk store
-    __syncthreads();
-    if (tid == 0) {
-      const uint32_t kvb = (uint32_t)m * d * 4;
-      const uint32_t src = tc::smem_u32(st);
-      for (uint32_t o = 0; o < kvb; o += 32768)
-        asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(
-                         reinterpret_cast<uint8_t*>(kv + (size_t)bh * m * d) + o),
-                     "r"(src + o), "r"(kvb - o < 32768 ? kvb - o : 32768)
-                     : "memory");
-      asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(
-                       z + (size_t)bh * m),
-                   "r"(src + kvb), "r"((uint32_t)m * 4)
-                   : "memory");
-      asm volatile("cp.async.bulk.commit_group;" ::: "memory");
-    }
-    float dtot = 0.f;
-#pragma unroll
-    for (int u = 0; u < kStreamThreads / 32; ++u) dtot += scratch[u];
-    for (int c = tid; c < d; c += kStreamThreads) {
-      float acc = 0.f;
-      for (int g = 0; g < rpp; ++g) acc += red[g * d + c];
-      const float o = dtot > 0.f ? acc / dtot : 0.f;
-      if (!isfinite(o)) report(dev_status, DARK_ERR_NUMERIC);
-      out[(size_t)bh * d + c] = __float2bfloat16_rn(o);
-    }
-    __syncthreads();                   // red, scratch and pk/pq are reused by the next item
-  }
-  if (!ok && tid == 0) {
-    report(dev_status, DARK_ERR_TIMEOUT);
-    // no copy may land after the block is gone (a completed phase passes at once)
-    for (int bb = 0; bb < 2; ++bb) {
-      if (s_last[bb] >= 0) tc::mbar_wait(bar_s + bb, (s_last[bb] >> 1) & 1);
-      if (w_loads[bb] > 0) tc::mbar_wait(bar_w + bb, (w_loads[bb] - 1) & 1);
-    }
-  }
-  if (tid == 0) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
-}
 }  // namespace
 
 cudaError_t launch_decode(const DecodeArgs& a) {
-  // the streaming kernel when the heads outnumber the SMs and two states and
-  // two W' copies fit in shared memory
-  if (a.dtype == DARK_BF16 && a.shift == nullptr && a.update == 1 && a.d % 8 == 0 && a.d <= 256 &&
-      a.m % 4 == 0 && a.B * a.H >= 2 * num_sms() && ((uintptr_t)a.w & 15) == 0 &&
-      ((uintptr_t)a.kv & 15) == 0 && ((uintptr_t)a.z & 15) == 0) {
-    const StreamLayout L = stream_layout(a.m, a.r, a.d);
-    if (L.total <= 227 * 1024 && L.wbytes % 16 == 0 && (a.m * 4) % 16 == 0) {
-      static int done[64];
-      cudaError_t err = set_smem_limit_once((const void*)decode_stream_kernel, (int)L.total, done);
-      if (err != cudaSuccess) return err;
-      const int n = a.B * a.H, grid = n < num_sms() ? n : num_sms();
-      decode_stream_kernel<<<grid, kStreamThreads, L.total, a.stream>>>(
-          (const __half*)a.w, a.heads_w, a.m, a.r, a.d, a.kv, a.z, a.B, a.H,
-          (const __nv_bfloat16*)a.q, (const __nv_bfloat16*)a.k, (const __nv_bfloat16*)a.v,
-          (__nv_bfloat16*)a.out, a.valid, a.dev_status, n);
-      return cudaGetLastError();
-    }
-  }
   const int tpr = a.d / 4;
   const int rpp = kThreads / tpr;
   const size_t welt = a.dtype == DARK_BF16 ? sizeof(__half) : sizeof(float);

@@ -80,7 +80,8 @@ bool tc_make_maps(FwdArgs& a);
 long long test_stall_cycles();
 // Streaming multiprocessors of the current device (looked up once per device).
 int num_sms();
-// Sets a kernel's dynamic shared memory limit once per device.
+// Raises a kernel's dynamic shared memory limit to `bytes` on the current device
+// when it is below (done_per_device keeps the size set so far per device).
 cudaError_t set_smem_limit_once(const void* kernel, int bytes, int* done_per_device);
 
 bool tc_causal_supported(FwdArgs& a);
@@ -141,6 +142,15 @@ struct BwdArgs {
 };
 size_t bwd_workspace_bytes(int B, int H, int L, int m, int r, int d, int heads_w);
 cudaError_t launch_backward(const BwdArgs& a);
+// bf16 I/O on the tensor cores (kind::tf32): d a multiple of 32 up to 128, m a
+// multiple of 64 up to 256, r a multiple of 32 up to 256.
+bool tc_backward_supported(const BwdArgs& a);
+size_t tc_bwd_workspace_bytes(int B, int H, int L, int m, int r, int d, int heads_w);
+cudaError_t launch_backward_tc(const BwdArgs& a);
+cudaError_t bwd_fill_ordered(int* p, int n, float v, cudaStream_t s);
+cudaError_t bwd_shift_keys(float* phik, const int* ck, int L, int m, size_t n, cudaStream_t s);
+cudaError_t bwd_tile_scan(float* st, int n, int nt, int bh, int mode, cudaStream_t s);
+cudaError_t bwd_dgeom(const float* G, const BwdArgs& a);
 
 // Projection sampler (Philox4x64-10 + Box-Muller; orthogonal blocks by fp64
 // Gram-Schmidt).

@@ -1,0 +1,876 @@
+// Backward pass of PRF self-attention for bf16 I/O on the tensor cores:
+// every contraction of the chain rule runs as tcgen05 MMAs of kind::tf32 on
+// fp32 operands (tf32 keeps 10 explicit mantissa bits; bf16 operands would
+// not hold the gradients' tolerance), with fp32 accumulators in TMEM.
+//
+// DARKformer README, section "Kernel": phi(x)_j = m^{-1/2} exp(omega_j^T M x~
+// - 1/2 |M x~|^2), x~ = d^{-1/4} x, out = Phi(Q)(Phi(K)^T V) / Phi(Q)(Phi(K)^T 1);
+// section "Self-attention" gives the key mask and the causal constraint; M is
+// learned (Sigma = M^T M), Omega is a fixed draw.
+//
+// The chain rule is the one of the fp32 path (backward.cu) in the associative
+// order, on 128-token tiles (the causal chunk is one tile). For query i with
+// the key statistics S_i, z_i it sees and g_i = dout_i:
+//   w_i = g_i / den_i, c_i = (g_i . o_i) / den_i, P_i = [w_i | -c_i],
+//   dphi(q_i) = S_i w_i - z_i c_i = P_i [S_i | z_i]^T,
+//   dv_j = sum_i phi(q_i)^T phi(k_j) w_i,  dphi(k_j) = dS_j [v_j ; 1],
+//   coef = [ln2 phi dphi ; -2 (sum_j ln2 phi_j dphi_j) (W' x)_bot],
+//   dx = W'^T coef, dW' = sum_t coef_t x_t^T, dM = c_w Omega^T dW'_top + c_m dW'_bot.
+//
+// Launches: features (P = X W'^T, exp2 epilogue) -> tile states
+// Phi(K_c)^T [V_c | 1] -> exclusive prefix (causal) or total -> query pass
+// ([num | den], P = [w | -c], dphi(q), coef) -> tile states Phi(Q_c)^T [w | -c]
+// -> exclusive suffix or total -> key pass (dv, dphi(k), coef) -> dx -> dW'.
+// Operands are staged into shared memory by the CTA's threads (tc_tf32.cuh
+// layouts) through a two-slot ring: the threads fill one slot while the MMAs
+// of the other run.
+#include <math.h>
+
+#include "common.cuh"
+#include "internal.h"
+#include "tc_tf32.cuh"
+
+namespace dark {
+namespace {
+
+using tc::km_bytes;
+using tc::mn_bytes;
+
+constexpr int kTT = 128;                        // tokens per tile
+constexpr int kThr = 256;                       // threads per CTA
+constexpr float kLn2f = 0.69314718055994530942f;
+
+__host__ __device__ constexpr int round_up(int x, int a) { return (x + a - 1) / a * a; }
+
+// The shared-memory ring: slot g & 1 takes chunk g; a chunk's MMAs commit to
+// the slot's barrier, which the next user of the slot waits for. Every
+// thread calls every member in the same order; `failed` is uniform.
+struct Ring {
+  uint8_t* base;
+  uint32_t slot_bytes;
+  uint64_t* bar;                  // 2 slot barriers
+  int g;                          // chunks issued
+  bool failed;
+
+  __device__ uint8_t* acquire() {
+    const int s = g & 1;
+    if (g >= 2 && !failed) {
+      const bool ok = tc::mbar_wait(bar + s, ((g - 2) >> 1) & 1);
+      if (__syncthreads_or(ok ? 0 : 1)) failed = true;
+    }
+    return base + s * slot_bytes;
+  }
+  // After staging: thread 0 issues the chunk's MMAs and commits them.
+  template <class F>
+  __device__ void issue(F fn) {
+    tc::fence_async_smem();
+    tc::tc_fence_before();
+    __syncthreads();
+    if (!failed && threadIdx.x == 0) {
+      tc::tc_fence_after();
+      fn();
+      tc::mma_commit(bar + (g & 1));
+    }
+    ++g;
+  }
+  // Every MMA issued so far has completed (their results are readable).
+  __device__ void wait_all() {
+    if (g > 0 && !failed) {
+      const bool ok = tc::mbar_wait(bar + ((g - 1) & 1), ((g - 1) >> 1) & 1);
+      if (__syncthreads_or(ok ? 0 : 1)) failed = true;
+    }
+    tc::tc_fence_after();
+  }
+};
+
+// Shared prologue: barriers, TMEM allocation (warp 0). Returns the TMEM base.
+__device__ __forceinline__ uint32_t setup(uint64_t* bars, int nbars, uint32_t* tslot,
+                                          uint32_t ncols) {
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < nbars; ++i) tc::mbar_init(bars + i, 1);
+    tc::fence_mbar_init();
+  }
+  if (threadIdx.x < 32) tc::tmem_alloc(tslot, ncols);
+  tc::tc_fence_before();
+  __syncthreads();
+  tc::tc_fence_after();
+  return *tslot;
+}
+
+// Shared epilogue: on a failed wait, drain the issued MMAs before TMEM is freed.
+__device__ __forceinline__ void teardown(Ring& ring, uint64_t* bar_drain, uint32_t tmem,
+                                         uint32_t ncols, int* dev_status) {
+  if (ring.failed && threadIdx.x == 0) {
+    report(dev_status, DARK_ERR_TIMEOUT);
+    tc::drain_mmas(bar_drain);
+  }
+  tc::tc_fence_before();
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    tc::tc_fence_after();
+    tc::tmem_dealloc(tmem, ncols);
+  }
+}
+
+// TMEM address of this thread's lane (row 32 * (warp % 4) + lane) at column col.
+__device__ __forceinline__ uint32_t lane_addr(uint32_t tmem, int col) {
+  return tmem + ((uint32_t)((threadIdx.x >> 5) & 3) * 32u << 16) + (uint32_t)col;
+}
+
+__device__ __forceinline__ float4 ld_bf16x4(const __nv_bfloat16* p) {
+  return make_float4(__bfloat162float(p[0]), __bfloat162float(p[1]), __bfloat162float(p[2]),
+                     __bfloat162float(p[3]));
+}
+__device__ __forceinline__ void st_f4(float* p, float a, float b, float c, float d) {
+  *reinterpret_cast<float4*>(p) = make_float4(a, b, c, d);
+}
+
+// ---------------------------------------------------------------------------
+// Features of one side for a tile of 128 tokens: P = X W'^T on the tensor
+// cores (fp32 W', rows m + r for keys, m for queries). Keys: phi = 2^(P_top -
+// |P_bot|^2 - 1/2 log2 m), masked keys 0, and P_bot kept for the key
+// coefficients; with the stabiliser the exponent is stored (-inf when masked)
+// and the head maximum collected for a shift pass. Queries: 2^(P_top - max_j
+// P_top) (a per-query factor cancels from every query gradient).
+// Grid (tiles, B * H, 2 sides); TMEM columns 0 .. m + r - 1 hold P.
+struct FeatArgs {
+  const __nv_bfloat16 *xq, *xk;
+  int64_t sb, sh, sl;
+  const float* w;
+  int heads_w, m, r, d, H, L;
+  const uint8_t* mask;
+  int stabilise;
+  float *phiq, *phik, *pbot;
+  int* ck;
+  int* dev_status;
+};
+
+__global__ void __launch_bounds__(kThr, 1) tbf_features_kernel(FeatArgs a) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  const int side = blockIdx.z, bh = blockIdx.y, b = bh / a.H, h = bh % a.H;
+  const int t0 = blockIdx.x * kTT;
+  const int m = a.m, r = a.r, d = a.d, L = a.L;
+  const int nrow = side ? m + r : m;                          // W' rows = P columns
+  const uint32_t slot = km_bytes(kTT) + km_bytes(round_up(m + r, 32));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + 2 * slot);
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(bars + 4);
+  float* red = reinterpret_cast<float*>(tslot + 4);           // [2][128]
+  const uint32_t tmem = setup(bars, 3, tslot, 512);
+  Ring ring{smem, slot, bars, 0, false};
+  const __nv_bfloat16* x = (side ? a.xk : a.xq) + (int64_t)b * a.sb + (int64_t)h * a.sh;
+  const float* wh = a.w + (size_t)(a.heads_w == 1 ? 0 : h) * (m + r) * d;
+
+  for (int kc = 0; kc < d / 32; ++kc) {
+    uint8_t* s = ring.acquire();
+    tc::stage_km(s, kTT, [&](int row, int c) {
+      const int t = t0 + row;
+      return t < L ? ld_bf16x4(x + (int64_t)t * a.sl + kc * 32 + 4 * c) : make_float4(0.f, 0.f, 0.f, 0.f);
+    });
+    tc::stage_km(s + km_bytes(kTT), round_up(nrow, 32), [&](int row, int c) {
+      return row < nrow ? *reinterpret_cast<const float4*>(wh + (size_t)row * d + kc * 32 + 4 * c)
+                        : make_float4(0.f, 0.f, 0.f, 0.f);
+    });
+    ring.issue([&] {
+      const uint32_t sa = tc::smem_u32(s), sw = sa + km_bytes(kTT);
+      for (int c0 = 0; c0 < nrow; c0 += 256) {
+        const int n = nrow - c0 < 256 ? nrow - c0 : 256;
+        tc::mma_chunk(tmem + c0, sa, false, sw + (uint32_t)c0 * 128u, false, n, kc > 0);
+      }
+    });
+  }
+  ring.wait_all();
+
+  // epilogue: warps w and w + 4 share TMEM lanes 32 (w % 4) .. +31, each
+  // taking half of the columns; row statistics are combined through `red`.
+  const int q = (threadIdx.x >> 5) & 3, hf = threadIdx.x >> 7;
+  const int row = q * 32 + (threadIdx.x & 31), t = t0 + row;
+  const bool in = t < L;
+  float* dst = (side ? a.phik : a.phiq) + ((size_t)bh * L + (in ? t : 0)) * m;
+  const int half = m / 2;
+  if (side) {
+    // key norm |P_bot|^2 and P_bot itself
+    float nrm = 0.f;
+    float* pb = a.pbot + ((size_t)bh * L + (in ? t : 0)) * r;
+    for (int c0 = hf * (r / 2); c0 < (hf + 1) * (r / 2); c0 += 16) {
+      float v[16];
+      tc::tmem_ld16(lane_addr(tmem, m + c0), v);
+#pragma unroll
+      for (int j = 0; j < 16; ++j) nrm = fmaf(v[j], v[j], nrm);
+      if (in)
+#pragma unroll
+        for (int j = 0; j < 16; j += 4) st_f4(pb + c0 + j, v[j], v[j + 1], v[j + 2], v[j + 3]);
+    }
+    red[hf * kTT + row] = nrm;
+    __syncthreads();
+    const float rowc = red[row] + red[kTT + row] + 0.5f * log2f((float)m);
+    const bool ok = a.mask == nullptr || (in && a.mask[(size_t)b * L + t] != 0);
+    float kmax = -INFINITY;
+    for (int c0 = hf * half; c0 < (hf + 1) * half; c0 += 32) {
+      float v[32];
+      tc::tmem_ld32(lane_addr(tmem, c0), v);
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        const float e = v[j] - rowc;
+        if (a.stabilise) {
+          v[j] = ok ? e : -INFINITY;
+          kmax = fmaxf(kmax, v[j]);
+        } else {
+          v[j] = ok ? exp2f(e) : 0.f;
+        }
+      }
+      if (in)
+#pragma unroll
+        for (int j = 0; j < 32; j += 4) st_f4(dst + c0 + j, v[j], v[j + 1], v[j + 2], v[j + 3]);
+    }
+    if (a.stabilise) {
+      kmax = warp_max(in ? kmax : -INFINITY);
+      if ((threadIdx.x & 31) == 0 && kmax > -INFINITY) atomicMax(a.ck + bh, float_to_ordered(kmax));
+    }
+  } else {
+    float mx = -INFINITY;
+    for (int c0 = hf * half; c0 < (hf + 1) * half; c0 += 32) {
+      float v[32];
+      tc::tmem_ld32(lane_addr(tmem, c0), v);
+#pragma unroll
+      for (int j = 0; j < 32; ++j) mx = fmaxf(mx, v[j]);
+    }
+    red[hf * kTT + row] = mx;
+    __syncthreads();
+    mx = fmaxf(red[row], red[kTT + row]);
+    for (int c0 = hf * half; c0 < (hf + 1) * half; c0 += 32) {
+      float v[32];
+      tc::tmem_ld32(lane_addr(tmem, c0), v);
+#pragma unroll
+      for (int j = 0; j < 32; ++j) v[j] = exp2f(v[j] - mx);
+      if (in)
+#pragma unroll
+        for (int j = 0; j < 32; j += 4) st_f4(dst + c0 + j, v[j], v[j + 1], v[j + 2], v[j + 3]);
+    }
+  }
+  teardown(ring, bars + 2, tmem, 512, a.dev_status);
+}
+
+// ---------------------------------------------------------------------------
+// Tile states st_c = X_c^T U_c as [m][dp] fp32 (dp = d + 1 rounded up to 32,
+// the padding columns zero): X the feature rows of one side, U = [v | 1] for
+// keys (SIDE 1) or the rows [w | -c] the query pass stored (SIDE 0). M = m
+// features in one or two 128-row accumulators (TMEM columns 0 and 256), K =
+// the tile's 128 tokens, N = d + 1 rounded up to 16. Grid (tiles, B * H).
+struct StateArgs {
+  const float* X;                 // [B*H][L][m]
+  const __nv_bfloat16* v;         // keys: values
+  int64_t vb, vh, vl;
+  const float* wrow;              // queries: [B*H][L][dp]
+  int m, d, dp, H, L, nt;
+  float* st;                      // [B*H][nt][m][dp]
+  int* dev_status;
+};
+
+template <int SIDE>
+__global__ void __launch_bounds__(kThr, 1) tbf_state_kernel(StateArgs a) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  const int c = blockIdx.x, bh = blockIdx.y, b = bh / a.H, h = bh % a.H;
+  const int t0 = c * kTT, m = a.m, d = a.d, dp = a.dp, L = a.L;
+  const int mt = (m + 127) / 128, dn = round_up(d + 1, 16);
+  const uint32_t abytes = mn_bytes(mt * 128), slot = abytes + mn_bytes(dp);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + 2 * slot);
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(bars + 4);
+  const uint32_t tmem = setup(bars, 3, tslot, 512);
+  Ring ring{smem, slot, bars, 0, false};
+  const float* X = a.X + (size_t)bh * L * m;
+  const __nv_bfloat16* vh = a.v + (int64_t)b * a.vb + (int64_t)h * a.vh;
+  const float* wr = a.wrow + (size_t)bh * L * dp;
+
+  for (int kc = 0; kc < kTT / 32; ++kc) {
+    uint8_t* s = ring.acquire();
+    tc::stage_mn(s, mt * 128, [&](int k, int cc) {
+      const int t = t0 + kc * 32 + k;
+      return (t < L && 4 * cc < m) ? *reinterpret_cast<const float4*>(X + (size_t)t * m + 4 * cc)
+                                   : make_float4(0.f, 0.f, 0.f, 0.f);
+    });
+    tc::stage_mn(s + abytes, dp, [&](int k, int cc) {
+      const int t = t0 + kc * 32 + k, e = 4 * cc;
+      if (t >= L) return make_float4(0.f, 0.f, 0.f, 0.f);
+      if constexpr (SIDE == 0) return *reinterpret_cast<const float4*>(wr + (size_t)t * dp + e);
+      float u[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        u[j] = e + j < d ? __bfloat162float(vh[(int64_t)t * a.vl + e + j]) : (e + j == d ? 1.f : 0.f);
+      return make_float4(u[0], u[1], u[2], u[3]);
+    });
+    ring.issue([&] {
+      const uint32_t sa = tc::smem_u32(s), sb = sa + abytes;
+      for (int i = 0; i < mt; ++i)
+        tc::mma_chunk(tmem + 256 * i, sa + i * 4 * tc::kMnBlockBytes, true, sb, true, dn, kc > 0);
+    });
+  }
+  ring.wait_all();
+  // warps 0-3 read accumulator 0, warps 4-7 accumulator 1 (feature rows 128..)
+  const int q = (threadIdx.x >> 5) & 3, acc = threadIdx.x >> 7;
+  const int f = acc * 128 + q * 32 + (threadIdx.x & 31);
+  if (acc < mt) {
+    float* out = a.st + (((size_t)bh * a.nt + c) * m + (f < m ? f : 0)) * dp;
+    for (int c0 = 0; c0 < dp; c0 += 16) {
+      float v[16];
+      if (c0 < dn) tc::tmem_ld16(lane_addr(tmem, 256 * acc + c0), v);
+#pragma unroll
+      for (int j = 0; j < 16; ++j)
+        if (c0 + j > d) v[j] = 0.f;
+      if (f < m)
+#pragma unroll
+        for (int j = 0; j < 16; j += 4) st_f4(out + c0 + j, v[j], v[j + 1], v[j + 2], v[j + 3]);
+    }
+  }
+  teardown(ring, bars + 2, tmem, 512, a.dev_status);
+}
+
+// ---------------------------------------------------------------------------
+// One tile of 128 tokens of one side. SIDE 0 (queries): X = Phi(Q), Y = Phi(K),
+// state = [S | z] over earlier tiles (or all keys), U = [v | 1]; phase 1 gives
+// [num | den], hence P = [w | -c] (stored for the key side). SIDE 1 (keys):
+// X = Phi(K), Y = Phi(Q), state = [dS] over later tiles (or all queries),
+// U = [w | -c]; phase 1 gives dv, and P = [v | 1]. Phase 2 on both sides:
+// dphi(X) = P state^T + tri(P U^T) Y, coef = ln2 X dphi (keys add the norm
+// part). tri keeps key <= query inside the tile (causal only).
+// TMEM: columns 0..255 hold [num | den] / dv, later dphi; 256..383 the
+// diagonal tile's scores. Shared memory: a two-slot ring and, causal, the
+// masked 128 x 128 scores as a K-major operand.
+struct PassArgs {
+  const float *phiq, *phik;       // [B*H][L][m]
+  const float* state;             // [B*H][nt][m][dp]
+  const __nv_bfloat16* v;
+  int64_t vb, vh, vl;
+  const __nv_bfloat16* g;
+  int64_t gb, gh, gl;
+  float* wrow;                    // [B*H][L][dp]
+  __nv_bfloat16* dv;
+  int64_t ob, oh, ol;
+  float* coef;                    // [B*H][L][m + r]
+  const float* pbot;              // [B*H][L][r]
+  int m, r, d, dp, H, L, nt, causal;
+  int* dev_status;
+};
+
+__host__ __device__ inline uint32_t pass_slot_bytes(int m, int dp, int causal) {
+  const uint32_t p1 = km_bytes(kTT) + mn_bytes(dp) + (causal ? km_bytes(kTT) : 0);
+  const uint32_t p2 = km_bytes(kTT) + km_bytes(m) + (causal ? km_bytes(kTT) : 0);
+  const uint32_t p3 = mn_bytes(m);
+  uint32_t s = p1 > p2 ? p1 : p2;
+  return s > p3 ? s : p3;
+}
+__host__ __device__ inline uint32_t pass_smem_bytes(int m, int dp, int causal) {
+  return 1024 + 2 * pass_slot_bytes(m, dp, causal) + (causal ? 4 * km_bytes(kTT) : 0) + 64 +
+         2 * kTT * 4;
+}
+
+template <int SIDE>
+__global__ void __launch_bounds__(kThr, 1) tbf_pass_kernel(PassArgs a) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  const int c = blockIdx.x, bh = blockIdx.y, b = bh / a.H, h = bh % a.H;
+  const int t0 = c * kTT, m = a.m, r = a.r, d = a.d, dp = a.dp, L = a.L;
+  const int causal = a.causal, dn = round_up(d + 1, 16);
+  const uint32_t slot = pass_slot_bytes(m, dp, causal);
+  uint8_t* scores = smem + 2 * slot;                              // 4 K-major chunks
+  uint64_t* bars = reinterpret_cast<uint64_t*>(scores + (causal ? 4 * km_bytes(kTT) : 0));
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(bars + 4);
+  float* red = reinterpret_cast<float*>(tslot + 4);               // [2][128]
+  const uint32_t tmem = setup(bars, 3, tslot, 512);
+  const uint32_t tD = tmem, tS = tmem + 256;
+  Ring ring{smem, slot, bars, 0, false};
+
+  const size_t rowbase = (size_t)bh * L;
+  const float* X = (SIDE == 0 ? a.phiq : a.phik) + rowbase * m;
+  const float* Y = (SIDE == 0 ? a.phik : a.phiq) + rowbase * m;
+  const float* st = a.state + ((size_t)bh * a.nt + (causal ? c : 0)) * m * dp;
+  float* wr = a.wrow + rowbase * dp;
+  const __nv_bfloat16* vh = a.v + (int64_t)b * a.vb + (int64_t)h * a.vh;
+  // [v | 1 | 0 ...] at token t, columns e .. e + 3
+  auto vone4 = [&](int t, int e) -> float4 {
+    if (t >= L) return make_float4(0.f, 0.f, 0.f, 0.f);
+    float u[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+      u[j] = e + j < d ? __bfloat162float(vh[(int64_t)t * a.vl + e + j]) : (e + j == d ? 1.f : 0.f);
+    return make_float4(u[0], u[1], u[2], u[3]);
+  };
+  auto wrow4 = [&](int t, int e) -> float4 {
+    return t < L ? *reinterpret_cast<const float4*>(wr + (size_t)t * dp + e) : make_float4(0.f, 0.f, 0.f, 0.f);
+  };
+  // U rows of the tile: [v | 1] (queries) or [w | -c] (keys)
+  auto u4 = [&](int t, int e) -> float4 { return SIDE == 0 ? vone4(t, e) : wrow4(t, e); };
+  // P rows of the tile: [w | -c] (queries) or [v | 1] (keys)
+  auto p4 = [&](int t, int e) -> float4 { return SIDE == 0 ? wrow4(t, e) : vone4(t, e); };
+  auto feat4 = [&](const float* F, int t, int f) -> float4 {
+    return t < L ? *reinterpret_cast<const float4*>(F + (size_t)t * m + f) : make_float4(0.f, 0.f, 0.f, 0.f);
+  };
+
+  const int q = (threadIdx.x >> 5) & 3, hf = threadIdx.x >> 7;
+  const int row = q * 32 + (threadIdx.x & 31), t = t0 + row;
+  const bool in = t < L;
+  // masked diagonal scores (TMEM columns 256..383) -> K-major operand in `scores`
+  auto scores_to_smem = [&]() {
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int c0 = hf * 64 + u * 32;
+      float v[32];
+      tc::tmem_ld32(lane_addr(tS, c0), v);
+      uint8_t* chunk = scores + (c0 >> 5) * km_bytes(kTT);
+#pragma unroll
+      for (int j4 = 0; j4 < 8; ++j4) {
+        float o[4];
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj) {
+          const int col = c0 + 4 * j4 + jj;
+          const bool keep = SIDE == 0 ? col <= row : col >= row;
+          o[jj] = keep ? v[4 * j4 + jj] : 0.f;
+        }
+        *reinterpret_cast<float4*>(chunk + (row >> 3) * 1024 + (row & 7) * 128 +
+                                   (((j4 ^ row) & 7) << 4)) = make_float4(o[0], o[1], o[2], o[3]);
+      }
+    }
+  };
+
+  // ---- phase 1: D = X state + tri(X Y^T) U ----
+  for (int fc = 0; fc < m / 32; ++fc) {
+    uint8_t* s = ring.acquire();
+    tc::stage_km(s, kTT, [&](int rr, int cc) { return feat4(X, t0 + rr, fc * 32 + 4 * cc); });
+    tc::stage_mn(s + km_bytes(kTT), dp, [&](int k, int cc) {
+      return *reinterpret_cast<const float4*>(st + (size_t)(fc * 32 + k) * dp + 4 * cc);
+    });
+    if (causal)
+      tc::stage_km(s + km_bytes(kTT) + mn_bytes(dp), kTT,
+                   [&](int rr, int cc) { return feat4(Y, t0 + rr, fc * 32 + 4 * cc); });
+    ring.issue([&] {
+      const uint32_t sa = tc::smem_u32(s);
+      tc::mma_chunk(tD, sa, false, sa + km_bytes(kTT), true, dn, fc > 0);
+      if (causal)
+        tc::mma_chunk(tS, sa, false, sa + km_bytes(kTT) + mn_bytes(dp), false, kTT, fc > 0);
+    });
+  }
+  if (causal) {
+    ring.wait_all();
+    scores_to_smem();
+    for (int kc = 0; kc < kTT / 32; ++kc) {
+      uint8_t* s = ring.acquire();
+      tc::stage_mn(s, dp, [&](int k, int cc) { return u4(t0 + kc * 32 + k, 4 * cc); });
+      ring.issue([&] {
+        tc::mma_chunk(tD, tc::smem_u32(scores + kc * km_bytes(kTT)), false, tc::smem_u32(s), true,
+                      dn, true);
+      });
+    }
+  }
+  ring.wait_all();
+
+  // ---- epilogue of phase 1 ----
+  const int dh = d / 2;
+  if (SIDE == 0) {
+    const __nv_bfloat16* gh = a.g + (int64_t)b * a.gb + (int64_t)h * a.gh + (int64_t)(in ? t : 0) * a.gl;
+    const float den = tc::tmem_ld1(lane_addr(tD, d));
+    float go = 0.f;
+    for (int c0 = hf * dh; c0 < (hf + 1) * dh; c0 += 16) {
+      float v[16];
+      tc::tmem_ld16(lane_addr(tD, c0), v);
+      if (in)
+#pragma unroll
+        for (int j = 0; j < 16; ++j) go = fmaf(__bfloat162float(gh[c0 + j]), v[j], go);
+    }
+    red[hf * kTT + row] = go;
+    __syncthreads();
+    go = red[row] + red[kTT + row];
+    const float inv = (in && den > 0.f) ? 1.f / den : 0.f;
+    const float cc = go * inv * inv;
+    if (in) {
+      float* wt = wr + (size_t)t * dp;
+      for (int c0 = hf * dh; c0 < (hf + 1) * dh; c0 += 4) {
+        float p[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          p[j] = __bfloat162float(gh[c0 + j]) * inv;
+          if (!isfinite(p[j])) report(a.dev_status, DARK_ERR_NUMERIC);
+        }
+        st_f4(wt + c0, p[0], p[1], p[2], p[3]);
+      }
+      if (hf == 1) {
+        if (!isfinite(cc)) report(a.dev_status, DARK_ERR_NUMERIC);
+        for (int e = d; e < dp; e += 4) st_f4(wt + e, e == d ? -cc : 0.f, 0.f, 0.f, 0.f);
+      }
+    }
+  } else {
+    __nv_bfloat16* dvh = a.dv + (int64_t)b * a.ob + (int64_t)h * a.oh + (int64_t)(in ? t : 0) * a.ol;
+    for (int c0 = hf * dh; c0 < (hf + 1) * dh; c0 += 16) {
+      float v[16];
+      tc::tmem_ld16(lane_addr(tD, c0), v);
+      if (in)
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          if (!isfinite(v[j])) report(a.dev_status, DARK_ERR_NUMERIC);
+          dvh[c0 + j] = __float2bfloat16_rn(v[j]);
+        }
+    }
+  }
+  tc::tc_fence_before();
+  __syncthreads();                // the P rows above are read back by the staging below
+
+  // ---- phase 2: dphi(X) = P state^T + tri(P U^T) Y ----
+  for (int pc = 0; pc < dp / 32; ++pc) {
+    uint8_t* s = ring.acquire();
+    tc::stage_km(s, kTT, [&](int rr, int cc) { return p4(t0 + rr, pc * 32 + 4 * cc); });
+    tc::stage_km(s + km_bytes(kTT), m, [&](int f, int cc) {
+      return *reinterpret_cast<const float4*>(st + (size_t)f * dp + pc * 32 + 4 * cc);
+    });
+    if (causal)
+      tc::stage_km(s + km_bytes(kTT) + km_bytes(m), kTT,
+                   [&](int rr, int cc) { return u4(t0 + rr, pc * 32 + 4 * cc); });
+    ring.issue([&] {
+      const uint32_t sa = tc::smem_u32(s);
+      tc::mma_chunk(tD, sa, false, sa + km_bytes(kTT), false, m, pc > 0);
+      if (causal)
+        tc::mma_chunk(tS, sa, false, sa + km_bytes(kTT) + km_bytes(m), false, kTT, pc > 0);
+    });
+  }
+  if (causal) {
+    ring.wait_all();
+    scores_to_smem();
+    for (int kc = 0; kc < kTT / 32; ++kc) {
+      uint8_t* s = ring.acquire();
+      tc::stage_mn(s, m, [&](int k, int cc) { return feat4(Y, t0 + kc * 32 + k, 4 * cc); });
+      ring.issue([&] {
+        tc::mma_chunk(tD, tc::smem_u32(scores + kc * km_bytes(kTT)), false, tc::smem_u32(s), true,
+                      m, true);
+      });
+    }
+  }
+  ring.wait_all();
+
+  // ---- coef = ln2 X dphi; keys add -2 (sum_j coef_j) P_bot ----
+  const int mh = m / 2, rh = r / 2;
+  float* cf = a.coef + (rowbase + (in ? t : 0)) * (size_t)(m + r);
+  const float* xr = X + (size_t)(in ? t : 0) * m;
+  float rs = 0.f;
+  for (int c0 = hf * mh; c0 < (hf + 1) * mh; c0 += 32) {
+    float v[32];
+    tc::tmem_ld32(lane_addr(tD, c0), v);
+    if (in) {
+#pragma unroll
+      for (int j = 0; j < 32; j += 4) {
+        const float4 x4 = *reinterpret_cast<const float4*>(xr + c0 + j);
+        const float o0 = kLn2f * x4.x * v[j], o1 = kLn2f * x4.y * v[j + 1];
+        const float o2 = kLn2f * x4.z * v[j + 2], o3 = kLn2f * x4.w * v[j + 3];
+        rs += (o0 + o1) + (o2 + o3);
+        st_f4(cf + c0 + j, o0, o1, o2, o3);
+      }
+    }
+  }
+  if (SIDE == 1) {
+    red[hf * kTT + row] = rs;
+    __syncthreads();
+    rs = red[row] + red[kTT + row];
+  }
+  if (in) {
+    const float* pb = a.pbot + (rowbase + t) * (size_t)r;
+    for (int j = hf * rh; j < (hf + 1) * rh; j += 4) {
+      if (SIDE == 1) {
+        const float4 p = *reinterpret_cast<const float4*>(pb + j);
+        st_f4(cf + m + j, -2.f * rs * p.x, -2.f * rs * p.y, -2.f * rs * p.z, -2.f * rs * p.w);
+      } else {
+        st_f4(cf + m + j, 0.f, 0.f, 0.f, 0.f);
+      }
+    }
+  }
+  teardown(ring, bars + 2, tmem, 512, a.dev_status);
+}
+
+// ---------------------------------------------------------------------------
+// dx = coef W' for a tile of 128 tokens of one side (queries: K = m, their norm
+// part is zero; keys: K = m + r). A = coef rows (K-major), B = W' (MN-major,
+// N = d). Grid (tiles, B * H, 2 sides).
+struct DxArgs {
+  const float *cfq, *cfk;         // [B*H][L][m + r]
+  const float* w;                 // [heads_w][m + r][d]
+  int heads_w, m, r, d, H, L;
+  __nv_bfloat16 *dq, *dk;
+  int64_t ob, oh, ol;
+  int* dev_status;
+};
+
+__global__ void __launch_bounds__(kThr) tbf_dx_kernel(DxArgs a) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  const int side = blockIdx.z, bh = blockIdx.y, b = bh / a.H, h = bh % a.H;
+  const int t0 = blockIdx.x * kTT, m = a.m, r = a.r, d = a.d, L = a.L, mr = m + r;
+  const uint32_t slot = km_bytes(kTT) + mn_bytes(d);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + 2 * slot);
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(bars + 4);
+  const uint32_t tmem = setup(bars, 3, tslot, 128);
+  Ring ring{smem, slot, bars, 0, false};
+  const float* cf = (side ? a.cfk : a.cfq) + (size_t)bh * L * mr;
+  const float* wh = a.w + (size_t)(a.heads_w == 1 ? 0 : h) * mr * d;
+  const int kend = side ? mr : m;
+  for (int kc = 0; kc < kend / 32; ++kc) {
+    uint8_t* s = ring.acquire();
+    tc::stage_km(s, kTT, [&](int rr, int cc) {
+      const int t = t0 + rr;
+      return t < L ? *reinterpret_cast<const float4*>(cf + (size_t)t * mr + kc * 32 + 4 * cc)
+                   : make_float4(0.f, 0.f, 0.f, 0.f);
+    });
+    tc::stage_mn(s + km_bytes(kTT), d, [&](int k, int cc) {
+      return *reinterpret_cast<const float4*>(wh + (size_t)(kc * 32 + k) * d + 4 * cc);
+    });
+    ring.issue([&] {
+      const uint32_t sa = tc::smem_u32(s);
+      tc::mma_chunk(tmem, sa, false, sa + km_bytes(kTT), true, d, kc > 0);
+    });
+  }
+  ring.wait_all();
+  const int q = (threadIdx.x >> 5) & 3, hf = threadIdx.x >> 7;
+  const int row = q * 32 + (threadIdx.x & 31), t = t0 + row;
+  __nv_bfloat16* out = (side ? a.dk : a.dq) + (int64_t)b * a.ob + (int64_t)h * a.oh +
+                       (int64_t)(t < L ? t : 0) * a.ol;
+  for (int c0 = hf * (d / 2); c0 < (hf + 1) * (d / 2); c0 += 16) {
+    float v[16];
+    tc::tmem_ld16(lane_addr(tmem, c0), v);
+    if (t < L)
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        if (!isfinite(v[j])) report(a.dev_status, DARK_ERR_NUMERIC);
+        out[c0 + j] = __float2bfloat16_rn(v[j]);
+      }
+  }
+  teardown(ring, bars + 2, tmem, 128, a.dev_status);
+}
+
+// dW'[hw] += sum over a token range of one (batch, head), both sides, of
+// coef_t x_t^T: a 128-row block of [m + r][d] per CTA, K = tokens, A = coef^T
+// and B = x both MN-major; fp32 atomics into dW' at the end.
+// Grid (row blocks, B * H, token splits).
+struct DwArgs {
+  const __nv_bfloat16 *xq, *xk;
+  int64_t sb, sh, sl;
+  const float *cfq, *cfk;
+  int m, r, d, H, L, heads_w, nsplit;
+  float* G;                       // [heads_w][m + r][d]
+  int* dev_status;
+};
+
+__global__ void __launch_bounds__(kThr) tbf_dw_kernel(DwArgs a) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  const int j0 = blockIdx.x * 128, bh = blockIdx.y, split = blockIdx.z;
+  const int b = bh / a.H, h = bh % a.H, d = a.d, L = a.L, mr = a.m + a.r;
+  const int per = round_up((L + a.nsplit - 1) / a.nsplit, 32);
+  const int tb = split * per, te = min(L, tb + per);
+  const uint32_t slot = mn_bytes(128) + mn_bytes(d);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + 2 * slot);
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(bars + 4);
+  const uint32_t tmem = setup(bars, 3, tslot, 128);
+  Ring ring{smem, slot, bars, 0, false};
+  for (int side = 0; side < 2; ++side) {
+    const __nv_bfloat16* x = (side ? a.xk : a.xq) + (int64_t)b * a.sb + (int64_t)h * a.sh;
+    const float* cf = (side ? a.cfk : a.cfq) + (size_t)bh * L * mr;
+    for (int k0 = tb; k0 < te; k0 += 32) {
+      uint8_t* s = ring.acquire();
+      tc::stage_mn(s, 128, [&](int k, int cc) {
+        const int t = k0 + k, j = j0 + 4 * cc;
+        return (t < te && j < mr) ? *reinterpret_cast<const float4*>(cf + (size_t)t * mr + j)
+                                  : make_float4(0.f, 0.f, 0.f, 0.f);
+      });
+      tc::stage_mn(s + mn_bytes(128), d, [&](int k, int cc) {
+        const int t = k0 + k;
+        return t < te ? ld_bf16x4(x + (int64_t)t * a.sl + 4 * cc) : make_float4(0.f, 0.f, 0.f, 0.f);
+      });
+      const bool first = ring.g == 0;
+      ring.issue([&] {
+        const uint32_t sa = tc::smem_u32(s);
+        tc::mma_chunk(tmem, sa, true, sa + mn_bytes(128), true, d, !first);
+      });
+    }
+  }
+  ring.wait_all();
+  const int q = (threadIdx.x >> 5) & 3, hf = threadIdx.x >> 7;
+  const int j = j0 + q * 32 + (threadIdx.x & 31);
+  float* gh = a.G + ((size_t)(a.heads_w == 1 ? 0 : h) * mr + (j < mr ? j : 0)) * d;
+  if (ring.g > 0)
+    for (int c0 = hf * (d / 2); c0 < (hf + 1) * (d / 2); c0 += 16) {
+      float v[16];
+      tc::tmem_ld16(lane_addr(tmem, c0), v);
+      if (j < mr)
+#pragma unroll
+        for (int u = 0; u < 16; ++u) atomicAdd(gh + c0 + u, v[u]);
+    }
+  teardown(ring, bars + 2, tmem, 128, a.dev_status);
+}
+
+struct TcLayout {
+  int nt, dp;
+  size_t off_w, off_ck, off_phiq, off_phik, off_pbot, off_cs, off_ds, off_wq, off_cfq, off_cfk,
+      off_g, total;
+};
+
+TcLayout tc_layout(int B, int H, int L, int m, int r, int d, int heads_w) {
+  TcLayout s;
+  const size_t bh = (size_t)B * H, mr = (size_t)m + r;
+  s.nt = (L + kTT - 1) / kTT;
+  s.dp = round_up(d + 1, 32);
+  size_t o = kWsHeader;
+  auto take = [&o](size_t bytes) {
+    const size_t at = o;
+    o = align_up(o + bytes, 256);
+    return at;
+  };
+  s.off_w = take(sizeof(float) * heads_w * mr * d);
+  s.off_ck = take(sizeof(int) * bh);
+  s.off_phiq = take(sizeof(float) * bh * L * m);
+  s.off_phik = take(sizeof(float) * bh * L * m);
+  s.off_pbot = take(sizeof(float) * bh * L * r);
+  s.off_cs = take(sizeof(float) * bh * s.nt * m * s.dp);
+  s.off_ds = take(sizeof(float) * bh * s.nt * m * s.dp);
+  s.off_wq = take(sizeof(float) * bh * L * s.dp);
+  s.off_cfq = take(sizeof(float) * bh * L * mr);
+  s.off_cfk = take(sizeof(float) * bh * L * mr);
+  s.off_g = take(sizeof(float) * heads_w * mr * d);
+  s.total = o;
+  return s;
+}
+
+template <class K>
+cudaError_t set_smem(K kernel, size_t bytes, int* done) {
+  return set_smem_limit_once((const void*)kernel, (int)bytes, done);
+}
+
+// The kernels that allocate all 512 TMEM columns ask for enough shared memory
+// to keep a single CTA per SM.
+constexpr size_t kOneCtaSmem = 116 * 1024;
+size_t one_cta(size_t bytes) { return bytes > kOneCtaSmem ? bytes : kOneCtaSmem; }
+
+}  // namespace
+
+size_t tc_bwd_workspace_bytes(int B, int H, int L, int m, int r, int d, int heads_w) {
+  return tc_layout(B, H, L, m, r, d, heads_w).total;
+}
+
+bool tc_backward_supported(const BwdArgs& a) {
+  if (a.dtype != DARK_BF16) return false;
+  if (a.d % 32 != 0 || a.d > 128 || a.m % 64 != 0 || a.m > 256 || a.r % 32 != 0 || a.r > 256)
+    return false;
+  const int dp = round_up(a.d + 1, 32);
+  if (pass_smem_bytes(a.m, dp, 1) > 227 * 1024) return false;
+  return true;
+}
+
+cudaError_t launch_backward_tc(const BwdArgs& a) {
+  const TcLayout s = tc_layout(a.B, a.H, a.L, a.m, a.r, a.d, a.heads_w);
+  char* ws = (char*)a.ws;
+  float* wf = (float*)(ws + s.off_w);
+  int* ck = (int*)(ws + s.off_ck);
+  float* phiq = (float*)(ws + s.off_phiq);
+  float* phik = (float*)(ws + s.off_phik);
+  float* pbot = (float*)(ws + s.off_pbot);
+  float* cs = (float*)(ws + s.off_cs);
+  float* dsn = (float*)(ws + s.off_ds);
+  float* wq = (float*)(ws + s.off_wq);
+  float* cfq = (float*)(ws + s.off_cfq);
+  float* cfk = (float*)(ws + s.off_cfk);
+  float* G = (float*)(ws + s.off_g);
+  const int bh = a.B * a.H, m = a.m, r = a.r, d = a.d, L = a.L, nt = s.nt, dp = s.dp;
+  const int stab = (a.flags & DARK_STABILISE) ? 1 : 0;
+  const int causal = (a.flags & DARK_CAUSAL) ? 1 : 0;
+  const __nv_bfloat16* q = (const __nv_bfloat16*)a.q;
+  const __nv_bfloat16* k = (const __nv_bfloat16*)a.k;
+  const __nv_bfloat16* v = (const __nv_bfloat16*)a.v;
+  cudaStream_t st = a.stream;
+  cudaError_t err;
+
+  err = launch_projection(a.omega, a.heads_omega, a.geom, a.heads_geom, a.heads_w, m, r, d,
+                          DARK_F32, wf, st);
+  if (err != cudaSuccess) return err;
+  if (stab && (err = bwd_fill_ordered(ck, bh, -INFINITY, st)) != cudaSuccess) return err;
+
+  {
+    static int done[64];
+    const size_t bytes = one_cta(1024 + 2 * (km_bytes(kTT) + km_bytes(round_up(m + r, 32))) + 64 +
+                                 2 * kTT * 4);
+    if ((err = set_smem(tbf_features_kernel, bytes, done)) != cudaSuccess) return err;
+    FeatArgs fa{q, k, a.xs[0], a.xs[1], a.xs[2], wf, a.heads_w, m, r, d, a.H, L, a.mask, stab,
+                phiq, phik, pbot, ck, a.dev_status};
+    tbf_features_kernel<<<dim3(nt, bh, 2), kThr, bytes, st>>>(fa);
+    if ((err = cudaGetLastError()) != cudaSuccess) return err;
+  }
+  if (stab && (err = bwd_shift_keys(phik, ck, L, m, (size_t)bh * L * m, st)) != cudaSuccess)
+    return err;
+
+  const size_t st_bytes = one_cta(1024 + 2 * (mn_bytes(round_up(m, 128)) + mn_bytes(dp)) + 64);
+  StateArgs sa{phik, v, a.xs[0], a.xs[1], a.xs[2], wq, m, d, dp, a.H, L, nt, cs, a.dev_status};
+  {
+    static int done[64];
+    if ((err = set_smem(tbf_state_kernel<1>, st_bytes, done)) != cudaSuccess) return err;
+    tbf_state_kernel<1><<<dim3(nt, bh), kThr, st_bytes, st>>>(sa);
+    if ((err = cudaGetLastError()) != cudaSuccess) return err;
+  }
+  if ((err = bwd_tile_scan(cs, m * dp, nt, bh, causal ? 0 : 2, st)) != cudaSuccess) return err;
+
+  const size_t pass_bytes = one_cta(pass_smem_bytes(m, dp, causal));
+  PassArgs pa{phiq, phik, cs, v, a.xs[0], a.xs[1], a.xs[2],
+              (const __nv_bfloat16*)a.dout, a.gs[0], a.gs[1], a.gs[2], wq,
+              nullptr, 0, 0, 0, cfq, pbot, m, r, d, dp, a.H, L, nt, causal, a.dev_status};
+  {
+    static int done[64];
+    if ((err = set_smem(tbf_pass_kernel<0>, pass_bytes, done)) != cudaSuccess) return err;
+    tbf_pass_kernel<0><<<dim3(nt, bh), kThr, pass_bytes, st>>>(pa);
+    if ((err = cudaGetLastError()) != cudaSuccess) return err;
+  }
+  sa.X = phiq;
+  sa.st = dsn;
+  {
+    static int done[64];
+    if ((err = set_smem(tbf_state_kernel<0>, st_bytes, done)) != cudaSuccess) return err;
+    tbf_state_kernel<0><<<dim3(nt, bh), kThr, st_bytes, st>>>(sa);
+    if ((err = cudaGetLastError()) != cudaSuccess) return err;
+  }
+  if ((err = bwd_tile_scan(dsn, m * dp, nt, bh, causal ? 1 : 2, st)) != cudaSuccess) return err;
+  pa.state = dsn;
+  pa.g = nullptr;
+  pa.gb = pa.gh = pa.gl = 0;
+  pa.dv = (__nv_bfloat16*)a.dv;
+  pa.ob = a.ds[0];
+  pa.oh = a.ds[1];
+  pa.ol = a.ds[2];
+  pa.coef = cfk;
+  {
+    static int done[64];
+    if ((err = set_smem(tbf_pass_kernel<1>, pass_bytes, done)) != cudaSuccess) return err;
+    tbf_pass_kernel<1><<<dim3(nt, bh), kThr, pass_bytes, st>>>(pa);
+    if ((err = cudaGetLastError()) != cudaSuccess) return err;
+  }
+  {
+    static int done[64];
+    const size_t bytes = 1024 + 2 * (km_bytes(kTT) + mn_bytes(d)) + 64;
+    if ((err = set_smem(tbf_dx_kernel, bytes, done)) != cudaSuccess) return err;
+    DxArgs xa{cfq, cfk, wf, a.heads_w, m, r, d, a.H, L, (__nv_bfloat16*)a.dq,
+              (__nv_bfloat16*)a.dk, a.ds[0], a.ds[1], a.ds[2], a.dev_status};
+    tbf_dx_kernel<<<dim3(nt, bh, 2), kThr, bytes, st>>>(xa);
+    if ((err = cudaGetLastError()) != cudaSuccess) return err;
+  }
+  if (a.dgeom != nullptr) {
+    err = cudaMemsetAsync(G, 0, sizeof(float) * (size_t)a.heads_w * (m + r) * d, st);
+    if (err != cudaSuccess) return err;
+    const int blocks = (m + r + 127) / 128;
+    int nsplit = (2 * num_sms() + blocks * bh - 1) / (blocks * bh);
+    const int max_split = (L + 127) / 128;
+    if (nsplit > max_split) nsplit = max_split;
+    if (nsplit < 1) nsplit = 1;
+    static int done[64];
+    const size_t bytes = 1024 + 2 * (mn_bytes(128) + mn_bytes(d)) + 64;
+    if ((err = set_smem(tbf_dw_kernel, bytes, done)) != cudaSuccess) return err;
+    DwArgs wa{q, k, a.xs[0], a.xs[1], a.xs[2], cfq, cfk, m, r, d, a.H, L, a.heads_w, nsplit, G,
+              a.dev_status};
+    tbf_dw_kernel<<<dim3(blocks, bh, nsplit), kThr, bytes, st>>>(wa);
+    if ((err = cudaGetLastError()) != cudaSuccess) return err;
+    if ((err = bwd_dgeom(G, a)) != cudaSuccess) return err;
+  }
+  return cudaSuccess;
+}
+
+}  // namespace dark

@@ -74,9 +74,10 @@ cudaError_t set_smem_limit_once(const void* kernel, int bytes, int* done_per_dev
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  if (dev >= 0 && dev < 64 && done_per_device[dev]) return cudaSuccess;
+  // done_per_device[dev] holds the largest size set so far on that device
+  if (dev >= 0 && dev < 64 && done_per_device[dev] >= bytes) return cudaSuccess;
   e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
-  if (e == cudaSuccess && dev >= 0 && dev < 64) done_per_device[dev] = 1;
+  if (e == cudaSuccess && dev >= 0 && dev < 64) done_per_device[dev] = bytes;
   return e;
 }
 

@@ -2,9 +2,12 @@
 C ABI with the fp64 oracle, on seeded synthetic inputs.
 
 Tolerances (per (batch, head), relative to the largest reference entry): fp32
-I/O 1e-4; bf16 I/O 8e-3 for dq, dk, dv (the kernels compute in fp32 from
-bf16-exact inputs, and rounding the gradients to bf16 moves each entry by up
-to 2^-9 of itself); the geometry gradient is fp32 for both and held to 1e-4.
+I/O 1e-4 (fp32 arithmetic throughout); bf16 I/O 8e-3 for dq, dk, dv and the
+geometry gradient: the bf16 path runs every contraction on the tensor cores
+with tf32 operands (10 explicit mantissa bits, unit roundoff 2^-11) and fp32
+accumulation, and rounding dq, dk, dv to bf16 moves each entry by up to 2^-9
+of itself. A numpy emulation of that arithmetic on the causal workload gives
+about 1.5e-3 for the gradients.
 """
 import numpy as np
 import pytest
@@ -77,7 +80,7 @@ def check_grads(w, got, ref):
     dg, rg = got[3], ref[3]
     assert np.all(np.isfinite(dg))
     err = max(np.abs(dg[i] - rg[i]).max() / np.abs(rg[i]).max() for i in range(rg.shape[0]))
-    assert err <= 1e-4, f"dgeom: relative error {err:.3e}"
+    assert err <= tol, f"dgeom: relative error {err:.3e} > {tol}"
 
 
 SMALL = {
