@@ -791,6 +791,13 @@ def run_backward(args, w: synth.Workload, rank: int, world: int, dev) -> dict | 
         D.dark_attention_bwd(omega, geom, q_, k_, v_, g_, dq, dk, dv, w.B, w.H, w.L, dt,
                              key_mask=m_, flags=flags, dgeom=dgeom, ws=ws, dev_status=status)
 
+    if args.ncu:
+        # capture mode for Nsight Compute: warmup + steps backward calls only
+        for _ in range(args.warmup + args.steps):
+            call(q, k, v, g, mask)
+        torch.cuda.synchronize()
+        assert int(status.item()) == 0, D.dark_status_string(int(status.item()))
+        return None
     for _ in range(args.warmup):
         flush.zero_()
         call(q, k, v, g, mask)

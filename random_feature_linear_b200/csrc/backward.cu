@@ -258,22 +258,22 @@ __global__ void __launch_bounds__(256) chunk_state_kernel(const float* __restric
 }
 
 // mode 0: exclusive prefix over tiles (causal forward statistics); 1: exclusive
-// suffix (causal gradient statistics); 2: total into tile 0 (non-causal). Eight
-// tiles' values are loaded before any is stored, so the loads overlap.
+// suffix (causal gradient statistics); 2: total into tile 0 (non-causal).
+// Sixteen tiles' values are loaded before any is stored, so the loads overlap.
 __global__ void tile_scan_kernel(float* __restrict__ st, int n, int nt, int mode) {
   const int idx = blockIdx.x * blockDim.x + threadIdx.x;
   if (idx >= n) return;
   float* base = st + (size_t)blockIdx.y * nt * n + idx;
   float run = 0.f;
-  for (int s0 = 0; s0 < nt; s0 += 8) {
-    float v[8];
+  for (int s0 = 0; s0 < nt; s0 += 16) {
+    float v[16];
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {
+    for (int u = 0; u < 16; ++u) {
       const int s = s0 + u, c = mode == 1 ? nt - 1 - s : s;
       v[u] = s < nt ? base[(size_t)c * n] : 0.f;
     }
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {
+    for (int u = 0; u < 16; ++u) {
       const int s = s0 + u, c = mode == 1 ? nt - 1 - s : s;
       if (s < nt && mode != 2) base[(size_t)c * n] = run;
       run += v[u];
@@ -660,8 +660,15 @@ __global__ void dgeom_kernel(const float* __restrict__ G, const float* __restric
       if (heads_geom != 1 && hw != hm) continue;
       const float* om = omega + (size_t)(heads_omega == 1 ? 0 : hw) * m * r;
       const float* g = G + (size_t)hw * mr * d;
-      float s = 0.f;
-      for (int j = 0; j < m; ++j) s = fmaf(om[(size_t)j * r + i], g[(size_t)j * d + c], s);
+      float s4[4] = {0.f, 0.f, 0.f, 0.f};
+      int j = 0;
+#pragma unroll 4
+      for (; j + 4 <= m; j += 4)
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+          s4[u] = fmaf(om[(size_t)(j + u) * r + i], g[(size_t)(j + u) * d + c], s4[u]);
+      for (; j < m; ++j) s4[0] = fmaf(om[(size_t)j * r + i], g[(size_t)j * d + c], s4[0]);
+      const float s = (s4[0] + s4[1]) + (s4[2] + s4[3]);
       acc += cw * s + cm * g[(size_t)(m + i) * d + c];
     }
     dgeom[((size_t)hm * r + i) * d + c] = acc;

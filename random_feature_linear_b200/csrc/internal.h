@@ -143,7 +143,7 @@ struct BwdArgs {
 size_t bwd_workspace_bytes(int B, int H, int L, int m, int r, int d, int heads_w);
 cudaError_t launch_backward(const BwdArgs& a);
 // bf16 I/O on the tensor cores (kind::tf32): d a multiple of 32 up to 128, m a
-// multiple of 64 up to 256, r a multiple of 32 up to 256.
+// multiple of 64 up to 256, r a multiple of 32 up to 128.
 bool tc_backward_supported(const BwdArgs& a);
 size_t tc_bwd_workspace_bytes(int B, int H, int L, int m, int r, int d, int heads_w);
 cudaError_t launch_backward_tc(const BwdArgs& a);

@@ -39,46 +39,75 @@ using tc::mn_bytes;
 constexpr int kTT = 128;                        // tokens per tile
 constexpr int kThr = 256;                       // threads per CTA
 constexpr float kLn2f = 0.69314718055994530942f;
+constexpr int kFeatSlots = 3, kStateSlots = 4, kPassSlots = 3, kGemmSlots = 4;
+// Shared memory past the ring: 8 barriers (slots, drain), the TMEM slot and a
+// [2][128] fp32 reduction buffer.
+constexpr uint32_t kTailBytes = 128 + 2 * 128 * 4;
 
 __host__ __device__ constexpr int round_up(int x, int a) { return (x + a - 1) / a * a; }
 
-// The shared-memory ring: slot g & 1 takes chunk g; a chunk's MMAs commit to
-// the slot's barrier, which the next user of the slot waits for. Every
-// thread calls every member in the same order; `failed` is uniform.
+// The shared-memory ring of NS slots: chunk i is staged into slot i % NS; its
+// MMAs commit to that slot's barrier, which the stager of chunk i + NS waits
+// for. The MMAs of chunk i are issued once chunk i + NS - 1 has been staged,
+// so the copies of NS - 1 chunks are in flight behind the MMAs. Every thread
+// calls every member in the same order; `failed` is uniform.
+template <int NS>
 struct Ring {
   uint8_t* base;
   uint32_t slot_bytes;
-  uint64_t* bar;                  // 2 slot barriers
-  int g;                          // chunks issued
+  uint64_t* bar;                  // NS slot barriers
+  int staged;                     // chunks staged
+  int issued;                     // chunks whose MMAs are issued
   bool failed;
 
-  __device__ uint8_t* acquire() {
-    const int s = g & 1;
-    if (g >= 2 && !failed) {
-      const bool ok = tc::mbar_wait(bar + s, ((g - 2) >> 1) & 1);
+  __device__ uint8_t* slot(int i) const { return base + (i % NS) * slot_bytes; }
+  __device__ void wait_chunk(int i) {   // the MMAs of chunk i completed
+    if (i >= 0 && !failed) {
+      const bool ok = tc::mbar_wait(bar + (i % NS), (i / NS) & 1);
       if (__syncthreads_or(ok ? 0 : 1)) failed = true;
     }
-    return base + s * slot_bytes;
   }
-  // After staging: thread 0 issues the chunk's MMAs and commits them.
+  __device__ uint8_t* acquire() {
+    wait_chunk(staged - NS);
+    return slot(staged);
+  }
+  __device__ void staged_one() {
+    tc::cp_async_commit();
+    ++staged;
+  }
+  // Thread 0 issues the MMAs of the oldest staged chunk once its copies have
+  // landed (the copies of the `newer` chunks staged after it may be in flight).
   template <class F>
-  __device__ void issue(F fn) {
+  __device__ void issue(F fn, int newer) {
+    if (newer >= 2) tc::cp_async_wait<2>();
+    else if (newer == 1) tc::cp_async_wait<1>();
+    else tc::cp_async_wait<0>();
     tc::fence_async_smem();
     tc::tc_fence_before();
     __syncthreads();
     if (!failed && threadIdx.x == 0) {
       tc::tc_fence_after();
-      fn();
-      tc::mma_commit(bar + (g & 1));
+      fn(issued, slot(issued));
+      tc::mma_commit(bar + (issued % NS));
     }
-    ++g;
+    ++issued;
+  }
+  // Stages and issues n chunks: stage(i, slot) fills chunk i's slot,
+  // mma(i, slot) issues its MMAs (thread 0).
+  template <class S, class M>
+  __device__ void run(int n, S stage, M mma) {
+    constexpr int D = NS - 1 < 2 ? NS - 1 : 2;          // chunks in flight behind the MMAs
+    for (int i = 0; i < n; ++i) {
+      stage(i, acquire());
+      staged_one();
+      if (i >= D) issue([&](int, uint8_t* p) { mma(i - D, p); }, D);
+    }
+    for (int j = n - D > 0 ? n - D : 0; j < n; ++j)
+      issue([&](int, uint8_t* p) { mma(j, p); }, n - 1 - j);
   }
   // Every MMA issued so far has completed (their results are readable).
   __device__ void wait_all() {
-    if (g > 0 && !failed) {
-      const bool ok = tc::mbar_wait(bar + ((g - 1) & 1), ((g - 1) >> 1) & 1);
-      if (__syncthreads_or(ok ? 0 : 1)) failed = true;
-    }
+    wait_chunk(issued - 1);
     tc::tc_fence_after();
   }
 };
@@ -98,9 +127,9 @@ __device__ __forceinline__ uint32_t setup(uint64_t* bars, int nbars, uint32_t* t
 }
 
 // Shared epilogue: on a failed wait, drain the issued MMAs before TMEM is freed.
-__device__ __forceinline__ void teardown(Ring& ring, uint64_t* bar_drain, uint32_t tmem,
+__device__ __forceinline__ void teardown(bool failed, uint64_t* bar_drain, uint32_t tmem,
                                          uint32_t ncols, int* dev_status) {
-  if (ring.failed && threadIdx.x == 0) {
+  if (failed && threadIdx.x == 0) {
     report(dev_status, DARK_ERR_TIMEOUT);
     tc::drain_mmas(bar_drain);
   }
@@ -117,12 +146,63 @@ __device__ __forceinline__ uint32_t lane_addr(uint32_t tmem, int col) {
   return tmem + ((uint32_t)((threadIdx.x >> 5) & 3) * 32u << 16) + (uint32_t)col;
 }
 
-__device__ __forceinline__ float4 ld_bf16x4(const __nv_bfloat16* p) {
+// Four consecutive bf16 values as floats; `vec`: the address is 8-byte aligned.
+__device__ __forceinline__ float4 ld_bf16x4(const __nv_bfloat16* p, bool vec) {
+  if (vec) {
+    const uint2 u = *reinterpret_cast<const uint2*>(p);
+    const float2 lo = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.x));
+    const float2 hi = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.y));
+    return make_float4(lo.x, lo.y, hi.x, hi.y);
+  }
   return make_float4(__bfloat162float(p[0]), __bfloat162float(p[1]), __bfloat162float(p[2]),
                      __bfloat162float(p[3]));
 }
 __device__ __forceinline__ void st_f4(float* p, float a, float b, float c, float d) {
   *reinterpret_cast<float4*>(p) = make_float4(a, b, c, d);
+}
+__device__ __forceinline__ void st_bf16x4(__nv_bfloat16* p, float4 v, bool vec) {
+  const __nv_bfloat162 lo = __floats2bfloat162_rn(v.x, v.y), hi = __floats2bfloat162_rn(v.z, v.w);
+  if (vec) {
+    uint2 u;
+    u.x = *reinterpret_cast<const uint32_t*>(&lo);
+    u.y = *reinterpret_cast<const uint32_t*>(&hi);
+    *reinterpret_cast<uint2*>(p) = u;
+  } else {
+    p[0] = lo.x;
+    p[1] = lo.y;
+    p[2] = hi.x;
+    p[3] = hi.y;
+  }
+}
+
+// Epilogue blocks of 128 rows x W fp32 values in shared memory (row stride
+// W + 4 floats, so that one float4 per row and thread meets no bank conflict):
+// each epilogue thread fills its own row, then all threads move the block
+// row by row so that global accesses are coalesced.
+constexpr int kPad = 4;
+// store(row, c, v): values 4c..4c+3 of the block's row.
+template <int W, class S>
+__device__ __forceinline__ void block_out(const float* buf, S store) {
+  constexpr int per = W / 4;
+  __syncthreads();
+  for (int i = threadIdx.x; i < kTT * per; i += blockDim.x) {
+    const int row = i / per, c = i % per;
+    store(row, c, *reinterpret_cast<const float4*>(buf + row * (W + kPad) + 4 * c));
+  }
+  __syncthreads();
+}
+// Copies rows in: src(row, c) is the 16-byte aligned source of values
+// 4c..4c+3 of the row, or nullptr for zeros (then `any` stands in, unread).
+template <int W, class S>
+__device__ __forceinline__ void block_in(float* buf, S src, const float* any) {
+  constexpr int per = W / 4;
+  for (int i = threadIdx.x; i < kTT * per; i += blockDim.x) {
+    const int row = i / per, c = i % per;
+    const float* p = src(row, c);
+    tc::cp_async16(tc::smem_u32(buf + row * (W + kPad) + 4 * c), p != nullptr ? p : any,
+                   p != nullptr);
+  }
+  tc::cp_async_commit();
 }
 
 // ---------------------------------------------------------------------------
@@ -140,10 +220,15 @@ struct FeatArgs {
   int heads_w, m, r, d, H, L;
   const uint8_t* mask;
   int stabilise;
+  int xvec;                       // q, k rows 8-byte aligned (4-value loads)
   float *phiq, *phik, *pbot;
   int* ck;
   int* dev_status;
 };
+
+__host__ __device__ inline uint32_t feat_slot_bytes(int m, int r) {
+  return km_bytes(kTT) + km_bytes(round_up(m + r, 32));
+}
 
 __global__ void __launch_bounds__(kThr, 1) tbf_features_kernel(FeatArgs a) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -152,84 +237,71 @@ __global__ void __launch_bounds__(kThr, 1) tbf_features_kernel(FeatArgs a) {
   const int t0 = blockIdx.x * kTT;
   const int m = a.m, r = a.r, d = a.d, L = a.L;
   const int nrow = side ? m + r : m;                          // W' rows = P columns
-  const uint32_t slot = km_bytes(kTT) + km_bytes(round_up(m + r, 32));
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + 2 * slot);
-  uint32_t* tslot = reinterpret_cast<uint32_t*>(bars + 4);
-  float* red = reinterpret_cast<float*>(tslot + 4);           // [2][128]
-  const uint32_t tmem = setup(bars, 3, tslot, 512);
-  Ring ring{smem, slot, bars, 0, false};
+  const uint32_t slot = feat_slot_bytes(m, r);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kFeatSlots * slot);   // slots, drain (7)
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(bars + 8);
+  float* red = reinterpret_cast<float*>(bars + 16);                        // [2][128]
+  const uint32_t tmem = setup(bars, 8, tslot, 512);
+  Ring<kFeatSlots> ring{smem, slot, bars, 0, 0, false};
   const __nv_bfloat16* x = (side ? a.xk : a.xq) + (int64_t)b * a.sb + (int64_t)h * a.sh;
   const float* wh = a.w + (size_t)(a.heads_w == 1 ? 0 : h) * (m + r) * d;
 
-  for (int kc = 0; kc < d / 32; ++kc) {
-    uint8_t* s = ring.acquire();
-    tc::stage_km(s, kTT, [&](int row, int c) {
-      const int t = t0 + row;
-      return t < L ? ld_bf16x4(x + (int64_t)t * a.sl + kc * 32 + 4 * c) : make_float4(0.f, 0.f, 0.f, 0.f);
-    });
-    tc::stage_km(s + km_bytes(kTT), round_up(nrow, 32), [&](int row, int c) {
-      return row < nrow ? *reinterpret_cast<const float4*>(wh + (size_t)row * d + kc * 32 + 4 * c)
-                        : make_float4(0.f, 0.f, 0.f, 0.f);
-    });
-    ring.issue([&] {
-      const uint32_t sa = tc::smem_u32(s), sw = sa + km_bytes(kTT);
-      for (int c0 = 0; c0 < nrow; c0 += 256) {
-        const int n = nrow - c0 < 256 ? nrow - c0 : 256;
-        tc::mma_chunk(tmem + c0, sa, false, sw + (uint32_t)c0 * 128u, false, n, kc > 0);
-      }
-    });
-  }
+  ring.run(
+      d / 32,
+      [&](int kc, uint8_t* s) {
+        tc::stage_km_async(s + km_bytes(kTT), round_up(nrow, 32), [&](int row, int c) {
+          return row < nrow ? wh + (size_t)row * d + kc * 32 + 4 * c : nullptr;
+        }, wh);
+        tc::stage_km(s, kTT, [&](int row, int c) {
+          const int t = t0 + row;
+          return t < L ? ld_bf16x4(x + (int64_t)t * a.sl + kc * 32 + 4 * c, a.xvec)
+                       : make_float4(0.f, 0.f, 0.f, 0.f);
+        });
+      },
+      [&](int kc, uint8_t* s) {
+        const uint32_t sa = tc::smem_u32(s), sw = sa + km_bytes(kTT);
+        for (int c0 = 0; c0 < nrow; c0 += 256) {
+          const int n = nrow - c0 < 256 ? nrow - c0 : 256;
+          tc::mma_chunk(tmem + c0, sa, false, sw + (uint32_t)c0 * 128u, false, n, kc > 0);
+        }
+      });
   ring.wait_all();
 
   // epilogue: warps w and w + 4 share TMEM lanes 32 (w % 4) .. +31, each
-  // taking half of the columns; row statistics are combined through `red`.
+  // taking half of a block's columns; row statistics are combined through
+  // `red`, outputs leave through shared memory (the ring is idle now).
   const int q = (threadIdx.x >> 5) & 3, hf = threadIdx.x >> 7;
   const int row = q * 32 + (threadIdx.x & 31), t = t0 + row;
   const bool in = t < L;
-  float* dst = (side ? a.phik : a.phiq) + ((size_t)bh * L + (in ? t : 0)) * m;
-  const int half = m / 2;
+  float* buf = reinterpret_cast<float*>(smem);
+  float* dst = (side ? a.phik : a.phiq) + (size_t)bh * L * m;
+  auto store_rows = [&](float* base, int stride, int c0) {
+    return [=](int rr, int c, float4 v) {
+      if (t0 + rr < L) *reinterpret_cast<float4*>(base + (size_t)(t0 + rr) * stride + c0 + 4 * c) = v;
+    };
+  };
+  float rowc = 0.f;
   if (side) {
-    // key norm |P_bot|^2 and P_bot itself
+    // P_bot (kept for the key coefficients) and the key norm |P_bot|^2
     float nrm = 0.f;
-    float* pb = a.pbot + ((size_t)bh * L + (in ? t : 0)) * r;
-    for (int c0 = hf * (r / 2); c0 < (hf + 1) * (r / 2); c0 += 16) {
+    float* pb = a.pbot + (size_t)bh * L * r;
+    for (int c0 = 0; c0 < r; c0 += 32) {
       float v[16];
-      tc::tmem_ld16(lane_addr(tmem, m + c0), v);
+      tc::tmem_ld16(lane_addr(tmem, m + c0 + hf * 16), v);
+      float* o = buf + row * (32 + kPad) + hf * 16;
 #pragma unroll
       for (int j = 0; j < 16; ++j) nrm = fmaf(v[j], v[j], nrm);
-      if (in)
 #pragma unroll
-        for (int j = 0; j < 16; j += 4) st_f4(pb + c0 + j, v[j], v[j + 1], v[j + 2], v[j + 3]);
+      for (int j = 0; j < 16; j += 4) st_f4(o + j, v[j], v[j + 1], v[j + 2], v[j + 3]);
+      block_out<32>(buf, store_rows(pb, r, c0));
     }
     red[hf * kTT + row] = nrm;
     __syncthreads();
-    const float rowc = red[row] + red[kTT + row] + 0.5f * log2f((float)m);
-    const bool ok = a.mask == nullptr || (in && a.mask[(size_t)b * L + t] != 0);
-    float kmax = -INFINITY;
-    for (int c0 = hf * half; c0 < (hf + 1) * half; c0 += 32) {
-      float v[32];
-      tc::tmem_ld32(lane_addr(tmem, c0), v);
-#pragma unroll
-      for (int j = 0; j < 32; ++j) {
-        const float e = v[j] - rowc;
-        if (a.stabilise) {
-          v[j] = ok ? e : -INFINITY;
-          kmax = fmaxf(kmax, v[j]);
-        } else {
-          v[j] = ok ? exp2f(e) : 0.f;
-        }
-      }
-      if (in)
-#pragma unroll
-        for (int j = 0; j < 32; j += 4) st_f4(dst + c0 + j, v[j], v[j + 1], v[j + 2], v[j + 3]);
-    }
-    if (a.stabilise) {
-      kmax = warp_max(in ? kmax : -INFINITY);
-      if ((threadIdx.x & 31) == 0 && kmax > -INFINITY) atomicMax(a.ck + bh, float_to_ordered(kmax));
-    }
+    rowc = red[row] + red[kTT + row] + 0.5f * log2f((float)m);
   } else {
+    // queries: exponents relative to the row maximum
     float mx = -INFINITY;
-    for (int c0 = hf * half; c0 < (hf + 1) * half; c0 += 32) {
+    for (int c0 = hf * 32; c0 < m; c0 += 64) {
       float v[32];
       tc::tmem_ld32(lane_addr(tmem, c0), v);
 #pragma unroll
@@ -237,18 +309,33 @@ __global__ void __launch_bounds__(kThr, 1) tbf_features_kernel(FeatArgs a) {
     }
     red[hf * kTT + row] = mx;
     __syncthreads();
-    mx = fmaxf(red[row], red[kTT + row]);
-    for (int c0 = hf * half; c0 < (hf + 1) * half; c0 += 32) {
-      float v[32];
-      tc::tmem_ld32(lane_addr(tmem, c0), v);
-#pragma unroll
-      for (int j = 0; j < 32; ++j) v[j] = exp2f(v[j] - mx);
-      if (in)
-#pragma unroll
-        for (int j = 0; j < 32; j += 4) st_f4(dst + c0 + j, v[j], v[j + 1], v[j + 2], v[j + 3]);
-    }
+    rowc = fmaxf(red[row], red[kTT + row]);
   }
-  teardown(ring, bars + 2, tmem, 512, a.dev_status);
+  const bool ok = !side || a.mask == nullptr || (in && a.mask[(size_t)b * L + t] != 0);
+  float kmax = -INFINITY;
+  for (int c0 = 0; c0 < m; c0 += 64) {
+    float v[32];
+    tc::tmem_ld32(lane_addr(tmem, c0 + hf * 32), v);
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+      const float e = v[j] - rowc;
+      if (side && a.stabilise) {
+        v[j] = ok ? e : -INFINITY;
+        kmax = fmaxf(kmax, v[j]);
+      } else {
+        v[j] = ok ? exp2f(e) : 0.f;
+      }
+    }
+    float* o = buf + row * (64 + kPad) + hf * 32;
+#pragma unroll
+    for (int j = 0; j < 32; j += 4) st_f4(o + j, v[j], v[j + 1], v[j + 2], v[j + 3]);
+    block_out<64>(buf, store_rows(dst, m, c0));
+  }
+  if (side && a.stabilise) {
+    kmax = warp_max(in ? kmax : -INFINITY);
+    if ((threadIdx.x & 31) == 0 && kmax > -INFINITY) atomicMax(a.ck + bh, float_to_ordered(kmax));
+  }
+  teardown(ring.failed, bars + 7, tmem, 512, a.dev_status);
 }
 
 // ---------------------------------------------------------------------------
@@ -261,6 +348,7 @@ struct StateArgs {
   const float* X;                 // [B*H][L][m]
   const __nv_bfloat16* v;         // keys: values
   int64_t vb, vh, vl;
+  int vvec;                       // v rows 8-byte aligned
   const float* wrow;              // queries: [B*H][L][dp]
   int m, d, dp, H, L, nt;
   float* st;                      // [B*H][nt][m][dp]
@@ -275,55 +363,73 @@ __global__ void __launch_bounds__(kThr, 1) tbf_state_kernel(StateArgs a) {
   const int t0 = c * kTT, m = a.m, d = a.d, dp = a.dp, L = a.L;
   const int mt = (m + 127) / 128, dn = round_up(d + 1, 16);
   const uint32_t abytes = mn_bytes(mt * 128), slot = abytes + mn_bytes(dp);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + 2 * slot);
-  uint32_t* tslot = reinterpret_cast<uint32_t*>(bars + 4);
-  const uint32_t tmem = setup(bars, 3, tslot, 512);
-  Ring ring{smem, slot, bars, 0, false};
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kStateSlots * slot);
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(bars + 8);
+  const uint32_t tmem = setup(bars, 8, tslot, 512);
+  Ring<kStateSlots> ring{smem, slot, bars, 0, 0, false};
   const float* X = a.X + (size_t)bh * L * m;
   const __nv_bfloat16* vh = a.v + (int64_t)b * a.vb + (int64_t)h * a.vh;
   const float* wr = a.wrow + (size_t)bh * L * dp;
 
-  for (int kc = 0; kc < kTT / 32; ++kc) {
-    uint8_t* s = ring.acquire();
-    tc::stage_mn(s, mt * 128, [&](int k, int cc) {
-      const int t = t0 + kc * 32 + k;
-      return (t < L && 4 * cc < m) ? *reinterpret_cast<const float4*>(X + (size_t)t * m + 4 * cc)
-                                   : make_float4(0.f, 0.f, 0.f, 0.f);
-    });
-    tc::stage_mn(s + abytes, dp, [&](int k, int cc) {
-      const int t = t0 + kc * 32 + k, e = 4 * cc;
-      if (t >= L) return make_float4(0.f, 0.f, 0.f, 0.f);
-      if constexpr (SIDE == 0) return *reinterpret_cast<const float4*>(wr + (size_t)t * dp + e);
-      float u[4];
-#pragma unroll
-      for (int j = 0; j < 4; ++j)
-        u[j] = e + j < d ? __bfloat162float(vh[(int64_t)t * a.vl + e + j]) : (e + j == d ? 1.f : 0.f);
-      return make_float4(u[0], u[1], u[2], u[3]);
-    });
-    ring.issue([&] {
-      const uint32_t sa = tc::smem_u32(s), sb = sa + abytes;
-      for (int i = 0; i < mt; ++i)
-        tc::mma_chunk(tmem + 256 * i, sa + i * 4 * tc::kMnBlockBytes, true, sb, true, dn, kc > 0);
-    });
-  }
+  ring.run(
+      kTT / 32,
+      [&](int kc, uint8_t* s) {
+        tc::stage_mn_async(s, mt * 128, [&](int k, int cc) -> const float* {
+          const int t = t0 + kc * 32 + k;
+          return (t < L && 4 * cc < m) ? X + (size_t)t * m + 4 * cc : nullptr;
+        }, X);
+        if constexpr (SIDE == 0) {
+          tc::stage_mn_async(s + abytes, dp, [&](int k, int cc) -> const float* {
+            const int t = t0 + kc * 32 + k;
+            return t < L ? wr + (size_t)t * dp + 4 * cc : nullptr;
+          }, wr);
+        } else {
+          tc::stage_mn(s + abytes, dp, [&](int k, int cc) {
+            const int t = t0 + kc * 32 + k, e = 4 * cc;
+            if (t >= L || e > d) return make_float4(0.f, 0.f, 0.f, 0.f);
+            if (e == d) return make_float4(1.f, 0.f, 0.f, 0.f);
+            return ld_bf16x4(vh + (int64_t)t * a.vl + e, a.vvec);
+          });
+        }
+      },
+      [&](int kc, uint8_t* s) {
+        const uint32_t sa = tc::smem_u32(s), sb = sa + abytes;
+        for (int i = 0; i < mt; ++i)
+          tc::mma_chunk(tmem + 256 * i, sa + i * 4 * tc::kMnBlockBytes, true, sb, true, dn,
+                        kc > 0);
+      });
   ring.wait_all();
-  // warps 0-3 read accumulator 0, warps 4-7 accumulator 1 (feature rows 128..)
+  // warps 0-3 read accumulator 0, warps 4-7 accumulator 1 (feature rows 128..);
+  // the rows [m][dp] (contiguous in the state array) leave through shared memory
   const int q = (threadIdx.x >> 5) & 3, acc = threadIdx.x >> 7;
   const int f = acc * 128 + q * 32 + (threadIdx.x & 31);
-  if (acc < mt) {
-    float* out = a.st + (((size_t)bh * a.nt + c) * m + (f < m ? f : 0)) * dp;
+  float* buf = reinterpret_cast<float*>(smem);           // [m][dp + 4]
+  const int ld = dp + kPad;
+  if (acc < mt && f < m) {
     for (int c0 = 0; c0 < dp; c0 += 16) {
       float v[16];
       if (c0 < dn) tc::tmem_ld16(lane_addr(tmem, 256 * acc + c0), v);
 #pragma unroll
       for (int j = 0; j < 16; ++j)
         if (c0 + j > d) v[j] = 0.f;
-      if (f < m)
 #pragma unroll
-        for (int j = 0; j < 16; j += 4) st_f4(out + c0 + j, v[j], v[j + 1], v[j + 2], v[j + 3]);
+      for (int j = 0; j < 16; j += 4) st_f4(buf + f * ld + c0 + j, v[j], v[j + 1], v[j + 2], v[j + 3]);
+    }
+  } else if (acc < mt) {
+    for (int c0 = 0; c0 < dn; c0 += 16) {   // the warp's loads are collective
+      float v[16];
+      tc::tmem_ld16(lane_addr(tmem, 256 * acc + c0), v);
     }
   }
-  teardown(ring, bars + 2, tmem, 512, a.dev_status);
+  __syncthreads();
+  float* out = a.st + ((size_t)bh * a.nt + c) * m * dp;
+  const int per = dp / 4;
+  for (int i = threadIdx.x; i < m * per; i += blockDim.x) {
+    const int rr = i / per, cc = i - rr * per;
+    *reinterpret_cast<float4*>(out + (size_t)rr * dp + 4 * cc) =
+        *reinterpret_cast<const float4*>(buf + rr * ld + 4 * cc);
+  }
+  teardown(ring.failed, bars + 7, tmem, 512, a.dev_status);
 }
 
 // ---------------------------------------------------------------------------
@@ -344,9 +450,11 @@ struct PassArgs {
   int64_t vb, vh, vl;
   const __nv_bfloat16* g;
   int64_t gb, gh, gl;
+  int vvec, gvec;                 // v / dout rows 8-byte aligned
   float* wrow;                    // [B*H][L][dp]
   __nv_bfloat16* dv;
   int64_t ob, oh, ol;
+  int ovec;                       // dv rows 8-byte aligned
   float* coef;                    // [B*H][L][m + r]
   const float* pbot;              // [B*H][L][r]
   int m, r, d, dp, H, L, nt, causal;
@@ -355,14 +463,14 @@ struct PassArgs {
 
 __host__ __device__ inline uint32_t pass_slot_bytes(int m, int dp, int causal) {
   const uint32_t p1 = km_bytes(kTT) + mn_bytes(dp) + (causal ? km_bytes(kTT) : 0);
-  const uint32_t p2 = km_bytes(kTT) + km_bytes(m) + (causal ? km_bytes(kTT) : 0);
-  const uint32_t p3 = mn_bytes(m);
+  const uint32_t p2 = km_bytes(kTT) + km_bytes(m);      // P and the state rows
+  const uint32_t p3 = mn_bytes(m);                      // feature rows (diagonal)
   uint32_t s = p1 > p2 ? p1 : p2;
   return s > p3 ? s : p3;
 }
 __host__ __device__ inline uint32_t pass_smem_bytes(int m, int dp, int causal) {
-  return 1024 + 2 * pass_slot_bytes(m, dp, causal) + (causal ? 4 * km_bytes(kTT) : 0) + 64 +
-         2 * kTT * 4;
+  return 1024 + kPassSlots * pass_slot_bytes(m, dp, causal) + (causal ? 4 * km_bytes(kTT) : 0) +
+         kTailBytes;
 }
 
 template <int SIDE>
@@ -373,13 +481,13 @@ __global__ void __launch_bounds__(kThr, 1) tbf_pass_kernel(PassArgs a) {
   const int t0 = c * kTT, m = a.m, r = a.r, d = a.d, dp = a.dp, L = a.L;
   const int causal = a.causal, dn = round_up(d + 1, 16);
   const uint32_t slot = pass_slot_bytes(m, dp, causal);
-  uint8_t* scores = smem + 2 * slot;                              // 4 K-major chunks
+  uint8_t* scores = smem + kPassSlots * slot;                     // 4 K-major chunks
   uint64_t* bars = reinterpret_cast<uint64_t*>(scores + (causal ? 4 * km_bytes(kTT) : 0));
-  uint32_t* tslot = reinterpret_cast<uint32_t*>(bars + 4);
-  float* red = reinterpret_cast<float*>(tslot + 4);               // [2][128]
-  const uint32_t tmem = setup(bars, 3, tslot, 512);
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(bars + 8);
+  float* red = reinterpret_cast<float*>(bars + 16);               // [2][128]
+  const uint32_t tmem = setup(bars, 8, tslot, 512);
   const uint32_t tD = tmem, tS = tmem + 256;
-  Ring ring{smem, slot, bars, 0, false};
+  Ring<kPassSlots> ring{smem, slot, bars, 0, 0, false};
 
   const size_t rowbase = (size_t)bh * L;
   const float* X = (SIDE == 0 ? a.phiq : a.phik) + rowbase * m;
@@ -389,22 +497,51 @@ __global__ void __launch_bounds__(kThr, 1) tbf_pass_kernel(PassArgs a) {
   const __nv_bfloat16* vh = a.v + (int64_t)b * a.vb + (int64_t)h * a.vh;
   // [v | 1 | 0 ...] at token t, columns e .. e + 3
   auto vone4 = [&](int t, int e) -> float4 {
-    if (t >= L) return make_float4(0.f, 0.f, 0.f, 0.f);
-    float u[4];
-#pragma unroll
-    for (int j = 0; j < 4; ++j)
-      u[j] = e + j < d ? __bfloat162float(vh[(int64_t)t * a.vl + e + j]) : (e + j == d ? 1.f : 0.f);
-    return make_float4(u[0], u[1], u[2], u[3]);
+    if (t >= L || e > d) return make_float4(0.f, 0.f, 0.f, 0.f);
+    if (e == d) return make_float4(1.f, 0.f, 0.f, 0.f);
+    return ld_bf16x4(vh + (int64_t)t * a.vl + e, a.vvec);
   };
-  auto wrow4 = [&](int t, int e) -> float4 {
-    return t < L ? *reinterpret_cast<const float4*>(wr + (size_t)t * dp + e) : make_float4(0.f, 0.f, 0.f, 0.f);
+  // Staging of the tile's operands. [v | 1] is converted through registers;
+  // fp32 rows ([w | -c], features, states) are copied asynchronously.
+  auto v_km = [&](uint8_t* dst, int e0) {        // rows: tile tokens, K: columns e0..
+    tc::stage_km(dst, kTT, [&](int rr, int cc) { return vone4(t0 + rr, e0 + 4 * cc); });
   };
-  // U rows of the tile: [v | 1] (queries) or [w | -c] (keys)
-  auto u4 = [&](int t, int e) -> float4 { return SIDE == 0 ? vone4(t, e) : wrow4(t, e); };
-  // P rows of the tile: [w | -c] (queries) or [v | 1] (keys)
-  auto p4 = [&](int t, int e) -> float4 { return SIDE == 0 ? wrow4(t, e) : vone4(t, e); };
-  auto feat4 = [&](const float* F, int t, int f) -> float4 {
-    return t < L ? *reinterpret_cast<const float4*>(F + (size_t)t * m + f) : make_float4(0.f, 0.f, 0.f, 0.f);
+  auto w_km = [&](uint8_t* dst, int e0) {
+    tc::stage_km_async(dst, kTT, [&](int rr, int cc) -> const float* {
+      const int tt = t0 + rr;
+      return tt < L ? wr + (size_t)tt * dp + e0 + 4 * cc : nullptr;
+    }, wr);
+  };
+  auto v_mn = [&](uint8_t* dst, int tk0) {       // K: tokens tk0.., MN: columns
+    tc::stage_mn(dst, dp, [&](int k, int cc) { return vone4(tk0 + k, 4 * cc); });
+  };
+  auto w_mn = [&](uint8_t* dst, int tk0) {
+    tc::stage_mn_async(dst, dp, [&](int k, int cc) -> const float* {
+      const int tt = tk0 + k;
+      return tt < L ? wr + (size_t)tt * dp + 4 * cc : nullptr;
+    }, wr);
+  };
+  auto feat_km = [&](uint8_t* dst, const float* F, int f0) {   // rows: tokens, K: features
+    tc::stage_km_async(dst, kTT, [&](int rr, int cc) -> const float* {
+      const int tt = t0 + rr;
+      return tt < L ? F + (size_t)tt * m + f0 + 4 * cc : nullptr;
+    }, F);
+  };
+  auto feat_mn = [&](uint8_t* dst, const float* F, int tk0) {  // K: tokens, MN: features
+    tc::stage_mn_async(dst, m, [&](int k, int cc) -> const float* {
+      const int tt = tk0 + k;
+      return tt < L ? F + (size_t)tt * m + 4 * cc : nullptr;
+    }, F);
+  };
+  // U = [v | 1] (queries) or [w | -c] (keys); P the other one
+  auto u_mn = [&](uint8_t* dst, int tk0) {
+    if constexpr (SIDE == 0) v_mn(dst, tk0); else w_mn(dst, tk0);
+  };
+  auto u_km = [&](uint8_t* dst, int e0) {
+    if constexpr (SIDE == 0) v_km(dst, e0); else w_km(dst, e0);
+  };
+  auto p_km = [&](uint8_t* dst, int e0) {
+    if constexpr (SIDE == 0) w_km(dst, e0); else v_km(dst, e0);
   };
 
   const int q = (threadIdx.x >> 5) & 3, hf = threadIdx.x >> 7;
@@ -434,153 +571,213 @@ __global__ void __launch_bounds__(kThr, 1) tbf_pass_kernel(PassArgs a) {
   };
 
   // ---- phase 1: D = X state + tri(X Y^T) U ----
-  for (int fc = 0; fc < m / 32; ++fc) {
-    uint8_t* s = ring.acquire();
-    tc::stage_km(s, kTT, [&](int rr, int cc) { return feat4(X, t0 + rr, fc * 32 + 4 * cc); });
-    tc::stage_mn(s + km_bytes(kTT), dp, [&](int k, int cc) {
-      return *reinterpret_cast<const float4*>(st + (size_t)(fc * 32 + k) * dp + 4 * cc);
-    });
-    if (causal)
-      tc::stage_km(s + km_bytes(kTT) + mn_bytes(dp), kTT,
-                   [&](int rr, int cc) { return feat4(Y, t0 + rr, fc * 32 + 4 * cc); });
-    ring.issue([&] {
-      const uint32_t sa = tc::smem_u32(s);
-      tc::mma_chunk(tD, sa, false, sa + km_bytes(kTT), true, dn, fc > 0);
-      if (causal)
-        tc::mma_chunk(tS, sa, false, sa + km_bytes(kTT) + mn_bytes(dp), false, kTT, fc > 0);
-    });
-  }
+  ring.run(
+      m / 32,
+      [&](int fc, uint8_t* s) {
+        feat_km(s, X, fc * 32);
+        tc::stage_mn_async(s + km_bytes(kTT), dp, [&](int k, int cc) -> const float* {
+          return st + (size_t)(fc * 32 + k) * dp + 4 * cc;
+        }, st);
+        if (causal) feat_km(s + km_bytes(kTT) + mn_bytes(dp), Y, fc * 32);
+      },
+      [&](int fc, uint8_t* s) {
+        const uint32_t sa = tc::smem_u32(s);
+        tc::mma_chunk(tD, sa, false, sa + km_bytes(kTT), true, dn, fc > 0);
+        if (causal)
+          tc::mma_chunk(tS, sa, false, sa + km_bytes(kTT) + mn_bytes(dp), false, kTT, fc > 0);
+      });
   if (causal) {
     ring.wait_all();
     scores_to_smem();
-    for (int kc = 0; kc < kTT / 32; ++kc) {
-      uint8_t* s = ring.acquire();
-      tc::stage_mn(s, dp, [&](int k, int cc) { return u4(t0 + kc * 32 + k, 4 * cc); });
-      ring.issue([&] {
-        tc::mma_chunk(tD, tc::smem_u32(scores + kc * km_bytes(kTT)), false, tc::smem_u32(s), true,
-                      dn, true);
-      });
-    }
+    ring.run(
+        kTT / 32, [&](int kc, uint8_t* s) { u_mn(s, t0 + kc * 32); },
+        [&](int kc, uint8_t* s) {
+          tc::mma_chunk(tD, tc::smem_u32(scores + kc * km_bytes(kTT)), false, tc::smem_u32(s),
+                        true, dn, true);
+        });
   }
   ring.wait_all();
 
-  // ---- epilogue of phase 1 ----
+  // ---- epilogue of phase 1 (rows through shared memory; the ring is idle) ----
   const int dh = d / 2;
+  float* buf = reinterpret_cast<float*>(smem);
   if (SIDE == 0) {
-    const __nv_bfloat16* gh = a.g + (int64_t)b * a.gb + (int64_t)h * a.gh + (int64_t)(in ? t : 0) * a.gl;
+    // g rows in, then P = [g / den | -(g . num) / den^2 | 0 ...] in their place
+    const int ld = dp + kPad, per = d / 4;
+    const __nv_bfloat16* gb = a.g + (int64_t)b * a.gb + (int64_t)h * a.gh;
+    for (int i = threadIdx.x; i < kTT * per; i += blockDim.x) {
+      const int rr = i / per, cc = i - rr * per, tt = t0 + rr;
+      const float4 g4 = tt < L ? ld_bf16x4(gb + (int64_t)tt * a.gl + 4 * cc, a.gvec)
+                               : make_float4(0.f, 0.f, 0.f, 0.f);
+      *reinterpret_cast<float4*>(buf + rr * ld + 4 * cc) = g4;
+    }
+    __syncthreads();
     const float den = tc::tmem_ld1(lane_addr(tD, d));
+    float* gr = buf + row * ld;
     float go = 0.f;
     for (int c0 = hf * dh; c0 < (hf + 1) * dh; c0 += 16) {
       float v[16];
       tc::tmem_ld16(lane_addr(tD, c0), v);
-      if (in)
 #pragma unroll
-        for (int j = 0; j < 16; ++j) go = fmaf(__bfloat162float(gh[c0 + j]), v[j], go);
+      for (int j = 0; j < 16; ++j) go = fmaf(gr[c0 + j], v[j], go);
     }
     red[hf * kTT + row] = go;
     __syncthreads();
     go = red[row] + red[kTT + row];
     const float inv = (in && den > 0.f) ? 1.f / den : 0.f;
     const float cc = go * inv * inv;
-    if (in) {
-      float* wt = wr + (size_t)t * dp;
-      for (int c0 = hf * dh; c0 < (hf + 1) * dh; c0 += 4) {
-        float p[4];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          p[j] = __bfloat162float(gh[c0 + j]) * inv;
-          if (!isfinite(p[j])) report(a.dev_status, DARK_ERR_NUMERIC);
-        }
-        st_f4(wt + c0, p[0], p[1], p[2], p[3]);
-      }
-      if (hf == 1) {
-        if (!isfinite(cc)) report(a.dev_status, DARK_ERR_NUMERIC);
-        for (int e = d; e < dp; e += 4) st_f4(wt + e, e == d ? -cc : 0.f, 0.f, 0.f, 0.f);
-      }
+    for (int c0 = hf * dh; c0 < (hf + 1) * dh; c0 += 4) {
+      float4 g4 = *reinterpret_cast<const float4*>(gr + c0);
+      g4.x *= inv; g4.y *= inv; g4.z *= inv; g4.w *= inv;
+      if (!(isfinite(g4.x) && isfinite(g4.y) && isfinite(g4.z) && isfinite(g4.w)))
+        report(a.dev_status, DARK_ERR_NUMERIC);
+      *reinterpret_cast<float4*>(gr + c0) = g4;
+    }
+    if (hf == 1) {
+      if (!isfinite(cc)) report(a.dev_status, DARK_ERR_NUMERIC);
+      for (int e = d; e < dp; e += 4) st_f4(gr + e, e == d ? -cc : 0.f, 0.f, 0.f, 0.f);
+    }
+    __syncthreads();
+    const int pw = dp / 4;
+    for (int i = threadIdx.x; i < kTT * pw; i += blockDim.x) {
+      const int rr = i / pw, c4 = i - rr * pw;
+      if (t0 + rr < L)
+        *reinterpret_cast<float4*>(wr + (size_t)(t0 + rr) * dp + 4 * c4) =
+            *reinterpret_cast<const float4*>(buf + rr * ld + 4 * c4);
     }
   } else {
-    __nv_bfloat16* dvh = a.dv + (int64_t)b * a.ob + (int64_t)h * a.oh + (int64_t)(in ? t : 0) * a.ol;
+    // dv rows out as bf16
+    const int ld = d + kPad, per = d / 4;
     for (int c0 = hf * dh; c0 < (hf + 1) * dh; c0 += 16) {
       float v[16];
       tc::tmem_ld16(lane_addr(tD, c0), v);
-      if (in)
 #pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          if (!isfinite(v[j])) report(a.dev_status, DARK_ERR_NUMERIC);
-          dvh[c0 + j] = __float2bfloat16_rn(v[j]);
-        }
+      for (int j = 0; j < 16; ++j)
+        if (in && !isfinite(v[j])) report(a.dev_status, DARK_ERR_NUMERIC);
+#pragma unroll
+      for (int j = 0; j < 16; j += 4) st_f4(buf + row * ld + c0 + j, v[j], v[j + 1], v[j + 2], v[j + 3]);
+    }
+    __syncthreads();
+    __nv_bfloat16* dvb = a.dv + (int64_t)b * a.ob + (int64_t)h * a.oh;
+    for (int i = threadIdx.x; i < kTT * per; i += blockDim.x) {
+      const int rr = i / per, c4 = i - rr * per;
+      if (t0 + rr < L)
+        st_bf16x4(dvb + (int64_t)(t0 + rr) * a.ol + 4 * c4,
+                  *reinterpret_cast<const float4*>(buf + rr * ld + 4 * c4), a.ovec);
     }
   }
   tc::tc_fence_before();
   __syncthreads();                // the P rows above are read back by the staging below
 
   // ---- phase 2: dphi(X) = P state^T + tri(P U^T) Y ----
-  for (int pc = 0; pc < dp / 32; ++pc) {
-    uint8_t* s = ring.acquire();
-    tc::stage_km(s, kTT, [&](int rr, int cc) { return p4(t0 + rr, pc * 32 + 4 * cc); });
-    tc::stage_km(s + km_bytes(kTT), m, [&](int f, int cc) {
-      return *reinterpret_cast<const float4*>(st + (size_t)f * dp + pc * 32 + 4 * cc);
-    });
-    if (causal)
-      tc::stage_km(s + km_bytes(kTT) + km_bytes(m), kTT,
-                   [&](int rr, int cc) { return u4(t0 + rr, pc * 32 + 4 * cc); });
-    ring.issue([&] {
-      const uint32_t sa = tc::smem_u32(s);
-      tc::mma_chunk(tD, sa, false, sa + km_bytes(kTT), false, m, pc > 0);
-      if (causal)
-        tc::mma_chunk(tS, sa, false, sa + km_bytes(kTT) + km_bytes(m), false, kTT, pc > 0);
-    });
-  }
+  if (causal)       // the diagonal tile's scores P U^T first
+    ring.run(
+        dp / 32,
+        [&](int pc, uint8_t* s) {
+          p_km(s, pc * 32);
+          u_km(s + km_bytes(kTT), pc * 32);
+        },
+        [&](int pc, uint8_t* s) {
+          const uint32_t sa = tc::smem_u32(s);
+          tc::mma_chunk(tS, sa, false, sa + km_bytes(kTT), false, kTT, pc > 0);
+        });
+  ring.run(
+      dp / 32,
+      [&](int pc, uint8_t* s) {
+        p_km(s, pc * 32);
+        tc::stage_km_async(s + km_bytes(kTT), m, [&](int f, int cc) -> const float* {
+          return st + (size_t)f * dp + pc * 32 + 4 * cc;
+        }, st);
+      },
+      [&](int pc, uint8_t* s) {
+        const uint32_t sa = tc::smem_u32(s);
+        tc::mma_chunk(tD, sa, false, sa + km_bytes(kTT), false, m, pc > 0);
+      });
   if (causal) {
     ring.wait_all();
     scores_to_smem();
-    for (int kc = 0; kc < kTT / 32; ++kc) {
-      uint8_t* s = ring.acquire();
-      tc::stage_mn(s, m, [&](int k, int cc) { return feat4(Y, t0 + kc * 32 + k, 4 * cc); });
-      ring.issue([&] {
-        tc::mma_chunk(tD, tc::smem_u32(scores + kc * km_bytes(kTT)), false, tc::smem_u32(s), true,
-                      m, true);
-      });
-    }
+    ring.run(
+        kTT / 32, [&](int kc, uint8_t* s) { feat_mn(s, Y, t0 + kc * 32); },
+        [&](int kc, uint8_t* s) {
+          tc::mma_chunk(tD, tc::smem_u32(scores + kc * km_bytes(kTT)), false, tc::smem_u32(s),
+                        true, m, true);
+        });
   }
   ring.wait_all();
 
   // ---- coef = ln2 X dphi; keys add -2 (sum_j coef_j) P_bot ----
-  const int mh = m / 2, rh = r / 2;
-  float* cf = a.coef + (rowbase + (in ? t : 0)) * (size_t)(m + r);
-  const float* xr = X + (size_t)(in ? t : 0) * m;
+  // 64-column blocks: the X rows come in by copies (double-buffered), the
+  // coefficients replace them and leave row by row
+  float* buf0 = reinterpret_cast<float*>(smem);
+  float* buf1 = buf0 + kTT * (64 + kPad);
+  float* cfb = a.coef + rowbase * (size_t)(m + r);
+  auto x_in = [&](int blk, float* bb) {
+    block_in<64>(bb, [&](int rr, int c) -> const float* {
+      const int tt = t0 + rr;
+      return tt < L ? X + (size_t)tt * m + blk * 64 + 4 * c : nullptr;
+    }, X);
+  };
+  const int nb = m / 64;
+  x_in(0, buf0);
   float rs = 0.f;
-  for (int c0 = hf * mh; c0 < (hf + 1) * mh; c0 += 32) {
-    float v[32];
-    tc::tmem_ld32(lane_addr(tD, c0), v);
-    if (in) {
-#pragma unroll
-      for (int j = 0; j < 32; j += 4) {
-        const float4 x4 = *reinterpret_cast<const float4*>(xr + c0 + j);
-        const float o0 = kLn2f * x4.x * v[j], o1 = kLn2f * x4.y * v[j + 1];
-        const float o2 = kLn2f * x4.z * v[j + 2], o3 = kLn2f * x4.w * v[j + 3];
-        rs += (o0 + o1) + (o2 + o3);
-        st_f4(cf + c0 + j, o0, o1, o2, o3);
-      }
+  for (int blk = 0; blk < nb; ++blk) {
+    float* cur = (blk & 1) ? buf1 : buf0;
+    if (blk + 1 < nb) {
+      x_in(blk + 1, (blk & 1) ? buf0 : buf1);
+      tc::cp_async_wait<1>();
+    } else {
+      tc::cp_async_wait<0>();
     }
+    __syncthreads();
+    float v[32];
+    tc::tmem_ld32(lane_addr(tD, blk * 64 + hf * 32), v);
+    float* xr = cur + row * (64 + kPad) + hf * 32;
+#pragma unroll
+    for (int j = 0; j < 32; j += 4) {
+      const float4 x4 = *reinterpret_cast<const float4*>(xr + j);
+      const float o0 = kLn2f * x4.x * v[j], o1 = kLn2f * x4.y * v[j + 1];
+      const float o2 = kLn2f * x4.z * v[j + 2], o3 = kLn2f * x4.w * v[j + 3];
+      rs += (o0 + o1) + (o2 + o3);
+      st_f4(xr + j, o0, o1, o2, o3);
+    }
+    block_out<64>(cur, [&](int rr, int c, float4 val) {
+      if (t0 + rr < L)
+        *reinterpret_cast<float4*>(cfb + (size_t)(t0 + rr) * (m + r) + blk * 64 + 4 * c) = val;
+    });
   }
   if (SIDE == 1) {
     red[hf * kTT + row] = rs;
     __syncthreads();
     rs = red[row] + red[kTT + row];
-  }
-  if (in) {
-    const float* pb = a.pbot + (rowbase + t) * (size_t)r;
-    for (int j = hf * rh; j < (hf + 1) * rh; j += 4) {
-      if (SIDE == 1) {
-        const float4 p = *reinterpret_cast<const float4*>(pb + j);
-        st_f4(cf + m + j, -2.f * rs * p.x, -2.f * rs * p.y, -2.f * rs * p.z, -2.f * rs * p.w);
-      } else {
-        st_f4(cf + m + j, 0.f, 0.f, 0.f, 0.f);
+    const float* pb = a.pbot + rowbase * (size_t)r;
+    for (int c0 = 0; c0 < r; c0 += 32) {
+      block_in<32>(buf0, [&](int rr, int c) -> const float* {
+        const int tt = t0 + rr;
+        return tt < L ? pb + (size_t)tt * r + c0 + 4 * c : nullptr;
+      }, pb);
+      tc::cp_async_wait<0>();
+      __syncthreads();
+      float* pr = buf0 + row * (32 + kPad) + hf * 16;
+#pragma unroll
+      for (int j = 0; j < 16; j += 4) {
+        const float4 p4 = *reinterpret_cast<const float4*>(pr + j);
+        st_f4(pr + j, -2.f * rs * p4.x, -2.f * rs * p4.y, -2.f * rs * p4.z, -2.f * rs * p4.w);
       }
+      block_out<32>(buf0, [&](int rr, int c, float4 val) {
+        if (t0 + rr < L)
+          *reinterpret_cast<float4*>(cfb + (size_t)(t0 + rr) * (m + r) + m + c0 + 4 * c) = val;
+      });
+    }
+  } else {
+    // the norm part of the query coefficients is zero
+    const int per = r / 4;
+    for (int i = threadIdx.x; i < kTT * per; i += blockDim.x) {
+      const int rr = i / per, c4 = i - rr * per;
+      if (t0 + rr < L)
+        st_f4(cfb + (size_t)(t0 + rr) * (m + r) + m + 4 * c4, 0.f, 0.f, 0.f, 0.f);
     }
   }
-  teardown(ring, bars + 2, tmem, 512, a.dev_status);
+  teardown(ring.failed, bars + 7, tmem, 512, a.dev_status);
 }
 
 // ---------------------------------------------------------------------------
@@ -593,6 +790,7 @@ struct DxArgs {
   int heads_w, m, r, d, H, L;
   __nv_bfloat16 *dq, *dk;
   int64_t ob, oh, ol;
+  int ovec;                       // dq, dk rows 8-byte aligned
   int* dev_status;
 };
 
@@ -602,44 +800,52 @@ __global__ void __launch_bounds__(kThr) tbf_dx_kernel(DxArgs a) {
   const int side = blockIdx.z, bh = blockIdx.y, b = bh / a.H, h = bh % a.H;
   const int t0 = blockIdx.x * kTT, m = a.m, r = a.r, d = a.d, L = a.L, mr = m + r;
   const uint32_t slot = km_bytes(kTT) + mn_bytes(d);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + 2 * slot);
-  uint32_t* tslot = reinterpret_cast<uint32_t*>(bars + 4);
-  const uint32_t tmem = setup(bars, 3, tslot, 128);
-  Ring ring{smem, slot, bars, 0, false};
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kGemmSlots * slot);
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(bars + 8);
+  const uint32_t tmem = setup(bars, 8, tslot, 128);
+  Ring<kGemmSlots> ring{smem, slot, bars, 0, 0, false};
   const float* cf = (side ? a.cfk : a.cfq) + (size_t)bh * L * mr;
   const float* wh = a.w + (size_t)(a.heads_w == 1 ? 0 : h) * mr * d;
   const int kend = side ? mr : m;
-  for (int kc = 0; kc < kend / 32; ++kc) {
-    uint8_t* s = ring.acquire();
-    tc::stage_km(s, kTT, [&](int rr, int cc) {
-      const int t = t0 + rr;
-      return t < L ? *reinterpret_cast<const float4*>(cf + (size_t)t * mr + kc * 32 + 4 * cc)
-                   : make_float4(0.f, 0.f, 0.f, 0.f);
-    });
-    tc::stage_mn(s + km_bytes(kTT), d, [&](int k, int cc) {
-      return *reinterpret_cast<const float4*>(wh + (size_t)(kc * 32 + k) * d + 4 * cc);
-    });
-    ring.issue([&] {
-      const uint32_t sa = tc::smem_u32(s);
-      tc::mma_chunk(tmem, sa, false, sa + km_bytes(kTT), true, d, kc > 0);
-    });
-  }
+  ring.run(
+      kend / 32,
+      [&](int kc, uint8_t* s) {
+        tc::stage_km_async(s, kTT, [&](int rr, int cc) -> const float* {
+          const int t = t0 + rr;
+          return t < L ? cf + (size_t)t * mr + kc * 32 + 4 * cc : nullptr;
+        }, cf);
+        tc::stage_mn_async(s + km_bytes(kTT), d, [&](int k, int cc) -> const float* {
+          return wh + (size_t)(kc * 32 + k) * d + 4 * cc;
+        }, wh);
+      },
+      [&](int kc, uint8_t* s) {
+        const uint32_t sa = tc::smem_u32(s);
+        tc::mma_chunk(tmem, sa, false, sa + km_bytes(kTT), true, d, kc > 0);
+      });
   ring.wait_all();
   const int q = (threadIdx.x >> 5) & 3, hf = threadIdx.x >> 7;
   const int row = q * 32 + (threadIdx.x & 31), t = t0 + row;
-  __nv_bfloat16* out = (side ? a.dk : a.dq) + (int64_t)b * a.ob + (int64_t)h * a.oh +
-                       (int64_t)(t < L ? t : 0) * a.ol;
+  // rows out through shared memory (the ring is idle), as bf16
+  float* buf = reinterpret_cast<float*>(smem);
+  const int ld = d + kPad, per = d / 4;
   for (int c0 = hf * (d / 2); c0 < (hf + 1) * (d / 2); c0 += 16) {
     float v[16];
     tc::tmem_ld16(lane_addr(tmem, c0), v);
-    if (t < L)
 #pragma unroll
-      for (int j = 0; j < 16; ++j) {
-        if (!isfinite(v[j])) report(a.dev_status, DARK_ERR_NUMERIC);
-        out[c0 + j] = __float2bfloat16_rn(v[j]);
-      }
+    for (int j = 0; j < 16; ++j)
+      if (t < L && !isfinite(v[j])) report(a.dev_status, DARK_ERR_NUMERIC);
+#pragma unroll
+    for (int j = 0; j < 16; j += 4) st_f4(buf + row * ld + c0 + j, v[j], v[j + 1], v[j + 2], v[j + 3]);
   }
-  teardown(ring, bars + 2, tmem, 128, a.dev_status);
+  __syncthreads();
+  __nv_bfloat16* out = (side ? a.dk : a.dq) + (int64_t)b * a.ob + (int64_t)h * a.oh;
+  for (int i = threadIdx.x; i < kTT * per; i += blockDim.x) {
+    const int rr = i / per, c4 = i - rr * per;
+    if (t0 + rr < L)
+      st_bf16x4(out + (int64_t)(t0 + rr) * a.ol + 4 * c4,
+                *reinterpret_cast<const float4*>(buf + rr * ld + 4 * c4), a.ovec);
+  }
+  teardown(ring.failed, bars + 7, tmem, 128, a.dev_status);
 }
 
 // dW'[hw] += sum over a token range of one (batch, head), both sides, of
@@ -651,6 +857,7 @@ struct DwArgs {
   int64_t sb, sh, sl;
   const float *cfq, *cfk;
   int m, r, d, H, L, heads_w, nsplit;
+  int xvec;                       // q, k rows 8-byte aligned
   float* G;                       // [heads_w][m + r][d]
   int* dev_status;
 };
@@ -663,44 +870,60 @@ __global__ void __launch_bounds__(kThr) tbf_dw_kernel(DwArgs a) {
   const int per = round_up((L + a.nsplit - 1) / a.nsplit, 32);
   const int tb = split * per, te = min(L, tb + per);
   const uint32_t slot = mn_bytes(128) + mn_bytes(d);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + 2 * slot);
-  uint32_t* tslot = reinterpret_cast<uint32_t*>(bars + 4);
-  const uint32_t tmem = setup(bars, 3, tslot, 128);
-  Ring ring{smem, slot, bars, 0, false};
-  for (int side = 0; side < 2; ++side) {
-    const __nv_bfloat16* x = (side ? a.xk : a.xq) + (int64_t)b * a.sb + (int64_t)h * a.sh;
-    const float* cf = (side ? a.cfk : a.cfq) + (size_t)bh * L * mr;
-    for (int k0 = tb; k0 < te; k0 += 32) {
-      uint8_t* s = ring.acquire();
-      tc::stage_mn(s, 128, [&](int k, int cc) {
-        const int t = k0 + k, j = j0 + 4 * cc;
-        return (t < te && j < mr) ? *reinterpret_cast<const float4*>(cf + (size_t)t * mr + j)
-                                  : make_float4(0.f, 0.f, 0.f, 0.f);
-      });
-      tc::stage_mn(s + mn_bytes(128), d, [&](int k, int cc) {
-        const int t = k0 + k;
-        return t < te ? ld_bf16x4(x + (int64_t)t * a.sl + 4 * cc) : make_float4(0.f, 0.f, 0.f, 0.f);
-      });
-      const bool first = ring.g == 0;
-      ring.issue([&] {
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kGemmSlots * slot);
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(bars + 8);
+  const uint32_t tmem = setup(bars, 8, tslot, 128);
+  Ring<kGemmSlots> ring{smem, slot, bars, 0, 0, false};
+  const int nc = (te - tb + 31) / 32 > 0 ? (te - tb + 31) / 32 : 0;   // chunks per side
+  ring.run(
+      2 * nc,
+      [&](int i, uint8_t* s) {
+        const int side = i / nc, k0 = tb + (i % nc) * 32;
+        const __nv_bfloat16* x = (side ? a.xk : a.xq) + (int64_t)b * a.sb + (int64_t)h * a.sh;
+        const float* cf = (side ? a.cfk : a.cfq) + (size_t)bh * L * mr;
+        tc::stage_mn_async(s, 128, [&](int k, int cc) -> const float* {
+          const int t = k0 + k, j = j0 + 4 * cc;
+          return (t < te && j < mr) ? cf + (size_t)t * mr + j : nullptr;
+        }, cf);
+        tc::stage_mn(s + mn_bytes(128), d, [&](int k, int cc) {
+          const int t = k0 + k;
+          return t < te ? ld_bf16x4(x + (int64_t)t * a.sl + 4 * cc, a.xvec)
+                        : make_float4(0.f, 0.f, 0.f, 0.f);
+        });
+      },
+      [&](int i, uint8_t* s) {
         const uint32_t sa = tc::smem_u32(s);
-        tc::mma_chunk(tmem, sa, true, sa + mn_bytes(128), true, d, !first);
+        tc::mma_chunk(tmem, sa, true, sa + mn_bytes(128), true, d, i > 0);
       });
-    }
-  }
   ring.wait_all();
   const int q = (threadIdx.x >> 5) & 3, hf = threadIdx.x >> 7;
   const int j = j0 + q * 32 + (threadIdx.x & 31);
-  float* gh = a.G + ((size_t)(a.heads_w == 1 ? 0 : h) * mr + (j < mr ? j : 0)) * d;
-  if (ring.g > 0)
+  // the block's rows through shared memory, then coalesced atomics
+  float* buf = reinterpret_cast<float*>(smem);
+  const int ld = d + kPad, pw = d / 4;
+  if (ring.issued > 0) {
     for (int c0 = hf * (d / 2); c0 < (hf + 1) * (d / 2); c0 += 16) {
       float v[16];
       tc::tmem_ld16(lane_addr(tmem, c0), v);
-      if (j < mr)
+      const int rr = j - j0;
 #pragma unroll
-        for (int u = 0; u < 16; ++u) atomicAdd(gh + c0 + u, v[u]);
+      for (int u = 0; u < 16; u += 4) st_f4(buf + rr * ld + c0 + u, v[u], v[u + 1], v[u + 2], v[u + 3]);
     }
-  teardown(ring, bars + 2, tmem, 128, a.dev_status);
+    __syncthreads();
+    float* gh = a.G + ((size_t)(a.heads_w == 1 ? 0 : h) * mr + j0) * d;
+    for (int i = threadIdx.x; i < 128 * pw; i += blockDim.x) {
+      const int rr = i / pw, c4 = i - rr * pw;
+      if (j0 + rr < mr) {
+        const float4 v4 = *reinterpret_cast<const float4*>(buf + rr * ld + 4 * c4);
+        float* g = gh + (size_t)rr * d + 4 * c4;
+        atomicAdd(g, v4.x);
+        atomicAdd(g + 1, v4.y);
+        atomicAdd(g + 2, v4.z);
+        atomicAdd(g + 3, v4.w);
+      }
+    }
+  }
+  teardown(ring.failed, bars + 7, tmem, 128, a.dev_status);
 }
 
 struct TcLayout {
@@ -753,10 +976,12 @@ size_t tc_bwd_workspace_bytes(int B, int H, int L, int m, int r, int d, int head
 
 bool tc_backward_supported(const BwdArgs& a) {
   if (a.dtype != DARK_BF16) return false;
-  if (a.d % 32 != 0 || a.d > 128 || a.m % 64 != 0 || a.m > 256 || a.r % 32 != 0 || a.r > 256)
+  if (a.d % 32 != 0 || a.d > 128 || a.m % 64 != 0 || a.m > 256 || a.r % 32 != 0 || a.r > 128)
     return false;
   const int dp = round_up(a.d + 1, 32);
-  if (pass_smem_bytes(a.m, dp, 1) > 227 * 1024) return false;
+  const uint32_t limit = 227 * 1024;
+  if (pass_smem_bytes(a.m, dp, 1) > limit) return false;
+  if (1024 + kFeatSlots * feat_slot_bytes(a.m, a.r) + kTailBytes > limit) return false;
   return true;
 }
 
@@ -782,6 +1007,12 @@ cudaError_t launch_backward_tc(const BwdArgs& a) {
   const __nv_bfloat16* v = (const __nv_bfloat16*)a.v;
   cudaStream_t st = a.stream;
   cudaError_t err;
+  auto rows8 = [](const void* p, const int64_t* s3) {
+    return ((uintptr_t)p % 8 == 0) && s3[0] % 4 == 0 && s3[1] % 4 == 0 && s3[2] % 4 == 0;
+  };
+  const int xvec = rows8(a.q, a.xs) && rows8(a.k, a.xs) ? 1 : 0;
+  const int vvec = rows8(a.v, a.xs) ? 1 : 0;
+  const int gvec = rows8(a.dout, a.gs) ? 1 : 0;
 
   err = launch_projection(a.omega, a.heads_omega, a.geom, a.heads_geom, a.heads_w, m, r, d,
                           DARK_F32, wf, st);
@@ -790,19 +1021,20 @@ cudaError_t launch_backward_tc(const BwdArgs& a) {
 
   {
     static int done[64];
-    const size_t bytes = one_cta(1024 + 2 * (km_bytes(kTT) + km_bytes(round_up(m + r, 32))) + 64 +
-                                 2 * kTT * 4);
+    const size_t bytes = one_cta(1024 + kFeatSlots * feat_slot_bytes(m, r) + kTailBytes);
     if ((err = set_smem(tbf_features_kernel, bytes, done)) != cudaSuccess) return err;
     FeatArgs fa{q, k, a.xs[0], a.xs[1], a.xs[2], wf, a.heads_w, m, r, d, a.H, L, a.mask, stab,
-                phiq, phik, pbot, ck, a.dev_status};
+                xvec, phiq, phik, pbot, ck, a.dev_status};
     tbf_features_kernel<<<dim3(nt, bh, 2), kThr, bytes, st>>>(fa);
     if ((err = cudaGetLastError()) != cudaSuccess) return err;
   }
   if (stab && (err = bwd_shift_keys(phik, ck, L, m, (size_t)bh * L * m, st)) != cudaSuccess)
     return err;
 
-  const size_t st_bytes = one_cta(1024 + 2 * (mn_bytes(round_up(m, 128)) + mn_bytes(dp)) + 64);
-  StateArgs sa{phik, v, a.xs[0], a.xs[1], a.xs[2], wq, m, d, dp, a.H, L, nt, cs, a.dev_status};
+  const size_t st_bytes =
+      one_cta(1024 + kStateSlots * (mn_bytes(round_up(m, 128)) + mn_bytes(dp)) + kTailBytes);
+  StateArgs sa{phik, v, a.xs[0], a.xs[1], a.xs[2], vvec, wq, m, d, dp, a.H, L, nt, cs,
+               a.dev_status};
   {
     static int done[64];
     if ((err = set_smem(tbf_state_kernel<1>, st_bytes, done)) != cudaSuccess) return err;
@@ -813,8 +1045,8 @@ cudaError_t launch_backward_tc(const BwdArgs& a) {
 
   const size_t pass_bytes = one_cta(pass_smem_bytes(m, dp, causal));
   PassArgs pa{phiq, phik, cs, v, a.xs[0], a.xs[1], a.xs[2],
-              (const __nv_bfloat16*)a.dout, a.gs[0], a.gs[1], a.gs[2], wq,
-              nullptr, 0, 0, 0, cfq, pbot, m, r, d, dp, a.H, L, nt, causal, a.dev_status};
+              (const __nv_bfloat16*)a.dout, a.gs[0], a.gs[1], a.gs[2], vvec, gvec, wq,
+              nullptr, 0, 0, 0, 0, cfq, pbot, m, r, d, dp, a.H, L, nt, causal, a.dev_status};
   {
     static int done[64];
     if ((err = set_smem(tbf_pass_kernel<0>, pass_bytes, done)) != cudaSuccess) return err;
@@ -837,6 +1069,7 @@ cudaError_t launch_backward_tc(const BwdArgs& a) {
   pa.ob = a.ds[0];
   pa.oh = a.ds[1];
   pa.ol = a.ds[2];
+  pa.ovec = rows8(a.dv, a.ds) ? 1 : 0;
   pa.coef = cfk;
   {
     static int done[64];
@@ -846,10 +1079,11 @@ cudaError_t launch_backward_tc(const BwdArgs& a) {
   }
   {
     static int done[64];
-    const size_t bytes = 1024 + 2 * (km_bytes(kTT) + mn_bytes(d)) + 64;
+    const size_t bytes = 1024 + kGemmSlots * (km_bytes(kTT) + mn_bytes(d)) + kTailBytes;
     if ((err = set_smem(tbf_dx_kernel, bytes, done)) != cudaSuccess) return err;
     DxArgs xa{cfq, cfk, wf, a.heads_w, m, r, d, a.H, L, (__nv_bfloat16*)a.dq,
-              (__nv_bfloat16*)a.dk, a.ds[0], a.ds[1], a.ds[2], a.dev_status};
+              (__nv_bfloat16*)a.dk, a.ds[0], a.ds[1], a.ds[2],
+              rows8(a.dq, a.ds) && rows8(a.dk, a.ds) ? 1 : 0, a.dev_status};
     tbf_dx_kernel<<<dim3(nt, bh, 2), kThr, bytes, st>>>(xa);
     if ((err = cudaGetLastError()) != cudaSuccess) return err;
   }
@@ -862,10 +1096,10 @@ cudaError_t launch_backward_tc(const BwdArgs& a) {
     if (nsplit > max_split) nsplit = max_split;
     if (nsplit < 1) nsplit = 1;
     static int done[64];
-    const size_t bytes = 1024 + 2 * (mn_bytes(128) + mn_bytes(d)) + 64;
+    const size_t bytes = 1024 + kGemmSlots * (mn_bytes(128) + mn_bytes(d)) + kTailBytes;
     if ((err = set_smem(tbf_dw_kernel, bytes, done)) != cudaSuccess) return err;
-    DwArgs wa{q, k, a.xs[0], a.xs[1], a.xs[2], cfq, cfk, m, r, d, a.H, L, a.heads_w, nsplit, G,
-              a.dev_status};
+    DwArgs wa{q, k, a.xs[0], a.xs[1], a.xs[2], cfq, cfk, m, r, d, a.H, L, a.heads_w, nsplit, xvec,
+              G, a.dev_status};
     tbf_dw_kernel<<<dim3(blocks, bh, nsplit), kThr, bytes, st>>>(wa);
     if ((err = cudaGetLastError()) != cudaSuccess) return err;
     if ((err = bwd_dgeom(G, a)) != cudaSuccess) return err;

@@ -54,28 +54,101 @@ __device__ __forceinline__ uint64_t mn_desc(uint32_t base, int j) {
   return sdesc(base + 1024u * j, kMnBlockBytes, 512, kSwizzle128Base32);
 }
 
-// Stages a K-major chunk: fn(row, c) returns values 4c..4c+3 of the row's 32.
-template <class F>
-__device__ __forceinline__ void stage_km(uint8_t* base, int R, F fn) {
-  for (int i = threadIdx.x; i < R * 8; i += blockDim.x) {
-    const int row = i >> 3, c = i & 7;
-    const float4 v = fn(row, c);
-    *reinterpret_cast<float4*>(base + (row >> 3) * 1024 + (row & 7) * 128 +
-                               (((c ^ row) & 7) << 4)) = v;
-  }
+// Shared-memory byte offsets of 16-byte piece c (values 4c..4c+3) of K-major
+// row `row`, and of MN-major K row k.
+__device__ __forceinline__ uint32_t km_off(int row, int c) {
+  return (uint32_t)((row >> 3) * 1024 + (row & 7) * 128 + (((c ^ row) & 7) << 4));
+}
+__device__ __forceinline__ uint32_t mn_off(int k, int c) {
+  return (uint32_t)((c >> 3) * kMnBlockBytes + (k >> 2) * 512 + (k & 3) * 128 +
+                    ((((c >> 1) ^ k) & 3) << 5) + ((c & 1) << 4));
 }
 
-// Stages an MN-major chunk: fn(k, c) returns MN values 4c..4c+3 at K row k
-// (0..31); R is the MN extent (a multiple of 32).
+// Register staging for values that need converting: fn(row, c) (K-major) or
+// fn(k, c) (MN-major) returns the four values; each thread issues up to four
+// loads before it stores any of them. Element i of the rows x per_row pieces
+// is (i / per_row, i % per_row); a thread steps its pair instead of dividing.
+template <bool MN, class F>
+__device__ __forceinline__ void stage_regs(uint8_t* base, int rows, int per_row, F fn) {
+  constexpr int U = 4;
+  const int total = rows * per_row, nt = blockDim.x;
+  const int da = nt / per_row, dc = nt - da * per_row;
+  int a = threadIdx.x / per_row, c = threadIdx.x - a * per_row;
+  for (int i0 = threadIdx.x; i0 < total; i0 += U * nt) {
+    float4 v[U];
+    uint32_t off[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const bool ok = i0 + u * nt < total;
+      v[u] = ok ? fn(a, c) : make_float4(0.f, 0.f, 0.f, 0.f);
+      off[u] = MN ? mn_off(a, c) : km_off(a, c);
+      a += da;
+      c += dc;
+      if (c >= per_row) {
+        c -= per_row;
+        ++a;
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u)
+      if (i0 + u * nt < total) *reinterpret_cast<float4*>(base + off[u]) = v[u];
+  }
+}
+// K-major chunk of R rows: fn(row, c) returns values 4c..4c+3 of the row's 32.
+template <class F>
+__device__ __forceinline__ void stage_km(uint8_t* base, int R, F fn) {
+  stage_regs<false>(base, R, 8, fn);
+}
+// MN-major chunk of MN extent R (a multiple of 32): fn(k, c) returns MN values
+// 4c..4c+3 at K row k (0..31).
 template <class F>
 __device__ __forceinline__ void stage_mn(uint8_t* base, int R, F fn) {
-  const int per_k = R >> 2;
-  for (int i = threadIdx.x; i < 32 * per_k; i += blockDim.x) {
-    const int k = i / per_k, c = i - k * per_k;
-    const float4 v = fn(k, c);
-    *reinterpret_cast<float4*>(base + (c >> 3) * kMnBlockBytes + (k >> 2) * 512 + (k & 3) * 128 +
-                               ((((c >> 1) ^ k) & 3) << 5) + ((c & 1) << 4)) = v;
+  stage_regs<true>(base, 32, R >> 2, fn);
+}
+
+// Asynchronous 16-byte copies global -> shared (zero-filled when `valid` is
+// false: no byte of `src` is read then, and `src` is any mapped address).
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, bool valid) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src),
+               "r"(valid ? 16 : 0)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+// Copy staging of fp32 values already in place: src(row, c) / src(k, c) gives
+// the 16-byte aligned source of the four values, or nullptr for zeros
+// (`any` then stands in as the unread source address).
+template <bool MN, class F>
+__device__ __forceinline__ void stage_async(uint8_t* base, int rows, int per_row, F src,
+                                            const float* any) {
+  const uint32_t b = smem_u32(base);
+  const int total = rows * per_row, nt = blockDim.x;
+  const int da = nt / per_row, dc = nt - da * per_row;
+  int a = threadIdx.x / per_row, c = threadIdx.x - a * per_row;
+#pragma unroll 4
+  for (int i = threadIdx.x; i < total; i += nt) {
+    const float* p = src(a, c);
+    cp_async16(b + (MN ? mn_off(a, c) : km_off(a, c)), p != nullptr ? p : any, p != nullptr);
+    a += da;
+    c += dc;
+    if (c >= per_row) {
+      c -= per_row;
+      ++a;
+    }
   }
+}
+template <class F>
+__device__ __forceinline__ void stage_km_async(uint8_t* base, int R, F src, const float* any) {
+  stage_async<false>(base, R, 8, src, any);
+}
+template <class F>
+__device__ __forceinline__ void stage_mn_async(uint8_t* base, int R, F src, const float* any) {
+  stage_async<true>(base, 32, R >> 2, src, any);
 }
 
 // Issues the four K-steps of one 32-deep chunk: D (+)= A * B with A an M = 128
