@@ -648,31 +648,54 @@ __global__ void __launch_bounds__(256) dw_kernel(
 }
 
 // dM[hm] = sum over the projection heads hw that use M_hm of
-// c_w Omega_hw^T dW'_top[hw] + c_m dW'_bot[hw].
-__global__ void dgeom_kernel(const float* __restrict__ G, const float* __restrict__ omega,
-                             int heads_omega, int heads_geom, int heads_w, int m, int r, int d,
-                             float cw, float cm, float* __restrict__ dgeom) {
-  const int i = blockIdx.x, hm = blockIdx.y;
+// c_w Omega_hw^T dW'_top[hw] + c_m dW'_bot[hw]: a 16 x 64 block of dM per CTA,
+// Omega columns and dW' rows staged 32 features at a time.
+__global__ void __launch_bounds__(256) dgeom_kernel(
+    const float* __restrict__ G, const float* __restrict__ omega, int heads_omega,
+    int heads_geom, int heads_w, int m, int r, int d, float cw, float cm,
+    float* __restrict__ dgeom) {
+  __shared__ float Os[32][17];
+  __shared__ __align__(16) float Gs[32][64];
+  const int c0 = blockIdx.x * 64, i0 = blockIdx.y * 16, hm = blockIdx.z;
+  const int ii = threadIdx.x >> 4, cq = threadIdx.x & 15;
+  const int i = i0 + ii, c = c0 + 4 * cq;
   const int mr = m + r;
-  for (int c = threadIdx.x; c < d; c += blockDim.x) {
-    float acc = 0.f;
-    for (int hw = 0; hw < heads_w; ++hw) {
-      if (heads_geom != 1 && hw != hm) continue;
-      const float* om = omega + (size_t)(heads_omega == 1 ? 0 : hw) * m * r;
-      const float* g = G + (size_t)hw * mr * d;
-      float s4[4] = {0.f, 0.f, 0.f, 0.f};
-      int j = 0;
-#pragma unroll 4
-      for (; j + 4 <= m; j += 4)
-#pragma unroll
-        for (int u = 0; u < 4; ++u)
-          s4[u] = fmaf(om[(size_t)(j + u) * r + i], g[(size_t)(j + u) * d + c], s4[u]);
-      for (; j < m; ++j) s4[0] = fmaf(om[(size_t)j * r + i], g[(size_t)j * d + c], s4[0]);
-      const float s = (s4[0] + s4[1]) + (s4[2] + s4[3]);
-      acc += cw * s + cm * g[(size_t)(m + i) * d + c];
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  for (int hw = 0; hw < heads_w; ++hw) {
+    if (heads_geom != 1 && hw != hm) continue;
+    const float* om = omega + (size_t)(heads_omega == 1 ? 0 : hw) * m * r;
+    const float* g = G + (size_t)hw * mr * d;
+    float s4[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int j0 = 0; j0 < m; j0 += 32) {
+      for (int e = threadIdx.x; e < 32 * 16; e += blockDim.x) {
+        const int jj = e >> 4, i2 = e & 15;
+        Os[jj][i2] = (j0 + jj < m && i0 + i2 < r) ? om[(size_t)(j0 + jj) * r + i0 + i2] : 0.f;
+      }
+      for (int e = threadIdx.x; e < 32 * 64; e += blockDim.x) {
+        const int jj = e >> 6, c2 = e & 63;
+        Gs[jj][c2] = (j0 + jj < m && c0 + c2 < d) ? g[(size_t)(j0 + jj) * d + c0 + c2] : 0.f;
+      }
+      __syncthreads();
+#pragma unroll 8
+      for (int jj = 0; jj < 32; ++jj) {
+        const float o = Os[jj][ii];
+        const float4 g4 = *reinterpret_cast<const float4*>(&Gs[jj][4 * cq]);
+        s4[0] = fmaf(o, g4.x, s4[0]);
+        s4[1] = fmaf(o, g4.y, s4[1]);
+        s4[2] = fmaf(o, g4.z, s4[2]);
+        s4[3] = fmaf(o, g4.w, s4[3]);
+      }
+      __syncthreads();
     }
-    dgeom[((size_t)hm * r + i) * d + c] = acc;
+    if (i < r)
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        if (c + u < d) acc[u] += cw * s4[u] + cm * g[(size_t)(m + i) * d + c + u];
   }
+  if (i < r)
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+      if (c + u < d) dgeom[((size_t)hm * r + i) * d + c + u] = acc[u];
 }
 
 size_t pass_smem_bytes(int et) {
@@ -790,7 +813,7 @@ cudaError_t backward_t(const BwdArgs& a) {
     dw_kernel<T><<<dim3((m + r + 63) / 64, (d + 63) / 64, bh * nsplit), 256, 0, a.stream>>>(
         q, k, a.xs[0], a.xs[1], a.xs[2], cfq, cfk, m, r, d, a.H, L, a.heads_w, nsplit, G);
     const double sc = pow((double)d, -0.25);
-    dgeom_kernel<<<dim3(r, a.heads_geom), 128, 0, a.stream>>>(
+    dgeom_kernel<<<dim3((d + 63) / 64, (r + 15) / 16, a.heads_geom), 256, 0, a.stream>>>(
         G, a.omega, a.heads_omega, a.heads_geom, a.heads_w, m, r, d, (float)(sc * kLog2e),
         (float)(sc * sqrt(0.5 * kLog2e)), a.dgeom);
   }
@@ -825,7 +848,7 @@ cudaError_t bwd_tile_scan(float* st, int n, int nt, int bh, int mode, cudaStream
 }
 cudaError_t bwd_dgeom(const float* G, const BwdArgs& a) {
   const double sc = pow((double)a.d, -0.25);
-  dgeom_kernel<<<dim3(a.r, a.heads_geom), 128, 0, a.stream>>>(
+  dgeom_kernel<<<dim3((a.d + 63) / 64, (a.r + 15) / 16, a.heads_geom), 256, 0, a.stream>>>(
       G, a.omega, a.heads_omega, a.heads_geom, a.heads_w, a.m, a.r, a.d, (float)(sc * kLog2e),
       (float)(sc * sqrt(0.5 * kLog2e)), a.dgeom);
   return cudaGetLastError();

@@ -37,86 +37,97 @@ using tc::km_bytes;
 using tc::mn_bytes;
 
 constexpr int kTT = 128;                        // tokens per tile
-constexpr int kThr = 256;                       // threads per CTA
+constexpr int kWorkers = 256;                   // staging and epilogue threads (warps 0-7)
+constexpr int kThr = kWorkers + 32;             // + warp 8, which issues the MMAs
 constexpr float kLn2f = 0.69314718055994530942f;
 constexpr int kFeatSlots = 3, kStateSlots = 4, kPassSlots = 3, kGemmSlots = 4;
-// Shared memory past the ring: 8 barriers (slots, drain), the TMEM slot and a
-// [2][128] fp32 reduction buffer.
-constexpr uint32_t kTailBytes = 128 + 2 * 128 * 4;
+// Shared memory past the ring: 16 barrier words (full, empty, drain), the
+// TMEM slot and a [2][128] fp32 reduction buffer.
+constexpr uint32_t kTailBytes = 160 + 2 * 128 * 4;
 
 __host__ __device__ constexpr int round_up(int x, int a) { return (x + a - 1) / a * a; }
 
-// The shared-memory ring of NS slots: chunk i is staged into slot i % NS; its
-// MMAs commit to that slot's barrier, which the stager of chunk i + NS waits
-// for. The MMAs of chunk i are issued once chunk i + NS - 1 has been staged,
-// so the copies of NS - 1 chunks are in flight behind the MMAs. Every thread
-// calls every member in the same order; `failed` is uniform.
+// The shared-memory ring of NS slots, between the workers (warps 0-7), which
+// stage the operands, and warp 8, whose lane 0 issues the MMAs. Chunk i goes
+// to slot i % NS. A worker arrives on full[slot] once its copies for the
+// chunk have landed (fenced for the tensor cores); the MMA thread waits for
+// all 256 arrivals, issues the chunk's MMAs and commits them to empty[slot],
+// which the stagers of chunk i + NS wait for. Workers keep the copies of two
+// chunks in flight before they signal. Every thread runs the same sequence
+// of run() calls; a wait that runs out sets `failed`, which later waits skip
+// and which is made uniform after each run().
 template <int NS>
 struct Ring {
+  // a worker signals chunk i after staging chunk i + 2, which needs the MMAs
+  // of chunk i + 2 - NS: NS must exceed 2
+  static_assert(NS > 2, "the ring needs more slots than chunks in flight");
   uint8_t* base;
   uint32_t slot_bytes;
-  uint64_t* bar;                  // NS slot barriers
-  int staged;                     // chunks staged
-  int issued;                     // chunks whose MMAs are issued
+  uint64_t* bar;                  // full[NS], then empty[NS]
+  int done;                       // chunks completed by both sides so far
   bool failed;
 
   __device__ uint8_t* slot(int i) const { return base + (i % NS) * slot_bytes; }
-  __device__ void wait_chunk(int i) {   // the MMAs of chunk i completed
-    if (i >= 0 && !failed) {
-      const bool ok = tc::mbar_wait(bar + (i % NS), (i / NS) & 1);
-      if (__syncthreads_or(ok ? 0 : 1)) failed = true;
-    }
+  __device__ uint64_t* full(int i) const { return bar + (i % NS); }
+  __device__ uint64_t* empty(int i) const { return bar + NS + (i % NS); }
+  __device__ void wait(uint64_t* b, int parity) {
+    if (!failed && !tc::mbar_wait(b, parity)) failed = true;
   }
-  __device__ uint8_t* acquire() {
-    wait_chunk(staged - NS);
-    return slot(staged);
-  }
-  __device__ void staged_one() {
-    tc::cp_async_commit();
-    ++staged;
-  }
-  // Thread 0 issues the MMAs of the oldest staged chunk once its copies have
-  // landed (the copies of the `newer` chunks staged after it may be in flight).
-  template <class F>
-  __device__ void issue(F fn, int newer) {
-    if (newer >= 2) tc::cp_async_wait<2>();
-    else if (newer == 1) tc::cp_async_wait<1>();
-    else tc::cp_async_wait<0>();
-    tc::fence_async_smem();
-    tc::tc_fence_before();
-    __syncthreads();
-    if (!failed && threadIdx.x == 0) {
-      tc::tc_fence_after();
-      fn(issued, slot(issued));
-      tc::mma_commit(bar + (issued % NS));
-    }
-    ++issued;
-  }
-  // Stages and issues n chunks: stage(i, slot) fills chunk i's slot,
-  // mma(i, slot) issues its MMAs (thread 0).
+  // Stages and issues n chunks: stage(i, slot) fills chunk i's slot (workers),
+  // mma(i, slot) issues its MMAs (warp 8, lane 0).
   template <class S, class M>
   __device__ void run(int n, S stage, M mma) {
-    constexpr int D = NS - 1 < 2 ? NS - 1 : 2;          // chunks in flight behind the MMAs
-    for (int i = 0; i < n; ++i) {
-      stage(i, acquire());
-      staged_one();
-      if (i >= D) issue([&](int, uint8_t* p) { mma(i - D, p); }, D);
+    const int g0 = done;
+    if (threadIdx.x < kWorkers) {
+      constexpr int D = 2;        // chunks whose copies may still be in flight
+      int arrived = 0;
+      auto signal = [&](int k) {
+        tc::fence_async_smem();
+        tc::tc_fence_before();
+        tc::mbar_arrive(full(g0 + k));
+      };
+      for (int i = 0; i < n; ++i) {
+        const int g = g0 + i;
+        if (g >= NS) wait(empty(g - NS), ((g - NS) / NS) & 1);
+        stage(i, slot(g));
+        tc::cp_async_commit();
+        if (i - arrived >= D) {
+          tc::cp_async_wait<D>();
+          signal(arrived++);
+        }
+      }
+      tc::cp_async_wait<0>();
+      while (arrived < n) signal(arrived++);
+    } else if (threadIdx.x == kWorkers) {
+      for (int i = 0; i < n; ++i) {
+        const int g = g0 + i;
+        wait(full(g), (g / NS) & 1);
+        tc::tc_fence_after();
+        if (!failed) mma(i, slot(g));
+        tc::mma_commit(empty(g));
+      }
     }
-    for (int j = n - D > 0 ? n - D : 0; j < n; ++j)
-      issue([&](int, uint8_t* p) { mma(j, p); }, n - 1 - j);
+    done = g0 + n;
+    failed = __syncthreads_or(failed ? 1 : 0) != 0;
   }
   // Every MMA issued so far has completed (their results are readable).
   __device__ void wait_all() {
-    wait_chunk(issued - 1);
+    if (done > 0) wait(empty(done - 1), ((done - 1) / NS) & 1);
+    failed = __syncthreads_or(failed ? 1 : 0) != 0;
     tc::tc_fence_after();
   }
 };
 
-// Shared prologue: barriers, TMEM allocation (warp 0). Returns the TMEM base.
-__device__ __forceinline__ uint32_t setup(uint64_t* bars, int nbars, uint32_t* tslot,
+// Shared prologue: barriers (full[ns] for the workers' arrivals, empty[ns] and
+// the drain barrier for MMA commits), TMEM allocation (warp 0). Returns the
+// TMEM base.
+constexpr int kDrainBar = 15;
+__device__ __forceinline__ uint32_t setup(uint64_t* bars, int ns, uint32_t* tslot,
                                           uint32_t ncols) {
   if (threadIdx.x == 0) {
-    for (int i = 0; i < nbars; ++i) tc::mbar_init(bars + i, 1);
+    for (int i = 0; i < ns; ++i) tc::mbar_init(bars + i, kWorkers);
+    for (int i = ns; i < 2 * ns; ++i) tc::mbar_init(bars + i, 1);
+    tc::mbar_init(bars + kDrainBar, 1);
     tc::fence_mbar_init();
   }
   if (threadIdx.x < 32) tc::tmem_alloc(tslot, ncols);
@@ -129,7 +140,7 @@ __device__ __forceinline__ uint32_t setup(uint64_t* bars, int nbars, uint32_t* t
 // Shared epilogue: on a failed wait, drain the issued MMAs before TMEM is freed.
 __device__ __forceinline__ void teardown(bool failed, uint64_t* bar_drain, uint32_t tmem,
                                          uint32_t ncols, int* dev_status) {
-  if (failed && threadIdx.x == 0) {
+  if (failed && threadIdx.x == kWorkers) {
     report(dev_status, DARK_ERR_TIMEOUT);
     tc::drain_mmas(bar_drain);
   }
@@ -239,10 +250,10 @@ __global__ void __launch_bounds__(kThr, 1) tbf_features_kernel(FeatArgs a) {
   const int nrow = side ? m + r : m;                          // W' rows = P columns
   const uint32_t slot = feat_slot_bytes(m, r);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kFeatSlots * slot);   // slots, drain (7)
-  uint32_t* tslot = reinterpret_cast<uint32_t*>(bars + 8);
-  float* red = reinterpret_cast<float*>(bars + 16);                        // [2][128]
-  const uint32_t tmem = setup(bars, 8, tslot, 512);
-  Ring<kFeatSlots> ring{smem, slot, bars, 0, 0, false};
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(bars + 16);
+  float* red = reinterpret_cast<float*>(bars + 20);                        // [2][128]
+  const uint32_t tmem = setup(bars, kFeatSlots, tslot, 512);
+  Ring<kFeatSlots> ring{smem, slot, bars, 0, false};
   const __nv_bfloat16* x = (side ? a.xk : a.xq) + (int64_t)b * a.sb + (int64_t)h * a.sh;
   const float* wh = a.w + (size_t)(a.heads_w == 1 ? 0 : h) * (m + r) * d;
 
@@ -251,12 +262,12 @@ __global__ void __launch_bounds__(kThr, 1) tbf_features_kernel(FeatArgs a) {
       [&](int kc, uint8_t* s) {
         tc::stage_km_async(s + km_bytes(kTT), round_up(nrow, 32), [&](int row, int c) {
           return row < nrow ? wh + (size_t)row * d + kc * 32 + 4 * c : nullptr;
-        }, wh);
+        }, wh, kWorkers);
         tc::stage_km(s, kTT, [&](int row, int c) {
           const int t = t0 + row;
           return t < L ? ld_bf16x4(x + (int64_t)t * a.sl + kc * 32 + 4 * c, a.xvec)
                        : make_float4(0.f, 0.f, 0.f, 0.f);
-        });
+        }, kWorkers);
       },
       [&](int kc, uint8_t* s) {
         const uint32_t sa = tc::smem_u32(s), sw = sa + km_bytes(kTT);
@@ -270,7 +281,9 @@ __global__ void __launch_bounds__(kThr, 1) tbf_features_kernel(FeatArgs a) {
   // epilogue: warps w and w + 4 share TMEM lanes 32 (w % 4) .. +31, each
   // taking half of a block's columns; row statistics are combined through
   // `red`, outputs leave through shared memory (the ring is idle now).
-  const int q = (threadIdx.x >> 5) & 3, hf = threadIdx.x >> 7;
+  // (warp 8 only joins the block-wide steps)
+  const bool wk = threadIdx.x < kWorkers;
+  const int q = (threadIdx.x >> 5) & 3, hf = (threadIdx.x >> 7) & 1;
   const int row = q * 32 + (threadIdx.x & 31), t = t0 + row;
   const bool in = t < L;
   float* buf = reinterpret_cast<float*>(smem);
@@ -286,56 +299,61 @@ __global__ void __launch_bounds__(kThr, 1) tbf_features_kernel(FeatArgs a) {
     float nrm = 0.f;
     float* pb = a.pbot + (size_t)bh * L * r;
     for (int c0 = 0; c0 < r; c0 += 32) {
-      float v[16];
-      tc::tmem_ld16(lane_addr(tmem, m + c0 + hf * 16), v);
-      float* o = buf + row * (32 + kPad) + hf * 16;
+      if (wk) {
+        float v[16];
+        tc::tmem_ld16(lane_addr(tmem, m + c0 + hf * 16), v);
+        float* o = buf + row * (32 + kPad) + hf * 16;
 #pragma unroll
-      for (int j = 0; j < 16; ++j) nrm = fmaf(v[j], v[j], nrm);
+        for (int j = 0; j < 16; ++j) nrm = fmaf(v[j], v[j], nrm);
 #pragma unroll
-      for (int j = 0; j < 16; j += 4) st_f4(o + j, v[j], v[j + 1], v[j + 2], v[j + 3]);
+        for (int j = 0; j < 16; j += 4) st_f4(o + j, v[j], v[j + 1], v[j + 2], v[j + 3]);
+      }
       block_out<32>(buf, store_rows(pb, r, c0));
     }
-    red[hf * kTT + row] = nrm;
+    if (wk) red[hf * kTT + row] = nrm;
     __syncthreads();
     rowc = red[row] + red[kTT + row] + 0.5f * log2f((float)m);
   } else {
     // queries: exponents relative to the row maximum
     float mx = -INFINITY;
-    for (int c0 = hf * 32; c0 < m; c0 += 64) {
-      float v[32];
-      tc::tmem_ld32(lane_addr(tmem, c0), v);
+    if (wk)
+      for (int c0 = hf * 32; c0 < m; c0 += 64) {
+        float v[32];
+        tc::tmem_ld32(lane_addr(tmem, c0), v);
 #pragma unroll
-      for (int j = 0; j < 32; ++j) mx = fmaxf(mx, v[j]);
-    }
-    red[hf * kTT + row] = mx;
+        for (int j = 0; j < 32; ++j) mx = fmaxf(mx, v[j]);
+      }
+    if (wk) red[hf * kTT + row] = mx;
     __syncthreads();
     rowc = fmaxf(red[row], red[kTT + row]);
   }
   const bool ok = !side || a.mask == nullptr || (in && a.mask[(size_t)b * L + t] != 0);
   float kmax = -INFINITY;
   for (int c0 = 0; c0 < m; c0 += 64) {
-    float v[32];
-    tc::tmem_ld32(lane_addr(tmem, c0 + hf * 32), v);
+    if (wk) {
+      float v[32];
+      tc::tmem_ld32(lane_addr(tmem, c0 + hf * 32), v);
 #pragma unroll
-    for (int j = 0; j < 32; ++j) {
-      const float e = v[j] - rowc;
-      if (side && a.stabilise) {
-        v[j] = ok ? e : -INFINITY;
-        kmax = fmaxf(kmax, v[j]);
-      } else {
-        v[j] = ok ? exp2f(e) : 0.f;
+      for (int j = 0; j < 32; ++j) {
+        const float e = v[j] - rowc;
+        if (side && a.stabilise) {
+          v[j] = ok ? e : -INFINITY;
+          kmax = fmaxf(kmax, v[j]);
+        } else {
+          v[j] = ok ? exp2f(e) : 0.f;
+        }
       }
-    }
-    float* o = buf + row * (64 + kPad) + hf * 32;
+      float* o = buf + row * (64 + kPad) + hf * 32;
 #pragma unroll
-    for (int j = 0; j < 32; j += 4) st_f4(o + j, v[j], v[j + 1], v[j + 2], v[j + 3]);
+      for (int j = 0; j < 32; j += 4) st_f4(o + j, v[j], v[j + 1], v[j + 2], v[j + 3]);
+    }
     block_out<64>(buf, store_rows(dst, m, c0));
   }
-  if (side && a.stabilise) {
+  if (wk && side && a.stabilise) {
     kmax = warp_max(in ? kmax : -INFINITY);
     if ((threadIdx.x & 31) == 0 && kmax > -INFINITY) atomicMax(a.ck + bh, float_to_ordered(kmax));
   }
-  teardown(ring.failed, bars + 7, tmem, 512, a.dev_status);
+  teardown(ring.failed, bars + kDrainBar, tmem, 512, a.dev_status);
 }
 
 // ---------------------------------------------------------------------------
@@ -364,9 +382,9 @@ __global__ void __launch_bounds__(kThr, 1) tbf_state_kernel(StateArgs a) {
   const int mt = (m + 127) / 128, dn = round_up(d + 1, 16);
   const uint32_t abytes = mn_bytes(mt * 128), slot = abytes + mn_bytes(dp);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kStateSlots * slot);
-  uint32_t* tslot = reinterpret_cast<uint32_t*>(bars + 8);
-  const uint32_t tmem = setup(bars, 8, tslot, 512);
-  Ring<kStateSlots> ring{smem, slot, bars, 0, 0, false};
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(bars + 16);
+  const uint32_t tmem = setup(bars, kStateSlots, tslot, 512);
+  Ring<kStateSlots> ring{smem, slot, bars, 0, false};
   const float* X = a.X + (size_t)bh * L * m;
   const __nv_bfloat16* vh = a.v + (int64_t)b * a.vb + (int64_t)h * a.vh;
   const float* wr = a.wrow + (size_t)bh * L * dp;
@@ -377,19 +395,19 @@ __global__ void __launch_bounds__(kThr, 1) tbf_state_kernel(StateArgs a) {
         tc::stage_mn_async(s, mt * 128, [&](int k, int cc) -> const float* {
           const int t = t0 + kc * 32 + k;
           return (t < L && 4 * cc < m) ? X + (size_t)t * m + 4 * cc : nullptr;
-        }, X);
+        }, X, kWorkers);
         if constexpr (SIDE == 0) {
           tc::stage_mn_async(s + abytes, dp, [&](int k, int cc) -> const float* {
             const int t = t0 + kc * 32 + k;
             return t < L ? wr + (size_t)t * dp + 4 * cc : nullptr;
-          }, wr);
+          }, wr, kWorkers);
         } else {
           tc::stage_mn(s + abytes, dp, [&](int k, int cc) {
             const int t = t0 + kc * 32 + k, e = 4 * cc;
             if (t >= L || e > d) return make_float4(0.f, 0.f, 0.f, 0.f);
             if (e == d) return make_float4(1.f, 0.f, 0.f, 0.f);
             return ld_bf16x4(vh + (int64_t)t * a.vl + e, a.vvec);
-          });
+          }, kWorkers);
         }
       },
       [&](int kc, uint8_t* s) {
@@ -429,7 +447,7 @@ __global__ void __launch_bounds__(kThr, 1) tbf_state_kernel(StateArgs a) {
     *reinterpret_cast<float4*>(out + (size_t)rr * dp + 4 * cc) =
         *reinterpret_cast<const float4*>(buf + rr * ld + 4 * cc);
   }
-  teardown(ring.failed, bars + 7, tmem, 512, a.dev_status);
+  teardown(ring.failed, bars + kDrainBar, tmem, 512, a.dev_status);
 }
 
 // ---------------------------------------------------------------------------
@@ -483,11 +501,11 @@ __global__ void __launch_bounds__(kThr, 1) tbf_pass_kernel(PassArgs a) {
   const uint32_t slot = pass_slot_bytes(m, dp, causal);
   uint8_t* scores = smem + kPassSlots * slot;                     // 4 K-major chunks
   uint64_t* bars = reinterpret_cast<uint64_t*>(scores + (causal ? 4 * km_bytes(kTT) : 0));
-  uint32_t* tslot = reinterpret_cast<uint32_t*>(bars + 8);
-  float* red = reinterpret_cast<float*>(bars + 16);               // [2][128]
-  const uint32_t tmem = setup(bars, 8, tslot, 512);
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(bars + 16);
+  float* red = reinterpret_cast<float*>(bars + 20);               // [2][128]
+  const uint32_t tmem = setup(bars, kPassSlots, tslot, 512);
   const uint32_t tD = tmem, tS = tmem + 256;
-  Ring<kPassSlots> ring{smem, slot, bars, 0, 0, false};
+  Ring<kPassSlots> ring{smem, slot, bars, 0, false};
 
   const size_t rowbase = (size_t)bh * L;
   const float* X = (SIDE == 0 ? a.phiq : a.phik) + rowbase * m;
@@ -504,34 +522,34 @@ __global__ void __launch_bounds__(kThr, 1) tbf_pass_kernel(PassArgs a) {
   // Staging of the tile's operands. [v | 1] is converted through registers;
   // fp32 rows ([w | -c], features, states) are copied asynchronously.
   auto v_km = [&](uint8_t* dst, int e0) {        // rows: tile tokens, K: columns e0..
-    tc::stage_km(dst, kTT, [&](int rr, int cc) { return vone4(t0 + rr, e0 + 4 * cc); });
+    tc::stage_km(dst, kTT, [&](int rr, int cc) { return vone4(t0 + rr, e0 + 4 * cc); }, kWorkers);
   };
   auto w_km = [&](uint8_t* dst, int e0) {
     tc::stage_km_async(dst, kTT, [&](int rr, int cc) -> const float* {
       const int tt = t0 + rr;
       return tt < L ? wr + (size_t)tt * dp + e0 + 4 * cc : nullptr;
-    }, wr);
+    }, wr, kWorkers);
   };
   auto v_mn = [&](uint8_t* dst, int tk0) {       // K: tokens tk0.., MN: columns
-    tc::stage_mn(dst, dp, [&](int k, int cc) { return vone4(tk0 + k, 4 * cc); });
+    tc::stage_mn(dst, dp, [&](int k, int cc) { return vone4(tk0 + k, 4 * cc); }, kWorkers);
   };
   auto w_mn = [&](uint8_t* dst, int tk0) {
     tc::stage_mn_async(dst, dp, [&](int k, int cc) -> const float* {
       const int tt = tk0 + k;
       return tt < L ? wr + (size_t)tt * dp + 4 * cc : nullptr;
-    }, wr);
+    }, wr, kWorkers);
   };
   auto feat_km = [&](uint8_t* dst, const float* F, int f0) {   // rows: tokens, K: features
     tc::stage_km_async(dst, kTT, [&](int rr, int cc) -> const float* {
       const int tt = t0 + rr;
       return tt < L ? F + (size_t)tt * m + f0 + 4 * cc : nullptr;
-    }, F);
+    }, F, kWorkers);
   };
   auto feat_mn = [&](uint8_t* dst, const float* F, int tk0) {  // K: tokens, MN: features
     tc::stage_mn_async(dst, m, [&](int k, int cc) -> const float* {
       const int tt = tk0 + k;
       return tt < L ? F + (size_t)tt * m + 4 * cc : nullptr;
-    }, F);
+    }, F, kWorkers);
   };
   // U = [v | 1] (queries) or [w | -c] (keys); P the other one
   auto u_mn = [&](uint8_t* dst, int tk0) {
@@ -544,11 +562,14 @@ __global__ void __launch_bounds__(kThr, 1) tbf_pass_kernel(PassArgs a) {
     if constexpr (SIDE == 0) w_km(dst, e0); else v_km(dst, e0);
   };
 
-  const int q = (threadIdx.x >> 5) & 3, hf = threadIdx.x >> 7;
+  // per-row work of the epilogues on warps 0-7 (warp 8 joins the block-wide steps)
+  const bool wk = threadIdx.x < kWorkers;
+  const int q = (threadIdx.x >> 5) & 3, hf = (threadIdx.x >> 7) & 1;
   const int row = q * 32 + (threadIdx.x & 31), t = t0 + row;
   const bool in = t < L;
   // masked diagonal scores (TMEM columns 256..383) -> K-major operand in `scores`
   auto scores_to_smem = [&]() {
+    if (!wk) return;
 #pragma unroll
     for (int u = 0; u < 2; ++u) {
       const int c0 = hf * 64 + u * 32;
@@ -577,7 +598,7 @@ __global__ void __launch_bounds__(kThr, 1) tbf_pass_kernel(PassArgs a) {
         feat_km(s, X, fc * 32);
         tc::stage_mn_async(s + km_bytes(kTT), dp, [&](int k, int cc) -> const float* {
           return st + (size_t)(fc * 32 + k) * dp + 4 * cc;
-        }, st);
+        }, st, kWorkers);
         if (causal) feat_km(s + km_bytes(kTT) + mn_bytes(dp), Y, fc * 32);
       },
       [&](int fc, uint8_t* s) {
@@ -612,20 +633,22 @@ __global__ void __launch_bounds__(kThr, 1) tbf_pass_kernel(PassArgs a) {
       *reinterpret_cast<float4*>(buf + rr * ld + 4 * cc) = g4;
     }
     __syncthreads();
-    const float den = tc::tmem_ld1(lane_addr(tD, d));
+    const float den = wk ? tc::tmem_ld1(lane_addr(tD, d)) : 0.f;
     float* gr = buf + row * ld;
     float go = 0.f;
-    for (int c0 = hf * dh; c0 < (hf + 1) * dh; c0 += 16) {
-      float v[16];
-      tc::tmem_ld16(lane_addr(tD, c0), v);
+    if (wk)
+      for (int c0 = hf * dh; c0 < (hf + 1) * dh; c0 += 16) {
+        float v[16];
+        tc::tmem_ld16(lane_addr(tD, c0), v);
 #pragma unroll
-      for (int j = 0; j < 16; ++j) go = fmaf(gr[c0 + j], v[j], go);
-    }
-    red[hf * kTT + row] = go;
+        for (int j = 0; j < 16; ++j) go = fmaf(gr[c0 + j], v[j], go);
+      }
+    if (wk) red[hf * kTT + row] = go;
     __syncthreads();
     go = red[row] + red[kTT + row];
     const float inv = (in && den > 0.f) ? 1.f / den : 0.f;
     const float cc = go * inv * inv;
+    if (wk)
     for (int c0 = hf * dh; c0 < (hf + 1) * dh; c0 += 4) {
       float4 g4 = *reinterpret_cast<const float4*>(gr + c0);
       g4.x *= inv; g4.y *= inv; g4.z *= inv; g4.w *= inv;
@@ -633,7 +656,7 @@ __global__ void __launch_bounds__(kThr, 1) tbf_pass_kernel(PassArgs a) {
         report(a.dev_status, DARK_ERR_NUMERIC);
       *reinterpret_cast<float4*>(gr + c0) = g4;
     }
-    if (hf == 1) {
+    if (wk && hf == 1) {
       if (!isfinite(cc)) report(a.dev_status, DARK_ERR_NUMERIC);
       for (int e = d; e < dp; e += 4) st_f4(gr + e, e == d ? -cc : 0.f, 0.f, 0.f, 0.f);
     }
@@ -648,6 +671,7 @@ __global__ void __launch_bounds__(kThr, 1) tbf_pass_kernel(PassArgs a) {
   } else {
     // dv rows out as bf16
     const int ld = d + kPad, per = d / 4;
+    if (wk)
     for (int c0 = hf * dh; c0 < (hf + 1) * dh; c0 += 16) {
       float v[16];
       tc::tmem_ld16(lane_addr(tD, c0), v);
@@ -687,7 +711,7 @@ __global__ void __launch_bounds__(kThr, 1) tbf_pass_kernel(PassArgs a) {
         p_km(s, pc * 32);
         tc::stage_km_async(s + km_bytes(kTT), m, [&](int f, int cc) -> const float* {
           return st + (size_t)f * dp + pc * 32 + 4 * cc;
-        }, st);
+        }, st, kWorkers);
       },
       [&](int pc, uint8_t* s) {
         const uint32_t sa = tc::smem_u32(s);
@@ -729,16 +753,18 @@ __global__ void __launch_bounds__(kThr, 1) tbf_pass_kernel(PassArgs a) {
       tc::cp_async_wait<0>();
     }
     __syncthreads();
-    float v[32];
-    tc::tmem_ld32(lane_addr(tD, blk * 64 + hf * 32), v);
-    float* xr = cur + row * (64 + kPad) + hf * 32;
+    if (wk) {
+      float v[32];
+      tc::tmem_ld32(lane_addr(tD, blk * 64 + hf * 32), v);
+      float* xr = cur + row * (64 + kPad) + hf * 32;
 #pragma unroll
-    for (int j = 0; j < 32; j += 4) {
-      const float4 x4 = *reinterpret_cast<const float4*>(xr + j);
-      const float o0 = kLn2f * x4.x * v[j], o1 = kLn2f * x4.y * v[j + 1];
-      const float o2 = kLn2f * x4.z * v[j + 2], o3 = kLn2f * x4.w * v[j + 3];
-      rs += (o0 + o1) + (o2 + o3);
-      st_f4(xr + j, o0, o1, o2, o3);
+      for (int j = 0; j < 32; j += 4) {
+        const float4 x4 = *reinterpret_cast<const float4*>(xr + j);
+        const float o0 = kLn2f * x4.x * v[j], o1 = kLn2f * x4.y * v[j + 1];
+        const float o2 = kLn2f * x4.z * v[j + 2], o3 = kLn2f * x4.w * v[j + 3];
+        rs += (o0 + o1) + (o2 + o3);
+        st_f4(xr + j, o0, o1, o2, o3);
+      }
     }
     block_out<64>(cur, [&](int rr, int c, float4 val) {
       if (t0 + rr < L)
@@ -746,7 +772,7 @@ __global__ void __launch_bounds__(kThr, 1) tbf_pass_kernel(PassArgs a) {
     });
   }
   if (SIDE == 1) {
-    red[hf * kTT + row] = rs;
+    if (wk) red[hf * kTT + row] = rs;
     __syncthreads();
     rs = red[row] + red[kTT + row];
     const float* pb = a.pbot + rowbase * (size_t)r;
@@ -758,6 +784,7 @@ __global__ void __launch_bounds__(kThr, 1) tbf_pass_kernel(PassArgs a) {
       tc::cp_async_wait<0>();
       __syncthreads();
       float* pr = buf0 + row * (32 + kPad) + hf * 16;
+      if (wk)
 #pragma unroll
       for (int j = 0; j < 16; j += 4) {
         const float4 p4 = *reinterpret_cast<const float4*>(pr + j);
@@ -777,7 +804,7 @@ __global__ void __launch_bounds__(kThr, 1) tbf_pass_kernel(PassArgs a) {
         st_f4(cfb + (size_t)(t0 + rr) * (m + r) + m + 4 * c4, 0.f, 0.f, 0.f, 0.f);
     }
   }
-  teardown(ring.failed, bars + 7, tmem, 512, a.dev_status);
+  teardown(ring.failed, bars + kDrainBar, tmem, 512, a.dev_status);
 }
 
 // ---------------------------------------------------------------------------
@@ -801,9 +828,9 @@ __global__ void __launch_bounds__(kThr) tbf_dx_kernel(DxArgs a) {
   const int t0 = blockIdx.x * kTT, m = a.m, r = a.r, d = a.d, L = a.L, mr = m + r;
   const uint32_t slot = km_bytes(kTT) + mn_bytes(d);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kGemmSlots * slot);
-  uint32_t* tslot = reinterpret_cast<uint32_t*>(bars + 8);
-  const uint32_t tmem = setup(bars, 8, tslot, 128);
-  Ring<kGemmSlots> ring{smem, slot, bars, 0, 0, false};
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(bars + 16);
+  const uint32_t tmem = setup(bars, kGemmSlots, tslot, 128);
+  Ring<kGemmSlots> ring{smem, slot, bars, 0, false};
   const float* cf = (side ? a.cfk : a.cfq) + (size_t)bh * L * mr;
   const float* wh = a.w + (size_t)(a.heads_w == 1 ? 0 : h) * mr * d;
   const int kend = side ? mr : m;
@@ -813,21 +840,22 @@ __global__ void __launch_bounds__(kThr) tbf_dx_kernel(DxArgs a) {
         tc::stage_km_async(s, kTT, [&](int rr, int cc) -> const float* {
           const int t = t0 + rr;
           return t < L ? cf + (size_t)t * mr + kc * 32 + 4 * cc : nullptr;
-        }, cf);
+        }, cf, kWorkers);
         tc::stage_mn_async(s + km_bytes(kTT), d, [&](int k, int cc) -> const float* {
           return wh + (size_t)(kc * 32 + k) * d + 4 * cc;
-        }, wh);
+        }, wh, kWorkers);
       },
       [&](int kc, uint8_t* s) {
         const uint32_t sa = tc::smem_u32(s);
         tc::mma_chunk(tmem, sa, false, sa + km_bytes(kTT), true, d, kc > 0);
       });
   ring.wait_all();
-  const int q = (threadIdx.x >> 5) & 3, hf = threadIdx.x >> 7;
+  const int q = (threadIdx.x >> 5) & 3, hf = (threadIdx.x >> 7) & 1;
   const int row = q * 32 + (threadIdx.x & 31), t = t0 + row;
   // rows out through shared memory (the ring is idle), as bf16
   float* buf = reinterpret_cast<float*>(smem);
   const int ld = d + kPad, per = d / 4;
+  if (threadIdx.x < kWorkers)
   for (int c0 = hf * (d / 2); c0 < (hf + 1) * (d / 2); c0 += 16) {
     float v[16];
     tc::tmem_ld16(lane_addr(tmem, c0), v);
@@ -845,7 +873,7 @@ __global__ void __launch_bounds__(kThr) tbf_dx_kernel(DxArgs a) {
       st_bf16x4(out + (int64_t)(t0 + rr) * a.ol + 4 * c4,
                 *reinterpret_cast<const float4*>(buf + rr * ld + 4 * c4), a.ovec);
   }
-  teardown(ring.failed, bars + 7, tmem, 128, a.dev_status);
+  teardown(ring.failed, bars + kDrainBar, tmem, 128, a.dev_status);
 }
 
 // dW'[hw] += sum over a token range of one (batch, head), both sides, of
@@ -871,9 +899,9 @@ __global__ void __launch_bounds__(kThr) tbf_dw_kernel(DwArgs a) {
   const int tb = split * per, te = min(L, tb + per);
   const uint32_t slot = mn_bytes(128) + mn_bytes(d);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kGemmSlots * slot);
-  uint32_t* tslot = reinterpret_cast<uint32_t*>(bars + 8);
-  const uint32_t tmem = setup(bars, 8, tslot, 128);
-  Ring<kGemmSlots> ring{smem, slot, bars, 0, 0, false};
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(bars + 16);
+  const uint32_t tmem = setup(bars, kGemmSlots, tslot, 128);
+  Ring<kGemmSlots> ring{smem, slot, bars, 0, false};
   const int nc = (te - tb + 31) / 32 > 0 ? (te - tb + 31) / 32 : 0;   // chunks per side
   ring.run(
       2 * nc,
@@ -884,24 +912,25 @@ __global__ void __launch_bounds__(kThr) tbf_dw_kernel(DwArgs a) {
         tc::stage_mn_async(s, 128, [&](int k, int cc) -> const float* {
           const int t = k0 + k, j = j0 + 4 * cc;
           return (t < te && j < mr) ? cf + (size_t)t * mr + j : nullptr;
-        }, cf);
+        }, cf, kWorkers);
         tc::stage_mn(s + mn_bytes(128), d, [&](int k, int cc) {
           const int t = k0 + k;
           return t < te ? ld_bf16x4(x + (int64_t)t * a.sl + 4 * cc, a.xvec)
                         : make_float4(0.f, 0.f, 0.f, 0.f);
-        });
+        }, kWorkers);
       },
       [&](int i, uint8_t* s) {
         const uint32_t sa = tc::smem_u32(s);
         tc::mma_chunk(tmem, sa, true, sa + mn_bytes(128), true, d, i > 0);
       });
   ring.wait_all();
-  const int q = (threadIdx.x >> 5) & 3, hf = threadIdx.x >> 7;
+  const int q = (threadIdx.x >> 5) & 3, hf = (threadIdx.x >> 7) & 1;
   const int j = j0 + q * 32 + (threadIdx.x & 31);
   // the block's rows through shared memory, then coalesced atomics
   float* buf = reinterpret_cast<float*>(smem);
   const int ld = d + kPad, pw = d / 4;
-  if (ring.issued > 0) {
+  if (ring.done > 0) {
+    if (threadIdx.x < kWorkers)
     for (int c0 = hf * (d / 2); c0 < (hf + 1) * (d / 2); c0 += 16) {
       float v[16];
       tc::tmem_ld16(lane_addr(tmem, c0), v);
@@ -923,7 +952,7 @@ __global__ void __launch_bounds__(kThr) tbf_dw_kernel(DwArgs a) {
       }
     }
   }
-  teardown(ring.failed, bars + 7, tmem, 128, a.dev_status);
+  teardown(ring.failed, bars + kDrainBar, tmem, 128, a.dev_status);
 }
 
 struct TcLayout {

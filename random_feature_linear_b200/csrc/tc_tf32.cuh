@@ -38,6 +38,11 @@ __device__ __forceinline__ void mma_tf32(uint32_t tmem_d, uint64_t adesc, uint64
       : "memory");
 }
 
+// One arrival of this thread on a shared-memory mbarrier.
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
 constexpr uint32_t kKmRowBytes = 128;      // one K-major row of a chunk
 constexpr uint32_t kMnBlockBytes = 4096;   // one 32-wide MN block of an MN-major chunk
 
@@ -69,9 +74,9 @@ __device__ __forceinline__ uint32_t mn_off(int k, int c) {
 // loads before it stores any of them. Element i of the rows x per_row pieces
 // is (i / per_row, i % per_row); a thread steps its pair instead of dividing.
 template <bool MN, class F>
-__device__ __forceinline__ void stage_regs(uint8_t* base, int rows, int per_row, F fn) {
+__device__ __forceinline__ void stage_regs(uint8_t* base, int rows, int per_row, F fn, int nt) {
   constexpr int U = 4;
-  const int total = rows * per_row, nt = blockDim.x;
+  const int total = rows * per_row;
   const int da = nt / per_row, dc = nt - da * per_row;
   int a = threadIdx.x / per_row, c = threadIdx.x - a * per_row;
   for (int i0 = threadIdx.x; i0 < total; i0 += U * nt) {
@@ -94,16 +99,17 @@ __device__ __forceinline__ void stage_regs(uint8_t* base, int rows, int per_row,
       if (i0 + u * nt < total) *reinterpret_cast<float4*>(base + off[u]) = v[u];
   }
 }
+// The staging helpers are called by threads 0 .. nt - 1 of the CTA.
 // K-major chunk of R rows: fn(row, c) returns values 4c..4c+3 of the row's 32.
 template <class F>
-__device__ __forceinline__ void stage_km(uint8_t* base, int R, F fn) {
-  stage_regs<false>(base, R, 8, fn);
+__device__ __forceinline__ void stage_km(uint8_t* base, int R, F fn, int nt) {
+  stage_regs<false>(base, R, 8, fn, nt);
 }
 // MN-major chunk of MN extent R (a multiple of 32): fn(k, c) returns MN values
 // 4c..4c+3 at K row k (0..31).
 template <class F>
-__device__ __forceinline__ void stage_mn(uint8_t* base, int R, F fn) {
-  stage_regs<true>(base, 32, R >> 2, fn);
+__device__ __forceinline__ void stage_mn(uint8_t* base, int R, F fn, int nt) {
+  stage_regs<true>(base, 32, R >> 2, fn, nt);
 }
 
 // Asynchronous 16-byte copies global -> shared (zero-filled when `valid` is
@@ -125,9 +131,9 @@ __device__ __forceinline__ void cp_async_wait() {
 // (`any` then stands in as the unread source address).
 template <bool MN, class F>
 __device__ __forceinline__ void stage_async(uint8_t* base, int rows, int per_row, F src,
-                                            const float* any) {
+                                            const float* any, int nt) {
   const uint32_t b = smem_u32(base);
-  const int total = rows * per_row, nt = blockDim.x;
+  const int total = rows * per_row;
   const int da = nt / per_row, dc = nt - da * per_row;
   int a = threadIdx.x / per_row, c = threadIdx.x - a * per_row;
 #pragma unroll 4
@@ -143,12 +149,14 @@ __device__ __forceinline__ void stage_async(uint8_t* base, int rows, int per_row
   }
 }
 template <class F>
-__device__ __forceinline__ void stage_km_async(uint8_t* base, int R, F src, const float* any) {
-  stage_async<false>(base, R, 8, src, any);
+__device__ __forceinline__ void stage_km_async(uint8_t* base, int R, F src, const float* any,
+                                               int nt) {
+  stage_async<false>(base, R, 8, src, any, nt);
 }
 template <class F>
-__device__ __forceinline__ void stage_mn_async(uint8_t* base, int R, F src, const float* any) {
-  stage_async<true>(base, 32, R >> 2, src, any);
+__device__ __forceinline__ void stage_mn_async(uint8_t* base, int R, F src, const float* any,
+                                               int nt) {
+  stage_async<true>(base, 32, R >> 2, src, any, nt);
 }
 
 // Issues the four K-steps of one 32-deep chunk: D (+)= A * B with A an M = 128
