@@ -240,7 +240,8 @@ def run_native(args, w: synth.Workload, rank: int, world: int, dev) -> dict | No
     q, k, v = (torch.from_numpy(inp[n]).to(dev).to(tdt) for n in ("q", "k", "v"))
     mask = None if inp["mask"] is None else torch.from_numpy(inp["mask"]).to(dev)
     out = torch.empty_like(q)
-    flags = (D.DARK_CAUSAL if w.causal else 0) | (D.DARK_EXACT if args.exact else 0)
+    flags = (D.DARK_CAUSAL if w.causal else 0) | (D.DARK_EXACT if args.exact else 0) | \
+        (D.DARK_STABILISE if args.stabilise else 0)
     ws = D.alloc_workspace(proj, w.B, w.H, w.L, flags, dev)
     status = torch.zeros(1, dtype=torch.int32, device=dev)
     flush = None if args.ncu else torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.int32, device=dev)
@@ -390,7 +391,9 @@ def run_native(args, w: synth.Workload, rank: int, world: int, dev) -> dict | No
         "vs_baseline": None,
         "dtype": "bf16" if w.dtype == "bf16" else "f32",
         "data": "synthetic (seeded numpy, orthogonal Gaussian features)",
-        "config": {"workload": ("exact mode: " if args.exact else "") + w.name, "B": w.B, "H": w.H,
+        "config": {"workload": ("exact mode: " if args.exact else "") +
+                               ("stabilised: " if args.stabilise else "") + w.name,
+                   "B": w.B, "H": w.H,
                    "L": w.L, "d": w.d, "r": w.r, "m": w.m,
                    "causal": w.causal, "lengths": list(w.lengths) if w.lengths else None,
                    "l2": "flushed (512 MiB write) before every timed step",
@@ -1027,6 +1030,8 @@ def main():
                     help="do not count launches with the CUDA profiler (for runs under ncu)")
     ap.add_argument("--decode", action="store_true",
                     help="time the streaming decode step (workload 5) instead of the forward")
+    ap.add_argument("--stabilise", action="store_true",
+                    help="forward with the overflow stabiliser (DARK_STABILISE)")
     ap.add_argument("--exact", action="store_true",
                     help="time the exact learned-kernel mode of --workload instead")
     ap.add_argument("--sample", action="store_true",

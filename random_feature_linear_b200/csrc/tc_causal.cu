@@ -66,7 +66,8 @@ struct Cfg {
   static constexpr uint32_t oPsi = oPhi + kPhi;
   static constexpr uint32_t oOnes = oPsi + kPhi;
   static constexpr uint32_t oBar = oOnes + 2048;
-  static constexpr uint32_t kSmem = oBar + 64 + 1024;     // + alignment slack
+  static constexpr uint32_t oRed = oBar + 64;              // [2][128] fp32 row maxima
+  static constexpr uint32_t kSmem = oRed + 1024 + 1024;    // + alignment slack
   // TMEM columns
   // key features [0, M_) and norms [M_, M_ + R_); query features [256, 256 + M_)
   // (issued once the norms are read); once both feature blocks are consumed:
@@ -86,6 +87,10 @@ struct Params {
   int nseg;                     // segments per head
   const float* seg_sums;        // [B*H*nseg][65][m] per-segment key states (nseg > 1)
   float *st_kv, *st_z;          // state after the last chunk
+  // stabiliser: per-(batch, head) key constants (null: none) and whether query
+  // exponents are taken relative to their row maximum
+  const float* kshift;
+  int stab_q;
   int* dev_status;
   long long stall;              // testing stall before the first wait (0: none)
 };
@@ -205,6 +210,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int i = 0; i < 16; ++i) nrm = fmaf(v[i], v[i], nrm);
       }
       nrm += 0.5f * __log2f((float)M_);
+      if (p.kshift != nullptr) nrm += p.kshift[bh];
       // the norm columns are read: the query GEMM may now overwrite them
       tc_fence_before();
       __syncthreads();
@@ -230,8 +236,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     ph_mma ^= 1;
     tc_fence_after();
     // ------------------------------------------------- epilogue: Psi(Q_c)
-    exp2_rows_to_smem(lane_tm + G::tQ, half * (M_ / 2), (half + 1) * (M_ / 2), 0.f, false,
-                      s0 + G::oPsi, row);
+    {
+      const float qoff = p.stab_q ? row_max_pair(lane_tm + G::tQ, half, M_ / 2,
+                                                  (float*)(sm + G::oRed), row)
+                                  : 0.f;
+      exp2_rows_to_smem(lane_tm + G::tQ, half * (M_ / 2), (half + 1) * (M_ / 2), qoff, false,
+                        s0 + G::oPsi, row);
+    }
     for (int i = tid; i < kTileBytes / 16; i += kThreads)   // the key tile is consumed
       st_shared_v4(s0 + G::oK + i * 16, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u);
     fence_async_smem();
@@ -432,7 +443,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 struct Layout {
   int nc, nseg;
-  size_t off_seg, total;
+  size_t off_seg, off_kmax, off_shift, total;   // kmax, shift: stabiliser scratch
 };
 
 // Segments per head: 1 when the heads alone fill the SMs, else enough to give
@@ -444,7 +455,9 @@ Layout layout(int B, int H, int L, int m) {
   s.nseg = bh >= kSms ? 1 : kSms / bh;
   if (s.nseg > s.nc) s.nseg = s.nc;
   s.off_seg = kWsHeader;
-  s.total = align_up(s.off_seg + (s.nseg > 1 ? (size_t)bh * s.nseg * 65 * m * 4 : 0), 256);
+  s.off_kmax = align_up(s.off_seg + (s.nseg > 1 ? (size_t)bh * s.nseg * 65 * m * 4 : 0), 256);
+  s.off_shift = align_up(s.off_kmax + (size_t)bh * 4, 256);
+  s.total = align_up(s.off_shift + (size_t)bh * 4, 256);
   return s;
 }
 
@@ -456,8 +469,14 @@ cudaError_t launch(const FwdArgs& a, const CUtensorMap& tw, const CUtensorMap& t
   const int bh = a.B * a.H;
   float* seg = (float*)((char*)a.ws + s.off_seg);
   cudaError_t e;
+  const bool stab = (a.flags & DARK_STABILISE) != 0;
+  float* kshift = (float*)((char*)a.ws + s.off_shift);
+  if (stab) {
+    e = tc_key_shift(a, tw, tk, tv, (int*)((char*)a.ws + s.off_kmax), kshift);
+    if (e != cudaSuccess) return e;
+  }
   if (s.nseg > 1) {
-    e = tc_launch_key_states(a, tw, tk, tv, s.nc, s.nseg, seg);
+    e = tc_launch_key_states(a, tw, tk, tv, s.nc, s.nseg, seg, stab ? kshift : nullptr);
     if (e != cudaSuccess) return e;
   }
   Params p;
@@ -476,6 +495,8 @@ cudaError_t launch(const FwdArgs& a, const CUtensorMap& tw, const CUtensorMap& t
   p.seg_sums = seg;
   p.st_kv = a.st_kv;
   p.st_z = a.st_z;
+  p.kshift = stab ? kshift : nullptr;
+  p.stab_q = stab ? 1 : 0;
   p.dev_status = a.dev_status;
   p.stall = test_stall_cycles();
   static int smem_set[64];
@@ -503,7 +524,7 @@ cudaError_t launch(const FwdArgs& a, const CUtensorMap& tw, const CUtensorMap& t
 }  // namespace
 
 bool tc_causal_supported(FwdArgs& a) {
-  if (a.dtype != DARK_BF16 || a.d != kD || (a.flags & DARK_STABILISE)) return false;
+  if (a.dtype != DARK_BF16 || a.d != kD) return false;
   if (!(a.m == 128 || a.m == 256) || a.r % 16 != 0 || a.r < 16 || a.r > 64) return false;
   return tc_make_maps(a);
 }

@@ -27,6 +27,11 @@ struct KeyParams {
   const uint8_t* mask;
   int B, H, L, ntiles, nsplit, heads_w;
   float* partials;                 // [B*H*nsplit][65][m]
+  // stabiliser: kmax non-null -> max pass only (the largest valid key exponent
+  // of each (batch, head) into kmax as an ordered int, nothing else written);
+  // kshift non-null -> the per-(batch, head) key constant subtracted in base 2
+  int* kmax;
+  const float* kshift;
   int* dev_status;
   long long stall;                 // testing stall before the first wait (0: none)
 };
@@ -79,11 +84,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(bar_never, 1);
     fence_mbar_init();
     if (te > tb) {
-      mbar_arrive_expect_tx(&bar_kv[0], G::kW + 2 * kTileBytes);
+      // the max pass reads no values
+      mbar_arrive_expect_tx(&bar_kv[0], G::kW + (p.kmax ? 1 : 2) * kTileBytes);
       for (int r0 = 0; r0 < G::NW; r0 += 16)
         tma_load_2d(sm + G::oW + r0 * 128, &tm_w, 0, hw * G::NW + r0, &bar_kv[0]);
       tma_load_4d(sm + G::oK, &tm_k, 0, tb * kT, h, b, &bar_kv[0]);
-      tma_load_4d(sm + G::oV, &tm_v, 0, tb * kT, h, b, &bar_kv[0]);
+      if (!p.kmax) tma_load_4d(sm + G::oV, &tm_v, 0, tb * kT, h, b, &bar_kv[0]);
     }
   }
   __syncwarp();
@@ -132,9 +138,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (tid == 0 && t + 1 < te) {
       const int nb = buf ^ 1;
       ++issued[nb];
-      mbar_arrive_expect_tx(&bar_kv[nb], 2 * kTileBytes);
+      mbar_arrive_expect_tx(&bar_kv[nb], (p.kmax ? 1 : 2) * kTileBytes);
       tma_load_4d(sm + G::oK + nb * kTileBytes, &tm_k, 0, (t + 1) * kT, h, b, &bar_kv[nb]);
-      tma_load_4d(sm + G::oV + nb * kTileBytes, &tm_v, 0, (t + 1) * kT, h, b, &bar_kv[nb]);
+      if (!p.kmax)
+        tma_load_4d(sm + G::oV + nb * kTileBytes, &tm_v, 0, (t + 1) * kT, h, b, &bar_kv[nb]);
     }
     {
       float nrm = 0.f;
@@ -146,9 +153,25 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int e = 0; e < 16; ++e) nrm = fmaf(v[e], v[e], nrm);
       }
       nrm += 0.5f * __log2f((float)M_);
+      if (p.kshift != nullptr) nrm += p.kshift[bh];
       const int tok = t * kT + row;
       bool valid = tok < p.L;
       if (valid && p.mask != nullptr) valid = p.mask[(size_t)b * p.L + tok] != 0;
+      if (p.kmax != nullptr) {
+        // max pass: the largest exponent of this thread's half of the features
+        float mx = -INFINITY;
+        for (int c0 = half * (M_ / 2); c0 < (half + 1) * (M_ / 2); c0 += 32) {
+          float v[32];
+          tmem_ld32(lane_tm + G::tP + c0, v);
+#pragma unroll
+          for (int e = 0; e < 32; ++e) mx = fmaxf(mx, v[e]);
+        }
+        mx = warp_max(valid ? mx - nrm : -INFINITY);
+        if (lane == 0 && mx > -INFINITY) atomicMax(p.kmax + bh, float_to_ordered(mx));
+        tc_fence_before();
+        __syncthreads();           // the next feature GEMM overwrites these columns
+        continue;
+      }
       exp2_rows_to_smem(lane_tm + G::tP, half * (M_ / 2), (half + 1) * (M_ / 2), nrm, !valid,
                         s0 + G::oPhi, row);
     }
@@ -183,7 +206,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     drain_loads(&bar_kv[1], issued[1], waited[1]);
     drain_mmas(bar_drain);
   }
-  if (!abort && half < G::MB) {
+  if (!abort && half < G::MB && p.kmax == nullptr) {
     const int f = half * 128 + row;
     float* dst = p.partials + ((size_t)bh * p.nsplit + split) * 65 * M_;
     if (te > tb) {
@@ -211,8 +234,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 template <int M_, int R_>
 cudaError_t launch_keys_t(const FwdArgs& a, const CUtensorMap& tw, const CUtensorMap& tk,
-                          const CUtensorMap& tv, int ntiles, int nsplit, float* partials) {
+                          const CUtensorMap& tv, int ntiles, int nsplit, float* partials,
+                          int* kmax, const float* kshift) {
   KeyParams kp;
+  kp.kmax = kmax;
+  kp.kshift = kshift;
   kp.mask = a.mask;
   kp.B = a.B;
   kp.H = a.H;
@@ -233,10 +259,14 @@ cudaError_t launch_keys_t(const FwdArgs& a, const CUtensorMap& tw, const CUtenso
 
 }  // namespace
 
-cudaError_t tc_launch_key_states(const FwdArgs& a, const CUtensorMap& tw, const CUtensorMap& tk,
-                                 const CUtensorMap& tv, int ntiles, int nsplit, float* partials) {
-#define DARK_KEYS_CASE(MM, RR) \
-  if (a.m == MM && a.r == RR) return launch_keys_t<MM, RR>(a, tw, tk, tv, ntiles, nsplit, partials);
+namespace {
+
+cudaError_t launch_keys(const FwdArgs& a, const CUtensorMap& tw, const CUtensorMap& tk,
+                        const CUtensorMap& tv, int ntiles, int nsplit, float* partials, int* kmax,
+                        const float* kshift) {
+#define DARK_KEYS_CASE(MM, RR)                                                              \
+  if (a.m == MM && a.r == RR)                                                               \
+    return launch_keys_t<MM, RR>(a, tw, tk, tv, ntiles, nsplit, partials, kmax, kshift);
   DARK_KEYS_CASE(256, 64)
   DARK_KEYS_CASE(256, 48)
   DARK_KEYS_CASE(256, 32)
@@ -247,6 +277,44 @@ cudaError_t tc_launch_key_states(const FwdArgs& a, const CUtensorMap& tw, const 
   DARK_KEYS_CASE(128, 16)
 #undef DARK_KEYS_CASE
   return cudaErrorInvalidValue;
+}
+
+__global__ void fill_ordered(int* p, int n) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < n) p[i] = float_to_ordered(-INFINITY);
+}
+
+// c_K = the largest valid key exponent (0 for a head without valid keys)
+__global__ void finalize_shift(const int* kmax, float* shift, float* st_shift, int n) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= n) return;
+  float c = ordered_to_float(kmax[i]);
+  if (!(c > -INFINITY)) c = 0.f;
+  shift[i] = c;
+  if (st_shift != nullptr) st_shift[i] = c;
+}
+
+}  // namespace
+
+cudaError_t tc_launch_key_states(const FwdArgs& a, const CUtensorMap& tw, const CUtensorMap& tk,
+                                 const CUtensorMap& tv, int ntiles, int nsplit, float* partials,
+                                 const float* kshift) {
+  return launch_keys(a, tw, tk, tv, ntiles, nsplit, partials, nullptr, kshift);
+}
+
+cudaError_t tc_key_shift(const FwdArgs& a, const CUtensorMap& tw, const CUtensorMap& tk,
+                         const CUtensorMap& tv, int* kmax, float* shift) {
+  const int bh = a.B * a.H, ntiles = (a.Lk + 127) / 128;
+  int nsplit = (2 * num_sms() + bh - 1) / bh;
+  if (nsplit > ntiles) nsplit = ntiles;
+  if (nsplit < 1) nsplit = 1;
+  fill_ordered<<<(bh + 255) / 256, 256, 0, a.stream>>>(kmax, bh);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  e = launch_keys(a, tw, tk, tv, ntiles, nsplit, nullptr, kmax, nullptr);
+  if (e != cudaSuccess) return e;
+  finalize_shift<<<(bh + 255) / 256, 256, 0, a.stream>>>(kmax, shift, a.st_shift, bh);
+  return cudaGetLastError();
 }
 
 }  // namespace dark

@@ -39,5 +39,25 @@ __device__ __forceinline__ void to_fp16_inplace(uint32_t saddr, int bytes, int* 
   if (bad) report(dev_status, DARK_ERR_NUMERIC);
 }
 
+// Stabiliser: the maximum of a row of `ncols_half` * 2 TMEM columns whose two
+// halves are read by the threads of warps w and w + 4 (half = 0, 1) at
+// lane_taddr + half * ncols_half; the halves meet in red[2][128]. Called by
+// every thread of the CTA (it holds a block-wide barrier).
+__device__ __forceinline__ float row_max_pair(uint32_t lane_taddr, int half, int ncols_half,
+                                              float* red, int row) {
+  float mx = -INFINITY;
+  for (int c0 = half * ncols_half; c0 < (half + 1) * ncols_half; c0 += 32) {
+    float v[32];
+    tmem_ld32(lane_taddr + c0, v);
+#pragma unroll
+    for (int e = 0; e < 32; ++e) mx = fmaxf(mx, v[e]);
+  }
+  red[half * 128 + row] = mx;
+  __syncthreads();
+  mx = fmaxf(red[row], red[128 + row]);
+  __syncthreads();               // red may be reused
+  return mx;
+}
+
 }  // namespace tc
 }  // namespace dark

@@ -78,6 +78,7 @@ struct QueryParams {
   int B, H, L, ntiles, heads_w, total_tiles;   // L, ntiles: queries
   const uint8_t* qmask;         // [B][L] or null: a masked query row outputs 0
   const uint8_t* images;
+  int stab_q;                   // stabiliser: query exponents relative to their row maximum
   int* dev_status;
   long long stall;              // testing stall before the first wait (0: none)
 };
@@ -92,7 +93,8 @@ struct QueryCfg {
   static constexpr uint32_t oQ = oImg + (img_bytes(M_) + 1023) / 1024 * 1024;   // 2 buffers
   static constexpr uint32_t oPsi = oQ + 2 * kTileBytes;
   static constexpr uint32_t oBar = oPsi + kPsi;
-  static constexpr uint32_t kSmem = oBar + 64 + 1024;
+  static constexpr uint32_t oRed = oBar + 64;              // [2][128] fp32 row maxima
+  static constexpr uint32_t kSmem = oRed + 1024 + 1024;
   static constexpr uint32_t tP = 0, tO = 256;
   static_assert(kSmem <= 232448, "shared memory");
 };
@@ -193,8 +195,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       tma_load_4d(sm + G::oQ + (buf ^ 1) * kTileBytes, &tm_q, 0, nt * kT, nbh % p.H, nbh / p.H,
                   &bar_q[buf ^ 1]);
     }
-    exp2_rows_to_smem(lane_tm + G::tP, half * (M_ / 2), (half + 1) * (M_ / 2), 0.f, false,
-                      s0 + G::oPsi, row);
+    {
+      const float qoff = p.stab_q ? row_max_pair(lane_tm + G::tP, half, M_ / 2,
+                                                  (float*)(sm + G::oRed), row)
+                                  : 0.f;
+      exp2_rows_to_smem(lane_tm + G::tP, half * (M_ / 2), (half + 1) * (M_ / 2), qoff, false,
+                        s0 + G::oPsi, row);
+    }
     fence_async_smem();
     tc_fence_before();
     __syncthreads();
@@ -259,7 +266,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 struct Layout {
   int ntiles, nsplit;           // key tiles per head and key ranges per head
   int qtiles;                   // query tiles per head
-  size_t off_part, off_img, total;
+  size_t off_part, off_img, off_kmax, off_shift, total;   // kmax, shift: stabiliser scratch
 };
 
 // Lq queries over Lk keys (equal for self-attention).
@@ -273,7 +280,9 @@ Layout layout(int B, int H, int Lq, int Lk, int m) {
   if (s.nsplit > s.ntiles) s.nsplit = s.ntiles;
   s.off_part = kWsHeader;
   s.off_img = align_up(s.off_part + (size_t)bh * s.nsplit * 65 * m * 4, 1024);
-  s.total = align_up(s.off_img + (size_t)bh * img_bytes(m), 256);
+  s.off_kmax = align_up(s.off_img + (size_t)bh * img_bytes(m), 256);
+  s.off_shift = align_up(s.off_kmax + (size_t)bh * 4, 256);
+  s.total = align_up(s.off_shift + (size_t)bh * 4, 256);
   return s;
 }
 
@@ -288,7 +297,14 @@ cudaError_t launch(const FwdArgs& a, const CUtensorMap& tw, const CUtensorMap& t
   uint8_t* images = (uint8_t*)(ws + s.off_img);
   const int bh = a.B * a.H;
 
-  cudaError_t e = tc_launch_key_states(a, tw, tk, tv, s.ntiles, s.nsplit, partials);
+  const bool stab = (a.flags & DARK_STABILISE) != 0;
+  float* kshift = (float*)(ws + s.off_shift);
+  cudaError_t e;
+  if (stab) {
+    e = tc_key_shift(a, tw, tk, tv, (int*)(ws + s.off_kmax), kshift);
+    if (e != cudaSuccess) return e;
+  }
+  e = tc_launch_key_states(a, tw, tk, tv, s.ntiles, s.nsplit, partials, stab ? kshift : nullptr);
   if (e != cudaSuccess) return e;
   reduce_kernel<<<dim3((65 * a.m + 255) / 256, bh), 256, 0, a.stream>>>(partials, s.nsplit, a.m,
                                                                          images, a.st_kv, a.st_z);
@@ -306,6 +322,7 @@ cudaError_t launch(const FwdArgs& a, const CUtensorMap& tw, const CUtensorMap& t
   qp.total_tiles = bh * s.qtiles;
   qp.qmask = a.qmask;
   qp.images = images;
+  qp.stab_q = stab ? 1 : 0;
   qp.dev_status = a.dev_status;
   qp.stall = test_stall_cycles();
   using QG = QueryCfg<M_, R_>;
@@ -320,7 +337,7 @@ cudaError_t launch(const FwdArgs& a, const CUtensorMap& tw, const CUtensorMap& t
 }  // namespace
 
 bool tc_noncausal_supported(FwdArgs& a) {
-  if (a.dtype != DARK_BF16 || a.d != kD || (a.flags & DARK_STABILISE)) return false;
+  if (a.dtype != DARK_BF16 || a.d != kD) return false;
   if (!(a.m == 128 || a.m == 256) || a.r % 16 != 0 || a.r < 16 || a.r > 64) return false;
   return tc_make_maps(a);
 }

@@ -86,20 +86,45 @@ def test_stabiliser_changes_nothing(D, cuda_ok, name):
     assert np.abs(res["z"] - zs).max() <= 2e-2 * np.abs(zs).max()
 
 
-def test_stabiliser_avoids_overflow(D, cuda_ok):
+@pytest.mark.parametrize("recipe", ["f32-causal", "bf16-causal", "bf16-noncausal"])
+def test_stabiliser_avoids_overflow(D, cuda_ok, recipe):
     # Queries scaled by 6: their exponents reach ~2^138 and overflow fp32 unless
     # the per-query constant is subtracted (key exponents are bounded by
     # |omega_j|^2 / 2 and stay in range). Without the flag the device reports a
-    # non-finite output; with it the result matches the oracle.
-    w = synth.WORKLOADS[1].with_sizes(L=130, causal=True)
+    # non-finite output; with it the result matches the oracle. fp32 runs the
+    # FFMA kernels, bf16 (d = 64) the tensor-core kernels.
+    w = {"f32-causal": synth.WORKLOADS[1].with_sizes(L=130, causal=True),
+         "bf16-causal": synth.WORKLOADS[2].with_sizes(H=2, L=260, lengths=(260, 199)),
+         "bf16-noncausal": synth.WORKLOADS[3].with_sizes(H=2, L=300)}[recipe]
     inp = synth.make_inputs(w)
     inp = dict(inp, q=inp["q"] * 6.0)
-    res = forward(D, w, inp, cuda_ok, flags=D.DARK_CAUSAL)
+    causal = D.DARK_CAUSAL if w.causal else 0
+    res = forward(D, w, inp, cuda_ok, flags=causal)
     assert res["status"] == D.DARK_ERR_NUMERIC
-    res = forward(D, w, inp, cuda_ok, flags=D.DARK_CAUSAL | D.DARK_STABILISE)
+    res = forward(D, w, inp, cuda_ok, flags=causal | D.DARK_STABILISE)
     assert res["status"] == 0
-    out, _, _ = _oracle(inp, True)
-    check(w, res["out"], out)
+    out, _, _ = _oracle(inp, w.causal)
+    if w.dtype == "f32":
+        check(w, res["out"], out)
+    else:
+        # bf16 tokens meet an fp16 W' (each entry within 2^-11 of itself), so
+        # the base-2 query exponent j of token i moves by at most
+        # 2^-11 sum_t |W'_jt q_it|: about 0.1 at these 2^138 exponents. A
+        # convex mix whose feature weights move by the factor 2^(+-de) moves by
+        # at most 2 ln2 de max|v|; that bound, over the usual 2e-2, is the
+        # tolerance here.
+        d = inp["q"].shape[-1]
+        de = 0.0
+        for h in range(w.H):
+            wtop = np.log2(np.e) * d ** -0.25 * (inp["omega"][0].astype(np.float64)
+                                                 @ inp["geom"][h % inp["geom"].shape[0]]
+                                                 .astype(np.float64))
+            qh = np.abs(inp["q"][:, h].astype(np.float64)).reshape(-1, d)
+            de = max(de, 2.0 ** -11 * float((qh @ np.abs(wtop).T).max()))
+        tol = 2e-2 + 2 * np.log(2) * de * float(np.abs(inp["v"]).max())
+        assert np.all(np.isfinite(res["out"]))
+        err = float(np.abs(res["out"] - out).max())
+        assert err <= tol, (err, tol, de)
 
 
 def test_rows_without_valid_keys_are_zero(D, cuda_ok):

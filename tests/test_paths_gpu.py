@@ -42,6 +42,20 @@ if case.startswith("bwd"):
     mask = torch.from_numpy(inp["mask"]).to(dev)
     fn = lambda: D.dark_attention_bwd(omega, geom, q, k, v, g, *grads, w.B, w.H, w.L, D.DARK_BF16,
                                       key_mask=mask, flags=flags, dgeom=dgeom, ws=ws)
+elif case.startswith("fwd"):
+    w = {"fwd-stab-causal": synth.WORKLOADS[2].with_sizes(H=2, L=300, lengths=(300, 217)),
+         "fwd-stab-noncausal": synth.WORKLOADS[3].with_sizes(H=2, L=300)}[case]
+    inp = synth.make_inputs(w)
+    omega = torch.from_numpy(inp["omega"]).to(dev)
+    geom = torch.from_numpy(inp["geom"]).to(dev)
+    proj, _wb = D.dark_make_projection(omega, geom, w.H, D.DARK_BF16)
+    q, k, v = (torch.from_numpy(inp[n]).to(dev).to(torch.bfloat16) for n in ("q", "k", "v"))
+    out = torch.empty_like(q)
+    mask = None if inp["mask"] is None else torch.from_numpy(inp["mask"]).to(dev)
+    flags = (D.DARK_CAUSAL if w.causal else 0) | D.DARK_STABILISE
+    ws = D.alloc_workspace(proj, w.B, w.H, w.L, flags, dev)
+    fn = lambda: D.dark_attention_fwd(proj, q, k, v, out, w.B, w.H, w.L, key_mask=mask,
+                                      flags=flags, ws=ws)
 print(json.dumps(kernels(fn)))
 '''
 
@@ -60,3 +74,14 @@ def test_bf16_backward_runs_on_tensor_cores(cuda_ok, case):
                    "tbf_dw_kernel"):
         assert any(kernel in n for n in names), (kernel, names)
     assert not any("pass_kernel<" in n and "tbf_" not in n for n in names), names
+
+
+@pytest.mark.parametrize("case,kernel", [("fwd-stab-causal", "causal_kernel"),
+                                         ("fwd-stab-noncausal", "queries_kernel")])
+def test_stabilised_forward_runs_on_tensor_cores(cuda_ok, case, kernel):
+    # DARK_STABILISE on bf16 d = 64: the key-constant pass runs in keys_kernel,
+    # the attention in the tensor-core kernels; none of the FFMA kernels
+    names = launched(case)
+    assert any(kernel in n for n in names), names
+    assert any("keys_kernel" in n for n in names), names
+    assert not any(("out_kernel" in n or "scan_kernel" in n) for n in names), names
