@@ -37,20 +37,23 @@ L2_FLUSH_BYTES = 512 << 20        # > 126 MB L2
 
 METRIC = "DARK attention fwd tokens/s (B\u00b7H\u00b7L/s) on 1 B200; % of BF16-tensor/HBM roofline"
 
-# DRAM bytes (read + write) per forward call from one ncu capture of the causal
-# masked workload (B2 H8 L2048 d64 r64 m256), summed over its two launches
-# (key states, causal chunks; no bytes written back within either launch).
-# Reported only while the kernel sources hash to what was captured.
-_CAUSAL_SOURCES = ("tc_causal.cu", "tc_keys.cu", "tc_keys.cuh", "tc_common.cuh")
-_NCU_TRAFFIC = {2: ("2d9f70c43543c0ba", 8.759040e6 + 21.510656e6)}
+# DRAM bytes (read + write) per forward call from one ncu capture per kernel
+# of the call, summed over its launches: the large-head causal workload
+# (B4 H8 L8192 d256 r256 m512; features_kernel 271.8 + 553.5 MB, values_kernel
+# 745.4 + 121.8 MB). Reported only while the kernel sources hash to what was
+# captured.
+_NCU_TRAFFIC = {
+    4: (("tc_wide.cu", "tc_common.cuh", "common.cuh", "internal.h"), "890d6f26930e3504",
+        271.831040e6 + 553.532416e6 + 745.381120e6 + 121.838592e6),
+}
 
 
 def captured_traffic(cfg: int):
     if cfg not in _NCU_TRAFFIC:
         return None
-    digest, nbytes = _NCU_TRAFFIC[cfg]
+    sources, digest, nbytes = _NCU_TRAFFIC[cfg]
     h = hashlib.sha256()
-    for f in _CAUSAL_SOURCES:
+    for f in sources:
         with open(os.path.join(ROOT, "random_feature_linear_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return nbytes if h.hexdigest()[:16] == digest else None
@@ -370,7 +373,8 @@ def run_native(args, w: synth.Workload, rank: int, world: int, dev) -> dict | No
         short = sorted({k.replace("(anonymous namespace)::", "").split("(")[0].split("<")[0].split("::")[-1]
                         for k in kernel_names if "dark::" in k})
         roof["kernel"] = "forward call" + (" (" + ", ".join(short) + ")" if short else "")
-        roof["traffic"] = captured_traffic(args.workload)
+        # the capture is of the plain call's kernels (not the stabilised one)
+        roof["traffic"] = None if args.stabilise else captured_traffic(args.workload)
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
         with oracle_threads() as ot:
