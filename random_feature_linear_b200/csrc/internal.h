@@ -89,16 +89,12 @@ size_t tc_causal_workspace_bytes(int B, int H, int L, int m, int d);
 cudaError_t tc_causal_forward(const FwdArgs& a);
 
 bool tc_noncausal_supported(FwdArgs& a);
-// Per-range key states Phi(K)^T [V | 1] as fp32 [B*H*nsplit][65][m] (tcgen05);
-// kshift: null, or the per-(batch, head) key constant of the stabiliser.
+// Per-range key states Phi(K)^T [V | 1] as fp32 [B*H*nsplit][65][m] (tcgen05).
+// shifts: null, or (stabiliser) [B*H*nsplit] receiving each range's largest
+// valid key exponent (-inf without one), which its state is scaled by 2^-shift.
 cudaError_t tc_launch_key_states(const FwdArgs& a, const CUtensorMap& tw, const CUtensorMap& tk,
                                  const CUtensorMap& tv, int ntiles, int nsplit, float* partials,
-                                 const float* kshift);
-// The stabiliser's key constant c_K per (batch, head): the largest exponent of
-// a valid key (0 without one), into shift[B*H] and the state's shift when
-// a.st_shift is set; kmax is [B*H] ints of scratch.
-cudaError_t tc_key_shift(const FwdArgs& a, const CUtensorMap& tw, const CUtensorMap& tk,
-                         const CUtensorMap& tv, int* kmax, float* shift);
+                                 float* shifts);
 size_t tc_noncausal_workspace_bytes(int B, int H, int Lq, int Lk, int m, int d);
 cudaError_t tc_noncausal_forward(const FwdArgs& a);
 

@@ -87,10 +87,13 @@ struct Params {
   int nseg;                     // segments per head
   const float* seg_sums;        // [B*H*nseg][65][m] per-segment key states (nseg > 1)
   float *st_kv, *st_z;          // state after the last chunk
-  // stabiliser: per-(batch, head) key constants (null: none) and whether query
-  // exponents are taken relative to their row maximum
-  const float* kshift;
-  int stab_q;
+  // stabiliser (stab != 0): the key exponents of a CTA are taken relative to the
+  // running maximum over the keys seen so far (the earlier segments' maxima in
+  // seg_shift, then this segment's chunks), the prefix rescaled when it grows;
+  // the query exponents relative to their row maximum
+  const float* seg_shift;       // [B*H*nseg] (nseg > 1)
+  float* st_shift;              // the state's key constant (state output)
+  int stab;
   int* dev_status;
   long long stall;              // testing stall before the first wait (0: none)
 };
@@ -148,6 +151,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   uint32_t ph_tma = 0, ph_mma = 0;
   float run[65];                               // prefix state row `feat` (fp32)
+  float c_run = -INFINITY;                     // stabiliser: running key maximum
 #pragma unroll
   for (int i = 0; i < 65; ++i) run[i] = 0.f;
   bool abort = false;
@@ -210,7 +214,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int i = 0; i < 16; ++i) nrm = fmaf(v[i], v[i], nrm);
       }
       nrm += 0.5f * __log2f((float)M_);
-      if (p.kshift != nullptr) nrm += p.kshift[bh];
       // the norm columns are read: the query GEMM may now overwrite them
       tc_fence_before();
       __syncthreads();
@@ -226,6 +229,39 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int tok = t0 + row;
       bool valid = tok < p.L;
       if (valid && p.mask != nullptr) valid = p.mask[(size_t)b * p.L + tok] != 0;
+      if (p.stab) {
+        // the running maximum starts from the earlier segments' maxima (the
+        // key-state launch's results), then takes each chunk's largest valid
+        // key exponent; the prefix carried in registers follows it
+        if (c == c_begin && seg > 0) {
+          asm volatile("griddepcontrol.wait;" ::: "memory");
+          for (int g = 0; g < seg; ++g) c_run = fmaxf(c_run, p.seg_shift[bh * p.nseg + g]);
+        }
+        float mx = -INFINITY;
+        for (int c0 = half * (M_ / 2); c0 < (half + 1) * (M_ / 2); c0 += 32) {
+          float v[32];
+          tmem_ld32(lane_tm + G::tP + c0, v);
+#pragma unroll
+          for (int e = 0; e < 32; ++e) mx = fmaxf(mx, v[e]);
+        }
+        mx = warp_max(valid ? mx - nrm : -INFINITY);
+        float* red = (float*)(sm + G::oRed);
+        if (lane == 0) red[warp] = mx;
+        __syncthreads();
+        float cmx = red[0];
+#pragma unroll
+        for (int w = 1; w < kThreads / 32; ++w) cmx = fmaxf(cmx, red[w]);
+        __syncthreads();
+        if (cmx > c_run) {
+          if (c_run > -INFINITY) {
+            const float sc = exp2f(c_run - cmx);
+#pragma unroll
+            for (int i = 0; i < 65; ++i) run[i] *= sc;
+          }
+          c_run = cmx;
+        }
+        if (c_run > -INFINITY) nrm += c_run;
+      }
       exp2_rows_to_smem(lane_tm + G::tP, half * (M_ / 2), (half + 1) * (M_ / 2), nrm, !valid,
                         s0 + G::oPhi, row);
     }
@@ -237,7 +273,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     // ------------------------------------------------- epilogue: Psi(Q_c)
     {
-      const float qoff = p.stab_q ? row_max_pair(lane_tm + G::tQ, half, M_ / 2,
+      const float qoff = p.stab ? row_max_pair(lane_tm + G::tQ, half, M_ / 2,
                                                   (float*)(sm + G::oRed), row)
                                   : 0.f;
       exp2_rows_to_smem(lane_tm + G::tQ, half * (M_ / 2), (half + 1) * (M_ / 2), qoff, false,
@@ -273,11 +309,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       // (written by the key-state launch, which may still be finishing: this
       // launch starts early and waits for it only here), added in segment order
       asm volatile("griddepcontrol.wait;" ::: "memory");
+      // stabiliser: segment g's sum is scaled by 2^-(its maximum); c_run (set
+      // in the key epilogue above) is at least every one of them
       if (has_feat) {
         for (int g = 0; g < seg; ++g) {
           const float* sp = p.seg_sums + (size_t)(bh * p.nseg + g) * 65 * M_ + feat;
+          float sc = 1.f;
+          if (p.stab) {
+            const float cg = p.seg_shift[bh * p.nseg + g];
+            if (!(cg > -INFINITY)) continue;
+            sc = exp2f(cg - c_run);
+          }
 #pragma unroll
-          for (int i = 0; i < 65; ++i) run[i] += sp[(size_t)i * M_];
+          for (int i = 0; i < 65; ++i) run[i] += sc * sp[(size_t)i * M_];
         }
       }
     }
@@ -428,6 +472,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int i = 0; i < 64; ++i) kv[i] = run[i];
     p.st_z[(size_t)bh * M_ + feat] = run[64];
   }
+  if (!abort && p.st_shift != nullptr && tid == 0 && c_end == p.nc)
+    p.st_shift[bh] = c_run > -INFINITY ? c_run : 0.f;
   if (abort && tid == 0) {
     // no copy or MMA of this CTA may still be running when TMEM is freed
     drain_loads(bar_tma, tma_issued, tma_waited);
@@ -443,7 +489,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 struct Layout {
   int nc, nseg;
-  size_t off_seg, off_kmax, off_shift, total;   // kmax, shift: stabiliser scratch
+  size_t off_seg, off_shift, total;   // shift: the stabiliser's per-segment maxima
 };
 
 // Segments per head: 1 when the heads alone fill the SMs, else enough to give
@@ -455,9 +501,8 @@ Layout layout(int B, int H, int L, int m) {
   s.nseg = bh >= kSms ? 1 : kSms / bh;
   if (s.nseg > s.nc) s.nseg = s.nc;
   s.off_seg = kWsHeader;
-  s.off_kmax = align_up(s.off_seg + (s.nseg > 1 ? (size_t)bh * s.nseg * 65 * m * 4 : 0), 256);
-  s.off_shift = align_up(s.off_kmax + (size_t)bh * 4, 256);
-  s.total = align_up(s.off_shift + (size_t)bh * 4, 256);
+  s.off_shift = align_up(s.off_seg + (s.nseg > 1 ? (size_t)bh * s.nseg * 65 * m * 4 : 0), 256);
+  s.total = align_up(s.off_shift + (size_t)bh * s.nseg * 4, 256);
   return s;
 }
 
@@ -470,13 +515,9 @@ cudaError_t launch(const FwdArgs& a, const CUtensorMap& tw, const CUtensorMap& t
   float* seg = (float*)((char*)a.ws + s.off_seg);
   cudaError_t e;
   const bool stab = (a.flags & DARK_STABILISE) != 0;
-  float* kshift = (float*)((char*)a.ws + s.off_shift);
-  if (stab) {
-    e = tc_key_shift(a, tw, tk, tv, (int*)((char*)a.ws + s.off_kmax), kshift);
-    if (e != cudaSuccess) return e;
-  }
+  float* seg_shift = (float*)((char*)a.ws + s.off_shift);
   if (s.nseg > 1) {
-    e = tc_launch_key_states(a, tw, tk, tv, s.nc, s.nseg, seg, stab ? kshift : nullptr);
+    e = tc_launch_key_states(a, tw, tk, tv, s.nc, s.nseg, seg, stab ? seg_shift : nullptr);
     if (e != cudaSuccess) return e;
   }
   Params p;
@@ -495,8 +536,9 @@ cudaError_t launch(const FwdArgs& a, const CUtensorMap& tw, const CUtensorMap& t
   p.seg_sums = seg;
   p.st_kv = a.st_kv;
   p.st_z = a.st_z;
-  p.kshift = stab ? kshift : nullptr;
-  p.stab_q = stab ? 1 : 0;
+  p.seg_shift = seg_shift;
+  p.st_shift = stab ? a.st_shift : nullptr;
+  p.stab = stab ? 1 : 0;
   p.dev_status = a.dev_status;
   p.stall = test_stall_cycles();
   static int smem_set[64];

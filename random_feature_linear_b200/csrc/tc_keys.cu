@@ -27,11 +27,10 @@ struct KeyParams {
   const uint8_t* mask;
   int B, H, L, ntiles, nsplit, heads_w;
   float* partials;                 // [B*H*nsplit][65][m]
-  // stabiliser: kmax non-null -> max pass only (the largest valid key exponent
-  // of each (batch, head) into kmax as an ordered int, nothing else written);
-  // kshift non-null -> the per-(batch, head) key constant subtracted in base 2
-  int* kmax;
-  const float* kshift;
+  // stabiliser (null: off): each CTA subtracts the running maximum of its valid
+  // key exponents, rescaling the state accumulated so far when it grows, and
+  // writes that maximum (-inf without a valid key) to shifts[B*H*nsplit]
+  float* shifts;
   int* dev_status;
   long long stall;                 // testing stall before the first wait (0: none)
 };
@@ -49,7 +48,8 @@ struct KeyCfg {
   static constexpr uint32_t oOnes = oV + 2 * kTileBytes;
   static constexpr uint32_t oPhi = oOnes + kTileBytes;
   static constexpr uint32_t oBar = oPhi + kPhi;
-  static constexpr uint32_t kSmem = oBar + 64 + 1024;
+  static constexpr uint32_t oRed = oBar + 64;              // [8] per-warp maxima
+  static constexpr uint32_t kSmem = oRed + 64 + 1024;
   static_assert(kSmem <= 232448, "shared memory");
   static constexpr uint32_t tP = 0, tD = 320;
 };
@@ -84,12 +84,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(bar_never, 1);
     fence_mbar_init();
     if (te > tb) {
-      // the max pass reads no values
-      mbar_arrive_expect_tx(&bar_kv[0], G::kW + (p.kmax ? 1 : 2) * kTileBytes);
+      mbar_arrive_expect_tx(&bar_kv[0], G::kW + 2 * kTileBytes);
       for (int r0 = 0; r0 < G::NW; r0 += 16)
         tma_load_2d(sm + G::oW + r0 * 128, &tm_w, 0, hw * G::NW + r0, &bar_kv[0]);
       tma_load_4d(sm + G::oK, &tm_k, 0, tb * kT, h, b, &bar_kv[0]);
-      if (!p.kmax) tma_load_4d(sm + G::oV, &tm_v, 0, tb * kT, h, b, &bar_kv[0]);
+      tma_load_4d(sm + G::oV, &tm_v, 0, tb * kT, h, b, &bar_kv[0]);
     }
   }
   __syncwarp();
@@ -106,6 +105,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t lane_tm = tmem + ((uint32_t)(quad * 32) << 16);
 
   uint32_t ph_kv = 0, ph_mma = 0;             // bit i: phase parity of buffer i
+  float c_run = -INFINITY;                     // stabiliser: running key maximum
   bool abort = false;
   int issued[2] = {te > tb ? 1 : 0, 0}, waited[2] = {0, 0};   // load phases per buffer
   if (te > tb && p.stall > 0 && !wait_all(bar_never, 0, p.dev_status, p.stall)) abort = true;
@@ -138,10 +138,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (tid == 0 && t + 1 < te) {
       const int nb = buf ^ 1;
       ++issued[nb];
-      mbar_arrive_expect_tx(&bar_kv[nb], (p.kmax ? 1 : 2) * kTileBytes);
+      mbar_arrive_expect_tx(&bar_kv[nb], 2 * kTileBytes);
       tma_load_4d(sm + G::oK + nb * kTileBytes, &tm_k, 0, (t + 1) * kT, h, b, &bar_kv[nb]);
-      if (!p.kmax)
-        tma_load_4d(sm + G::oV + nb * kTileBytes, &tm_v, 0, (t + 1) * kT, h, b, &bar_kv[nb]);
+      tma_load_4d(sm + G::oV + nb * kTileBytes, &tm_v, 0, (t + 1) * kT, h, b, &bar_kv[nb]);
     }
     {
       float nrm = 0.f;
@@ -153,12 +152,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int e = 0; e < 16; ++e) nrm = fmaf(v[e], v[e], nrm);
       }
       nrm += 0.5f * __log2f((float)M_);
-      if (p.kshift != nullptr) nrm += p.kshift[bh];
       const int tok = t * kT + row;
       bool valid = tok < p.L;
       if (valid && p.mask != nullptr) valid = p.mask[(size_t)b * p.L + tok] != 0;
-      if (p.kmax != nullptr) {
-        // max pass: the largest exponent of this thread's half of the features
+      if (p.shifts != nullptr) {
+        // the tile's largest valid exponent, then the running maximum; the
+        // state accumulated so far (its MMAs completed with this tile's
+        // feature GEMM) is rescaled when the maximum grows
         float mx = -INFINITY;
         for (int c0 = half * (M_ / 2); c0 < (half + 1) * (M_ / 2); c0 += 32) {
           float v[32];
@@ -167,10 +167,30 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int e = 0; e < 32; ++e) mx = fmaxf(mx, v[e]);
         }
         mx = warp_max(valid ? mx - nrm : -INFINITY);
-        if (lane == 0 && mx > -INFINITY) atomicMax(p.kmax + bh, float_to_ordered(mx));
-        tc_fence_before();
-        __syncthreads();           // the next feature GEMM overwrites these columns
-        continue;
+        float* red = (float*)(sm + G::oRed);
+        if (lane == 0) red[warp] = mx;
+        __syncthreads();
+        float tmx = red[0];
+#pragma unroll
+        for (int w = 1; w < kThreads / 32; ++w) tmx = fmaxf(tmx, red[w]);
+        __syncthreads();
+        if (tmx > c_run) {
+          if (t > tb && c_run > -INFINITY && half < G::MB) {
+            const float sc = exp2f(c_run - tmx);
+            const uint32_t base = lane_tm + G::tD + 80 * half;
+            float v[32];
+#pragma unroll
+            for (int c0 = 0; c0 < 64; c0 += 32) {
+              tmem_ld32(base + c0, v);
+#pragma unroll
+              for (int e = 0; e < 32; ++e) v[e] *= sc;
+              tmem_st32(base + c0, v);
+            }
+            tmem_st1(base + 64, tmem_ld1(base + 64) * sc);
+          }
+          c_run = tmx;
+        }
+        if (c_run > -INFINITY) nrm += c_run;
       }
       exp2_rows_to_smem(lane_tm + G::tP, half * (M_ / 2), (half + 1) * (M_ / 2), nrm, !valid,
                         s0 + G::oPhi, row);
@@ -206,7 +226,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     drain_loads(&bar_kv[1], issued[1], waited[1]);
     drain_mmas(bar_drain);
   }
-  if (!abort && half < G::MB && p.kmax == nullptr) {
+  if (!abort && tid == 0 && p.shifts != nullptr) p.shifts[(size_t)bh * p.nsplit + split] = c_run;
+  if (!abort && half < G::MB) {
     const int f = half * 128 + row;
     float* dst = p.partials + ((size_t)bh * p.nsplit + split) * 65 * M_;
     if (te > tb) {
@@ -235,10 +256,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 template <int M_, int R_>
 cudaError_t launch_keys_t(const FwdArgs& a, const CUtensorMap& tw, const CUtensorMap& tk,
                           const CUtensorMap& tv, int ntiles, int nsplit, float* partials,
-                          int* kmax, const float* kshift) {
+                          float* shifts) {
   KeyParams kp;
-  kp.kmax = kmax;
-  kp.kshift = kshift;
+  kp.shifts = shifts;
   kp.mask = a.mask;
   kp.B = a.B;
   kp.H = a.H;
@@ -259,14 +279,12 @@ cudaError_t launch_keys_t(const FwdArgs& a, const CUtensorMap& tw, const CUtenso
 
 }  // namespace
 
-namespace {
-
-cudaError_t launch_keys(const FwdArgs& a, const CUtensorMap& tw, const CUtensorMap& tk,
-                        const CUtensorMap& tv, int ntiles, int nsplit, float* partials, int* kmax,
-                        const float* kshift) {
+cudaError_t tc_launch_key_states(const FwdArgs& a, const CUtensorMap& tw, const CUtensorMap& tk,
+                                 const CUtensorMap& tv, int ntiles, int nsplit, float* partials,
+                                 float* shifts) {
 #define DARK_KEYS_CASE(MM, RR)                                                              \
   if (a.m == MM && a.r == RR)                                                               \
-    return launch_keys_t<MM, RR>(a, tw, tk, tv, ntiles, nsplit, partials, kmax, kshift);
+    return launch_keys_t<MM, RR>(a, tw, tk, tv, ntiles, nsplit, partials, shifts);
   DARK_KEYS_CASE(256, 64)
   DARK_KEYS_CASE(256, 48)
   DARK_KEYS_CASE(256, 32)
@@ -277,44 +295,6 @@ cudaError_t launch_keys(const FwdArgs& a, const CUtensorMap& tw, const CUtensorM
   DARK_KEYS_CASE(128, 16)
 #undef DARK_KEYS_CASE
   return cudaErrorInvalidValue;
-}
-
-__global__ void fill_ordered(int* p, int n) {
-  const int i = blockIdx.x * blockDim.x + threadIdx.x;
-  if (i < n) p[i] = float_to_ordered(-INFINITY);
-}
-
-// c_K = the largest valid key exponent (0 for a head without valid keys)
-__global__ void finalize_shift(const int* kmax, float* shift, float* st_shift, int n) {
-  const int i = blockIdx.x * blockDim.x + threadIdx.x;
-  if (i >= n) return;
-  float c = ordered_to_float(kmax[i]);
-  if (!(c > -INFINITY)) c = 0.f;
-  shift[i] = c;
-  if (st_shift != nullptr) st_shift[i] = c;
-}
-
-}  // namespace
-
-cudaError_t tc_launch_key_states(const FwdArgs& a, const CUtensorMap& tw, const CUtensorMap& tk,
-                                 const CUtensorMap& tv, int ntiles, int nsplit, float* partials,
-                                 const float* kshift) {
-  return launch_keys(a, tw, tk, tv, ntiles, nsplit, partials, nullptr, kshift);
-}
-
-cudaError_t tc_key_shift(const FwdArgs& a, const CUtensorMap& tw, const CUtensorMap& tk,
-                         const CUtensorMap& tv, int* kmax, float* shift) {
-  const int bh = a.B * a.H, ntiles = (a.Lk + 127) / 128;
-  int nsplit = (2 * num_sms() + bh - 1) / bh;
-  if (nsplit > ntiles) nsplit = ntiles;
-  if (nsplit < 1) nsplit = 1;
-  fill_ordered<<<(bh + 255) / 256, 256, 0, a.stream>>>(kmax, bh);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
-  e = launch_keys(a, tw, tk, tv, ntiles, nsplit, nullptr, kmax, nullptr);
-  if (e != cudaSuccess) return e;
-  finalize_shift<<<(bh + 255) / 256, 256, 0, a.stream>>>(kmax, shift, a.st_shift, bh);
-  return cudaGetLastError();
 }
 
 }  // namespace dark

@@ -43,16 +43,29 @@ __host__ __device__ constexpr uint32_t img_bytes(int m) { return 3 * img_s_bytes
 
 // Sums the split partials of each head in split order and writes the query
 // kernel's operand image (hi + lo bf16) and, if requested, the fp32 state.
+// Stabiliser (shifts non-null): partial s is scaled by 2^-shifts[s]; the sum is
+// taken relative to the largest of them, c_K (0 when no key is valid), which
+// is the state's shift.
 __global__ void reduce_kernel(const float* __restrict__ partials, int nsplit, int m,
-                              uint8_t* __restrict__ images, float* __restrict__ st_kv,
-                              float* __restrict__ st_z) {
+                              const float* __restrict__ shifts, uint8_t* __restrict__ images,
+                              float* __restrict__ st_kv, float* __restrict__ st_z,
+                              float* __restrict__ st_shift) {
   const int bh = blockIdx.y;
   const int idx = blockIdx.x * blockDim.x + threadIdx.x;
   if (idx >= 65 * m) return;
   const int col = idx / m, f = idx % m;
   const float* src = partials + (size_t)bh * nsplit * 65 * m + idx;
   float acc = 0.f;
-  for (int s = 0; s < nsplit; ++s) acc += src[(size_t)s * 65 * m];
+  if (shifts == nullptr) {
+    for (int s = 0; s < nsplit; ++s) acc += src[(size_t)s * 65 * m];
+  } else {
+    const float* sh = shifts + (size_t)bh * nsplit;
+    float cmax = -INFINITY;
+    for (int s = 0; s < nsplit; ++s) cmax = fmaxf(cmax, sh[s]);
+    for (int s = 0; s < nsplit; ++s)
+      if (sh[s] > -INFINITY) acc += exp2f(sh[s] - cmax) * src[(size_t)s * 65 * m];
+    if (idx == 0 && st_shift != nullptr) st_shift[bh] = cmax > -INFINITY ? cmax : 0.f;
+  }
   const __nv_bfloat16 hi = __float2bfloat16_rn(acc);
   const __nv_bfloat16 lo = __float2bfloat16_rn(acc - __bfloat162float(hi));
   uint8_t* img = images + (size_t)bh * img_bytes(m);
@@ -266,7 +279,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 struct Layout {
   int ntiles, nsplit;           // key tiles per head and key ranges per head
   int qtiles;                   // query tiles per head
-  size_t off_part, off_img, off_kmax, off_shift, total;   // kmax, shift: stabiliser scratch
+  size_t off_part, off_img, off_shift, total;   // shift: the stabiliser's per-range maxima
 };
 
 // Lq queries over Lk keys (equal for self-attention).
@@ -280,9 +293,8 @@ Layout layout(int B, int H, int Lq, int Lk, int m) {
   if (s.nsplit > s.ntiles) s.nsplit = s.ntiles;
   s.off_part = kWsHeader;
   s.off_img = align_up(s.off_part + (size_t)bh * s.nsplit * 65 * m * 4, 1024);
-  s.off_kmax = align_up(s.off_img + (size_t)bh * img_bytes(m), 256);
-  s.off_shift = align_up(s.off_kmax + (size_t)bh * 4, 256);
-  s.total = align_up(s.off_shift + (size_t)bh * 4, 256);
+  s.off_shift = align_up(s.off_img + (size_t)bh * img_bytes(m), 256);
+  s.total = align_up(s.off_shift + (size_t)bh * s.nsplit * 4, 256);
   return s;
 }
 
@@ -298,16 +310,11 @@ cudaError_t launch(const FwdArgs& a, const CUtensorMap& tw, const CUtensorMap& t
   const int bh = a.B * a.H;
 
   const bool stab = (a.flags & DARK_STABILISE) != 0;
-  float* kshift = (float*)(ws + s.off_shift);
-  cudaError_t e;
-  if (stab) {
-    e = tc_key_shift(a, tw, tk, tv, (int*)(ws + s.off_kmax), kshift);
-    if (e != cudaSuccess) return e;
-  }
-  e = tc_launch_key_states(a, tw, tk, tv, s.ntiles, s.nsplit, partials, stab ? kshift : nullptr);
+  float* shifts = stab ? (float*)(ws + s.off_shift) : nullptr;
+  cudaError_t e = tc_launch_key_states(a, tw, tk, tv, s.ntiles, s.nsplit, partials, shifts);
   if (e != cudaSuccess) return e;
-  reduce_kernel<<<dim3((65 * a.m + 255) / 256, bh), 256, 0, a.stream>>>(partials, s.nsplit, a.m,
-                                                                         images, a.st_kv, a.st_z);
+  reduce_kernel<<<dim3((65 * a.m + 255) / 256, bh), 256, 0, a.stream>>>(
+      partials, s.nsplit, a.m, shifts, images, a.st_kv, a.st_z, a.st_shift);
 
   QueryParams qp;
   qp.out = (__nv_bfloat16*)a.out;
