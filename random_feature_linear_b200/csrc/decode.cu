@@ -416,9 +416,205 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(
 }
 
 
+
+// Two batch rows of one projection head per CTA, for bf16 tokens without the
+// stabiliser: the rows b = 2i and 2i + 1 share the staged W' (one bulk copy)
+// and the block's two feature GEMVs. The tokens load first and alone (queued
+// behind the step's 34 MB of state they took several microseconds); once the
+// GEMVs are done the first row's state streams into registers and the second
+// row's into shared memory by bulk copies (B * H / 2 CTAs, two per SM: one wave
+// for 512 heads).
+struct PairLayout {
+  uint32_t vec, w, st, total;     // byte offsets: vectors, W', second state; total
+};
+__host__ __device__ inline PairLayout pair_layout(int m, int r, int d) {
+  PairLayout L;
+  const int rpp = kThreads / (d / 4);
+  // xq, xk, xv (2 rows), pk (2 x (m + r)), pq (2 x m), scratch [32], barriers
+  L.vec = 0;
+  const uint32_t vec_bytes = (uint32_t)(6 * d + 2 * (m + r) + 2 * m + 32) * 4 + 32;
+  L.w = (vec_bytes + 127) / 128 * 128;
+  // W' (fp16); once the GEMVs are done the same bytes hold the partial sums
+  const uint32_t wb = (uint32_t)(m + r) * d * 2, red = (uint32_t)rpp * d * 4;
+  L.st = L.w + ((wb > red ? wb : red) + 127) / 128 * 128;
+  L.total = L.st + (uint32_t)m * d * 4;
+  return L;
+}
+
+__global__ void __launch_bounds__(kThreads, 2) decode_pair_kernel(
+    const __half* __restrict__ w, int heads_w, int m, int r, int d, float* __restrict__ kv,
+    float* __restrict__ z, int H, const __nv_bfloat16* __restrict__ q,
+    const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ v,
+    __nv_bfloat16* __restrict__ out, const uint8_t* __restrict__ valid, int* dev_status) {
+  extern __shared__ __align__(128) uint8_t smp[];
+  const PairLayout Lp = pair_layout(m, r, d);
+  const int tpr = d / 4, rpp = kThreads / tpr, nb = m / rpp;   // nb <= kBatchRows
+  float* xq = reinterpret_cast<float*>(smp + Lp.vec);           // [2][d]
+  float* xk = xq + 2 * d;                                       // [2][d]
+  float* xv = xk + 2 * d;                                       // [2][d]
+  float* pk = xv + 2 * d;                                       // [2][m + r]
+  float* pq = pk + 2 * (m + r);                                 // [2][m]
+  float* scratch = pq + 2 * m;                                  // [32]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(scratch + 32);   // W', second state
+  __half* w_sm = reinterpret_cast<__half*>(smp + Lp.w);
+  float* red = reinterpret_cast<float*>(smp + Lp.w);            // after the GEMVs
+  const float* st2 = reinterpret_cast<const float*>(smp + Lp.st);
+  const int h = blockIdx.x % H, bp = blockIdx.x / H;
+  const int bhs[2] = {(2 * bp) * H + h, (2 * bp + 1) * H + h};
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const uint32_t w_bytes = (uint32_t)(m + r) * d * 2, s_bytes = (uint32_t)m * d * 4;
+  if (tid == 0) {
+    tc::mbar_init(bars, 1);
+    tc::mbar_init(bars + 1, 1);
+    tc::fence_mbar_init();
+    const uint8_t* wg = reinterpret_cast<const uint8_t*>(w + (size_t)(heads_w == 1 ? 0 : h) * (m + r) * d);
+    tc::mbar_arrive_expect_tx(bars, w_bytes);
+    for (uint32_t o = 0; o < w_bytes; o += 16384)
+      tc::bulk_load(smp + Lp.w + o, wg + o, w_bytes - o < 16384 ? w_bytes - o : 16384, bars);
+  }
+  const int c4 = tid % tpr, r0 = tid / tpr;
+  // the tokens of both rows (they gate the feature GEMVs)
+  const bool has_c = tid < d;
+  if (has_c) {
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      xq[i * d + tid] = __bfloat162float(q[(size_t)bhs[i] * d + tid]);
+      xk[i * d + tid] = __bfloat162float(k[(size_t)bhs[i] * d + tid]);
+      xv[i * d + tid] = __bfloat162float(v[(size_t)bhs[i] * d + tid]);
+    }
+  }
+  __syncthreads();
+  bool ok = tc::mbar_wait(bars, 0);
+  if (__syncthreads_or(ok ? 0 : 1)) {
+    if (tid == 0) {
+      report(dev_status, DARK_ERR_TIMEOUT);
+      tc::mbar_wait(bars, 0);        // no copy may land after the block is gone
+    }
+    __syncthreads();
+    return;
+  }
+  // feature exponents of both rows from the staged W'; key norms per row
+  float ks[2];
+  float4 s[kBatchRows];
+  float zp[2][2];
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    const float part =
+        warp_sum(feature_gemv_shared(w_sm, m, r, d, xk + i * d, xq + i * d, pk + i * (m + r),
+                                     pq + i * m));
+    if (lane == 0) scratch[warp] = part;
+    __syncthreads();
+    float nrm = 0.f;
+#pragma unroll
+    for (int u = 0; u < kThreads / 32; ++u) nrm += scratch[u];
+    ks[i] = nrm + 0.5f * log2f((float)m);
+    __syncthreads();
+  }
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    const bool upd = valid == nullptr || valid[bhs[i] / H] != 0;
+    for (int j = tid; j < m; j += kThreads) {
+      pk[i * (m + r) + j] = upd ? exp2f(pk[i * (m + r) + j] - ks[i]) : 0.f;
+      pq[i * m + j] = exp2f(pq[i * m + j]);
+    }
+  }
+  __syncthreads();                   // W' is read: its bytes now hold partial sums
+  // the state, once this block's GEMVs are done: the second row's by bulk
+  // copies into shared memory, the first row's into registers
+  if (tid == 0) {
+    const uint8_t* sg = reinterpret_cast<const uint8_t*>(kv + (size_t)bhs[1] * m * d);
+    tc::mbar_arrive_expect_tx(bars + 1, s_bytes);
+    for (uint32_t o = 0; o < s_bytes; o += 16384)
+      tc::bulk_load(smp + Lp.st + o, sg + o, s_bytes - o < 16384 ? s_bytes - o : 16384, bars + 1);
+  }
+  float4* base1 = reinterpret_cast<float4*>(kv + (size_t)bhs[0] * m * d) + c4;
+#pragma unroll
+  for (int u = 0; u < kBatchRows; ++u)
+    if (u < nb) s[u] = __ldcs(base1 + (size_t)(r0 + u * rpp) * tpr);
+#pragma unroll
+  for (int i = 0; i < 2; ++i)
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int j = tid + u * kThreads;
+      zp[i][u] = j < m ? __ldcs(z + (size_t)bhs[i] * m + j) : 0.f;
+    }
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    const float* fk = pk + i * (m + r);
+    const float* fq = pq + i * m;
+    if (i == 1) {
+      ok = tc::mbar_wait(bars + 1, 0);
+      if (__syncthreads_or(ok ? 0 : 1)) {
+        if (tid == 0) {
+          report(dev_status, DARK_ERR_TIMEOUT);
+          tc::mbar_wait(bars + 1, 0);
+        }
+        __syncthreads();
+        return;
+      }
+    }
+    float4* base = reinterpret_cast<float4*>(kv + (size_t)bhs[i] * m * d) + c4;
+    const float4 vv = make_float4(xv[i * d + 4 * c4], xv[i * d + 4 * c4 + 1],
+                                  xv[i * d + 4 * c4 + 2], xv[i * d + 4 * c4 + 3]);
+    float4 num = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int u = 0; u < kBatchRows; ++u) {
+      if (u >= nb) break;
+      const int j = r0 + u * rpp;
+      float4 x = i == 0 ? s[u] : reinterpret_cast<const float4*>(st2)[(size_t)j * tpr + c4];
+      const float a = fk[j], c = fq[j];
+      x.x = fmaf(a, vv.x, x.x); x.y = fmaf(a, vv.y, x.y);
+      x.z = fmaf(a, vv.z, x.z); x.w = fmaf(a, vv.w, x.w);
+      __stcs(base + (size_t)j * tpr, x);
+      num.x = fmaf(c, x.x, num.x); num.y = fmaf(c, x.y, num.y);
+      num.z = fmaf(c, x.z, num.z); num.w = fmaf(c, x.w, num.w);
+    }
+    float* rr = red + r0 * d + 4 * c4;
+    rr[0] = num.x; rr[1] = num.y; rr[2] = num.z; rr[3] = num.w;
+    float den = 0.f;
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int j = tid + u * kThreads;
+      if (j < m) {
+        const float zj = zp[i][u] + fk[j];
+        __stcs(z + (size_t)bhs[i] * m + j, zj);
+        den = fmaf(fq[j], zj, den);
+      }
+    }
+    den = block_sum(den, scratch);   // contains the barrier that publishes `red`
+    for (int c = tid; c < d; c += kThreads) {
+      float acc = 0.f;
+      for (int g = 0; g < rpp; ++g) acc += red[g * d + c];
+      const float o = den > 0.f ? acc / den : 0.f;
+      if (!isfinite(o)) report(dev_status, DARK_ERR_NUMERIC);
+      out[(size_t)bhs[i] * d + c] = __float2bfloat16_rn(o);
+    }
+    __syncthreads();                 // red and scratch are reused by the second row
+  }
+}
 }  // namespace
 
 cudaError_t launch_decode(const DecodeArgs& a) {
+  // two batch rows per CTA when the step's tokens are bf16 with an fp16 W' that
+  // fits the staging, no stabiliser, an even batch, and every row's state in
+  // one register pass
+  if (a.dtype == DARK_BF16 && a.shift == nullptr && a.update == 1 && a.B % 2 == 0 &&
+      a.d % 8 == 0 && a.d <= 256 && (size_t)(a.m + a.r) * a.d * 2 <= kStageW &&
+      ((size_t)(a.m + a.r) * a.d * 2) % 16 == 0 && ((uintptr_t)a.w & 15) == 0 &&
+      ((uintptr_t)a.kv & 15) == 0 && (a.m % (kThreads / (a.d / 4))) == 0 &&
+      a.m / (kThreads / (a.d / 4)) <= kBatchRows && a.m <= 2 * kThreads) {
+    const PairLayout L = pair_layout(a.m, a.r, a.d);
+    if (L.total <= 227 * 1024) {
+      static int done[64];
+      cudaError_t err = set_smem_limit_once((const void*)decode_pair_kernel, (int)L.total, done);
+      if (err != cudaSuccess) return err;
+      decode_pair_kernel<<<a.B / 2 * a.H, kThreads, L.total, a.stream>>>(
+          (const __half*)a.w, a.heads_w, a.m, a.r, a.d, a.kv, a.z, a.H,
+          (const __nv_bfloat16*)a.q, (const __nv_bfloat16*)a.k, (const __nv_bfloat16*)a.v,
+          (__nv_bfloat16*)a.out, a.valid, a.dev_status);
+      return cudaGetLastError();
+    }
+  }
   const int tpr = a.d / 4;
   const int rpp = kThreads / tpr;
   const size_t welt = a.dtype == DARK_BF16 ? sizeof(__half) : sizeof(float);

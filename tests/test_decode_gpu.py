@@ -150,13 +150,14 @@ def test_decode_staged_projection_small_m(D, cuda_ok):
         check(w, g[:, :, None], r_[:, :, None])
 
 
-@pytest.mark.parametrize("per_head", [True, False], ids=["per-head-geometry", "shared-geometry"])
-def test_decode_many_heads(D, cuda_ok, per_head):
-    # More heads than twice the SM count: the streaming path (one block per SM
-    # walking heads in projection order, state copied through shared memory),
-    # with invalid tokens in some batch rows and heads of one projection row
-    # spread over several blocks
-    w = synth.WORKLOADS[5].with_sizes(B=41, H=8, L=130, per_head_geom=per_head)
+@pytest.mark.parametrize("per_head,B", [(True, 41), (False, 41), (True, 40), (False, 40)],
+                         ids=["per-head-geometry-odd", "shared-geometry-odd",
+                              "per-head-geometry-even", "shared-geometry-even"])
+def test_decode_many_heads(D, cuda_ok, per_head, B):
+    # More heads than twice the SM count, with invalid tokens in some batch rows:
+    # an even batch runs two batch rows per block (the second row's state through
+    # shared memory), an odd one a row per block
+    w = synth.WORKLOADS[5].with_sizes(B=B, H=8, L=130, per_head_geom=per_head)
     inp = synth.make_inputs(w)
     steps = 3
     stream = synth.decode_stream(w, steps)
