@@ -33,6 +33,24 @@ sys.path.insert(0, ROOT)
 from random_feature_linear_b200 import synth  # noqa: E402
 
 L2_FLUSH_BYTES = 512 << 20        # > 126 MB L2
+L2_CLEAN_BYTES = 256 << 20
+L2_NOTE = ("flushed before every timed step: 512 MiB written, then 256 MiB of other data read "
+           "(no line of the step's data and no dirty line left in L2)")
+
+
+class L2Flush:
+    """Writes a buffer larger than L2, then reads a second one: the write evicts
+    every line the timed call could reuse, the read leaves L2 holding clean
+    lines, so that writing back the flush's own dirty lines is not charged to
+    the next timed call."""
+
+    def __init__(self, dev):
+        self.w = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.int32, device=dev)
+        self.r = torch.zeros(L2_CLEAN_BYTES // 4, dtype=torch.int32, device=dev)
+
+    def __call__(self):
+        self.w.zero_()
+        self.r.sum()
 
 
 METRIC = "DARK attention fwd tokens/s (B\u00b7H\u00b7L/s) on 1 B200; % of BF16-tensor/HBM roofline"
@@ -247,7 +265,7 @@ def run_native(args, w: synth.Workload, rank: int, world: int, dev) -> dict | No
         (D.DARK_STABILISE if args.stabilise else 0)
     ws = D.alloc_workspace(proj, w.B, w.H, w.L, flags, dev)
     status = torch.zeros(1, dtype=torch.int32, device=dev)
-    flush = None if args.ncu else torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.int32, device=dev)
+    flush = None if args.ncu else L2Flush(dev)
     stream = torch.cuda.current_stream()
 
     def step():
@@ -263,7 +281,7 @@ def run_native(args, w: synth.Workload, rank: int, world: int, dev) -> dict | No
         assert int(status.item()) == 0, D.dark_status_string(int(status.item()))
         return None
     for _ in range(args.warmup):
-        flush.zero_()
+        flush()
         step()
     torch.cuda.synchronize()
     # The timed forward is one replay of a CUDA graph holding the API call's
@@ -292,7 +310,7 @@ def run_native(args, w: synth.Workload, rank: int, world: int, dev) -> dict | No
     with ClockSampler(dev.index) as clk:
         wall0 = time.perf_counter()
         for i in range(args.steps):
-            flush.zero_()                       # L2 flush, outside the timed interval
+            flush()                       # L2 flush, outside the timed interval
             starts[i].record(stream)
             graph.replay()
             ends[i].record(stream)
@@ -400,7 +418,7 @@ def run_native(args, w: synth.Workload, rank: int, world: int, dev) -> dict | No
                    "B": w.B, "H": w.H,
                    "L": w.L, "d": w.d, "r": w.r, "m": w.m,
                    "causal": w.causal, "lengths": list(w.lengths) if w.lengths else None,
-                   "l2": "flushed (512 MiB write) before every timed step",
+                   "l2": L2_NOTE,
                    "timing": "CUDA events around one CUDA-graph replay of the forward call per step",
                    "parallelism": f"replicas x{world} (independent batches, no collective)"},
         "e2e": {"value": tokens / (e2e_ms / 1e3), "unit": "tokens/s",
@@ -467,7 +485,7 @@ def run_decode(args, rank: int, world: int, dev) -> dict | None:
     stream_np = synth.decode_stream(w, n_graph, salt=rank)
     sq, sk, sv = (torch.from_numpy(stream_np[n]).to(dev).to(torch.bfloat16) for n in ("q", "k", "v"))
     so = torch.empty_like(sq)
-    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.int32, device=dev)
+    flush = L2Flush(dev)
     stream = torch.cuda.current_stream()
 
     def one(i):
@@ -503,7 +521,7 @@ def run_decode(args, rank: int, world: int, dev) -> dict | None:
     torch.cuda.synchronize()
     with ClockSampler(dev.index) as clk:
         for i in range(args.steps):
-            flush.zero_()
+            flush()
             starts[i].record(stream)
             g1.replay()
             ends[i].record(stream)
@@ -562,7 +580,7 @@ def run_decode(args, rank: int, world: int, dev) -> dict | None:
         "data": "synthetic (seeded numpy, orthogonal Gaussian features)",
         "config": {"workload": "decode after a 4096-token causal prefill (B64 H8 d64 r64 m256, "
                                "fp32 state)", "B": w.B, "H": w.H, "d": w.d, "r": w.r, "m": w.m,
-                   "l2": "flushed (512 MiB write) before every timed step",
+                   "l2": L2_NOTE,
                    "timing": "CUDA events around a one-step CUDA-graph replay",
                    "parallelism": f"replicas x{world} (independent batches, no collective)"},
         "e2e": {"value": rows / (e2e_ms / 1e3), "unit": "tokens/s",
@@ -621,7 +639,7 @@ def run_cross(args, rank: int, world: int, dev) -> dict | None:
     out = torch.empty_like(q)
     ws = D.alloc_cross_workspace(proj, w.B, w.H, lq, lk, 0, dev)
     status = torch.zeros(1, dtype=torch.int32, device=dev)
-    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.int32, device=dev)
+    flush = L2Flush(dev)
     stream = torch.cuda.current_stream()
 
     def call(q_, k_, v_, qm_, cm_):
@@ -629,7 +647,7 @@ def run_cross(args, rank: int, world: int, dev) -> dict | None:
                                    context_mask=cm_, ws=ws, dev_status=status)
 
     for _ in range(args.warmup):
-        flush.zero_()
+        flush()
         call(q, k, v, qm, cm)
     torch.cuda.synchronize()
     graph = torch.cuda.CUDAGraph()
@@ -651,7 +669,7 @@ def run_cross(args, rank: int, world: int, dev) -> dict | None:
     torch.cuda.synchronize()
     with ClockSampler(dev.index) as clk:
         for i in range(args.steps):
-            flush.zero_()
+            flush()
             starts[i].record(stream)
             graph.replay()
             ends[i].record(stream)
@@ -724,7 +742,7 @@ def run_cross(args, rank: int, world: int, dev) -> dict | None:
         "data": "synthetic (seeded numpy, orthogonal Gaussian features)",
         "config": {"workload": f"cross-attention bf16 (B{w.B} H{w.H} Lq{lq} Lk{lk} d{w.d} r{w.r} "
                                f"m{w.m}, all-valid query and context masks)",
-                   "l2": "flushed (512 MiB write) before every timed step",
+                   "l2": L2_NOTE,
                    "timing": "CUDA events around one CUDA-graph replay of the forward call per step",
                    "parallelism": f"replicas x{world} (independent batches, no collective)"},
         "e2e": {"value": tokens / (e2e_ms / 1e3), "unit": "tokens/s",
@@ -791,7 +809,7 @@ def run_backward(args, w: synth.Workload, rank: int, world: int, dev) -> dict | 
     flags = D.DARK_CAUSAL if w.causal else 0
     ws = D.alloc_bwd_workspace(omega, geom, w.B, w.H, w.L, dev)
     status = torch.zeros(1, dtype=torch.int32, device=dev)
-    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.int32, device=dev)
+    flush = L2Flush(dev)
     stream = torch.cuda.current_stream()
 
     def call(q_, k_, v_, g_, m_):
@@ -806,7 +824,7 @@ def run_backward(args, w: synth.Workload, rank: int, world: int, dev) -> dict | 
         assert int(status.item()) == 0, D.dark_status_string(int(status.item()))
         return None
     for _ in range(args.warmup):
-        flush.zero_()
+        flush()
         call(q, k, v, g, mask)
     torch.cuda.synchronize()
     assert int(status.item()) == 0, D.dark_status_string(int(status.item()))
@@ -829,7 +847,7 @@ def run_backward(args, w: synth.Workload, rank: int, world: int, dev) -> dict | 
     torch.cuda.synchronize()
     with ClockSampler(dev.index) as clk:
         for i in range(args.steps):
-            flush.zero_()
+            flush()
             starts[i].record(stream)
             graph.replay()
             ends[i].record(stream)
@@ -909,7 +927,7 @@ def run_backward(args, w: synth.Workload, rank: int, world: int, dev) -> dict | 
         "data": "synthetic (seeded numpy, orthogonal Gaussian features; dout ~ N(0,1))",
         "config": {"workload": "backward of " + w.name, "B": w.B, "H": w.H, "L": w.L, "d": w.d,
                    "r": w.r, "m": w.m, "causal": w.causal,
-                   "l2": "flushed (512 MiB write) before every timed step",
+                   "l2": L2_NOTE,
                    "timing": "CUDA events around one CUDA-graph replay of the backward call per step",
                    "parallelism": f"replicas x{world} (independent batches, no collective)"},
         "e2e": {"value": tokens / (e2e_ms / 1e3), "unit": "tokens/s",
