@@ -57,12 +57,12 @@ METRIC = "DARK attention fwd tokens/s (B\u00b7H\u00b7L/s) on 1 B200; % of BF16-t
 
 # DRAM bytes (read + write) per forward call from one ncu capture per kernel
 # of the call, summed over its launches: the large-head causal workload
-# (B4 H8 L8192 d256 r256 m512; features_kernel 271.8 + 553.5 MB, values_kernel
-# 745.4 + 121.8 MB). Reported only while the kernel sources hash to what was
+# (B4 H8 L8192 d256 r256 m512; features_kernel 271.9 + 553.0 MB, values_kernel
+# 745.5 + 118.0 MB). Reported only while the kernel sources hash to what was
 # captured.
 _NCU_TRAFFIC = {
-    4: (("tc_wide.cu", "tc_common.cuh", "common.cuh", "internal.h"), "890d6f26930e3504",
-        271.831040e6 + 553.532416e6 + 745.381120e6 + 121.838592e6),
+    4: (("tc_wide.cu", "tc_common.cuh", "common.cuh", "internal.h"), "1dd8e5b001a2a74d",
+        271.933440e6 + 552.986624e6 + 745.497088e6 + 118.045952e6),
 }
 
 

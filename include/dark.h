@@ -338,7 +338,10 @@ dark_status dark_attention_bwd(const float* omega, int heads_omega, const float*
  * rows (c_m M); Omega is not used. A query row with no visible key outputs 0.
  * state_out / context_out must be NULL (the mode keeps no recurrent statistics);
  * DARK_STABILISE is accepted and has no effect (the softmax is computed with a
- * running maximum). The workspace queries account for the flag.
+ * running maximum). The workspace queries account for the flag. bf16 I/O with
+ * d = 64 (r <= 64) or d = 128 (r <= 128), r a multiple of 16 and 16-byte aligned
+ * rows runs on the tensor cores; every other shape on the fp32 SIMT kernels, with
+ * the same results within rounding.
  *
  * Auto mode ("exact_threshold"): the exact mode for sequences up to the threshold
  * length, random features for longer ones. dark_auto_uses_exact returns 1 when L <= exact_threshold and

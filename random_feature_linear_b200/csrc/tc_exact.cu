@@ -1,5 +1,6 @@
-// Exact learned-kernel attention on sm_100a tensor cores (bf16 I/O, d = 64,
-// r <= 64): out_i = sum_j softmax_j(u_i . w_j) v_j with u = M q~, w = M k~
+// Exact learned-kernel attention on sm_100a tensor cores (bf16 I/O; d = 64 with
+// r <= 64, d = 128 with r <= 128): out_i = sum_j softmax_j(u_i . w_j) v_j with
+// u = M q~, w = M k~
 // (README, section "Attention modes": in the exact mode M acts on queries and
 // keys and ordinary softmax attention with scaled scores follows).
 //
@@ -11,7 +12,7 @@
 //     scores S = (2 p_q) p_k^T                              tcgen05, N = 128
 //     key mask, causal mask, running row maximum (the two thread halves of a
 //     row exchange their maxima), P = 2^(S - max) as bf16 into shared memory
-//     [num | den] = P [V | 1]                               tcgen05, N = 80
+//     [num | den] = P [V | 1]                               tcgen05, N = d + 16
 //     O = O * 2^(old max - new max) + num, l likewise with den (registers)
 //   out = O / l.
 // The next key tile loads while the current scores are processed, the next
@@ -29,26 +30,34 @@ namespace {
 
 using namespace tc;
 
-constexpr int kD = 64;
 constexpr int kT = 128;                    // queries per CTA, keys per tile
 constexpr int kThreads = kFwdThreads;
-constexpr int kTile = kT * kD * 2;         // one 128 x 64 tile of 16-bit elements
-constexpr uint32_t kTmemCols = 256;
+constexpr int kBlk = kT * 64 * 2;          // one 128 x 64 block of 16-bit elements (16 KB)
 
-// shared memory (all 1024-byte aligned)
-constexpr uint32_t oW = 0;                 // W'_bot: up to 64 rows x 128 B (fp16)
-constexpr uint32_t oQ = 8192;              // Q tile, then 2 p_q (fp16, K-major)
-constexpr uint32_t oK = oQ + kTile;        // K tile, then p_k (fp16, K-major)
-constexpr uint32_t oV = oK + kTile;        // V tile (bf16, keys x d)
-constexpr uint32_t oOnes = oV + kTile;     // bf16 ones: [V | 1] as one N = 80 operand
-constexpr uint32_t oP = oOnes + kTile;     // P: 128 queries x 128 keys bf16, two K blocks
-constexpr uint32_t oMax = oP + 2 * kTile;  // row maxima of the two thread halves
-constexpr uint32_t oKv = oMax + 2 * kT * 4; // validity of the tile's 128 keys (bytes)
-constexpr uint32_t oBar = oKv + kT;
-constexpr uint32_t kSmem = oBar + 64 + 1024;
-// TMEM columns: scores [0, 128); projection [128, 128 + r) and, later in the
-// same tile, [num | den] [128, 208)
-constexpr uint32_t tS = 0, tX = 128;
+// Shared memory (1024-byte aligned blocks) and TMEM of the kernel for head
+// dimension D_: d = 64 fits two CTAs per SM (~106 KB, 256 TMEM columns each),
+// d = 128 one (~177 KB, 512 columns).
+template <int D_>
+struct ExCfg {
+  static constexpr int DS = D_ / 64;                  // 64-column slabs of d
+  static constexpr int RMAX = D_;                     // r <= d (projection blocks fit the tiles)
+  static constexpr uint32_t kWslab = RMAX * 128;      // W'_bot rows of one slab (fp16)
+  static constexpr uint32_t oW = 0;
+  static constexpr uint32_t oQ = oW + DS * kWslab;    // Q tile, then 2 p_q (fp16, K-major blocks)
+  static constexpr uint32_t oK = oQ + DS * kBlk;      // K tile, then p_k
+  static constexpr uint32_t oV = oK + DS * kBlk;      // V tile (bf16, keys x d, DS blocks)
+  static constexpr uint32_t oOnes = oV + DS * kBlk;   // bf16 ones: [V | 1] as one N = d + 16 operand
+  static constexpr uint32_t oP = oOnes + kBlk;        // P: 128 queries x 128 keys bf16, two K blocks
+  static constexpr uint32_t oMax = oP + 2 * kBlk;     // row maxima of the two thread halves
+  static constexpr uint32_t oKv = oMax + 2 * kT * 4;  // validity of the tile's 128 keys (bytes)
+  static constexpr uint32_t oBar = oKv + kT;
+  static constexpr uint32_t kSmem = oBar + 64 + 1024;
+  // TMEM columns: scores [0, 128); projection [128, 128 + r) and, later in the
+  // same tile, [num | den] [128, 128 + d + 16)
+  static constexpr uint32_t tS = 0, tX = 128;
+  static constexpr uint32_t kTmemCols = D_ == 64 ? 256 : 512;
+  static_assert(tX + D_ + 16 <= kTmemCols, "tmem");
+};
 
 struct Params {
   __nv_bfloat16* out;
@@ -61,46 +70,55 @@ struct Params {
 };
 
 // Projection epilogue: this thread's row of the N = r projection in TMEM, times
-// `scale`, as fp16 into a K-major 128B-swizzled tile (columns r..63 zero).
-__device__ __forceinline__ void proj_to_smem(uint32_t lane_taddr, int r, float scale,
+// `scale`, as fp16 into K-major 128B-swizzled 64-column blocks 16 KB apart
+// (columns r and up zero); each thread half writes 32 columns of every block.
+__device__ __forceinline__ void proj_to_smem(uint32_t lane_taddr, int r, int nblk, float scale,
                                              uint32_t tile, int row, int half) {
-  const int c0 = half * 32;
-  uint32_t w[16];
-  if (c0 < r) {
-    float v[32];
-    tmem_ld32(lane_taddr + c0, v);
+  for (int kb = 0; kb < nblk; ++kb) {
+    const int c0 = kb * 64 + half * 32;
+    uint32_t w[16];
+    if (c0 < r) {
+      float v[32];
+      tmem_ld32(lane_taddr + c0, v);
 #pragma unroll
-    for (int e = 0; e < 16; ++e) {
-      const float a = c0 + 2 * e < r ? v[2 * e] * scale : 0.f;
-      const float b = c0 + 2 * e + 1 < r ? v[2 * e + 1] * scale : 0.f;
-      const __half2 hv = __floats2half2_rn(a, b);
-      w[e] = *reinterpret_cast<const uint32_t*>(&hv);
+      for (int e = 0; e < 16; ++e) {
+        const float a = c0 + 2 * e < r ? v[2 * e] * scale : 0.f;
+        const float b = c0 + 2 * e + 1 < r ? v[2 * e + 1] * scale : 0.f;
+        const __half2 hv = __floats2half2_rn(a, b);
+        w[e] = *reinterpret_cast<const uint32_t*>(&hv);
+      }
+    } else {
+#pragma unroll
+      for (int e = 0; e < 16; ++e) w[e] = 0u;
     }
-  } else {
 #pragma unroll
-    for (int e = 0; e < 16; ++e) w[e] = 0u;
+    for (int g = 0; g < 4; ++g)
+      st_shared_v4(tile + kb * kBlk + kmajor_off(row, half * 32 + 8 * g, 0), w[4 * g],
+                   w[4 * g + 1], w[4 * g + 2], w[4 * g + 3]);
   }
-#pragma unroll
-  for (int g = 0; g < 4; ++g)
-    st_shared_v4(tile + kmajor_off(row, c0 + 8 * g, 0), w[4 * g], w[4 * g + 1], w[4 * g + 2],
-                 w[4 * g + 3]);
 }
 
-__global__ void __launch_bounds__(kThreads, 2)
+template <int D_>
+__global__ void __launch_bounds__(kThreads, D_ == 64 ? 2 : 1)
     exact_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_q,
                     const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                     const Params p) {
+  using G = ExCfg<D_>;
+  constexpr int DS = G::DS;
+  constexpr uint32_t oW = G::oW, oQ = G::oQ, oK = G::oK, oV = G::oV, oOnes = G::oOnes, oP = G::oP;
+  constexpr uint32_t tS = G::tS, tX = G::tX;
+  constexpr uint32_t kTile = DS * kBlk;         // one 128-token tile of d columns (bf16)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   const uint32_t s0 = smem_u32(sm);
-  uint64_t* bar_k = (uint64_t*)(sm + oBar);     // Q, W' (first), then each K tile
+  uint64_t* bar_k = (uint64_t*)(sm + G::oBar);  // Q, W' (first), then each K tile
   uint64_t* bar_v = bar_k + 1;                  // each V tile
   uint64_t* bar_mma = bar_k + 2;
   uint32_t* tmem_slot = (uint32_t*)(bar_k + 3);
   uint64_t* bar_drain = bar_k + 4;              // abort path: the issued MMAs completed
   uint64_t* bar_never = bar_k + 5;              // completed by nothing (testing stall)
-  float* smax = (float*)(sm + oMax);
-  uint8_t* kval = sm + oKv;
+  float* smax = (float*)(sm + G::oMax);
+  uint8_t* kval = sm + G::oKv;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int quad = warp & 3, half = warp >> 2;
@@ -119,8 +137,8 @@ __global__ void __launch_bounds__(kThreads, 2)
     prefetch_tmap(&tm_v);
   }
   __syncwarp();
-  if (warp == 0) tmem_alloc(tmem_slot, kTmemCols);
-  for (int i = tid; i < kTile / 16; i += kThreads)
+  if (warp == 0) tmem_alloc(tmem_slot, G::kTmemCols);
+  for (int i = tid; i < kBlk / 16; i += kThreads)
     st_shared_v4(s0 + oOnes + i * 16, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u);
   fence_async_smem();
   tc_fence_before();
@@ -138,20 +156,25 @@ __global__ void __launch_bounds__(kThreads, 2)
   const int qi = q0 + row;
   const int nk = p.causal ? qt + 1 : (p.Lk + kT - 1) / kT;
   const int r = p.r;
+  const int rb = (r + 63) / 64;                 // 64-column blocks of the projections
 
   uint32_t ph_k = 0, ph_v = 0, ph_mma = 0;
   bool abort = false;
   int k_issued = 1, k_waited = 0, v_issued = 0, v_waited = 0;   // load phases started / waited
-  float o[32], l = 0.f, mrow = -INFINITY;
+  constexpr int kHalfD = D_ / 2;                // output columns per thread
+  float o[kHalfD], l = 0.f, mrow = -INFINITY;
 #pragma unroll
-  for (int i = 0; i < 32; ++i) o[i] = 0.f;
+  for (int i = 0; i < kHalfD; ++i) o[i] = 0.f;
 
   // ---- Q and W'_bot, then K_0 and V_0
   if (tid == 0) {
-    mbar_arrive_expect_tx(bar_k, (uint32_t)r * 128 + kTile);
-    for (int r0 = 0; r0 < r; r0 += 16)
-      tma_load_2d(sm + oW + r0 * 128, &tm_w, 0, hw * (p.m + r) + p.m + r0, bar_k);
-    tma_load_4d(sm + oQ, &tm_q, 0, q0, h, b, bar_k);
+    mbar_arrive_expect_tx(bar_k, (uint32_t)r * 128 * DS + kTile);
+    for (int sl = 0; sl < DS; ++sl) {
+      for (int r0 = 0; r0 < r; r0 += 16)
+        tma_load_2d(sm + oW + sl * G::kWslab + r0 * 128, &tm_w, 64 * sl,
+                    hw * (p.m + r) + p.m + r0, bar_k);
+      tma_load_4d(sm + oQ + sl * kBlk, &tm_q, 64 * sl, q0, h, b, bar_k);
+    }
   }
   if (p.stall > 0 && !wait_all(bar_never, 0, p.dev_status, p.stall)) abort = true;
   if (!abort && !wait_all(bar_k, ph_k, p.dev_status)) abort = true;
@@ -162,9 +185,11 @@ __global__ void __launch_bounds__(kThreads, 2)
     ++v_issued;
     if (tid == 0) {
       mbar_arrive_expect_tx(bar_k, kTile);
-      tma_load_4d(sm + oK, &tm_k, 0, 0, h, b, bar_k);
+      for (int sl = 0; sl < DS; ++sl)
+        tma_load_4d(sm + oK + sl * kBlk, &tm_k, 64 * sl, 0, h, b, bar_k);
       mbar_arrive_expect_tx(bar_v, kTile);
-      tma_load_4d(sm + oV, &tm_v, 0, 0, h, b, bar_v);
+      for (int sl = 0; sl < DS; ++sl)
+        tma_load_4d(sm + oV + sl * kBlk, &tm_v, 64 * sl, 0, h, b, bar_v);
     }
     to_fp16_inplace(s0 + oQ, kTile, p.dev_status);
     fence_async_smem();
@@ -173,16 +198,16 @@ __global__ void __launch_bounds__(kThreads, 2)
       tc_fence_after();
       const uint32_t idp = idesc(128, r, false, false, true);
 #pragma unroll
-      for (int s = 0; s < kD / 16; ++s)
-        mma(tmem + tX, sdesc(s0 + oQ + s * 32, 16, 1024), sdesc(s0 + oW + s * 32, 16, 1024), idp,
-            s > 0);
+      for (int s = 0; s < D_ / 16; ++s)
+        mma(tmem + tX, sdesc(s0 + oQ + (s / 4) * kBlk + (s % 4) * 32, 16, 1024),
+            sdesc(s0 + oW + (s / 4) * G::kWslab + (s % 4) * 32, 16, 1024), idp, s > 0);
       mma_commit(bar_mma);
     }
     if (!wait_all(bar_mma, ph_mma, p.dev_status)) abort = true;
     ph_mma ^= 1;
     tc_fence_after();
     // the projection MMA has read the Q tile: 2 p_q over it
-    if (!abort) proj_to_smem(lane_tm + tX, r, 2.f, s0 + oQ, row, half);
+    if (!abort) proj_to_smem(lane_tm + tX, r, rb, 2.f, s0 + oQ, row, half);
     fence_async_smem();
     tc_fence_before();
     __syncthreads();
@@ -201,15 +226,15 @@ __global__ void __launch_bounds__(kThreads, 2)
       tc_fence_after();
       const uint32_t idp = idesc(128, r, false, false, true);
 #pragma unroll
-      for (int s = 0; s < kD / 16; ++s)
-        mma(tmem + tX, sdesc(s0 + oK + s * 32, 16, 1024), sdesc(s0 + oW + s * 32, 16, 1024), idp,
-            s > 0);
+      for (int s = 0; s < D_ / 16; ++s)
+        mma(tmem + tX, sdesc(s0 + oK + (s / 4) * kBlk + (s % 4) * 32, 16, 1024),
+            sdesc(s0 + oW + (s / 4) * G::kWslab + (s % 4) * 32, 16, 1024), idp, s > 0);
       mma_commit(bar_mma);
     }
     if (!wait_all(bar_mma, ph_mma, p.dev_status)) { abort = true; break; }
     ph_mma ^= 1;
     tc_fence_after();
-    proj_to_smem(lane_tm + tX, r, 1.f, s0 + oK, row, half);
+    proj_to_smem(lane_tm + tX, r, rb, 1.f, s0 + oK, row, half);
     fence_async_smem();
     tc_fence_before();
     __syncthreads();
@@ -217,10 +242,9 @@ __global__ void __launch_bounds__(kThreads, 2)
     if (tid == 0) {
       tc_fence_after();
       constexpr uint32_t ids = idesc(128, 128, false, false, true);
-#pragma unroll
-      for (int s = 0; s < kD / 16; ++s)
-        mma(tmem + tS, sdesc(s0 + oQ + s * 32, 16, 1024), sdesc(s0 + oK + s * 32, 16, 1024), ids,
-            s > 0);
+      for (int s = 0; s < rb * 4; ++s)
+        mma(tmem + tS, sdesc(s0 + oQ + (s / 4) * kBlk + (s % 4) * 32, 16, 1024),
+            sdesc(s0 + oK + (s / 4) * kBlk + (s % 4) * 32, 16, 1024), ids, s > 0);
       mma_commit(bar_mma);
     }
     // key validity of this tile, read from global memory once (the wait below
@@ -236,7 +260,8 @@ __global__ void __launch_bounds__(kThreads, 2)
     if (j + 1 < nk) ++k_issued;
     if (tid == 0 && j + 1 < nk) {
       mbar_arrive_expect_tx(bar_k, kTile);
-      tma_load_4d(sm + oK, &tm_k, 0, k0 + kT, h, b, bar_k);
+      for (int sl = 0; sl < DS; ++sl)
+        tma_load_4d(sm + oK + sl * kBlk, &tm_k, 64 * sl, k0 + kT, h, b, bar_k);
     }
     // ---- masks, row maximum, P = 2^(S - max) (this half: keys half*64 .. +63);
     // the scores are read from TMEM twice (maximum, then exponentials) rather
@@ -284,11 +309,11 @@ __global__ void __launch_bounds__(kThreads, 2)
     ++v_waited;
     if (tid == 0) {
       tc_fence_after();
-      constexpr uint32_t idv = idesc(128, 80, false, true, false);
+      constexpr uint32_t idv = idesc(128, D_ + 16, false, true, false);
 #pragma unroll
       for (int s = 0; s < kT / 16; ++s)
         mma(tmem + tX, sdesc(s0 + oP + (s / 4) * 16384 + (s % 4) * 32, 16, 1024),
-            sdesc(s0 + oV + s * 2048, oOnes - oV, 1024), idv, s > 0);
+            sdesc(s0 + oV + s * 2048, kBlk, 1024), idv, s > 0);
       mma_commit(bar_mma);
     }
     if (!wait_all(bar_mma, ph_mma, p.dev_status)) { abort = true; break; }
@@ -298,14 +323,18 @@ __global__ void __launch_bounds__(kThreads, 2)
     if (j + 1 < nk) ++v_issued;
     if (tid == 0 && j + 1 < nk) {
       mbar_arrive_expect_tx(bar_v, kTile);
-      tma_load_4d(sm + oV, &tm_v, 0, k0 + kT, h, b, bar_v);
+      for (int sl = 0; sl < DS; ++sl)
+        tma_load_4d(sm + oV + sl * kBlk, &tm_v, 64 * sl, k0 + kT, h, b, bar_v);
     }
     {
-      float v[32];
-      tmem_ld32(lane_tm + tX + half * 32, v);
-      const float den = tmem_ld1(lane_tm + tX + 64);
 #pragma unroll
-      for (int i = 0; i < 32; ++i) o[i] = fmaf(o[i], scale, v[i]);
+      for (int c = 0; c < kHalfD; c += 32) {
+        float v[32];
+        tmem_ld32(lane_tm + tX + half * kHalfD + c, v);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) o[c + i] = fmaf(o[c + i], scale, v[i]);
+      }
+      const float den = tmem_ld1(lane_tm + tX + D_);
       l = fmaf(l, scale, den);
     }
     tc_fence_before();
@@ -320,33 +349,62 @@ __global__ void __launch_bounds__(kThreads, 2)
   if (!abort && qi < p.Lq) {
     const bool live = p.qmask == nullptr || p.qmask[(size_t)b * p.Lq + qi] != 0;
     const float inv = (live && l > 0.f) ? 1.f / l : 0.f;
-    uint32_t w[16];
+    uint4* dst = reinterpret_cast<uint4*>(p.out + (int64_t)b * p.ob + (int64_t)h * p.oh +
+                                          (int64_t)qi * p.ol + half * kHalfD);
     bool bad = false;
 #pragma unroll
-    for (int e = 0; e < 16; ++e) {
-      const float a = o[2 * e] * inv, c = o[2 * e + 1] * inv;
-      bad |= !isfinite(a) || !isfinite(c);
-      w[e] = pack_bf16(a, c);
+    for (int q4 = 0; q4 < kHalfD / 8; ++q4) {
+      uint32_t w[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float a = o[8 * q4 + 2 * e] * inv, c = o[8 * q4 + 2 * e + 1] * inv;
+        bad |= !isfinite(a) || !isfinite(c);
+        w[e] = pack_bf16(a, c);
+      }
+      dst[q4] = make_uint4(w[0], w[1], w[2], w[3]);
     }
     if (bad) report(p.dev_status, DARK_ERR_NUMERIC);
-    uint4* dst = reinterpret_cast<uint4*>(p.out + (int64_t)b * p.ob + (int64_t)h * p.oh +
-                                          (int64_t)qi * p.ol + half * 32);
-#pragma unroll
-    for (int q4 = 0; q4 < 4; ++q4)
-      dst[q4] = make_uint4(w[4 * q4], w[4 * q4 + 1], w[4 * q4 + 2], w[4 * q4 + 3]);
   }
   tc_fence_before();
   __syncthreads();
   if (warp == 0) {
     tc_fence_after();
-    tmem_dealloc(tmem, kTmemCols);
+    tmem_dealloc(tmem, G::kTmemCols);
   }
 }
 
 }  // namespace
 
+template <int D_>
+cudaError_t launch_exact(const FwdArgs& a, const Params& p) {
+  using G = ExCfg<D_>;
+  static int smem_set[64];
+  cudaError_t e = set_smem_limit_once((const void*)exact_tc_kernel<D_>, (int)G::kSmem, smem_set);
+  if (e != cudaSuccess) return e;
+  if (D_ == 64) {
+    // two CTAs per SM (2 x 106 KB of shared memory, 2 x 256 TMEM columns); set
+    // once per device, outside any later stream capture
+    static int carveout_set[64];
+    int dev = 0;
+    e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev >= 0 && dev < 64 && !carveout_set[dev]) {
+      e = cudaFuncSetAttribute((const void*)exact_tc_kernel<D_>,
+                               cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+      if (e != cudaSuccess) return e;
+      carveout_set[dev] = 1;
+    }
+  }
+  exact_tc_kernel<D_><<<a.B * a.H * p.nq, kThreads, G::kSmem, a.stream>>>(a.tm_w, a.tm_q, a.tm_k,
+                                                                         a.tm_v, p);
+  return cudaGetLastError();
+}
+
+// d = 64 (r <= 64, two CTAs per SM) and d = 128 (r <= 128, one CTA per SM):
+// the projections p_q, p_k overwrite the Q and K tiles, so r <= d
 bool tc_exact_supported(FwdArgs& a) {
-  if (a.dtype != DARK_BF16 || a.d != kD || a.r % 16 != 0 || a.r < 16 || a.r > 64) return false;
+  if (a.dtype != DARK_BF16 || !(a.d == 64 || a.d == 128)) return false;
+  if (a.r % 16 != 0 || a.r < 16 || a.r > a.d) return false;
   if (a.os[2] % 8 != 0) return false;          // 16-byte output stores
   return tc_make_maps(a);
 }
@@ -372,24 +430,7 @@ cudaError_t tc_exact_forward(const FwdArgs& a) {
   p.r = a.r;
   p.dev_status = a.dev_status;
   p.stall = test_stall_cycles();
-  static int smem_set[64];
-  cudaError_t e = set_smem_limit_once((const void*)exact_tc_kernel, (int)kSmem, smem_set);
-  if (e != cudaSuccess) return e;
-  // two CTAs per SM (2 x 106 KB of shared memory, 2 x 256 TMEM columns); set
-  // once per device, outside any later stream capture
-  static int carveout_set[64];
-  int dev = 0;
-  e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return e;
-  if (dev >= 0 && dev < 64 && !carveout_set[dev]) {
-    e = cudaFuncSetAttribute((const void*)exact_tc_kernel,
-                             cudaFuncAttributePreferredSharedMemoryCarveout, 100);
-    if (e != cudaSuccess) return e;
-    carveout_set[dev] = 1;
-  }
-  exact_tc_kernel<<<a.B * a.H * p.nq, kThreads, kSmem, a.stream>>>(a.tm_w, a.tm_q, a.tm_k, a.tm_v,
-                                                                   p);
-  return cudaGetLastError();
+  return a.d == 64 ? launch_exact<64>(a, p) : launch_exact<128>(a, p);
 }
 
 }  // namespace dark

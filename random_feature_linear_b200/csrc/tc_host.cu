@@ -37,7 +37,8 @@ bool encode_tmap(CUtensorMap* map, CUtensorMapDataType type, int rank, const voi
 bool tc_make_maps(FwdArgs& a) {
   if (a.maps_ready) return true;
   auto al16 = [](const void* p) { return ((uintptr_t)p & 15) == 0; };
-  if (a.dtype != DARK_BF16 || a.d != 64) return false;
+  // 64-column boxes: d = 64 is one box per row, d = 128 two
+  if (a.dtype != DARK_BF16 || !(a.d == 64 || a.d == 128)) return false;
   if (!al16(a.q) || !al16(a.k) || !al16(a.v) || !al16(a.out) || !al16(a.w)) return false;
   for (int i = 0; i < 3; ++i)
     if (a.qs[i] % 8 != 0 || a.ks[i] % 8 != 0 || a.os[i] % 8 != 0) return false;

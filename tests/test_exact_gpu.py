@@ -25,6 +25,11 @@ CASES = {
     "f32-noncausal-masked": synth.WORKLOADS[1].with_sizes(B=2, H=2, L=150, lengths=(150, 97)),
     "f32-causal": synth.WORKLOADS[1].with_sizes(B=1, H=2, L=130, causal=True),
     "bf16-causal-d128": synth.WORKLOADS[4].with_sizes(B=1, H=2, L=130, d=128, r=128, m=256),
+    # d = 128 on the tensor cores: r = 64 (one projection block), key masks
+    # and a ragged last tile over three 128-token tiles
+    "bf16-noncausal-d128-r64": synth.WORKLOADS[3].with_sizes(H=2, L=300, d=128, r=64, m=128),
+    "bf16-causal-d128-masked": synth.WORKLOADS[2].with_sizes(H=2, L=300, lengths=(300, 211),
+                                                             d=128, r=96, m=256),
     "f32-causal-d256": synth.WORKLOADS[4].with_sizes(B=1, H=1, L=70, d=256, r=64, m=128,
                                                       dtype="f32"),
     "bf16-single-token": synth.WORKLOADS[2].with_sizes(H=1, L=1, lengths=(1, 1)),
@@ -50,7 +55,8 @@ def test_exact_matches_oracle(D, cuda_ok, name):
     check(w, res["out"], _ref(inp, w.causal))
 
 
-@pytest.mark.parametrize("name", ["bf16-causal-c2", "f32-noncausal-masked"])
+@pytest.mark.parametrize("name", ["bf16-causal-c2", "f32-noncausal-masked",
+                                  "bf16-causal-d128-masked"])
 def test_exact_strided(D, cuda_ok, name):
     w = CASES[name]
     inp = synth.make_inputs(w)

@@ -42,9 +42,12 @@ if case.startswith("bwd"):
     mask = torch.from_numpy(inp["mask"]).to(dev)
     fn = lambda: D.dark_attention_bwd(omega, geom, q, k, v, g, *grads, w.B, w.H, w.L, D.DARK_BF16,
                                       key_mask=mask, flags=flags, dgeom=dgeom, ws=ws)
-elif case.startswith("fwd"):
+elif case.startswith("fwd") or case.startswith("exact"):
     w = {"fwd-stab-causal": synth.WORKLOADS[2].with_sizes(H=2, L=300, lengths=(300, 217)),
-         "fwd-stab-noncausal": synth.WORKLOADS[3].with_sizes(H=2, L=300)}[case]
+         "fwd-stab-noncausal": synth.WORKLOADS[3].with_sizes(H=2, L=300),
+         "exact-d64": synth.WORKLOADS[2].with_sizes(H=2, L=300, lengths=(300, 217)),
+         "exact-d128": synth.WORKLOADS[2].with_sizes(H=2, L=300, lengths=(300, 217), d=128,
+                                                     r=128)}[case]
     inp = synth.make_inputs(w)
     omega = torch.from_numpy(inp["omega"]).to(dev)
     geom = torch.from_numpy(inp["geom"]).to(dev)
@@ -52,7 +55,8 @@ elif case.startswith("fwd"):
     q, k, v = (torch.from_numpy(inp[n]).to(dev).to(torch.bfloat16) for n in ("q", "k", "v"))
     out = torch.empty_like(q)
     mask = None if inp["mask"] is None else torch.from_numpy(inp["mask"]).to(dev)
-    flags = (D.DARK_CAUSAL if w.causal else 0) | D.DARK_STABILISE
+    flags = (D.DARK_CAUSAL if w.causal else 0) | (
+        D.DARK_EXACT if case.startswith("exact") else D.DARK_STABILISE)
     ws = D.alloc_workspace(proj, w.B, w.H, w.L, flags, dev)
     fn = lambda: D.dark_attention_fwd(proj, q, k, v, out, w.B, w.H, w.L, key_mask=mask,
                                       flags=flags, ws=ws)
@@ -85,3 +89,10 @@ def test_stabilised_forward_runs_on_tensor_cores(cuda_ok, case, kernel):
     assert any(kernel in n for n in names), names
     assert any("keys_kernel" in n for n in names), names
     assert not any(("out_kernel" in n or "scan_kernel" in n) for n in names), names
+
+
+@pytest.mark.parametrize("case", ["exact-d64", "exact-d128"])
+def test_bf16_exact_runs_on_tensor_cores(cuda_ok, case):
+    names = launched(case)
+    assert any("exact_tc_kernel" in n for n in names), names
+    assert not any("exact_attn_kernel" in n for n in names), names
