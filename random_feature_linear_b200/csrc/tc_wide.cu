@@ -14,20 +14,30 @@
 // more than one SM's shared memory or TMEM, so it cannot ride along with one
 // CTA as in the d = 64 kernel. The work is split in two launches:
 //
-//  1. features_kernel, one CTA per (head, chunk): the feature GEMMs K_c W'^T
-//     and Q_c W^T (fp16 operands, fp32 in TMEM) share every streamed W' slab;
-//     the epilogue warps turn them into Phi(K_c), Psi(Q_c) (bf16) in 64-feature
-//     blocks while the next block's GEMM runs, the scores Psi Phi^T accumulate
-//     on the tensor cores block by block, and Phi, Psi and the masked causal
-//     scores A_c are bulk-copied to the workspace as ready shared-memory operand
-//     images (128B-swizzled, so the second launch copies them back verbatim).
-//  2. values_kernel, one CTA per (head, 64 value columns): walks the chunks in
-//     order with its slice of the state, m x (64 + 1) fp32, resident in TMEM
-//     (m/128 tiles of 128 features x 80 columns). Per chunk and feature tile f
-//     the epilogue warps copy S_f to shared memory as hi + lo bf16 operands
-//     (bf16 alone moves outputs by ~1e-2), then the tensor cores run
-//       num += Psi_f [S_f | z_f]  (hi and lo)   and   S_f += Phi_f^T [V_c | 1]
-//     after num = A_c [V_c | 1]; the epilogue divides and stores out_c.
+//  1. features_kernel, persistent (one CTA per SM walking a contiguous range of
+//     (head, chunk) items): per item the key norms, then per 128-feature block
+//     one N = 256 MMA chain over the chunk's keys and queries together (the W'
+//     block is the M = 128 operand); the epilogue warps turn the block into
+//     Phi(K_c), Psi(Q_c) (bf16), the scores Psi Phi^T accumulate on the tensor
+//     cores block by block, and Phi, Psi, the masked causal scores A_c, the
+//     chunk's key-feature sums and the row sums of A_c go to the workspace as
+//     ready shared-memory operand images (128B-swizzled, so the second launch
+//     copies them back verbatim).
+//  2. values_kernel, one CTA per (head, 128 value columns, feature half), the
+//     two feature halves of a (head, value block) forming a 2-CTA cluster: each
+//     CTA walks the chunks in order with its 256 x 128 block of the state in
+//     TMEM; per chunk the epilogue warps copy S to shared memory as hi + lo
+//     bf16 operands (bf16 alone moves outputs by ~1e-2), the tensor cores run
+//       num = A_c [V_c] + Psi [S hi | S lo]   and   S += Phi^T V_c,
+//     the denominators come from the key sums on the CUDA cores, and the two
+//     halves exchange their partial outputs through distributed shared memory.
+//
+// The stabiliser (DARK_STABILISE) adds a statistics pass of the features
+// kernel before the features: the same GEMMs with an epilogue that only takes
+// maxima, the largest valid key exponent of every (b, h) and the largest
+// exponent of every query. The features pass subtracts them before exp2, so
+// every image, key sum and score is relative to those constants and the values
+// launch runs unchanged; the key constant is the state's shift.
 //
 // In both kernels warp 9 is the producer (TMA / bulk copies), warp 8 issues
 // the MMAs and warps 0-7 are the epilogue (TMEM lane quadrant = warp % 4). Every
@@ -164,11 +174,33 @@ struct FeatParams {
   const uint8_t* mask;
   uint8_t* img;            // chunk records [B*H][nc]
   int B, H, L, nc, heads_w, nitems;
+  // stabiliser: per-(b,h) key maximum as an order-preserving integer (zero
+  // before the statistics pass), per-query maxima [B*H][nc*128], the state's
+  // key constant (state output, or null)
+  unsigned* kmax;
+  float* qc;
+  float* st_shift;
   int* dev_status;
   long long stall;         // testing stall before the first wait (0: none)
 };
 
-template <int D_, int M_, int R_>
+// The three forms of the features launch: plain; the statistics pass of the
+// stabiliser (feature exponents only: per-(b,h) maximum of the valid key
+// exponents, per-query maximum of the query exponents; no images); and the
+// stabilised pass, which subtracts those maxima before exp2.
+constexpr int kPlain = 0, kStats = 1, kStab = 2;
+
+// float <-> unsigned with the order of the floats (for integer max reductions);
+// 0 lies below every float, -inf included
+__device__ __forceinline__ unsigned f2ord(float f) {
+  const unsigned u = __float_as_uint(f);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+__device__ __forceinline__ float ord2f(unsigned o) {
+  return __uint_as_float((o & 0x80000000u) ? (o & 0x7fffffffu) : ~o);
+}
+
+template <int D_, int M_, int R_, int MODE>
 __global__ void __launch_bounds__(kThreadsF, 1)
     features_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_q,
                     const __grid_constant__ CUtensorMap tm_k, const FeatParams p) {
@@ -195,6 +227,10 @@ __global__ void __launch_bounds__(kThreadsF, 1)
   volatile int* abort_flag = (volatile int*)(bars + 33);
   float* nrm_s = (float*)(sm + G::oBar + 1024);          // [128] key offsets
   float* nrm_x = (float*)(sm + G::oBar + 1536);          // [128] second half sums
+  // stabiliser: the chunk's query maxima (statistics pass: order-preserving
+  // integers; stabilised pass: floats)
+  unsigned* qmax_s = (unsigned*)(sm + G::oBar + 512);
+  float* qc_s = (float*)(sm + G::oBar + 512);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   // this CTA's contiguous range of (head, chunk) items
@@ -223,6 +259,7 @@ __global__ void __launch_bounds__(kThreadsF, 1)
     fence_mbar_init();
   }
   if (warp == 0) tmem_alloc(tmem_slot, kTmemCols);
+  if (MODE == kStats && tid < kC) qmax_s[tid] = 0u;
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -340,7 +377,7 @@ __global__ void __launch_bounds__(kThreadsF, 1)
           mma_commit(bar_ffull);
           if (f == G::NB - 1) mma_commit(bar_xfree);
           // scores of the previous block, staged meanwhile by the epilogue
-          if (f > 0) {
+          if (MODE != kStats && f > 0) {
             if (f == 1 && !(ok = wait_one(bar_nread, j & 1, abort_flag, p.dev_status))) break;
             if (!(ok = wait_one(bar_stage, (nblk - 1) & 1, abort_flag, p.dev_status))) break;
             tc_fence_after();
@@ -348,6 +385,7 @@ __global__ void __launch_bounds__(kThreadsF, 1)
           }
         }
         if (!ok) break;
+        if (MODE == kStats) continue;
         if (G::NB == 1 && !(ok = wait_one(bar_nread, j & 1, abort_flag, p.dev_status))) break;
         if (!(ok = wait_one(bar_stage, (nblk - 1) & 1, abort_flag, p.dev_status))) break;
         tc_fence_after();
@@ -368,6 +406,7 @@ __global__ void __launch_bounds__(kThreadsF, 1)
     const uint32_t lane_tm = tmem + ((uint32_t)(quad * 32) << 16);
     bool ok = true;
     int nblk = 0;
+    float kmax_t = -INFINITY;   // statistics pass: this thread's key maximum
     if (nit > 0 && p.stall > 0) ok = epi_wait(bar_never, 0, abort_flag, p.dev_status, p.stall);
     for (int j = 0; ok && j < nit; ++j) {
       const int item = it0 + j, bh = item / p.nc, c = item % p.nc;
@@ -396,8 +435,17 @@ __global__ void __launch_bounds__(kThreadsF, 1)
       fence_async_smem();
       tc_fence_before();
       warp_arrive(bar_conv);
-      // ---- key offsets: sum of squares of the norm columns + 1/2 log2 m;
-      // +inf for a masked or missing key
+      // ---- key offsets: sum of squares of the norm columns + 1/2 log2 m
+      // (+ the head's key maximum when stabilised); +inf for a masked or
+      // missing key
+      float kconst = 0.f;
+      if (MODE == kStab) {
+        // the statistics pass's maxima: 0 for a head without a valid key
+        const float km = ord2f(p.kmax[bh]);
+        kconst = km > -INFINITY ? km : 0.f;
+        if (etid < kC) qc_s[etid] = p.qc[(size_t)item * kC + etid];
+        if (p.st_shift != nullptr && c == 0 && etid == 0) p.st_shift[bh] = kconst;
+      }
       if (!(ok = epi_wait(bar_norm, j & 1, abort_flag, p.dev_status))) break;
       tc_fence_after();
       {
@@ -415,7 +463,8 @@ __global__ void __launch_bounds__(kThreadsF, 1)
           const int tok = c * kC + row;
           bool valid = tok < p.L;
           if (valid && p.mask != nullptr) valid = p.mask[(size_t)b * p.L + tok] != 0;
-          nrm_s[row] = valid ? part + nrm_x[row] + 0.5f * __log2f((float)M_) : __int_as_float(0x7f800000);
+          nrm_s[row] = valid ? part + nrm_x[row] + 0.5f * __log2f((float)M_) + kconst
+                             : __int_as_float(0x7f800000);
         }
         tc_fence_before();
         epi_sync();
@@ -432,6 +481,32 @@ __global__ void __launch_bounds__(kThreadsF, 1)
         for (int q = 0; q < 4; ++q) tmem_wait_ld(v[q]);
         tc_fence_before();
         warp_arrive(bar_ffree);
+        if (MODE == kStats) {
+          if (half == 0) {
+            // keys: the largest exponent over this thread's feature and the
+            // chunk's valid keys (a masked key's offset is +inf)
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+#pragma unroll
+              for (int e = 0; e < 32; ++e)
+                kmax_t = fmaxf(kmax_t, __uint_as_float(v[q][e]) - nrm_s[32 * q + e]);
+          } else {
+            // queries: the maximum over the block's 128 features (TMEM lanes)
+            // of every query (column): a warp reduction per column, then
+            // across the four warps of the half in shared memory
+            unsigned mine[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+#pragma unroll
+              for (int e = 0; e < 32; ++e) {
+                const unsigned r = __reduce_max_sync(0xffffffffu, f2ord(__uint_as_float(v[q][e])));
+                if (lane == e) mine[q] = r;
+              }
+#pragma unroll
+            for (int q = 0; q < 4; ++q) atomicMax(&qmax_s[32 * q + lane], mine[q]);
+          }
+          continue;
+        }
         // exp2 and bf16 packing (keys: minus the key offset; their sum over the
         // chunk, of the rounded values, is the chunk's increment of z)
         uint32_t pk[64];
@@ -445,6 +520,9 @@ __global__ void __launch_bounds__(kThreadsF, 1)
             if (half == 0) {
               x0 -= nrm_s[t];
               x1 -= nrm_s[t + 1];
+            } else if (MODE == kStab) {
+              x0 -= qc_s[t];
+              x1 -= qc_s[t + 1];
             }
             const __nv_bfloat162 pv = __floats2bfloat162_rn(ex2(x0), ex2(x1));
             pk[16 * q + e] = *reinterpret_cast<const uint32_t*>(&pv);
@@ -482,6 +560,21 @@ __global__ void __launch_bounds__(kThreadsF, 1)
         warp_arrive(bar_stage);
       }
       if (!ok) break;
+      if (MODE == kStats) {
+        // the chunk's maxima: keys into the head's running maximum, queries
+        // (their own, one per query) to the workspace
+        if (half == 0) {
+          const unsigned km = __reduce_max_sync(0xffffffffu, f2ord(kmax_t));
+          if (lane == 0) atomicMax(p.kmax + bh, km);
+        }
+        kmax_t = -INFINITY;
+        epi_sync();
+        if (etid < kC) {
+          p.qc[(size_t)item * kC + etid] = ord2f(qmax_s[etid]);
+          qmax_s[etid] = 0u;
+        }
+        continue;
+      }
       // ---- masked causal scores -> A image (query rows, keys as K)
       if (!(ok = epi_wait(bar_sc, j & 1, abort_flag, p.dev_status))) break;
       if (etid == 0) bulk_wait_read_all();
@@ -1205,13 +1298,36 @@ bool shape_ok(int d, int m, int r) {
          (d == 128 && m == 128 && r == 64);
 }
 
+// Workspace after the chunk records: the stabiliser's per-(b,h) key maxima
+// (order-preserving integers) and per-query maxima.
+size_t stab_kmax_off(int B, int H, int nc, int m) {
+  return align_up(kWsHeader + (size_t)B * H * nc * chunk_record_bytes(m), 256);
+}
+size_t stab_qc_off(int B, int H, int nc, int m) {
+  return align_up(stab_kmax_off(B, H, nc, m) + (size_t)B * H * 4, 256);
+}
+
+template <int D_, int M_, int R_, int MODE>
+cudaError_t launch_features(const FwdArgs& a, const FeatParams& fp) {
+  using F = FeatCfg<D_, M_, R_>;
+  static int smem_f[64];
+  cudaError_t e =
+      set_smem_limit_once((const void*)features_kernel<D_, M_, R_, MODE>, (int)F::kSmem, smem_f);
+  if (e != cudaSuccess) return e;
+  const int grid_f = fp.nitems < num_sms() ? fp.nitems : num_sms();
+  features_kernel<D_, M_, R_, MODE><<<grid_f, kThreadsF, F::kSmem, a.stream>>>(a.tm_w, a.tm_q,
+                                                                               a.tm_k, fp);
+  return cudaGetLastError();
+}
+
 template <int D_, int M_, int R_>
 cudaError_t launch(const FwdArgs& a) {
-  using F = FeatCfg<D_, M_, R_>;
   using V = ValCfg<D_, M_>;
   const int nc = (a.L + kC - 1) / kC;
   uint8_t* img = (uint8_t*)a.ws + kWsHeader;
+  const bool stab = (a.flags & DARK_STABILISE) != 0;
   FeatParams fp;
+  memset(&fp, 0, sizeof(fp));
   fp.mask = a.mask;
   fp.img = img;
   fp.B = a.B;
@@ -1221,15 +1337,23 @@ cudaError_t launch(const FwdArgs& a) {
   fp.heads_w = a.heads_w;
   fp.dev_status = a.dev_status;
   fp.stall = test_stall_cycles();
-  static int smem_f[64], smem_v[64];
-  cudaError_t e = set_smem_limit_once((const void*)features_kernel<D_, M_, R_>, (int)F::kSmem, smem_f);
-  if (e != cudaSuccess) return e;
-  e = set_smem_limit_once((const void*)values_kernel<D_, M_>, (int)V::kSmem, smem_v);
+  static int smem_v[64];
+  cudaError_t e = set_smem_limit_once((const void*)values_kernel<D_, M_>, (int)V::kSmem, smem_v);
   if (e != cudaSuccess) return e;
   fp.nitems = a.B * a.H * nc;
-  const int grid_f = fp.nitems < num_sms() ? fp.nitems : num_sms();
-  features_kernel<D_, M_, R_><<<grid_f, kThreadsF, F::kSmem, a.stream>>>(a.tm_w, a.tm_q, a.tm_k, fp);
-  e = cudaGetLastError();
+  if (stab) {
+    // statistics pass, then the features with the maxima subtracted
+    fp.kmax = (unsigned*)((uint8_t*)a.ws + stab_kmax_off(a.B, a.H, nc, M_));
+    fp.qc = (float*)((uint8_t*)a.ws + stab_qc_off(a.B, a.H, nc, M_));
+    fp.st_shift = a.st_shift;
+    e = cudaMemsetAsync(fp.kmax, 0, (size_t)a.B * a.H * 4, a.stream);
+    if (e != cudaSuccess) return e;
+    e = launch_features<D_, M_, R_, kStats>(a, fp);
+    if (e != cudaSuccess) return e;
+    e = launch_features<D_, M_, R_, kStab>(a, fp);
+  } else {
+    e = launch_features<D_, M_, R_, kPlain>(a, fp);
+  }
   if (e != cudaSuccess) return e;
   ValParams vp;
   memset(&vp, 0, sizeof(vp));
@@ -1269,15 +1393,15 @@ cudaError_t launch(const FwdArgs& a) {
 }  // namespace
 
 bool tc_wide_supported(FwdArgs& a) {
-  if (a.dtype != DARK_BF16 || !(a.flags & DARK_CAUSAL) || (a.flags & DARK_STABILISE)) return false;
+  if (a.dtype != DARK_BF16 || !(a.flags & DARK_CAUSAL)) return false;
   if (!shape_ok(a.d, a.m, a.r)) return false;
   return make_wide_maps(a);
 }
 
 size_t tc_wide_workspace_bytes(int B, int H, int L, int m, int d, int r) {
   if (!shape_ok(d, m, r)) return 0;
-  const size_t nc = (size_t)(L + kC - 1) / kC;
-  return align_up(kWsHeader + (size_t)B * H * nc * chunk_record_bytes(m), 256);
+  const int nc = (L + kC - 1) / kC;
+  return align_up(stab_qc_off(B, H, nc, m) + (size_t)B * H * nc * kC * 4, 256);
 }
 
 cudaError_t tc_wide_forward(const FwdArgs& a) {

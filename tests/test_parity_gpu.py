@@ -1,6 +1,7 @@
 """Parity of the CUDA forward path (through the C ABI) with the fp64 oracle."""
 import numpy as np
 import pytest
+import torch
 
 from oracle import dark_oracle as O
 from random_feature_linear_b200 import synth
@@ -71,7 +72,8 @@ def test_strided_inputs(D, cuda_ok, recipe):
     check(w, res["out"], out)
 
 
-@pytest.mark.parametrize("name", ["c1-causal", "c2", "c3"])
+@pytest.mark.parametrize("name", ["c1-causal", "c2", "c3", "c4-masked", "wide-d128-m256",
+                                  "wide-d128-m128-shared"])
 def test_stabiliser_changes_nothing(D, cuda_ok, name):
     w = SMALL[name]
     inp = synth.make_inputs(w)
@@ -86,18 +88,42 @@ def test_stabiliser_changes_nothing(D, cuda_ok, name):
     assert np.abs(res["z"] - zs).max() <= 2e-2 * np.abs(zs).max()
 
 
-@pytest.mark.parametrize("recipe", ["f32-causal", "bf16-causal", "bf16-noncausal"])
+def _query_exponent_max(inp):
+    """Largest base-2 query exponent max_j log2(e) (omega_j . M q~) over all
+    heads and tokens (the oracle's feature exponent without the key terms)."""
+    d = inp["q"].shape[-1]
+    top = 0.0
+    for h in range(inp["q"].shape[1]):
+        wtop = np.log2(np.e) * d ** -0.25 * (inp["omega"][0].astype(np.float64)
+                                             @ inp["geom"][h % inp["geom"].shape[0]]
+                                             .astype(np.float64))
+        qh = inp["q"][:, h].astype(np.float64).reshape(-1, d)
+        top = max(top, float((qh @ wtop.T).max()))
+    return top
+
+
+@pytest.mark.parametrize("recipe", ["f32-causal", "bf16-causal", "bf16-noncausal",
+                                    "bf16-wide-d256", "bf16-wide-d128"])
 def test_stabiliser_avoids_overflow(D, cuda_ok, recipe):
-    # Queries scaled by 6: their exponents reach ~2^138 and overflow fp32 unless
-    # the per-query constant is subtracted (key exponents are bounded by
-    # |omega_j|^2 / 2 and stay in range). Without the flag the device reports a
-    # non-finite output; with it the result matches the oracle. fp32 runs the
-    # FFMA kernels, bf16 (d = 64) the tensor-core kernels.
+    # Queries scaled so that their largest exponent is ~2^138 (by 6 for the
+    # d = 64 recipes): that overflows fp32 unless the per-query constant is
+    # subtracted (key exponents are bounded by |omega_j|^2 / 2 and stay in
+    # range). Without the flag the device reports a non-finite output; with it
+    # the result matches the oracle. fp32 runs the FFMA kernels, bf16 the
+    # tensor-core kernels (d = 64, and the wide-head pair for d = 128, 256).
     w = {"f32-causal": synth.WORKLOADS[1].with_sizes(L=130, causal=True),
          "bf16-causal": synth.WORKLOADS[2].with_sizes(H=2, L=260, lengths=(260, 199)),
-         "bf16-noncausal": synth.WORKLOADS[3].with_sizes(H=2, L=300)}[recipe]
+         "bf16-noncausal": synth.WORKLOADS[3].with_sizes(H=2, L=300),
+         "bf16-wide-d256": synth.WORKLOADS[4].with_sizes(B=1, H=2, L=300, lengths=(300,)),
+         "bf16-wide-d128": synth.WORKLOADS[4].with_sizes(B=2, H=2, L=270, d=128, r=128, m=256,
+                                                          lengths=(270, 150))}[recipe]
     inp = synth.make_inputs(w)
-    inp = dict(inp, q=inp["q"] * 6.0)
+    scale = 6.0 if w.d == 64 else 138.0 / _query_exponent_max(inp)
+    q = inp["q"] * scale
+    if w.dtype == "bf16":
+        # the device reads bf16 tokens: give the oracle the same rounded values
+        q = torch.from_numpy(q).to(torch.bfloat16).double().numpy()
+    inp = dict(inp, q=q)
     causal = D.DARK_CAUSAL if w.causal else 0
     res = forward(D, w, inp, cuda_ok, flags=causal)
     assert res["status"] == D.DARK_ERR_NUMERIC

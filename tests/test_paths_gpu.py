@@ -45,6 +45,7 @@ if case.startswith("bwd"):
 elif case.startswith("fwd") or case.startswith("exact"):
     w = {"fwd-stab-causal": synth.WORKLOADS[2].with_sizes(H=2, L=300, lengths=(300, 217)),
          "fwd-stab-noncausal": synth.WORKLOADS[3].with_sizes(H=2, L=300),
+         "fwd-stab-wide": synth.WORKLOADS[4].with_sizes(B=1, H=2, L=300, lengths=(300,)),
          "exact-d64": synth.WORKLOADS[2].with_sizes(H=2, L=300, lengths=(300, 217)),
          "exact-d128": synth.WORKLOADS[2].with_sizes(H=2, L=300, lengths=(300, 217), d=128,
                                                      r=128)}[case]
@@ -96,3 +97,13 @@ def test_bf16_exact_runs_on_tensor_cores(cuda_ok, case):
     names = launched(case)
     assert any("exact_tc_kernel" in n for n in names), names
     assert not any("exact_attn_kernel" in n for n in names), names
+
+
+def test_stabilised_wide_forward_runs_on_tensor_cores(cuda_ok):
+    # DARK_STABILISE at d = 256: the statistics pass and the stabilised pass of
+    # features_kernel, then values_kernel; none of the FFMA kernels
+    names = launched("fwd-stab-wide")
+    assert sum("features_kernel<256, 512, 256" in n for n in names) == 2, names
+    assert any("values_kernel" in n for n in names), names
+    assert not any(("out_kernel" in n or "scan_kernel" in n or "chunk_state_kernel" in n)
+                   for n in names), names
