@@ -17,6 +17,7 @@
 #pragma once
 
 #include "tc_common.cuh"
+#include "tc_roles.cuh"
 
 namespace dark {
 namespace tc {
@@ -36,11 +37,6 @@ __device__ __forceinline__ void mma_tf32(uint32_t tmem_d, uint64_t adesc, uint64
       "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
       "l"(adesc), "l"(bdesc), "r"(id), "r"(accumulate)
       : "memory");
-}
-
-// One arrival of this thread on a shared-memory mbarrier.
-__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
 constexpr uint32_t kKmRowBytes = 128;      // one K-major row of a chunk

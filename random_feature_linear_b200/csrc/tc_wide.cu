@@ -49,6 +49,7 @@
 #include "common.cuh"
 #include "internal.h"
 #include "tc_common.cuh"
+#include "tc_roles.cuh"
 
 namespace dark {
 namespace {
@@ -61,10 +62,7 @@ constexpr int kThreadsF = kEpiThreads + 64;   // + MMA warp 8 + producer warp 9
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kSmemBudget = 229376;   // 224 KB of operands + barriers + alignment slack
 
-// ------------------------------------------------------------ sync helpers --
-__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
-}
+// ----------------------------------------------------------- bulk copies --
 // shared -> global bulk copy (16-byte aligned, size a multiple of 16) with an
 // L2 eviction policy for the written lines
 __device__ __forceinline__ void bulk_store_hint(void* gdst, uint32_t ssrc, uint32_t bytes,
@@ -83,49 +81,6 @@ __device__ __forceinline__ void bulk_wait_read_all() {
 __device__ __forceinline__ void bulk_wait_all() {
   asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
 }
-// Barrier 1 over the 256 epilogue threads; true if any of them passes `bad`.
-__device__ __forceinline__ bool epi_sync_or(bool bad) {
-  uint32_t r;
-  asm volatile(
-      "{\n\t.reg .pred p, q;\n\t"
-      "setp.ne.u32 p, %1, 0;\n\t"
-      "barrier.cta.red.or.pred q, 1, 256, p;\n\t"
-      "selp.u32 %0, 1, 0, q;\n\t}"
-      : "=r"(r)
-      : "r"((uint32_t)bad)
-      : "memory");
-  return r != 0;
-}
-__device__ __forceinline__ void epi_sync() { asm volatile("barrier.cta.sync 1, 256;" ::: "memory"); }
-
-// Bounded wait of one thread. A wait that runs out records DARK_ERR_TIMEOUT and
-// raises the abort flag; a raised flag ends every other wait of the CTA.
-__device__ __forceinline__ bool wait_one(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
-                                         int* dev_status, long long limit = kWaitCycles) {
-  if (mbar_try_wait(bar, parity)) return true;
-  const long long t0 = clock64();
-  while (!mbar_try_wait(bar, parity)) {
-    if (*abort_flag) return false;
-    if (clock64() - t0 > limit) {
-      *abort_flag = 1;
-      report(dev_status, DARK_ERR_TIMEOUT);
-      return false;
-    }
-  }
-  return true;
-}
-// The same for the epilogue warps: all 256 wait, then agree.
-__device__ __forceinline__ bool epi_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
-                                         int* dev_status, long long limit = kWaitCycles) {
-  const bool ok = wait_one(bar, parity, abort_flag, dev_status, limit);
-  return !epi_sync_or(!ok);
-}
-// Epilogue warp -> producer/MMA thread: one arrival per warp (barrier count 8).
-__device__ __forceinline__ void warp_arrive(uint64_t* bar) {
-  __syncwarp();
-  if ((threadIdx.x & 31) == 0) mbar_arrive(bar);
-}
-
 // ================================================================ launch 1 ==
 // Persistent: each CTA walks a contiguous range of (head, chunk) items. Per
 // item the key and query tiles sit side by side in shared memory as one
