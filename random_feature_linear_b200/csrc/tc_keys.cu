@@ -63,23 +63,6 @@ struct KeyCfg {
 };
 
 
-// exp2 of 32 values (minus `offset`) packed to bf16 pairs (zeros for a masked key).
-__device__ __forceinline__ void exp2_pack32(const uint32_t (&r)[32], float offset, bool zero,
-                                            uint32_t (&w)[16]) {
-#pragma unroll
-  for (int e = 0; e < 16; ++e) {
-    const float x0 = __uint_as_float(r[2 * e]) - offset;
-    const float x1 = __uint_as_float(r[2 * e + 1]) - offset;
-    w[e] = zero ? 0u : pack_bf16(ex2(x0), ex2(x1));
-  }
-}
-// 32 packed bf16 pairs as four 16-byte chunks of a K-major 128B-swizzled row.
-__device__ __forceinline__ void store_row32(const uint32_t (&w)[16], uint32_t tile, int row, int f0) {
-#pragma unroll
-  for (int g = 0; g < 4; ++g)
-    st_shared_v4(tile + kmajor_off(row, f0 + 8 * g, 16384), w[4 * g], w[4 * g + 1], w[4 * g + 2],
-                 w[4 * g + 3]);
-}
 // The fp16 W' image at `hi` (as loaded) -> bf16 hi in place and bf16 lo at
 // `lo` (the same layout), by the 256 epilogue threads. An fp16 value has 11
 // significant bits: hi = bf16(x) keeps 8 of them and x - hi, exact in fp32,

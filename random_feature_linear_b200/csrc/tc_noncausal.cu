@@ -20,6 +20,7 @@
 #include "internal.h"
 #include "tc_common.cuh"
 #include "tc_keys.cuh"
+#include "tc_roles.cuh"
 
 namespace dark {
 namespace {
@@ -28,7 +29,7 @@ using namespace tc;
 
 constexpr int kD = 64;
 constexpr int kT = 128;                     // tokens per tile
-constexpr int kThreads = kFwdThreads;
+constexpr int kThreads = kFwdThreads + 128;   // query kernel: + MMA, producer, 2 converter warps
 constexpr int kSms = 148;
 constexpr int kTileBytes = kT * kD * 2;
 constexpr uint32_t kTmemCols = 512;
@@ -106,138 +107,249 @@ struct QueryCfg {
   static constexpr uint32_t oQ = oImg + (img_bytes(M_) + 1023) / 1024 * 1024;   // 2 buffers
   static constexpr uint32_t oPsi = oQ + 2 * kTileBytes;
   static constexpr uint32_t oBar = oPsi + kPsi;
-  static constexpr uint32_t oRed = oBar + 64;              // [2][128] fp32 row maxima
+  static constexpr uint32_t oRed = oBar + 256;             // [2][128] fp32 row maxima
   static constexpr uint32_t kSmem = oRed + 1024 + 1024;
   static constexpr uint32_t tP = 0, tO = 256;
   static_assert(kSmem <= 232448, "shared memory");
 };
 
+// bf16 -> fp16 in place for one Q tile by the 64 converter threads. A bf16
+// value is out of fp16 range (|x| > 65504) exactly when its magnitude bits are
+// 0x4780 (65536) or more.
+__device__ __forceinline__ void q_to_fp16(uint32_t saddr, int ctid, int* dev_status) {
+  uint32_t mag = 0;
+#pragma unroll 4
+  for (int i = ctid; i < kTileBytes / 16; i += 64) {
+    const uint32_t a = saddr + i * 16;
+    uint4 u = ld_shared_v4(a);
+    uint32_t* w32 = &u.x;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      mag = __vmaxu2(mag, w32[e] & 0x7FFF7FFFu);
+      const __half2 hv = __floats2half2_rn(__uint_as_float(w32[e] << 16),
+                                           __uint_as_float(w32[e] & 0xFFFF0000u));
+      w32[e] = *reinterpret_cast<const uint32_t*>(&hv);
+    }
+    st_shared_v4(a, u.x, u.y, u.z, u.w);
+  }
+  if ((mag & 0xFFFFu) >= 0x4780u || (mag >> 16) >= 0x4780u) report(dev_status, DARK_ERR_NUMERIC);
+}
+
+// Query kernel: each CTA walks a contiguous range of (head, query tile) items
+// with four roles. Warp 9 loads the head operands (W' feature rows and the
+// [S | z] image, once per head) and the Q tiles (two buffers); warps 10-11
+// convert each Q tile to fp16 as it lands; warp 8 issues the MMAs; warps 0-7
+// run the epilogue. The feature GEMM Q W^T comes in two parts (features [0, M/2) and
+// [M/2, M)), each released by the epilogue as soon as it has read it, so the
+// next tile's features are computed during this tile's exponentials; the
+// output GEMM of a tile is read back (and the tile's rows stored) while the
+// next tile is exponentiated.
 template <int M_, int R_>
 __global__ void __launch_bounds__(kThreads, 1)
     queries_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_q,
                    const QueryParams p) {
   using G = QueryCfg<M_, R_>;
+  constexpr int NH = M_ / 128;                // 32-column chunks per round
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   const uint32_t s0 = smem_u32(sm);
-  uint64_t* bar_q = (uint64_t*)(sm + G::oBar);      // [2]
-  uint64_t* bar_mma = bar_q + 2;
-  uint64_t* bar_head = bar_q + 3;
-  uint32_t* tmem_slot = (uint32_t*)(bar_q + 4);
-  uint64_t* bar_drain = bar_q + 5;      // abort path: the issued MMAs completed
-  uint64_t* bar_never = bar_q + 6;      // completed by nothing (testing stall)
+  uint64_t* bars = (uint64_t*)(sm + G::oBar);
+  uint64_t* q_full = bars + 0;       // [2] producer: Q tile loaded
+  uint64_t* q_conv = bars + 2;       // [2] converters: Q tile converted to fp16 (2)
+  uint64_t* q_empty = bars + 4;      // [2] MMA: the feature GEMM has read the Q tile
+  uint64_t* h_full = bars + 6;       // producer: a head's W' rows and image loaded
+  uint64_t* h_free = bars + 7;       // MMA: the last GEMMs of a head are done
+  uint64_t* bar_ffullA = bars + 8;   // MMA: features [0, M/2) in TMEM
+  uint64_t* bar_ffreeA = bars + 9;   // epilogue: read (8)
+  uint64_t* bar_ffullB = bars + 10;  // MMA: features [M/2, M) in TMEM
+  uint64_t* bar_ffreeB = bars + 11;  // epilogue: read (8)
+  uint64_t* bar_pfull = bars + 12;   // epilogue: Psi staged, the previous output read (8)
+  uint64_t* bar_ofull = bars + 13;   // MMA: output GEMM done (Psi free)
+  uint64_t* bar_drain = bars + 14;   // abort path: the issued MMAs completed
+  uint64_t* bar_never = bars + 15;   // completed by nothing (testing stall)
+  uint32_t* tmem_slot = (uint32_t*)(bars + 16);
+  volatile int* abort_flag = (volatile int*)(bars + 16) + 1;
+  float* red = (float*)(sm + G::oRed);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int quad = warp & 3, half = warp >> 2;
-  const int row = quad * 32 + lane;
   const int ub = (int)((long long)blockIdx.x * p.total_tiles / gridDim.x);
   const int ue = (int)((long long)(blockIdx.x + 1) * p.total_tiles / gridDim.x);
+  const int n = ue > ub ? ue - ub : 0;
+  // a new head starts at item i (its operands must be loaded first)
+  auto head_starts = [&](int i) { return i == 0 || (ub + i) % p.ntiles == 0; };
 
   if (tid == 0) {
-    mbar_init(&bar_q[0], 1);
-    mbar_init(&bar_q[1], 1);
-    mbar_init(bar_mma, 1);
-    mbar_init(bar_head, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(q_full + i, 1);
+      mbar_init(q_conv + i, 2);
+      mbar_init(q_empty + i, 1);
+    }
+    mbar_init(h_full, 1);
+    mbar_init(h_free, 1);
+    mbar_init(bar_ffullA, 1);
+    mbar_init(bar_ffreeA, 8);
+    mbar_init(bar_ffullB, 1);
+    mbar_init(bar_ffreeB, 8);
+    mbar_init(bar_pfull, 8);
+    mbar_init(bar_ofull, 1);
     mbar_init(bar_drain, 1);
     mbar_init(bar_never, 1);
+    *abort_flag = 0;
     fence_mbar_init();
-    if (ue > ub) {
-      const int bh = ub / p.ntiles, t = ub % p.ntiles;
-      mbar_arrive_expect_tx(&bar_q[0], kTileBytes);
-      tma_load_4d(sm + G::oQ, &tm_q, 0, t * kT, bh % p.H, bh / p.H, &bar_q[0]);
-    }
   }
-  __syncwarp();
   if (warp == 0) tmem_alloc(tmem_slot, kTmemCols);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t lane_tm = tmem + ((uint32_t)(quad * 32) << 16);
 
-  uint32_t ph_q = 0, ph_mma = 0, ph_head = 0;  // ph_q bit i: parity of buffer i
-  int cur_bh = -1;
-  bool abort = false;
-  // load phases started / waited for: query buffers, head operands
-  int q_issued[2] = {ue > ub ? 1 : 0, 0}, q_waited[2] = {0, 0}, h_issued = 0, h_waited = 0;
-  if (ue > ub && p.stall > 0 && !wait_all(bar_never, 0, p.dev_status, p.stall)) abort = true;
-  for (int u = ub; u < ue && !abort; ++u) {
-    const int i = u - ub, buf = i & 1;
-    const int bh = u / p.ntiles, t = u % p.ntiles, b = bh / p.H, h = bh % p.H;
-    if (bh != cur_bh) {
-      // W' rows and the [S | z] image of this head (all earlier MMAs have completed)
-      if (tid == 0) {
+  if (warp >= 10) {
+    // ---------------------------------------------------------- converters
+    const int ctid = tid - 320;
+    for (int i = 0; i < n; ++i) {
+      const int buf = i & 1;
+      bool w = true;
+      if (lane == 0) w = wait_one(q_full + buf, (i >> 1) & 1, abort_flag, p.dev_status);
+      if (__shfl_sync(0xffffffffu, w ? 1 : 0, 0) == 0) break;
+      mbar_wait(q_full + buf, (i >> 1) & 1);   // passes at once (the data's visibility)
+      q_to_fp16(s0 + G::oQ + buf * kTileBytes, ctid, p.dev_status);
+      fence_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(q_conv + buf);
+    }
+    __syncwarp();
+  } else if (warp == 9) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0 && n > 0) {
+      int nq[2] = {0, 0}, nh = 0;        // loads issued: per Q buffer, head operands
+      auto load_head = [&](int i) {
+        const int bh = (ub + i) / p.ntiles, h = bh % p.H;
         const int hw = p.heads_w == 1 ? 0 : h;
-        ++h_issued;
-        mbar_arrive_expect_tx(bar_head, G::kWq + img_bytes(M_));
+        mbar_arrive_expect_tx(h_full, G::kWq + img_bytes(M_));
         for (int r0 = 0; r0 < M_; r0 += 16)
-          tma_load_2d(sm + G::oW + r0 * 128, &tm_w, 0, hw * G::NW + r0, bar_head);
+          tma_load_2d(sm + G::oW + r0 * 128, &tm_w, 0, hw * G::NW + r0, h_full);
         const uint8_t* src = p.images + (size_t)bh * img_bytes(M_);
         for (uint32_t o = 0; o < img_bytes(M_); o += 16384)
-          bulk_load(sm + G::oImg + o, src + o, img_bytes(M_) - o < 16384 ? img_bytes(M_) - o : 16384,
-                    bar_head);
+          bulk_load(sm + G::oImg + o, src + o,
+                    img_bytes(M_) - o < 16384 ? img_bytes(M_) - o : 16384, h_full);
+        ++nh;
+      };
+      auto load_q = [&](int i) {
+        const int u = ub + i, bh = u / p.ntiles, t = u % p.ntiles, buf = i & 1;
+        mbar_arrive_expect_tx(q_full + buf, kTileBytes);
+        tma_load_4d(sm + G::oQ + buf * kTileBytes, &tm_q, 0, t * kT, bh % p.H, bh / p.H,
+                    q_full + buf);
+        ++nq[buf];
+      };
+      prefetch_tmap(&tm_w);
+      prefetch_tmap(&tm_q);
+      load_head(0);
+      load_q(0);
+      if (n > 1) load_q(1);
+      bool ok = true;
+      int heads_done = 0;                 // h_free phases passed
+      for (int i = 0; ok && i + 1 < n; ++i) {
+        // Q tile i + 2 into tile i's buffer once tile i's feature GEMM has read it
+        if (i + 2 < n) {
+          if (!(ok = wait_one(q_empty + (i & 1), (i >> 1) & 1, abort_flag, p.dev_status))) break;
+          load_q(i + 2);
+        }
+        // the next head's operands once this head's last GEMMs are done
+        if (head_starts(i + 1)) {
+          if (!(ok = wait_one(h_free, heads_done & 1, abort_flag, p.dev_status))) break;
+          ++heads_done;
+          load_head(i + 1);
+        }
       }
-      if (!wait_all(bar_head, ph_head, p.dev_status)) { abort = true; break; }
-      ph_head ^= 1;
-      ++h_waited;
-      cur_bh = bh;
+      if (!ok) {
+        // aborted: leave no copy in flight (a completed phase passes at once)
+        for (int i = 0; i < 2; ++i)
+          if (nq[i] > 0) mbar_wait(q_full + i, (uint32_t)(nq[i] - 1) & 1u);
+        if (nh > 0) mbar_wait(h_full, (uint32_t)(nh - 1) & 1u);
+      }
     }
-    if (!wait_all(&bar_q[buf], (ph_q >> buf) & 1u, p.dev_status)) { abort = true; break; }
-    ph_q ^= 1u << buf;
-    ++q_waited[buf];
-    to_fp16_inplace(s0 + G::oQ + buf * kTileBytes, kTileBytes, p.dev_status);
-    fence_async_smem();
-    __syncthreads();
-    if (tid == 0) {
-      tc_fence_after();
-      constexpr uint32_t idq = idesc(128, M_, false, false, true);
+    __syncwarp();
+  } else if (warp == 8) {
+    // ---------------------------------------------------------- MMA issuer
+    if (lane == 0 && n > 0) {
+      bool ok = true;
+      int heads_seen = 0;
+      // Q W^T, part A (features [0, M/2)) or B ([M/2, M)); fp16, fp32 in TMEM
+      auto features = [&](int i, int part) {
+        const uint32_t sq = s0 + G::oQ + (i & 1) * kTileBytes;
+        constexpr uint32_t idh = idesc(128, M_ / 2, false, false, true);
 #pragma unroll
-      for (int s = 0; s < kD / 16; ++s)
-        mma(tmem + G::tP, sdesc(s0 + G::oQ + buf * kTileBytes + s * 32, 16, 1024),
-            sdesc(s0 + G::oW + s * 32, 16, 1024), idq, s > 0);
-      mma_commit(bar_mma);
-    }
-    if (!wait_all(bar_mma, ph_mma, p.dev_status)) { abort = true; break; }
-    ph_mma ^= 1;
-    tc_fence_after();
-    // prefetch the next query tile into the other buffer (its GEMM completed)
-    if (tid == 0 && u + 1 < ue) {
-      const int nbh = (u + 1) / p.ntiles, nt = (u + 1) % p.ntiles;
-      ++q_issued[buf ^ 1];
-      mbar_arrive_expect_tx(&bar_q[buf ^ 1], kTileBytes);
-      tma_load_4d(sm + G::oQ + (buf ^ 1) * kTileBytes, &tm_q, 0, nt * kT, nbh % p.H, nbh / p.H,
-                  &bar_q[buf ^ 1]);
-    }
-    {
-      const float qoff = p.stab_q ? row_max_pair(lane_tm + G::tP, half, M_ / 2,
-                                                  (float*)(sm + G::oRed), row)
-                                  : 0.f;
-      exp2_rows_to_smem(lane_tm + G::tP, half * (M_ / 2), (half + 1) * (M_ / 2), qoff, false,
-                        s0 + G::oPsi, row);
-    }
-    fence_async_smem();
-    tc_fence_before();
-    __syncthreads();
-    if (tid == 0) {
-      tc_fence_after();
-      // [num hi | num lo | den hi, den lo] = Psi [S hi | S lo | (z hi, z lo)]
-      constexpr uint32_t id = idesc(128, 144, false, true, false);
+        for (int s = 0; s < kD / 16; ++s)
+          mma(tmem + G::tP + part * (M_ / 2), sdesc(sq + s * 32, 16, 1024),
+              sdesc(s0 + G::oW + part * (M_ / 2) * 128 + s * 32, 16, 1024), idh, s > 0);
+        if (part == 0) {
+          mma_commit(bar_ffullA);
+        } else {
+          mma_commit(bar_ffullB);
+          mma_commit(q_empty + (i & 1));
+        }
+      };
+      // features of item i: the head's operands (first item of a head), the
+      // converted Q tile, the previous item's TMEM columns released
+      auto issue_features = [&](int i) -> bool {
+        if (head_starts(i)) {
+          if (!wait_one(h_full, heads_seen & 1, abort_flag, p.dev_status)) return false;
+          ++heads_seen;
+        }
+        if (!wait_one(q_conv + (i & 1), (i >> 1) & 1, abort_flag, p.dev_status)) return false;
+        if (i > 0 && !wait_one(bar_ffreeA, (i - 1) & 1, abort_flag, p.dev_status)) return false;
+        tc_fence_after();
+        features(i, 0);
+        if (i > 0 && !wait_one(bar_ffreeB, (i - 1) & 1, abort_flag, p.dev_status)) return false;
+        tc_fence_after();
+        features(i, 1);
+        return true;
+      };
+      auto output = [&](int i) -> bool {
+        // [num hi | num lo | den hi, den lo] = Psi [S hi | S lo | (z hi, z lo)]
+        if (!wait_one(bar_pfull, i & 1, abort_flag, p.dev_status)) return false;
+        tc_fence_after();
+        constexpr uint32_t id = idesc(128, 144, false, true, false);
 #pragma unroll
-      for (int s = 0; s < M_ / 16; ++s)
-        mma(tmem + G::tO, sdesc(s0 + G::oPsi + (s / 4) * 16384 + (s % 4) * 32, 16, 1024),
-            sdesc(s0 + G::oImg + s * 2048, img_s_bytes(M_), 1024), id, s > 0);
-      mma_commit(bar_mma);
+        for (int s = 0; s < M_ / 16; ++s)
+          mma(tmem + G::tO, sdesc(s0 + G::oPsi + (s / 4) * 16384 + (s % 4) * 32, 16, 1024),
+              sdesc(s0 + G::oImg + s * 2048, img_s_bytes(M_), 1024), id, s > 0);
+        mma_commit(bar_ofull);
+        return true;
+      };
+      ok = issue_features(0);
+      for (int i = 0; ok && i < n; ++i) {
+        if (i + 1 < n && !head_starts(i + 1)) {
+          // the next tile's features first: they run under this tile's exponentials
+          if (!(ok = issue_features(i + 1))) break;
+          if (!(ok = output(i))) break;
+        } else {
+          // last tile of a head: its output GEMM, then the head's operands are free
+          if (!(ok = output(i))) break;
+          if (i + 1 < n) {
+            mma_commit(h_free);
+            if (!(ok = issue_features(i + 1))) break;
+          }
+        }
+      }
+      if (!ok) drain_mmas(bar_drain);
     }
-    if (!wait_all(bar_mma, ph_mma, p.dev_status)) { abort = true; break; }
-    ph_mma ^= 1;
-    tc_fence_after();
-    {
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int quad = warp & 3, half = warp >> 2;
+    const int row = quad * 32 + lane;
+    const uint32_t lane_tm = tmem + ((uint32_t)(quad * 32) << 16);
+    const int f_r0 = half * (M_ / 4), f_r1 = M_ / 2 + half * (M_ / 4);
+    // the output rows of item i (num / den read from TMEM)
+    auto store_out = [&](int i) {
+      const int u = ub + i, bh = u / p.ntiles, t = u % p.ntiles, b = bh / p.H, h = bh % p.H;
       const float den = tmem_ld1(lane_tm + G::tO + 128) + tmem_ld1(lane_tm + G::tO + 129);
       float v[32], vl[32];
       tmem_ld32(lane_tm + G::tO + half * 32, v);
       tmem_ld32(lane_tm + G::tO + 64 + half * 32, vl);
 #pragma unroll
-      for (int i = 0; i < 32; ++i) v[i] += vl[i];
+      for (int e = 0; e < 32; ++e) v[e] += vl[e];
       const int tok = t * kT + row;
       if (tok < p.L) {
         const bool live = p.qmask == nullptr || p.qmask[(size_t)b * p.L + tok] != 0;
@@ -257,16 +369,76 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int q4 = 0; q4 < 4; ++q4)
           dst[q4] = make_uint4(w[4 * q4], w[4 * q4 + 1], w[4 * q4 + 2], w[4 * q4 + 3]);
       }
+    };
+    bool ok = n > 0;
+    if (ok && p.stall > 0) ok = epi_wait(bar_never, 0, abort_flag, p.dev_status, p.stall);
+    for (int i = 0; ok && i < n; ++i) {
+      if (!(ok = epi_wait(bar_ffullA, i & 1, abort_flag, p.dev_status))) break;
+      tc_fence_after();
+      bool have_b = false;
+      float qoff = 0.f;
+      if (p.stab_q) {
+        // the row maximum over all M features (both parts, both thread halves)
+        if (!(ok = epi_wait(bar_ffullB, i & 1, abort_flag, p.dev_status))) break;
+        tc_fence_after();
+        have_b = true;
+        float mx = -INFINITY;
+#pragma unroll 1
+        for (int q = 0; q < 2 * NH; ++q) {
+          float v[32];
+          tmem_ld32(lane_tm + G::tP + (q < NH ? f_r0 + 32 * q : f_r1 + 32 * (q - NH)), v);
+#pragma unroll
+          for (int e = 0; e < 32; ++e) mx = fmaxf(mx, v[e]);
+        }
+        red[half * 128 + row] = mx;
+        epi_sync();
+        qoff = fmaxf(red[row], red[128 + row]);
+        epi_sync();                     // red may be reused
+      }
+      // ---- round 0 (part A)
+      uint32_t fv[NH][32], pk[NH][16];
+#pragma unroll
+      for (int q = 0; q < NH; ++q) tmem_ld32_async(lane_tm + G::tP + f_r0 + 32 * q, fv[q]);
+#pragma unroll
+      for (int q = 0; q < NH; ++q) tmem_wait_ld(fv[q]);
+      tc_fence_before();
+      warp_arrive(bar_ffreeA);
+#pragma unroll
+      for (int q = 0; q < NH; ++q) exp2_pack32(fv[q], qoff, false, pk[q]);
+      // ---- the previous tile's output GEMM is done: its rows out, Psi free
+      if (i > 0) {
+        if (!(ok = epi_wait(bar_ofull, (i - 1) & 1, abort_flag, p.dev_status))) break;
+        tc_fence_after();
+        store_out(i - 1);
+      }
+#pragma unroll
+      for (int q = 0; q < NH; ++q) store_row32(pk[q], s0 + G::oPsi, row, f_r0 + 32 * q);
+      // ---- round 1 (part B)
+      if (!have_b) {
+        if (!(ok = epi_wait(bar_ffullB, i & 1, abort_flag, p.dev_status))) break;
+        tc_fence_after();
+      }
+#pragma unroll
+      for (int q = 0; q < NH; ++q) tmem_ld32_async(lane_tm + G::tP + f_r1 + 32 * q, fv[q]);
+#pragma unroll
+      for (int q = 0; q < NH; ++q) tmem_wait_ld(fv[q]);
+      tc_fence_before();
+      warp_arrive(bar_ffreeB);
+#pragma unroll
+      for (int q = 0; q < NH; ++q) {
+        exp2_pack32(fv[q], qoff, false, pk[q]);
+        store_row32(pk[q], s0 + G::oPsi, row, f_r1 + 32 * q);
+      }
+      fence_async_smem();
+      tc_fence_before();
+      warp_arrive(bar_pfull);
     }
-    tc_fence_before();
-    __syncthreads();
-  }
-  if (abort && tid == 0) {
-    // no copy or MMA of this CTA may still be running when TMEM is freed
-    drain_loads(bar_head, h_issued, h_waited);
-    drain_loads(&bar_q[0], q_issued[0], q_waited[0]);
-    drain_loads(&bar_q[1], q_issued[1], q_waited[1]);
-    drain_mmas(bar_drain);
+    if (ok) {
+      // the last tile's rows
+      ok = epi_wait(bar_ofull, (n - 1) & 1, abort_flag, p.dev_status);
+      tc_fence_after();
+      if (ok) store_out(n - 1);
+    }
   }
   tc_fence_before();
   __syncthreads();
