@@ -31,6 +31,7 @@ struct FwdArgs {
   cudaStream_t stream;
   // TMA descriptors of W', q, k, v, encoded once per call by tc_make_maps
   CUtensorMap tm_w, tm_q, tm_k, tm_v;
+  CUtensorMap tm_o;               // out, 64 x 128 boxes (tensor stores of the d = 64 paths)
   bool maps_ready;
   int path;                       // kernel path chosen by fwd_prepare
 };

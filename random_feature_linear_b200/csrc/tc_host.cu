@@ -55,6 +55,10 @@ bool tc_make_maps(FwdArgs& a) {
                  encode_tmap(&a.tm_q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, a.q, qd, qst, xb) &&
                  encode_tmap(&a.tm_k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, a.k, kd, kst, xb) &&
                  encode_tmap(&a.tm_v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, a.v, kd, kst, xb);
+  // out: L query rows with strides os
+  const uint64_t ost[3] = {(uint64_t)a.os[2] * 2, (uint64_t)a.os[1] * 2, (uint64_t)a.os[0] * 2};
+  a.maps_ready = a.maps_ready &&
+                 encode_tmap(&a.tm_o, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, a.out, qd, ost, xb);
   return a.maps_ready;
 }
 

@@ -135,6 +135,26 @@ __device__ __forceinline__ void q_to_fp16(uint32_t saddr, int ctid, int* dev_sta
   if ((mag & 0xFFFFu) >= 0x4780u || (mag >> 16) >= 0x4780u) report(dev_status, DARK_ERR_NUMERIC);
 }
 
+// Tensor store of one 128-row tile from shared memory (128B-swizzled, as the
+// map says) to global memory; rows past the tensor's end are not written.
+__device__ __forceinline__ void tma_store_4d(const CUtensorMap* map, uint32_t ssrc, int x, int y,
+                                             int z, int w) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.global.shared::cta.bulk_group [%0, {%2, %3, %4, %5}], [%1];" ::"l"(
+          (uint64_t)map),
+      "r"(ssrc), "r"(x), "r"(y), "r"(z), "r"(w)
+      : "memory");
+}
+__device__ __forceinline__ void bulk_commit_group() {
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+__device__ __forceinline__ void bulk_wait_group_read() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+__device__ __forceinline__ void bulk_wait_group() {
+  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+}
+
 // Query kernel: each CTA walks a contiguous range of (head, query tile) items
 // with four roles. Warp 9 loads the head operands (W' feature rows and the
 // [S | z] image, once per head) and the Q tiles (two buffers); warps 10-11
@@ -147,7 +167,7 @@ __device__ __forceinline__ void q_to_fp16(uint32_t saddr, int ctid, int* dev_sta
 template <int M_, int R_>
 __global__ void __launch_bounds__(kThreads, 1)
     queries_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_q,
-                   const QueryParams p) {
+                   const __grid_constant__ CUtensorMap tm_o, const QueryParams p) {
   using G = QueryCfg<M_, R_>;
   constexpr int NH = M_ / 128;                // 32-column chunks per round
   extern __shared__ uint8_t smem_raw[];
@@ -341,33 +361,45 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int row = quad * 32 + lane;
     const uint32_t lane_tm = tmem + ((uint32_t)(quad * 32) << 16);
     const int f_r0 = half * (M_ / 4), f_r1 = M_ / 2 + half * (M_ / 4);
-    // the output rows of item i (num / den read from TMEM)
+    // the output rows of item i (num / den read from TMEM): each thread packs
+    // its half row into the staging area (the second half of the Psi buffer,
+    // which the next tile's first round does not write; 16-byte chunks
+    // XOR-swizzled by row, as the output map's 128-byte swizzle expects), then
+    // one thread stores the tile with a tensor store. The staging is free again
+    // once that store has read it (thread 0 waits for that before the second
+    // round's Psi stores; an epilogue barrier follows).
+    const uint32_t stage = s0 + G::oPsi + M_ * 128;
     auto store_out = [&](int i) {
       const int u = ub + i, bh = u / p.ntiles, t = u % p.ntiles, b = bh / p.H, h = bh % p.H;
+      uint32_t vh[32], vl[32];
+      tmem_ld32_async(lane_tm + G::tO + half * 32, vh);
+      tmem_ld32_async(lane_tm + G::tO + 64 + half * 32, vl);
+      // (each synchronous load waits for every load of the thread)
       const float den = tmem_ld1(lane_tm + G::tO + 128) + tmem_ld1(lane_tm + G::tO + 129);
-      float v[32], vl[32];
-      tmem_ld32(lane_tm + G::tO + half * 32, v);
-      tmem_ld32(lane_tm + G::tO + 64 + half * 32, vl);
-#pragma unroll
-      for (int e = 0; e < 32; ++e) v[e] += vl[e];
+      tmem_wait_ld(vh);
+      tmem_wait_ld(vl);
       const int tok = t * kT + row;
-      if (tok < p.L) {
-        const bool live = p.qmask == nullptr || p.qmask[(size_t)b * p.L + tok] != 0;
-        const float inv = live && den > 0.f ? 1.f / den : 0.f;
-        uint32_t w[16];
-        bool bad = !isfinite(den);
+      const bool live = tok < p.L && (p.qmask == nullptr || p.qmask[(size_t)b * p.L + tok] != 0);
+      const float inv = live && den > 0.f ? 1.f / den : 0.f;
+      float sum = den;                  // non-finite if any value is
+      uint32_t w[16];
 #pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const float a = v[2 * e] * inv, c = v[2 * e + 1] * inv;
-          bad |= !isfinite(a) || !isfinite(c);
-          w[e] = pack_bf16(a, c);
-        }
-        if (bad) report(p.dev_status, DARK_ERR_NUMERIC);
-        uint4* dst = reinterpret_cast<uint4*>(p.out + (int64_t)b * p.ob + (int64_t)h * p.oh +
-                                              (int64_t)tok * p.ol + half * 32);
+      for (int e = 0; e < 16; ++e) {
+        const float a = (__uint_as_float(vh[2 * e]) + __uint_as_float(vl[2 * e])) * inv;
+        const float c = (__uint_as_float(vh[2 * e + 1]) + __uint_as_float(vl[2 * e + 1])) * inv;
+        sum += a + c;
+        w[e] = pack_bf16(a, c);
+      }
+      if (tok < p.L && !isfinite(sum)) report(p.dev_status, DARK_ERR_NUMERIC);
 #pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4)
-          dst[q4] = make_uint4(w[4 * q4], w[4 * q4 + 1], w[4 * q4 + 2], w[4 * q4 + 3]);
+      for (int c = 0; c < 4; ++c)
+        st_shared_v4(stage + row * 128 + (uint32_t)(((half * 4 + c) ^ (row & 7)) * 16), w[4 * c],
+                     w[4 * c + 1], w[4 * c + 2], w[4 * c + 3]);
+      fence_async_smem();
+      epi_sync();
+      if (tid == 0) {
+        tma_store_4d(&tm_o, stage, 0, t * kT, h, b);
+        bulk_commit_group();
       }
     };
     bool ok = n > 0;
@@ -425,10 +457,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       warp_arrive(bar_ffreeB);
 #pragma unroll
-      for (int q = 0; q < NH; ++q) {
-        exp2_pack32(fv[q], qoff, false, pk[q]);
-        store_row32(pk[q], s0 + G::oPsi, row, f_r1 + 32 * q);
+      for (int q = 0; q < NH; ++q) exp2_pack32(fv[q], qoff, false, pk[q]);
+      if (i > 0) {
+        // the previous tile's tensor store has read the staging
+        if (tid == 0) bulk_wait_group_read();
+        epi_sync();
       }
+#pragma unroll
+      for (int q = 0; q < NH; ++q) store_row32(pk[q], s0 + G::oPsi, row, f_r1 + 32 * q);
       fence_async_smem();
       tc_fence_before();
       warp_arrive(bar_pfull);
@@ -439,6 +475,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       if (ok) store_out(n - 1);
     }
+    if (tid == 0) bulk_wait_group();    // every tensor store has completed
   }
   tc_fence_before();
   __syncthreads();
@@ -509,7 +546,7 @@ cudaError_t launch(const FwdArgs& a, const CUtensorMap& tw, const CUtensorMap& t
   e = set_smem_limit_once((const void*)queries_kernel<M_, R_>, (int)QG::kSmem, smem_set);
   if (e != cudaSuccess) return e;
   const int grid = qp.total_tiles < kSms ? qp.total_tiles : kSms;
-  queries_kernel<M_, R_><<<grid, kThreads, QG::kSmem, a.stream>>>(tw, tq, qp);
+  queries_kernel<M_, R_><<<grid, kThreads, QG::kSmem, a.stream>>>(tw, tq, a.tm_o, qp);
   return cudaGetLastError();
 }
 
