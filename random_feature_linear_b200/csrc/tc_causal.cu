@@ -31,6 +31,7 @@
 #include "internal.h"
 #include "tc_common.cuh"
 #include "tc_keys.cuh"
+#include "tc_roles.cuh"
 
 namespace dark {
 namespace {
@@ -102,7 +103,7 @@ template <int M_, int R_>
 __global__ void __launch_bounds__(kThreads, 1)
     causal_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_q,
                   const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
-                  const Params p) {
+                  const __grid_constant__ CUtensorMap tm_o, const Params p) {
   using G = Cfg<M_, R_>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
@@ -179,6 +180,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (!wait_all(bar_tma, ph_tma, p.dev_status)) { abort = true; break; }
     ph_tma ^= 1;
     ++tma_waited;
+    // the previous chunk's output tensor store has read its staging (in the
+    // Psi region, written again below)
+    if (tid == 0) bulk_wait_group_read();
     // k, then q: bf16 -> fp16 in place (the feature GEMMs run on fp16 operands);
     // the key GEMM starts while the query tile converts
     to_fp16_inplace(s0 + G::oK, kTileBytes, p.dev_status);
@@ -444,24 +448,31 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int i = 0; i < 32; ++i) v[i] += vl[i];
         den += tmem_ld1(lane_tm + G::tDen + 1);
       }
+      // the chunk's rows staged in the Psi region (free once the inter GEMM is
+      // done; 16-byte chunks XOR-swizzled by row, as the output map's 128-byte
+      // swizzle expects), then one tensor store (rows past L are not written)
       const int tok = t0 + row;
-      if (tok < p.L) {
-        const float inv = den > 0.f ? 1.f / den : 0.f;
-        uint32_t w[16];
-        bool bad = false;
+      const float inv = den > 0.f ? 1.f / den : 0.f;
+      uint32_t w[16];
+      float sum = den;                  // non-finite if any value is
 #pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const float a = v[2 * e] * inv, bb = v[2 * e + 1] * inv;
-          bad |= !isfinite(a) || !isfinite(bb);
-          w[e] = pack_bf16(a, bb);
-        }
-        if (bad || !isfinite(den)) report(p.dev_status, DARK_ERR_NUMERIC);
-        uint4* dst = reinterpret_cast<uint4*>(p.out + (int64_t)b * p.ob + (int64_t)h * p.oh +
-                                              (int64_t)tok * p.ol + half * 32);
-#pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4)
-          dst[q4] = make_uint4(w[4 * q4], w[4 * q4 + 1], w[4 * q4 + 2], w[4 * q4 + 3]);
+      for (int e = 0; e < 16; ++e) {
+        const float a = v[2 * e] * inv, bb = v[2 * e + 1] * inv;
+        sum += a + bb;
+        w[e] = pack_bf16(a, bb);
       }
+      if (tok < p.L && !isfinite(sum)) report(p.dev_status, DARK_ERR_NUMERIC);
+      const uint32_t stage = s0 + G::oPsi;
+#pragma unroll
+      for (int q4 = 0; q4 < 4; ++q4)
+        st_shared_v4(stage + row * 128 + (uint32_t)(((half * 4 + q4) ^ (row & 7)) * 16), w[4 * q4],
+                     w[4 * q4 + 1], w[4 * q4 + 2], w[4 * q4 + 3]);
+      fence_async_smem();
+    }
+    __syncthreads();
+    if (tid == 0) {
+      tma_store_4d(&tm_o, s0 + G::oPsi, 0, t0, h, b);
+      bulk_commit_group();
     }
     tc_fence_before();
     __syncthreads();
@@ -474,6 +485,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   if (!abort && p.st_shift != nullptr && tid == 0 && c_end == p.nc)
     p.st_shift[bh] = c_run > -INFINITY ? c_run : 0.f;
+  if (tid == 0) bulk_wait_group();      // every output tensor store has completed
   if (abort && tid == 0) {
     // no copy or MMA of this CTA may still be running when TMEM is freed
     drain_loads(bar_tma, tma_issued, tma_waited);
@@ -558,7 +570,7 @@ cudaError_t launch(const FwdArgs& a, const CUtensorMap& tw, const CUtensorMap& t
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = s.nseg > 1 ? 1 : 0;
-  return cudaLaunchKernelEx(&cfg, causal_kernel<M_, R_>, tw, tq, tk, tv, p);
+  return cudaLaunchKernelEx(&cfg, causal_kernel<M_, R_>, tw, tq, tk, tv, a.tm_o, p);
 }
 
 

@@ -46,43 +46,72 @@ __host__ __device__ constexpr uint32_t img_bytes(int m) { return 3 * img_s_bytes
 // kernel's operand image (hi + lo bf16) and, if requested, the fp32 state.
 // Stabiliser (shifts non-null): partial s is scaled by 2^-shifts[s]; the sum is
 // taken relative to the largest of them, c_K (0 when no key is valid), which
-// is the state's shift.
+// is the state's shift. One thread per (feature f, group of 8 value columns),
+// consecutive threads over f (coalesced partial reads); group 8 is z.
 __global__ void reduce_kernel(const float* __restrict__ partials, int nsplit, int m,
                               const float* __restrict__ shifts, uint8_t* __restrict__ images,
                               float* __restrict__ st_kv, float* __restrict__ st_z,
                               float* __restrict__ st_shift) {
   const int bh = blockIdx.y;
   const int idx = blockIdx.x * blockDim.x + threadIdx.x;
-  if (idx >= 65 * m) return;
-  const int col = idx / m, f = idx % m;
-  const float* src = partials + (size_t)bh * nsplit * 65 * m + idx;
-  float acc = 0.f;
-  if (shifts == nullptr) {
-    for (int s = 0; s < nsplit; ++s) acc += src[(size_t)s * 65 * m];
-  } else {
-    const float* sh = shifts + (size_t)bh * nsplit;
-    float cmax = -INFINITY;
+  if (idx >= 9 * m) return;
+  const int cg = idx / m, f = idx % m;
+  const int ncol = cg < 8 ? 8 : 1;
+  const float* src = partials + (size_t)bh * nsplit * 65 * m + (size_t)(cg * 8) * m + f;
+  float acc[8];
+#pragma unroll
+  for (int c = 0; c < 8; ++c) acc[c] = 0.f;
+  const float* sh = shifts == nullptr ? nullptr : shifts + (size_t)bh * nsplit;
+  float cmax = -INFINITY;
+  if (sh != nullptr)
     for (int s = 0; s < nsplit; ++s) cmax = fmaxf(cmax, sh[s]);
-    for (int s = 0; s < nsplit; ++s)
-      if (sh[s] > -INFINITY) acc += exp2f(sh[s] - cmax) * src[(size_t)s * 65 * m];
-    if (idx == 0 && st_shift != nullptr) st_shift[bh] = cmax > -INFINITY ? cmax : 0.f;
+  for (int s = 0; s < nsplit; ++s) {
+    float sc = 1.f;
+    if (sh != nullptr) {
+      if (!(sh[s] > -INFINITY)) continue;
+      sc = exp2f(sh[s] - cmax);
+    }
+    const float* ps = src + (size_t)s * 65 * m;
+#pragma unroll
+    for (int c = 0; c < 8; ++c)
+      if (c < ncol) acc[c] += (sh != nullptr ? sc * ps[(size_t)c * m] : ps[(size_t)c * m]);
   }
-  const __nv_bfloat16 hi = __float2bfloat16_rn(acc);
-  const __nv_bfloat16 lo = __float2bfloat16_rn(acc - __bfloat162float(hi));
+  if (sh != nullptr && idx == 0 && st_shift != nullptr)
+    st_shift[bh] = cmax > -INFINITY ? cmax : 0.f;
+  uint32_t hi2[4], lo2[4];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const __nv_bfloat16 h0 = __float2bfloat16_rn(acc[2 * e]), h1 = __float2bfloat16_rn(acc[2 * e + 1]);
+    const __nv_bfloat16 l0 = __float2bfloat16_rn(acc[2 * e] - __bfloat162float(h0));
+    const __nv_bfloat16 l1 = __float2bfloat16_rn(acc[2 * e + 1] - __bfloat162float(h1));
+    hi2[e] = (uint32_t)__bfloat16_as_ushort(h0) | ((uint32_t)__bfloat16_as_ushort(h1) << 16);
+    lo2[e] = (uint32_t)__bfloat16_as_ushort(l0) | ((uint32_t)__bfloat16_as_ushort(l1) << 16);
+  }
   uint8_t* img = images + (size_t)bh * img_bytes(m);
   const uint32_t row = (uint32_t)(f / 8) * 1024 + (uint32_t)(f % 8) * 128;
-  if (col < 64) {
-    const uint32_t off = row + (uint32_t)((((col / 8) ^ (f % 8)) * 16)) + (uint32_t)(col % 8) * 2;
-    *reinterpret_cast<__nv_bfloat16*>(img + off) = hi;
-    *reinterpret_cast<__nv_bfloat16*>(img + img_s_bytes(m) + off) = lo;
-    if (st_kv != nullptr) st_kv[((size_t)bh * m + f) * 64 + col] = acc;
+  if (cg < 8) {
+    // columns 8 cg .. 8 cg + 7: one 16-byte chunk of row f in each of the S
+    // blocks (hi, lo), chunk index XOR-swizzled by f % 8
+    const uint32_t off = row + (uint32_t)((cg ^ (f % 8)) * 16);
+    *reinterpret_cast<uint4*>(img + off) = make_uint4(hi2[0], hi2[1], hi2[2], hi2[3]);
+    *reinterpret_cast<uint4*>(img + img_s_bytes(m) + off) = make_uint4(lo2[0], lo2[1], lo2[2], lo2[3]);
+    if (st_kv != nullptr) {
+      float* d = st_kv + ((size_t)bh * m + f) * 64 + cg * 8;
+      if ((reinterpret_cast<uintptr_t>(d) & 15) == 0) {
+        reinterpret_cast<float4*>(d)[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+        reinterpret_cast<float4*>(d)[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
+      } else {
+#pragma unroll
+        for (int c = 0; c < 8; ++c) d[c] = acc[c];
+      }
+    }
   } else {
     // columns 0-7 and 8-15 of the third block: (z hi, z lo, 0, ...), zeros
     uint8_t* zz = img + 2 * img_s_bytes(m) + row;
-    const uint32_t w0 = (uint32_t)__bfloat16_as_ushort(hi) | ((uint32_t)__bfloat16_as_ushort(lo) << 16);
+    const uint32_t w0 = (hi2[0] & 0xFFFFu) | ((lo2[0] & 0xFFFFu) << 16);
     *reinterpret_cast<uint4*>(zz + (uint32_t)((0 ^ (f % 8)) * 16)) = make_uint4(w0, 0u, 0u, 0u);
     *reinterpret_cast<uint4*>(zz + (uint32_t)((1 ^ (f % 8)) * 16)) = make_uint4(0u, 0u, 0u, 0u);
-    if (st_z != nullptr) st_z[(size_t)bh * m + f] = acc;
+    if (st_z != nullptr) st_z[(size_t)bh * m + f] = acc[0];
   }
 }
 
@@ -133,26 +162,6 @@ __device__ __forceinline__ void q_to_fp16(uint32_t saddr, int ctid, int* dev_sta
     st_shared_v4(a, u.x, u.y, u.z, u.w);
   }
   if ((mag & 0xFFFFu) >= 0x4780u || (mag >> 16) >= 0x4780u) report(dev_status, DARK_ERR_NUMERIC);
-}
-
-// Tensor store of one 128-row tile from shared memory (128B-swizzled, as the
-// map says) to global memory; rows past the tensor's end are not written.
-__device__ __forceinline__ void tma_store_4d(const CUtensorMap* map, uint32_t ssrc, int x, int y,
-                                             int z, int w) {
-  asm volatile(
-      "cp.async.bulk.tensor.4d.global.shared::cta.bulk_group [%0, {%2, %3, %4, %5}], [%1];" ::"l"(
-          (uint64_t)map),
-      "r"(ssrc), "r"(x), "r"(y), "r"(z), "r"(w)
-      : "memory");
-}
-__device__ __forceinline__ void bulk_commit_group() {
-  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
-}
-__device__ __forceinline__ void bulk_wait_group_read() {
-  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
-}
-__device__ __forceinline__ void bulk_wait_group() {
-  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
 }
 
 // Query kernel: each CTA walks a contiguous range of (head, query tile) items
@@ -522,7 +531,7 @@ cudaError_t launch(const FwdArgs& a, const CUtensorMap& tw, const CUtensorMap& t
   float* shifts = stab ? (float*)(ws + s.off_shift) : nullptr;
   cudaError_t e = tc_launch_key_states(a, tw, tk, tv, s.ntiles, s.nsplit, partials, shifts);
   if (e != cudaSuccess) return e;
-  reduce_kernel<<<dim3((65 * a.m + 255) / 256, bh), 256, 0, a.stream>>>(
+  reduce_kernel<<<dim3((9 * a.m + 255) / 256, bh), 256, 0, a.stream>>>(
       partials, s.nsplit, a.m, shifts, images, a.st_kv, a.st_z, a.st_shift);
 
   QueryParams qp;
