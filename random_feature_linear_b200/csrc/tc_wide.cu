@@ -723,7 +723,8 @@ __device__ __forceinline__ bool grp_wait(int g, uint64_t* bar, uint32_t parity,
 
 template <int D_, int M_>
 __global__ void __launch_bounds__(kThreadsV, 1)
-    values_kernel(const __grid_constant__ CUtensorMap tm_v, const ValParams p) {
+    values_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
+                  const ValParams p) {
   using G = ValCfg<D_, M_>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
@@ -1001,16 +1002,38 @@ __global__ void __launch_bounds__(kThreadsV, 1)
           nm[8 * q4 + 2 * e + 1] = fmaf(pden, mf.y, dp * of.y);
         }
       }
-      // every reader of the group is done: expect the peer's chunk cc + 2 in this
-      // buffer and tell the peer it may send it
+      // every reader of the group is done with o': the rows go out through the
+      // same buffer (two 64-column halves, 64 rows x 128 B each, 16-byte chunks
+      // XOR-swizzled by row as the output map's 128-byte swizzle expects) by two
+      // tensor stores; then the peer may send its chunk cc + 2 into the buffer
+      grp_sync_or(grp, false);
+      const float dt = pden + dp;
+      const float invd = dt > 0.f ? 1.f / dt : 0.f;
+      float sum = dt;                   // non-finite if any value is
+      uint32_t w[32];
+#pragma unroll
+      for (int e = 0; e < 32; ++e) {
+        const float o0 = nm[2 * e] * invd, o1 = nm[2 * e + 1] * invd;
+        sum += o0 + o1;
+        w[e] = pack_bf16(o0, o1);
+      }
+      if (cc * kC + row < p.L && !isfinite(sum)) report(p.dev_status, DARK_ERR_NUMERIC);
+      const int r = row & 63;
+      const uint32_t stg = xb + colh * 8192 + (uint32_t)r * 128;
+#pragma unroll
+      for (int q4 = 0; q4 < 8; ++q4)
+        st_shared_v4(stg + (uint32_t)((q4 ^ (r & 7)) * 16), w[4 * q4], w[4 * q4 + 1], w[4 * q4 + 2],
+                     w[4 * q4 + 3]);
+      fence_async_smem();
       grp_sync_or(grp, false);
       if (gi == 0) {
+        tma_store_4d(&tm_o, xb, 128 * vb, cc * kC + 64 * fh, h, b);
+        tma_store_4d(&tm_o, xb + 8192, 128 * vb + 64, cc * kC + 64 * fh, h, b);
+        bulk_commit_group();
+        bulk_wait_group_read();
         if (cc + 2 < p.nc) mbar_arrive_expect_tx(bar_recv + (cc & 1), G::kXBytes);
         arrive_peer_relaxed(peer_addr(smem_u32(bar_rfree + (cc & 1)), peer));
       }
-      const float dt = pden + dp;
-      if (cc * kC + row < p.L && !store_row(cc, nm, dt > 0.f ? 1.f / dt : 0.f, dt))
-        report(p.dev_status, DARK_ERR_NUMERIC);
       return true;
     };
     // S operand half of feature tile t for chunk c (group grp's features)
@@ -1198,6 +1221,7 @@ __global__ void __launch_bounds__(kThreadsV, 1)
       warp_arrive(bar_smfree + (c & 1));
     }
     if (ok && G::FS == 2 && (row >> 6) == fh && p.nc > 0) ok = finish_prev(p.nc - 1);
+    if (G::FS == 2 && (row >> 6) == fh && gi == 0) bulk_wait_group();   // the output stores are done
     ok = !epi_sync_or(!ok);
     // final state: S_t (my features x my 128 value columns) and z (first value block)
     if (ok && p.st_kv != nullptr) {
@@ -1245,6 +1269,12 @@ bool make_wide_maps(FwdArgs& a) {
                  encode_tmap(&a.tm_q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, a.q, xd, xs, xb) &&
                  encode_tmap(&a.tm_k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, a.k, xd, xs, xb) &&
                  encode_tmap(&a.tm_v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, a.v, xd, xs, xb);
+  // out: 64-column x 64-row boxes (the half-chunk rows one CTA of a cluster finishes)
+  const uint64_t od[4] = {(uint64_t)a.d, (uint64_t)a.L, (uint64_t)a.H, (uint64_t)a.B};
+  const uint64_t ost[3] = {(uint64_t)a.os[2] * 2, (uint64_t)a.os[1] * 2, (uint64_t)a.os[0] * 2};
+  const uint32_t ob[4] = {64, 64, 1, 1};
+  a.maps_ready = a.maps_ready &&
+                 encode_tmap(&a.tm_o, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, a.out, od, ost, ob);
   return a.maps_ready;
 }
 
@@ -1340,7 +1370,7 @@ cudaError_t launch(const FwdArgs& a) {
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  e = cudaLaunchKernelEx(&cfg, values_kernel<D_, M_>, a.tm_v, vp);
+  e = cudaLaunchKernelEx(&cfg, values_kernel<D_, M_>, a.tm_v, a.tm_o, vp);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
