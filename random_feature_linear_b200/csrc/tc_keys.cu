@@ -91,7 +91,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     keys_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, const KeyParams p) {
   using G = KeyCfg<M_, R_>;
-  constexpr int NH = M_ / 128;                // 32-column groups per round (two rounds per half)
+  constexpr int NH = M_ / 128;                // 32-column groups per pass (two passes per half)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   const uint32_t s0 = smem_u32(sm);
@@ -292,10 +292,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int i = 0; ok && i < n; ++i) {
       const int t = tb + i;
-      // ---- this tile's features: the norm columns and round 0 (part A), the
-      // first round exponentiated while the previous chunk-state GEMM may
-      // still read Phi, then round 1 (part B); each part's TMEM columns are
-      // released as soon as they are read. Round r, chunk q of thread half h
+      // ---- this tile's features: the norm columns and pass 0 (part A), the
+      // first pass exponentiated while the previous chunk-state GEMM may
+      // still read Phi, then pass 1 (part B); each part's TMEM columns are
+      // released as soon as they are read. Pass r, chunk q of thread half h
       // holds features r M/2 + h M/4 + 32 q.
       if (!(ok = epi_wait(bar_ffullA, i & 1, abort_flag, p.dev_status))) break;
       tc_fence_after();
@@ -366,7 +366,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
 #pragma unroll
       for (int q = 0; q < NH; ++q) store_row32(pk[q], s0 + G::oPhi, row, f_r0 + 32 * q);
-      // ---- round 1 (part B)
+      // ---- pass 1 (part B)
       if (!have_b) {
         if (!(ok = epi_wait(bar_ffullB, i & 1, abort_flag, p.dev_status))) break;
         tc_fence_after();

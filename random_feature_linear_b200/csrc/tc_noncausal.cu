@@ -178,7 +178,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     queries_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_q,
                    const __grid_constant__ CUtensorMap tm_o, const QueryParams p) {
   using G = QueryCfg<M_, R_>;
-  constexpr int NH = M_ / 128;                // 32-column chunks per round
+  constexpr int NH = M_ / 128;                // 32-column chunks per pass
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   const uint32_t s0 = smem_u32(sm);
@@ -372,11 +372,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int f_r0 = half * (M_ / 4), f_r1 = M_ / 2 + half * (M_ / 4);
     // the output rows of item i (num / den read from TMEM): each thread packs
     // its half row into the staging area (the second half of the Psi buffer,
-    // which the next tile's first round does not write; 16-byte chunks
+    // which the next tile's first pass does not write; 16-byte chunks
     // XOR-swizzled by row, as the output map's 128-byte swizzle expects), then
     // one thread stores the tile with a tensor store. The staging is free again
     // once that store has read it (thread 0 waits for that before the second
-    // round's Psi stores; an epilogue barrier follows).
+    // pass's Psi stores; an epilogue barrier follows).
     const uint32_t stage = s0 + G::oPsi + M_ * 128;
     auto store_out = [&](int i) {
       const int u = ub + i, bh = u / p.ntiles, t = u % p.ntiles, b = bh / p.H, h = bh % p.H;
@@ -436,7 +436,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         qoff = fmaxf(red[row], red[128 + row]);
         epi_sync();                     // red may be reused
       }
-      // ---- round 0 (part A)
+      // ---- pass 0 (part A)
       uint32_t fv[NH][32], pk[NH][16];
 #pragma unroll
       for (int q = 0; q < NH; ++q) tmem_ld32_async(lane_tm + G::tP + f_r0 + 32 * q, fv[q]);
@@ -454,7 +454,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
 #pragma unroll
       for (int q = 0; q < NH; ++q) store_row32(pk[q], s0 + G::oPsi, row, f_r0 + 32 * q);
-      // ---- round 1 (part B)
+      // ---- pass 1 (part B)
       if (!have_b) {
         if (!(ok = epi_wait(bar_ffullB, i & 1, abort_flag, p.dev_status))) break;
         tc_fence_after();
