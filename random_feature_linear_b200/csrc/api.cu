@@ -49,6 +49,8 @@ size_t ws_need(Path p, int B, int H, int Lq, int Lk, int m, int r, int d, int fl
     case Path::TcWide: return dark::tc_wide_workspace_bytes(B, H, Lq, m, d, r);
     case Path::TcNonCausal: return dark::tc_noncausal_workspace_bytes(B, H, Lq, Lk, m, d);
     case Path::Exact: return dark::exact_workspace_bytes(B, H, Lq, Lk, r);
+    // the key-range splits run only when the caller's workspace holds them
+    // (the public workspace queries include them)
     case Path::TcExact: return dark::kWsHeader;
     default: return dark::simt_workspace_bytes(B, H, Lq, Lk, m, d, flags);
   }
@@ -215,7 +217,15 @@ dark_status dark_make_projection(const float* omega, int heads_omega, const floa
 size_t dark_attention_workspace_bytes(const dark_projection* proj, int B, int H, int L,
                                       int flags) {
   if (!proj_ok(proj) || B < 1 || H < 1 || L < 1) return 0;
-  if (flags & DARK_EXACT) return dark::exact_workspace_bytes(B, H, L, L, proj->r);
+  if (flags & DARK_EXACT) {
+    // either exact path may run (the tensor-core one for bf16 d = 64, 128)
+    const size_t simt = dark::exact_workspace_bytes(B, H, L, L, proj->r);
+    const size_t tc = (proj->d == 64 || proj->d == 128)
+                          ? dark::tc_exact_workspace_bytes(B, H, L, L, proj->d,
+                                                           (flags & DARK_CAUSAL) != 0)
+                          : 0;
+    return simt > tc ? simt : tc;
+  }
   const int m = proj->m, d = proj->d;
   size_t need = dark::simt_workspace_bytes(B, H, L, L, m, d, flags);
   const size_t tc = (flags & DARK_CAUSAL) ? dark::tc_causal_workspace_bytes(B, H, L, m, d)
@@ -243,7 +253,13 @@ dark_status dark_attention_fwd(const dark_projection* proj, const void* q, const
 size_t dark_cross_attention_workspace_bytes(const dark_projection* proj, int B, int H, int Lq,
                                             int Lk, int flags) {
   if (!proj_ok(proj) || B < 1 || H < 1 || Lq < 1 || Lk < 1 || (flags & DARK_CAUSAL)) return 0;
-  if (flags & DARK_EXACT) return dark::exact_workspace_bytes(B, H, Lq, Lk, proj->r);
+  if (flags & DARK_EXACT) {
+    const size_t simt = dark::exact_workspace_bytes(B, H, Lq, Lk, proj->r);
+    const size_t tc = (proj->d == 64 || proj->d == 128)
+                          ? dark::tc_exact_workspace_bytes(B, H, Lq, Lk, proj->d, 0)
+                          : 0;
+    return simt > tc ? simt : tc;
+  }
   const size_t simt = dark::simt_workspace_bytes(B, H, Lq, Lk, proj->m, proj->d, flags);
   const size_t tc = dark::tc_noncausal_workspace_bytes(B, H, Lq, Lk, proj->m, proj->d);
   return simt > tc ? simt : tc;

@@ -111,6 +111,9 @@ cudaError_t exact_forward(const FwdArgs& a);
 // ... and on tcgen05 for bf16, d = 64, r in {16, 32, 48, 64} (no workspace).
 bool tc_exact_supported(FwdArgs& a);
 cudaError_t tc_exact_forward(const FwdArgs& a);
+// Workspace of the tensor-core exact path (d = 64 or 128): the key-range
+// splits' partial results when the query tiles alone are too few for the GPU.
+size_t tc_exact_workspace_bytes(int B, int H, int Lq, int Lk, int d, int causal);
 
 // Decode step over [B][H] heads.
 struct DecodeArgs {

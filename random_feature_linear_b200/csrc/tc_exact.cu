@@ -65,9 +65,21 @@ struct Params {
   const uint8_t* kmask;                    // [B][Lk] or null
   const uint8_t* qmask;                    // [B][Lq] or null
   int B, H, Lq, Lk, nq, causal, heads_w, m, r;
+  // key ranges: a query tile's key tiles are cut into splits of at most S
+  // tiles, one CTA each (blockIdx: head fastest, then query tile, then split);
+  // a tile with more than one split leaves (O, l, m) per split in `part`
+  // ([B*H][nq][maxsplits] slots of 128 (d + 2) floats) for the combine kernel
+  int S, maxsplits;
+  float* part;
   int* dev_status;
   long long stall;                         // testing stall before the first wait (0: none)
 };
+
+// Key tiles of query tile qt.
+__host__ __device__ inline int exact_key_tiles(int qt, int Lk, int causal) {
+  const int nk_all = (Lk + 127) / 128;
+  return causal ? (qt + 1 < nk_all ? qt + 1 : nk_all) : nk_all;
+}
 
 // Projection epilogue: this thread's row of the N = r projection in TMEM, times
 // `scale`, as fp16 into K-major 128B-swizzled 64-column blocks 16 KB apart
@@ -105,6 +117,15 @@ __global__ void __launch_bounds__(kThreads, D_ == 64 ? 2 : 1)
                     const Params p) {
   using G = ExCfg<D_>;
   constexpr int DS = G::DS;
+  // this CTA's (head, query tile, split); a split past the tile's key tiles
+  // has nothing to do
+  const int nbh = p.B * p.H;
+  const int bh = blockIdx.x % nbh, qt = p.nq - 1 - (blockIdx.x / nbh) % p.nq;
+  const int split = blockIdx.x / (nbh * p.nq);
+  const int nk_q = exact_key_tiles(qt, p.Lk, p.causal);
+  const int jb = split * p.S, je = jb + p.S < nk_q ? jb + p.S : nk_q;
+  if (jb >= je) return;
+  const bool whole = jb == 0 && je == nk_q;     // the tile's only split: output directly
   constexpr uint32_t oW = G::oW, oQ = G::oQ, oK = G::oK, oV = G::oV, oOnes = G::oOnes, oP = G::oP;
   constexpr uint32_t tS = G::tS, tX = G::tX;
   constexpr uint32_t kTile = DS * kBlk;         // one 128-token tile of d columns (bf16)
@@ -148,13 +169,10 @@ __global__ void __launch_bounds__(kThreads, D_ == 64 ? 2 : 1)
   const uint32_t lane_tm = tmem + ((uint32_t)(quad * 32) << 16);
   // query tiles in decreasing order of work first (causal: tile qt walks qt + 1
   // key tiles), so that the short ones fill in behind the long ones
-  const int nbh = p.B * p.H;
-  const int bh = blockIdx.x % nbh, qt = p.nq - 1 - blockIdx.x / nbh;
   const int b = bh / p.H, h = bh % p.H;
   const int hw = p.heads_w == 1 ? 0 : h;
   const int q0 = qt * kT;
   const int qi = q0 + row;
-  const int nk = p.causal ? qt + 1 : (p.Lk + kT - 1) / kT;
   const int r = p.r;
   const int rb = (r + 63) / 64;                 // 64-column blocks of the projections
 
@@ -186,10 +204,10 @@ __global__ void __launch_bounds__(kThreads, D_ == 64 ? 2 : 1)
     if (tid == 0) {
       mbar_arrive_expect_tx(bar_k, kTile);
       for (int sl = 0; sl < DS; ++sl)
-        tma_load_4d(sm + oK + sl * kBlk, &tm_k, 64 * sl, 0, h, b, bar_k);
+        tma_load_4d(sm + oK + sl * kBlk, &tm_k, 64 * sl, jb * kT, h, b, bar_k);
       mbar_arrive_expect_tx(bar_v, kTile);
       for (int sl = 0; sl < DS; ++sl)
-        tma_load_4d(sm + oV + sl * kBlk, &tm_v, 64 * sl, 0, h, b, bar_v);
+        tma_load_4d(sm + oV + sl * kBlk, &tm_v, 64 * sl, jb * kT, h, b, bar_v);
     }
     to_fp16_inplace(s0 + oQ, kTile, p.dev_status);
     fence_async_smem();
@@ -213,7 +231,7 @@ __global__ void __launch_bounds__(kThreads, D_ == 64 ? 2 : 1)
     __syncthreads();
   }
 
-  for (int j = 0; j < nk && !abort; ++j) {
+  for (int j = jb; j < je && !abort; ++j) {
     const int k0 = j * kT;
     // ---- K_j: projection p_k
     if (!wait_all(bar_k, ph_k, p.dev_status)) { abort = true; break; }
@@ -257,8 +275,8 @@ __global__ void __launch_bounds__(kThreads, D_ == 64 ? 2 : 1)
     ph_mma ^= 1;
     tc_fence_after();
     // the scores MMA has read p_k: the next key tile may load over it
-    if (j + 1 < nk) ++k_issued;
-    if (tid == 0 && j + 1 < nk) {
+    if (j + 1 < je) ++k_issued;
+    if (tid == 0 && j + 1 < je) {
       mbar_arrive_expect_tx(bar_k, kTile);
       for (int sl = 0; sl < DS; ++sl)
         tma_load_4d(sm + oK + sl * kBlk, &tm_k, 64 * sl, k0 + kT, h, b, bar_k);
@@ -320,8 +338,8 @@ __global__ void __launch_bounds__(kThreads, D_ == 64 ? 2 : 1)
     ph_mma ^= 1;
     tc_fence_after();
     // the value MMA has read V: the next value tile may load
-    if (j + 1 < nk) ++v_issued;
-    if (tid == 0 && j + 1 < nk) {
+    if (j + 1 < je) ++v_issued;
+    if (tid == 0 && j + 1 < je) {
       mbar_arrive_expect_tx(bar_v, kTile);
       for (int sl = 0; sl < DS; ++sl)
         tma_load_4d(sm + oV + sl * kBlk, &tm_v, 64 * sl, k0 + kT, h, b, bar_v);
@@ -346,7 +364,19 @@ __global__ void __launch_bounds__(kThreads, D_ == 64 ? 2 : 1)
     drain_loads(bar_v, v_issued, v_waited);
     drain_mmas(bar_drain);
   }
-  if (!abort && qi < p.Lq) {
+  if (!abort && !whole) {
+    // a partial result: the unnormalised numerator, l and the running maximum
+    float* slot = p.part + ((size_t)(bh * p.nq + qt) * p.maxsplits + split) * (kT * (D_ + 2));
+    float4* od = reinterpret_cast<float4*>(slot + (size_t)row * D_ + half * kHalfD);
+#pragma unroll
+    for (int i = 0; i < kHalfD / 4; ++i)
+      od[i] = make_float4(o[4 * i], o[4 * i + 1], o[4 * i + 2], o[4 * i + 3]);
+    if (half == 0) {
+      slot[kT * D_ + row] = l;
+      slot[kT * D_ + kT + row] = mrow;
+    }
+  }
+  if (!abort && whole && qi < p.Lq) {
     const bool live = p.qmask == nullptr || p.qmask[(size_t)b * p.Lq + qi] != 0;
     const float inv = (live && l > 0.f) ? 1.f / l : 0.f;
     uint4* dst = reinterpret_cast<uint4*>(p.out + (int64_t)b * p.ob + (int64_t)h * p.oh +
@@ -375,6 +405,64 @@ __global__ void __launch_bounds__(kThreads, D_ == 64 ? 2 : 1)
 
 }  // namespace
 
+// Query tiles with more than one split: per row, m = max_s m_s and
+// out = sum_s 2^(m_s - m) O_s / sum_s 2^(m_s - m) l_s (the splits' running
+// maxima are base-2 exponents); 256 threads per (query tile, head), each thread
+// half a row.
+template <int D_>
+__global__ void __launch_bounds__(256) exact_combine_kernel(const Params p) {
+  const int qt = blockIdx.x, bh = blockIdx.y;
+  const int ns = (exact_key_tiles(qt, p.Lk, p.causal) + p.S - 1) / p.S;
+  if (ns <= 1) return;
+  const int row = threadIdx.x & 127, half = threadIdx.x >> 7;
+  const int qi = qt * kT + row;
+  if (qi >= p.Lq) return;
+  const int b = bh / p.H, h = bh % p.H;
+  constexpr int kHalfD = D_ / 2;
+  const size_t stride = (size_t)kT * (D_ + 2);
+  const float* base = p.part + (size_t)(bh * p.nq + qt) * p.maxsplits * stride;
+  float mx = -INFINITY;
+  for (int s = 0; s < ns; ++s) mx = fmaxf(mx, base[s * stride + kT * D_ + kT + row]);
+  float o[kHalfD], l = 0.f;
+#pragma unroll
+  for (int i = 0; i < kHalfD; ++i) o[i] = 0.f;
+  if (mx > -INFINITY) {
+    for (int s = 0; s < ns; ++s) {
+      const float* sl = base + s * stride;
+      const float ms = sl[kT * D_ + kT + row];
+      if (!(ms > -INFINITY)) continue;       // no visible key in this split
+      const float sc = exp2f(ms - mx);
+      l = fmaf(sc, sl[kT * D_ + row], l);
+      const float4* src = reinterpret_cast<const float4*>(sl + (size_t)row * D_ + half * kHalfD);
+#pragma unroll
+      for (int i = 0; i < kHalfD / 4; ++i) {
+        const float4 x = src[i];
+        o[4 * i] = fmaf(sc, x.x, o[4 * i]);
+        o[4 * i + 1] = fmaf(sc, x.y, o[4 * i + 1]);
+        o[4 * i + 2] = fmaf(sc, x.z, o[4 * i + 2]);
+        o[4 * i + 3] = fmaf(sc, x.w, o[4 * i + 3]);
+      }
+    }
+  }
+  const bool live = p.qmask == nullptr || p.qmask[(size_t)b * p.Lq + qi] != 0;
+  const float inv = (live && l > 0.f) ? 1.f / l : 0.f;
+  uint4* dst = reinterpret_cast<uint4*>(p.out + (int64_t)b * p.ob + (int64_t)h * p.oh +
+                                        (int64_t)qi * p.ol + half * kHalfD);
+  bool bad = false;
+#pragma unroll
+  for (int q4 = 0; q4 < kHalfD / 8; ++q4) {
+    uint32_t w[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float x0 = o[8 * q4 + 2 * e] * inv, x1 = o[8 * q4 + 2 * e + 1] * inv;
+      bad |= !isfinite(x0) || !isfinite(x1);
+      w[e] = pack_bf16(x0, x1);
+    }
+    dst[q4] = make_uint4(w[0], w[1], w[2], w[3]);
+  }
+  if (bad) report(p.dev_status, DARK_ERR_NUMERIC);
+}
+
 template <int D_>
 cudaError_t launch_exact(const FwdArgs& a, const Params& p) {
   using G = ExCfg<D_>;
@@ -395,9 +483,41 @@ cudaError_t launch_exact(const FwdArgs& a, const Params& p) {
       carveout_set[dev] = 1;
     }
   }
-  exact_tc_kernel<D_><<<a.B * a.H * p.nq, kThreads, G::kSmem, a.stream>>>(a.tm_w, a.tm_q, a.tm_k,
-                                                                         a.tm_v, p);
+  exact_tc_kernel<D_><<<a.B * a.H * p.nq * p.maxsplits, kThreads, G::kSmem, a.stream>>>(
+      a.tm_w, a.tm_q, a.tm_k, a.tm_v, p);
+  e = cudaGetLastError();
+  if (e != cudaSuccess || p.maxsplits == 1) return e;
+  exact_combine_kernel<D_><<<dim3(p.nq, a.B * a.H), 256, 0, a.stream>>>(p);
   return cudaGetLastError();
+}
+
+// Key tiles per split (d = 64 only): none while the query tiles alone give
+// two waves of CTAs; otherwise the total key-tile work spread over about two
+// waves (at least 2 tiles per split), so that the longest query tiles no
+// longer set the time. (At d = 128, one CTA per SM, the splits' repeated
+// query projections and the combine cost more than they gain: measured.)
+void exact_split_plan(int B, int H, int Lq, int Lk, int causal, int d, int* S, int* maxsplits) {
+  const int nq = (Lq + kT - 1) / kT, nk_all = (Lk + kT - 1) / kT;
+  const long long ctas = (long long)B * H * nq;
+  const long long slots = 2LL * num_sms();
+  if (d != 64 || ctas >= 2 * slots || nk_all <= 2) {
+    *S = nk_all;
+    *maxsplits = 1;
+    return;
+  }
+  long long total = 0;
+  for (int qt = 0; qt < nq; ++qt) total += exact_key_tiles(qt, Lk, causal);
+  total *= (long long)B * H;
+  long long s = (total + 2 * slots - 1) / (2 * slots);
+  if (s < 2) s = 2;
+  if (s > nk_all) s = nk_all;
+  int nk_max = 0;
+  for (int qt = 0; qt < nq; ++qt) {
+    const int k = exact_key_tiles(qt, Lk, causal);
+    nk_max = k > nk_max ? k : nk_max;
+  }
+  *S = (int)s;
+  *maxsplits = (int)((nk_max + s - 1) / s);
 }
 
 // d = 64 (r <= 64, two CTAs per SM) and d = 128 (r <= 128, one CTA per SM):
@@ -430,7 +550,22 @@ cudaError_t tc_exact_forward(const FwdArgs& a) {
   p.r = a.r;
   p.dev_status = a.dev_status;
   p.stall = test_stall_cycles();
+  exact_split_plan(a.B, a.H, a.L, a.Lk, p.causal, a.d, &p.S, &p.maxsplits);
+  if (p.maxsplits > 1 && a.ws_bytes < tc_exact_workspace_bytes(a.B, a.H, a.L, a.Lk, a.d, p.causal)) {
+    // a workspace without room for the splits' partials: one CTA per query tile
+    p.S = (a.Lk + kT - 1) / kT;
+    p.maxsplits = 1;
+  }
+  p.part = p.maxsplits > 1 ? (float*)((char*)a.ws + kWsHeader) : nullptr;
   return a.d == 64 ? launch_exact<64>(a, p) : launch_exact<128>(a, p);
+}
+
+size_t tc_exact_workspace_bytes(int B, int H, int Lq, int Lk, int d, int causal) {
+  int S = 0, ms = 1;
+  exact_split_plan(B, H, Lq, Lk, causal, d, &S, &ms);
+  if (ms <= 1) return kWsHeader;
+  const size_t nq = (size_t)(Lq + kT - 1) / kT;
+  return align_up(kWsHeader + (size_t)B * H * nq * ms * kT * (d + 2) * 4, 256);
 }
 
 }  // namespace dark

@@ -32,6 +32,9 @@ CASES = {
                                                              d=128, r=96, m=256),
     "f32-causal-d256": synth.WORKLOADS[4].with_sizes(B=1, H=1, L=70, d=256, r=64, m=128,
                                                       dtype="f32"),
+    # six query tiles on a few heads: the key ranges are split across CTAs and
+    # the splits' partial results combined
+    "bf16-causal-split": synth.WORKLOADS[2].with_sizes(H=2, L=700, lengths=(700, 517)),
     "bf16-single-token": synth.WORKLOADS[2].with_sizes(H=1, L=1, lengths=(1, 1)),
     "bf16-empty-row": synth.WORKLOADS[2].with_sizes(H=1, L=90, lengths=(0, 90)),
 }

@@ -38,6 +38,12 @@ SMALL = {
     "c4-masked": synth.WORKLOADS[4].with_sizes(B=2, H=1, L=260, lengths=(260, 100)),
     "wide-d128-m256": synth.WORKLOADS[4].with_sizes(B=2, H=2, L=270, d=128, r=128, m=256,
                                                       lengths=(270, 150)),
+    # other (m, r) instances of the d = 64 tensor-core kernels
+    "c2-m128-r48": synth.WORKLOADS[2].with_sizes(H=2, L=300, lengths=(300, 211), m=128, r=48),
+    "c3-m128-r16": synth.WORKLOADS[3].with_sizes(H=3, L=700, m=128, r=16),
+    "c3-r64": synth.WORKLOADS[3].with_sizes(H=2, L=520, r=64),
+    "c2-noncausal-r48": synth.WORKLOADS[2].with_sizes(H=2, L=390, lengths=(390, 260), r=48,
+                                                      causal=False),
     "wide-d128-m128-shared": synth.WORKLOADS[4].with_sizes(B=1, H=3, L=140, d=128, r=64, m=128,
                                                              per_head_geom=False),
 }
