@@ -57,13 +57,12 @@ METRIC = "DARK attention fwd tokens/s (B\u00b7H\u00b7L/s) on 1 B200; % of BF16-t
 
 # DRAM bytes (read + write) per forward call from one ncu capture per kernel
 # of the call, summed over its launches: the large-head causal workload
-# (B4 H8 L8192 d256 r256 m512; features_kernel 271.8 + 553.3 MB, values_kernel
-# 745.3 + 117.0 MB). Reported only while the kernel sources hash to what was
+# (B4 H8 L8192 d256 r256 m512; features_kernel 271.9 + 553.5 MB, values_kernel
+# 745.9 + 118.6 MB). Reported only while the kernel sources hash to what was
 # captured.
 _NCU_TRAFFIC = {
     4: (("tc_wide.cu", "tc_common.cuh", "common.cuh", "internal.h", "tc_roles.cuh"),
-        "7c0598b92cb57444",
-        271.750144e6 + 553.273344e6 + 745.261312e6 + 116.957696e6),
+        "4a858da67aea70b2", 271.875328e6 + 553.454336e6 + 745.856000e6 + 118.560000e6),
 }
 
 
