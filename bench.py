@@ -588,7 +588,7 @@ def run_decode(args, rank: int, world: int, dev) -> dict | None:
                 "d2h_bytes_per_step": do.numel() * do.element_size()},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm"], "unit": "GB/s",
                      "frac": achieved / peaks["hbm"], "traffic": None,
-                     "peak_source": peaks["source"], "kernel": "decode_kernel"},
+                     "peak_source": peaks["source"], "kernel": "decode step (decode_pair_kernel for this workload)"},
         "warm_graph_1024": {"ms_per_step": warm_ms, "value": rows / (warm_ms / 1e3),
                             "GBps_algorithmic": nbytes / (warm_ms / 1e3) / 1e9,
                             "note": "state L2-resident between steps"},
