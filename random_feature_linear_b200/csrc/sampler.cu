@@ -114,23 +114,30 @@ __global__ void orth_draw_kernel(uint64_t seed, uint64_t draw, int nblk, int r,
   }
 }
 
-// Step 2: Q of one block (one CTA, thread i owns row i) by classical Gram-Schmidt
-// with a second pass, fp64; columns of Q stored like G (qc[j][i] = Q[i][j]).
-__global__ void __launch_bounds__(256) orth_qr_kernel(const double* __restrict__ gc, int r,
-                                                      double* __restrict__ qc) {
+// Step 2: Q of one block (one CTA of 1024 threads) by classical Gram-Schmidt with
+// a second pass, fp64; columns of Q stored like G (qc[j][i] = Q[i][j]). Thread
+// t < r owns row t of the column being orthogonalised; the projections
+// h_k = Q[:, k] . v are spread over the 32 warps, and the update
+// v -= sum_k Q[:, k] h_k over four groups of 256 threads, each summing a quarter
+// of the k range (the quarters are added in a fixed order).
+constexpr int kQrThreads = 1024;
+__global__ void __launch_bounds__(kQrThreads) orth_qr_kernel(const double* __restrict__ gc, int r,
+                                                             double* __restrict__ qc) {
   __shared__ double vs[256];
   __shared__ double hs[256];
+  __shared__ double part[4][256];
   __shared__ double red[8];
   const size_t off = (size_t)blockIdx.x * r * r;
   const double* g = gc + off;
   double* q = qc + off;
-  const int i = threadIdx.x, warp = i >> 5, lane = i & 31;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int i = tid & 255, grp = tid >> 8;
   for (int j = 0; j < r; ++j) {
-    double v = i < r ? g[(size_t)j * r + i] : 0.0;
+    double v = (grp == 0 && i < r) ? g[(size_t)j * r + i] : 0.0;
     for (int pass = 0; pass < 2; ++pass) {
-      vs[i] = v;
+      if (grp == 0) vs[i] = v;
       __syncthreads();
-      for (int k = warp; k < j; k += 8) {           // h_k = Q[:, k] . v
+      for (int k = warp; k < j; k += kQrThreads / 32) {    // h_k = Q[:, k] . v
         double s = 0.0;
         for (int t = lane; t < r; t += 32) s = fma(q[(size_t)k * r + t], vs[t], s);
 #pragma unroll
@@ -138,20 +145,29 @@ __global__ void __launch_bounds__(256) orth_qr_kernel(const double* __restrict__
         if (lane == 0) hs[k] = s;
       }
       __syncthreads();
-      if (i < r)
-        for (int k = 0; k < j; ++k) v = fma(-q[(size_t)k * r + i], hs[k], v);
+      {
+        const int kb = grp * j / 4, ke = (grp + 1) * j / 4;
+        double u = 0.0;
+        if (i < r)
+          for (int k = kb; k < ke; ++k) u = fma(q[(size_t)k * r + i], hs[k], u);
+        part[grp][i] = u;
+      }
+      __syncthreads();
+      if (grp == 0 && i < r) v -= ((part[0][i] + part[1][i]) + part[2][i]) + part[3][i];
       __syncthreads();
     }
-    double s = v * v;
+    if (grp == 0) {
+      double s = v * v;
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-    if (lane == 0) red[warp] = s;
+      for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+      if (lane == 0) red[warp] = s;
+    }
     __syncthreads();
     double nrm = 0.0;
 #pragma unroll
     for (int w = 0; w < 8; ++w) nrm += red[w];
     nrm = sqrt(nrm);
-    if (i < r) q[(size_t)j * r + i] = nrm > 0.0 ? v / nrm : 0.0;
+    if (grp == 0 && i < r) q[(size_t)j * r + i] = nrm > 0.0 ? v / nrm : 0.0;
     __syncthreads();                               // column j is visible before column j + 1
   }
 }
@@ -205,7 +221,7 @@ cudaError_t launch_sample_omega(uint64_t seed, uint64_t draw, int heads, int m, 
   const uint64_t work = per_head4 > (uint64_t)nblk * r ? per_head4 : (uint64_t)nblk * r;
   orth_draw_kernel<<<dim3((unsigned)((work + 255) / 256), heads), 256, 0, stream>>>(
       seed, draw, nblk, r, gc, norms);
-  orth_qr_kernel<<<heads * nblk, 256, 0, stream>>>(gc, r, qc);
+  orth_qr_kernel<<<heads * nblk, kQrThreads, 0, stream>>>(gc, r, qc);
   const uint64_t n = (uint64_t)m * r;
   orth_write_kernel<<<dim3((unsigned)((n + 255) / 256), heads), 256, 0, stream>>>(qc, norms, nblk,
                                                                                    m, r, omega);
