@@ -114,61 +114,105 @@ __global__ void orth_draw_kernel(uint64_t seed, uint64_t draw, int nblk, int r,
   }
 }
 
-// Step 2: Q of one block (one CTA of 1024 threads) by classical Gram-Schmidt with
-// a second pass, fp64; columns of Q stored like G (qc[j][i] = Q[i][j]). Thread
-// t < r owns row t of the column being orthogonalised; the projections
-// h_k = Q[:, k] . v are spread over the 32 warps, and the update
-// v -= sum_k Q[:, k] h_k over four groups of 256 threads, each summing a quarter
-// of the k range (the quarters are added in a fixed order).
+// Step 2: Q of one block (one CTA of 1024 threads), fp64, columns of Q stored
+// like G (qc[j][i] = Q[i][j]), by block classical Gram-Schmidt: the columns in
+// panels of kPanel, each panel held in shared memory. A panel is first cleared
+// of the earlier columns twice (H = Q_prev^T V, V -= Q_prev H: the
+// re-orthogonalisation pass of Gram-Schmidt, in blocks), then its columns are
+// orthonormalised among themselves by classical Gram-Schmidt with a second pass.
+// diag(R) > 0 as in the column-by-column form, so Q is the same up to rounding.
 constexpr int kQrThreads = 1024;
+constexpr int kPanel = 32;
+constexpr size_t kQrSmem = sizeof(double) * (kPanel * 256 + 256 * kPanel + 256 + 32);
 __global__ void __launch_bounds__(kQrThreads) orth_qr_kernel(const double* __restrict__ gc, int r,
                                                              double* __restrict__ qc) {
-  __shared__ double vs[256];
-  __shared__ double hs[256];
-  __shared__ double part[4][256];
-  __shared__ double red[8];
+  extern __shared__ double qsm[];
+  double* vs = qsm;                        // [kPanel][r] the panel, column-major
+  double* hs = vs + kPanel * 256;          // [256][kPanel] projections on the earlier columns
+  double* hj = hs + 256 * kPanel;          // [256] projections inside the panel
+  double* red = hj + 256;                  // [32]
   const size_t off = (size_t)blockIdx.x * r * r;
   const double* g = gc + off;
   double* q = qc + off;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int i = tid & 255, grp = tid >> 8;
-  for (int j = 0; j < r; ++j) {
-    double v = (grp == 0 && i < r) ? g[(size_t)j * r + i] : 0.0;
-    for (int pass = 0; pass < 2; ++pass) {
-      if (grp == 0) vs[i] = v;
+  const int i = tid & 255, cg = tid >> 8;  // update: row i, columns 8 cg .. 8 cg + 7
+  for (int c0 = 0; c0 < r; c0 += kPanel) {
+    const int pc = r - c0 < kPanel ? r - c0 : kPanel;
+    for (int e = tid; e < pc * r; e += kQrThreads) vs[e] = g[(size_t)c0 * r + e];
+    __syncthreads();
+    for (int pass = 0; pass < 2 && c0 > 0; ++pass) {
+      // hs[k][c] = Q[:, k] . V[:, c] for the c0 earlier columns k
+      for (int k = warp; k < c0; k += kQrThreads / 32) {
+        double qk[8];
+#pragma unroll
+        for (int t = 0; t < 8; ++t) {
+          const int ii = lane + 32 * t;
+          qk[t] = ii < r ? q[(size_t)k * r + ii] : 0.0;
+        }
+        for (int c = 0; c < pc; ++c) {
+          double s = 0.0;
+#pragma unroll
+          for (int t = 0; t < 8; ++t) {
+            const int ii = lane + 32 * t;
+            if (ii < r) s = fma(qk[t], vs[c * r + ii], s);
+          }
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+          if (lane == 0) hs[k * kPanel + c] = s;
+        }
+      }
       __syncthreads();
-      for (int k = warp; k < j; k += kQrThreads / 32) {    // h_k = Q[:, k] . v
-        double s = 0.0;
-        for (int t = lane; t < r; t += 32) s = fma(q[(size_t)k * r + t], vs[t], s);
+      // V[:, c] -= sum_k Q[:, k] hs[k][c]
+      if (i < r) {
+        double acc[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) acc[u] = 0.0;
+        for (int k = 0; k < c0; ++k) {
+          const double qik = q[(size_t)k * r + i];
+#pragma unroll
+          for (int u = 0; u < 8; ++u) acc[u] = fma(qik, hs[k * kPanel + 8 * cg + u], acc[u]);
+        }
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+          if (8 * cg + u < pc) vs[(8 * cg + u) * r + i] -= acc[u];
+      }
+      __syncthreads();
+    }
+    // the panel's columns among themselves: Gram-Schmidt with a second pass
+    for (int j = 0; j < pc; ++j) {
+      for (int pass = 0; pass < 2 && j > 0; ++pass) {
+        if (warp < j) {                    // hj[k] = V[:, k] . V[:, j], k < j
+          double s = 0.0;
+          for (int ii = lane; ii < r; ii += 32) s = fma(vs[warp * r + ii], vs[j * r + ii], s);
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+          if (lane == 0) hj[warp] = s;
+        }
+        __syncthreads();
+        if (tid < r) {
+          double v = vs[j * r + tid];
+          for (int k = 0; k < j; ++k) v = fma(-vs[k * r + tid], hj[k], v);
+          vs[j * r + tid] = v;
+        }
+        __syncthreads();
+      }
+      if (warp < 8) {
+        const double v = tid < r ? vs[j * r + tid] : 0.0;
+        double s = v * v;
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-        if (lane == 0) hs[k] = s;
+        if (lane == 0) red[warp] = s;
       }
       __syncthreads();
-      {
-        const int kb = grp * j / 4, ke = (grp + 1) * j / 4;
-        double u = 0.0;
-        if (i < r)
-          for (int k = kb; k < ke; ++k) u = fma(q[(size_t)k * r + i], hs[k], u);
-        part[grp][i] = u;
-      }
-      __syncthreads();
-      if (grp == 0 && i < r) v -= ((part[0][i] + part[1][i]) + part[2][i]) + part[3][i];
+      double nrm = 0.0;
+#pragma unroll
+      for (int w = 0; w < 8; ++w) nrm += red[w];
+      nrm = sqrt(nrm);
+      if (tid < r) vs[j * r + tid] = nrm > 0.0 ? vs[j * r + tid] / nrm : 0.0;
       __syncthreads();
     }
-    if (grp == 0) {
-      double s = v * v;
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-      if (lane == 0) red[warp] = s;
-    }
-    __syncthreads();
-    double nrm = 0.0;
-#pragma unroll
-    for (int w = 0; w < 8; ++w) nrm += red[w];
-    nrm = sqrt(nrm);
-    if (grp == 0 && i < r) q[(size_t)j * r + i] = nrm > 0.0 ? v / nrm : 0.0;
-    __syncthreads();                               // column j is visible before column j + 1
+    for (int e = tid; e < pc * r; e += kQrThreads) q[(size_t)c0 * r + e] = vs[e];
+    __syncthreads();                       // the panel is in Q before the next panel reads it
   }
 }
 
@@ -221,7 +265,10 @@ cudaError_t launch_sample_omega(uint64_t seed, uint64_t draw, int heads, int m, 
   const uint64_t work = per_head4 > (uint64_t)nblk * r ? per_head4 : (uint64_t)nblk * r;
   orth_draw_kernel<<<dim3((unsigned)((work + 255) / 256), heads), 256, 0, stream>>>(
       seed, draw, nblk, r, gc, norms);
-  orth_qr_kernel<<<heads * nblk, kQrThreads, 0, stream>>>(gc, r, qc);
+  static int smem_set[64];
+  cudaError_t e = set_smem_limit_once((const void*)orth_qr_kernel, (int)kQrSmem, smem_set);
+  if (e != cudaSuccess) return e;
+  orth_qr_kernel<<<heads * nblk, kQrThreads, kQrSmem, stream>>>(gc, r, qc);
   const uint64_t n = (uint64_t)m * r;
   orth_write_kernel<<<dim3((unsigned)((n + 255) / 256), heads), 256, 0, stream>>>(qc, norms, nblk,
                                                                                    m, r, omega);
