@@ -180,6 +180,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (!wait_all(bar_tma, ph_tma, p.dev_status)) { abort = true; break; }
     ph_tma ^= 1;
     ++tma_waited;
+    // this chunk's key validity, read now so that the load's latency passes
+    // under the conversion and the key GEMM
+    const int tok = t0 + row;
+    const bool valid = tok < p.L && (p.mask == nullptr || p.mask[(size_t)b * p.L + tok] != 0);
     // the previous chunk's output tensor store has read its staging (in the
     // Psi region, written again below)
     if (tid == 0) bulk_wait_group_read();
@@ -230,9 +234,6 @@ __global__ void __launch_bounds__(kThreads, 1)
               sdesc(s0 + G::oW + s * 32, 16, 1024), idq, s > 0);
         mma_commit(bar_mma);
       }
-      const int tok = t0 + row;
-      bool valid = tok < p.L;
-      if (valid && p.mask != nullptr) valid = p.mask[(size_t)b * p.L + tok] != 0;
       if (p.stab) {
         // the running maximum starts from the earlier segments' maxima (the
         // key-state launch's results), then takes each chunk's largest valid
@@ -451,7 +452,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       // the chunk's rows staged in the Psi region (free once the inter GEMM is
       // done; 16-byte chunks XOR-swizzled by row, as the output map's 128-byte
       // swizzle expects), then one tensor store (rows past L are not written)
-      const int tok = t0 + row;
       const float inv = den > 0.f ? 1.f / den : 0.f;
       uint32_t w[16];
       float sum = den;                  // non-finite if any value is

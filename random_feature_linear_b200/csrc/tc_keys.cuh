@@ -21,22 +21,25 @@ __device__ __forceinline__ bool wait_all(uint64_t* bar, uint32_t parity, int* de
 }
 
 // bf16 -> fp16 in place for `bytes` of a shared tile (feature GEMM operand).
+// A bf16 value is out of fp16 range (|x| > 65504) exactly when its magnitude
+// bits are 0x4780 (65536) or more; that is reported.
 __device__ __forceinline__ void to_fp16_inplace(uint32_t saddr, int bytes, int* dev_status) {
-  bool bad = false;
+  uint32_t mag = 0;
+#pragma unroll 4
   for (int i = threadIdx.x; i < bytes / 16; i += kFwdThreads) {
     const uint32_t a = saddr + i * 16;
     uint4 u = ld_shared_v4(a);
     uint32_t* w32 = &u.x;
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
-      const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w32[e]));
-      bad |= fabsf(f.x) > 65504.f || fabsf(f.y) > 65504.f;
-      const __half2 hv = __floats2half2_rn(f.x, f.y);
+      mag = __vmaxu2(mag, w32[e] & 0x7FFF7FFFu);
+      const __half2 hv = __floats2half2_rn(__uint_as_float(w32[e] << 16),
+                                           __uint_as_float(w32[e] & 0xFFFF0000u));
       w32[e] = *reinterpret_cast<const uint32_t*>(&hv);
     }
     st_shared_v4(a, u.x, u.y, u.z, u.w);
   }
-  if (bad) report(dev_status, DARK_ERR_NUMERIC);
+  if ((mag & 0xFFFFu) >= 0x4780u || (mag >> 16) >= 0x4780u) report(dev_status, DARK_ERR_NUMERIC);
 }
 
 // Stabiliser: the maximum of a row of `ncols_half` * 2 TMEM columns whose two
