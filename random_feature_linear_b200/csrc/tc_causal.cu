@@ -559,8 +559,7 @@ cudaError_t launch(const FwdArgs& a, const CUtensorMap& tw, const CUtensorMap& t
   // after the key-state launch: programmatic dependent launch, so that CTAs
   // start on SMs the key-state CTAs leave and wait for its results only where
   // they read them
-  cudaLaunchConfig_t cfg;
-  memset(&cfg, 0, sizeof(cfg));
+  cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(bh * s.nseg);
   cfg.blockDim = dim3(kThreads);
   cfg.dynamicSmemBytes = G::kSmem;
