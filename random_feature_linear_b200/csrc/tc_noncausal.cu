@@ -52,6 +52,9 @@ __global__ void reduce_kernel(const float* __restrict__ partials, int nsplit, in
                               const float* __restrict__ shifts, uint8_t* __restrict__ images,
                               float* __restrict__ st_kv, float* __restrict__ st_z,
                               float* __restrict__ st_shift) {
+  // the query launch that follows may start now: it waits for this grid only
+  // where it reads the operand image
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int bh = blockIdx.y;
   const int idx = blockIdx.x * blockDim.x + threadIdx.x;
   if (idx >= 9 * m) return;
@@ -272,9 +275,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       };
       prefetch_tmap(&tm_w);
       prefetch_tmap(&tm_q);
-      load_head(0);
       load_q(0);
       if (n > 1) load_q(1);
+      // the head operands come from the split reduce (this launch may have
+      // started before it finished)
+      asm volatile("griddepcontrol.wait;" ::: "memory");
+      load_head(0);
       bool ok = true;
       int heads_done = 0;                 // h_free phases passed
       for (int i = 0; ok && i + 1 < n; ++i) {
@@ -555,8 +561,19 @@ cudaError_t launch(const FwdArgs& a, const CUtensorMap& tw, const CUtensorMap& t
   e = set_smem_limit_once((const void*)queries_kernel<M_, R_>, (int)QG::kSmem, smem_set);
   if (e != cudaSuccess) return e;
   const int grid = qp.total_tiles < kSms ? qp.total_tiles : kSms;
-  queries_kernel<M_, R_><<<grid, kThreads, QG::kSmem, a.stream>>>(tw, tq, a.tm_o, qp);
-  return cudaGetLastError();
+  // programmatic dependent launch after the reduce: the CTAs set up, load and
+  // convert their first Q tiles while the reduce finishes
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = QG::kSmem;
+  cfg.stream = a.stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, queries_kernel<M_, R_>, tw, tq, a.tm_o, qp);
 }
 
 }  // namespace
