@@ -368,9 +368,11 @@ __global__ void __launch_bounds__(kThreadsF, 1)
       const int b = bh / p.H;
       uint8_t* rec = p.img + (size_t)item * chunk_record_bytes(M_);
       if (!(ok = epi_wait(bar_x, j & 1, abort_flag, p.dev_status))) break;
-      // bf16 -> fp16 in place (|x| >= 65504 is reported)
+      // bf16 -> fp16 in place; a magnitude of 0x4780 (65536) or more in either
+      // half of a word (the running unsigned maximum of the magnitude bits) is
+      // out of fp16 range and reported
       {
-        bool bad = false;
+        uint32_t mag = 0;
 #pragma unroll 4
         for (int i = etid; i < (int)(G::DS * G::kXSlab / 16); i += kEpiThreads) {
           const uint32_t a = s0 + G::oX + i * 16;
@@ -378,14 +380,14 @@ __global__ void __launch_bounds__(kThreadsF, 1)
           uint32_t* w32 = &u.x;
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            const float2 f2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w32[e]));
-            bad |= fabsf(f2.x) > 65504.f || fabsf(f2.y) > 65504.f;
-            const __half2 hv = __floats2half2_rn(f2.x, f2.y);
+            mag = __vmaxu2(mag, w32[e] & 0x7FFF7FFFu);
+            const __half2 hv = __floats2half2_rn(__uint_as_float(w32[e] << 16),
+                                                 __uint_as_float(w32[e] & 0xFFFF0000u));
             w32[e] = *reinterpret_cast<const uint32_t*>(&hv);
           }
           st_shared_v4(a, u.x, u.y, u.z, u.w);
         }
-        if (bad) report(p.dev_status, DARK_ERR_NUMERIC);
+        if ((mag & 0xFFFFu) >= 0x4780u || (mag >> 16) >= 0x4780u) report(p.dev_status, DARK_ERR_NUMERIC);
       }
       fence_async_smem();
       tc_fence_before();
@@ -913,6 +915,9 @@ __global__ void __launch_bounds__(kThreadsV, 1)
                 1u);
           mma_commit(bar_empty + gA % G::NSLOT);
         }
+        // the numerators are complete: the epilogue reads them while the state
+        // update runs (its own barrier orders the next conversions)
+        if (ok) mma_commit(bar_nfull);
         // ---- S_t += Phi_t^T V_c, in blocks of 64 tokens
         for (int t = 0; ok && t < G::NTC; ++t) {
           for (int kb = 0; ok && kb < 2; ++kb) {
@@ -931,14 +936,12 @@ __global__ void __launch_bounds__(kThreadsV, 1)
           mma_commit(bar_ds + t);
         }
         if (!ok) break;
-        mma_commit(bar_nfull);
         mma_commit(bar_vfree);
       }
-      if (!ok) {
-        // let every issued MMA finish before TMEM is released
-        mma_commit(bar_drain);
-        mbar_wait(bar_drain, 0);
-      }
+      // let every issued MMA finish before TMEM is released (the last state
+      // update is waited for by no other role unless the state is output)
+      mma_commit(bar_drain);
+      mbar_wait(bar_drain, 0);
     }
     __syncwarp();
   } else {
