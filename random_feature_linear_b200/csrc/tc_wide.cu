@@ -616,7 +616,10 @@ struct ValCfg {
   static constexpr uint32_t oV = 0;                     // V_c block: 2 x 16 KB (MN-major)
   static constexpr uint32_t oS = 32768;                 // S operand halves: 2 x 32 KB
   static constexpr uint32_t oR = oS + 65536;            // ring: NSLOT x 16 KB
-  static constexpr uint32_t kXB = 16384 + 1024;         // received o' (fp16 [64][128]) + den' [64]
+  // received o' (fp16 [64 rows][128 columns], the 16-byte chunks of each
+  // 128-byte half-row XOR-swizzled by row, so that eight consecutive rows
+  // hit different banks) + den' [64]
+  static constexpr uint32_t kXB = 16384 + 1024;
   static constexpr uint32_t kXBytes = 16384 + 256;      // bytes the peer sends per chunk
   static constexpr uint32_t oX = oR + NSLOT * 16384;    // [2] receive buffers (chunk parity)
   static constexpr uint32_t oSm = oX + 2 * kXB;         // [2] small items: dz [NTC*128], den_a [256]
@@ -995,7 +998,7 @@ __global__ void __launch_bounds__(kThreadsV, 1)
       float nm[64];
 #pragma unroll
       for (int q4 = 0; q4 < 8; ++q4) {
-        const uint4 u = ld_shared_v4(xr + q4 * 16);
+        const uint4 u = ld_shared_v4(xr + (uint32_t)((q4 ^ (row & 7)) * 16));
         const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
@@ -1217,7 +1220,8 @@ __global__ void __launch_bounds__(kThreadsV, 1)
           const uint32_t rb = peer_addr(smem_u32(bar_recv + (c & 1)), peer);
 #pragma unroll
           for (int q4 = 0; q4 < 8; ++q4)
-            st_async_v4(xr + q4 * 16, o[4 * q4], o[4 * q4 + 1], o[4 * q4 + 2], o[4 * q4 + 3], rb);
+            st_async_v4(xr + (uint32_t)((q4 ^ (row & 7)) * 16), o[4 * q4], o[4 * q4 + 1], o[4 * q4 + 2],
+                        o[4 * q4 + 3], rb);
           if (colh == 0) st_async_f32(peer_addr(xb + 16384 + (uint32_t)(row & 63) * 4, peer), den, rb);
         }
       }
