@@ -987,8 +987,15 @@ __global__ void __launch_bounds__(kThreadsV, 1)
       return !bad;
     };
     // rows of chunk cc this CTA finishes: (den o + den' o') / (den + den') with
-    // o, den kept from that chunk and o', den' from the peer's buffer cc & 1
+    // o, den kept from that chunk and o', den' from the peer's buffer cc & 1.
+    // The buffer of chunk cc - 1 goes back to the peer here (its chunk cc + 1),
+    // once the tensor stores of cc - 1 have read it: the wait is a chunk late.
     auto finish_prev = [&](int cc) -> bool {
+      if (gi == 0 && cc > 0) {
+        bulk_wait_group_read();
+        if (cc + 1 < p.nc) mbar_arrive_expect_tx(bar_recv + ((cc - 1) & 1), G::kXBytes);
+        arrive_peer_relaxed(peer_addr(smem_u32(bar_rfree + ((cc - 1) & 1)), peer));
+      }
       const bool arrived = wait_cluster(bar_recv + (cc & 1), (cc >> 1) & 1, abort_flag, p.dev_status);
       if (grp_sync_or(grp, !arrived)) return false;
       const uint32_t xb = s0 + G::oX + (cc & 1) * G::kXB;
@@ -1011,7 +1018,7 @@ __global__ void __launch_bounds__(kThreadsV, 1)
       // every reader of the group is done with o': the rows go out through the
       // same buffer (two 64-column halves, 64 rows x 128 B each, 16-byte chunks
       // XOR-swizzled by row as the output map's 128-byte swizzle expects) by two
-      // tensor stores; then the peer may send its chunk cc + 2 into the buffer
+      // tensor stores
       grp_sync_or(grp, false);
       const float dt = pden + dp;
       const float invd = dt > 0.f ? 1.f / dt : 0.f;
@@ -1036,9 +1043,6 @@ __global__ void __launch_bounds__(kThreadsV, 1)
         tma_store_4d(&tm_o, xb, 128 * vb, cc * kC + 64 * fh, h, b);
         tma_store_4d(&tm_o, xb + 8192, 128 * vb + 64, cc * kC + 64 * fh, h, b);
         bulk_commit_group();
-        bulk_wait_group_read();
-        if (cc + 2 < p.nc) mbar_arrive_expect_tx(bar_recv + (cc & 1), G::kXBytes);
-        arrive_peer_relaxed(peer_addr(smem_u32(bar_rfree + (cc & 1)), peer));
       }
       return true;
     };
