@@ -895,13 +895,14 @@ __global__ void __launch_bounds__(kThreadsV, 1)
                   (t | hh | st) != 0);
             mma_commit(bar_sfree + hh);
           }
-        }
-        // the epilogue reads the Psi items too (denominators): release them after that
-        for (int t = 0; ok && t < G::NTC; ++t)
+          // the epilogue reads the tile's Psi items too (denominators): release
+          // them once it has, so that the Phi items taking their slots load
+          // while the next tile's prefix product runs
           for (int hh = 0; ok && hh < 2; ++hh) {
             if (!(ok = wait_one(bar_den + 2 * t + hh, c & 1, abort_flag, p.dev_status))) break;
             mma_commit(bar_empty + (g0 + item_psi(t, hh)) % G::NSLOT);
           }
+        }
         if (!ok) break;
         // ---- num[:, hi] += A_c[:, my keys] V_c[my keys]
         for (int j = 0; ok && j < G::NA; ++j) {
