@@ -92,6 +92,55 @@ def max_over_ranks(value: float, device) -> float:
     return float(t.item())
 
 
+E2E_NOTE = ("pinned host buffers, double-buffered over three streams: step i's "
+            "host-to-device copies overlap step i-1's call and its device-to-host copies; "
+            "every step copies all of its inputs in and its outputs out; time from the "
+            "first copy in to the last copy out")
+
+
+def pipelined_e2e(host_in, dev_in_like, call, dev_out_like, host_out, steps: int, warmup: int,
+                  dev) -> float:
+    """Milliseconds per step of `steps` end-to-end steps through the public
+    call: the inputs of step i (host_in(i), pinned) are copied in on one
+    stream, `call(inputs, outputs)` runs on a second, the outputs are copied
+    back into `host_out` (pinned) on a third, with two device buffer sets so
+    that the copies of neighbouring steps overlap the call (PCIe carries both
+    directions at once). Events order each buffer set's reuse."""
+    s_in, s_cmp, s_out = (torch.cuda.Stream(device=dev) for _ in range(3))
+    ins = [[torch.empty_like(t) for t in dev_in_like] for _ in range(2)]
+    outs = [[torch.empty_like(t) for t in dev_out_like] for _ in range(2)]
+    ev_in, ev_cmp, ev_out = ([torch.cuda.Event() for _ in range(2)] for _ in range(3))
+
+    def step(i):
+        k = i % 2
+        with torch.cuda.stream(s_in):
+            s_in.wait_event(ev_cmp[k])      # the call two steps back has read set k
+            for d, h in zip(ins[k], host_in(i)):
+                d.copy_(h, non_blocking=True)
+            ev_in[k].record(s_in)
+        with torch.cuda.stream(s_cmp):
+            s_cmp.wait_event(ev_in[k])
+            s_cmp.wait_event(ev_out[k])     # the copy out two steps back has read set k
+            call(ins[k], outs[k])
+            ev_cmp[k].record(s_cmp)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(ev_cmp[k])
+            for h, d in zip(host_out, outs[k]):
+                h.copy_(d, non_blocking=True)
+            ev_out[k].record(s_out)
+
+    for i in range(warmup):
+        step(i)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(s_in)
+    for i in range(steps):
+        step(i)
+    e1.record(s_out)
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / steps
+
+
 def alg_flops(w: synth.Workload) -> float:
     """Algorithmic FLOPs of one forward pass: per head 2Ldm (query features) +
     2Ld(m+r) (key features and norms) + 2Lm(d+1) (state) + 2Lm(d+1) (output)."""
@@ -323,36 +372,21 @@ def run_native(args, w: synth.Workload, rank: int, world: int, dev) -> dict | No
     assert int(status.item()) == 0, D.dark_status_string(int(status.item()))
 
     # end to end through the C ABI with pinned host buffers
-    hq, hk, hv = (t.cpu().pin_memory() for t in (q, k, v))
-    hmask = None if mask is None else mask.cpu().pin_memory()
+    srcs = [q, k, v] + ([] if mask is None else [mask])
+    host = [t.cpu().pin_memory() for t in srcs]
     hout = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
-    dmask = None if mask is None else torch.empty_like(mask)
 
-    def e2e_step():
-        dq.copy_(hq, non_blocking=True)
-        dk.copy_(hk, non_blocking=True)
-        dv.copy_(hv, non_blocking=True)
-        if dmask is not None:
-            dmask.copy_(hmask, non_blocking=True)
-        D.dark_attention_fwd(proj, dq, dk, dv, out, w.B, w.H, w.L, key_mask=dmask, flags=flags,
+    def e2e_call(ins, outs):
+        D.dark_attention_fwd(proj, ins[0], ins[1], ins[2], outs[0], w.B, w.H, w.L,
+                             key_mask=ins[3] if mask is not None else None, flags=flags,
                              ws=ws, dev_status=status)
-        hout.copy_(out, non_blocking=True)
 
-    for _ in range(args.warmup):
-        e2e_step()
-    torch.cuda.synchronize()
-    e_start, e_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if world > 1:
         dist.barrier()
-    e_start.record(stream)
-    for _ in range(args.steps):
-        e2e_step()
-    e_end.record(stream)
-    torch.cuda.synchronize()
-    e2e_ms = max_over_ranks(e_start.elapsed_time(e_end) / args.steps, dev)
-    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv)) + (
-        0 if hmask is None else hmask.numel())
+    e2e_ms = max_over_ranks(pipelined_e2e(lambda i: host, srcs, e2e_call, [out], [hout],
+                                          args.steps, args.warmup, dev), dev)
+    assert int(status.item()) == 0, D.dark_status_string(int(status.item()))
+    h2d = sum(t.numel() * t.element_size() for t in host)
     d2h = hout.numel() * hout.element_size()
 
     if rank != 0:
@@ -422,7 +456,7 @@ def run_native(args, w: synth.Workload, rank: int, world: int, dev) -> dict | No
                    "timing": "CUDA events around one CUDA-graph replay of the forward call per step",
                    "parallelism": f"replicas x{world} (independent batches, no collective)"},
         "e2e": {"value": tokens / (e2e_ms / 1e3), "unit": "tokens/s",
-                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "how": E2E_NOTE},
         "roofline": roof,
         "roofline_other": {"t_tensor_us": t_tc * 1e6, "t_hbm_us": t_hbm * 1e6,
                            "t_mufu_us_nominal": 2.0 * w.tokens * w.m / MUFU_EX2_PER_S * 1e6,
@@ -542,18 +576,15 @@ def run_decode(args, rank: int, world: int, dev) -> dict | None:
     # end to end: pinned host q, k, v in, the call, out back to the host, per step
     hq, hk, hv = (t[:args.steps].cpu().pin_memory() for t in (sq, sk, sv))
     ho = torch.empty_like(hq[0]).pin_memory()
-    dq, dk, dv = (torch.empty_like(sq[0]) for _ in range(3))
-    do = torch.empty_like(dq)
-    e0.record(stream)
-    for i in range(args.steps):
-        dq.copy_(hq[i], non_blocking=True)
-        dk.copy_(hk[i], non_blocking=True)
-        dv.copy_(hv[i], non_blocking=True)
-        D.dark_decode_step(proj, st, dq, dk, dv, do, dev_status=status)
-        ho.copy_(do, non_blocking=True)
-    e1.record(stream)
-    torch.cuda.synchronize()
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, dev)
+    dq, do = sq[0], sq[0]
+
+    def e2e_call(ins, outs):
+        D.dark_decode_step(proj, st, ins[0], ins[1], ins[2], outs[0], dev_status=status)
+
+    n_e2e = hq.shape[0]
+    e2e_ms = max_over_ranks(pipelined_e2e(
+        lambda i: [hq[i % n_e2e], hk[i % n_e2e], hv[i % n_e2e]], [sq[0], sk[0], sv[0]], e2e_call,
+        [sq[0]], [ho], args.steps, 0, dev), dev)
     ms = max_over_ranks(ms, dev)
     if rank != 0:
         return None
@@ -585,7 +616,7 @@ def run_decode(args, rank: int, world: int, dev) -> dict | None:
                    "parallelism": f"replicas x{world} (independent batches, no collective)"},
         "e2e": {"value": rows / (e2e_ms / 1e3), "unit": "tokens/s",
                 "h2d_bytes_per_step": 3 * dq.numel() * dq.element_size(),
-                "d2h_bytes_per_step": do.numel() * do.element_size()},
+                "d2h_bytes_per_step": do.numel() * do.element_size(), "how": E2E_NOTE},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm"], "unit": "GB/s",
                      "frac": achieved / peaks["hbm"], "traffic": None,
                      "peak_source": peaks["source"], "kernel": "decode step (decode_pair_kernel for this workload)"},
@@ -642,9 +673,9 @@ def run_cross(args, rank: int, world: int, dev) -> dict | None:
     flush = L2Flush(dev)
     stream = torch.cuda.current_stream()
 
-    def call(q_, k_, v_, qm_, cm_):
-        D.dark_cross_attention_fwd(proj, q_, k_, v_, out, w.B, w.H, lq, lk, query_mask=qm_,
-                                   context_mask=cm_, ws=ws, dev_status=status)
+    def call(q_, k_, v_, qm_, cm_, out_=None):
+        D.dark_cross_attention_fwd(proj, q_, k_, v_, out if out_ is None else out_, w.B, w.H, lq,
+                                   lk, query_mask=qm_, context_mask=cm_, ws=ws, dev_status=status)
 
     for _ in range(args.warmup):
         flush()
@@ -680,28 +711,13 @@ def run_cross(args, rank: int, world: int, dev) -> dict | None:
         / args.steps
     assert int(status.item()) == 0, D.dark_status_string(int(status.item()))
 
-    host = [t.cpu().pin_memory() for t in (q, k, v, qm, cm)]
-    devb = [torch.empty_like(t) for t in (q, k, v, qm, cm)]
+    srcs = [q, k, v, qm, cm]
+    host = [t.cpu().pin_memory() for t in srcs]
     hout = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-
-    def e2e_step():
-        for dst, src in zip(devb, host):
-            dst.copy_(src, non_blocking=True)
-        call(*devb)
-        hout.copy_(out, non_blocking=True)
-
-    for _ in range(args.warmup):
-        e2e_step()
-    torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if world > 1:
         dist.barrier()
-    e0.record(stream)
-    for _ in range(args.steps):
-        e2e_step()
-    e1.record(stream)
-    torch.cuda.synchronize()
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, dev)
+    e2e_ms = max_over_ranks(pipelined_e2e(lambda i: host, srcs, lambda ins, outs: call(*ins, out_=outs[0]),
+                                          [out], [hout], args.steps, args.warmup, dev), dev)
     if rank != 0:
         return None
     tokens = w.B * w.H * (lq + lk) * world
@@ -747,7 +763,7 @@ def run_cross(args, rank: int, world: int, dev) -> dict | None:
                    "parallelism": f"replicas x{world} (independent batches, no collective)"},
         "e2e": {"value": tokens / (e2e_ms / 1e3), "unit": "tokens/s",
                 "h2d_bytes_per_step": sum(x.numel() * x.element_size() for x in host),
-                "d2h_bytes_per_step": hout.numel() * hout.element_size()},
+                "d2h_bytes_per_step": hout.numel() * hout.element_size(), "how": E2E_NOTE},
         "roofline": roof,
         "roofline_other": {"t_tensor_us": t_tc * 1e6, "t_hbm_us": t_hbm * 1e6,
                            "alg_flops": flops, "alg_bytes": nbytes},
@@ -812,9 +828,10 @@ def run_backward(args, w: synth.Workload, rank: int, world: int, dev) -> dict | 
     flush = L2Flush(dev)
     stream = torch.cuda.current_stream()
 
-    def call(q_, k_, v_, g_, m_):
-        D.dark_attention_bwd(omega, geom, q_, k_, v_, g_, dq, dk, dv, w.B, w.H, w.L, dt,
-                             key_mask=m_, flags=flags, dgeom=dgeom, ws=ws, dev_status=status)
+    def call(q_, k_, v_, g_, m_, outs_=None):
+        o = (dq, dk, dv, dgeom) if outs_ is None else outs_
+        D.dark_attention_bwd(omega, geom, q_, k_, v_, g_, o[0], o[1], o[2], w.B, w.H, w.L, dt,
+                             key_mask=m_, flags=flags, dgeom=o[3], ws=ws, dev_status=status)
 
     if args.ncu:
         # capture mode for Nsight Compute: warmup + steps backward calls only
@@ -859,29 +876,15 @@ def run_backward(args, w: synth.Workload, rank: int, world: int, dev) -> dict | 
 
     srcs = [q, k, v, g] + ([] if mask is None else [mask])
     host = [t.cpu().pin_memory() for t in srcs]
-    devb = [torch.empty_like(t) for t in srcs]
     outs = [dq, dk, dv, dgeom]
     houts = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in outs]
-
-    def e2e_step():
-        for dst, src in zip(devb, host):
-            dst.copy_(src, non_blocking=True)
-        call(devb[0], devb[1], devb[2], devb[3], devb[4] if mask is not None else None)
-        for dst, src in zip(houts, outs):
-            dst.copy_(src, non_blocking=True)
-
-    for _ in range(args.warmup):
-        e2e_step()
-    torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if world > 1:
         dist.barrier()
-    e0.record(stream)
-    for _ in range(args.steps):
-        e2e_step()
-    e1.record(stream)
-    torch.cuda.synchronize()
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, dev)
+    e2e_ms = max_over_ranks(pipelined_e2e(
+        lambda i: host, srcs,
+        lambda ins, o: call(ins[0], ins[1], ins[2], ins[3], ins[4] if mask is not None else None,
+                            outs_=o),
+        outs, houts, args.steps, args.warmup, dev), dev)
     assert int(status.item()) == 0, D.dark_status_string(int(status.item()))
     if rank != 0:
         return None
@@ -932,7 +935,8 @@ def run_backward(args, w: synth.Workload, rank: int, world: int, dev) -> dict | 
                    "parallelism": f"replicas x{world} (independent batches, no collective)"},
         "e2e": {"value": tokens / (e2e_ms / 1e3), "unit": "tokens/s",
                 "h2d_bytes_per_step": sum(x.numel() * x.element_size() for x in host),
-                "d2h_bytes_per_step": sum(x.numel() * x.element_size() for x in houts)},
+                "d2h_bytes_per_step": sum(x.numel() * x.element_size() for x in houts),
+                "how": E2E_NOTE},
         "roofline": roof,
         "roofline_other": {"alg_flops": flops,
                            "frac_of_bf16_tensor_peak": flops / t / 1e12 / peaks["bf16"],
