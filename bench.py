@@ -92,10 +92,11 @@ def max_over_ranks(value: float, device) -> float:
     return float(t.item())
 
 
-E2E_NOTE = ("pinned host buffers, double-buffered over three streams: step i's "
-            "host-to-device copies overlap step i-1's call and its device-to-host copies; "
-            "every step copies all of its inputs in and its outputs out; time from the "
-            "first copy in to the last copy out")
+E2E_NOTE = ("pinned host buffers, double-buffered over three streams (one stream when a "
+            "step moves under 4 MiB): step i's host-to-device copies overlap step i-1's call "
+            "and its device-to-host copies; every step copies all of its inputs in and its "
+            "outputs out; time from the first copy in to the last copy out")
+E2E_OVERLAP_MIN_BYTES = 4 << 20
 
 
 def pipelined_e2e(host_in, dev_in_like, call, dev_out_like, host_out, steps: int, warmup: int,
@@ -105,8 +106,14 @@ def pipelined_e2e(host_in, dev_in_like, call, dev_out_like, host_out, steps: int
     stream, `call(inputs, outputs)` runs on a second, the outputs are copied
     back into `host_out` (pinned) on a third, with two device buffer sets so
     that the copies of neighbouring steps overlap the call (PCIe carries both
-    directions at once). Events order each buffer set's reuse."""
-    s_in, s_cmp, s_out = (torch.cuda.Stream(device=dev) for _ in range(3))
+    directions at once). Events order each buffer set's reuse. A step that
+    moves less than E2E_OVERLAP_MIN_BYTES runs all three parts on one stream:
+    there the cross-stream waits cost more than the overlap saves."""
+    moved = sum(t.numel() * t.element_size() for t in list(dev_in_like) + list(dev_out_like))
+    if moved < E2E_OVERLAP_MIN_BYTES:
+        s_in = s_cmp = s_out = torch.cuda.Stream(device=dev)
+    else:
+        s_in, s_cmp, s_out = (torch.cuda.Stream(device=dev) for _ in range(3))
     ins = [[torch.empty_like(t) for t in dev_in_like] for _ in range(2)]
     outs = [[torch.empty_like(t) for t in dev_out_like] for _ in range(2)]
     ev_in, ev_cmp, ev_out = ([torch.cuda.Event() for _ in range(2)] for _ in range(3))
