@@ -57,12 +57,12 @@ METRIC = "DARK attention fwd tokens/s (B\u00b7H\u00b7L/s) on 1 B200; % of BF16-t
 
 # DRAM bytes (read + write) per forward call from one ncu capture per kernel
 # of the call, summed over its launches: the large-head causal workload
-# (B4 H8 L8192 d256 r256 m512; features_kernel 271.8 + 552.3 MB, values_kernel
-# 744.7 + 117.9 MB). Reported only while the kernel sources hash to what was
+# (B4 H8 L8192 d256 r256 m512; features_kernel 271.8 + 552.4 MB, values_kernel
+# 744.6 + 117.9 MB). Reported only while the kernel sources hash to what was
 # captured.
 _NCU_TRAFFIC = {
     4: (("tc_wide.cu", "tc_common.cuh", "common.cuh", "internal.h", "tc_roles.cuh"),
-        "2687760ef240a970", 271.757824e6 + 552.337152e6 + 744.660224e6 + 117.919744e6),
+        "6615388094732260", 271.751936e6 + 552.398080e6 + 744.621312e6 + 117.852160e6),
 }
 
 

@@ -598,11 +598,14 @@ __global__ void __launch_bounds__(kThreadsF, 1)
 // other half through distributed shared memory, as num/den in fp16 plus den
 // in fp32 (out = (num + den' o') / (den + den')).
 //
-// Warp 9 streams V_c (TMA) and the images (bulk copies) through a 3-slot ring;
+// Warp 9 streams V_c (TMA) and the images (bulk copies) through a 5-slot ring;
 // warp 8 issues the MMAs; warps 0-7 are the epilogue. The S operand [S hi | S lo]
 // is rebuilt from TMEM for every chunk in halves of 64 features: epilogue group
 // h (the four warps whose TMEM lanes hold features 64h..64h+63) fills buffer h
-// while the MMAs read the other one.
+// while the MMAs read the other one. The numerators are signalled as soon as
+// the prefix and intra-chunk products are done, so the epilogue reads them
+// while the state update runs; each feature tile's Psi slots go back to the
+// producer once the epilogue has read them for the denominators.
 template <int D_, int M_>
 struct ValCfg {
   static constexpr int FS = M_ >= 256 ? 2 : 1;          // feature halves (cluster size)
@@ -742,7 +745,7 @@ __global__ void __launch_bounds__(kThreadsV, 1)
   uint64_t* bar_sfree = bars + 6;       // [2] MMA: GEMM reading S operand half h done
   uint64_t* bar_ds = bars + 8;          // [2] MMA: state tile t updated by the chunk
   uint64_t* bar_den = bars + 10;        // [2 t][2 h] group h: Psi_{t,h} read for the denominators (4)
-  uint64_t* bar_nfull = bars + 14;      // MMA: numerator complete
+  uint64_t* bar_nfull = bars + 14;      // MMA: numerators complete (before the state update)
   uint64_t* bar_nfree = bars + 15;      // epilogue: numerator read (8)
   uint64_t* bar_recv = bars + 38;       // [2] peer: its half-result for my rows arrived (128)
   uint64_t* bar_rfree = bars + 40;      // [2] peer: my half-result in its buffer consumed (128)
